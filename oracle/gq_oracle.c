@@ -1,0 +1,742 @@
+/*
+ * gq_oracle.c -- plain, slow, sequential CPU oracle for bucketed gradient quantization.
+ *
+ * TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU-baseline leg
+ * load it; the CUDA product path never does, and the two share no code.
+ *
+ * Page references ([P1], [P2], [P3]) are defined in gq_oracle.h.  Every loop runs over the
+ * elements of a bucket in index order.  Floating point is IEEE binary32/binary64 with
+ * round-to-nearest and no contraction (built with -ffp-contract=off).  The pages fix no
+ * precision; the level fits and rounding decisions are taken in binary32 (the precision of
+ * the gradients and of the CUDA kernels), and every fit decision is taken from exact integer
+ * data (fixed-point positions and sums), so that it does not depend on summation order.
+ *
+ * Pins (checked by the CPU test suite, not by re-typing these formulas):
+ *   - Philox4x32-10 against the published known-answer vectors of the generator;
+ *   - stochastic rounding against the 0.7 example of [P3] and Monte Carlo mean / variance;
+ *   - ORQ's greedy against an independent naive greedy on the raw values;
+ *   - BinGrad-b's split against brute force over all thresholds;
+ *   - BinGrad-pb's pair against brute force over all grid pairs, and the ordering of
+ *     quantization errors BinGrad-b <= BinGrad-pb stated in [P2] "Key findings";
+ *   - QSGD/TernGrad against hand-computed closed forms;
+ *   - packing against a bit-by-bit unpacker; error feedback against its telescoping sum.
+ * Parity of BinGrad-pb with the paper's own (unpublished on the pages) definition is unpinned:
+ * only this reading of it is pinned.
+ */
+#include "gq_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_GRIDPTS 64      /* candidate grid points j = 0..63 */
+#define OR_TOPCELL 62      /* cells 0..62 lie between grid points */
+#define OR_ORQ_FBITS 22    /* fraction bits of ORQ fixed-point positions */
+#define OR_PB_FBITS 16     /* fraction bits of BinGrad-pb fixed-point positions */
+
+/* ------------------------------------------------------------------------------------------ */
+/* Philox4x32-10 (counter-based generator, Salmon et al., "Parallel Random Numbers: As Easy as */
+/* 1, 2, 3", SC'11).  Written from the published definition: ten rounds of two 32x32->64      */
+/* multiplications, the key bumped by the two Weyl constants between rounds.                   */
+/* ------------------------------------------------------------------------------------------ */
+void or_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)x0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)x2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t y0 = hi1 ^ x1 ^ k0;
+        uint32_t y1 = lo1;
+        uint32_t y2 = hi0 ^ x3 ^ k1;
+        uint32_t y3 = lo0;
+        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/*
+ * Randomness of the rounding step.  [P2] "Proposed method" and [P3] (stochastic quantization)
+ * only ask for random rounding; the draw is keyed on (seed, step, worker, global element
+ * index) so that it is reproducible and independent of the launch shape.  Reading: key =
+ * (seed low word, seed high word), counter = (i/4 low word, i/4 high word, step low word,
+ * worker); element i takes output word i mod 4; U = (word >> 8) * 2^-24.
+ */
+float or_uniform(uint64_t seed, uint64_t step, uint32_t worker, int64_t i)
+{
+    uint64_t blk = (uint64_t)i >> 2;
+    uint32_t ctr[4] = {(uint32_t)blk, (uint32_t)(blk >> 32), (uint32_t)step, worker};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    or_philox4x32_10(ctr, key, out);
+    uint32_t word = out[(uint64_t)i & 3u];
+    return (float)(word >> 8) * 0x1p-24f;
+}
+
+/* floor(log2(m)) for finite m > 0, read from the binary32 encoding. */
+int or_fexpo(float m)
+{
+    uint32_t bits;
+    memcpy(&bits, &m, sizeof bits);
+    int ex = (int)((bits >> 23) & 0xffu);
+    if (ex != 0) return ex - 127;
+    uint32_t mant = bits & 0x7fffffu;
+    int msb = 31;
+    while (msb > 0 && !((mant >> msb) & 1u)) --msb;
+    return msb - 149;
+}
+
+/* Saturate to [0, 1]; NaN becomes 0. */
+static float sat01(float x)
+{
+    if (!(x > 0.0f)) return 0.0f;
+    if (x > 1.0f) return 1.0f;
+    return x;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Clipping.  [P2] "Proposed method": gradients are clipped in the distributed setting,        */
+/* notably for ORQ with few levels.  Reading: per bucket, symmetric about zero at +-c*sigma,   */
+/* sigma the population standard deviation of the bucket's values.  sigma is computed from    */
+/* exact integer sums of the values in fixed point with 20 fraction bits below the bucket's    */
+/* largest magnitude, so that it does not depend on summation order.                           */
+/* ------------------------------------------------------------------------------------------ */
+float or_clip_threshold(const float *v, int n, float c)
+{
+    float m0 = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(v[i]);
+        if (a > m0) m0 = a;
+    }
+    if (!(m0 > 0.0f) || n <= 0) return 0.0f;
+    int e = 20 - or_fexpo(m0);
+    int64_t sx = 0, sxx = 0;
+    for (int i = 0; i < n; ++i) {
+        int64_t x = llrint(ldexp((double)v[i], e));
+        sx += x;
+        sxx += x * x;
+    }
+    double mean = (double)sx / (double)n;
+    double var = (double)sxx / (double)n - mean * mean;
+    if (var < 0.0) var = 0.0;
+    double sigma = ldexp(sqrt(var), -e);
+    return (float)((double)c * sigma);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* The 64-point candidate grid shared by ORQ and BinGrad-pb: uniform from the bucket minimum   */
+/* to its maximum, both ends included (g_j = min + j*(max-min)/63, g_63 = max).  A value's     */
+/* position on the grid is kept in fixed point, floor((u - min) * 63/(max-min) * 2^F),        */
+/* clamped to [0, 63*2^F]; its cell is min(position >> F, 62).                                 */
+/* ------------------------------------------------------------------------------------------ */
+typedef struct {
+    float mn, mx, step, scale;
+    float grid[OR_GRIDPTS];
+} or_gridinfo;
+
+/* Returns 0 when the bucket is constant (min == max). */
+static int grid_setup(const float *u, int n, int fbits, or_gridinfo *gi)
+{
+    float mn = u[0], mx = u[0];
+    for (int i = 1; i < n; ++i) {
+        if (u[i] < mn) mn = u[i];
+        if (u[i] > mx) mx = u[i];
+    }
+    /* canonical zero: -0 + +0 = +0 */
+    mn = mn + 0.0f;
+    mx = mx + 0.0f;
+    gi->mn = mn;
+    gi->mx = mx;
+    if (!(mx > mn)) return 0;
+    float range = mx - mn;
+    gi->step = range / 63.0f;
+    gi->scale = (63.0f / range) * (float)(1 << fbits);
+    for (int j = 0; j < OR_GRIDPTS - 1; ++j) gi->grid[j] = mn + (float)j * gi->step;
+    gi->grid[OR_GRIDPTS - 1] = mx;
+    return 1;
+}
+
+static int32_t grid_pos(const or_gridinfo *gi, float u, int fbits)
+{
+    int32_t top = (int32_t)63 << fbits;
+    float y = (u - gi->mn) * gi->scale;
+    if (!(y > 0.0f)) return 0;
+    if (y >= (float)top) return top;
+    return (int32_t)y;
+}
+
+static int pos_cell(int32_t pos, int fbits)
+{
+    int c = pos >> fbits;
+    return c > OR_TOPCELL ? OR_TOPCELL : c;
+}
+
+int or_grid(const float *u, int n, float grid[64])
+{
+    or_gridinfo gi;
+    if (!grid_setup(u, n, OR_ORQ_FBITS, &gi)) return 0;
+    memcpy(grid, gi.grid, sizeof gi.grid);
+    return 1;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* ORQ-s.  [P2] "Proposed method" / abstract: unbiased multi-level quantization whose levels   */
+/* are chosen greedily to minimise the expected quantization variance.  Reading: the levels    */
+/* start as {min, max} (grid indices 0 and 63); each of s-2 rounds adds the grid index whose   */
+/* addition gives the smallest total variance sum (b - x)(x - a) over the bucket, ties to the  */
+/* smallest index; x in fixed point with 22 fraction bits per cell, the bracket [a, b] of a    */
+/* value being the chosen levels around its cell.                                              */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Index k of the bracket [lv[k], lv[k+1]] holding cell c (lv sorted, lv[0]=0, lv[nl-1]=63). */
+static int bracket_of(const int *lv, int nl, int c)
+{
+    int k = 0;
+    while (k + 2 < nl && lv[k + 1] <= c) ++k;
+    return k;
+}
+
+static __int128 orq_total_variance(const int32_t *pos, const int *cell, int n, const int *lv, int nl)
+{
+    __int128 tot = 0;
+    for (int i = 0; i < n; ++i) {
+        int k = bracket_of(lv, nl, cell[i]);
+        int64_t a = (int64_t)lv[k] << OR_ORQ_FBITS;
+        int64_t b = (int64_t)lv[k + 1] << OR_ORQ_FBITS;
+        tot += (__int128)(b - pos[i]) * (__int128)(pos[i] - a);
+    }
+    return tot;
+}
+
+/* Sorted insertion of c into lv[0..nl). */
+static void insert_level(int *lv, int nl, int c)
+{
+    int k = nl;
+    while (k > 0 && lv[k - 1] > c) {
+        lv[k] = lv[k - 1];
+        --k;
+    }
+    lv[k] = c;
+}
+
+/* Greedy selection; idx_out[0..s) receives the sorted grid indices.  Returns the final total
+ * variance in units of (cell * 2^-22)^2 as a double (0 for a constant bucket). */
+static double orq_select_pos(const int32_t *pos, const int *cell, int n, int s, int *lv)
+{
+    int nl = 2;
+    lv[0] = 0;
+    lv[1] = OR_GRIDPTS - 1;
+    __int128 best_v = orq_total_variance(pos, cell, n, lv, nl);
+    for (int round = 0; round < s - 2; ++round) {
+        int best_c = -1;
+        for (int c = 1; c < OR_GRIDPTS - 1; ++c) {
+            int used = 0;
+            for (int k = 0; k < nl; ++k) used |= (lv[k] == c);
+            if (used) continue;
+            int trial[OR_GRIDPTS];
+            memcpy(trial, lv, sizeof(int) * (size_t)nl);
+            insert_level(trial, nl, c);
+            __int128 v = orq_total_variance(pos, cell, n, trial, nl + 1);
+            if (best_c < 0 || v < best_v) {
+                best_c = c;
+                best_v = v;
+            }
+        }
+        insert_level(lv, nl, best_c);
+        ++nl;
+    }
+    return (double)best_v;
+}
+
+double or_orq_select(const float *u, int n, int s, int *idx_out)
+{
+    or_gridinfo gi;
+    if (!grid_setup(u, n, OR_ORQ_FBITS, &gi)) {
+        for (int k = 0; k < s; ++k) idx_out[k] = 0;
+        return 0.0;
+    }
+    int32_t *pos = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    int *cell = (int *)malloc(sizeof(int) * (size_t)n);
+    for (int i = 0; i < n; ++i) {
+        pos[i] = grid_pos(&gi, u[i], OR_ORQ_FBITS);
+        cell[i] = pos_cell(pos[i], OR_ORQ_FBITS);
+    }
+    double v = orq_select_pos(pos, cell, n, s, idx_out);
+    free(pos);
+    free(cell);
+    return v;
+}
+
+static void orq_bucket(const or_config *cfg, int worker, uint64_t step, int64_t base,
+                       const float *u, int n, uint8_t *code, float *q, float *table)
+{
+    int s = cfg->levels;
+    or_gridinfo gi;
+    if (!grid_setup(u, n, OR_ORQ_FBITS, &gi)) {
+        /* constant bucket: every level is the common value, every code 0 */
+        for (int k = 0; k < s; ++k) table[k] = gi.mn;
+        for (int i = 0; i < n; ++i) {
+            code[i] = 0;
+            q[i] = gi.mn;
+        }
+        return;
+    }
+    int32_t *pos = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    int *cell = (int *)malloc(sizeof(int) * (size_t)n);
+    for (int i = 0; i < n; ++i) {
+        pos[i] = grid_pos(&gi, u[i], OR_ORQ_FBITS);
+        cell[i] = pos_cell(pos[i], OR_ORQ_FBITS);
+    }
+    int lv[OR_GRIDPTS];
+    orq_select_pos(pos, cell, n, s, lv);
+    for (int k = 0; k < s; ++k) table[k] = gi.grid[lv[k]];
+    /* unbiased rounding inside the bracket [a, b]: up with probability (u - a)/(b - a) */
+    for (int i = 0; i < n; ++i) {
+        int k = bracket_of(lv, s, cell[i]);
+        float a = table[k], b = table[k + 1];
+        float rinv = 1.0f / (b - a);
+        float p = sat01((u[i] - a) * rinv);
+        float U = or_uniform(cfg->seed, step, (uint32_t)worker, base + i);
+        int c = k + (U < p ? 1 : 0);
+        code[i] = (uint8_t)c;
+        q[i] = table[c];
+    }
+    free(pos);
+    free(cell);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* QSGD-s / TernGrad.  [P3]: scale by the maximum magnitude and round stochastically to the    */
+/* nearest representable levels; TernGrad uses the three levels {-m, 0, m}.  Reading: per      */
+/* bucket, m = max|u|, s uniform levels m*(2k-(s-1))/(s-1), k = 0..s-1 (TernGrad is s = 3).    */
+/* The message carries m only.                                                                 */
+/* ------------------------------------------------------------------------------------------ */
+static float qsgd_ratio(int code, int s)
+{
+    return (float)(2 * code - (s - 1)) / (float)(s - 1);
+}
+
+static void qsgd_bucket(const or_config *cfg, int worker, uint64_t step, int64_t base,
+                        const float *u, int n, uint8_t *code, float *q, float *table)
+{
+    int s = cfg->levels;
+    float m = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(u[i]);
+        if (a > m) m = a;
+    }
+    table[0] = m;
+    float inv_m = m > 0.0f ? 1.0f / m : 0.0f;
+    float h = (float)(s - 1) * 0.5f;
+    for (int i = 0; i < n; ++i) {
+        float y = (u[i] * inv_m + 1.0f) * h;   /* position in level units, 0 .. s-1 */
+        int k = y > 0.0f ? (int)y : 0;
+        if (k > s - 2) k = s - 2;
+        float p = y - (float)k;
+        float U = or_uniform(cfg->seed, step, (uint32_t)worker, base + i);
+        int c = k + (U < p ? 1 : 0);
+        code[i] = (uint8_t)c;
+        q[i] = m * qsgd_ratio(c, s);
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* BinGrad-b.  [P2]: the biased binary scheme that minimises variance; its two levels adapt to */
+/* the gradient distribution.  Reading: the SSE-optimal two-level split (1-D two-means) with  */
+/* the levels at the means of each side, deterministic assignment (hence biased).  Sums are   */
+/* exact int64 in fixed point with 46 fraction bits below the bucket's largest magnitude; the  */
+/* split maximises J(k) = S_k^2/k + (S_n - S_k)^2/(n - k) (equivalently minimises the SSE),    */
+/* evaluated in binary64, ties to the smallest k, over splits between distinct values.         */
+/* ------------------------------------------------------------------------------------------ */
+static int cmp_float(const void *a, const void *b)
+{
+    float x = *(const float *)a, y = *(const float *)b;
+    return (x > y) - (x < y);
+}
+
+void or_bingrad_b_fit(const float *u, int n, float *a_out, float *b_out, float *thr, int *split)
+{
+    float m = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(u[i]);
+        if (a > m) m = a;
+    }
+    if (!(m > 0.0f)) {
+        *a_out = 0.0f;
+        *b_out = 0.0f;
+        *thr = 0.0f;
+        *split = 0;
+        return;
+    }
+    float *srt = (float *)malloc(sizeof(float) * (size_t)n);
+    memcpy(srt, u, sizeof(float) * (size_t)n);
+    qsort(srt, (size_t)n, sizeof(float), cmp_float);
+    int e = 46 - or_fexpo(m);
+    int64_t *S = (int64_t *)malloc(sizeof(int64_t) * (size_t)(n + 1));
+    S[0] = 0;
+    for (int i = 0; i < n; ++i) S[i + 1] = S[i] + llrint(ldexp((double)srt[i], e));
+    int best = -1;
+    double best_j = 0.0;
+    for (int k = 1; k < n; ++k) {
+        if (!(srt[k - 1] < srt[k])) continue;
+        double l = (double)S[k];
+        double r = (double)(S[n] - S[k]);
+        double j = l * l / (double)k + r * r / (double)(n - k);
+        if (best < 0 || j > best_j) {
+            best = k;
+            best_j = j;
+        }
+    }
+    if (best < 0) {
+        /* every value equal: one level, no split */
+        *a_out = srt[0] + 0.0f;
+        *b_out = srt[0] + 0.0f;
+        *thr = srt[0] + 0.0f;
+        *split = 0;
+    } else {
+        *a_out = (float)ldexp((double)S[best] / (double)best, -e);
+        *b_out = (float)ldexp((double)(S[n] - S[best]) / (double)(n - best), -e);
+        *thr = srt[best];
+        *split = best;
+    }
+    free(S);
+    free(srt);
+}
+
+static void bingrad_b_bucket(const float *u, int n, uint8_t *code, float *q, float *table)
+{
+    float a, b, thr;
+    int split;
+    or_bingrad_b_fit(u, n, &a, &b, &thr, &split);
+    table[0] = a;
+    table[1] = b;
+    for (int i = 0; i < n; ++i) {
+        int c = (split > 0 && u[i] >= thr) ? 1 : 0;
+        code[i] = (uint8_t)c;
+        q[i] = c ? b : a;
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* BinGrad-pb.  [P2]: the binary variant that trades some variance for less bias by a wider   */
+/* range, with a larger quantization error than BinGrad-b.  Reading ("partially biased"):     */
+/* two levels (g_A, g_B) from the 64-point grid; values between them are rounded             */
+/* stochastically (unbiased), values outside are clamped to the nearer level (biased).  The    */
+/* pair minimises the expected squared error                                                  */
+/*   sum_{x<a} (a-x)^2 + sum_{a<=x<b} (b-x)(x-a) + sum_{x>=b} (x-b)^2                         */
+/* in fixed point with 16 fraction bits per cell (exact int128), ties to the smallest (A, B).  */
+/* ------------------------------------------------------------------------------------------ */
+static void pb_select_pos(const int32_t *pos, int n, int *A_out, int *B_out)
+{
+    int bestA = -1, bestB = -1;
+    __int128 best_e = 0;
+    for (int A = 0; A < OR_GRIDPTS - 1; ++A) {
+        for (int B = A + 1; B < OR_GRIDPTS; ++B) {
+            int64_t a = (int64_t)A << OR_PB_FBITS, b = (int64_t)B << OR_PB_FBITS;
+            __int128 e = 0;
+            for (int i = 0; i < n; ++i) {
+                int64_t x = pos[i];
+                if (x < a) e += (__int128)(a - x) * (a - x);
+                else if (x >= b) e += (__int128)(x - b) * (x - b);
+                else e += (__int128)(b - x) * (x - a);
+            }
+            if (bestA < 0 || e < best_e) {
+                bestA = A;
+                bestB = B;
+                best_e = e;
+            }
+        }
+    }
+    *A_out = bestA;
+    *B_out = bestB;
+}
+
+void or_bingrad_pb_fit(const float *u, int n, int *A, int *B, float *ga, float *gb)
+{
+    or_gridinfo gi;
+    if (!grid_setup(u, n, OR_PB_FBITS, &gi)) {
+        *A = 0;
+        *B = 0;
+        *ga = gi.mn;
+        *gb = gi.mn;
+        return;
+    }
+    int32_t *pos = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    for (int i = 0; i < n; ++i) pos[i] = grid_pos(&gi, u[i], OR_PB_FBITS);
+    pb_select_pos(pos, n, A, B);
+    *ga = gi.grid[*A];
+    *gb = gi.grid[*B];
+    free(pos);
+}
+
+static void bingrad_pb_bucket(const or_config *cfg, int worker, uint64_t step, int64_t base,
+                              const float *u, int n, uint8_t *code, float *q, float *table)
+{
+    or_gridinfo gi;
+    if (!grid_setup(u, n, OR_PB_FBITS, &gi)) {
+        table[0] = gi.mn;
+        table[1] = gi.mn;
+        for (int i = 0; i < n; ++i) {
+            code[i] = 0;
+            q[i] = gi.mn;
+        }
+        return;
+    }
+    int32_t *pos = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    for (int i = 0; i < n; ++i) pos[i] = grid_pos(&gi, u[i], OR_PB_FBITS);
+    int A, B;
+    pb_select_pos(pos, n, &A, &B);
+    float a = gi.grid[A], b = gi.grid[B];
+    table[0] = a;
+    table[1] = b;
+    float rinv = 1.0f / (b - a);
+    int32_t pa = (int32_t)A << OR_PB_FBITS, pbv = (int32_t)B << OR_PB_FBITS;
+    for (int i = 0; i < n; ++i) {
+        int c;
+        if (pos[i] < pa) {
+            c = 0;
+        } else if (pos[i] >= pbv) {
+            c = 1;
+        } else {
+            float p = sat01((u[i] - a) * rinv);
+            float U = or_uniform(cfg->seed, step, (uint32_t)worker, base + i);
+            c = U < p ? 1 : 0;
+        }
+        code[i] = (uint8_t)c;
+        q[i] = c ? b : a;
+    }
+    free(pos);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Sizes and message layout.                                                                   */
+/* ------------------------------------------------------------------------------------------ */
+int or_bits(int levels)
+{
+    int b = 0;
+    while ((1 << b) < levels) ++b;
+    return b;
+}
+
+int or_table_len(int scheme, int levels)
+{
+    if (scheme == OR_QSGD || scheme == OR_TERNGRAD) return 1;
+    if (scheme == OR_BINGRAD_B || scheme == OR_BINGRAD_PB) return 2;
+    return levels;
+}
+
+int64_t or_num_buckets(const or_config *cfg)
+{
+    return (cfg->n + cfg->bucket - 1) / cfg->bucket;
+}
+
+/*
+ * A worker's message: the packed codes of every bucket, bucket after bucket (d*b/32 words
+ * each), then the level tables, bucket after bucket (L floats each), the second region
+ * starting on a 16-byte boundary and the total rounded up to 16 bytes.
+ */
+void or_message_layout(const or_config *cfg, int64_t *bytes, int64_t *codes_off, int64_t *levels_off)
+{
+    int64_t nb = or_num_buckets(cfg);
+    int64_t words = (int64_t)cfg->bucket * or_bits(cfg->levels) / 32;
+    int64_t cbytes = nb * words * 4;
+    int64_t lbytes = nb * or_table_len(cfg->scheme, cfg->levels) * 4;
+    cbytes = (cbytes + 15) / 16 * 16;
+    lbytes = (lbytes + 15) / 16 * 16;
+    *codes_off = 0;
+    *levels_off = cbytes;
+    *bytes = cbytes + lbytes;
+}
+
+/*
+ * Bit-plane packing of one bucket (b bits per code).  The bucket is cut into chunks of 128
+ * elements; in chunk m, element e = 128m + 4l + c (l = 0..31, c = 0..3) puts bit j of its
+ * code at bit l of word (m*b + j)*4 + c.  Codes of padding elements (e >= n) are 0.
+ */
+void or_pack_bucket(const or_config *cfg, const uint8_t *code, int n, uint32_t *words)
+{
+    int b = or_bits(cfg->levels);
+    int d = cfg->bucket;
+    memset(words, 0, sizeof(uint32_t) * (size_t)(d * b / 32));
+    for (int e = 0; e < n; ++e) {
+        int m = e / 128, l = (e % 128) / 4, c = e % 4;
+        for (int j = 0; j < b; ++j)
+            if ((code[e] >> j) & 1) words[(m * b + j) * 4 + c] |= 1u << l;
+    }
+}
+
+void or_unpack_bucket(const or_config *cfg, const uint32_t *words, int n, uint8_t *code)
+{
+    int b = or_bits(cfg->levels);
+    for (int e = 0; e < n; ++e) {
+        int m = e / 128, l = (e % 128) / 4, c = e % 4;
+        int v = 0;
+        for (int j = 0; j < b; ++j) v |= (int)((words[(m * b + j) * 4 + c] >> l) & 1u) << j;
+        code[e] = (uint8_t)v;
+    }
+}
+
+float or_dequant(const or_config *cfg, const float *table, int code)
+{
+    if (cfg->scheme == OR_QSGD || cfg->scheme == OR_TERNGRAD)
+        return table[0] * qsgd_ratio(code, cfg->levels);
+    return table[code];
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* One bucket of one worker.                                                                   */
+/* ------------------------------------------------------------------------------------------ */
+int or_encode_bucket(const or_config *cfg, int worker, uint64_t step, int64_t bucket,
+                     const float *v, int n, uint8_t *code, float *q, float *table)
+{
+    if (n <= 0) return 0;
+    int64_t base = bucket * (int64_t)cfg->bucket;
+    float *u = (float *)malloc(sizeof(float) * (size_t)n);
+    memcpy(u, v, sizeof(float) * (size_t)n);
+    if (cfg->clip_sigma > 0.0f) {
+        float t = or_clip_threshold(v, n, cfg->clip_sigma);
+        for (int i = 0; i < n; ++i) {
+            if (u[i] < -t) u[i] = -t;
+            if (u[i] > t) u[i] = t;
+        }
+    }
+    switch (cfg->scheme) {
+    case OR_QSGD:
+    case OR_TERNGRAD:
+        qsgd_bucket(cfg, worker, step, base, u, n, code, q, table);
+        break;
+    case OR_BINGRAD_B:
+        bingrad_b_bucket(u, n, code, q, table);
+        break;
+    case OR_BINGRAD_PB:
+        bingrad_pb_bucket(cfg, worker, step, base, u, n, code, q, table);
+        break;
+    case OR_ORQ:
+        orq_bucket(cfg, worker, step, base, u, n, code, q, table);
+        break;
+    default:
+        free(u);
+        return 1;
+    }
+    free(u);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Whole-vector calls.                                                                         */
+/* ------------------------------------------------------------------------------------------ */
+static int bucket_len(const or_config *cfg, int64_t bucket)
+{
+    int64_t lo = bucket * (int64_t)cfg->bucket;
+    int64_t hi = lo + cfg->bucket;
+    if (hi > cfg->n) hi = cfg->n;
+    return (int)(hi - lo);
+}
+
+/* Error feedback ([P1] "Quantization Schemes", [P3]): quantize v = g + r, keep r' = v - Q(v). */
+int or_encode(const or_config *cfg, int worker, uint64_t step, int64_t b0, int64_t b1,
+              const float *g, float *r, uint8_t *msg)
+{
+    int d = cfg->bucket;
+    int L = or_table_len(cfg->scheme, cfg->levels);
+    int64_t words = (int64_t)d * or_bits(cfg->levels) / 32;
+    int64_t bytes, coff, loff;
+    or_message_layout(cfg, &bytes, &coff, &loff);
+    float *v = (float *)malloc(sizeof(float) * (size_t)d);
+    float *q = (float *)malloc(sizeof(float) * (size_t)d);
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    int rc = 0;
+    for (int64_t bk = b0; bk < b1 && rc == 0; ++bk) {
+        int n = bucket_len(cfg, bk);
+        int64_t base = bk * d;
+        for (int i = 0; i < n; ++i) v[i] = (cfg->error_feedback && r) ? g[base + i] + r[base + i] : g[base + i];
+        float *table = (float *)(msg + loff) + bk * L;
+        rc = or_encode_bucket(cfg, worker, step, bk, v, n, code, q, table);
+        if (cfg->error_feedback && r)
+            for (int i = 0; i < n; ++i) r[base + i] = v[i] - q[i];
+        or_pack_bucket(cfg, code, n, (uint32_t *)(msg + coff) + bk * words);
+    }
+    free(v);
+    free(q);
+    free(code);
+    return rc;
+}
+
+/* Dequantize and aggregate ([P1] "How Gradient Quantization Works"): the mean over workers,
+ * summed in worker order in binary32, then multiplied by 1/W. */
+int or_decode_accumulate(const or_config *cfg, const uint8_t *const *msgs, int nmsgs,
+                         int64_t b0, int64_t b1, float *avg)
+{
+    int d = cfg->bucket;
+    int L = or_table_len(cfg->scheme, cfg->levels);
+    int64_t words = (int64_t)d * or_bits(cfg->levels) / 32;
+    int64_t bytes, coff, loff;
+    or_message_layout(cfg, &bytes, &coff, &loff);
+    float inv_w = 1.0f / (float)nmsgs;
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    float *acc = (float *)malloc(sizeof(float) * (size_t)d);
+    for (int64_t bk = b0; bk < b1; ++bk) {
+        int n = bucket_len(cfg, bk);
+        for (int i = 0; i < n; ++i) acc[i] = 0.0f;
+        for (int w = 0; w < nmsgs; ++w) {
+            const uint32_t *cw = (const uint32_t *)(msgs[w] + coff) + bk * words;
+            const float *table = (const float *)(msgs[w] + loff) + bk * L;
+            or_unpack_bucket(cfg, cw, n, code);
+            for (int i = 0; i < n; ++i) acc[i] = acc[i] + or_dequant(cfg, table, code[i]);
+        }
+        for (int i = 0; i < n; ++i) avg[bk * d + i] = acc[i] * inv_w;
+    }
+    free(code);
+    free(acc);
+    return 0;
+}
+
+/* The whole step for W workers: encode each worker (messages optional), average the
+ * dequantized values in worker order. */
+int or_fused_step(const or_config *cfg, uint64_t step, int64_t b0, int64_t b1,
+                  const float *const *g, float *const *r, uint8_t *const *msgs, float *avg)
+{
+    int d = cfg->bucket;
+    int W = cfg->workers;
+    int L = or_table_len(cfg->scheme, cfg->levels);
+    int64_t words = (int64_t)d * or_bits(cfg->levels) / 32;
+    int64_t bytes, coff, loff;
+    or_message_layout(cfg, &bytes, &coff, &loff);
+    float inv_w = 1.0f / (float)W;
+    float *v = (float *)malloc(sizeof(float) * (size_t)d);
+    float *q = (float *)malloc(sizeof(float) * (size_t)d);
+    float *acc = (float *)malloc(sizeof(float) * (size_t)d);
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    float table[16];
+    int rc = 0;
+    for (int64_t bk = b0; bk < b1 && rc == 0; ++bk) {
+        int n = bucket_len(cfg, bk);
+        int64_t base = bk * d;
+        for (int i = 0; i < n; ++i) acc[i] = 0.0f;
+        for (int w = 0; w < W && rc == 0; ++w) {
+            const float *gw = g[w];
+            float *rw = (cfg->error_feedback && r) ? r[w] : NULL;
+            for (int i = 0; i < n; ++i) v[i] = rw ? gw[base + i] + rw[base + i] : gw[base + i];
+            rc = or_encode_bucket(cfg, w, step, bk, v, n, code, q, table);
+            if (rw)
+                for (int i = 0; i < n; ++i) rw[base + i] = v[i] - q[i];
+            if (msgs && msgs[w]) {
+                or_pack_bucket(cfg, code, n, (uint32_t *)(msgs[w] + coff) + bk * words);
+                memcpy((float *)(msgs[w] + loff) + bk * L, table, sizeof(float) * (size_t)L);
+            }
+            for (int i = 0; i < n; ++i) acc[i] = acc[i] + q[i];
+        }
+        for (int i = 0; i < n; ++i) avg[base + i] = acc[i] * inv_w;
+    }
+    free(v);
+    free(q);
+    free(acc);
+    free(code);
+    return rc;
+}

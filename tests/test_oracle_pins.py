@@ -1,0 +1,492 @@
+"""Pins of the CPU oracle against what the pages and mathematics fix (no GPU needed).
+
+Each test checks the oracle against something other than itself: published known answers,
+the pages' worked example, brute force on tiny inputs, an independent naive greedy, Monte
+Carlo moments, closed forms and invariants.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+# ------------------------------------------------------------------------------------------
+# Philox4x32-10
+# ------------------------------------------------------------------------------------------
+def test_philox_known_answers():
+    rows = _rows("philox4x32_10_kat.txt")
+    assert len(rows) == 3
+    for r in rows:
+        v = [int(x, 16) for x in r]
+        out = O.philox(v[0:4], v[4:6])
+        assert [int(x) for x in out] == v[6:10]
+
+
+def test_uniform_statistics():
+    # 2^16 draws: mean 1/2, chi-square over 64 bins, 24-bit resolution
+    n = 1 << 16
+    u = np.array([O.uniform(7, 3, 1, i) for i in range(n)], dtype=np.float64)
+    assert u.min() >= 0.0 and u.max() < 1.0
+    assert abs(u.mean() - 0.5) < 4 * math.sqrt(1 / 12 / n)
+    h, _ = np.histogram(u, bins=64, range=(0, 1))
+    chi2 = ((h - n / 64) ** 2 / (n / 64)).sum()
+    assert chi2 < 63 + 6 * math.sqrt(2 * 63)
+    assert np.all(np.round(u * 2 ** 24) == u * 2 ** 24)
+    # distinct workers / steps give distinct streams
+    a = [O.uniform(7, 3, 1, i) for i in range(64)]
+    b = [O.uniform(7, 3, 2, i) for i in range(64)]
+    c = [O.uniform(7, 4, 1, i) for i in range(64)]
+    assert a != b and a != c
+
+
+def test_fexpo_matches_frexp():
+    rng = np.random.default_rng(0)
+    vals = np.concatenate([rng.standard_normal(2000) * 10.0 ** rng.uniform(-40, 38, 2000),
+                           [1.0, 2.0, 0.5, 1e-45, 1.4e-45, 3e-39, 1.1754942e-38, 1.1754944e-38, 3.4e38]])
+    for v in np.abs(vals.astype(np.float32)):
+        if v == 0:
+            continue
+        m, e = math.frexp(float(v))
+        assert O.fexpo(float(v)) == e - 1
+
+
+# ------------------------------------------------------------------------------------------
+# Stochastic rounding: the pages' worked example and Monte Carlo moments
+# ------------------------------------------------------------------------------------------
+def _mc(cfg, v, steps):
+    qs = np.stack([O.encode_bucket(cfg, 0, t, 0, v)[1] for t in range(steps)]).astype(np.float64)
+    return qs
+
+
+def test_worked_example_point_seven():
+    (val, lo, hi, p_up), = [[float(x) for x in r] for r in _rows("stochastic_rounding_example.txt")]
+    d = 512
+    v = np.full(d, val, dtype=np.float32)
+    v[0], v[1] = lo, hi          # ORQ-2 levels are the bucket's min and max: exactly {0, 1}
+    cfg = O.Config(O.ORQ, 2, d, 1, 1, 0.0, 42, d)
+    _, _, table = O.encode_bucket(cfg, 0, 0, 0, v)
+    assert list(table) == [lo, hi]
+    steps = 200                   # 510 draws per step: 102,000 draws
+    qs = _mc(cfg, v, steps)[:, 2:]
+    frac_up = (qs == hi).mean()
+    assert set(np.unique(qs)) <= {lo, hi}
+    sigma = math.sqrt(p_up * (1 - p_up) / qs.size)
+    assert abs(frac_up - p_up) < 3 * sigma
+    # QSGD-3 with m = 1 has levels {-1, 0, 1}: 0.7 lies between 0 and 1 as well
+    v2 = np.full(d, val, dtype=np.float32)
+    v2[0] = -1.0
+    cfgq = O.Config(O.QSGD, 3, d, 1, 1, 0.0, 42, d)
+    qq = _mc(cfgq, v2, steps)[:, 1:]
+    assert set(np.unique(qq)) <= {0.0, 1.0}
+    assert abs((qq == 1.0).mean() - p_up) < 3 * math.sqrt(0.21 / qq.size)
+
+
+def _bracket_moments(levels, u):
+    """(lower, upper) adjacent levels of each value in an ascending level list."""
+    lv = np.asarray(levels, dtype=np.float64)
+    k = np.clip(np.searchsorted(lv, u, side="right") - 1, 0, len(lv) - 2)
+    return lv[k], lv[k + 1]
+
+
+@pytest.mark.parametrize("scheme,levels", [(O.ORQ, 3), (O.ORQ, 5), (O.ORQ, 9), (O.QSGD, 5),
+                                           (O.TERNGRAD, 3), (O.QSGD, 9)])
+def test_unbiased_and_variance_monte_carlo(scheme, levels):
+    rng = np.random.default_rng(scheme * 10 + levels)
+    d = 128
+    v = (rng.laplace(0, 1e-3, d)).astype(np.float32)
+    cfg = O.Config(scheme, levels, d, 1, 1, 0.0, 99, d)
+    steps = 1000                  # 1000 draws per element, 128,000 draws
+    qs = _mc(cfg, v, steps)
+    _, _, table = O.encode_bucket(cfg, 0, 0, 0, v)
+    if scheme in (O.QSGD, O.TERNGRAD):
+        m = float(table[0])
+        lv = [m * (2 * k - (levels - 1)) / (levels - 1) for k in range(levels)]
+    else:
+        lv = [float(t) for t in table]
+    assert all(lv[i] <= lv[i + 1] for i in range(len(lv) - 1))
+    u = v.astype(np.float64)
+    a, b = _bracket_moments(lv, u)
+    var = (b - u) * (u - a)
+    # every output is a level and lies in the fitted range
+    assert qs.min() >= lv[0] and qs.max() <= lv[-1]
+    assert np.isin(qs.astype(np.float32), np.asarray(lv, dtype=np.float32)).all()
+    mean = qs.mean(axis=0)
+    se = np.sqrt(np.maximum(var, 1e-30) / steps)
+    z = (mean - u) / se
+    ok = var > 0
+    assert np.abs(z[ok]).max() < 5.5
+    assert 0.75 < np.mean(z[ok] ** 2) < 1.25
+    # deterministic where the value sits on a level
+    assert np.allclose(mean[~ok], u[~ok], rtol=0, atol=1e-6 * abs(lv[-1] - lv[0]))
+    # expected variance sum (b-x)(x-a) against the empirical one
+    emp = qs.var(axis=0).sum()
+    assert abs(emp - var.sum()) < 0.1 * var.sum()
+
+
+# ------------------------------------------------------------------------------------------
+# ORQ greedy
+# ------------------------------------------------------------------------------------------
+def _naive_orq(u, s):
+    """Independent greedy on the raw values in float64 (no fixed point, no prefix sums)."""
+    x = np.asarray(u, dtype=np.float64)
+    mn, mx = x.min(), x.max()
+    grid = mn + np.arange(64) * (mx - mn) / 63.0
+    grid[63] = mx
+
+    def total(lvset):
+        a, b = _bracket_moments(grid[sorted(lvset)], x)
+        return float(np.sum((b - x) * (x - a)))
+
+    lv = [0, 63]
+    for _ in range(s - 2):
+        best = None
+        for c in range(1, 63):
+            if c in lv:
+                continue
+            t = total(lv + [c])
+            if best is None or t < best[0]:
+                best = (t, c)
+        lv.append(best[1])
+    return sorted(lv), total(lv), total
+
+
+@pytest.mark.parametrize("s", [2, 3, 5, 9])
+def test_orq_matches_naive_greedy(s):
+    rng = np.random.default_rng(s)
+    same = 0
+    trials = 12
+    for t in range(trials):
+        n = int(rng.integers(40, 300))
+        dist = t % 3
+        if dist == 0:
+            u = rng.standard_normal(n)
+        elif dist == 1:
+            u = rng.laplace(0, 1, n)
+        else:
+            u = rng.standard_t(3, n)
+        u = (u * 1e-3).astype(np.float32)
+        var_fixed, idx = O.orq_select(u, s)
+        lv, tot, total = _naive_orq(u, s)
+        assert sorted(idx.tolist()) == idx.tolist()
+        assert idx[0] == 0 and idx[-1] == 63
+        mine = total(list(idx))
+        assert mine <= tot * (1 + 1e-5) + 1e-30
+        same += list(idx) == lv
+    assert same >= trials - 1
+
+
+def test_orq_greedy_nested_and_monotone():
+    rng = np.random.default_rng(5)
+    u = (rng.standard_normal(512) * 1e-3).astype(np.float32)
+    prev_idx, prev_var = None, None
+    for s in range(2, 12):
+        var, idx = O.orq_select(u, s)
+        if prev_idx is not None:
+            assert set(prev_idx.tolist()) <= set(idx.tolist())
+            assert var <= prev_var
+        prev_idx, prev_var = idx, var
+
+
+def test_orq_three_point_special_case():
+    # values only on grid points {g_0, g_k, g_63}: ORQ-3 picks k, zero variance, no randomness
+    d = 256
+    k = 23
+    lo, hi = -0.5, 1.0
+    rng = np.random.default_rng(3)
+    ok, grid = O.grid(np.array([lo, hi], dtype=np.float32))
+    assert ok
+    v = grid[rng.choice([0, k, 63], size=d)].astype(np.float32)
+    v[0], v[1], v[2] = grid[0], grid[k], grid[63]
+    var, idx = O.orq_select(v, 3)
+    assert idx.tolist() == [0, k, 63]
+    assert var == 0.0
+    cfg = O.Config(O.ORQ, 3, d, 1, 1, 0.0, 5, d)
+    for step in range(4):
+        code, q, table = O.encode_bucket(cfg, 0, step, 0, v)
+        assert np.array_equal(q, v)
+
+
+def test_orq2_is_min_max():
+    rng = np.random.default_rng(8)
+    u = (rng.standard_normal(300)).astype(np.float32)
+    cfg = O.Config(O.ORQ, 2, 512, 1, 1, 0.0, 1, 300)
+    _, q, table = O.encode_bucket(cfg, 0, 0, 0, u)
+    assert table[0] == u.min() and table[1] == u.max()
+    assert set(np.unique(q)) <= {u.min(), u.max()}
+
+
+def test_orq_constant_bucket():
+    cfg = O.Config(O.ORQ, 5, 128, 1, 1, 0.0, 1, 128)
+    v = np.full(128, 0.25, dtype=np.float32)
+    code, q, table = O.encode_bucket(cfg, 0, 0, 0, v)
+    assert (code == 0).all() and (q == 0.25).all() and (table == 0.25).all()
+
+
+# ------------------------------------------------------------------------------------------
+# BinGrad-b: brute force over every threshold (exact rational arithmetic)
+# ------------------------------------------------------------------------------------------
+def _sse_split(vals, k):
+    left, right = vals[:k], vals[k:]
+    fl = [Fraction(float(x)) for x in left]
+    fr = [Fraction(float(x)) for x in right]
+    ml = sum(fl) / len(fl)
+    mr = sum(fr) / len(fr)
+    return sum((x - ml) ** 2 for x in fl) + sum((x - mr) ** 2 for x in fr)
+
+
+def test_bingrad_b_brute_force():
+    rng = np.random.default_rng(11)
+    for t in range(60):
+        n = int(rng.integers(2, 17))
+        if t % 4 == 0:
+            u = rng.choice([-1.0, 0.5, 2.0], size=n)      # many ties
+        else:
+            u = rng.standard_normal(n) * 10.0 ** rng.uniform(-5, 1)
+        u = u.astype(np.float32)
+        a, b, thr, split = O.bingrad_b_fit(u)
+        srt = np.sort(u)
+        cands = [k for k in range(1, n) if srt[k - 1] < srt[k]]
+        if not cands:
+            assert split == 0 and a == b == srt[0]
+            continue
+        best = min(_sse_split(srt, k) for k in cands)
+        mine = _sse_split(srt, split)
+        assert srt[split - 1] < srt[split] and thr == srt[split]
+        assert float(mine) <= float(best) * (1 + 1e-9) + 1e-300
+        # levels are the side means (rounded to binary32)
+        ml = float(sum(Fraction(float(x)) for x in srt[:split]) / split)
+        mr = float(sum(Fraction(float(x)) for x in srt[split:]) / (n - split))
+        assert abs(a - ml) <= 2e-7 * max(abs(ml), 1e-30) and abs(b - mr) <= 2e-7 * max(abs(mr), 1e-30)
+        # Lloyd condition: every value is at least as near its own level
+        for x in srt[:split]:
+            assert abs(float(x) - ml) <= abs(float(x) - mr) * (1 + 1e-6) + 1e-12 * abs(mr - ml)
+        for x in srt[split:]:
+            assert abs(float(x) - mr) <= abs(float(x) - ml) * (1 + 1e-6) + 1e-12 * abs(mr - ml)
+
+
+def test_bingrad_b_codes_deterministic():
+    rng = np.random.default_rng(12)
+    v = (rng.standard_normal(512) * 1e-3).astype(np.float32)
+    cfg = O.Config(O.BINGRAD_B, 2, 512, 1, 1, 0.0, 3, 512)
+    c0, q0, t0 = O.encode_bucket(cfg, 0, 0, 0, v)
+    c1, q1, t1 = O.encode_bucket(cfg, 0, 7, 0, v)
+    assert np.array_equal(c0, c1) and np.array_equal(q0, q1)
+    a, b, thr, _ = O.bingrad_b_fit(v)
+    assert np.array_equal(c0, (v >= thr).astype(np.uint8))
+
+
+# ------------------------------------------------------------------------------------------
+# BinGrad-pb: brute force over every grid pair, and the b <= pb ordering of [P2]
+# ------------------------------------------------------------------------------------------
+def _pb_error(x, a, b):
+    x = np.asarray(x, dtype=np.float64)
+    e = np.where(x < a, (a - x) ** 2, np.where(x >= b, (x - b) ** 2, (b - x) * (x - a)))
+    return float(e.sum())
+
+
+def test_bingrad_pb_brute_force():
+    rng = np.random.default_rng(13)
+    for t in range(8):
+        n = int(rng.integers(8, 40))
+        u = (rng.standard_t(3, n) * 1e-3).astype(np.float32)
+        A, B, ga, gb = O.bingrad_pb_fit(u)
+        x = u.astype(np.float64)
+        mn, mx = x.min(), x.max()
+        grid = mn + np.arange(64) * (mx - mn) / 63.0
+        grid[63] = mx
+        best = min(_pb_error(x, grid[i], grid[j]) for i in range(63) for j in range(i + 1, 64))
+        assert 0 <= A < B <= 63
+        assert _pb_error(x, grid[A], grid[B]) <= best * (1 + 1e-4) + 1e-30
+
+
+def test_bingrad_b_error_below_pb():
+    """[P2] Key findings: BinGrad-b's quantization error is lower than BinGrad-pb's."""
+    rng = np.random.default_rng(14)
+    for t in range(10):
+        n = 128
+        u = [rng.standard_normal(n), rng.laplace(0, 1, n), rng.standard_t(3, n)][t % 3]
+        u = (u * 1e-3).astype(np.float32)
+        a, b, thr, split = O.bingrad_b_fit(u)
+        x = u.astype(np.float64)
+        sse_b = float(np.sum(np.where(x >= thr, (x - b) ** 2, (x - a) ** 2)))
+        _, _, ga, gb = O.bingrad_pb_fit(u)
+        assert sse_b <= _pb_error(x, ga, gb) * (1 + 1e-6)
+
+
+def test_bingrad_pb_unbiased_inside_range():
+    rng = np.random.default_rng(15)
+    d = 128
+    v = (rng.standard_normal(d) * 1e-3).astype(np.float32)
+    cfg = O.Config(O.BINGRAD_PB, 2, d, 1, 1, 0.0, 17, d)
+    qs = _mc(cfg, v, 600)
+    _, _, table = O.encode_bucket(cfg, 0, 0, 0, v)
+    a, b = float(table[0]), float(table[1])
+    x = v.astype(np.float64)
+    inside = (x > a) & (x < b)
+    assert inside.sum() > 10
+    mean = qs.mean(axis=0)
+    se = np.sqrt(np.maximum((b - x) * (x - a), 0) / qs.shape[0])
+    z = (mean[inside] - x[inside]) / se[inside]
+    assert np.abs(z).max() < 5.5
+    assert np.all(mean[x <= a] == a) and np.all(mean[x >= b] == b)
+
+
+# ------------------------------------------------------------------------------------------
+# QSGD / TernGrad closed forms
+# ------------------------------------------------------------------------------------------
+def test_qsgd_levels_and_exact_points():
+    d = 128
+    for s in (3, 5, 9):
+        m = 0.75
+        levels = [m * (2 * k - (s - 1)) / (s - 1) for k in range(s)]
+        v = np.array([levels[i % s] for i in range(d)], dtype=np.float32)
+        cfg = O.Config(O.QSGD, s, d, 1, 1, 0.0, 2, d)
+        for step in range(3):
+            code, q, table = O.encode_bucket(cfg, 0, step, 0, v)
+            assert table[0] == np.float32(m)
+            assert np.array_equal(q, v)                 # values on levels are exact
+            assert np.array_equal(code, np.arange(d) % s)
+
+
+def test_terngrad_is_qsgd3():
+    rng = np.random.default_rng(16)
+    v = (rng.standard_normal(512) * 1e-3).astype(np.float32)
+    a = O.encode_bucket(O.Config(O.TERNGRAD, 3, 512, 1, 1, 0.0, 4, 512), 0, 2, 3, v)
+    b = O.encode_bucket(O.Config(O.QSGD, 3, 512, 1, 1, 0.0, 4, 512), 0, 2, 3, v)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+    m = float(np.abs(v).max())
+    assert set(np.unique(a[1]).tolist()) <= {-m, 0.0, m}
+
+
+def test_zero_bucket_all_schemes():
+    v = np.zeros(256, dtype=np.float32)
+    for sch, s in [(O.QSGD, 5), (O.TERNGRAD, 3), (O.BINGRAD_B, 2), (O.BINGRAD_PB, 2), (O.ORQ, 5)]:
+        code, q, table = O.encode_bucket(O.Config(sch, s, 256, 1, 1, 0.0, 1, 256), 0, 0, 0, v)
+        assert (q == 0).all()
+
+
+# ------------------------------------------------------------------------------------------
+# Clipping, packing, error feedback, aggregation
+# ------------------------------------------------------------------------------------------
+def test_clip_threshold_is_c_sigma():
+    rng = np.random.default_rng(17)
+    for t in range(20):
+        n = int(rng.integers(2, 600))
+        v = (rng.standard_t(3, n) * 10.0 ** rng.uniform(-6, 0)).astype(np.float32)
+        T = O.clip_threshold(v, 2.5)
+        sigma = v.astype(np.float64).std()
+        assert abs(T - 2.5 * sigma) <= 2e-5 * 2.5 * sigma + 1e-30
+    assert O.clip_threshold(np.zeros(10, dtype=np.float32), 2.5) == 0.0
+    v = (rng.standard_normal(512) * 1e-3).astype(np.float32)
+    v[5] = 1.0
+    cfg = O.Config(O.ORQ, 3, 512, 1, 1, 2.5, 1, 512)
+    _, q, table = O.encode_bucket(cfg, 0, 0, 0, v)
+    T = O.clip_threshold(v, 2.5)
+    assert table[-1] <= T and table[0] >= -T and np.abs(q).max() <= T
+
+
+@pytest.mark.parametrize("levels", [2, 3, 4, 5, 9, 16])
+def test_pack_roundtrip(levels):
+    rng = np.random.default_rng(levels)
+    for d in (128, 512, 2048):
+        for n in (d, d - 1, 40, 1):
+            cfg = O.Config(O.ORQ, levels, d, 1, 1, 0.0, 0, n)
+            code = rng.integers(0, levels, n).astype(np.uint8)
+            words = O.pack_bucket(cfg, code)
+            assert words.size == d * O.bits(levels) // 32
+            assert np.array_equal(O.unpack_bucket(cfg, words, n), code)
+            ones = sum(bin(int(w)).count("1") for w in words)
+            assert ones == sum(bin(int(c)).count("1") for c in code)
+            if n < d:  # padding codes are zero
+                assert np.array_equal(O.unpack_bucket(cfg, words, d)[n:], np.zeros(d - n, np.uint8))
+
+
+def test_error_feedback_telescopes():
+    """[P3] error feedback: nothing is lost, only delayed: sum_t Q_t = sum_t g_t + r_0 - r_T."""
+    rng = np.random.default_rng(18)
+    n, d, T = 1000, 128, 6
+    cfg = O.Config(O.ORQ, 3, d, 1, 1, 0.0, 9, n)
+    r = np.zeros(n, dtype=np.float32)
+    r0 = r.copy()
+    gsum = np.zeros(n)
+    qsum = np.zeros(n)
+    for t in range(T):
+        g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+        gsum += g
+        rin = r.copy()
+        msg = O.encode(cfg, 0, t, g, r)
+        avg = O.decode_accumulate(O.Config(O.ORQ, 3, d, 1, 1, 0.0, 9, n), [msg])
+        qsum += avg
+        assert np.allclose(avg, (g + rin) - r, rtol=0, atol=1e-9)
+    assert np.allclose(qsum, gsum + r0 - r, rtol=0, atol=5e-9)
+
+
+def test_fused_equals_encode_then_decode():
+    rng = np.random.default_rng(19)
+    n, d, W = 1000, 128, 3
+    for sch, s in [(O.ORQ, 5), (O.QSGD, 5), (O.BINGRAD_B, 2), (O.BINGRAD_PB, 2)]:
+        cfg = O.Config(sch, s, d, W, 1, 0.0, 21, n)
+        gs = [(rng.standard_normal(n) * 1e-3).astype(np.float32) for _ in range(W)]
+        rs = [(rng.standard_normal(n) * 1e-5).astype(np.float32) for _ in range(W)]
+        rs2 = [r.copy() for r in rs]
+        avg, msgs = O.fused_step(cfg, 4, gs, rs)
+        msgs2 = [O.encode(cfg, w, 4, gs[w], rs2[w]) for w in range(W)]
+        avg2 = O.decode_accumulate(cfg, msgs2)
+        assert all(np.array_equal(a, b) for a, b in zip(msgs, msgs2))
+        assert all(np.array_equal(a, b) for a, b in zip(rs, rs2))
+        assert np.array_equal(avg, avg2)
+        # the average is the mean of the workers' dequantized values, read back from the
+        # messages bucket by bucket
+        _, coff, loff = O.message_layout(cfg)
+        L = O.table_len(sch, s)
+        wpb = d * O.bits(s) // 32
+        deq = np.zeros((W, n))
+        for w in range(W):
+            words = msgs[w][coff:loff].view(np.uint32)
+            tables = msgs[w][loff:].view(np.float32)
+            for bk in range(O.num_buckets(cfg)):
+                nb_ = min(d, n - bk * d)
+                codes = O.unpack_bucket(cfg, words[bk * wpb:(bk + 1) * wpb], nb_)
+                tab = tables[bk * L:(bk + 1) * L]
+                deq[w, bk * d:bk * d + nb_] = [O.dequant(cfg, tab, int(c)) for c in codes]
+        assert np.allclose(avg, deq.mean(axis=0), rtol=1e-6, atol=1e-12)
+
+
+def test_message_sizes_and_compression():
+    rows = _rows("compression_ratios.txt")
+    for s, bits, ratio in rows[:2]:
+        assert round(32 / math.log2(int(s)), 1) == float(ratio)
+    assert O.bits(3) == 2 and O.bits(5) == 3 and O.bits(9) == 4 and O.bits(2) == 1
+    n = 512 * 1000
+    cfg = O.Config(O.ORQ, 5, 512, 1, 1, 0.0, 0, n)
+    nbytes, coff, loff = O.message_layout(cfg)
+    assert loff == n * 3 // 8 and nbytes == loff + 1000 * 5 * 4
+    assert abs(32 * n / (8 * nbytes) - 32 / (3 + 5 * 32 / 512)) < 1e-9
+
+
+def test_tie_rules():
+    # Only the two end values: every candidate leaves the variance at 0, so ORQ must take the
+    # smallest unused grid indices, one per round.
+    u = np.array([-1.0, 2.0] * 50, dtype=np.float32)
+    assert O.orq_select(u, 3)[1].tolist() == [0, 1, 63]
+    assert O.orq_select(u, 5)[1].tolist() == [0, 1, 2, 3, 63]
+    # {-1, 0, 1}: the splits after the first and after the second value have equal SSE (1/2);
+    # the smaller split wins.
+    a, b, thr, split = O.bingrad_b_fit(np.array([1.0, -1.0, 0.0], dtype=np.float32))
+    assert (split, thr, a, b) == (1, 0.0, -1.0, 0.5)
+    # BinGrad-pb on the integer grid 0..63 (min 0, max 63): the pairs (9, 51) and (9, 52) both
+    # give the least expected squared error (663, found by exhaustive search); the smaller wins.
+    A, B, ga, gb = O.bingrad_pb_fit(np.array([0.0, 8.0, 32.0, 63.0], dtype=np.float32))
+    assert (A, B, ga, gb) == (9, 51, 9.0, 51.0)
