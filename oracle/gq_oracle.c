@@ -336,8 +336,10 @@ static void qsgd_bucket(const or_config *cfg, int worker, uint64_t step, int64_t
     float h = (float)(s - 1) * 0.5f;
     for (int i = 0; i < n; ++i) {
         float y = (u[i] * inv_m + 1.0f) * h;   /* position in level units, 0 .. s-1 */
-        int k = y > 0.0f ? (int)y : 0;
-        if (k > s - 2) k = s - 2;
+        /* k = trunc(y) clamped to [0, s-2]; y may be infinite (1/m overflows for a subnormal
+         * m) or NaN (0 * inf), so the clamp is taken before any conversion to int */
+        int k = 0;
+        if (y > 0.0f) k = (y >= (float)(s - 2)) ? s - 2 : (int)y;
         float p = y - (float)k;
         float U = or_uniform(cfg->seed, step, (uint32_t)worker, base + i);
         int c = k + (U < p ? 1 : 0);
@@ -697,8 +699,45 @@ int or_decode_accumulate(const or_config *cfg, const uint8_t *const *msgs, int n
     return 0;
 }
 
-/* The whole step for W workers: encode each worker (messages optional), average the
- * dequantized values in worker order. */
+/* One bucket of the whole step.  g[w] / r_in[w] hold the n values of bucket `bucket` of
+ * worker w (r_in NULL when error feedback is off).  Outputs (each may be NULL): r_out[w] the new
+ * residuals, words[w] the packed codes (d*b/32 words), tables[w] the level table (L floats),
+ * avg the n averaged values. */
+int or_fused_bucket(const or_config *cfg, uint64_t step, int64_t bucket, int n,
+                    const float *const *g, const float *const *r_in, float *const *r_out,
+                    uint32_t *const *words, float *const *tables, float *avg)
+{
+    int W = cfg->workers;
+    float inv_w = 1.0f / (float)W;
+    float *v = (float *)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+    float *q = (float *)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+    float *acc = (float *)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+    uint8_t *code = (uint8_t *)malloc((size_t)(n > 0 ? n : 1));
+    float table[16];
+    int rc = 0;
+    for (int i = 0; i < n; ++i) acc[i] = 0.0f;
+    for (int w = 0; w < W && rc == 0; ++w) {
+        int ef = cfg->error_feedback && r_in && r_in[w];
+        for (int i = 0; i < n; ++i) v[i] = ef ? g[w][i] + r_in[w][i] : g[w][i];
+        rc = or_encode_bucket(cfg, w, step, bucket, v, n, code, q, table);
+        if (ef && r_out && r_out[w])
+            for (int i = 0; i < n; ++i) r_out[w][i] = v[i] - q[i];
+        if (words && words[w]) or_pack_bucket(cfg, code, n, words[w]);
+        if (tables && tables[w])
+            memcpy(tables[w], table, sizeof(float) * (size_t)or_table_len(cfg->scheme, cfg->levels));
+        for (int i = 0; i < n; ++i) acc[i] = acc[i] + q[i];
+    }
+    if (avg)
+        for (int i = 0; i < n; ++i) avg[i] = acc[i] * inv_w;
+    free(v);
+    free(q);
+    free(acc);
+    free(code);
+    return rc;
+}
+
+/* The whole step for W workers over the bucket range [b0, b1): every worker quantized
+ * (messages optional), the dequantized values averaged in worker order. */
 int or_fused_step(const or_config *cfg, uint64_t step, int64_t b0, int64_t b1,
                   const float *const *g, float *const *r, uint8_t *const *msgs, float *avg)
 {
@@ -708,35 +747,24 @@ int or_fused_step(const or_config *cfg, uint64_t step, int64_t b0, int64_t b1,
     int64_t words = (int64_t)d * or_bits(cfg->levels) / 32;
     int64_t bytes, coff, loff;
     or_message_layout(cfg, &bytes, &coff, &loff);
-    float inv_w = 1.0f / (float)W;
-    float *v = (float *)malloc(sizeof(float) * (size_t)d);
-    float *q = (float *)malloc(sizeof(float) * (size_t)d);
-    float *acc = (float *)malloc(sizeof(float) * (size_t)d);
-    uint8_t *code = (uint8_t *)malloc((size_t)d);
-    float table[16];
+    const float *gb[64];
+    const float *rb[64];
+    float *ro[64];
+    uint32_t *wb[64];
+    float *tb[64];
+    int ef = cfg->error_feedback && r;
     int rc = 0;
     for (int64_t bk = b0; bk < b1 && rc == 0; ++bk) {
         int n = bucket_len(cfg, bk);
         int64_t base = bk * d;
-        for (int i = 0; i < n; ++i) acc[i] = 0.0f;
-        for (int w = 0; w < W && rc == 0; ++w) {
-            const float *gw = g[w];
-            float *rw = (cfg->error_feedback && r) ? r[w] : NULL;
-            for (int i = 0; i < n; ++i) v[i] = rw ? gw[base + i] + rw[base + i] : gw[base + i];
-            rc = or_encode_bucket(cfg, w, step, bk, v, n, code, q, table);
-            if (rw)
-                for (int i = 0; i < n; ++i) rw[base + i] = v[i] - q[i];
-            if (msgs && msgs[w]) {
-                or_pack_bucket(cfg, code, n, (uint32_t *)(msgs[w] + coff) + bk * words);
-                memcpy((float *)(msgs[w] + loff) + bk * L, table, sizeof(float) * (size_t)L);
-            }
-            for (int i = 0; i < n; ++i) acc[i] = acc[i] + q[i];
+        for (int w = 0; w < W; ++w) {
+            gb[w] = g[w] + base;
+            rb[w] = ef ? r[w] + base : NULL;
+            ro[w] = ef ? r[w] + base : NULL;
+            wb[w] = (msgs && msgs[w]) ? (uint32_t *)(msgs[w] + coff) + bk * words : NULL;
+            tb[w] = (msgs && msgs[w]) ? (float *)(msgs[w] + loff) + bk * L : NULL;
         }
-        for (int i = 0; i < n; ++i) avg[base + i] = acc[i] * inv_w;
+        rc = or_fused_bucket(cfg, step, bk, n, gb, ef ? rb : NULL, ef ? ro : NULL, wb, tb, avg + base);
     }
-    free(v);
-    free(q);
-    free(acc);
-    free(code);
     return rc;
 }
