@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Throughput of the bucketed gradient-quantization step on B200.
+
+One step = one pass of the whole hot path over one batch: for each of W simulated workers,
+error feedback (v = g + r), per-bucket level fit, Philox stochastic rounding, bit-plane packing
+into the worker's message, residual update, and the decode + average of the W dequantized
+gradients (gq_fused_step, messages written).
+
+Default workload: 1e9-element fp32 gradient per worker (1000 blocks of 1e6 elements, block
+sigma log-uniform in [1e-5, 1e-2]), W = 8 workers on one GPU, ORQ-5, d = 512, error feedback
+on: 71 GB resident in HBM, far larger than L2.  Metric: gradient worker-elements per second.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gq|reference]
+
+--impl reference times the CPU oracle (plain C, all host cores) on bounded samples of the same
+workload.  With N > 1 (torchrun) every rank runs an independent replica on its GPU: the path
+has no exchange between GPUs.
+"""
+import argparse
+import concurrent.futures as cf
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gradient elems/s (encode+pack+decode+sum), ORQ-5 d=512; % of HBM peak"
+UNIT = "elem/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="gq", choices=["gq", "reference"])
+    ap.add_argument("--workload", default="blocks1b")
+    ap.add_argument("--scheme", default="orq")
+    ap.add_argument("--levels", type=int, default=5)
+    ap.add_argument("--bucket", type=int, default=512)
+    ap.add_argument("--clip", type=float, default=0.0)
+    ap.add_argument("--elements", type=int, default=0, help="truncate the workload (profiling runs)")
+    ap.add_argument("--no-msgs", action="store_true", help="do not write the messages")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------------
+# bookkeeping shared by both arms
+# ---------------------------------------------------------------------------------------------
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def bytes_per_worker_elem(scheme_id, levels, d, W, ef, msgs):
+    """Algorithmic HBM bytes per worker-element of the fused step: read g (and r), write r',
+    the message (b/8 bits + level table share) and the worker's share of the average."""
+    bits = (levels - 1).bit_length()
+    L = 1 if scheme_id in (0, 1) else (2 if scheme_id in (2, 3) else levels)
+    b = 4.0 + (8.0 if ef else 0.0) + 4.0 / W
+    if msgs:
+        b += bits / 8.0 + 4.0 * L / d
+    return b
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gradient_quantization_communication_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel_key):
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel_key)
+    except Exception:
+        return None
+    if rec and rec.get("source_hash") == source_hash():
+        return rec
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region (one GPU)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = bus_id
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+
+    def start(self):
+        cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.bus_id:
+            cmd += ["-i", self.bus_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [ln.split(", ") for ln in self.out.read().splitlines() if ln.strip()]
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, r[5:9]):
+                if val.strip() == "Active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def pci_bus_id(dev):
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------------------------
+def oracle_sample_rate(wl, args, gs_host, nbuckets, threads):
+    """Worker-elements per second of the oracle's fused step over the first nbuckets buckets of
+    every worker (host arrays gs_host), split over `threads` host threads."""
+    import numpy as np
+
+    import oracle as O
+    d = args.bucket
+    n = nbuckets * d
+    sid = O.SCHEMES[args.scheme]
+    cfg = O.Config(sid, args.levels, d, wl.workers, int(wl.error_feedback), args.clip, wl.rounding_seed, n)
+    gs = [np.ascontiguousarray(g[:n]) for g in gs_host]
+    rs = [np.zeros(n, np.float32) for _ in gs] if wl.error_feedback else None
+    bounds = [(nbuckets * i // threads, nbuckets * (i + 1) // threads) for i in range(threads)]
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda b: O.fused_step(cfg, 0, gs, rs, not args.no_msgs, b[0], b[1]), bounds))
+    dt = time.perf_counter() - t0
+    return wl.workers * n / dt, dt
+
+
+def host_sample(wl_name, workers, nelem):
+    import torch
+
+    from gradient_quantization_communication_b200 import synth
+    return [synth.gradient(wl_name, w, 0, n=nelem).numpy() for w in range(workers)]
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def calibrated_buckets(wl, args, gs_host, threads, seconds):
+    probe = 8 * threads
+    rate, dt = oracle_sample_rate(wl, args, gs_host, probe, threads)
+    per_bucket = dt / probe
+    return max(threads, int(seconds / per_bucket)), rate
+
+
+# ---------------------------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from gradient_quantization_communication_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    threads = cpu_threads()
+    max_buckets = 64 * threads * 8
+    gs_host = host_sample(args.workload, wl.workers, max_buckets * args.bucket)
+    # size each step to about half a second of work on all host cores
+    nbk, _ = calibrated_buckets(wl, args, gs_host, threads, 0.5)
+    nbk = min(nbk, max_buckets)
+    for _ in range(args.warmup):
+        oracle_sample_rate(wl, args, gs_host, nbk, threads)
+    times = []
+    for _ in range(args.steps):
+        _, dt = oracle_sample_rate(wl, args, gs_host, nbk, threads)
+        times.append(dt)
+    total = sum(times)
+    value = wl.workers * nbk * args.bucket * args.steps / total
+    sample = "first %d buckets (d=%d) of each of the %d workers per step" % (nbk, args.bucket, wl.workers)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(args, wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(args, wl):
+    return {"workload": "%s: %d fp32 elements x W=%d workers, %s-%d, d=%d, error feedback %s%s" % (
+        args.workload, wl.n, wl.workers, args.scheme, args.levels, args.bucket,
+        "on" if wl.error_feedback else "off", (", clip %.1f sigma" % args.clip) if args.clip else ""),
+        "elements": wl.n, "workers": wl.workers, "scheme": args.scheme, "levels": args.levels,
+        "bucket": args.bucket, "messages_written": not args.no_msgs,
+        "l2": "inputs larger than L2 (working set far above 126 MB)",
+        "gradients": "drawn once in HBM before timing; the residual evolves every step"}
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+def run_gq(args):
+    import torch
+    import torch.distributed as dist
+
+    import gradient_quantization_communication_b200.gq as G
+    from gradient_quantization_communication_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = synth.WORKLOADS[args.workload]
+    if args.elements:
+        wl = dataclasses.replace(wl, n=min(wl.n, args.elements))
+    W, n, d, ef = wl.workers, wl.n, args.bucket, wl.error_feedback
+    sid = G.SCHEMES[args.scheme]
+    cfg = G.gq_config(sid, args.levels, d, W, ef, args.clip, wl.rounding_seed, n)
+    plan = G.Plan(cfg)
+    stream = torch.cuda.current_stream()
+    g = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
+    for w in range(W):
+        synth.gradient(args.workload, w, 0, out=g[w])
+    r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)] if ef else None
+    write_msgs = not args.no_msgs or d > 512
+    msgs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)] if write_msgs else None
+    avg = torch.empty(n, dtype=torch.float32, device=dev)
+    launches_per_step = 1 if d <= 512 else W + 1
+
+    def step(t):
+        G.gq_fused_step(plan.handle, t, g, r, msgs, avg, stream)
+
+    for t in range(args.warmup):
+        step(t)
+    torch.cuda.synchronize()
+    if G.gq_plan_status(plan.handle, stream) != G.GQ_OK:
+        raise RuntimeError("non-finite input in the benchmark workload")
+
+    sampler = ClockSampler(pci_bus_id(dev)) if rank == 0 else None
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        step(args.warmup + k)
+        ev[k][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * W * n * args.steps / (elapsed_ms / 1000.0)
+
+    bpe = bytes_per_worker_elem(sid, args.levels, d, W, ef, write_msgs)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = bpe * W * n / (per_launch_ms / 1000.0) / 1e9 if d <= 512 else None
+    kernel_key = "fused_%s%d_d%d_w%d" % (args.scheme, args.levels, d, W)
+    traffic = traffic_record(kernel_key)
+    roofline = None
+    if achieved is not None:
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                    "traffic": traffic["bytes_per_launch"] if traffic else None,
+                    "algorithmic_bytes_per_launch": bpe * W * n, "kernel": kernel_key}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, G, plan, W, n, g, r, msgs, avg, dev, stream, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = run_cpu_baseline(args, wl, g)
+
+    plan.close()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(args, wl),
+            "hbm_gbs_achieved": round(bpe * W * n * world / (ms_per_step / 1000.0) / 1e9 / world, 1),
+            "pct_hbm_peak": round(100.0 * bpe * W * n / (ms_per_step / 1000.0) / 1e9 / peak, 2),
+            "bytes_per_worker_elem": bpe,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, G, plan, W, n, g, r, msgs, avg, dev, stream, world):
+    """The same step through the C ABI with the gradients in pinned host memory: every step
+    copies the W gradients host -> device, runs gq_fused_step and reads the average back."""
+    import torch
+    need = 4 * (W + 1) * n
+    try:
+        with open("/proc/meminfo") as f:
+            avail = 1024 * int(next(ln for ln in f if ln.startswith("MemAvailable")).split()[1])
+    except Exception:
+        avail = None
+    if avail is not None and avail < 1.5 * need:
+        return {"value": None, "unit": UNIT, "error": "host memory: %d GB available, %d GB of pinned buffers needed"
+                % (avail >> 30, need >> 30)}
+    try:
+        host_g = [torch.empty(n, dtype=torch.float32, pin_memory=True) for _ in range(W)]
+        host_avg = torch.empty(n, dtype=torch.float32, pin_memory=True)
+    except Exception as e:  # host memory
+        return {"value": None, "unit": UNIT, "error": "pinned host allocation failed: %s" % str(e)[:80]}
+    for w in range(W):
+        host_g[w].copy_(g[w])
+
+    def step(t):
+        for w in range(W):
+            g[w].copy_(host_g[w], non_blocking=True)
+        G.gq_fused_step(plan.handle, 1000 + t, g, r, msgs, avg, stream)
+        host_avg.copy_(avg, non_blocking=True)
+
+    step(0)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for t in range(args.e2e_steps):
+        step(1 + t)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    del host_g, host_avg
+    return {"value": world * W * n * args.e2e_steps / (ms / 1000.0), "unit": UNIT,
+            "h2d_bytes_per_step": 4 * W * n, "d2h_bytes_per_step": 4 * n, "steps": args.e2e_steps}
+
+
+def run_cpu_baseline(args, wl, g):
+    threads = cpu_threads()
+    max_buckets = 64 * threads * 16
+    nelem = min(wl.n, max_buckets * args.bucket)
+    gs_host = [x[:nelem].cpu().numpy() for x in g]
+    nbk, _ = calibrated_buckets(wl, args, gs_host, threads, args.cpu_seconds)
+    nbk = min(nbk, nelem // args.bucket)
+    rate, dt = oracle_sample_rate(wl, args, gs_host, nbk, threads)
+    return {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "seconds": round(dt, 2),
+            "sample": "first %d buckets (d=%d) of each of the %d workers, one step" % (nbk, args.bucket, wl.workers)}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

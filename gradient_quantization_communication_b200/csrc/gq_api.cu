@@ -1,0 +1,277 @@
+// gq_api.cu -- host side of the C ABI declared in include/gq.h: argument checks, the plan,
+// kernel selection and the status word.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "gq_internal.h"
+
+struct gq_plan {
+    gq_config_t cfg;  // normalised (levels filled in)
+    int bits;
+    int L;
+    int64_t nb;
+    int tail;
+    size_t msg_bytes, codes_off, levels_off;
+    int device;
+    unsigned int *status;  // device word
+};
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int bits_for(int s)
+{
+    int b = 0;
+    while ((1 << b) < s) ++b;
+    return b;
+}
+
+int table_len(int scheme, int s)
+{
+    if (scheme == GQ_QSGD || scheme == GQ_TERNGRAD) return 1;
+    if (scheme == GQ_BINGRAD_B || scheme == GQ_BINGRAD_PB) return 2;
+    return s;
+}
+
+// Validates *in and writes the normalised configuration to *out.
+gq_status_t normalise(const gq_config_t *in, gq_config_t *out)
+{
+    if (!in) return GQ_ERR_INVALID;
+    gq_config_t c = *in;
+    switch (c.scheme) {
+    case GQ_QSGD:
+    case GQ_ORQ:
+        if (c.levels < 2 || c.levels > GQ_MAX_LEVELS) return GQ_ERR_INVALID;
+        break;
+    case GQ_TERNGRAD:
+        if (c.levels == 0) c.levels = 3;
+        if (c.levels != 3) return GQ_ERR_INVALID;
+        break;
+    case GQ_BINGRAD_B:
+    case GQ_BINGRAD_PB:
+        if (c.levels == 0) c.levels = 2;
+        if (c.levels != 2) return GQ_ERR_INVALID;
+        break;
+    default: return GQ_ERR_INVALID;
+    }
+    if (c.bucket < GQ_MIN_BUCKET || c.bucket > GQ_MAX_BUCKET || (c.bucket & (c.bucket - 1)) != 0) return GQ_ERR_INVALID;
+    if (c.workers < 1 || c.workers > GQ_MAX_WORKERS) return GQ_ERR_INVALID;
+    if (c.error_feedback != 0 && c.error_feedback != 1) return GQ_ERR_INVALID;
+    if (!(c.clip_sigma >= 0.0f) || !std::isfinite(c.clip_sigma)) return GQ_ERR_INVALID;
+    if (c.n < 0 || c.n >= (int64_t(1) << 40)) return GQ_ERR_INVALID;
+    *out = c;
+    return GQ_OK;
+}
+
+void layout(const gq_config_t &c, size_t *bytes, size_t *codes_off, size_t *levels_off)
+{
+    const int64_t nb = (c.n + c.bucket - 1) / c.bucket;
+    int64_t cbytes = nb * (int64_t)c.bucket * bits_for(c.levels) / 8;
+    int64_t lbytes = nb * table_len(c.scheme, c.levels) * 4;
+    cbytes = (cbytes + 15) / 16 * 16;
+    lbytes = (lbytes + 15) / 16 * 16;
+    if (bytes) *bytes = (size_t)(cbytes + lbytes);
+    if (codes_off) *codes_off = 0;
+    if (levels_off) *levels_off = (size_t)cbytes;
+}
+
+gq::KParams base_params(const gq_plan &pl, uint64_t step)
+{
+    gq::KParams p;
+    std::memset(&p, 0, sizeof p);
+    p.scheme = pl.cfg.scheme;
+    p.s = pl.cfg.levels;
+    p.bits = pl.bits;
+    p.L = pl.L;
+    p.d = pl.cfg.bucket;
+    p.W = 1;
+    p.n = pl.cfg.n;
+    p.nb = pl.nb;
+    p.tail = pl.tail;
+    p.clip = pl.cfg.clip_sigma;
+    p.key0 = (uint32_t)pl.cfg.seed;
+    p.key1 = (uint32_t)(pl.cfg.seed >> 32);
+    p.step_lo = (uint32_t)step;
+    p.worker0 = 0;
+    p.inv_w = 1.0f;
+    p.codes_words = (int64_t)pl.cfg.bucket * pl.bits / 32;
+    p.levels_off = (int64_t)pl.levels_off;
+    p.status = pl.status;
+    return p;
+}
+
+gq_status_t check_device(const gq_plan &pl)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+    return dev == pl.device ? GQ_OK : GQ_ERR_INVALID;
+}
+
+gq_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GQ_OK : GQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+gq_status_t gq_config_check(const gq_config_t *cfg)
+{
+    gq_config_t c;
+    return normalise(cfg, &c);
+}
+
+gq_status_t gq_message_layout(const gq_config_t *cfg, size_t *bytes, size_t *codes_off, size_t *levels_off)
+{
+    gq_config_t c;
+    const gq_status_t st = normalise(cfg, &c);
+    if (st != GQ_OK) return st;
+    layout(c, bytes, codes_off, levels_off);
+    return GQ_OK;
+}
+
+gq_status_t gq_plan_create(const gq_config_t *cfg, gq_plan_t *out)
+{
+    if (!out) return GQ_ERR_INVALID;
+    *out = nullptr;
+    gq_config_t c;
+    const gq_status_t st = normalise(cfg, &c);
+    if (st != GQ_OK) return st;
+    gq_plan *pl = new (std::nothrow) gq_plan;
+    if (!pl) return GQ_ERR_NOMEM;
+    pl->cfg = c;
+    pl->bits = bits_for(c.levels);
+    pl->L = table_len(c.scheme, c.levels);
+    pl->nb = (c.n + c.bucket - 1) / c.bucket;
+    pl->tail = c.n > 0 ? (int)(c.n - (pl->nb - 1) * c.bucket) : 0;
+    layout(c, &pl->msg_bytes, &pl->codes_off, &pl->levels_off);
+    pl->status = nullptr;
+    if (cudaGetDevice(&pl->device) != cudaSuccess || cudaMalloc(&pl->status, sizeof(unsigned int)) != cudaSuccess ||
+        cudaMemset(pl->status, 0, sizeof(unsigned int)) != cudaSuccess) {
+        if (pl->status) cudaFree(pl->status);
+        delete pl;
+        return GQ_ERR_CUDA;
+    }
+    *out = pl;
+    return GQ_OK;
+}
+
+gq_status_t gq_plan_destroy(gq_plan_t plan)
+{
+    if (!plan) return GQ_ERR_INVALID;
+    const cudaError_t e = cudaFree(plan->status);
+    delete plan;
+    return from_cuda(e);
+}
+
+gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, float *residual, void *msg,
+                      void *stream)
+{
+    if (!plan || !grad || !msg || !aligned16(grad) || !aligned16(msg)) return GQ_ERR_INVALID;
+    if ((plan->cfg.error_feedback != 0) != (residual != nullptr)) return GQ_ERR_INVALID;
+    if (residual && !aligned16(residual)) return GQ_ERR_INVALID;
+    gq_status_t st = check_device(*plan);
+    if (st != GQ_OK) return st;
+    if (plan->cfg.n == 0) return GQ_OK;
+    gq::KParams p = base_params(*plan, step);
+    p.worker0 = worker;
+    p.g[0] = grad;
+    p.r[0] = residual;
+    p.msg[0] = static_cast<unsigned char *>(msg);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (plan->cfg.bucket <= 512) return from_cuda(gq::launch_warp_encode(p, false, s));
+    return from_cuda(gq::launch_cta_encode(p, s));
+}
+
+gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs, int nmsgs, float *avg, void *stream)
+{
+    if (!plan || !msgs || !avg || nmsgs < 1 || nmsgs > GQ_MAX_WORKERS || !aligned16(avg)) return GQ_ERR_INVALID;
+    for (int w = 0; w < nmsgs; ++w)
+        if (!msgs[w] || !aligned16(msgs[w])) return GQ_ERR_INVALID;
+    gq_status_t st = check_device(*plan);
+    if (st != GQ_OK) return st;
+    if (plan->cfg.n == 0) return GQ_OK;
+    gq::KParams p = base_params(*plan, 0);
+    p.W = nmsgs;
+    p.inv_w = 1.0f / (float)nmsgs;
+    for (int w = 0; w < nmsgs; ++w) p.msg[w] = static_cast<unsigned char *>(const_cast<void *>(msgs[w]));
+    p.avg = avg;
+    return from_cuda(gq::launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *grads, float *const *residuals,
+                          void *const *msgs, float *avg, void *stream)
+{
+    if (!plan || !grads || !avg || !aligned16(avg)) return GQ_ERR_INVALID;
+    const int W = plan->cfg.workers;
+    const bool ef = plan->cfg.error_feedback != 0;
+    if (ef != (residuals != nullptr)) return GQ_ERR_INVALID;
+    for (int w = 0; w < W; ++w) {
+        if (!grads[w] || !aligned16(grads[w])) return GQ_ERR_INVALID;
+        if (ef && (!residuals[w] || !aligned16(residuals[w]))) return GQ_ERR_INVALID;
+        if (msgs && (!msgs[w] || !aligned16(msgs[w]))) return GQ_ERR_INVALID;
+    }
+    if (!msgs && plan->cfg.bucket > 512) return GQ_ERR_INVALID;
+    gq_status_t st = check_device(*plan);
+    if (st != GQ_OK) return st;
+    if (plan->cfg.n == 0) return GQ_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    gq::KParams p = base_params(*plan, step);
+    if (plan->cfg.bucket <= 512) {
+        p.W = W;
+        p.inv_w = 1.0f / (float)W;
+        for (int w = 0; w < W; ++w) {
+            p.g[w] = grads[w];
+            p.r[w] = ef ? residuals[w] : nullptr;
+            p.msg[w] = msgs ? static_cast<unsigned char *>(msgs[w]) : nullptr;
+        }
+        p.avg = avg;
+        return from_cuda(gq::launch_warp_encode(p, true, s));
+    }
+    // large buckets: quantize each worker into its message, then decode + aggregate
+    for (int w = 0; w < W; ++w) {
+        gq::KParams q = p;
+        q.worker0 = (uint32_t)w;
+        q.g[0] = grads[w];
+        q.r[0] = ef ? residuals[w] : nullptr;
+        q.msg[0] = static_cast<unsigned char *>(msgs[w]);
+        const cudaError_t e = gq::launch_cta_encode(q, s);
+        if (e != cudaSuccess) return GQ_ERR_CUDA;
+    }
+    p.W = W;
+    p.inv_w = 1.0f / (float)W;
+    for (int w = 0; w < W; ++w) p.msg[w] = static_cast<unsigned char *>(msgs[w]);
+    p.avg = avg;
+    return from_cuda(gq::launch_decode(p, s));
+}
+
+gq_status_t gq_plan_status(gq_plan_t plan, void *stream)
+{
+    if (!plan) return GQ_ERR_INVALID;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int flags = 0;
+    if (cudaMemcpyAsync(&flags, plan->status, sizeof flags, cudaMemcpyDeviceToHost, s) != cudaSuccess) return GQ_ERR_CUDA;
+    if (cudaMemsetAsync(plan->status, 0, sizeof(unsigned int), s) != cudaSuccess) return GQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GQ_ERR_CUDA;
+    if (flags & gq::kStatusNonFinite) return GQ_ERR_NONFINITE;
+    return GQ_OK;
+}
+
+const char *gq_status_string(gq_status_t status)
+{
+    switch (status) {
+    case GQ_OK: return "ok";
+    case GQ_ERR_INVALID: return "invalid argument";
+    case GQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case GQ_ERR_CUDA: return "CUDA error";
+    case GQ_ERR_NONFINITE: return "non-finite input value";
+    case GQ_ERR_NOMEM: return "out of host memory";
+    }
+    return "unknown status";
+}
+
+const char *gq_version(void) { return "0.1.0"; }
+
+}  // extern "C"

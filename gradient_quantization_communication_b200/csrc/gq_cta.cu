@@ -1,0 +1,583 @@
+// gq_cta.cu -- quantization of large buckets (d = 1024 .. 32768): one CTA per bucket.
+//
+// The CTA (8 warps) stages the bucket's error-fed values v = g + r in shared memory (16-byte
+// coalesced loads), reduces the bucket statistics across its warps, fits the levels and then
+// rounds, packs and writes the residual chunk by chunk (warp k takes the 128-element chunks
+// k, k+8, ...).  Fits:
+//   QSGD / TernGrad : block max of |u|
+//   ORQ             : lane-private histograms per warp, flushed every 16 values per lane into
+//                     a block histogram (shared atomics); warp 0 runs the greedy
+//   BinGrad-pb      : block moments per cell (shared atomics), all 2016 pairs searched by
+//                     the 256 threads
+//   BinGrad-b       : block bitonic sort of u in place, exact int64 block scan, argmax of
+//                     J(k); the final pass re-reads g and r because the sort overwrote v
+// The per-element rules and the chunk step are those of the register path (gq_round.cuh), so
+// both paths produce identical codes.
+#include "gq_round.cuh"
+
+namespace gq {
+namespace {
+
+constexpr int kCtaWarps = 8;
+constexpr int kCtaThreads = kCtaWarps * 32;
+
+struct alignas(16) CtaShared {
+    float redf[2][kCtaWarps];
+    long long redl[3][kCtaWarps];
+    double redd[kCtaWarps];
+    int redi[kCtaWarps];
+    unsigned long long cs1[64], cs2[64];  // block histogram: sum of positions, of squares
+    unsigned int ccnt[64];                // block histogram: count
+    long long P1[64];
+    int P0[64];
+    long long al[64], be[64], ga[64], de[64];
+    float4 tab[16];
+    float lev[16];
+    unsigned char lut[64];
+    float bcast_f[4];
+    long long bcast_l[2];
+};
+
+// --- block reductions (every thread receives the result) -------------------------------------
+__device__ float block_max(float x, CtaShared &sh, int slot)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    x = warp_max(x);
+    if (lane == 0) sh.redf[slot][wid] = x;
+    __syncthreads();
+    float y = sh.redf[slot][lane & (kCtaWarps - 1)];
+    y = warp_max(y);
+    __syncthreads();
+    return y;
+}
+__device__ float block_min(float x, CtaShared &sh, int slot)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    x = warp_min(x);
+    if (lane == 0) sh.redf[slot][wid] = x;
+    __syncthreads();
+    float y = sh.redf[slot][lane & (kCtaWarps - 1)];
+    y = warp_min(y);
+    __syncthreads();
+    return y;
+}
+__device__ float block_max_nan(float x, CtaShared &sh, int slot)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    x = warp_max_nan(x);
+    if (lane == 0) sh.redf[slot][wid] = x;
+    __syncthreads();
+    float y = sh.redf[slot][lane & (kCtaWarps - 1)];
+    y = warp_max_nan(y);
+    __syncthreads();
+    return y;
+}
+__device__ long long block_sum(long long x, CtaShared &sh, int slot)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    x = warp_sum(x);
+    if (lane == 0) sh.redl[slot][wid] = x;
+    __syncthreads();
+    long long y = lane < kCtaWarps ? sh.redl[slot][lane] : 0ll;
+    y = warp_sum(y);
+    __syncthreads();
+    return y;
+}
+
+// --- ORQ: lane-private histogram of one warp -> block histogram --------------------------------
+__device__ __forceinline__ void flush_hist(uint32_t *hist, CtaShared &sh, int lane)
+{
+    __syncwarp();
+    uint32_t ca = 0, fa = 0, cb = 0, fb = 0;
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+        const int col = (lane + k) & 31;
+        const uint32_t xa = hist[lane * 32 + col];
+        const uint32_t xb = hist[(lane + 32) * 32 + col];
+        hist[lane * 32 + col] = 0u;
+        hist[(lane + 32) * 32 + col] = 0u;
+        ca += xa >> 27;
+        fa += xa & 0x7ffffffu;
+        cb += xb >> 27;
+        fb += xb & 0x7ffffffu;
+    }
+    if (ca) {
+        atomicAdd(&sh.ccnt[lane], ca);
+        atomicAdd(&sh.cs1[lane], (unsigned long long)ca * ((unsigned long long)lane << kOrqFBits) + fa);
+    }
+    if (cb) {
+        atomicAdd(&sh.ccnt[lane + 32], cb);
+        atomicAdd(&sh.cs1[lane + 32], (unsigned long long)cb * ((unsigned long long)(lane + 32) << kOrqFBits) + fb);
+    }
+    __syncwarp();
+}
+
+template <int SCHEME>
+__global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KParams p)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ CtaShared sh;
+    const int d = p.d;
+    float *vs = reinterpret_cast<float *>(smem_raw);                      // d floats
+    uint32_t *hist_all = reinterpret_cast<uint32_t *>(smem_raw + (size_t)d * 4);  // ORQ: 8 x 64 x 32
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    uint32_t *hist = hist_all + wid * 64 * 32;
+
+    if constexpr (SCHEME == GQ_ORQ) {
+        for (int i = lane; i < 64 * 32; i += 32) hist[i] = 0u;
+    }
+    for (int i = tid; i < 64; i += kCtaThreads) {
+        sh.ccnt[i] = 0u;
+        sh.cs1[i] = 0ull;
+        sh.cs2[i] = 0ull;
+    }
+    __syncthreads();
+
+    const float *g = p.g[0];
+    float *r = p.r[0];
+    unsigned char *msg = p.msg[0];
+    const uint32_t worker = p.worker0;
+    const int nchunks = d >> 7;
+
+    for (int64_t beta = blockIdx.x; beta < p.nb; beta += gridDim.x) {
+        const int64_t base = beta * (int64_t)d;
+        const int nvalid = (beta == p.nb - 1) ? p.tail : d;
+        // ---- stage v = g + r in shared memory; NaN-propagating max |v| --------------------------
+        float am = 0.0f;
+        for (int i4 = tid; i4 < (d >> 2); i4 += kCtaThreads) {
+            const int e = 4 * i4;
+            float4 x;
+            if (e + 3 < nvalid) {
+                x = __ldcs(reinterpret_cast<const float4 *>(g + base + e));
+                if (r) {
+                    const float4 y = __ldcs(reinterpret_cast<const float4 *>(r + base + e));
+                    x.x = __fadd_rn(x.x, y.x);
+                    x.y = __fadd_rn(x.y, y.y);
+                    x.z = __fadd_rn(x.z, y.z);
+                    x.w = __fadd_rn(x.w, y.w);
+                }
+                am = fmax_nan(am, fmax_nan(fmax_nan(fabsf(x.x), fabsf(x.y)), fmax_nan(fabsf(x.z), fabsf(x.w))));
+            } else {
+                float t[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    t[c] = 0.0f;
+                    if (e + c < nvalid) {
+                        t[c] = g[base + e + c];
+                        if (r) t[c] = __fadd_rn(t[c], r[base + e + c]);
+                        am = fmax_nan(am, fabsf(t[c]));
+                    }
+                }
+                x = make_float4(t[0], t[1], t[2], t[3]);
+            }
+            reinterpret_cast<float4 *>(vs)[i4] = x;
+        }
+        am = block_max_nan(am, sh, 0);
+        if (!(am <= FLT_MAX) && tid == 0) atomicOr(p.status, kStatusNonFinite);
+
+        // ---- clip threshold ---------------------------------------------------------------------
+        float T = INFINITY;
+        const bool clip = p.clip > 0.0f;
+        if (clip) {
+            T = 0.0f;
+            if (am > 0.0f) {
+                const int e = 20 - fexpo(am);
+                const double sc = pow2d(e);
+                long long sx = 0, sxx = 0;
+                for (int i = tid; i < nvalid; i += kCtaThreads) {
+                    const long long X = fixed_point(vs[i], sc);
+                    sx += X;
+                    sxx += X * X;
+                }
+                sx = block_sum(sx, sh, 0);
+                sxx = block_sum(sxx, sh, 1);
+                T = clip_threshold_from_sums(sx, sxx, nvalid, e, p.clip);
+            }
+        }
+        auto clipped = [&](float x) {
+            if (!clip) return x;
+            x = x < -T ? -T : x;
+            return x > T ? T : x;
+        };
+
+        // ---- fit ------------------------------------------------------------------------------
+        RoundQSGD rq;
+        RoundORQ ro{sh.lut, sh.tab, sh.lev};
+        RoundB rb{0.0f, 0.0f, 0.0f, false};
+        RoundPB rp;
+        bool constant = false;
+        float mn = 0.0f, mx = 0.0f, scale = 0.0f;
+        if constexpr (SCHEME == GQ_QSGD) {
+            float m = 0.0f;
+            for (int i = tid; i < nvalid; i += kCtaThreads) m = fmaxf(m, fabsf(clipped(vs[i])));
+            m = block_max(m, sh, 0);
+            const int s = p.s;
+            if (tid < s) sh.lev[tid] = __fmul_rn(m, __fdiv_rn((float)(2 * tid - (s - 1)), (float)(s - 1)));
+            if (tid == 0) sh.bcast_f[0] = m;
+            __syncthreads();
+            rq.inv_m = m > 0.0f ? __fdiv_rn(1.0f, m) : 0.0f;
+            rq.h = __fmul_rn((float)(s - 1), 0.5f);
+            rq.s = s;
+            rq.lev = sh.lev;
+        } else if constexpr (SCHEME == GQ_ORQ || SCHEME == GQ_BINGRAD_PB) {
+            float lo = INFINITY, hi = -INFINITY;
+            for (int i = tid; i < nvalid; i += kCtaThreads) {
+                const float x = clipped(vs[i]);
+                lo = fminf(lo, x);
+                hi = fmaxf(hi, x);
+            }
+            mn = __fadd_rn(block_min(lo, sh, 0), 0.0f);
+            mx = __fadd_rn(block_max(hi, sh, 1), 0.0f);
+            constant = !(mx > mn);
+            if (!constant) {
+                const float range = __fsub_rn(mx, mn);
+                const float step = __fdiv_rn(range, 63.0f);
+                if constexpr (SCHEME == GQ_ORQ) {
+                    scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kOrqFBits));
+                    // warp k: chunks k, k+8, ...; flush every 4 chunks (16 values per lane)
+                    int pending = 0;
+                    for (int ch = wid; ch < nchunks; ch += kCtaWarps) {
+                        const float4 x = reinterpret_cast<const float4 *>(vs)[ch * 32 + lane];
+                        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int e = ch * 128 + 4 * lane + c;
+                            if (e < nvalid) {
+                                const int ps = grid_pos<kOrqFBits>(clipped(xs[c]), mn, scale);
+                                const int cell = min(ps >> kOrqFBits, kTopCell);
+                                hist[cell * 32 + lane] += (1u << 27) + (uint32_t)(ps - (cell << kOrqFBits));
+                            }
+                        }
+                        if (++pending == 4) {
+                            flush_hist(hist, sh, lane);
+                            pending = 0;
+                        }
+                    }
+                    if (pending) flush_hist(hist, sh, lane);
+                    __syncthreads();
+                    if (wid == 0) {
+                        const long long c0 = sh.ccnt[lane], c1 = sh.ccnt[lane + 32];
+                        const long long s0 = (long long)sh.cs1[lane], s1 = (long long)sh.cs1[lane + 32];
+                        const long long ic0 = warp_inclusive_scan(c0, lane), ic1 = warp_inclusive_scan(c1, lane);
+                        const long long is0 = warp_inclusive_scan(s0, lane), is1 = warp_inclusive_scan(s1, lane);
+                        const long long tc = __shfl_sync(kFull, ic0, 31), ts = __shfl_sync(kFull, is0, 31);
+                        sh.P0[lane] = (int)(ic0 - c0);
+                        sh.P1[lane] = is0 - s0;
+                        sh.P0[lane + 32] = (int)(tc + ic1 - c1);
+                        sh.P1[lane + 32] = ts + is1 - s1;
+                        sh.ccnt[lane] = 0u;
+                        sh.ccnt[lane + 32] = 0u;
+                        sh.cs1[lane] = 0ull;
+                        sh.cs1[lane + 32] = 0ull;
+                        __syncwarp();
+                        const unsigned long long mask = orq_greedy(sh.P0, sh.P1, p.s, lane);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int j = lane + 32 * h;
+                            if ((mask >> j) & 1ull) sh.lev[__popcll(mask & ((1ull << j) - 1ull))] = grid_point(mn, mx, step, j);
+                            if (j <= kTopCell) sh.lut[j] = (unsigned char)(__popcll(mask & ((2ull << j) - 1ull)) - 1);
+                        }
+                        __syncwarp();
+                        if (lane < p.s - 1) {
+                            const float l0 = sh.lev[lane], l1 = sh.lev[lane + 1];
+                            sh.tab[lane] = make_float4(l0, l1, __fdiv_rn(1.0f, __fsub_rn(l1, l0)), 0.0f);
+                        }
+                    }
+                    __syncthreads();
+                } else {
+                    scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kPbFBits));
+                    for (int i = tid; i < nvalid; i += kCtaThreads) {
+                        const int ps = grid_pos<kPbFBits>(clipped(vs[i]), mn, scale);
+                        const int cell = min(ps >> kPbFBits, kTopCell);
+                        const unsigned long long x = (unsigned long long)ps;
+                        atomicAdd(&sh.ccnt[cell], 1u);
+                        atomicAdd(&sh.cs1[cell], x);
+                        atomicAdd(&sh.cs2[cell], x * x);
+                    }
+                    __syncthreads();
+                    if (wid == 0) {
+                        const long long c0 = sh.ccnt[lane], c1 = sh.ccnt[lane + 32];
+                        const long long x0 = (long long)sh.cs1[lane], x1 = (long long)sh.cs1[lane + 32];
+                        const long long y0 = (long long)sh.cs2[lane], y1 = (long long)sh.cs2[lane + 32];
+                        sh.ccnt[lane] = 0u;
+                        sh.ccnt[lane + 32] = 0u;
+                        sh.cs1[lane] = 0ull;
+                        sh.cs1[lane + 32] = 0ull;
+                        sh.cs2[lane] = 0ull;
+                        sh.cs2[lane + 32] = 0ull;
+                        const long long ic0 = warp_inclusive_scan(c0, lane), ic1 = warp_inclusive_scan(c1, lane);
+                        const long long ix0 = warp_inclusive_scan(x0, lane), ix1 = warp_inclusive_scan(x1, lane);
+                        const long long iy0 = warp_inclusive_scan(y0, lane), iy1 = warp_inclusive_scan(y1, lane);
+                        const long long tc = __shfl_sync(kFull, ic0, 31), tx = __shfl_sync(kFull, ix0, 31),
+                                        ty = __shfl_sync(kFull, iy0, 31);
+                        const long long tc_all = __shfl_sync(kFull, tc + ic1, 31);
+                        const long long tx_all = __shfl_sync(kFull, tx + ix1, 31);
+                        const long long ty_all = __shfl_sync(kFull, ty + iy1, 31);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int K = lane + 32 * h;
+                            const unsigned long long uQ0 = h ? tc + ic1 - c1 : ic0 - c0;
+                            const unsigned long long uQ1 = h ? tx + ix1 - x1 : ix0 - x0;
+                            const unsigned long long uQ2 = h ? ty + iy1 - y1 : iy0 - y0;
+                            const unsigned long long k = (unsigned long long)K << kPbFBits;
+                            sh.al[K] = (long long)(k * k * uQ0 - 3ull * k * uQ1 + 2ull * uQ2);
+                            sh.be[K] = (long long)(3ull * k * uQ1 - 2ull * uQ2 + (unsigned long long)ty_all -
+                                                   2ull * k * (unsigned long long)tx_all +
+                                                   k * k * ((unsigned long long)tc_all - uQ0));
+                            sh.ga[K] = (long long)(uQ1 - k * uQ0);
+                            sh.de[K] = (long long)(k * uQ0 - uQ1);
+                        }
+                    }
+                    __syncthreads();
+                    // thread (B = tid % 64, group tid / 64) searches A in [16*group, 16*group + 16) below B
+                    const int B = tid & 63, grp = tid >> 6;
+                    const unsigned long long bb = (unsigned long long)B << kPbFBits;
+                    const unsigned long long beB = sh.be[B], gaB = sh.ga[B];
+                    long long best_e = 0x7fffffffffffffffll;
+                    int best_ab = 0x7fffffff;
+                    for (int A = 16 * grp; A < 16 * grp + 16 && A < B; ++A) {
+                        const unsigned long long aa = (unsigned long long)A << kPbFBits;
+                        const long long e = (long long)((unsigned long long)sh.al[A] + beB + aa * gaB + bb * (unsigned long long)sh.de[A]);
+                        const int ab = A * 64 + B;
+                        if (e < best_e || (e == best_e && ab < best_ab)) {
+                            best_e = e;
+                            best_ab = ab;
+                        }
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const long long oe = __shfl_xor_sync(kFull, best_e, o);
+                        const int oab = __shfl_xor_sync(kFull, best_ab, o);
+                        if (oe < best_e || (oe == best_e && oab < best_ab)) {
+                            best_e = oe;
+                            best_ab = oab;
+                        }
+                    }
+                    if (lane == 0) {
+                        sh.redl[0][wid] = best_e;
+                        sh.redi[wid] = best_ab;
+                    }
+                    __syncthreads();
+                    best_e = sh.redl[0][lane & 7];
+                    best_ab = sh.redi[lane & 7];
+#pragma unroll
+                    for (int o = 4; o > 0; o >>= 1) {
+                        const long long oe = __shfl_xor_sync(kFull, best_e, o);
+                        const int oab = __shfl_xor_sync(kFull, best_ab, o);
+                        if (oe < best_e || (oe == best_e && oab < best_ab)) {
+                            best_e = oe;
+                            best_ab = oab;
+                        }
+                    }
+                    __syncthreads();
+                    const int A = best_ab >> 6, Bs = best_ab & 63;
+                    rp.a = grid_point(mn, mx, step, A);
+                    rp.b = grid_point(mn, mx, step, Bs);
+                    rp.rinv = __fdiv_rn(1.0f, __fsub_rn(rp.b, rp.a));
+                    rp.pa = A << kPbFBits;
+                    rp.pb = Bs << kPbFBits;
+                }
+            }
+        } else {  // BinGrad-b
+            float m = 0.0f;
+            for (int i = tid; i < nvalid; i += kCtaThreads) m = fmaxf(m, fabsf(clipped(vs[i])));
+            m = block_max(m, sh, 0);
+            if (m > 0.0f) {
+                // sort u in place (padding = +inf)
+                for (int i = tid; i < d; i += kCtaThreads) vs[i] = i < nvalid ? clipped(vs[i]) : INFINITY;
+                __syncthreads();
+                for (int k = 2; k <= d; k <<= 1) {
+                    for (int j = k >> 1; j > 0; j >>= 1) {
+                        for (int i = tid; i < d; i += kCtaThreads) {
+                            const int ixj = i ^ j;
+                            if (ixj > i) {
+                                const float a = vs[i], b = vs[ixj];
+                                const bool up = (i & k) == 0;
+                                if ((a > b) == up) {
+                                    vs[i] = b;
+                                    vs[ixj] = a;
+                                }
+                            }
+                        }
+                        __syncthreads();
+                    }
+                }
+                // exact prefix sums of the fixed-point values: thread t owns positions [t*seg, (t+1)*seg)
+                const int e2 = 46 - fexpo(m);
+                const double sc = pow2d(e2);
+                const int seg = d / kCtaThreads;
+                long long run = 0;
+                for (int i = tid * seg; i < tid * seg + seg; ++i) run += (i < nvalid) ? fixed_point(vs[i], sc) : 0ll;
+                const long long incl = warp_inclusive_scan(run, lane);
+                if (lane == 31) sh.redl[0][wid] = incl;
+                __syncthreads();
+                long long wpre = 0, total = 0;
+                for (int k = 0; k < kCtaWarps; ++k) {
+                    const long long t = sh.redl[0][k];
+                    if (k < wid) wpre += t;
+                    total += t;
+                }
+                __syncthreads();
+                long long S = wpre + incl - run;  // sum of positions before tid*seg
+                double best_j = -1.0;
+                int best_i = 0x7fffffff;
+                long long best_s = 0;
+                for (int i = tid * seg; i < tid * seg + seg; ++i) {
+                    if (i >= 1 && i < nvalid && vs[i - 1] < vs[i]) {
+                        const double l = __ll2double_rn(S);
+                        const double rr = __ll2double_rn(total - S);
+                        const double J = __dadd_rn(__ddiv_rn(__dmul_rn(l, l), (double)i),
+                                                   __ddiv_rn(__dmul_rn(rr, rr), (double)(nvalid - i)));
+                        if (J > best_j) {
+                            best_j = J;
+                            best_i = i;
+                            best_s = S;
+                        }
+                    }
+                    if (i < nvalid) S += fixed_point(vs[i], sc);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const double oj = __shfl_xor_sync(kFull, best_j, o);
+                    const int oi = __shfl_xor_sync(kFull, best_i, o);
+                    const long long os = __shfl_xor_sync(kFull, best_s, o);
+                    if (oj > best_j || (oj == best_j && oi < best_i)) {
+                        best_j = oj;
+                        best_i = oi;
+                        best_s = os;
+                    }
+                }
+                if (lane == 0) {
+                    sh.redd[wid] = best_j;
+                    sh.redi[wid] = best_i;
+                    sh.redl[1][wid] = best_s;
+                }
+                __syncthreads();
+                best_j = sh.redd[lane & 7];
+                best_i = sh.redi[lane & 7];
+                best_s = sh.redl[1][lane & 7];
+#pragma unroll
+                for (int o = 4; o > 0; o >>= 1) {
+                    const double oj = __shfl_xor_sync(kFull, best_j, o);
+                    const int oi = __shfl_xor_sync(kFull, best_i, o);
+                    const long long os = __shfl_xor_sync(kFull, best_s, o);
+                    if (oj > best_j || (oj == best_j && oi < best_i)) {
+                        best_j = oj;
+                        best_i = oi;
+                        best_s = os;
+                    }
+                }
+                if (best_i == 0x7fffffff) {
+                    const float v0 = __fadd_rn(vs[0], 0.0f);
+                    rb = RoundB{v0, v0, v0, false};
+                } else {
+                    const double inv_sc = pow2d(-e2);
+                    const float a = __double2float_rn(__dmul_rn(__ddiv_rn(__ll2double_rn(best_s), (double)best_i), inv_sc));
+                    const float b = __double2float_rn(
+                        __dmul_rn(__ddiv_rn(__ll2double_rn(total - best_s), (double)(nvalid - best_i)), inv_sc));
+                    rb = RoundB{a, b, vs[best_i], true};
+                }
+                __syncthreads();
+            }
+        }
+
+        // ---- round, pack, write residual and message ---------------------------------------------
+        uint32_t *cw = msg ? reinterpret_cast<uint32_t *>(msg) + beta * p.codes_words : nullptr;
+        for (int ch = wid; ch < nchunks; ch += kCtaWarps) {
+            const int e0 = ch * 128 + 4 * lane;
+            float v4[4];
+            if constexpr (SCHEME == GQ_BINGRAD_B) {
+                // the sort overwrote the staged values: read g (+ r) again
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    v4[c] = 0.0f;
+                    if (e0 + c < nvalid) {
+                        v4[c] = g[base + e0 + c];
+                        if (r) v4[c] = __fadd_rn(v4[c], r[base + e0 + c]);
+                    }
+                }
+            } else {
+                const float4 x = reinterpret_cast<const float4 *>(vs)[ch * 32 + lane];
+                v4[0] = x.x;
+                v4[1] = x.y;
+                v4[2] = x.z;
+                v4[3] = x.w;
+            }
+            float u4[4];
+            int pos4[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                u4[c] = clipped(v4[c]);
+                pos4[c] = 0;
+                if constexpr (SCHEME == GQ_ORQ) pos4[c] = constant ? 0 : grid_pos<kOrqFBits>(u4[c], mn, scale);
+                if constexpr (SCHEME == GQ_BINGRAD_PB) pos4[c] = constant ? 0 : grid_pos<kPbFBits>(u4[c], mn, scale);
+            }
+            uint32_t valid = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) valid |= (e0 + c < nvalid ? 1u : 0u) << c;
+            const uint64_t blk = (uint64_t)(base >> 2) + (uint64_t)(32 * ch);
+            float *rout = r ? r + base + 128 * ch : nullptr;
+            uint32_t *cwc = cw ? cw + ch * 4 * p.bits : nullptr;
+            float q[4];
+            if constexpr (SCHEME == GQ_QSGD) {
+                round_chunk<true>(p, rq, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+            } else if constexpr (SCHEME == GQ_ORQ) {
+                if (constant)
+                    round_chunk<false>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                else
+                    round_chunk<true>(p, ro, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+            } else if constexpr (SCHEME == GQ_BINGRAD_PB) {
+                if (constant)
+                    round_chunk<false>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                else
+                    round_chunk<true>(p, rp, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+            } else {
+                round_chunk<false>(p, rb, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+            }
+        }
+        // ---- level table --------------------------------------------------------------------------
+        if (msg && tid < p.L) {
+            float lv;
+            if constexpr (SCHEME == GQ_QSGD) lv = sh.bcast_f[0];
+            else if constexpr (SCHEME == GQ_ORQ) lv = constant ? mn : sh.lev[tid];
+            else if constexpr (SCHEME == GQ_BINGRAD_PB) lv = constant ? mn : (tid == 0 ? rp.a : rp.b);
+            else lv = tid == 0 ? rb.a : rb.b;
+            reinterpret_cast<float *>(msg + p.levels_off)[beta * p.L + tid] = lv;
+        }
+        __syncthreads();
+    }
+}
+
+template <int SCHEME>
+cudaError_t launch(const KParams &p, cudaStream_t stream)
+{
+    auto kern = k_cta<SCHEME>;
+    const size_t smem = (size_t)p.d * 4 + (SCHEME == GQ_ORQ ? (size_t)kCtaWarps * 64 * 32 * 4 : 0);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCtaThreads, smem);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t cap = (int64_t)sms * per_sm;
+    const int grid = (int)(p.nb < cap ? p.nb : cap);
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, kCtaThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream)
+{
+    switch (p.scheme) {
+    case GQ_QSGD:
+    case GQ_TERNGRAD: return launch<GQ_QSGD>(p, stream);
+    case GQ_BINGRAD_B: return launch<GQ_BINGRAD_B>(p, stream);
+    case GQ_BINGRAD_PB: return launch<GQ_BINGRAD_PB>(p, stream);
+    default: return launch<GQ_ORQ>(p, stream);
+    }
+}
+
+}  // namespace gq

@@ -1,0 +1,105 @@
+// gq_decode.cu -- Dequantize + Aggregate: avg[i] = (sum_w level_w(code_w[i])) * (1/W).
+//
+// One warp owns a tile of 512 consecutive elements (four 128-element chunks of the packed
+// layout), for any bucket size.  Per worker and chunk the warp reads the b uint4 words of the
+// chunk (the same 16 bytes for all lanes: one broadcast transaction each) and the bucket's
+// level table; lane l pulls bit l of each word, which gives the codes of its elements
+// 128m + 4l + c, and looks the level up with a register shuffle (lane k holds level k).  The
+// sum runs in worker order in registers; the average is written once, with 16-byte stores.
+#include "gq_device.cuh"
+
+namespace gq {
+namespace {
+
+constexpr int kDecodeWarps = 8;
+
+template <bool QSGD>
+__global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_constant__ KParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t ntiles = (p.n + 511) / 512;
+    const int64_t first = (int64_t)blockIdx.x * kDecodeWarps + (threadIdx.x >> 5);
+    const int64_t stride = (int64_t)gridDim.x * kDecodeWarps;
+    const int log2d = 31 - __clz(p.d);
+    const int chunks_per_bucket = p.d >> 7;
+    for (int64_t tile = first; tile < ntiles; tile += stride) {
+        float acc[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) acc[t] = 0.0f;
+        for (int w = 0; w < p.W; ++w) {
+            const unsigned char *msg = p.msg[w];
+            const uint32_t *codes = reinterpret_cast<const uint32_t *>(msg);
+            const float *tables = reinterpret_cast<const float *>(msg + p.levels_off);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int64_t e0 = tile * 512 + 128 * m;
+                if (e0 >= p.n) break;
+                const int64_t bk = e0 >> log2d;
+                const int cb = (int)((e0 >> 7) & (chunks_per_bucket - 1));
+                const uint32_t *cw = codes + bk * p.codes_words + (int64_t)cb * 4 * p.bits;
+                // lane k holds level k of this bucket
+                float lv = 0.0f;
+                if (QSGD) {
+                    const float mscale = __ldg(tables + bk);
+                    if (lane < p.s) lv = __fmul_rn(mscale, __fdiv_rn((float)(2 * lane - (p.s - 1)), (float)(p.s - 1)));
+                } else if (lane < p.L) {
+                    lv = __ldg(tables + bk * p.L + lane);
+                }
+                uint32_t code0 = 0, code1 = 0, code2 = 0, code3 = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (j < p.bits) {
+                        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(cw) + j);
+                        code0 |= ((x.x >> lane) & 1u) << j;
+                        code1 |= ((x.y >> lane) & 1u) << j;
+                        code2 |= ((x.z >> lane) & 1u) << j;
+                        code3 |= ((x.w >> lane) & 1u) << j;
+                    }
+                }
+                acc[4 * m + 0] = __fadd_rn(acc[4 * m + 0], __shfl_sync(kFull, lv, (int)code0));
+                acc[4 * m + 1] = __fadd_rn(acc[4 * m + 1], __shfl_sync(kFull, lv, (int)code1));
+                acc[4 * m + 2] = __fadd_rn(acc[4 * m + 2], __shfl_sync(kFull, lv, (int)code2));
+                acc[4 * m + 3] = __fadd_rn(acc[4 * m + 3], __shfl_sync(kFull, lv, (int)code3));
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int64_t e = tile * 512 + 128 * m + 4 * lane;
+            if (e + 3 < p.n) {
+                __stcs(reinterpret_cast<float4 *>(p.avg + e),
+                       make_float4(__fmul_rn(acc[4 * m], p.inv_w), __fmul_rn(acc[4 * m + 1], p.inv_w),
+                                   __fmul_rn(acc[4 * m + 2], p.inv_w), __fmul_rn(acc[4 * m + 3], p.inv_w)));
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (e + c < p.n) p.avg[e + c] = __fmul_rn(acc[4 * m + c], p.inv_w);
+            }
+        }
+    }
+}
+
+template <bool QSGD>
+cudaError_t launch(const KParams &p, cudaStream_t stream)
+{
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<QSGD>, kDecodeWarps * 32, 0);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t ntiles = (p.n + 511) / 512;
+    const int64_t need = (ntiles + kDecodeWarps - 1) / kDecodeWarps;
+    const int64_t cap = (int64_t)sms * per_sm;
+    const int grid = (int)(need < cap ? need : cap);
+    if (grid <= 0) return cudaSuccess;
+    k_decode<QSGD><<<grid, kDecodeWarps * 32, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const KParams &p, cudaStream_t stream)
+{
+    return (p.scheme == GQ_QSGD || p.scheme == GQ_TERNGRAD) ? launch<true>(p, stream) : launch<false>(p, stream);
+}
+
+}  // namespace gq

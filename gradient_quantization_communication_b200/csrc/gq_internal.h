@@ -1,0 +1,47 @@
+// gq_internal.h -- kernel parameter block and launch entry points shared by the library's
+// translation units (not part of the public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "gq.h"
+
+namespace gq {
+
+// Everything a quantization kernel needs, passed by value as a __grid_constant__ parameter.
+struct KParams {
+    int scheme;          // gq_scheme_t
+    int s;               // levels
+    int bits;            // ceil(log2 s)
+    int L;               // floats per level table in the message
+    int d;               // bucket size (power of two)
+    int W;               // workers handled by this launch
+    int64_t n;           // elements per worker
+    int64_t nb;          // buckets per worker
+    int tail;            // valid elements of the last bucket (1..d)
+    float clip;          // c of the +-c*sigma clip, 0 = off
+    uint32_t key0, key1; // Philox key (seed)
+    uint32_t step_lo;    // step, low word
+    uint32_t worker0;    // Philox worker index of worker slot 0
+    float inv_w;         // 1/W for the average
+    int64_t codes_words; // words of packed codes per bucket (d*b/32)
+    int64_t levels_off;  // byte offset of the level tables inside a message
+    const float *g[GQ_MAX_WORKERS];
+    float *r[GQ_MAX_WORKERS];          // NULL when error feedback is off
+    unsigned char *msg[GQ_MAX_WORKERS];// NULL: do not write the message
+    float *avg;                        // fused kernels only
+    unsigned int *status;              // plan status word
+};
+
+// Status bits raised by kernels.
+constexpr unsigned kStatusNonFinite = 1u;
+
+// Register-resident path (d = 128, 256, 512): one warp per bucket index.
+cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream);
+// Shared-memory path (d = 1024 .. 32768): one CTA per bucket, one worker per launch.
+cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream);
+// Dequantize + aggregate for any d.
+cudaError_t launch_decode(const KParams &p, cudaStream_t stream);
+
+}  // namespace gq

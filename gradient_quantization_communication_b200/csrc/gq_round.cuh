@@ -1,0 +1,116 @@
+// gq_round.cuh -- per-element rounding rules of the five schemes and the 128-element chunk
+// step shared by the register path (d <= 512) and the shared-memory path (d >= 1024):
+// draw, round, dequantize, write the residual, bit-plane pack with warp ballots.
+#pragma once
+
+#include "gq_device.cuh"
+
+namespace gq {
+
+// QSGD / TernGrad: position y = (u/m + 1) * (s-1)/2 in level units; up with probability frac(y).
+struct RoundQSGD {
+    float inv_m, h;
+    int s;
+    const float *lev;
+    __device__ __forceinline__ int code(float u, int, float U) const
+    {
+        const float y = __fmul_rn(__fadd_rn(__fmul_rn(u, inv_m), 1.0f), h);
+        const int k = min(max(__float2int_rz(y), 0), s - 2);
+        const float pu = __fsub_rn(y, (float)k);
+        return k + (U < pu ? 1 : 0);
+    }
+    __device__ __forceinline__ float level(int c) const { return lev[c]; }
+};
+
+// ORQ: bracket of the value's grid cell, up with probability (u - lower)/(upper - lower).
+struct RoundORQ {
+    const unsigned char *lut;
+    const float4 *tab;
+    const float *lev;
+    __device__ __forceinline__ int code(float u, int pos, float U) const
+    {
+        const int cell = min(pos >> kOrqFBits, kTopCell);
+        const int k = lut[cell];
+        const float4 b = tab[k];
+        const float pu = sat01(__fmul_rn(__fsub_rn(u, b.x), b.z));
+        return k + (U < pu ? 1 : 0);
+    }
+    __device__ __forceinline__ float level(int c) const { return lev[c]; }
+};
+
+// Constant bucket: one level, code 0.
+struct RoundConst {
+    float lv;
+    __device__ __forceinline__ int code(float, int, float) const { return 0; }
+    __device__ __forceinline__ float level(int) const { return lv; }
+};
+
+// BinGrad-b: deterministic, code 1 at or above the split value.
+struct RoundB {
+    float a, b, thr;
+    bool split;
+    __device__ __forceinline__ int code(float u, int, float) const { return (split && u >= thr) ? 1 : 0; }
+    __device__ __forceinline__ float level(int c) const { return c ? b : a; }
+};
+
+// BinGrad-pb: clamped below the lower / at or above the upper grid level, stochastic between.
+struct RoundPB {
+    float a, b, rinv;
+    int pa, pb;
+    __device__ __forceinline__ int code(float u, int pos, float U) const
+    {
+        if (pos < pa) return 0;
+        if (pos >= pb) return 1;
+        const float pu = sat01(__fmul_rn(__fsub_rn(u, a), rinv));
+        return U < pu ? 1 : 0;
+    }
+    __device__ __forceinline__ float level(int c) const { return c ? b : a; }
+};
+
+// One 128-element chunk of a bucket: lane l holds elements 4l .. 4l+3 of the chunk
+// (v: error-fed values, u: clipped values, pos: grid positions; valid: 4-bit mask).
+//   blk      global element index of the chunk's first element, divided by 4
+//   rout     residual of the chunk's first element (NULL: no residual), 16-byte aligned
+//   cw       packed words of the chunk (b uint4: plane j = words 4j..4j+3), NULL: no message
+// Returns the dequantized values in q.
+template <bool RANDOM, class R>
+__device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uint64_t blk, uint32_t worker, int lane,
+                                            uint32_t valid, const float (&v)[4], const float (&u)[4],
+                                            const int (&pos)[4], float *rout, uint32_t *cw, float (&q)[4])
+{
+    uint4 rnd = make_uint4(0u, 0u, 0u, 0u);
+    if (RANDOM) rnd = draws4(p, blk + (uint64_t)lane, worker);
+    const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+    int code[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int k = rule.code(u[c], pos[c], RANDOM ? unit_float(words[c]) : 0.0f);
+        code[c] = ((valid >> c) & 1u) ? k : 0;
+        q[c] = rule.level(code[c]);
+    }
+    if (rout) {
+        if (valid == 0xfu) {
+            __stcs(reinterpret_cast<float4 *>(rout + 4 * lane),
+                   make_float4(__fsub_rn(v[0], q[0]), __fsub_rn(v[1], q[1]), __fsub_rn(v[2], q[2]), __fsub_rn(v[3], q[3])));
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if ((valid >> c) & 1u) rout[4 * lane + c] = __fsub_rn(v[c], q[c]);
+        }
+    }
+    if (cw) {
+        // bit j of the code of element 4l + c -> bit l of word 4j + c of the chunk
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (j < p.bits) {
+                const uint32_t w0 = __ballot_sync(kFull, (code[0] >> j) & 1);
+                const uint32_t w1 = __ballot_sync(kFull, (code[1] >> j) & 1);
+                const uint32_t w2 = __ballot_sync(kFull, (code[2] >> j) & 1);
+                const uint32_t w3 = __ballot_sync(kFull, (code[3] >> j) & 1);
+                if (lane == 0) __stcs(reinterpret_cast<uint4 *>(cw) + j, make_uint4(w0, w1, w2, w3));
+            }
+        }
+    }
+}
+
+}  // namespace gq

@@ -1,0 +1,174 @@
+"""Python binding of the C ABI in ``include/gq.h`` (``libgq.so``): argument marshalling only.
+
+Every function keeps the C name.  Tensors are passed as ``data_ptr()``; the stream defaults to
+torch's current CUDA stream.  There is no fallback: if ``libgq.so`` is missing the import of the
+library fails with an error that says how to build it.
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgq.so")
+
+GQ_QSGD, GQ_TERNGRAD, GQ_BINGRAD_B, GQ_BINGRAD_PB, GQ_ORQ = 0, 1, 2, 3, 4
+GQ_OK, GQ_ERR_INVALID, GQ_ERR_UNSUPPORTED, GQ_ERR_CUDA, GQ_ERR_NONFINITE, GQ_ERR_NOMEM = 0, 1, 2, 3, 4, 5
+GQ_MAX_WORKERS = 64
+SCHEMES = {"qsgd": GQ_QSGD, "terngrad": GQ_TERNGRAD, "bingrad_b": GQ_BINGRAD_B,
+           "bingrad_pb": GQ_BINGRAD_PB, "orq": GQ_ORQ}
+
+
+class gq_config_t(ctypes.Structure):
+    _fields_ = [("scheme", ctypes.c_int32), ("levels", ctypes.c_int32), ("bucket", ctypes.c_int32),
+                ("workers", ctypes.c_int32), ("error_feedback", ctypes.c_int32),
+                ("clip_sigma", ctypes.c_float), ("seed", ctypes.c_uint64), ("n", ctypes.c_int64)]
+
+
+class GQError(RuntimeError):
+    def __init__(self, status, what):
+        super().__init__("%s: %s (status %d)" % (what, gq_status_string(status), status))
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libgq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libgq.so is not built (%s); run gradient_quantization_communication_b200/build.py"
+                              % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        cfgp = ctypes.POINTER(gq_config_t)
+        L.gq_config_check.argtypes = [cfgp]
+        L.gq_message_layout.argtypes = [cfgp, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.gq_plan_create.argtypes = [cfgp, ctypes.POINTER(vp)]
+        L.gq_plan_destroy.argtypes = [vp]
+        L.gq_encode.argtypes = [vp, ctypes.c_uint32, ctypes.c_uint64, vp, vp, vp, vp]
+        L.gq_decode_accumulate.argtypes = [vp, ctypes.POINTER(vp), ctypes.c_int, vp, vp]
+        L.gq_fused_step.argtypes = [vp, ctypes.c_uint64, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                    ctypes.POINTER(vp), vp, vp]
+        L.gq_plan_status.argtypes = [vp, vp]
+        L.gq_status_string.argtypes = [ctypes.c_int]
+        L.gq_status_string.restype = ctypes.c_char_p
+        L.gq_version.restype = ctypes.c_char_p
+        for f in ("gq_config_check", "gq_message_layout", "gq_plan_create", "gq_plan_destroy", "gq_encode",
+                  "gq_decode_accumulate", "gq_fused_step", "gq_plan_status"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------------------------
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptr_array(xs):
+    if xs is None:
+        return None
+    return (ctypes.c_void_p * len(xs))(*[_ptr(x) for x in xs])
+
+
+def _check(st, what):
+    if st != GQ_OK:
+        raise GQError(st, what)
+
+
+def gq_config(scheme, levels=0, bucket=512, workers=1, error_feedback=True, clip_sigma=0.0, seed=0, n=0):
+    if isinstance(scheme, str):
+        scheme = SCHEMES[scheme]
+    return gq_config_t(scheme, levels, bucket, workers, int(bool(error_feedback)), clip_sigma, seed, n)
+
+
+# ---------------------------------------------------------------------------------------------
+# the C entry points
+# ---------------------------------------------------------------------------------------------
+def gq_config_check(cfg):
+    return lib().gq_config_check(ctypes.byref(cfg))
+
+
+def gq_message_layout(cfg):
+    b, c, l = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().gq_message_layout(ctypes.byref(cfg), ctypes.byref(b), ctypes.byref(c), ctypes.byref(l)),
+           "gq_message_layout")
+    return b.value, c.value, l.value
+
+
+def gq_plan_create(cfg):
+    h = ctypes.c_void_p()
+    _check(lib().gq_plan_create(ctypes.byref(cfg), ctypes.byref(h)), "gq_plan_create")
+    return h
+
+
+def gq_plan_destroy(plan):
+    _check(lib().gq_plan_destroy(plan), "gq_plan_destroy")
+
+
+def gq_encode(plan, worker, step, grad, residual, msg, stream=None):
+    _check(lib().gq_encode(plan, worker, step, _ptr(grad), _ptr(residual), _ptr(msg), _stream(stream)), "gq_encode")
+
+
+def gq_decode_accumulate(plan, msgs, avg, stream=None):
+    _check(lib().gq_decode_accumulate(plan, _ptr_array(msgs), len(msgs), _ptr(avg), _stream(stream)),
+           "gq_decode_accumulate")
+
+
+def gq_fused_step(plan, step, grads, residuals, msgs, avg, stream=None):
+    _check(lib().gq_fused_step(plan, step, _ptr_array(grads), _ptr_array(residuals), _ptr_array(msgs), _ptr(avg),
+                               _stream(stream)), "gq_fused_step")
+
+
+def gq_plan_status(plan, stream=None):
+    return lib().gq_plan_status(plan, _stream(stream))
+
+
+def gq_status_string(status):
+    return lib().gq_status_string(status).decode()
+
+
+def gq_version():
+    return lib().gq_version().decode()
+
+
+class Plan:
+    """Owner of a gq_plan_t (destroyed on close / exit of a ``with`` block)."""
+
+    def __init__(self, cfg):
+        self.cfg = cfg
+        self.handle = gq_plan_create(cfg)
+        self.msg_bytes, self.codes_off, self.levels_off = gq_message_layout(cfg)
+
+    def close(self):
+        if self.handle:
+            gq_plan_destroy(self.handle)
+            self.handle = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

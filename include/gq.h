@@ -1,0 +1,167 @@
+/*
+ * gq.h -- C ABI of the B200 library for bucketed gradient quantization (libgq.so).
+ *
+ * The library implements the data-parallel step that the page "gradient quantization for
+ * communication" (glossary) describes in its section "How Gradient Quantization Works":
+ * Quantize -> Transmit -> Dequantize -> Aggregate, with the error feedback of its section
+ * "Quantization Schemes".  Quantize is bucketed (buckets of d elements, the review
+ * "[Paper Review] Optimal Gradient Quantization Condition for Communication-Efficient
+ * Distributed Training", section "Proposed method") with one of five level fits:
+ *   QSGD-s and TernGrad (max-abs scaling; "Gradient Quantization" glossary),
+ *   BinGrad-b, BinGrad-pb and ORQ-s (the review's proposed schemes).
+ * W workers are W separate buffers on one GPU; "Transmit" is the message each worker writes to
+ * device memory, and Dequantize + Aggregate read it back (or, in gq_fused_step, never leave
+ * the chip).
+ *
+ * Conventions for every call:
+ *   - Pointers named "device" are CUDA device (or managed) memory owned by the caller, 16-byte
+ *     aligned.  Arrays of pointers (grads[], residuals[], msgs[]) are HOST arrays of W device
+ *     pointers.  The library keeps no pointer after a call returns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only enqueue
+ *     work; results are ready when the stream is.  Calls on one plan must not overlap on the
+ *     GPU (the plan's status word is shared).
+ *   - Argument errors are reported synchronously (GQ_ERR_INVALID / GQ_ERR_UNSUPPORTED) and
+ *     nothing is enqueued.  A launch failure returns GQ_ERR_CUDA.  Non-finite input does not
+ *     fail the call: it raises a flag on the plan that gq_plan_status reports; the outputs of
+ *     the affected bucket are then unspecified (but every access stays in bounds).
+ *   - The library never allocates inside a call except gq_plan_create.
+ */
+#ifndef GQ_H
+#define GQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GQ_API __attribute__((visibility("default")))
+#else
+#define GQ_API
+#endif
+
+#define GQ_MAX_WORKERS 64
+#define GQ_MIN_BUCKET 128
+#define GQ_MAX_BUCKET 32768
+#define GQ_MAX_LEVELS 16
+
+typedef enum {
+    GQ_QSGD = 0,       /* s uniform levels on [-m, m], m = max|u| of the bucket, stochastic rounding */
+    GQ_TERNGRAD = 1,   /* QSGD with s = 3: levels {-m, 0, m} */
+    GQ_BINGRAD_B = 2,  /* two levels at the side means of the SSE-optimal split, deterministic */
+    GQ_BINGRAD_PB = 3, /* two grid levels minimising expected squared error; stochastic inside, clamped outside */
+    GQ_ORQ = 4         /* s levels: {min, max} plus s-2 greedy picks from a 64-point grid, stochastic rounding */
+} gq_scheme_t;
+
+typedef enum {
+    GQ_OK = 0,
+    GQ_ERR_INVALID = 1,     /* an argument is out of range, NULL where required, or misaligned */
+    GQ_ERR_UNSUPPORTED = 2, /* a valid combination this build does not implement */
+    GQ_ERR_CUDA = 3,        /* a CUDA call failed (launch, allocation of the plan's status word) */
+    GQ_ERR_NONFINITE = 4,   /* gq_plan_status: some input value was NaN or infinite */
+    GQ_ERR_NOMEM = 5        /* host allocation failed */
+} gq_status_t;
+
+/*
+ * Configuration of a plan.
+ *   scheme         gq_scheme_t.
+ *   levels         s.  QSGD: 2..16.  TernGrad: 3 (0 means 3).  BinGrad-b/pb: 2 (0 means 2).
+ *                  ORQ: 2..16.  Codes take b = ceil(log2 s) bits (1..4).
+ *   bucket         d, elements per bucket: a power of two in [128, 32768].  The vector is cut
+ *                  into ceil(n/d) buckets; the last one may hold fewer than d elements.
+ *   workers        W in [1, 64] for gq_fused_step (gq_encode ignores it).
+ *   error_feedback 1: v = g + r is quantized and r <- v - Q(v); 0: v = g, no residual.
+ *   clip_sigma     c >= 0.  c > 0 clips each bucket to [-c*sigma, c*sigma] before the fit
+ *                  (sigma: the bucket's population standard deviation); the residual keeps the
+ *                  clipped part.  0 disables clipping.
+ *   seed           key of the Philox4x32-10 stream used for stochastic rounding.
+ *   n              elements per worker, 0 <= n < 2^40.
+ */
+typedef struct {
+    int32_t scheme;
+    int32_t levels;
+    int32_t bucket;
+    int32_t workers;
+    int32_t error_feedback;
+    float clip_sigma;
+    uint64_t seed;
+    int64_t n;
+} gq_config_t;
+
+typedef struct gq_plan *gq_plan_t; /* opaque; owned by the library */
+
+/* Validate a configuration without touching any device.  GQ_OK if a plan can be made. */
+GQ_API gq_status_t gq_config_check(const gq_config_t *cfg);
+
+/*
+ * Layout of one worker's message, the bytes a worker would transmit (host computation, no
+ * device needed).  *bytes: total size.  *codes_off: offset of the packed codes, ceil(n/d)
+ * buckets of d*b/32 uint32 words each.  *levels_off: offset (16-byte aligned) of the level
+ * tables, ceil(n/d) tables of L float32 each (L = 1 for QSGD/TernGrad: the scale m; 2 for
+ * BinGrad-b/pb: the two levels; s for ORQ: the ascending levels).
+ * Packing inside a bucket: chunk m holds elements 128m .. 128m+127; element 128m + 4l + c
+ * (l = 0..31, c = 0..3) stores bit j of its code (the index of its level) at bit l of word
+ * (m*b + j)*4 + c.  Padding elements of the last bucket have code 0.
+ * Any output pointer may be NULL.
+ */
+GQ_API gq_status_t gq_message_layout(const gq_config_t *cfg, size_t *bytes, size_t *codes_off, size_t *levels_off);
+
+/* Create a plan: validates cfg, selects kernels and allocates the plan's 4-byte device status
+ * word on the current device (the only device allocation the library makes).  The plan must
+ * be used on that device only. */
+GQ_API gq_status_t gq_plan_create(const gq_config_t *cfg, gq_plan_t *out);
+/* Free the plan (synchronous; the caller must make sure no work of the plan is pending). */
+GQ_API gq_status_t gq_plan_destroy(gq_plan_t plan);
+
+/*
+ * Quantize: one worker's gradient into its message (the "Quantize" step, with error feedback).
+ *   worker    Philox worker index of this gradient (any 32-bit value; the draws for element i
+ *             are keyed on (seed, step, worker, i)).
+ *   step      training step; its low 32 bits key the draws.
+ *   grad      device, n float32, read only.
+ *   residual  device, n float32, read and overwritten with v - Q(v); must be NULL iff the
+ *             plan's error_feedback is 0.
+ *   msg       device, gq_message_layout bytes, written completely.
+ */
+GQ_API gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, float *residual,
+                      void *msg, void *stream);
+
+/*
+ * Dequantize + Aggregate: avg[i] = (sum over w = 0..nmsgs-1, in that order, of the level of
+ * element i in msgs[w]) * (1/nmsgs), in float32.
+ *   msgs      host array of nmsgs (1..64) device pointers to messages written by gq_encode
+ *             or gq_fused_step with this plan's configuration.
+ *   avg       device, n float32, overwritten.
+ */
+GQ_API gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs, int nmsgs, float *avg, void *stream);
+
+/*
+ * The whole step for the plan's W workers: worker w (w = 0..W-1, Philox worker index w) is
+ * quantized as by gq_encode and the mean of the W dequantized gradients is written to avg,
+ * as by gq_decode_accumulate; for d <= 512 the dequantized values never leave the chip.
+ *   grads      host array of W device pointers (n float32 each).
+ *   residuals  host array of W device pointers (in/out), or NULL iff error_feedback is 0.
+ *   msgs       host array of W device pointers receiving the messages, or NULL not to write
+ *              messages (allowed for d <= 512 only; larger buckets go through the messages).
+ *   avg        device, n float32, overwritten.
+ */
+GQ_API gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *grads, float *const *residuals,
+                          void *const *msgs, float *avg, void *stream);
+
+/* Synchronize `stream`, then report and clear the plan's status flags: GQ_ERR_NONFINITE if
+ * a non-finite input was seen since the last call, GQ_ERR_CUDA if the stream failed. */
+GQ_API gq_status_t gq_plan_status(gq_plan_t plan, void *stream);
+
+/* Static description of a status code. */
+GQ_API const char *gq_status_string(gq_status_t status);
+
+/* Library version, "major.minor.patch". */
+GQ_API const char *gq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQ_H */

@@ -75,6 +75,8 @@ def lib():
         L.or_encode.argtypes = [P(_Cfg), ctypes.c_int, ctypes.c_uint64, i64, i64, f32p, f32p, u8p]
         L.or_decode_accumulate.argtypes = [P(_Cfg), P(u8p), ctypes.c_int, i64, i64, f32p]
         L.or_fused_step.argtypes = [P(_Cfg), ctypes.c_uint64, i64, i64, P(f32p), P(f32p), P(u8p), f32p]
+        L.or_fused_bucket.argtypes = [P(_Cfg), ctypes.c_uint64, i64, ctypes.c_int, P(f32p), P(f32p), P(f32p),
+                                      P(u32p), P(f32p), f32p]
         _lib = L
     return _lib
 
@@ -230,3 +232,34 @@ def fused_step(cfg: Config, step, gs, rs=None, with_msgs=True, b0=0, b1=None):
     rc = lib().or_fused_step(ctypes.byref(cfg.c()), step, b0, b1, garr, rarr, marr, _p(avg, ctypes.c_float))
     assert rc == 0
     return avg, msgs
+
+
+def fused_bucket(cfg: Config, step, bucket, gs, rs=None):
+    """One bucket of the whole step from per-bucket slices.
+
+    gs / rs: W float32 arrays holding the bucket's n values of each worker (rs None when error
+    feedback is off).  Returns (avg, new residuals or None, packed words per worker, level
+    tables per worker)."""
+    W = len(gs)
+    assert W == cfg.workers
+    n = len(gs[0])
+    f32p = ctypes.POINTER(ctypes.c_float)
+    u32p = ctypes.POINTER(ctypes.c_uint32)
+    gs = [_f32(g) for g in gs]
+    garr = (f32p * W)(*[_p(g, ctypes.c_float) for g in gs])
+    rin = rout = None
+    routs = None
+    if rs is not None:
+        rs = [_f32(r) for r in rs]
+        routs = [np.zeros(n, dtype=np.float32) for _ in range(W)]
+        rin = (f32p * W)(*[_p(r, ctypes.c_float) for r in rs])
+        rout = (f32p * W)(*[_p(r, ctypes.c_float) for r in routs])
+    words = [np.zeros(cfg.bucket * bits(cfg.levels) // 32, dtype=np.uint32) for _ in range(W)]
+    tables = [np.zeros(table_len(cfg.scheme, cfg.levels), dtype=np.float32) for _ in range(W)]
+    warr = (u32p * W)(*[_p(x, ctypes.c_uint32) for x in words])
+    tarr = (f32p * W)(*[_p(x, ctypes.c_float) for x in tables])
+    avg = np.zeros(max(n, 1), dtype=np.float32)
+    rc = lib().or_fused_bucket(ctypes.byref(cfg.c()), step, bucket, n, garr, rin, rout, warr, tarr,
+                               _p(avg, ctypes.c_float))
+    assert rc == 0
+    return avg[:n], routs, words, tables

@@ -90,6 +90,10 @@ int or_decode_accumulate(const or_config *cfg, const uint8_t *const *msgs, int n
                          int64_t b0, int64_t b1, float *avg);
 int or_fused_step(const or_config *cfg, uint64_t step, int64_t b0, int64_t b1,
                   const float *const *g, float *const *r, uint8_t *const *msgs, float *avg);
+/* One bucket of the whole step, from per-bucket slices (see gq_oracle.c). */
+int or_fused_bucket(const or_config *cfg, uint64_t step, int64_t bucket, int n,
+                    const float *const *g, const float *const *r_in, float *const *r_out,
+                    uint32_t *const *words, float *const *tables, float *avg);
 
 #ifdef __cplusplus
 }

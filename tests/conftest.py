@@ -8,3 +8,12 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (runs on a B200)")
+
+
+def pytest_sessionstart(session):
+    # build the oracle and the CUDA library in-tree if they are missing or stale (nvcc
+    # cross-compiles without a GPU)
+    from oracle import build as obuild
+    from gradient_quantization_communication_b200 import build as gbuild
+    obuild.build()
+    gbuild.build()

@@ -1,0 +1,101 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol include/gq.h declares, and
+its host-side logic (argument checks, message layout, status strings) is right.  The layout is
+checked against the oracle's own, independently written, layout computation."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import gradient_quantization_communication_b200.gq as G
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "gq.h")) as f:
+        hdr = f.read()
+    return re.findall(r"GQ_API\s+[\w\s\*]+?\b(gq_\w+)\s*\(", hdr)
+
+
+def test_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 10
+    L = ctypes.CDLL(G.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", G.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln and ln.split()[-1].startswith("gq_")}
+    assert exported == set(names)
+
+
+def test_library_has_sm100a_code():
+    out = subprocess.run(["cuobjdump", "--list-elf", G.LIB_PATH], capture_output=True, text=True).stdout
+    assert "sm_100a" in out
+
+
+def test_version_and_status_strings():
+    assert G.gq_version().count(".") == 2
+    assert G.gq_status_string(G.GQ_OK) == "ok"
+    assert G.gq_status_string(G.GQ_ERR_NONFINITE) == "non-finite input value"
+    assert "unknown" in G.gq_status_string(99)
+
+
+@pytest.mark.parametrize("kw,ok", [
+    (dict(scheme="orq", levels=5), True),
+    (dict(scheme="orq", levels=16), True),
+    (dict(scheme="orq", levels=17), False),
+    (dict(scheme="orq", levels=1), False),
+    (dict(scheme="qsgd", levels=2), True),
+    (dict(scheme="terngrad", levels=0), True),
+    (dict(scheme="terngrad", levels=5), False),
+    (dict(scheme="bingrad_b", levels=0), True),
+    (dict(scheme="bingrad_pb", levels=3), False),
+    (dict(scheme=7, levels=3), False),
+    (dict(scheme="orq", levels=5, bucket=64), False),
+    (dict(scheme="orq", levels=5, bucket=384), False),
+    (dict(scheme="orq", levels=5, bucket=65536), False),
+    (dict(scheme="orq", levels=5, bucket=32768), True),
+    (dict(scheme="orq", levels=5, workers=0), False),
+    (dict(scheme="orq", levels=5, workers=65), False),
+    (dict(scheme="orq", levels=5, clip_sigma=-1.0), False),
+    (dict(scheme="orq", levels=5, clip_sigma=float("inf")), False),
+    (dict(scheme="orq", levels=5, n=-1), False),
+    (dict(scheme="orq", levels=5, n=1 << 40), False),
+    (dict(scheme="orq", levels=5, n=0), True),
+])
+def test_config_check(kw, ok):
+    base = dict(bucket=512, workers=2, error_feedback=True, clip_sigma=0.0, seed=1, n=1000)
+    base.update(kw)
+    st = G.gq_config_check(G.gq_config(**base))
+    assert (st == G.GQ_OK) == ok
+    if not ok:
+        assert st == G.GQ_ERR_INVALID
+
+
+@pytest.mark.parametrize("scheme,levels", [(0, 5), (1, 3), (2, 2), (3, 2), (4, 2), (4, 5), (4, 9), (0, 16), (4, 3)])
+@pytest.mark.parametrize("d", [128, 512, 4096, 32768])
+@pytest.mark.parametrize("n", [0, 1, 127, 1000, 11689512, 10 ** 9])
+def test_message_layout_matches_oracle(scheme, levels, d, n):
+    mine = G.gq_message_layout(G.gq_config(scheme, levels, d, 1, True, 0.0, 0, n))
+    ref = O.message_layout(O.Config(scheme, levels, d, 1, 1, 0.0, 0, n))
+    assert mine == ref
+    assert mine[2] % 16 == 0 and mine[0] % 16 == 0
+
+
+def test_compression_ratio_orq5_d512():
+    # 3 bits per element plus a 5-float table per 512-element bucket
+    n = 512 * 1000
+    nbytes, _, _ = G.gq_message_layout(G.gq_config("orq", 5, 512, 1, True, 0.0, 0, n))
+    assert abs(32 * n / (8 * nbytes) - 9.6603773) < 1e-6
+
+
+def test_plan_create_without_device_fails_cleanly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    with pytest.raises(G.GQError) as ei:
+        G.gq_plan_create(G.gq_config("orq", 5, 512, 1, True, 0.0, 0, 100))
+    assert ei.value.status == G.GQ_ERR_CUDA

@@ -1,0 +1,213 @@
+"""GPU parity: the CUDA library against the CPU oracle, element by element.
+
+Expected agreement is bit-exact for codes, level tables, residuals and averages: every fit
+decision is taken from exact integer data on both sides and every floating-point operation
+is a single IEEE rounding.  (The acceptance bar is looser: codes bit-exact for QSGD, TernGrad
+and BinGrad, >= 99.99 % for ORQ, average within 1e-5 relative L2, residuals within 1e-6.)
+Sizes span several buckets and a ragged tail; edge cases cover constant, zero, grid-aligned,
+tiny and subnormal buckets, n < d, a single element, clipping, no error feedback, and every
+bucket size 128 .. 32768.
+"""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+from gpu_harness import compare_steps, configs, run_gpu_fused, run_oracle_fused
+from gradient_quantization_communication_b200 import synth
+
+
+def _grads(n, W, steps, seed, dist="laplace"):
+    rng = np.random.default_rng(seed)
+    out = []
+    for t in range(steps):
+        row = []
+        for w in range(W):
+            if dist == "laplace":
+                x = rng.laplace(0, 1e-3, n)
+            elif dist == "t3":
+                x = rng.standard_t(3, n) * 1e-3
+            else:
+                x = rng.standard_normal(n) * 1e-3
+            row.append(x.astype(np.float32))
+        out.append(row)
+    return out
+
+
+SCHEMES = [("qsgd", 5), ("qsgd", 2), ("qsgd", 9), ("terngrad", 3), ("bingrad_b", 2), ("bingrad_pb", 2),
+           ("orq", 2), ("orq", 3), ("orq", 4), ("orq", 5), ("orq", 9), ("orq", 16), ("qsgd", 16)]
+
+
+@pytest.mark.parametrize("scheme,levels", SCHEMES)
+@pytest.mark.parametrize("d", [128, 256, 512])
+def test_fused_register_path(scheme, levels, d):
+    n, W, steps = 9 * d + 37, 3, 2
+    cg, co = configs(scheme, levels, d, W, True, 0.0, 42, n)
+    g = _grads(n, W, steps, seed=d + levels)
+    compare_steps(run_gpu_fused(cg, steps, g), run_oracle_fused(co, steps, g), co, "%s-%d d=%d" % (scheme, levels, d))
+
+
+@pytest.mark.parametrize("scheme,levels", [("qsgd", 5), ("terngrad", 3), ("bingrad_b", 2), ("bingrad_pb", 2),
+                                           ("orq", 3), ("orq", 5), ("orq", 9)])
+@pytest.mark.parametrize("d", [128, 512])
+def test_unfused_matches_oracle(scheme, levels, d):
+    n, W, steps = 7 * d + 40, 2, 2
+    cg, co = configs(scheme, levels, d, W, True, 0.0, 7, n)
+    g = _grads(n, W, steps, seed=3 * d + levels, dist="t3")
+    compare_steps(run_gpu_fused(cg, steps, g, unfused=True), run_oracle_fused(co, steps, g), co, "unfused")
+
+
+@pytest.mark.parametrize("scheme,levels", [("qsgd", 5), ("orq", 5), ("orq", 3), ("bingrad_b", 2), ("bingrad_pb", 2),
+                                           ("terngrad", 3)])
+@pytest.mark.parametrize("d", [1024, 2048, 8192, 32768])
+def test_large_buckets(scheme, levels, d):
+    nbk = {1024: 5, 2048: 3, 8192: 2, 32768: 2}[d]
+    if scheme == "bingrad_pb" and d >= 8192:
+        nbk = 1          # the oracle's exhaustive pair search is slow on big buckets
+    n, W, steps = nbk * d - 37 if nbk > 1 else d - 37, 2, 2
+    cg, co = configs(scheme, levels, d, W, True, 0.0, 11, n)
+    g = _grads(n, W, steps, seed=d + levels, dist="t3")
+    compare_steps(run_gpu_fused(cg, steps, g), run_oracle_fused(co, steps, g), co, "%s-%d d=%d" % (scheme, levels, d))
+
+
+@pytest.mark.parametrize("scheme,levels", [("qsgd", 5), ("orq", 3), ("orq", 5), ("bingrad_b", 2), ("bingrad_pb", 2)])
+@pytest.mark.parametrize("d", [512, 2048])
+def test_clip(scheme, levels, d):
+    n, W, steps = 4 * d + 100, 2, 2
+    cg, co = configs(scheme, levels, d, W, True, 2.5, 5, n)
+    g = _grads(n, W, steps, seed=99, dist="t3")
+    g[0][0][17] = 0.5   # an outlier the clip must catch
+    compare_steps(run_gpu_fused(cg, steps, g), run_oracle_fused(co, steps, g), co, "clip")
+
+
+@pytest.mark.parametrize("scheme,levels", [("qsgd", 5), ("orq", 5), ("bingrad_b", 2)])
+@pytest.mark.parametrize("d", [128, 512, 2048])
+def test_no_error_feedback(scheme, levels, d):
+    n, W, steps = 6 * d + 3, 8, 1
+    cg, co = configs(scheme, levels, d, W, False, 0.0, 1, n)
+    g = _grads(n, W, steps, seed=5, dist="normal")
+    compare_steps(run_gpu_fused(cg, steps, g), run_oracle_fused(co, steps, g), co, "no-ef")
+
+
+@pytest.mark.parametrize("kind", ["zero", "constant", "negconst", "grid", "twovalue", "tiny", "spike", "subnormal"])
+@pytest.mark.parametrize("scheme,levels", [("qsgd", 5), ("orq", 5), ("orq", 9), ("bingrad_b", 2), ("bingrad_pb", 2)])
+@pytest.mark.parametrize("d", [512, 1024])
+def test_special_buckets(kind, scheme, levels, d):
+    W = 2
+    parts = [synth.special_bucket(kind, d, seed=w).numpy() for w in range(W)]
+    # a normal bucket after the special one, then a ragged tail
+    rng = np.random.default_rng(0)
+    g = [[np.concatenate([parts[w], (rng.standard_normal(d + 40) * 1e-3).astype(np.float32)]) for w in range(W)]]
+    n = g[0][0].size
+    cg, co = configs(scheme, levels, d, W, True, 0.0, 3, n)
+    compare_steps(run_gpu_fused(cg, 1, g), run_oracle_fused(co, 1, g), co, kind)
+
+
+@pytest.mark.parametrize("n", [1, 3, 4, 127, 129, 500])
+@pytest.mark.parametrize("scheme,levels", [("orq", 5), ("qsgd", 3), ("bingrad_b", 2), ("bingrad_pb", 2)])
+def test_short_vectors(n, scheme, levels):
+    for d in (128, 512, 2048):
+        cg, co = configs(scheme, levels, d, 2, True, 0.0, 9, n)
+        g = _grads(n, 2, 2, seed=n)
+        compare_steps(run_gpu_fused(cg, 2, g), run_oracle_fused(co, 2, g), co, "n=%d d=%d" % (n, d))
+
+
+def test_fused_without_messages_matches():
+    n, W = 20 * 512 + 5, 4
+    cg, co = configs("orq", 5, 512, W, True, 0.0, 42, n)
+    g = _grads(n, W, 2, seed=1)
+    a = run_gpu_fused(cg, 2, g, with_msgs=False)
+    o = run_oracle_fused(co, 2, g)
+    for (ga, gr, _), (oa, orr, _) in zip(a, o):
+        assert np.array_equal(ga.view(np.uint32), oa.view(np.uint32))
+        assert all(np.array_equal(x, y) for x, y in zip(gr, orr))
+
+
+def test_many_workers():
+    n, W = 3 * 512 + 11, 64
+    cg, co = configs("orq", 5, 512, W, True, 0.0, 2, n)
+    g = _grads(n, W, 1, seed=64)
+    compare_steps(run_gpu_fused(cg, 1, g), run_oracle_fused(co, 1, g), co, "W=64")
+
+
+def test_empty_vector():
+    import gradient_quantization_communication_b200.gq as G
+    cg, _ = configs("orq", 5, 512, 2, True, 0.0, 1, 0)
+    with G.Plan(cg) as plan:
+        e = torch.empty(0, device="cuda")
+        G.gq_fused_step(plan.handle, 0, [e, e], [e, e], None, e)
+        assert G.gq_plan_status(plan.handle) == G.GQ_OK
+
+
+def test_nonfinite_input_is_flagged():
+    import gradient_quantization_communication_b200.gq as G
+    for d in (512, 2048):
+        n = 3 * d
+        cg, _ = configs("orq", 5, d, 2, True, 0.0, 1, n)
+        g = [torch.randn(n, device="cuda") * 1e-3 for _ in range(2)]
+        g[1][d + 5] = float("nan")
+        g[0][7] = float("inf")
+        r = [torch.zeros(n, device="cuda") for _ in range(2)]
+        with G.Plan(cg) as plan:
+            msgs = [torch.zeros(plan.msg_bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+            avg = torch.zeros(n, device="cuda")
+            G.gq_fused_step(plan.handle, 0, g, r, msgs, avg)
+            assert G.gq_plan_status(plan.handle) == G.GQ_ERR_NONFINITE
+            # the flag is cleared by reading it; clean input raises nothing
+            g[1][d + 5] = 0.0
+            g[0][7] = 0.0
+            G.gq_fused_step(plan.handle, 1, g, [torch.zeros(n, device="cuda") for _ in range(2)], msgs, avg)
+            assert G.gq_plan_status(plan.handle) == G.GQ_OK
+
+
+def test_invalid_arguments_rejected():
+    import gradient_quantization_communication_b200.gq as G
+    cg, _ = configs("orq", 5, 512, 2, True, 0.0, 1, 1024)
+    with G.Plan(cg) as plan:
+        g = torch.zeros(1024, device="cuda")
+        msg = torch.zeros(plan.msg_bytes, dtype=torch.uint8, device="cuda")
+        with pytest.raises(G.GQError) as ei:   # residual required with error feedback on
+            G.gq_encode(plan.handle, 0, 0, g, None, msg)
+        assert ei.value.status == G.GQ_ERR_INVALID
+        with pytest.raises(G.GQError):         # misaligned gradient
+            G.gq_encode(plan.handle, 0, 0, g.data_ptr() + 4, g, msg)
+        with pytest.raises(G.GQError):         # no messages for a fused step with d > 512 is
+            cg2, _ = configs("orq", 5, 2048, 2, True, 0.0, 1, 4096)      # checked per plan
+            with G.Plan(cg2) as p2:
+                x = torch.zeros(4096, device="cuda")
+                G.gq_fused_step(p2.handle, 0, [x, x], [x.clone(), x.clone()], None, x.clone())
+
+
+def test_deterministic_repeat():
+    """Two runs on the same inputs are bitwise identical (catches races in shared memory)."""
+    n, W = 50 * 512 + 9, 4
+    cg, _ = configs("orq", 5, 512, W, True, 0.0, 3, n)
+    g = _grads(n, W, 2, seed=8)
+    a = run_gpu_fused(cg, 2, g)
+    b = run_gpu_fused(cg, 2, g)
+    for (aa, ar, am), (ba, br, bm) in zip(a, b):
+        assert np.array_equal(aa.view(np.uint32), ba.view(np.uint32))
+        assert all(np.array_equal(x, y) for x, y in zip(am, bm))
+
+
+def test_checkpoint_resume_is_bit_identical():
+    """The only state is the residual and the step: 4 steps in one go equal 2 + save/restore + 2."""
+    import gradient_quantization_communication_b200.gq as G
+    n, W = 10 * 512 + 3, 2
+    cg, _ = configs("orq", 3, 512, W, True, 0.0, 77, n)
+    g = _grads(n, W, 4, seed=12)
+    full = run_gpu_fused(cg, 4, g)
+    with G.Plan(cg) as plan:
+        r = [torch.zeros(n, device="cuda") for _ in range(W)]
+        for t in range(2):
+            G.gq_fused_step(plan.handle, t, [torch.from_numpy(x).cuda() for x in g[t]], r, None,
+                            torch.empty(n, device="cuda"))
+        saved = [x.cpu().clone() for x in r]
+    with G.Plan(cg) as plan:
+        r = [x.cuda() for x in saved]
+        for t in range(2, 4):
+            avg = torch.empty(n, device="cuda")
+            G.gq_fused_step(plan.handle, t, [torch.from_numpy(x).cuda() for x in g[t]], r, None, avg)
+            assert np.array_equal(avg.cpu().numpy().view(np.uint32), full[t][0].view(np.uint32))
+        assert all(np.array_equal(x.cpu().numpy(), y) for x, y in zip(r, full[3][1]))
