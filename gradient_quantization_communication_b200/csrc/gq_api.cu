@@ -95,6 +95,10 @@ gq::KParams base_params(const gq_plan &pl, uint64_t step)
     p.clip = pl.cfg.clip_sigma;
     p.key0 = (uint32_t)pl.cfg.seed;
     p.key1 = (uint32_t)(pl.cfg.seed >> 32);
+    for (int i = 0; i < 10; ++i) {
+        p.rk0[i] = p.key0 + (uint32_t)i * 0x9E3779B9u;
+        p.rk1[i] = p.key1 + (uint32_t)i * 0xBB67AE85u;
+    }
     p.step_lo = (uint32_t)step;
     p.worker0 = 0;
     p.inv_w = 1.0f;
@@ -169,12 +173,13 @@ gq_status_t gq_plan_destroy(gq_plan_t plan)
 gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, float *residual, void *msg,
                       void *stream)
 {
-    if (!plan || !grad || !msg || !aligned16(grad) || !aligned16(msg)) return GQ_ERR_INVALID;
+    if (!plan) return GQ_ERR_INVALID;
+    if (plan->cfg.n == 0) return GQ_OK;  // nothing to read or write: pointers may be NULL
+    if (!grad || !msg || !aligned16(grad) || !aligned16(msg)) return GQ_ERR_INVALID;
     if ((plan->cfg.error_feedback != 0) != (residual != nullptr)) return GQ_ERR_INVALID;
     if (residual && !aligned16(residual)) return GQ_ERR_INVALID;
     gq_status_t st = check_device(*plan);
     if (st != GQ_OK) return st;
-    if (plan->cfg.n == 0) return GQ_OK;
     gq::KParams p = base_params(*plan, step);
     p.worker0 = worker;
     p.g[0] = grad;
@@ -187,12 +192,13 @@ gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const floa
 
 gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs, int nmsgs, float *avg, void *stream)
 {
-    if (!plan || !msgs || !avg || nmsgs < 1 || nmsgs > GQ_MAX_WORKERS || !aligned16(avg)) return GQ_ERR_INVALID;
+    if (!plan || nmsgs < 1 || nmsgs > GQ_MAX_WORKERS) return GQ_ERR_INVALID;
+    if (plan->cfg.n == 0) return GQ_OK;  // nothing to read or write: pointers may be NULL
+    if (!msgs || !avg || !aligned16(avg)) return GQ_ERR_INVALID;
     for (int w = 0; w < nmsgs; ++w)
         if (!msgs[w] || !aligned16(msgs[w])) return GQ_ERR_INVALID;
     gq_status_t st = check_device(*plan);
     if (st != GQ_OK) return st;
-    if (plan->cfg.n == 0) return GQ_OK;
     gq::KParams p = base_params(*plan, 0);
     p.W = nmsgs;
     p.inv_w = 1.0f / (float)nmsgs;
@@ -204,7 +210,9 @@ gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs, int nm
 gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *grads, float *const *residuals,
                           void *const *msgs, float *avg, void *stream)
 {
-    if (!plan || !grads || !avg || !aligned16(avg)) return GQ_ERR_INVALID;
+    if (!plan) return GQ_ERR_INVALID;
+    if (plan->cfg.n == 0) return GQ_OK;  // nothing to read or write: pointers may be NULL
+    if (!grads || !avg || !aligned16(avg)) return GQ_ERR_INVALID;
     const int W = plan->cfg.workers;
     const bool ef = plan->cfg.error_feedback != 0;
     if (ef != (residuals != nullptr)) return GQ_ERR_INVALID;
@@ -216,7 +224,6 @@ gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *gra
     if (!msgs && plan->cfg.bucket > 512) return GQ_ERR_INVALID;
     gq_status_t st = check_device(*plan);
     if (st != GQ_OK) return st;
-    if (plan->cfg.n == 0) return GQ_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     gq::KParams p = base_params(*plan, step);
     if (plan->cfg.bucket <= 512) {
@@ -255,6 +262,7 @@ gq_status_t gq_plan_status(gq_plan_t plan, void *stream)
     if (cudaMemcpyAsync(&flags, plan->status, sizeof flags, cudaMemcpyDeviceToHost, s) != cudaSuccess) return GQ_ERR_CUDA;
     if (cudaMemsetAsync(plan->status, 0, sizeof(unsigned int), s) != cudaSuccess) return GQ_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return GQ_ERR_CUDA;
+    if (flags & gq::kStatusTimeout) return GQ_ERR_CUDA;
     if (flags & gq::kStatusNonFinite) return GQ_ERR_NONFINITE;
     return GQ_OK;
 }

@@ -32,6 +32,7 @@ struct alignas(16) CtaShared {
     int P0[64];
     long long al[64], be[64], ga[64], de[64];
     float4 tab[16];
+    float2 pair[16];
     float lev[16];
     unsigned char lut[64];
     float bcast_f[4];
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
 
         // ---- fit ------------------------------------------------------------------------------
         RoundQSGD rq;
-        RoundORQ ro{sh.lut, sh.tab, sh.lev};
+        RoundORQ ro{sh.lut, sh.tab};
         RoundB rb{0.0f, 0.0f, 0.0f, false};
         RoundPB rp;
         bool constant = false;
@@ -212,13 +213,17 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
             for (int i = tid; i < nvalid; i += kCtaThreads) m = fmaxf(m, fabsf(clipped(vs[i])));
             m = block_max(m, sh, 0);
             const int s = p.s;
-            if (tid < s) sh.lev[tid] = __fmul_rn(m, __fdiv_rn((float)(2 * tid - (s - 1)), (float)(s - 1)));
+            if (wid == 0) {
+                const float lv = lane < s ? __fmul_rn(m, __fdiv_rn((float)(2 * lane - (s - 1)), (float)(s - 1))) : 0.0f;
+                const float lv_next = __shfl_down_sync(kFull, lv, 1);
+                if (lane < s - 1) sh.pair[lane] = make_float2(lv, lv_next);
+            }
             if (tid == 0) sh.bcast_f[0] = m;
             __syncthreads();
             rq.inv_m = m > 0.0f ? __fdiv_rn(1.0f, m) : 0.0f;
             rq.h = __fmul_rn((float)(s - 1), 0.5f);
-            rq.s = s;
-            rq.lev = sh.lev;
+            rq.kmax = s - 2;
+            rq.pair = sh.pair;
         } else if constexpr (SCHEME == GQ_ORQ || SCHEME == GQ_BINGRAD_PB) {
             float lo = INFINITY, hi = -INFINITY;
             for (int i = tid; i < nvalid; i += kCtaThreads) {
@@ -280,7 +285,7 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                         __syncwarp();
                         if (lane < p.s - 1) {
                             const float l0 = sh.lev[lane], l1 = sh.lev[lane + 1];
-                            sh.tab[lane] = make_float4(l0, l1, __fdiv_rn(1.0f, __fsub_rn(l1, l0)), 0.0f);
+                            sh.tab[lane] = make_float4(l0, l1, __fdiv_rn(1.0f, __fsub_rn(l1, l0)), __int_as_float(lane));
                         }
                     }
                     __syncthreads();
@@ -520,19 +525,19 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
             uint32_t *cwc = cw ? cw + ch * 4 * p.bits : nullptr;
             float q[4];
             if constexpr (SCHEME == GQ_QSGD) {
-                round_chunk<true>(p, rq, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                round_chunk<true, false>(p, rq, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             } else if constexpr (SCHEME == GQ_ORQ) {
                 if (constant)
-                    round_chunk<false>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    round_chunk<false, false>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
                 else
-                    round_chunk<true>(p, ro, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    round_chunk<true, false>(p, ro, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             } else if constexpr (SCHEME == GQ_BINGRAD_PB) {
                 if (constant)
-                    round_chunk<false>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    round_chunk<false, false>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
                 else
-                    round_chunk<true>(p, rp, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    round_chunk<true, false>(p, rp, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             } else {
-                round_chunk<false>(p, rb, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                round_chunk<false, false>(p, rb, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             }
         }
         // ---- level table --------------------------------------------------------------------------

@@ -24,29 +24,24 @@ constexpr int kPbFBits = 16;          // fraction bits of BinGrad-pb fixed-point
 
 // ---------------------------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3",
-// SC'11): ten rounds, each two 32x32->64-bit products of counter words 0 and 2 with the
-// round multipliers, the high halves xor-ed with the other counter words and the round key;
-// the key advances by the two Weyl increments between rounds.
+// SC'11): ten rounds, each two 32x32->64-bit products of counter words 0 and 2 with the round
+// multipliers, the high halves xor-ed with the other counter words and the round key; the key
+// advances by the two Weyl increments between rounds.  The ten round keys are computed once on
+// the host (KParams::rk0 / rk1), so a round costs two wide multiplies and two xors.
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
-                                               uint32_t k0, uint32_t k1)
+                                               const uint32_t *rk0, const uint32_t *rk1)
 {
 #pragma unroll
     for (int round = 0; round < 10; ++round) {
-        if (round > 0) {
-            k0 += 0x9E3779B9u;
-            k1 += 0xBB67AE85u;
-        }
-        const uint32_t lo0 = 0xD2511F53u * c0;
-        const uint32_t hi0 = __umulhi(0xD2511F53u, c0);
-        const uint32_t lo1 = 0xCD9E8D57u * c2;
-        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2);
-        const uint32_t y0 = hi1 ^ c1 ^ k0;
-        const uint32_t y2 = hi0 ^ c3 ^ k1;
+        const unsigned long long p0 = (unsigned long long)0xD2511F53u * c0;
+        const unsigned long long p1 = (unsigned long long)0xCD9E8D57u * c2;
+        const uint32_t y0 = (uint32_t)(p1 >> 32) ^ c1 ^ rk0[round];
+        const uint32_t y2 = (uint32_t)(p0 >> 32) ^ c3 ^ rk1[round];
+        c1 = (uint32_t)p1;
+        c3 = (uint32_t)p0;
         c0 = y0;
-        c1 = lo1;
         c2 = y2;
-        c3 = lo0;
     }
     return make_uint4(c0, c1, c2, c3);
 }
@@ -55,7 +50,7 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
 // (blk low word, blk high word, step low word, worker), the key the two words of the seed.
 __device__ __forceinline__ uint4 draws4(const KParams &p, uint64_t blk, uint32_t worker)
 {
-    return philox4x32_10((uint32_t)blk, (uint32_t)(blk >> 32), p.step_lo, worker, p.key0, p.key1);
+    return philox4x32_10((uint32_t)blk, (uint32_t)(blk >> 32), p.step_lo, worker, p.rk0, p.rk1);
 }
 
 // Uniform in [0, 1) at 24-bit resolution from one Philox output word.
@@ -98,6 +93,14 @@ __device__ __forceinline__ float fmax_nan(float a, float b)
     return r;
 }
 
+// min that propagates NaN.
+__device__ __forceinline__ float fmin_nan(float a, float b)
+{
+    float r;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
 // Round to nearest even, float64 -> int64.
 __device__ __forceinline__ long long fixed_point(float x, double scale)
 {
@@ -123,6 +126,12 @@ __device__ __forceinline__ float warp_max_nan(float x)
 {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x = fmax_nan(x, __shfl_xor_sync(kFull, x, o));
+    return x;
+}
+__device__ __forceinline__ float warp_min_nan(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmin_nan(x, __shfl_xor_sync(kFull, x, o));
     return x;
 }
 __device__ __forceinline__ long long warp_sum(long long x)
@@ -178,6 +187,9 @@ __device__ __forceinline__ float clip_threshold_from_sums(long long sx, long lon
 __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const long long *P1, int s, int lane)
 {
     unsigned long long mask = 1ull | (1ull << 63);
+    // the lane's two candidates and their own prefix values do not change across rounds
+    const int P0c[2] = {P0[lane], P0[lane + 32]};
+    const long long P1c[2] = {P1[lane], P1[lane + 32]};
     for (int round = 0; round < s - 2; ++round) {
         unsigned long long best = 0;
 #pragma unroll
@@ -188,15 +200,17 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const lo
                 const unsigned long long above = mask & ~((2ull << C) - 1ull);
                 const int A = 63 - __clzll((long long)below);
                 const int B = __ffsll((long long)above) - 1;
-                const long long lows = (P1[C] - P1[A]) - ((long long)A << kOrqFBits) * (long long)(P0[C] - P0[A]);
-                const long long highs = ((long long)B << kOrqFBits) * (long long)(P0[B] - P0[C]) - (P1[B] - P1[C]);
+                const long long lows = (P1c[h] - P1[A]) - (long long)(A << kOrqFBits) * (P0c[h] - P0[A]);
+                const long long highs = (long long)(B << kOrqFBits) * (P0[B] - P0c[h]) - (P1[B] - P1c[h]);
                 const long long delta = (long long)(B - C) * lows + (long long)(C - A) * highs;
                 const unsigned long long key = ((unsigned long long)delta << 6) | (unsigned long long)(63 - C);
                 best = key > best ? key : best;
             }
         }
-        best = warp_max_u64(best);
-        mask |= 1ull << (63 - (int)(best & 63ull));
+        // warp argmax of the 64-bit key: high words first, then low words among the lanes that tie
+        const unsigned hi = __reduce_max_sync(kFull, (unsigned)(best >> 32));
+        const unsigned lo = __reduce_max_sync(kFull, (unsigned)(best >> 32) == hi ? (unsigned)best : 0u);
+        mask |= 1ull << (63 - (int)(lo & 63u));
     }
     return mask;
 }
@@ -213,6 +227,73 @@ __device__ __forceinline__ int grid_pos(float u, float mn, float scale)
 {
     const int y = __float2int_rz(__fmul_rn(__fsub_rn(u, mn), scale));
     return min(max(y, 0), 63 << F);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Bulk asynchronous copies (TMA, no multicast) into shared memory, completed on an mbarrier.
+// Every wait is bounded: after kWaitLimitNs of global time it gives up and reports failure.
+// ---------------------------------------------------------------------------------------------
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // one second
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(unsigned long long *bar, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make barrier initialisation (generic proxy) visible to the copy engine (async proxy).
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order this thread's earlier generic accesses of shared memory before later async-proxy writes.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long *bar, unsigned bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+// 1-D bulk copy global -> shared of `bytes` (multiple of 16, both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned bytes, unsigned long long *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long *bar, unsigned parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Warp-uniform bounded wait for the phase `parity` of `bar`; false if it timed out.
+__device__ __forceinline__ bool mbar_wait_warp(unsigned long long *bar, unsigned parity)
+{
+    if (__all_sync(kFull, mbar_try_wait(bar, parity))) return true;
+    const unsigned long long t0 = global_ns();
+    for (;;) {
+        if (__all_sync(kFull, mbar_try_wait(bar, parity))) return true;
+        const bool late = global_ns() - t0 > kWaitLimitNs;
+        if (__any_sync(kFull, late)) return false;
+    }
 }
 
 }  // namespace gq

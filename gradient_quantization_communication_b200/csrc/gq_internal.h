@@ -22,6 +22,8 @@ struct KParams {
     int tail;            // valid elements of the last bucket (1..d)
     float clip;          // c of the +-c*sigma clip, 0 = off
     uint32_t key0, key1; // Philox key (seed)
+    uint32_t rk0[10];    // Philox round keys: key0 + i * 0x9E3779B9
+    uint32_t rk1[10];    //                    key1 + i * 0xBB67AE85
     uint32_t step_lo;    // step, low word
     uint32_t worker0;    // Philox worker index of worker slot 0
     float inv_w;         // 1/W for the average
@@ -36,6 +38,7 @@ struct KParams {
 
 // Status bits raised by kernels.
 constexpr unsigned kStatusNonFinite = 1u;
+constexpr unsigned kStatusTimeout = 2u;  // a bounded wait on a bulk copy gave up
 
 // Register-resident path (d = 128, 256, 512): one warp per bucket index.
 cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream);

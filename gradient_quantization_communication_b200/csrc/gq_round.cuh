@@ -1,79 +1,94 @@
 // gq_round.cuh -- per-element rounding rules of the five schemes and the 128-element chunk
 // step shared by the register path (d <= 512) and the shared-memory path (d >= 1024):
 // draw, round, dequantize, write the residual, bit-plane pack with warp ballots.
+//
+// Every stochastic rule compares U (in [0, 1)) with the unsaturated probability p: U < p has
+// the same truth value as U < clamp(p, 0, 1) for every p, NaN included, so no clamp is needed.
 #pragma once
 
 #include "gq_device.cuh"
 
 namespace gq {
 
-// QSGD / TernGrad: position y = (u/m + 1) * (s-1)/2 in level units; up with probability frac(y).
+// QSGD / TernGrad: position y = (u/m + 1) * (s-1)/2 in level units, bracket k = trunc(y)
+// clamped to [0, s-2], up with probability y - k.  pair[k] = {level k, level k+1}.
 struct RoundQSGD {
     float inv_m, h;
-    int s;
-    const float *lev;
-    __device__ __forceinline__ int code(float u, int, float U) const
+    int kmax;
+    const float2 *pair;
+    __device__ __forceinline__ void round(float u, int, uint32_t word, int &code, float &q) const
     {
         const float y = __fmul_rn(__fadd_rn(__fmul_rn(u, inv_m), 1.0f), h);
-        const int k = min(max(__float2int_rz(y), 0), s - 2);
+        const int k = min(max(__float2int_rz(y), 0), kmax);
         const float pu = __fsub_rn(y, (float)k);
-        return k + (U < pu ? 1 : 0);
+        const bool up = unit_float(word) < pu;
+        const float2 lp = pair[k];
+        code = k + (up ? 1 : 0);
+        q = up ? lp.y : lp.x;
     }
-    __device__ __forceinline__ float level(int c) const { return lev[c]; }
 };
 
-// ORQ: bracket of the value's grid cell, up with probability (u - lower)/(upper - lower).
+// ORQ: bracket of the value's grid cell; tab[k] = {lower, upper, 1/(upper-lower), k as bits};
+// up with probability (u - lower) / (upper - lower).
 struct RoundORQ {
     const unsigned char *lut;
     const float4 *tab;
-    const float *lev;
-    __device__ __forceinline__ int code(float u, int pos, float U) const
+    __device__ __forceinline__ void round(float u, int pos, uint32_t word, int &code, float &q) const
     {
         const int cell = min(pos >> kOrqFBits, kTopCell);
-        const int k = lut[cell];
-        const float4 b = tab[k];
-        const float pu = sat01(__fmul_rn(__fsub_rn(u, b.x), b.z));
-        return k + (U < pu ? 1 : 0);
+        const float4 b = tab[lut[cell]];
+        const float pu = __fmul_rn(__fsub_rn(u, b.x), b.z);
+        const bool up = unit_float(word) < pu;
+        code = __float_as_int(b.w) + (up ? 1 : 0);
+        q = up ? b.y : b.x;
     }
-    __device__ __forceinline__ float level(int c) const { return lev[c]; }
 };
 
 // Constant bucket: one level, code 0.
 struct RoundConst {
     float lv;
-    __device__ __forceinline__ int code(float, int, float) const { return 0; }
-    __device__ __forceinline__ float level(int) const { return lv; }
+    __device__ __forceinline__ void round(float, int, uint32_t, int &code, float &q) const
+    {
+        code = 0;
+        q = lv;
+    }
 };
 
 // BinGrad-b: deterministic, code 1 at or above the split value.
 struct RoundB {
     float a, b, thr;
     bool split;
-    __device__ __forceinline__ int code(float u, int, float) const { return (split && u >= thr) ? 1 : 0; }
-    __device__ __forceinline__ float level(int c) const { return c ? b : a; }
+    __device__ __forceinline__ void round(float u, int, uint32_t, int &code, float &q) const
+    {
+        const bool up = split && u >= thr;
+        code = up ? 1 : 0;
+        q = up ? b : a;
+    }
 };
 
 // BinGrad-pb: clamped below the lower / at or above the upper grid level, stochastic between.
 struct RoundPB {
     float a, b, rinv;
     int pa, pb;
-    __device__ __forceinline__ int code(float u, int pos, float U) const
+    __device__ __forceinline__ void round(float u, int pos, uint32_t word, int &code, float &q) const
     {
-        if (pos < pa) return 0;
-        if (pos >= pb) return 1;
-        const float pu = sat01(__fmul_rn(__fsub_rn(u, a), rinv));
-        return U < pu ? 1 : 0;
+        bool up;
+        if (pos < pa) up = false;
+        else if (pos >= pb) up = true;
+        else up = unit_float(word) < __fmul_rn(__fsub_rn(u, a), rinv);
+        code = up ? 1 : 0;
+        q = up ? b : a;
     }
-    __device__ __forceinline__ float level(int c) const { return c ? b : a; }
 };
 
 // One 128-element chunk of a bucket: lane l holds elements 4l .. 4l+3 of the chunk
-// (v: error-fed values, u: clipped values, pos: grid positions; valid: 4-bit mask).
-//   blk      global element index of the chunk's first element, divided by 4
-//   rout     residual of the chunk's first element (NULL: no residual), 16-byte aligned
-//   cw       packed words of the chunk (b uint4: plane j = words 4j..4j+3), NULL: no message
+// (v: error-fed values, u: clipped values, pos: grid positions; valid: 4-bit mask, ignored
+// when ALLVALID).
+//   blk   global element index of the chunk's first element, divided by 4
+//   rout  residual of the chunk's first element (NULL: no residual), 16-byte aligned
+//   cw    packed words of the chunk (b uint4: plane j = words 4j..4j+3), NULL: no message
 // Returns the dequantized values in q.
-template <bool RANDOM, class R>
+template <bool RANDOM, bool ALLVALID, class R>
 __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uint64_t blk, uint32_t worker, int lane,
                                             uint32_t valid, const float (&v)[4], const float (&u)[4],
                                             const int (&pos)[4], float *rout, uint32_t *cw, float (&q)[4])
@@ -84,12 +99,11 @@ __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uin
     int code[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        const int k = rule.code(u[c], pos[c], RANDOM ? unit_float(words[c]) : 0.0f);
-        code[c] = ((valid >> c) & 1u) ? k : 0;
-        q[c] = rule.level(code[c]);
+        rule.round(u[c], pos[c], words[c], code[c], q[c]);
+        if (!ALLVALID && !((valid >> c) & 1u)) code[c] = 0;
     }
     if (rout) {
-        if (valid == 0xfu) {
+        if (ALLVALID || valid == 0xfu) {
             __stcs(reinterpret_cast<float4 *>(rout + 4 * lane),
                    make_float4(__fsub_rn(v[0], q[0]), __fsub_rn(v[1], q[1]), __fsub_rn(v[2], q[2]), __fsub_rn(v[3], q[3])));
         } else {

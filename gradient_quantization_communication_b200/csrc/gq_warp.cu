@@ -1,100 +1,76 @@
 // gq_warp.cu -- register-resident quantization kernels for buckets of d = 128, 256, 512.
 //
-// One warp owns one bucket index.  Lane l holds EPL = d/32 values in registers, slot t being
-// element 128*(t/4) + 4*l + t%4 of the bucket, so every load and store is a coalesced 16-byte
-// access and the four values of a slot group share one Philox call.  For the fused step the
-// warp walks the W workers of its bucket in worker order, quantizes each, writes the residual
-// (and optionally the message) and accumulates the dequantized values in registers; the
-// average leaves the chip once, after the last worker.  Level fits per bucket:
+// One warp owns one bucket index at a time and walks its items (bucket, worker) in order.  The
+// g and r of each item (2 x d floats) are staged into the warp's shared memory by bulk
+// asynchronous copies (TMA, 1-D, no multicast) two items ahead, completed on per-stage
+// mbarriers, so the copy engine keeps 8 KB per warp in flight while the warp computes and no
+// registers are spent on prefetching.  Lane l then holds EPL = d/32 values in registers, slot
+// t being element 128*(t/4) + 4*l + t%4 of the bucket, so that the four values of a slot
+// group share one Philox call and every global store is a coalesced 16-byte access.  In the
+// fused step the W workers of a bucket are consecutive items: the dequantized values are
+// summed in registers in worker order and the average leaves the chip once.
+//
+// Level fits per bucket:
 //   QSGD / TernGrad : m = max|u|, s uniform levels on [-m, m]
-//   ORQ             : lane-private shared-memory histogram of 22-bit fixed-point grid
-//                     positions -> exact int64 prefix sums -> s-2 greedy rounds
-//   BinGrad-b       : warp bitonic sort -> exact int64 prefix sums -> argmax of J(k)
-//   BinGrad-pb      : shared-memory moments of 16-bit positions -> exact search of all
-//                     2016 grid pairs
+//   ORQ             : shared-memory histogram of 22-bit fixed-point grid positions (8 columns
+//                     per cell, shared atomics), exact int64 prefix sums, s-2 greedy rounds
+//   BinGrad-b       : warp bitonic sort, exact int64 prefix sums, argmax of J(k)
+//   BinGrad-pb      : shared-memory moments of 16-bit positions, exact search of all pairs
+// The last (ragged) bucket is loaded with plain guarded loads instead of bulk copies.
 #include "gq_round.cuh"
 
 namespace gq {
 namespace {
 
 constexpr int kWarpsPerCta = 4;
+constexpr int kStages = 2;
+constexpr int kHistCols = 8;
 
-// ---------------------------------------------------------------------------------------------
-// Per-warp shared memory, one layout per scheme
-// ---------------------------------------------------------------------------------------------
-struct alignas(16) SmemORQ {
-    uint32_t hist[64 * 32];  // [cell][lane]: (count << 27) + sum of 22-bit fractions
-    long long P1[64];        // sum of positions over cells < k
-    int P0[64];              // count over cells < k
-    float4 tab[16];          // bracket k: {lower level, upper level, 1/(upper-lower), 0}
-    float lev[16];           // ascending levels
-    unsigned char lut[64];   // cell -> bracket
+template <int EPL>
+struct alignas(16) StageBuf {
+    float g[32 * EPL];
+    float r[32 * EPL];
 };
-struct alignas(16) SmemQSGD {
-    float lev[16];
+
+struct alignas(16) FitORQ {
+    uint32_t hcnt[64 * kHistCols];  // [cell][column]: element counts
+    uint32_t hsum[64 * kHistCols];  // [cell][column]: sums of 22-bit fractions
+    long long P1[64];               // sum of positions over cells < k
+    int P0[64];                     // count over cells < k
+    float4 tab[16];                 // bracket k: {lower, upper, 1/(upper-lower), k}
+    float lev[16];                  // ascending levels
+    unsigned char lut[64];          // cell -> bracket
 };
-struct alignas(16) SmemPB {
+struct alignas(16) FitQSGD {
+    float2 pair[16];  // {level k, level k+1}
+};
+struct alignas(16) FitPB {
     unsigned long long s1[64], s2[64];  // per cell: sum of positions, of squared positions
     unsigned int cnt[64];               // per cell: count
     long long al[64], be[64], ga[64], de[64];
 };
-struct alignas(16) SmemB {
-    float lev[4];
+struct alignas(16) FitB {
+    int unused;
 };
 
-template <int S> struct SmemFor { using type = SmemQSGD; };
-template <> struct SmemFor<GQ_ORQ> { using type = SmemORQ; };
-template <> struct SmemFor<GQ_BINGRAD_PB> { using type = SmemPB; };
-template <> struct SmemFor<GQ_BINGRAD_B> { using type = SmemB; };
+template <int S> struct FitFor { using type = FitQSGD; };
+template <> struct FitFor<GQ_ORQ> { using type = FitORQ; };
+template <> struct FitFor<GQ_BINGRAD_PB> { using type = FitPB; };
+template <> struct FitFor<GQ_BINGRAD_B> { using type = FitB; };
+
+template <int EPL, int SCHEME>
+struct alignas(16) WarpSmem {
+    StageBuf<EPL> stage[kStages];
+    unsigned long long bar[kStages];
+    typename FitFor<SCHEME>::type fit;
+};
 
 __device__ __forceinline__ int slot_elem(int t, int lane) { return 128 * (t >> 2) + 4 * lane + (t & 3); }
 
 // ---------------------------------------------------------------------------------------------
-// Loads: v = g (+ r)
-// ---------------------------------------------------------------------------------------------
-template <int EPL>
-__device__ __forceinline__ void load_bucket(const float *g, const float *r, int64_t base, int nvalid,
-                                            bool full, int lane, float (&v)[EPL])
-{
-    const float *gb = g + base;
-    if (full) {
-#pragma unroll
-        for (int m = 0; m < EPL / 4; ++m) {
-            const float4 x = __ldcs(reinterpret_cast<const float4 *>(gb + 128 * m + 4 * lane));
-            v[4 * m + 0] = x.x;
-            v[4 * m + 1] = x.y;
-            v[4 * m + 2] = x.z;
-            v[4 * m + 3] = x.w;
-        }
-        if (r) {
-            const float *rb = r + base;
-#pragma unroll
-            for (int m = 0; m < EPL / 4; ++m) {
-                const float4 y = __ldcs(reinterpret_cast<const float4 *>(rb + 128 * m + 4 * lane));
-                v[4 * m + 0] = __fadd_rn(v[4 * m + 0], y.x);
-                v[4 * m + 1] = __fadd_rn(v[4 * m + 1], y.y);
-                v[4 * m + 2] = __fadd_rn(v[4 * m + 2], y.z);
-                v[4 * m + 3] = __fadd_rn(v[4 * m + 3], y.w);
-            }
-        }
-    } else {
-#pragma unroll
-        for (int t = 0; t < EPL; ++t) {
-            const int e = slot_elem(t, lane);
-            float x = 0.0f;
-            if (e < nvalid) {
-                x = gb[e];
-                if (r) x = __fadd_rn(x, r[base + e]);
-            }
-            v[t] = x;
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------------------------
 // Round + pack + residual + accumulate for one worker-bucket, chunk by chunk.
 // ---------------------------------------------------------------------------------------------
-template <int EPL, bool FUSED, bool RANDOM, class R>
+template <int EPL, bool FUSED, bool RANDOM, bool TAIL, class R>
 __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t beta, int w, int lane, uint32_t vmask,
                                      const float (&v)[EPL], const float (&u)[EPL], const int (&pos)[EPL],
                                      float (&acc)[EPL])
@@ -109,14 +85,14 @@ __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t be
         const float vv[4] = {v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]};
         const float uu[4] = {u[4 * m], u[4 * m + 1], u[4 * m + 2], u[4 * m + 3]};
         const int pp[4] = {pos[4 * m], pos[4 * m + 1], pos[4 * m + 2], pos[4 * m + 3]};
-        const uint32_t valid = (vmask >> (4 * m)) & 0xfu;
+        const uint32_t valid = TAIL ? (vmask >> (4 * m)) & 0xfu : 0xfu;
         float q[4];
-        round_chunk<RANDOM>(p, rule, (uint64_t)(base >> 2) + (uint64_t)(32 * m), worker, lane, valid, vv, uu, pp,
-                            r ? r + base + 128 * m : nullptr, cw ? cw + m * 4 * p.bits : nullptr, q);
+        round_chunk<RANDOM, !TAIL>(p, rule, (uint64_t)(base >> 2) + (uint64_t)(32 * m), worker, lane, valid, vv, uu,
+                                   pp, r ? r + base + 128 * m : nullptr, cw ? cw + m * 4 * p.bits : nullptr, q);
         if (FUSED) {
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                if ((valid >> c) & 1u) acc[4 * m + c] = __fadd_rn(acc[4 * m + c], q[c]);
+                if (!TAIL || ((valid >> c) & 1u)) acc[4 * m + c] = __fadd_rn(acc[4 * m + c], q[c]);
         }
     }
 }
@@ -128,114 +104,129 @@ __device__ __forceinline__ void store_table(const KParams &p, int w, int64_t bet
     if (msg && lane < p.L) reinterpret_cast<float *>(msg + p.levels_off)[beta * p.L + lane] = value;
 }
 
+__device__ __forceinline__ void flag_nonfinite(const KParams &p, int lane)
+{
+    if (lane == 0) atomicOr(p.status, kStatusNonFinite);
+}
+
 // ---------------------------------------------------------------------------------------------
-// Per-scheme fits
+// Per-scheme fits (u: the values to quantize; v: the error-fed values the residual refers to)
 // ---------------------------------------------------------------------------------------------
-template <int EPL, bool FUSED>
-__device__ void fit_qsgd(const KParams &p, SmemQSGD &sm, int64_t beta, int w, int lane, bool full, uint32_t vmask,
+template <int EPL, bool FUSED, bool TAIL>
+__device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                          const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
 {
     float m = 0.0f;
 #pragma unroll
     for (int t = 0; t < EPL; ++t)
-        if ((vmask >> t) & 1u) m = fmaxf(m, fabsf(u[t]));
-    m = warp_max(m);
+        if (!TAIL || ((vmask >> t) & 1u)) m = fmax_nan(m, fabsf(u[t]));
+    m = warp_max_nan(m);
+    if (check && !(m <= FLT_MAX)) flag_nonfinite(p, lane);
     const int s = p.s;
+    const float lv = lane < s ? __fmul_rn(m, __fdiv_rn((float)(2 * lane - (s - 1)), (float)(s - 1))) : 0.0f;
+    const float lv_next = __shfl_down_sync(kFull, lv, 1);
     __syncwarp();
-    if (lane < s) sm.lev[lane] = __fmul_rn(m, __fdiv_rn((float)(2 * lane - (s - 1)), (float)(s - 1)));
+    if (lane < s - 1) sm.pair[lane] = make_float2(lv, lv_next);
     __syncwarp();
     RoundQSGD rule;
     rule.inv_m = m > 0.0f ? __fdiv_rn(1.0f, m) : 0.0f;
     rule.h = __fmul_rn((float)(s - 1), 0.5f);
-    rule.s = s;
-    rule.lev = sm.lev;
+    rule.kmax = s - 2;
+    rule.pair = sm.pair;
     int pos[EPL];
 #pragma unroll
     for (int t = 0; t < EPL; ++t) pos[t] = 0;
-    emit<EPL, FUSED, true>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
+    emit<EPL, FUSED, true, TAIL>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
     store_table(p, w, beta, lane, m);
 }
 
-template <int EPL, bool FUSED>
-__device__ void fit_orq(const KParams &p, SmemORQ &sm, int64_t beta, int w, int lane, bool full, uint32_t vmask,
+template <int EPL, bool FUSED, bool TAIL>
+__device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                         const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
 {
     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
     for (int t = 0; t < EPL; ++t)
-        if ((vmask >> t) & 1u) {
-            mn = fminf(mn, u[t]);
-            mx = fmaxf(mx, u[t]);
+        if (!TAIL || ((vmask >> t) & 1u)) {
+            mn = fmin_nan(mn, u[t]);
+            mx = fmax_nan(mx, u[t]);
         }
-    mn = __fadd_rn(warp_min(mn), 0.0f);
-    mx = __fadd_rn(warp_max(mx), 0.0f);
+    mn = warp_min_nan(mn);
+    mx = warp_max_nan(mx);
+    if (check && !(mn >= -FLT_MAX && mx <= FLT_MAX)) flag_nonfinite(p, lane);
+    mn = __fadd_rn(mn, 0.0f);
+    mx = __fadd_rn(mx, 0.0f);
     int pos[EPL];
-    if (!(mx > mn)) {
+    if (!(mx > mn)) {  // constant bucket (or NaN): one level, code 0
 #pragma unroll
         for (int t = 0; t < EPL; ++t) pos[t] = 0;
-        RoundConst rule{mn};
-        emit<EPL, FUSED, false>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
+        emit<EPL, FUSED, false, TAIL>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc);
         store_table(p, w, beta, lane, mn);
         return;
     }
     const float range = __fsub_rn(mx, mn);
     const float step = __fdiv_rn(range, 63.0f);
     const float scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kOrqFBits));
-    // lane-private histogram: no two lanes ever touch the same word
+    // histogram: 8 columns per cell, lane l adds into column l % 8 with shared atomics
+    const int col = lane & (kHistCols - 1);
 #pragma unroll
     for (int t = 0; t < EPL; ++t) {
-        pos[t] = grid_pos<kOrqFBits>(u[t], mn, scale);
-        if ((vmask >> t) & 1u) {
-            const int cell = min(pos[t] >> kOrqFBits, kTopCell);
-            sm.hist[cell * 32 + lane] += (1u << 27) + (uint32_t)(pos[t] - (cell << kOrqFBits));
+        // every valid value is finite and >= mn here, so the position is >= 0 without a clamp
+        int ps = min(__float2int_rz(__fmul_rn(__fsub_rn(u[t], mn), scale)), 63 << kOrqFBits);
+        if (TAIL) ps = max(ps, 0);
+        pos[t] = ps;
+        if (!TAIL || ((vmask >> t) & 1u)) {
+            const int cell = min(ps >> kOrqFBits, kTopCell);
+            atomicAdd(&sm.hcnt[cell * kHistCols + col], 1u);
+            atomicAdd(&sm.hsum[cell * kHistCols + col], (uint32_t)(ps - (cell << kOrqFBits)));
         }
     }
     __syncwarp();
-    // column sums for cells lane and lane+32 (skewed so that the 32 lanes hit 32 banks), then clear
-    uint32_t ca = 0, fa = 0, cb = 0, fb = 0;
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k) {
-        const int col = (lane + k) & 31;
-        const uint32_t xa = sm.hist[lane * 32 + col];
-        const uint32_t xb = sm.hist[(lane + 32) * 32 + col];
-        sm.hist[lane * 32 + col] = 0u;
-        sm.hist[(lane + 32) * 32 + col] = 0u;
-        ca += xa >> 27;
-        fa += xa & 0x7ffffffu;
-        cb += xb >> 27;
-        fb += xb & 0x7ffffffu;
+    // lane l reduces cells 2l and 2l+1 (16 consecutive words per array), clearing them; the
+    // four 16-byte reads are rotated by l/2 so that a quarter-warp touches 8 distinct bank groups
+    uint32_t c0 = 0, c1 = 0, f0 = 0, f1 = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int q4 = (k + (lane >> 1)) & 3;
+        uint4 *pc = reinterpret_cast<uint4 *>(sm.hcnt + lane * 16) + q4;
+        uint4 *pf = reinterpret_cast<uint4 *>(sm.hsum + lane * 16) + q4;
+        const uint4 xc = *pc, xf = *pf;
+        *pc = make_uint4(0u, 0u, 0u, 0u);
+        *pf = make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t sc = xc.x + xc.y + xc.z + xc.w;
+        const uint32_t sf = xf.x + xf.y + xf.z + xf.w;
+        if (q4 < 2) {
+            c0 += sc;
+            f0 += sf;
+        } else {
+            c1 += sc;
+            f1 += sf;
+        }
     }
-    const long long sa = (long long)ca * ((long long)lane << kOrqFBits) + (long long)fa;
-    const long long sb = (long long)cb * ((long long)(lane + 32) << kOrqFBits) + (long long)fb;
-    // exclusive prefix over cells 0..63
-    const int ica = warp_inclusive_scan((int)ca, lane);
-    const long long isa = warp_inclusive_scan(sa, lane);
-    const int icb = warp_inclusive_scan((int)cb, lane);
-    const long long isb = warp_inclusive_scan(sb, lane);
-    const int tca = __shfl_sync(kFull, ica, 31);
-    const long long tsa = __shfl_sync(kFull, isa, 31);
-    sm.P0[lane] = ica - (int)ca;
-    sm.P1[lane] = isa - sa;
-    sm.P0[lane + 32] = tca + icb - (int)cb;
-    sm.P1[lane + 32] = tsa + isb - sb;
+    // sums of positions of the two cells, exclusive prefix over the cell pairs
+    const long long s0 = (long long)c0 * ((long long)(2 * lane) << kOrqFBits) + f0;
+    const long long s1 = (long long)c1 * ((long long)(2 * lane + 1) << kOrqFBits) + f1;
+    const int ic = warp_inclusive_scan((int)(c0 + c1), lane);
+    const long long is = warp_inclusive_scan(s0 + s1, lane);
+    const int ec = ic - (int)(c0 + c1);
+    const long long es = is - (s0 + s1);
+    reinterpret_cast<int2 *>(sm.P0)[lane] = make_int2(ec, ec + (int)c0);
+    reinterpret_cast<longlong2 *>(sm.P1)[lane] = make_longlong2(es, es + s0);
     __syncwarp();
     const unsigned long long mask = orq_greedy(sm.P0, sm.P1, p.s, lane);
-    // levels, cell -> bracket table, brackets
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int j = lane + 32 * h;
-        const unsigned long long upto = (j == 63) ? ~0ull : ((2ull << j) - 1ull);
         if ((mask >> j) & 1ull) sm.lev[__popcll(mask & ((1ull << j) - 1ull))] = grid_point(mn, mx, step, j);
-        if (j <= kTopCell) sm.lut[j] = (unsigned char)(__popcll(mask & upto) - 1);
+        if (j <= kTopCell) sm.lut[j] = (unsigned char)(__popcll(mask & ((2ull << j) - 1ull)) - 1);
     }
     __syncwarp();
     if (lane < p.s - 1) {
         const float lo = sm.lev[lane], hi = sm.lev[lane + 1];
-        sm.tab[lane] = make_float4(lo, hi, __fdiv_rn(1.0f, __fsub_rn(hi, lo)), 0.0f);
+        sm.tab[lane] = make_float4(lo, hi, __fdiv_rn(1.0f, __fsub_rn(hi, lo)), __int_as_float(lane));
     }
     __syncwarp();
-    RoundORQ rule{sm.lut, sm.tab, sm.lev};
-    emit<EPL, FUSED, true>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
+    emit<EPL, FUSED, true, TAIL>(p, RoundORQ{sm.lut, sm.tab}, beta, w, lane, vmask, v, u, pos, acc);
     store_table(p, w, beta, lane, lane < p.s ? sm.lev[lane] : 0.0f);
     __syncwarp();
 }
@@ -275,15 +266,16 @@ __device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
     }
 }
 
-template <int EPL, bool FUSED>
-__device__ void fit_bingrad_b(const KParams &p, SmemB &, int64_t beta, int w, int lane, bool full, uint32_t vmask,
+template <int EPL, bool FUSED, bool TAIL>
+__device__ void fit_bingrad_b(const KParams &p, FitB &, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                               int nvalid, const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
 {
     float m = 0.0f;
 #pragma unroll
     for (int t = 0; t < EPL; ++t)
-        if ((vmask >> t) & 1u) m = fmaxf(m, fabsf(u[t]));
-    m = warp_max(m);
+        if (!TAIL || ((vmask >> t) & 1u)) m = fmax_nan(m, fabsf(u[t]));
+    m = warp_max_nan(m);
+    if (check && !(m <= FLT_MAX)) flag_nonfinite(p, lane);
     int pos[EPL];
 #pragma unroll
     for (int t = 0; t < EPL; ++t) pos[t] = 0;
@@ -291,7 +283,7 @@ __device__ void fit_bingrad_b(const KParams &p, SmemB &, int64_t beta, int w, in
     if (m > 0.0f) {
         float key[EPL];
 #pragma unroll
-        for (int t = 0; t < EPL; ++t) key[t] = ((vmask >> t) & 1u) ? u[t] : INFINITY;
+        for (int t = 0; t < EPL; ++t) key[t] = (!TAIL || ((vmask >> t) & 1u)) ? u[t] : INFINITY;
         warp_bitonic_sort<EPL>(key, lane);
         const int e = 46 - fexpo(m);
         const double sc = pow2d(e);
@@ -301,7 +293,7 @@ __device__ void fit_bingrad_b(const KParams &p, SmemB &, int64_t beta, int w, in
 #pragma unroll
         for (int r = 0; r < EPL; ++r) {
             const int i = lane * EPL + r;
-            run += (i < nvalid) ? fixed_point(key[r], sc) : 0ll;
+            run += (!TAIL || i < nvalid) ? fixed_point(key[r], sc) : 0ll;
             pre[r] = run;
         }
         const long long incl = warp_inclusive_scan(run, lane);
@@ -359,29 +351,31 @@ __device__ void fit_bingrad_b(const KParams &p, SmemB &, int64_t beta, int w, in
             rule = RoundB{a, b, tv, true};
         }
     }
-    emit<EPL, FUSED, false>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
+    emit<EPL, FUSED, false, TAIL>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
     store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
 }
 
-template <int EPL, bool FUSED>
-__device__ void fit_bingrad_pb(const KParams &p, SmemPB &sm, int64_t beta, int w, int lane, bool full, uint32_t vmask,
+template <int EPL, bool FUSED, bool TAIL>
+__device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                                const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
 {
     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
     for (int t = 0; t < EPL; ++t)
-        if ((vmask >> t) & 1u) {
-            mn = fminf(mn, u[t]);
-            mx = fmaxf(mx, u[t]);
+        if (!TAIL || ((vmask >> t) & 1u)) {
+            mn = fmin_nan(mn, u[t]);
+            mx = fmax_nan(mx, u[t]);
         }
-    mn = __fadd_rn(warp_min(mn), 0.0f);
-    mx = __fadd_rn(warp_max(mx), 0.0f);
+    mn = warp_min_nan(mn);
+    mx = warp_max_nan(mx);
+    if (check && !(mn >= -FLT_MAX && mx <= FLT_MAX)) flag_nonfinite(p, lane);
+    mn = __fadd_rn(mn, 0.0f);
+    mx = __fadd_rn(mx, 0.0f);
     int pos[EPL];
     if (!(mx > mn)) {
 #pragma unroll
         for (int t = 0; t < EPL; ++t) pos[t] = 0;
-        RoundConst rule{mn};
-        emit<EPL, FUSED, false>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
+        emit<EPL, FUSED, false, TAIL>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc);
         store_table(p, w, beta, lane, mn);
         return;
     }
@@ -391,7 +385,7 @@ __device__ void fit_bingrad_pb(const KParams &p, SmemPB &sm, int64_t beta, int w
 #pragma unroll
     for (int t = 0; t < EPL; ++t) {
         pos[t] = grid_pos<kPbFBits>(u[t], mn, scale);
-        if ((vmask >> t) & 1u) {
+        if (!TAIL || ((vmask >> t) & 1u)) {
             const int cell = min(pos[t] >> kPbFBits, kTopCell);
             const unsigned long long x = (unsigned long long)pos[t];
             atomicAdd(&sm.cnt[cell], 1u);
@@ -436,7 +430,7 @@ __device__ void fit_bingrad_pb(const KParams &p, SmemPB &sm, int64_t beta, int w
     }
     __syncwarp();
     // exhaustive search over A < B, ties to the smallest (A, B)
-    unsigned long long best_e = ~0ull;
+    long long best_e = 0x7fffffffffffffffll;
     int best_ab = 0x7fffffff;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -445,9 +439,9 @@ __device__ void fit_bingrad_pb(const KParams &p, SmemPB &sm, int64_t beta, int w
         const unsigned long long beB = sm.be[B], gaB = sm.ga[B];
         for (int A = 0; A < B; ++A) {
             const unsigned long long aa = (unsigned long long)A << kPbFBits;
-            const unsigned long long e = (unsigned long long)sm.al[A] + beB + aa * gaB + bb * (unsigned long long)sm.de[A];
+            const long long e = (long long)((unsigned long long)sm.al[A] + beB + aa * gaB + bb * (unsigned long long)sm.de[A]);
             const int ab = A * 64 + B;
-            if ((long long)e < (long long)best_e || ((long long)e == (long long)best_e && ab < best_ab) || best_ab == 0x7fffffff) {
+            if (e < best_e || (e == best_e && ab < best_ab)) {
                 best_e = e;
                 best_ab = ab;
             }
@@ -455,10 +449,9 @@ __device__ void fit_bingrad_pb(const KParams &p, SmemPB &sm, int64_t beta, int w
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long oe = __shfl_xor_sync(kFull, best_e, o);
+        const long long oe = __shfl_xor_sync(kFull, best_e, o);
         const int oab = __shfl_xor_sync(kFull, best_ab, o);
-        if (oab != 0x7fffffff &&
-            (best_ab == 0x7fffffff || (long long)oe < (long long)best_e || ((long long)oe == (long long)best_e && oab < best_ab))) {
+        if (oe < best_e || (oe == best_e && oab < best_ab)) {
             best_e = oe;
             best_ab = oab;
         }
@@ -470,106 +463,219 @@ __device__ void fit_bingrad_pb(const KParams &p, SmemPB &sm, int64_t beta, int w
     rule.rinv = __fdiv_rn(1.0f, __fsub_rn(rule.b, rule.a));
     rule.pa = A << kPbFBits;
     rule.pb = B << kPbFBits;
-    emit<EPL, FUSED, true>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
+    emit<EPL, FUSED, true, TAIL>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
     store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
+}
+
+// ---------------------------------------------------------------------------------------------
+// One item: clip, fit, round, write
+// ---------------------------------------------------------------------------------------------
+template <int EPL, int SCHEME, bool FUSED, bool TAIL>
+__device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME>::type &fit, int64_t beta, int w,
+                                        int lane, int nvalid, uint32_t vmask, const float (&v)[EPL], float (&acc)[EPL])
+{
+    float u[EPL];
+    bool check = true;  // the fit flags non-finite values unless the clip pass already did
+    if (p.clip > 0.0f) {
+        float am = 0.0f;
+#pragma unroll
+        for (int t = 0; t < EPL; ++t)
+            if (!TAIL || ((vmask >> t) & 1u)) am = fmax_nan(am, fabsf(v[t]));
+        am = warp_max_nan(am);
+        if (!(am <= FLT_MAX)) flag_nonfinite(p, lane);
+        check = false;
+        float T = 0.0f;
+        if (am > 0.0f) {
+            const int e = 20 - fexpo(am);
+            const double sc = pow2d(e);
+            long long sx = 0, sxx = 0;
+#pragma unroll
+            for (int t = 0; t < EPL; ++t)
+                if (!TAIL || ((vmask >> t) & 1u)) {
+                    const long long X = fixed_point(v[t], sc);
+                    sx += X;
+                    sxx += X * X;
+                }
+            sx = warp_sum(sx);
+            sxx = warp_sum(sxx);
+            T = clip_threshold_from_sums(sx, sxx, nvalid, e, p.clip);
+        }
+#pragma unroll
+        for (int t = 0; t < EPL; ++t) {
+            float x = v[t];
+            x = x < -T ? -T : x;
+            x = x > T ? T : x;
+            u[t] = x;
+        }
+    } else {
+#pragma unroll
+        for (int t = 0; t < EPL; ++t) u[t] = v[t];
+    }
+    if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD)
+        fit_qsgd<EPL, FUSED, TAIL>(p, fit, beta, w, lane, vmask, check, v, u, acc);
+    else if constexpr (SCHEME == GQ_ORQ)
+        fit_orq<EPL, FUSED, TAIL>(p, fit, beta, w, lane, vmask, check, v, u, acc);
+    else if constexpr (SCHEME == GQ_BINGRAD_B)
+        fit_bingrad_b<EPL, FUSED, TAIL>(p, fit, beta, w, lane, vmask, check, nvalid, v, u, acc);
+    else
+        fit_bingrad_pb<EPL, FUSED, TAIL>(p, fit, beta, w, lane, vmask, check, v, u, acc);
 }
 
 // ---------------------------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------------------------
+template <int EPL, int SCHEME>
+constexpr int min_blocks() { return (SCHEME == GQ_BINGRAD_B || SCHEME == GQ_BINGRAD_PB) ? 2 : 4; }
+
 template <int EPL, int SCHEME, bool FUSED>
-__global__ void __launch_bounds__(kWarpsPerCta * 32) k_warp(const __grid_constant__ KParams p)
+__global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME>()))
+    k_warp(const __grid_constant__ KParams p)
 {
-    using Sm = typename SmemFor<SCHEME>::type;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    using Smem = WarpSmem<EPL, SCHEME>;
+    constexpr int D = 32 * EPL;
+    constexpr unsigned kBytes = D * 4;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
-    Sm &sm = reinterpret_cast<Sm *>(smem_raw)[wib];
+    Smem &sm = reinterpret_cast<Smem *>(smem_raw)[wib];
+
     if constexpr (SCHEME == GQ_ORQ) {
-        for (int i = lane; i < 64 * 32; i += 32) sm.hist[i] = 0u;
+        for (int i = lane; i < 64 * kHistCols; i += 32) {
+            sm.fit.hcnt[i] = 0u;
+            sm.fit.hsum[i] = 0u;
+        }
     }
     if constexpr (SCHEME == GQ_BINGRAD_PB) {
         for (int i = lane; i < 64; i += 32) {
-            sm.cnt[i] = 0u;
-            sm.s1[i] = 0ull;
-            sm.s2[i] = 0ull;
+            sm.fit.cnt[i] = 0u;
+            sm.fit.s1[i] = 0ull;
+            sm.fit.s2[i] = 0ull;
         }
+    }
+    if (lane == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
+        fence_barrier_init();
     }
     __syncwarp();
 
-    constexpr int D = 32 * EPL;
     const int64_t first = (int64_t)blockIdx.x * kWarpsPerCta + wib;
     const int64_t stride = (int64_t)gridDim.x * kWarpsPerCta;
-    for (int64_t beta = first; beta < p.nb; beta += stride) {
-        const int nvalid = (beta == p.nb - 1) ? p.tail : D;
-        const bool full = nvalid == D;
-        uint32_t vmask = 0;
+    if (first >= p.nb) return;
+    const int W = p.W;
+    const int64_t nitems = ((p.nb - 1 - first) / stride + 1) * W;
+    const bool ef = p.r[0] != nullptr;
+    const unsigned tx = ef ? 2 * kBytes : kBytes;
+
+    // the producer side (lane 0): item (beta, w) into stage s
+    auto bulk = [&](int64_t beta) { return !(beta == p.nb - 1 && p.tail < D); };
+    auto issue = [&](int64_t beta, int w, int s) {
+        fence_proxy_async();
+        mbar_arrive_expect_tx(&sm.bar[s], tx);
+        bulk_load(sm.stage[s].g, p.g[w] + beta * D, kBytes, &sm.bar[s]);
+        if (ef) bulk_load(sm.stage[s].r, p.r[w] + beta * D, kBytes, &sm.bar[s]);
+    };
+    // consumer position (beta, w) and producer position two items ahead
+    int64_t beta = first;
+    int w = 0;
+    int64_t pbeta = first;
+    int pw = 0;
+    unsigned pending = 0, parity = 0;
 #pragma unroll
-        for (int t = 0; t < EPL; ++t) vmask |= (slot_elem(t, lane) < nvalid ? 1u : 0u) << t;
-        float acc[EPL];
-#pragma unroll
-        for (int t = 0; t < EPL; ++t) acc[t] = 0.0f;
-        for (int w = 0; w < p.W; ++w) {
-            float v[EPL];
-            load_bucket<EPL>(p.g[w], p.r[w], beta * D, nvalid, full, lane, v);
-            // non-finite input: flag it (NaN-propagating max of |v|)
-            float am = 0.0f;
-#pragma unroll
-            for (int t = 0; t < EPL; ++t)
-                if ((vmask >> t) & 1u) am = fmax_nan(am, fabsf(v[t]));
-            am = warp_max_nan(am);
-            if (!(am <= FLT_MAX) && lane == 0) atomicOr(p.status, kStatusNonFinite);
-            // clip to +-c*sigma
-            float u[EPL];
-            if (p.clip > 0.0f) {
-                float T = 0.0f;
-                if (am > 0.0f) {
-                    const int e = 20 - fexpo(am);
-                    const double sc = pow2d(e);
-                    long long sx = 0, sxx = 0;
-#pragma unroll
-                    for (int t = 0; t < EPL; ++t)
-                        if ((vmask >> t) & 1u) {
-                            const long long X = fixed_point(v[t], sc);
-                            sx += X;
-                            sxx += X * X;
-                        }
-                    sx = warp_sum(sx);
-                    sxx = warp_sum(sxx);
-                    T = clip_threshold_from_sums(sx, sxx, nvalid, e, p.clip);
-                }
-#pragma unroll
-                for (int t = 0; t < EPL; ++t) {
-                    float x = v[t];
-                    x = x < -T ? -T : x;
-                    x = x > T ? T : x;
-                    u[t] = x;
-                }
-            } else {
-#pragma unroll
-                for (int t = 0; t < EPL; ++t) u[t] = v[t];
-            }
-            if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD)
-                fit_qsgd<EPL, FUSED>(p, sm, beta, w, lane, full, vmask, v, u, acc);
-            else if constexpr (SCHEME == GQ_ORQ)
-                fit_orq<EPL, FUSED>(p, sm, beta, w, lane, full, vmask, v, u, acc);
-            else if constexpr (SCHEME == GQ_BINGRAD_B)
-                fit_bingrad_b<EPL, FUSED>(p, sm, beta, w, lane, full, vmask, nvalid, v, u, acc);
-            else
-                fit_bingrad_pb<EPL, FUSED>(p, sm, beta, w, lane, full, vmask, v, u, acc);
+    for (int k = 0; k < kStages; ++k) {
+        if ((int64_t)k < nitems && bulk(pbeta)) {
+            if (lane == 0) issue(pbeta, pw, k);
+            pending |= 1u << k;
         }
-        if constexpr (FUSED) {
-            float *ab = p.avg + beta * D;
-            if (full) {
+        if (++pw == W) {
+            pw = 0;
+            pbeta += stride;
+        }
+    }
+
+    float acc[EPL];
+    for (int64_t it = 0; it < nitems; ++it) {
+        const int s = (int)(it % kStages);
+        if (w == 0) {
 #pragma unroll
-                for (int m = 0; m < EPL / 4; ++m)
-                    __stcs(reinterpret_cast<float4 *>(ab + 128 * m + 4 * lane),
-                           make_float4(__fmul_rn(acc[4 * m], p.inv_w), __fmul_rn(acc[4 * m + 1], p.inv_w),
-                                       __fmul_rn(acc[4 * m + 2], p.inv_w), __fmul_rn(acc[4 * m + 3], p.inv_w)));
-            } else {
+            for (int t = 0; t < EPL; ++t) acc[t] = 0.0f;
+        }
+        float v[EPL];
+        if (bulk(beta)) {
+            if (!mbar_wait_warp(&sm.bar[s], (parity >> s) & 1u)) {
+                // the copy did not complete in time: report, let the other copy land, stop
+                if (lane == 0) atomicOr(p.status, kStatusTimeout);
+                const int o = s ^ 1;
+                if ((pending >> o) & 1u) mbar_wait_warp(&sm.bar[o], (parity >> o) & 1u);
+                return;
+            }
+            parity ^= 1u << s;
+            pending &= ~(1u << s);
+            const float *sg = sm.stage[s].g;
+            const float *sr = sm.stage[s].r;
+#pragma unroll
+            for (int m = 0; m < EPL / 4; ++m) {
+                float4 x = *reinterpret_cast<const float4 *>(sg + 128 * m + 4 * lane);
+                if (ef) {
+                    const float4 y = *reinterpret_cast<const float4 *>(sr + 128 * m + 4 * lane);
+                    x = make_float4(__fadd_rn(x.x, y.x), __fadd_rn(x.y, y.y), __fadd_rn(x.z, y.z), __fadd_rn(x.w, y.w));
+                }
+                v[4 * m + 0] = x.x;
+                v[4 * m + 1] = x.y;
+                v[4 * m + 2] = x.z;
+                v[4 * m + 3] = x.w;
+            }
+            __syncwarp();
+            // stage s is free again: fetch the item two ahead into it
+            if (it + kStages < nitems && bulk(pbeta)) {
+                if (lane == 0) issue(pbeta, pw, s);
+                pending |= 1u << s;
+            }
+            process<EPL, SCHEME, FUSED, false>(p, sm.fit, beta, w, lane, D, 0xffffffffu, v, acc);
+        } else {
+            // the ragged last bucket: guarded plain loads
+            const int nvalid = p.tail;
+            uint32_t vmask = 0;
+            const float *gb = p.g[w] + beta * D;
+            const float *rb = ef ? p.r[w] + beta * D : nullptr;
+#pragma unroll
+            for (int t = 0; t < EPL; ++t) {
+                const int e = slot_elem(t, lane);
+                float x = 0.0f;
+                if (e < nvalid) {
+                    vmask |= 1u << t;
+                    x = gb[e];
+                    if (rb) x = __fadd_rn(x, rb[e]);
+                }
+                v[t] = x;
+            }
+            if (it + kStages < nitems && bulk(pbeta)) {
+                if (lane == 0) issue(pbeta, pw, s);
+                pending |= 1u << s;
+            }
+            process<EPL, SCHEME, FUSED, true>(p, sm.fit, beta, w, lane, nvalid, vmask, v, acc);
+            if (FUSED && w == W - 1) {
+                float *ab = p.avg + beta * D;
 #pragma unroll
                 for (int t = 0; t < EPL; ++t)
                     if ((vmask >> t) & 1u) ab[slot_elem(t, lane)] = __fmul_rn(acc[t], p.inv_w);
+            }
+        }
+        if (FUSED && w == W - 1 && bulk(beta)) {
+            float *ab = p.avg + beta * D;
+#pragma unroll
+            for (int m = 0; m < EPL / 4; ++m)
+                __stcs(reinterpret_cast<float4 *>(ab + 128 * m + 4 * lane),
+                       make_float4(__fmul_rn(acc[4 * m], p.inv_w), __fmul_rn(acc[4 * m + 1], p.inv_w),
+                                   __fmul_rn(acc[4 * m + 2], p.inv_w), __fmul_rn(acc[4 * m + 3], p.inv_w)));
+        }
+        if (++w == W) {
+            w = 0;
+            beta += stride;
+        }
+        if (it + kStages < nitems) {
+            if (++pw == W) {
+                pw = 0;
+                pbeta += stride;
             }
         }
     }
@@ -578,15 +684,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) k_warp(const __grid_constan
 template <int EPL, int SCHEME, bool FUSED>
 cudaError_t launch_one(const KParams &p, cudaStream_t stream)
 {
-    using Sm = typename SmemFor<SCHEME>::type;
     auto kern = k_warp<EPL, SCHEME, FUSED>;
-    const size_t smem = sizeof(Sm) * kWarpsPerCta;
-    static bool configured = false;  // per instantiation; attribute setting is idempotent
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    const size_t smem = sizeof(WarpSmem<EPL, SCHEME>) * kWarpsPerCta;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -72,7 +72,9 @@ def _gen(seed: int, device) -> torch.Generator:
 def _laplace_(out: torch.Tensor, b, gen: torch.Generator) -> torch.Tensor:
     """Laplace(0, b) into ``out`` by inverse CDF; ``b`` a float or a broadcastable tensor."""
     u = torch.rand(out.shape, generator=gen, device=out.device, dtype=torch.float32) - 0.5
-    out.copy_(-torch.sign(u) * torch.log1p(-2.0 * u.abs()))
+    # |2u| < 1 strictly (torch.rand can return 0, i.e. u = -0.5, where the inverse CDF is infinite)
+    a = (2.0 * u.abs()).clamp_(max=1.0 - 2.0 ** -24)
+    out.copy_(-torch.sign(u) * torch.log1p(-a))
     out.mul_(b)
     return out
 
@@ -82,7 +84,7 @@ def _student_t3(n: int, gen: torch.Generator, device) -> torch.Tensor:
     chi2 = torch.zeros(n, device=device)
     for _ in range(3):
         chi2.add_(torch.randn(n, generator=gen, device=device).square_())
-    return z / torch.sqrt(chi2 / 3.0)
+    return z / torch.sqrt(chi2.clamp_(min=1e-30) / 3.0)
 
 
 def mix_seed(*parts: int) -> int:

@@ -25,6 +25,7 @@
  *     fail the call: it raises a flag on the plan that gq_plan_status reports; the outputs of
  *     the affected bucket are then unspecified (but every access stays in bounds).
  *   - The library never allocates inside a call except gq_plan_create.
+ *   - With n = 0 every call is a no-op that returns GQ_OK; data pointers may then be NULL.
  */
 #ifndef GQ_H
 #define GQ_H
