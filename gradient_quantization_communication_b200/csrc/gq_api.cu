@@ -100,6 +100,7 @@ gq::KParams base_params(const gq_plan &pl, uint64_t step)
         p.rk1[i] = p.key1 + (uint32_t)i * 0xBB67AE85u;
     }
     p.step_lo = (uint32_t)step;
+    p.step_m1 = 0xCD9E8D57ull * (unsigned long long)p.step_lo;
     p.worker0 = 0;
     p.inv_w = 1.0f;
     p.codes_words = (int64_t)pl.cfg.bucket * pl.bits / 32;

@@ -514,7 +514,8 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
             for (int c = 0; c < 4; ++c) {
                 u4[c] = clipped(v4[c]);
                 pos4[c] = 0;
-                if constexpr (SCHEME == GQ_ORQ) pos4[c] = constant ? 0 : grid_pos<kOrqFBits>(u4[c], mn, scale);
+                if constexpr (SCHEME == GQ_ORQ)
+                    pos4[c] = constant ? 0 : min(grid_pos<kOrqFBits>(u4[c], mn, scale) >> kOrqFBits, kTopCell);
                 if constexpr (SCHEME == GQ_BINGRAD_PB) pos4[c] = constant ? 0 : grid_pos<kPbFBits>(u4[c], mn, scale);
             }
             uint32_t valid = 0;

@@ -28,12 +28,14 @@ constexpr int kPbFBits = 16;          // fraction bits of BinGrad-pb fixed-point
 // multipliers, the high halves xor-ed with the other counter words and the round key; the key
 // advances by the two Weyl increments between rounds.  The ten round keys are computed once on
 // the host (KParams::rk0 / rk1), so a round costs two wide multiplies and two xors.
+// philox_rounds_2_to_10 runs the last nine rounds on the state left by round 1, which draws4
+// computes.
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+__device__ __forceinline__ uint4 philox_rounds_2_to_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
                                                const uint32_t *rk0, const uint32_t *rk1)
 {
 #pragma unroll
-    for (int round = 0; round < 10; ++round) {
+    for (int round = 0; round < 9; ++round) {
         const unsigned long long p0 = (unsigned long long)0xD2511F53u * c0;
         const unsigned long long p1 = (unsigned long long)0xCD9E8D57u * c2;
         const uint32_t y0 = (uint32_t)(p1 >> 32) ^ c1 ^ rk0[round];
@@ -48,9 +50,15 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
 
 // The four draws of the 4-element group starting at global element index 4*blk: the counter is
 // (blk low word, blk high word, step low word, worker), the key the two words of the seed.
+// Counter word 2 is the step for every group, so the first round's product of it (step_m1)
+// comes precomputed from the host.
 __device__ __forceinline__ uint4 draws4(const KParams &p, uint64_t blk, uint32_t worker)
 {
-    return philox4x32_10((uint32_t)blk, (uint32_t)(blk >> 32), p.step_lo, worker, p.rk0, p.rk1);
+    const uint32_t c0 = (uint32_t)blk, c1 = (uint32_t)(blk >> 32);
+    const unsigned long long p0 = (unsigned long long)0xD2511F53u * c0;
+    const uint32_t y0 = (uint32_t)(p.step_m1 >> 32) ^ c1 ^ p.rk0[0];
+    const uint32_t y2 = (uint32_t)(p0 >> 32) ^ worker ^ p.rk1[0];
+    return philox_rounds_2_to_10(y0, (uint32_t)p.step_m1, y2, (uint32_t)p0, p.rk0 + 1, p.rk1 + 1);
 }
 
 // Uniform in [0, 1) at 24-bit resolution from one Philox output word.
@@ -184,33 +192,74 @@ __device__ __forceinline__ float clip_threshold_from_sums(long long sx, long lon
 // (x in units of 2^-22 cell).  Each round takes the largest Delta, ties to the smallest C.
 // Returns the 64-bit mask of chosen grid indices.
 // ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ long long orq_delta(int A, int C, int B, int P0A, int P0C, int P0B, long long P1A,
+                                               long long P1C, long long P1B)
+{
+    const long long lows = (P1C - P1A) - (long long)(A << kOrqFBits) * (P0C - P0A);
+    const long long highs = (long long)(B << kOrqFBits) * (P0B - P0C) - (P1B - P1C);
+    return (long long)(B - C) * lows + (long long)(C - A) * highs;
+}
+
+// Incremental form: lane l owns candidates C = l and l + 32 with their current neighbours and
+// Delta in registers; after a level L is added only the candidates of the bracket it split
+// are re-evaluated (skipped warp-wide when no lane has one).
 __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const long long *P1, int s, int lane)
 {
     unsigned long long mask = 1ull | (1ull << 63);
-    // the lane's two candidates and their own prefix values do not change across rounds
-    const int P0c[2] = {P0[lane], P0[lane + 32]};
-    const long long P1c[2] = {P1[lane], P1[lane + 32]};
+    int A[2], B[2], P0A[2], P0B[2], P0C[2];
+    long long P1A[2], P1B[2], P1C[2], delta[2];
+    bool live[2];
+    const int P0lo = P0[0], P0hi = P0[63];
+    const long long P1lo = P1[0], P1hi = P1[63];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int C = lane + 32 * h;
+        live[h] = C >= 1 && C <= 62;
+        A[h] = 0;
+        B[h] = 63;
+        P0A[h] = P0lo;
+        P1A[h] = P1lo;
+        P0B[h] = P0hi;
+        P1B[h] = P1hi;
+        P0C[h] = P0[C];
+        P1C[h] = P1[C];
+        delta[h] = orq_delta(0, C, 63, P0lo, P0C[h], P0hi, P1lo, P1C[h], P1hi);
+    }
     for (int round = 0; round < s - 2; ++round) {
         unsigned long long best = 0;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int C = lane + 32 * h;
-            if (C >= 1 && C <= 62 && !((mask >> C) & 1ull)) {
-                const unsigned long long below = mask & ((1ull << C) - 1ull);
-                const unsigned long long above = mask & ~((2ull << C) - 1ull);
-                const int A = 63 - __clzll((long long)below);
-                const int B = __ffsll((long long)above) - 1;
-                const long long lows = (P1c[h] - P1[A]) - (long long)(A << kOrqFBits) * (P0c[h] - P0[A]);
-                const long long highs = (long long)(B << kOrqFBits) * (P0[B] - P0c[h]) - (P1[B] - P1c[h]);
-                const long long delta = (long long)(B - C) * lows + (long long)(C - A) * highs;
-                const unsigned long long key = ((unsigned long long)delta << 6) | (unsigned long long)(63 - C);
-                best = key > best ? key : best;
-            }
+            const unsigned long long key = ((unsigned long long)delta[h] << 6) | (unsigned long long)(63 - lane - 32 * h);
+            if (live[h]) best = key > best ? key : best;
         }
         // warp argmax of the 64-bit key: high words first, then low words among the lanes that tie
         const unsigned hi = __reduce_max_sync(kFull, (unsigned)(best >> 32));
         const unsigned lo = __reduce_max_sync(kFull, (unsigned)(best >> 32) == hi ? (unsigned)best : 0u);
-        mask |= 1ull << (63 - (int)(lo & 63u));
+        const int L = 63 - (int)(lo & 63u);
+        mask |= 1ull << L;
+        if (round + 1 == s - 2) break;
+        const int P0L = P0[L];
+        const long long P1L = P1[L];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int C = lane + 32 * h;
+            if (C == L) live[h] = false;
+            const bool split = live[h] && A[h] < L && L < B[h];
+            if (__any_sync(kFull, split)) {
+                if (split) {
+                    if (L < C) {
+                        A[h] = L;
+                        P0A[h] = P0L;
+                        P1A[h] = P1L;
+                    } else {
+                        B[h] = L;
+                        P0B[h] = P0L;
+                        P1B[h] = P1L;
+                    }
+                    delta[h] = orq_delta(A[h], C, B[h], P0A[h], P0C[h], P0B[h], P1A[h], P1C[h], P1B[h]);
+                }
+            }
+        }
     }
     return mask;
 }

@@ -25,6 +25,7 @@ struct KParams {
     uint32_t rk0[10];    // Philox round keys: key0 + i * 0x9E3779B9
     uint32_t rk1[10];    //                    key1 + i * 0xBB67AE85
     uint32_t step_lo;    // step, low word
+    unsigned long long step_m1;  // 0xCD9E8D57 * step_lo (Philox round-1 product of counter word 2)
     uint32_t worker0;    // Philox worker index of worker slot 0
     float inv_w;         // 1/W for the average
     int64_t codes_words; // words of packed codes per bucket (d*b/32)
@@ -41,6 +42,8 @@ constexpr unsigned kStatusNonFinite = 1u;
 constexpr unsigned kStatusTimeout = 2u;  // a bounded wait on a bulk copy gave up
 
 // Register-resident path (d = 128, 256, 512): one warp per bucket index.
+// The ragged last bucket (when n is not a multiple of d) goes to a one-warp launch of the same
+// code with guarded loads, so the main kernel carries no tail logic.
 cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream);
 // Shared-memory path (d = 1024 .. 32768): one CTA per bucket, one worker per launch.
 cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream);

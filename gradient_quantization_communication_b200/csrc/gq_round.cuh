@@ -28,14 +28,14 @@ struct RoundQSGD {
     }
 };
 
-// ORQ: bracket of the value's grid cell; tab[k] = {lower, upper, 1/(upper-lower), k as bits};
-// up with probability (u - lower) / (upper - lower).
+// ORQ: bracket of the value's grid cell (passed in place of the position);
+// tab[k] = {lower, upper, 1/(upper-lower), k as bits}; up with probability
+// (u - lower) / (upper - lower).
 struct RoundORQ {
     const unsigned char *lut;
     const float4 *tab;
-    __device__ __forceinline__ void round(float u, int pos, uint32_t word, int &code, float &q) const
+    __device__ __forceinline__ void round(float u, int cell, uint32_t word, int &code, float &q) const
     {
-        const int cell = min(pos >> kOrqFBits, kTopCell);
         const float4 b = tab[lut[cell]];
         const float pu = __fmul_rn(__fsub_rn(u, b.x), b.z);
         const bool up = unit_float(word) < pu;

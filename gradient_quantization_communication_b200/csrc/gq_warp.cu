@@ -2,9 +2,10 @@
 //
 // One warp owns one bucket index at a time and walks its items (bucket, worker) in order.  The
 // g and r of each item (2 x d floats) are staged into the warp's shared memory by bulk
-// asynchronous copies (TMA, 1-D, no multicast) two items ahead, completed on per-stage
-// mbarriers, so the copy engine keeps 8 KB per warp in flight while the warp computes and no
-// registers are spent on prefetching.  Lane l then holds EPL = d/32 values in registers, slot
+// asynchronous copies (TMA, 1-D, no multicast) completed on an mbarrier: as soon as an item's
+// values are in registers the copy of the next item is issued into the same buffer, so the
+// copy engine keeps 4 KB per warp in flight during the whole fit and no registers are spent on
+// prefetching.  Lane l then holds EPL = d/32 values in registers, slot
 // t being element 128*(t/4) + 4*l + t%4 of the bucket, so that the four values of a slot
 // group share one Philox call and every global store is a coalesced 16-byte access.  In the
 // fused step the W workers of a bucket are consecutive items: the dequantized values are
@@ -16,15 +17,20 @@
 //                     per cell, shared atomics), exact int64 prefix sums, s-2 greedy rounds
 //   BinGrad-b       : warp bitonic sort, exact int64 prefix sums, argmax of J(k)
 //   BinGrad-pb      : shared-memory moments of 16-bit positions, exact search of all pairs
-// The last (ragged) bucket is loaded with plain guarded loads instead of bulk copies.
+// The last bucket, when ragged, is handled by a one-warp launch of the same code with guarded
+// plain loads, so the main kernel carries no tail logic.
 #include "gq_round.cuh"
 
 namespace gq {
 namespace {
 
 constexpr int kWarpsPerCta = 4;
-constexpr int kStages = 2;
 constexpr int kHistCols = 8;
+// Items staged ahead per warp (bulk-copy buffers of 2 x d floats each).
+#ifndef GQ_WARP_STAGES
+#define GQ_WARP_STAGES 1
+#endif
+constexpr int kStages = GQ_WARP_STAGES;
 
 template <int EPL>
 struct alignas(16) StageBuf {
@@ -167,16 +173,17 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     const float range = __fsub_rn(mx, mn);
     const float step = __fdiv_rn(range, 63.0f);
     const float scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kOrqFBits));
-    // histogram: 8 columns per cell, lane l adds into column l % 8 with shared atomics
+    // histogram: 8 columns per cell, lane l adds into column l % 8 with shared atomics; the
+    // rounding pass needs only the cell of each value, so the cells are what is kept
     const int col = lane & (kHistCols - 1);
 #pragma unroll
     for (int t = 0; t < EPL; ++t) {
         // every valid value is finite and >= mn here, so the position is >= 0 without a clamp
         int ps = min(__float2int_rz(__fmul_rn(__fsub_rn(u[t], mn), scale)), 63 << kOrqFBits);
         if (TAIL) ps = max(ps, 0);
-        pos[t] = ps;
+        const int cell = min(ps >> kOrqFBits, kTopCell);
+        pos[t] = cell;
         if (!TAIL || ((vmask >> t) & 1u)) {
-            const int cell = min(ps >> kOrqFBits, kTopCell);
             atomicAdd(&sm.hcnt[cell * kHistCols + col], 1u);
             atomicAdd(&sm.hsum[cell * kHistCols + col], (uint32_t)(ps - (cell << kOrqFBits)));
         }
@@ -203,13 +210,14 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
             f1 += sf;
         }
     }
-    // sums of positions of the two cells, exclusive prefix over the cell pairs
+    // sums of positions of the two cells; one exclusive prefix over the cell pairs of the packed
+    // (sum << 16 | count): counts stay below 2^16 and sums below 2^37 for d <= 512
     const long long s0 = (long long)c0 * ((long long)(2 * lane) << kOrqFBits) + f0;
     const long long s1 = (long long)c1 * ((long long)(2 * lane + 1) << kOrqFBits) + f1;
-    const int ic = warp_inclusive_scan((int)(c0 + c1), lane);
-    const long long is = warp_inclusive_scan(s0 + s1, lane);
-    const int ec = ic - (int)(c0 + c1);
-    const long long es = is - (s0 + s1);
+    const unsigned long long own = ((unsigned long long)(s0 + s1) << 16) | (c0 + c1);
+    const unsigned long long ex = warp_inclusive_scan(own, lane) - own;
+    const int ec = (int)(ex & 0xffffu);
+    const long long es = (long long)(ex >> 16);
     reinterpret_cast<int2 *>(sm.P0)[lane] = make_int2(ec, ec + (int)c0);
     reinterpret_cast<longlong2 *>(sm.P1)[lane] = make_longlong2(es, es + s0);
     __syncwarp();
@@ -522,14 +530,49 @@ __device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME
 }
 
 // ---------------------------------------------------------------------------------------------
-// The kernel
+// The kernels
 // ---------------------------------------------------------------------------------------------
-template <int EPL, int SCHEME>
-constexpr int min_blocks() { return (SCHEME == GQ_BINGRAD_B || SCHEME == GQ_BINGRAD_PB) ? 2 : 4; }
+// Resident CTAs per SM the register allocation is sized for (4 x 4 warps: 128 registers; at
+// 5 x 4 warps the 96-register cap spills and measured slower).
+#ifndef GQ_WARP_MIN_BLOCKS
+#define GQ_WARP_MIN_BLOCKS 4
+#endif
+template <int EPL, int SCHEME, int WARPS>
+constexpr int min_blocks()
+{
+    return (SCHEME == GQ_BINGRAD_B || SCHEME == GQ_BINGRAD_PB) ? 2 : GQ_WARP_MIN_BLOCKS * 4 / WARPS;
+}
 
+template <int SCHEME, class Fit>
+__device__ __forceinline__ void init_fit(Fit &fit, int lane)
+{
+    if constexpr (SCHEME == GQ_ORQ) {
+        for (int i = lane; i < 64 * kHistCols; i += 32) {
+            fit.hcnt[i] = 0u;
+            fit.hsum[i] = 0u;
+        }
+    }
+    if constexpr (SCHEME == GQ_BINGRAD_PB) {
+        for (int i = lane; i < 64; i += 32) {
+            fit.cnt[i] = 0u;
+            fit.s1[i] = 0ull;
+            fit.s2[i] = 0ull;
+        }
+    }
+}
+
+__device__ __forceinline__ void store_avg4(float *ab, int m, int lane, const float *acc, float inv_w)
+{
+    __stcs(reinterpret_cast<float4 *>(ab + 128 * m + 4 * lane),
+           make_float4(__fmul_rn(acc[0], inv_w), __fmul_rn(acc[1], inv_w), __fmul_rn(acc[2], inv_w),
+                       __fmul_rn(acc[3], inv_w)));
+}
+
+// Full buckets 0 .. nfull-1: every warp walks its items (bucket, worker), bulk copies one item
+// ahead.
 template <int EPL, int SCHEME, bool FUSED>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME>()))
-    k_warp(const __grid_constant__ KParams p)
+__global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME, kWarpsPerCta>()))
+    k_warp(const __grid_constant__ KParams p, int64_t nfull)
 {
     using Smem = WarpSmem<EPL, SCHEME>;
     constexpr int D = 32 * EPL;
@@ -538,145 +581,139 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME>())
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
     Smem &sm = reinterpret_cast<Smem *>(smem_raw)[wib];
-
-    if constexpr (SCHEME == GQ_ORQ) {
-        for (int i = lane; i < 64 * kHistCols; i += 32) {
-            sm.fit.hcnt[i] = 0u;
-            sm.fit.hsum[i] = 0u;
-        }
-    }
-    if constexpr (SCHEME == GQ_BINGRAD_PB) {
-        for (int i = lane; i < 64; i += 32) {
-            sm.fit.cnt[i] = 0u;
-            sm.fit.s1[i] = 0ull;
-            sm.fit.s2[i] = 0ull;
-        }
-    }
+    init_fit<SCHEME>(sm.fit, lane);
     if (lane == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
+        for (int k = 0; k < kStages; ++k) mbar_init(&sm.bar[k], 1);
         fence_barrier_init();
     }
     __syncwarp();
 
     const int64_t first = (int64_t)blockIdx.x * kWarpsPerCta + wib;
     const int64_t stride = (int64_t)gridDim.x * kWarpsPerCta;
-    if (first >= p.nb) return;
+    if (first >= nfull) return;
     const int W = p.W;
-    const int64_t nitems = ((p.nb - 1 - first) / stride + 1) * W;
+    const int64_t nitems = ((nfull - 1 - first) / stride + 1) * W;
     const bool ef = p.r[0] != nullptr;
     const unsigned tx = ef ? 2 * kBytes : kBytes;
-
-    // the producer side (lane 0): item (beta, w) into stage s
-    auto bulk = [&](int64_t beta) { return !(beta == p.nb - 1 && p.tail < D); };
-    auto issue = [&](int64_t beta, int w, int s) {
+    auto issue = [&](int64_t beta, int w, int k) {  // lane 0
         fence_proxy_async();
-        mbar_arrive_expect_tx(&sm.bar[s], tx);
-        bulk_load(sm.stage[s].g, p.g[w] + beta * D, kBytes, &sm.bar[s]);
-        if (ef) bulk_load(sm.stage[s].r, p.r[w] + beta * D, kBytes, &sm.bar[s]);
+        mbar_arrive_expect_tx(&sm.bar[k], tx);
+        bulk_load(sm.stage[k].g, p.g[w] + beta * D, kBytes, &sm.bar[k]);
+        if (ef) bulk_load(sm.stage[k].r, p.r[w] + beta * D, kBytes, &sm.bar[k]);
     };
-    // consumer position (beta, w) and producer position two items ahead
-    int64_t beta = first;
-    int w = 0;
+    // producer position: kStages items ahead of the consumer
     int64_t pbeta = first;
     int pw = 0;
-    unsigned pending = 0, parity = 0;
-#pragma unroll
     for (int k = 0; k < kStages; ++k) {
-        if ((int64_t)k < nitems && bulk(pbeta)) {
-            if (lane == 0) issue(pbeta, pw, k);
-            pending |= 1u << k;
-        }
+        if (lane == 0 && (int64_t)k < nitems) issue(pbeta, pw, k);
         if (++pw == W) {
             pw = 0;
             pbeta += stride;
         }
     }
 
+    int64_t beta = first;
+    int w = 0;
+    unsigned parity = 0;  // bit k: phase parity awaited next on buffer k
     float acc[EPL];
     for (int64_t it = 0; it < nitems; ++it) {
-        const int s = (int)(it % kStages);
+        const int k = kStages == 1 ? 0 : (int)(it % kStages);
+        if (!mbar_wait_warp(&sm.bar[k], (parity >> k) & 1u)) {
+            // a copy did not complete in time: report it, give every copy still in flight one
+            // more bounded wait so that none can land after the warp has left, and stop
+            if (lane == 0) atomicOr(p.status, kStatusTimeout);
+            for (int j = 0; j < kStages; ++j)
+                if ((int64_t)j + it < nitems) mbar_wait_warp(&sm.bar[(k + j) % kStages], (parity >> ((k + j) % kStages)) & 1u);
+            return;
+        }
+        parity ^= 1u << k;
+        float v[EPL];
+#pragma unroll
+        for (int m = 0; m < EPL / 4; ++m) {
+            float4 x = *reinterpret_cast<const float4 *>(sm.stage[k].g + 128 * m + 4 * lane);
+            if (ef) {
+                const float4 y = *reinterpret_cast<const float4 *>(sm.stage[k].r + 128 * m + 4 * lane);
+                x = make_float4(__fadd_rn(x.x, y.x), __fadd_rn(x.y, y.y), __fadd_rn(x.z, y.z), __fadd_rn(x.w, y.w));
+            }
+            v[4 * m + 0] = x.x;
+            v[4 * m + 1] = x.y;
+            v[4 * m + 2] = x.z;
+            v[4 * m + 3] = x.w;
+        }
+        __syncwarp();
+        // the buffer is free again: fetch the item kStages ahead while this one is processed
+        if (lane == 0 && it + kStages < nitems) issue(pbeta, pw, k);
+        if (++pw == W) {
+            pw = 0;
+            pbeta += stride;
+        }
+        const bool last_w = w == W - 1;
         if (w == 0) {
 #pragma unroll
             for (int t = 0; t < EPL; ++t) acc[t] = 0.0f;
         }
-        float v[EPL];
-        if (bulk(beta)) {
-            if (!mbar_wait_warp(&sm.bar[s], (parity >> s) & 1u)) {
-                // the copy did not complete in time: report, let the other copy land, stop
-                if (lane == 0) atomicOr(p.status, kStatusTimeout);
-                const int o = s ^ 1;
-                if ((pending >> o) & 1u) mbar_wait_warp(&sm.bar[o], (parity >> o) & 1u);
-                return;
-            }
-            parity ^= 1u << s;
-            pending &= ~(1u << s);
-            const float *sg = sm.stage[s].g;
-            const float *sr = sm.stage[s].r;
+        process<EPL, SCHEME, FUSED, false>(p, sm.fit, beta, w, lane, D, 0xffffffffu, v, acc);
+        if (FUSED && last_w) {
 #pragma unroll
-            for (int m = 0; m < EPL / 4; ++m) {
-                float4 x = *reinterpret_cast<const float4 *>(sg + 128 * m + 4 * lane);
-                if (ef) {
-                    const float4 y = *reinterpret_cast<const float4 *>(sr + 128 * m + 4 * lane);
-                    x = make_float4(__fadd_rn(x.x, y.x), __fadd_rn(x.y, y.y), __fadd_rn(x.z, y.z), __fadd_rn(x.w, y.w));
-                }
-                v[4 * m + 0] = x.x;
-                v[4 * m + 1] = x.y;
-                v[4 * m + 2] = x.z;
-                v[4 * m + 3] = x.w;
-            }
-            __syncwarp();
-            // stage s is free again: fetch the item two ahead into it
-            if (it + kStages < nitems && bulk(pbeta)) {
-                if (lane == 0) issue(pbeta, pw, s);
-                pending |= 1u << s;
-            }
-            process<EPL, SCHEME, FUSED, false>(p, sm.fit, beta, w, lane, D, 0xffffffffu, v, acc);
-        } else {
-            // the ragged last bucket: guarded plain loads
-            const int nvalid = p.tail;
-            uint32_t vmask = 0;
-            const float *gb = p.g[w] + beta * D;
-            const float *rb = ef ? p.r[w] + beta * D : nullptr;
-#pragma unroll
-            for (int t = 0; t < EPL; ++t) {
-                const int e = slot_elem(t, lane);
-                float x = 0.0f;
-                if (e < nvalid) {
-                    vmask |= 1u << t;
-                    x = gb[e];
-                    if (rb) x = __fadd_rn(x, rb[e]);
-                }
-                v[t] = x;
-            }
-            if (it + kStages < nitems && bulk(pbeta)) {
-                if (lane == 0) issue(pbeta, pw, s);
-                pending |= 1u << s;
-            }
-            process<EPL, SCHEME, FUSED, true>(p, sm.fit, beta, w, lane, nvalid, vmask, v, acc);
-            if (FUSED && w == W - 1) {
-                float *ab = p.avg + beta * D;
-#pragma unroll
-                for (int t = 0; t < EPL; ++t)
-                    if ((vmask >> t) & 1u) ab[slot_elem(t, lane)] = __fmul_rn(acc[t], p.inv_w);
-            }
+            for (int m = 0; m < EPL / 4; ++m) store_avg4(p.avg + beta * D, m, lane, acc + 4 * m, p.inv_w);
         }
-        if (FUSED && w == W - 1 && bulk(beta)) {
-            float *ab = p.avg + beta * D;
-#pragma unroll
-            for (int m = 0; m < EPL / 4; ++m)
-                __stcs(reinterpret_cast<float4 *>(ab + 128 * m + 4 * lane),
-                       make_float4(__fmul_rn(acc[4 * m], p.inv_w), __fmul_rn(acc[4 * m + 1], p.inv_w),
-                                   __fmul_rn(acc[4 * m + 2], p.inv_w), __fmul_rn(acc[4 * m + 3], p.inv_w)));
-        }
-        if (++w == W) {
+        if (last_w) {
             w = 0;
             beta += stride;
+        } else {
+            ++w;
         }
-        if (it + kStages < nitems) {
-            if (++pw == W) {
-                pw = 0;
-                pbeta += stride;
+    }
+}
+
+// The ragged last bucket (n not a multiple of d): guarded plain loads, one warp per worker
+// (warp k takes workers k, k + nwarps, ...).  Each warp's dequantized values are parked in
+// shared memory (qbuf[w][e]) and summed afterwards in worker order, which gives the same bits
+// as the register sum of the main kernel: every partial sum starts from +0.
+template <int EPL, int SCHEME, bool FUSED>
+__global__ void __launch_bounds__(512) k_warp_tail(const __grid_constant__ KParams p)
+{
+    using Fit = typename FitFor<SCHEME>::type;
+    constexpr int D = 32 * EPL;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    Fit &fit = reinterpret_cast<Fit *>(smem_raw)[wid];
+    float *qbuf = reinterpret_cast<float *>(smem_raw + sizeof(Fit) * nwarps);  // [W][D]
+    init_fit<SCHEME>(fit, lane);
+    __syncwarp();
+    const int64_t beta = p.nb - 1;
+    const int nvalid = p.tail;
+    uint32_t vmask = 0;
+#pragma unroll
+    for (int t = 0; t < EPL; ++t) vmask |= (slot_elem(t, lane) < nvalid ? 1u : 0u) << t;
+    for (int w = wid; w < p.W; w += nwarps) {
+        const float *gb = p.g[w] + beta * D;
+        const float *rb = p.r[w] ? p.r[w] + beta * D : nullptr;
+        float v[EPL], acc[EPL];
+#pragma unroll
+        for (int t = 0; t < EPL; ++t) {
+            const int e = slot_elem(t, lane);
+            float x = 0.0f;
+            if (e < nvalid) {
+                x = gb[e];
+                if (rb) x = __fadd_rn(x, rb[e]);
             }
+            v[t] = x;
+            acc[t] = 0.0f;
+        }
+        process<EPL, SCHEME, FUSED, true>(p, fit, beta, w, lane, nvalid, vmask, v, acc);
+        if (FUSED) {
+#pragma unroll
+            for (int t = 0; t < EPL; ++t) qbuf[w * D + slot_elem(t, lane)] = acc[t];
+        }
+    }
+    if (FUSED) {
+        __syncthreads();
+        float *ab = p.avg + beta * D;
+        for (int e = threadIdx.x; e < nvalid; e += blockDim.x) {
+            float sum = 0.0f;
+            for (int w = 0; w < p.W; ++w) sum = __fadd_rn(sum, qbuf[w * D + e]);
+            ab[e] = __fmul_rn(sum, p.inv_w);
         }
     }
 }
@@ -684,21 +721,36 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME>())
 template <int EPL, int SCHEME, bool FUSED>
 cudaError_t launch_one(const KParams &p, cudaStream_t stream)
 {
-    auto kern = k_warp<EPL, SCHEME, FUSED>;
-    const size_t smem = sizeof(WarpSmem<EPL, SCHEME>) * kWarpsPerCta;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarpsPerCta * 32, smem);
-    if (per_sm < 1) per_sm = 1;
-    const int64_t need = (p.nb + kWarpsPerCta - 1) / kWarpsPerCta;
-    const int64_t cap = (int64_t)sms * per_sm;
-    const int grid = (int)(need < cap ? need : cap);
-    if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kWarpsPerCta * 32, smem, stream>>>(p);
-    return cudaGetLastError();
+    constexpr int D = 32 * EPL;
+    const int64_t nfull = p.tail == D ? p.nb : p.nb - 1;
+    if (nfull > 0) {
+        auto kern = k_warp<EPL, SCHEME, FUSED>;
+        const size_t smem = sizeof(WarpSmem<EPL, SCHEME>) * kWarpsPerCta;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        int dev = 0, sms = 0, per_sm = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarpsPerCta * 32, smem);
+        if (per_sm < 1) per_sm = 1;
+        const int64_t need = (nfull + kWarpsPerCta - 1) / kWarpsPerCta;
+        const int64_t cap = (int64_t)sms * per_sm;
+        const int grid = (int)(need < cap ? need : cap);
+        kern<<<grid, kWarpsPerCta * 32, smem, stream>>>(p, nfull);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (nfull < p.nb) {
+        using Fit = typename FitFor<SCHEME>::type;
+        auto tail = k_warp_tail<EPL, SCHEME, FUSED>;
+        const int nwarps = p.W < 16 ? p.W : 16;
+        const size_t smem = sizeof(Fit) * nwarps + (FUSED ? (size_t)p.W * D * 4 : 0);
+        cudaError_t e = cudaFuncSetAttribute(tail, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        tail<<<1, 32 * nwarps, smem, stream>>>(p);
+        return cudaGetLastError();
+    }
+    return cudaSuccess;
 }
 
 template <int EPL, bool FUSED>
