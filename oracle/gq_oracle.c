@@ -31,7 +31,7 @@
 
 #define OR_GRIDPTS 64      /* candidate grid points j = 0..63 */
 #define OR_TOPCELL 62      /* cells 0..62 lie between grid points */
-#define OR_ORQ_FBITS 22    /* fraction bits of ORQ fixed-point positions */
+#define OR_ORQ_FBITS 16    /* fraction bits of ORQ fixed-point positions */
 #define OR_PB_FBITS 16     /* fraction bits of BinGrad-pb fixed-point positions */
 
 /* ------------------------------------------------------------------------------------------ */
@@ -190,7 +190,7 @@ int or_grid(const float *u, int n, float grid[64])
 /* are chosen greedily to minimise the expected quantization variance.  Reading: the levels    */
 /* start as {min, max} (grid indices 0 and 63); each of s-2 rounds adds the grid index whose   */
 /* addition gives the smallest total variance sum (b - x)(x - a) over the bucket, ties to the  */
-/* smallest index; x in fixed point with 22 fraction bits per cell, the bracket [a, b] of a    */
+/* smallest index; x in fixed point with 16 fraction bits per cell, the bracket [a, b] of a    */
 /* value being the chosen levels around its cell.                                              */
 /* ------------------------------------------------------------------------------------------ */
 
