@@ -103,6 +103,8 @@ gq::KParams base_params(const gq_plan &pl, uint64_t step)
     p.step_m1 = 0xCD9E8D57ull * (unsigned long long)p.step_lo;
     p.worker0 = 0;
     p.inv_w = 1.0f;
+    for (int k = 0; k < pl.cfg.levels; ++k)
+        p.qratio[k] = (float)(2 * k - (pl.cfg.levels - 1)) / (float)(pl.cfg.levels - 1);
     p.codes_words = (int64_t)pl.cfg.bucket * pl.bits / 32;
     p.levels_off = (int64_t)pl.levels_off;
     p.status = pl.status;

@@ -31,10 +31,10 @@ struct alignas(16) CtaShared {
     long long P1[64];
     int P0[64];
     long long al[64], be[64], ga[64], de[64];
-    float4 tab[16];
+    float4 ctab[64];
     float2 pair[16];
     float lev[16];
-    unsigned char lut[64];
+    float rinv[16];
     float bcast_f[4];
     long long bcast_l[2];
 };
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
 
         // ---- fit ------------------------------------------------------------------------------
         RoundQSGD rq;
-        RoundORQ ro{sh.lut, sh.tab};
+        RoundORQ ro{sh.ctab};
         RoundB rb{0.0f, 0.0f, 0.0f, false};
         RoundPB rp;
         bool constant = false;
@@ -214,13 +214,13 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
             m = block_max(m, sh, 0);
             const int s = p.s;
             if (wid == 0) {
-                const float lv = lane < s ? __fmul_rn(m, __fdiv_rn((float)(2 * lane - (s - 1)), (float)(s - 1))) : 0.0f;
+                const float lv = lane < s ? __fmul_rn(m, p.qratio[lane]) : 0.0f;
                 const float lv_next = __shfl_down_sync(kFull, lv, 1);
                 if (lane < s - 1) sh.pair[lane] = make_float2(lv, lv_next);
             }
             if (tid == 0) sh.bcast_f[0] = m;
             __syncthreads();
-            rq.inv_m = m > 0.0f ? __fdiv_rn(1.0f, m) : 0.0f;
+            rq.inv_m = m > 0.0f ? __frcp_rn(m) : 0.0f;
             rq.h = __fmul_rn((float)(s - 1), 0.5f);
             rq.kmax = s - 2;
             rq.pair = sh.pair;
@@ -280,12 +280,17 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                         for (int h = 0; h < 2; ++h) {
                             const int j = lane + 32 * h;
                             if ((mask >> j) & 1ull) sh.lev[__popcll(mask & ((1ull << j) - 1ull))] = grid_point(mn, mx, step, j);
-                            if (j <= kTopCell) sh.lut[j] = (unsigned char)(__popcll(mask & ((2ull << j) - 1ull)) - 1);
                         }
                         __syncwarp();
-                        if (lane < p.s - 1) {
-                            const float l0 = sh.lev[lane], l1 = sh.lev[lane + 1];
-                            sh.tab[lane] = make_float4(l0, l1, __fdiv_rn(1.0f, __fsub_rn(l1, l0)), __int_as_float(lane));
+                        if (lane < p.s - 1) sh.rinv[lane] = __frcp_rn(__fsub_rn(sh.lev[lane + 1], sh.lev[lane]));
+                        __syncwarp();
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int j = lane + 32 * h;
+                            if (j <= kTopCell) {
+                                const int k = __popcll(mask & ((2ull << j) - 1ull)) - 1;
+                                sh.ctab[j] = make_float4(sh.lev[k], sh.lev[k + 1], sh.rinv[k], __int_as_float(k));
+                            }
                         }
                     }
                     __syncthreads();
@@ -378,7 +383,7 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                     const int A = best_ab >> 6, Bs = best_ab & 63;
                     rp.a = grid_point(mn, mx, step, A);
                     rp.b = grid_point(mn, mx, step, Bs);
-                    rp.rinv = __fdiv_rn(1.0f, __fsub_rn(rp.b, rp.a));
+                    rp.rinv = __frcp_rn(__fsub_rn(rp.b, rp.a));
                     rp.pa = A << kPbFBits;
                     rp.pb = Bs << kPbFBits;
                 }
@@ -526,19 +531,19 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
             uint32_t *cwc = cw ? cw + ch * 4 * p.bits : nullptr;
             float q[4];
             if constexpr (SCHEME == GQ_QSGD) {
-                round_chunk<true, false>(p, rq, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                round_chunk<true, false, 0>(p, rq, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             } else if constexpr (SCHEME == GQ_ORQ) {
                 if (constant)
-                    round_chunk<false, false>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    round_chunk<false, false, 0>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
                 else
-                    round_chunk<true, false>(p, ro, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    round_chunk<true, false, 0>(p, ro, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             } else if constexpr (SCHEME == GQ_BINGRAD_PB) {
                 if (constant)
-                    round_chunk<false, false>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    round_chunk<false, false, 0>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
                 else
-                    round_chunk<true, false>(p, rp, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    round_chunk<true, false, 0>(p, rp, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             } else {
-                round_chunk<false, false>(p, rb, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                round_chunk<false, false, 0>(p, rb, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             }
         }
         // ---- level table --------------------------------------------------------------------------

@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
                 float lv = 0.0f;
                 if (QSGD) {
                     const float mscale = __ldg(tables + bk);
-                    if (lane < p.s) lv = __fmul_rn(mscale, __fdiv_rn((float)(2 * lane - (p.s - 1)), (float)(p.s - 1)));
+                    if (lane < p.s) lv = __fmul_rn(mscale, p.qratio[lane]);
                 } else if (lane < p.L) {
                     lv = __ldg(tables + bk * p.L + lane);
                 }

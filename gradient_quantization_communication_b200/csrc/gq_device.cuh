@@ -19,7 +19,7 @@ namespace gq {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kGridPts = 64;          // candidate grid points j = 0..63 (both ends included)
 constexpr int kTopCell = 62;          // cells 0..62 lie between grid points
-constexpr int kOrqFBits = 22;         // fraction bits of ORQ fixed-point grid positions
+constexpr int kOrqFBits = 16;         // fraction bits of ORQ fixed-point grid positions
 constexpr int kPbFBits = 16;          // fraction bits of BinGrad-pb fixed-point grid positions
 
 // ---------------------------------------------------------------------------------------------
@@ -142,6 +142,21 @@ __device__ __forceinline__ float warp_min_nan(float x)
     for (int o = 16; o > 0; o >>= 1) x = fmin_nan(x, __shfl_xor_sync(kFull, x, o));
     return x;
 }
+// Order-preserving map of binary32 onto int32 (NaN of either sign lands beyond +-inf, so a
+// NaN anywhere surfaces in the max or the min): lets a single REDUX find a float min / max.
+__device__ __forceinline__ int float_key(float f)
+{
+    const int b = __float_as_int(f);
+    return b ^ ((b >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ float key_float(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7fffffff)); }
+__device__ __forceinline__ float warp_redux_min(float x) { return key_float(__reduce_min_sync(kFull, float_key(x))); }
+__device__ __forceinline__ float warp_redux_max(float x) { return key_float(__reduce_max_sync(kFull, float_key(x))); }
+// max of non-negative values (or NaN): their bit patterns order like unsigned integers.
+__device__ __forceinline__ float warp_redux_max_abs(float x)
+{
+    return __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(x)));
+}
 __device__ __forceinline__ long long warp_sum(long long x)
 {
 #pragma unroll
@@ -187,30 +202,42 @@ __device__ __forceinline__ float clip_threshold_from_sums(long long sx, long lon
 // ORQ greedy over the prefix sums of the fixed-point histogram.
 // P0[k] / P1[k]: count / sum of positions of the elements in cells < k (k = 0..63).
 // Adding grid index C between the chosen neighbours A < C < B lowers the bucket's variance
-// sum (b-x)(x-a) by 2^22 * Delta(C) with
+// sum (b-x)(x-a) by 2^16 * Delta(C) with
 //   Delta(C) = (B-C) * sum_{A<=cell<C} (x - A) + (C-A) * sum_{C<=cell<B} (B - x)
-// (x in units of 2^-22 cell).  Each round takes the largest Delta, ties to the smallest C.
+// (x in units of 2^-16 cell).  Each round takes the largest Delta, ties to the smallest C.
 // Returns the 64-bit mask of chosen grid indices.
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ long long orq_delta(int A, int C, int B, int P0A, int P0C, int P0B, long long P1A,
-                                               long long P1C, long long P1B)
+// Buckets of up to 512 values: every prefix sum is below 512 * 63 * 2^16 < 2^31, so both
+// partial sums are exact in 32 bits and Delta takes two wide multiply-adds.
+__device__ __forceinline__ unsigned long long orq_delta(int A, int C, int B, int P0A, int P0C, int P0B, uint32_t P1A,
+                                                        uint32_t P1C, uint32_t P1B)
+{
+    const uint32_t lows = (P1C - P1A) - (uint32_t)(A << kOrqFBits) * (uint32_t)(P0C - P0A);
+    const uint32_t highs = (uint32_t)(B << kOrqFBits) * (uint32_t)(P0B - P0C) - (P1B - P1C);
+    return (unsigned long long)(uint32_t)(B - C) * lows + (unsigned long long)(uint32_t)(C - A) * highs;
+}
+// Larger buckets: 64-bit prefix sums.
+__device__ __forceinline__ unsigned long long orq_delta(int A, int C, int B, int P0A, int P0C, int P0B, long long P1A,
+                                                        long long P1C, long long P1B)
 {
     const long long lows = (P1C - P1A) - (long long)(A << kOrqFBits) * (P0C - P0A);
     const long long highs = (long long)(B << kOrqFBits) * (P0B - P0C) - (P1B - P1C);
-    return (long long)(B - C) * lows + (long long)(C - A) * highs;
+    return (unsigned long long)((long long)(B - C) * lows + (long long)(C - A) * highs);
 }
 
 // Incremental form: lane l owns candidates C = l and l + 32 with their current neighbours and
 // Delta in registers; after a level L is added only the candidates of the bracket it split
 // are re-evaluated (skipped warp-wide when no lane has one).
-__device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const long long *P1, int s, int lane)
+template <class T>
+__device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T *P1, int s, int lane)
 {
     unsigned long long mask = 1ull | (1ull << 63);
     int A[2], B[2], P0A[2], P0B[2], P0C[2];
-    long long P1A[2], P1B[2], P1C[2], delta[2];
+    T P1A[2], P1B[2], P1C[2];
+    unsigned long long delta[2];
     bool live[2];
     const int P0lo = P0[0], P0hi = P0[63];
-    const long long P1lo = P1[0], P1hi = P1[63];
+    const T P1lo = P1[0], P1hi = P1[63];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int C = lane + 32 * h;
@@ -229,7 +256,7 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const lo
         unsigned long long best = 0;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const unsigned long long key = ((unsigned long long)delta[h] << 6) | (unsigned long long)(63 - lane - 32 * h);
+            const unsigned long long key = (delta[h] << 6) | (unsigned long long)(63 - lane - 32 * h);
             if (live[h]) best = key > best ? key : best;
         }
         // warp argmax of the 64-bit key: high words first, then low words among the lanes that tie
@@ -239,7 +266,7 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const lo
         mask |= 1ull << L;
         if (round + 1 == s - 2) break;
         const int P0L = P0[L];
-        const long long P1L = P1[L];
+        const T P1L = P1[L];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int C = lane + 32 * h;

@@ -28,15 +28,14 @@ struct RoundQSGD {
     }
 };
 
-// ORQ: bracket of the value's grid cell (passed in place of the position);
-// tab[k] = {lower, upper, 1/(upper-lower), k as bits}; up with probability
-// (u - lower) / (upper - lower).
+// ORQ: the bracket of the value's grid cell (the cell is passed in place of the position),
+// one entry per cell: ctab[cell] = {lower, upper, 1/(upper-lower), bracket index as bits};
+// up with probability (u - lower) / (upper - lower).
 struct RoundORQ {
-    const unsigned char *lut;
-    const float4 *tab;
+    const float4 *ctab;
     __device__ __forceinline__ void round(float u, int cell, uint32_t word, int &code, float &q) const
     {
-        const float4 b = tab[lut[cell]];
+        const float4 b = ctab[cell];
         const float pu = __fmul_rn(__fsub_rn(u, b.x), b.z);
         const bool up = unit_float(word) < pu;
         code = __float_as_int(b.w) + (up ? 1 : 0);
@@ -88,7 +87,8 @@ struct RoundPB {
 //   rout  residual of the chunk's first element (NULL: no residual), 16-byte aligned
 //   cw    packed words of the chunk (b uint4: plane j = words 4j..4j+3), NULL: no message
 // Returns the dequantized values in q.
-template <bool RANDOM, bool ALLVALID, class R>
+// BITS: bits per code when known at compile time, 0 to read it from p.bits.
+template <bool RANDOM, bool ALLVALID, int BITS, class R>
 __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uint64_t blk, uint32_t worker, int lane,
                                             uint32_t valid, const float (&v)[4], const float (&u)[4],
                                             const int (&pos)[4], float *rout, uint32_t *cw, float (&q)[4])
@@ -115,8 +115,8 @@ __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uin
     if (cw) {
         // bit j of the code of element 4l + c -> bit l of word 4j + c of the chunk
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            if (j < p.bits) {
+        for (int j = 0; j < (BITS ? BITS : 4); ++j) {
+            if (BITS || j < p.bits) {
                 const uint32_t w0 = __ballot_sync(kFull, (code[0] >> j) & 1);
                 const uint32_t w1 = __ballot_sync(kFull, (code[1] >> j) & 1);
                 const uint32_t w2 = __ballot_sync(kFull, (code[2] >> j) & 1);

@@ -1,785 +1,21 @@
-// gq_warp.cu -- register-resident quantization kernels for buckets of d = 128, 256, 512.
-//
-// One warp owns one bucket index at a time and walks its items (bucket, worker) in order.  The
-// g and r of each item (2 x d floats) are staged into the warp's shared memory by bulk
-// asynchronous copies (TMA, 1-D, no multicast) completed on an mbarrier: as soon as an item's
-// values are in registers the copy of the next item is issued into the same buffer, so the
-// copy engine keeps 4 KB per warp in flight during the whole fit and no registers are spent on
-// prefetching.  Lane l then holds EPL = d/32 values in registers, slot
-// t being element 128*(t/4) + 4*l + t%4 of the bucket, so that the four values of a slot
-// group share one Philox call and every global store is a coalesced 16-byte access.  In the
-// fused step the W workers of a bucket are consecutive items: the dequantized values are
-// summed in registers in worker order and the average leaves the chip once.
-//
-// Level fits per bucket:
-//   QSGD / TernGrad : m = max|u|, s uniform levels on [-m, m]
-//   ORQ             : shared-memory histogram of 22-bit fixed-point grid positions (8 columns
-//                     per cell, shared atomics), exact int64 prefix sums, s-2 greedy rounds
-//   BinGrad-b       : warp bitonic sort, exact int64 prefix sums, argmax of J(k)
-//   BinGrad-pb      : shared-memory moments of 16-bit positions, exact search of all pairs
-// The last bucket, when ragged, is handled by a one-warp launch of the same code with guarded
-// plain loads, so the main kernel carries no tail logic.
-#include "gq_round.cuh"
+// gq_warp.cu -- entry of the register path (d = 128, 256, 512): picks the per-scheme launcher.
+#include "gq_internal.h"
 
 namespace gq {
-namespace {
 
-constexpr int kWarpsPerCta = 4;
-constexpr int kHistCols = 8;
-// Items staged ahead per warp (bulk-copy buffers of 2 x d floats each).
-#ifndef GQ_WARP_STAGES
-#define GQ_WARP_STAGES 1
-#endif
-constexpr int kStages = GQ_WARP_STAGES;
-
-template <int EPL>
-struct alignas(16) StageBuf {
-    float g[32 * EPL];
-    float r[32 * EPL];
-};
-
-struct alignas(16) FitORQ {
-    uint32_t hcnt[64 * kHistCols];  // [cell][column]: element counts
-    uint32_t hsum[64 * kHistCols];  // [cell][column]: sums of 22-bit fractions
-    long long P1[64];               // sum of positions over cells < k
-    int P0[64];                     // count over cells < k
-    float4 tab[16];                 // bracket k: {lower, upper, 1/(upper-lower), k}
-    float lev[16];                  // ascending levels
-    unsigned char lut[64];          // cell -> bracket
-};
-struct alignas(16) FitQSGD {
-    float2 pair[16];  // {level k, level k+1}
-};
-struct alignas(16) FitPB {
-    unsigned long long s1[64], s2[64];  // per cell: sum of positions, of squared positions
-    unsigned int cnt[64];               // per cell: count
-    long long al[64], be[64], ga[64], de[64];
-};
-struct alignas(16) FitB {
-    int unused;
-};
-
-template <int S> struct FitFor { using type = FitQSGD; };
-template <> struct FitFor<GQ_ORQ> { using type = FitORQ; };
-template <> struct FitFor<GQ_BINGRAD_PB> { using type = FitPB; };
-template <> struct FitFor<GQ_BINGRAD_B> { using type = FitB; };
-
-template <int EPL, int SCHEME>
-struct alignas(16) WarpSmem {
-    StageBuf<EPL> stage[kStages];
-    unsigned long long bar[kStages];
-    typename FitFor<SCHEME>::type fit;
-};
-
-__device__ __forceinline__ int slot_elem(int t, int lane) { return 128 * (t >> 2) + 4 * lane + (t & 3); }
-
-// ---------------------------------------------------------------------------------------------
-// Round + pack + residual + accumulate for one worker-bucket, chunk by chunk.
-// ---------------------------------------------------------------------------------------------
-template <int EPL, bool FUSED, bool RANDOM, bool TAIL, class R>
-__device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t beta, int w, int lane, uint32_t vmask,
-                                     const float (&v)[EPL], const float (&u)[EPL], const int (&pos)[EPL],
-                                     float (&acc)[EPL])
-{
-    const int64_t base = beta * (int64_t)(32 * EPL);
-    float *r = p.r[w];
-    unsigned char *msg = p.msg[w];
-    uint32_t *cw = msg ? reinterpret_cast<uint32_t *>(msg) + beta * p.codes_words : nullptr;
-    const uint32_t worker = p.worker0 + (uint32_t)w;
-#pragma unroll
-    for (int m = 0; m < EPL / 4; ++m) {
-        const float vv[4] = {v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]};
-        const float uu[4] = {u[4 * m], u[4 * m + 1], u[4 * m + 2], u[4 * m + 3]};
-        const int pp[4] = {pos[4 * m], pos[4 * m + 1], pos[4 * m + 2], pos[4 * m + 3]};
-        const uint32_t valid = TAIL ? (vmask >> (4 * m)) & 0xfu : 0xfu;
-        float q[4];
-        round_chunk<RANDOM, !TAIL>(p, rule, (uint64_t)(base >> 2) + (uint64_t)(32 * m), worker, lane, valid, vv, uu,
-                                   pp, r ? r + base + 128 * m : nullptr, cw ? cw + m * 4 * p.bits : nullptr, q);
-        if (FUSED) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                if (!TAIL || ((valid >> c) & 1u)) acc[4 * m + c] = __fadd_rn(acc[4 * m + c], q[c]);
-        }
-    }
-}
-
-// Level table of the message (L floats per bucket).
-__device__ __forceinline__ void store_table(const KParams &p, int w, int64_t beta, int lane, float value)
-{
-    unsigned char *msg = p.msg[w];
-    if (msg && lane < p.L) reinterpret_cast<float *>(msg + p.levels_off)[beta * p.L + lane] = value;
-}
-
-__device__ __forceinline__ void flag_nonfinite(const KParams &p, int lane)
-{
-    if (lane == 0) atomicOr(p.status, kStatusNonFinite);
-}
-
-// ---------------------------------------------------------------------------------------------
-// Per-scheme fits (u: the values to quantize; v: the error-fed values the residual refers to)
-// ---------------------------------------------------------------------------------------------
-template <int EPL, bool FUSED, bool TAIL>
-__device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
-                         const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
-{
-    float m = 0.0f;
-#pragma unroll
-    for (int t = 0; t < EPL; ++t)
-        if (!TAIL || ((vmask >> t) & 1u)) m = fmax_nan(m, fabsf(u[t]));
-    m = warp_max_nan(m);
-    if (check && !(m <= FLT_MAX)) flag_nonfinite(p, lane);
-    const int s = p.s;
-    const float lv = lane < s ? __fmul_rn(m, __fdiv_rn((float)(2 * lane - (s - 1)), (float)(s - 1))) : 0.0f;
-    const float lv_next = __shfl_down_sync(kFull, lv, 1);
-    __syncwarp();
-    if (lane < s - 1) sm.pair[lane] = make_float2(lv, lv_next);
-    __syncwarp();
-    RoundQSGD rule;
-    rule.inv_m = m > 0.0f ? __fdiv_rn(1.0f, m) : 0.0f;
-    rule.h = __fmul_rn((float)(s - 1), 0.5f);
-    rule.kmax = s - 2;
-    rule.pair = sm.pair;
-    int pos[EPL];
-#pragma unroll
-    for (int t = 0; t < EPL; ++t) pos[t] = 0;
-    emit<EPL, FUSED, true, TAIL>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
-    store_table(p, w, beta, lane, m);
-}
-
-template <int EPL, bool FUSED, bool TAIL>
-__device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
-                        const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
-{
-    float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-    for (int t = 0; t < EPL; ++t)
-        if (!TAIL || ((vmask >> t) & 1u)) {
-            mn = fmin_nan(mn, u[t]);
-            mx = fmax_nan(mx, u[t]);
-        }
-    mn = warp_min_nan(mn);
-    mx = warp_max_nan(mx);
-    if (check && !(mn >= -FLT_MAX && mx <= FLT_MAX)) flag_nonfinite(p, lane);
-    mn = __fadd_rn(mn, 0.0f);
-    mx = __fadd_rn(mx, 0.0f);
-    int pos[EPL];
-    if (!(mx > mn)) {  // constant bucket (or NaN): one level, code 0
-#pragma unroll
-        for (int t = 0; t < EPL; ++t) pos[t] = 0;
-        emit<EPL, FUSED, false, TAIL>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc);
-        store_table(p, w, beta, lane, mn);
-        return;
-    }
-    const float range = __fsub_rn(mx, mn);
-    const float step = __fdiv_rn(range, 63.0f);
-    const float scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kOrqFBits));
-    // histogram: 8 columns per cell, lane l adds into column l % 8 with shared atomics; the
-    // rounding pass needs only the cell of each value, so the cells are what is kept
-    const int col = lane & (kHistCols - 1);
-#pragma unroll
-    for (int t = 0; t < EPL; ++t) {
-        // every valid value is finite and >= mn here, so the position is >= 0 without a clamp
-        int ps = min(__float2int_rz(__fmul_rn(__fsub_rn(u[t], mn), scale)), 63 << kOrqFBits);
-        if (TAIL) ps = max(ps, 0);
-        const int cell = min(ps >> kOrqFBits, kTopCell);
-        pos[t] = cell;
-        if (!TAIL || ((vmask >> t) & 1u)) {
-            atomicAdd(&sm.hcnt[cell * kHistCols + col], 1u);
-            atomicAdd(&sm.hsum[cell * kHistCols + col], (uint32_t)(ps - (cell << kOrqFBits)));
-        }
-    }
-    __syncwarp();
-    // lane l reduces cells 2l and 2l+1 (16 consecutive words per array), clearing them; the
-    // four 16-byte reads are rotated by l/2 so that a quarter-warp touches 8 distinct bank groups
-    uint32_t c0 = 0, c1 = 0, f0 = 0, f1 = 0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int q4 = (k + (lane >> 1)) & 3;
-        uint4 *pc = reinterpret_cast<uint4 *>(sm.hcnt + lane * 16) + q4;
-        uint4 *pf = reinterpret_cast<uint4 *>(sm.hsum + lane * 16) + q4;
-        const uint4 xc = *pc, xf = *pf;
-        *pc = make_uint4(0u, 0u, 0u, 0u);
-        *pf = make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t sc = xc.x + xc.y + xc.z + xc.w;
-        const uint32_t sf = xf.x + xf.y + xf.z + xf.w;
-        if (q4 < 2) {
-            c0 += sc;
-            f0 += sf;
-        } else {
-            c1 += sc;
-            f1 += sf;
-        }
-    }
-    // sums of positions of the two cells; one exclusive prefix over the cell pairs of the packed
-    // (sum << 16 | count): counts stay below 2^16 and sums below 2^37 for d <= 512
-    const long long s0 = (long long)c0 * ((long long)(2 * lane) << kOrqFBits) + f0;
-    const long long s1 = (long long)c1 * ((long long)(2 * lane + 1) << kOrqFBits) + f1;
-    const unsigned long long own = ((unsigned long long)(s0 + s1) << 16) | (c0 + c1);
-    const unsigned long long ex = warp_inclusive_scan(own, lane) - own;
-    const int ec = (int)(ex & 0xffffu);
-    const long long es = (long long)(ex >> 16);
-    reinterpret_cast<int2 *>(sm.P0)[lane] = make_int2(ec, ec + (int)c0);
-    reinterpret_cast<longlong2 *>(sm.P1)[lane] = make_longlong2(es, es + s0);
-    __syncwarp();
-    const unsigned long long mask = orq_greedy(sm.P0, sm.P1, p.s, lane);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int j = lane + 32 * h;
-        if ((mask >> j) & 1ull) sm.lev[__popcll(mask & ((1ull << j) - 1ull))] = grid_point(mn, mx, step, j);
-        if (j <= kTopCell) sm.lut[j] = (unsigned char)(__popcll(mask & ((2ull << j) - 1ull)) - 1);
-    }
-    __syncwarp();
-    if (lane < p.s - 1) {
-        const float lo = sm.lev[lane], hi = sm.lev[lane + 1];
-        sm.tab[lane] = make_float4(lo, hi, __fdiv_rn(1.0f, __fsub_rn(hi, lo)), __int_as_float(lane));
-    }
-    __syncwarp();
-    emit<EPL, FUSED, true, TAIL>(p, RoundORQ{sm.lut, sm.tab}, beta, w, lane, vmask, v, u, pos, acc);
-    store_table(p, w, beta, lane, lane < p.s ? sm.lev[lane] : 0.0f);
-    __syncwarp();
-}
-
-// Bitonic sort of the 32*EPL keys, position i = lane*EPL + r.
-template <int EPL>
-__device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
-{
-    constexpr int N = 32 * EPL;
-#pragma unroll
-    for (int k = 2; k <= N; k <<= 1) {
-#pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            if (j >= EPL) {
-                const int lm = j / EPL;
-#pragma unroll
-                for (int r = 0; r < EPL; ++r) {
-                    const int i = lane * EPL + r;
-                    const float o = __shfl_xor_sync(kFull, key[r], lm);
-                    const bool up = (i & k) == 0;
-                    const bool lower = (i & j) == 0;
-                    key[r] = (lower == up) ? fminf(key[r], o) : fmaxf(key[r], o);
-                }
-            } else {
-#pragma unroll
-                for (int r = 0; r < EPL; ++r) {
-                    if ((r & j) == 0) {
-                        const int i = lane * EPL + r;
-                        const bool up = (i & k) == 0;
-                        const float a = key[r], b = key[r ^ j];
-                        key[r] = up ? fminf(a, b) : fmaxf(a, b);
-                        key[r ^ j] = up ? fmaxf(a, b) : fminf(a, b);
-                    }
-                }
-            }
-        }
-    }
-}
-
-template <int EPL, bool FUSED, bool TAIL>
-__device__ void fit_bingrad_b(const KParams &p, FitB &, int64_t beta, int w, int lane, uint32_t vmask, bool check,
-                              int nvalid, const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
-{
-    float m = 0.0f;
-#pragma unroll
-    for (int t = 0; t < EPL; ++t)
-        if (!TAIL || ((vmask >> t) & 1u)) m = fmax_nan(m, fabsf(u[t]));
-    m = warp_max_nan(m);
-    if (check && !(m <= FLT_MAX)) flag_nonfinite(p, lane);
-    int pos[EPL];
-#pragma unroll
-    for (int t = 0; t < EPL; ++t) pos[t] = 0;
-    RoundB rule{0.0f, 0.0f, 0.0f, false};
-    if (m > 0.0f) {
-        float key[EPL];
-#pragma unroll
-        for (int t = 0; t < EPL; ++t) key[t] = (!TAIL || ((vmask >> t) & 1u)) ? u[t] : INFINITY;
-        warp_bitonic_sort<EPL>(key, lane);
-        const int e = 46 - fexpo(m);
-        const double sc = pow2d(e);
-        // inclusive prefix of the fixed-point values inside the lane, then across lanes
-        long long pre[EPL];
-        long long run = 0;
-#pragma unroll
-        for (int r = 0; r < EPL; ++r) {
-            const int i = lane * EPL + r;
-            run += (!TAIL || i < nvalid) ? fixed_point(key[r], sc) : 0ll;
-            pre[r] = run;
-        }
-        const long long incl = warp_inclusive_scan(run, lane);
-        const long long lane_excl = incl - run;
-        const long long total = __shfl_sync(kFull, incl, 31);
-        const float prev_last = __shfl_up_sync(kFull, key[EPL - 1], 1);
-        double best_j = -1.0;
-        int best_i = 0x7fffffff;
-#pragma unroll
-        for (int r = 0; r < EPL; ++r) {
-            const int i = lane * EPL + r;  // split: positions < i on the left
-            const float prev = r > 0 ? key[r - 1] : prev_last;
-            if (i >= 1 && i < nvalid && prev < key[r]) {
-                const long long Sl = lane_excl + (r > 0 ? pre[r - 1] : 0ll);
-                const double l = __ll2double_rn(Sl);
-                const double rr = __ll2double_rn(total - Sl);
-                const double J = __dadd_rn(__ddiv_rn(__dmul_rn(l, l), (double)i),
-                                           __ddiv_rn(__dmul_rn(rr, rr), (double)(nvalid - i)));
-                if (J > best_j) {
-                    best_j = J;
-                    best_i = i;
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double oj = __shfl_xor_sync(kFull, best_j, o);
-            const int oi = __shfl_xor_sync(kFull, best_i, o);
-            if (oj > best_j || (oj == best_j && oi < best_i)) {
-                best_j = oj;
-                best_i = oi;
-            }
-        }
-        if (best_i == 0x7fffffff) {
-            // every value equal: a single level, code 0
-            const float v0 = __fadd_rn(__shfl_sync(kFull, key[0], 0), 0.0f);
-            rule = RoundB{v0, v0, v0, false};
-        } else {
-            // owner lane publishes the threshold value and the left sum
-            float tv = 0.0f;
-            long long sl = 0;
-#pragma unroll
-            for (int r = 0; r < EPL; ++r)
-                if (lane * EPL + r == best_i) {
-                    tv = key[r];
-                    sl = lane_excl + (r > 0 ? pre[r - 1] : 0ll);
-                }
-            const int owner = best_i / EPL;
-            tv = __shfl_sync(kFull, tv, owner);
-            sl = __shfl_sync(kFull, sl, owner);
-            const double inv_sc = pow2d(-e);
-            const float a = __double2float_rn(__dmul_rn(__ddiv_rn(__ll2double_rn(sl), (double)best_i), inv_sc));
-            const float b = __double2float_rn(
-                __dmul_rn(__ddiv_rn(__ll2double_rn(total - sl), (double)(nvalid - best_i)), inv_sc));
-            rule = RoundB{a, b, tv, true};
-        }
-    }
-    emit<EPL, FUSED, false, TAIL>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
-    store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
-}
-
-template <int EPL, bool FUSED, bool TAIL>
-__device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
-                               const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
-{
-    float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-    for (int t = 0; t < EPL; ++t)
-        if (!TAIL || ((vmask >> t) & 1u)) {
-            mn = fmin_nan(mn, u[t]);
-            mx = fmax_nan(mx, u[t]);
-        }
-    mn = warp_min_nan(mn);
-    mx = warp_max_nan(mx);
-    if (check && !(mn >= -FLT_MAX && mx <= FLT_MAX)) flag_nonfinite(p, lane);
-    mn = __fadd_rn(mn, 0.0f);
-    mx = __fadd_rn(mx, 0.0f);
-    int pos[EPL];
-    if (!(mx > mn)) {
-#pragma unroll
-        for (int t = 0; t < EPL; ++t) pos[t] = 0;
-        emit<EPL, FUSED, false, TAIL>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc);
-        store_table(p, w, beta, lane, mn);
-        return;
-    }
-    const float range = __fsub_rn(mx, mn);
-    const float step = __fdiv_rn(range, 63.0f);
-    const float scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kPbFBits));
-#pragma unroll
-    for (int t = 0; t < EPL; ++t) {
-        pos[t] = grid_pos<kPbFBits>(u[t], mn, scale);
-        if (!TAIL || ((vmask >> t) & 1u)) {
-            const int cell = min(pos[t] >> kPbFBits, kTopCell);
-            const unsigned long long x = (unsigned long long)pos[t];
-            atomicAdd(&sm.cnt[cell], 1u);
-            atomicAdd(&sm.s1[cell], x);
-            atomicAdd(&sm.s2[cell], x * x);
-        }
-    }
-    __syncwarp();
-    // prefix sums Q0, Q1, Q2 over cells < k, then the per-index terms of
-    // E(A,B) = al[A] + be[B] + a*ga[B] + b*de[A]   (a = A*2^16, b = B*2^16)
-    const long long c0 = sm.cnt[lane], c1 = sm.cnt[lane + 32];
-    const long long x0 = (long long)sm.s1[lane], x1 = (long long)sm.s1[lane + 32];
-    const long long y0 = (long long)sm.s2[lane], y1 = (long long)sm.s2[lane + 32];
-    __syncwarp();
-    sm.cnt[lane] = 0u;
-    sm.cnt[lane + 32] = 0u;
-    sm.s1[lane] = 0ull;
-    sm.s1[lane + 32] = 0ull;
-    sm.s2[lane] = 0ull;
-    sm.s2[lane + 32] = 0ull;
-    const long long ic0 = warp_inclusive_scan(c0, lane), ic1 = warp_inclusive_scan(c1, lane);
-    const long long ix0 = warp_inclusive_scan(x0, lane), ix1 = warp_inclusive_scan(x1, lane);
-    const long long iy0 = warp_inclusive_scan(y0, lane), iy1 = warp_inclusive_scan(y1, lane);
-    const long long tc = __shfl_sync(kFull, ic0, 31), tx = __shfl_sync(kFull, ix0, 31), ty = __shfl_sync(kFull, iy0, 31);
-    const long long tc_all = __shfl_sync(kFull, tc + ic1, 31);
-    const long long tx_all = __shfl_sync(kFull, tx + ix1, 31);
-    const long long ty_all = __shfl_sync(kFull, ty + iy1, 31);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int K = lane + 32 * h;
-        const long long Q0 = h ? tc + ic1 - c1 : ic0 - c0;
-        const long long Q1 = h ? tx + ix1 - x1 : ix0 - x0;
-        const long long Q2 = h ? ty + iy1 - y1 : iy0 - y0;
-        const unsigned long long k = (unsigned long long)K << kPbFBits;
-        // modular 64-bit arithmetic: every E(A,B) fits in int64, so wrapped partial terms cancel
-        const unsigned long long uQ0 = Q0, uQ1 = Q1, uQ2 = Q2;
-        sm.al[K] = (long long)(k * k * uQ0 - 3ull * k * uQ1 + 2ull * uQ2);
-        sm.be[K] = (long long)(3ull * k * uQ1 - 2ull * uQ2 + (unsigned long long)ty_all - 2ull * k * (unsigned long long)tx_all +
-                               k * k * ((unsigned long long)tc_all - uQ0));
-        sm.ga[K] = (long long)(uQ1 - k * uQ0);
-        sm.de[K] = (long long)(k * uQ0 - uQ1);
-    }
-    __syncwarp();
-    // exhaustive search over A < B, ties to the smallest (A, B)
-    long long best_e = 0x7fffffffffffffffll;
-    int best_ab = 0x7fffffff;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int B = lane + 32 * h;
-        const unsigned long long bb = (unsigned long long)B << kPbFBits;
-        const unsigned long long beB = sm.be[B], gaB = sm.ga[B];
-        for (int A = 0; A < B; ++A) {
-            const unsigned long long aa = (unsigned long long)A << kPbFBits;
-            const long long e = (long long)((unsigned long long)sm.al[A] + beB + aa * gaB + bb * (unsigned long long)sm.de[A]);
-            const int ab = A * 64 + B;
-            if (e < best_e || (e == best_e && ab < best_ab)) {
-                best_e = e;
-                best_ab = ab;
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const long long oe = __shfl_xor_sync(kFull, best_e, o);
-        const int oab = __shfl_xor_sync(kFull, best_ab, o);
-        if (oe < best_e || (oe == best_e && oab < best_ab)) {
-            best_e = oe;
-            best_ab = oab;
-        }
-    }
-    const int A = best_ab >> 6, B = best_ab & 63;
-    RoundPB rule;
-    rule.a = grid_point(mn, mx, step, A);
-    rule.b = grid_point(mn, mx, step, B);
-    rule.rinv = __fdiv_rn(1.0f, __fsub_rn(rule.b, rule.a));
-    rule.pa = A << kPbFBits;
-    rule.pb = B << kPbFBits;
-    emit<EPL, FUSED, true, TAIL>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
-    store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
-}
-
-// ---------------------------------------------------------------------------------------------
-// One item: clip, fit, round, write
-// ---------------------------------------------------------------------------------------------
-template <int EPL, int SCHEME, bool FUSED, bool TAIL>
-__device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME>::type &fit, int64_t beta, int w,
-                                        int lane, int nvalid, uint32_t vmask, const float (&v)[EPL], float (&acc)[EPL])
-{
-    float u[EPL];
-    bool check = true;  // the fit flags non-finite values unless the clip pass already did
-    if (p.clip > 0.0f) {
-        float am = 0.0f;
-#pragma unroll
-        for (int t = 0; t < EPL; ++t)
-            if (!TAIL || ((vmask >> t) & 1u)) am = fmax_nan(am, fabsf(v[t]));
-        am = warp_max_nan(am);
-        if (!(am <= FLT_MAX)) flag_nonfinite(p, lane);
-        check = false;
-        float T = 0.0f;
-        if (am > 0.0f) {
-            const int e = 20 - fexpo(am);
-            const double sc = pow2d(e);
-            long long sx = 0, sxx = 0;
-#pragma unroll
-            for (int t = 0; t < EPL; ++t)
-                if (!TAIL || ((vmask >> t) & 1u)) {
-                    const long long X = fixed_point(v[t], sc);
-                    sx += X;
-                    sxx += X * X;
-                }
-            sx = warp_sum(sx);
-            sxx = warp_sum(sxx);
-            T = clip_threshold_from_sums(sx, sxx, nvalid, e, p.clip);
-        }
-#pragma unroll
-        for (int t = 0; t < EPL; ++t) {
-            float x = v[t];
-            x = x < -T ? -T : x;
-            x = x > T ? T : x;
-            u[t] = x;
-        }
-    } else {
-#pragma unroll
-        for (int t = 0; t < EPL; ++t) u[t] = v[t];
-    }
-    if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD)
-        fit_qsgd<EPL, FUSED, TAIL>(p, fit, beta, w, lane, vmask, check, v, u, acc);
-    else if constexpr (SCHEME == GQ_ORQ)
-        fit_orq<EPL, FUSED, TAIL>(p, fit, beta, w, lane, vmask, check, v, u, acc);
-    else if constexpr (SCHEME == GQ_BINGRAD_B)
-        fit_bingrad_b<EPL, FUSED, TAIL>(p, fit, beta, w, lane, vmask, check, nvalid, v, u, acc);
-    else
-        fit_bingrad_pb<EPL, FUSED, TAIL>(p, fit, beta, w, lane, vmask, check, v, u, acc);
-}
-
-// ---------------------------------------------------------------------------------------------
-// The kernels
-// ---------------------------------------------------------------------------------------------
-// Resident CTAs per SM the register allocation is sized for (4 x 4 warps: 128 registers; at
-// 5 x 4 warps the 96-register cap spills and measured slower).
-#ifndef GQ_WARP_MIN_BLOCKS
-#define GQ_WARP_MIN_BLOCKS 4
-#endif
-template <int EPL, int SCHEME, int WARPS>
-constexpr int min_blocks()
-{
-    return (SCHEME == GQ_BINGRAD_B || SCHEME == GQ_BINGRAD_PB) ? 2 : GQ_WARP_MIN_BLOCKS * 4 / WARPS;
-}
-
-template <int SCHEME, class Fit>
-__device__ __forceinline__ void init_fit(Fit &fit, int lane)
-{
-    if constexpr (SCHEME == GQ_ORQ) {
-        for (int i = lane; i < 64 * kHistCols; i += 32) {
-            fit.hcnt[i] = 0u;
-            fit.hsum[i] = 0u;
-        }
-    }
-    if constexpr (SCHEME == GQ_BINGRAD_PB) {
-        for (int i = lane; i < 64; i += 32) {
-            fit.cnt[i] = 0u;
-            fit.s1[i] = 0ull;
-            fit.s2[i] = 0ull;
-        }
-    }
-}
-
-__device__ __forceinline__ void store_avg4(float *ab, int m, int lane, const float *acc, float inv_w)
-{
-    __stcs(reinterpret_cast<float4 *>(ab + 128 * m + 4 * lane),
-           make_float4(__fmul_rn(acc[0], inv_w), __fmul_rn(acc[1], inv_w), __fmul_rn(acc[2], inv_w),
-                       __fmul_rn(acc[3], inv_w)));
-}
-
-// Full buckets 0 .. nfull-1: every warp walks its items (bucket, worker), bulk copies one item
-// ahead.
-template <int EPL, int SCHEME, bool FUSED>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME, kWarpsPerCta>()))
-    k_warp(const __grid_constant__ KParams p, int64_t nfull)
-{
-    using Smem = WarpSmem<EPL, SCHEME>;
-    constexpr int D = 32 * EPL;
-    constexpr unsigned kBytes = D * 4;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    const int lane = threadIdx.x & 31;
-    const int wib = threadIdx.x >> 5;
-    Smem &sm = reinterpret_cast<Smem *>(smem_raw)[wib];
-    init_fit<SCHEME>(sm.fit, lane);
-    if (lane == 0) {
-        for (int k = 0; k < kStages; ++k) mbar_init(&sm.bar[k], 1);
-        fence_barrier_init();
-    }
-    __syncwarp();
-
-    const int64_t first = (int64_t)blockIdx.x * kWarpsPerCta + wib;
-    const int64_t stride = (int64_t)gridDim.x * kWarpsPerCta;
-    if (first >= nfull) return;
-    const int W = p.W;
-    const int64_t nitems = ((nfull - 1 - first) / stride + 1) * W;
-    const bool ef = p.r[0] != nullptr;
-    const unsigned tx = ef ? 2 * kBytes : kBytes;
-    auto issue = [&](int64_t beta, int w, int k) {  // lane 0
-        fence_proxy_async();
-        mbar_arrive_expect_tx(&sm.bar[k], tx);
-        bulk_load(sm.stage[k].g, p.g[w] + beta * D, kBytes, &sm.bar[k]);
-        if (ef) bulk_load(sm.stage[k].r, p.r[w] + beta * D, kBytes, &sm.bar[k]);
-    };
-    // producer position: kStages items ahead of the consumer
-    int64_t pbeta = first;
-    int pw = 0;
-    for (int k = 0; k < kStages; ++k) {
-        if (lane == 0 && (int64_t)k < nitems) issue(pbeta, pw, k);
-        if (++pw == W) {
-            pw = 0;
-            pbeta += stride;
-        }
-    }
-
-    int64_t beta = first;
-    int w = 0;
-    unsigned parity = 0;  // bit k: phase parity awaited next on buffer k
-    float acc[EPL];
-    for (int64_t it = 0; it < nitems; ++it) {
-        const int k = kStages == 1 ? 0 : (int)(it % kStages);
-        if (!mbar_wait_warp(&sm.bar[k], (parity >> k) & 1u)) {
-            // a copy did not complete in time: report it, give every copy still in flight one
-            // more bounded wait so that none can land after the warp has left, and stop
-            if (lane == 0) atomicOr(p.status, kStatusTimeout);
-            for (int j = 0; j < kStages; ++j)
-                if ((int64_t)j + it < nitems) mbar_wait_warp(&sm.bar[(k + j) % kStages], (parity >> ((k + j) % kStages)) & 1u);
-            return;
-        }
-        parity ^= 1u << k;
-        float v[EPL];
-#pragma unroll
-        for (int m = 0; m < EPL / 4; ++m) {
-            float4 x = *reinterpret_cast<const float4 *>(sm.stage[k].g + 128 * m + 4 * lane);
-            if (ef) {
-                const float4 y = *reinterpret_cast<const float4 *>(sm.stage[k].r + 128 * m + 4 * lane);
-                x = make_float4(__fadd_rn(x.x, y.x), __fadd_rn(x.y, y.y), __fadd_rn(x.z, y.z), __fadd_rn(x.w, y.w));
-            }
-            v[4 * m + 0] = x.x;
-            v[4 * m + 1] = x.y;
-            v[4 * m + 2] = x.z;
-            v[4 * m + 3] = x.w;
-        }
-        __syncwarp();
-        // the buffer is free again: fetch the item kStages ahead while this one is processed
-        if (lane == 0 && it + kStages < nitems) issue(pbeta, pw, k);
-        if (++pw == W) {
-            pw = 0;
-            pbeta += stride;
-        }
-        const bool last_w = w == W - 1;
-        if (w == 0) {
-#pragma unroll
-            for (int t = 0; t < EPL; ++t) acc[t] = 0.0f;
-        }
-        process<EPL, SCHEME, FUSED, false>(p, sm.fit, beta, w, lane, D, 0xffffffffu, v, acc);
-        if (FUSED && last_w) {
-#pragma unroll
-            for (int m = 0; m < EPL / 4; ++m) store_avg4(p.avg + beta * D, m, lane, acc + 4 * m, p.inv_w);
-        }
-        if (last_w) {
-            w = 0;
-            beta += stride;
-        } else {
-            ++w;
-        }
-    }
-}
-
-// The ragged last bucket (n not a multiple of d): guarded plain loads, one warp per worker
-// (warp k takes workers k, k + nwarps, ...).  Each warp's dequantized values are parked in
-// shared memory (qbuf[w][e]) and summed afterwards in worker order, which gives the same bits
-// as the register sum of the main kernel: every partial sum starts from +0.
-template <int EPL, int SCHEME, bool FUSED>
-__global__ void __launch_bounds__(512) k_warp_tail(const __grid_constant__ KParams p)
-{
-    using Fit = typename FitFor<SCHEME>::type;
-    constexpr int D = 32 * EPL;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    Fit &fit = reinterpret_cast<Fit *>(smem_raw)[wid];
-    float *qbuf = reinterpret_cast<float *>(smem_raw + sizeof(Fit) * nwarps);  // [W][D]
-    init_fit<SCHEME>(fit, lane);
-    __syncwarp();
-    const int64_t beta = p.nb - 1;
-    const int nvalid = p.tail;
-    uint32_t vmask = 0;
-#pragma unroll
-    for (int t = 0; t < EPL; ++t) vmask |= (slot_elem(t, lane) < nvalid ? 1u : 0u) << t;
-    for (int w = wid; w < p.W; w += nwarps) {
-        const float *gb = p.g[w] + beta * D;
-        const float *rb = p.r[w] ? p.r[w] + beta * D : nullptr;
-        float v[EPL], acc[EPL];
-#pragma unroll
-        for (int t = 0; t < EPL; ++t) {
-            const int e = slot_elem(t, lane);
-            float x = 0.0f;
-            if (e < nvalid) {
-                x = gb[e];
-                if (rb) x = __fadd_rn(x, rb[e]);
-            }
-            v[t] = x;
-            acc[t] = 0.0f;
-        }
-        process<EPL, SCHEME, FUSED, true>(p, fit, beta, w, lane, nvalid, vmask, v, acc);
-        if (FUSED) {
-#pragma unroll
-            for (int t = 0; t < EPL; ++t) qbuf[w * D + slot_elem(t, lane)] = acc[t];
-        }
-    }
-    if (FUSED) {
-        __syncthreads();
-        float *ab = p.avg + beta * D;
-        for (int e = threadIdx.x; e < nvalid; e += blockDim.x) {
-            float sum = 0.0f;
-            for (int w = 0; w < p.W; ++w) sum = __fadd_rn(sum, qbuf[w * D + e]);
-            ab[e] = __fmul_rn(sum, p.inv_w);
-        }
-    }
-}
-
-template <int EPL, int SCHEME, bool FUSED>
-cudaError_t launch_one(const KParams &p, cudaStream_t stream)
-{
-    constexpr int D = 32 * EPL;
-    const int64_t nfull = p.tail == D ? p.nb : p.nb - 1;
-    if (nfull > 0) {
-        auto kern = k_warp<EPL, SCHEME, FUSED>;
-        const size_t smem = sizeof(WarpSmem<EPL, SCHEME>) * kWarpsPerCta;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        int dev = 0, sms = 0, per_sm = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarpsPerCta * 32, smem);
-        if (per_sm < 1) per_sm = 1;
-        const int64_t need = (nfull + kWarpsPerCta - 1) / kWarpsPerCta;
-        const int64_t cap = (int64_t)sms * per_sm;
-        const int grid = (int)(need < cap ? need : cap);
-        kern<<<grid, kWarpsPerCta * 32, smem, stream>>>(p, nfull);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    if (nfull < p.nb) {
-        using Fit = typename FitFor<SCHEME>::type;
-        auto tail = k_warp_tail<EPL, SCHEME, FUSED>;
-        const int nwarps = p.W < 16 ? p.W : 16;
-        const size_t smem = sizeof(Fit) * nwarps + (FUSED ? (size_t)p.W * D * 4 : 0);
-        cudaError_t e = cudaFuncSetAttribute(tail, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        tail<<<1, 32 * nwarps, smem, stream>>>(p);
-        return cudaGetLastError();
-    }
-    return cudaSuccess;
-}
-
-template <int EPL, bool FUSED>
-cudaError_t dispatch_scheme(const KParams &p, cudaStream_t stream)
-{
-    switch (p.scheme) {
-    case GQ_QSGD:
-    case GQ_TERNGRAD: return launch_one<EPL, GQ_QSGD, FUSED>(p, stream);
-    case GQ_BINGRAD_B: return launch_one<EPL, GQ_BINGRAD_B, FUSED>(p, stream);
-    case GQ_BINGRAD_PB: return launch_one<EPL, GQ_BINGRAD_PB, FUSED>(p, stream);
-    default: return launch_one<EPL, GQ_ORQ, FUSED>(p, stream);
-    }
-}
-
-template <bool FUSED>
-cudaError_t dispatch_bucket(const KParams &p, cudaStream_t stream)
-{
-    switch (p.d) {
-    case 128: return dispatch_scheme<4, FUSED>(p, stream);
-    case 256: return dispatch_scheme<8, FUSED>(p, stream);
-    default: return dispatch_scheme<16, FUSED>(p, stream);
-    }
-}
-
-}  // namespace
+cudaError_t launch_warp_orq(const KParams &p, bool fused, cudaStream_t stream);
+cudaError_t launch_warp_qsgd(const KParams &p, bool fused, cudaStream_t stream);
+cudaError_t launch_warp_bingrad(const KParams &p, bool fused, cudaStream_t stream);
 
 cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream)
 {
-    return fused ? dispatch_bucket<true>(p, stream) : dispatch_bucket<false>(p, stream);
+    switch (p.scheme) {
+    case GQ_QSGD:
+    case GQ_TERNGRAD: return launch_warp_qsgd(p, fused, stream);
+    case GQ_BINGRAD_B:
+    case GQ_BINGRAD_PB: return launch_warp_bingrad(p, fused, stream);
+    default: return launch_warp_orq(p, fused, stream);
+    }
 }
 
 }  // namespace gq

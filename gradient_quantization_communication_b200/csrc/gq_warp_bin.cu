@@ -1,0 +1,12 @@
+// gq_warp_bin.cu -- instantiation of the register-path kernels for GQ_BINGRAD_B, GQ_BINGRAD_PB.
+#include "gq_warp.cuh"
+
+namespace gq {
+
+cudaError_t launch_warp_bingrad(const KParams &p, bool fused, cudaStream_t stream)
+{
+    return p.scheme == GQ_BINGRAD_B ? warp_dispatch<GQ_BINGRAD_B>(p, fused, stream)
+                                    : warp_dispatch<GQ_BINGRAD_PB>(p, fused, stream);
+}
+
+}  // namespace gq
