@@ -75,6 +75,8 @@ def lib():
         L.or_encode.argtypes = [P(_Cfg), ctypes.c_int, ctypes.c_uint64, i64, i64, f32p, f32p, u8p]
         L.or_decode_accumulate.argtypes = [P(_Cfg), P(u8p), ctypes.c_int, i64, i64, f32p]
         L.or_fused_step.argtypes = [P(_Cfg), ctypes.c_uint64, i64, i64, P(f32p), P(f32p), P(u8p), f32p]
+        L.or_quant_error.argtypes = [P(_Cfg), ctypes.c_int, ctypes.c_uint64, i64, i64, f32p, f32p,
+                                     P(ctypes.c_double)]
         L.or_fused_bucket.argtypes = [P(_Cfg), ctypes.c_uint64, i64, ctypes.c_int, P(f32p), P(f32p), P(f32p),
                                       P(u32p), P(f32p), f32p]
         _lib = L
@@ -263,3 +265,15 @@ def fused_bucket(cfg: Config, step, bucket, gs, rs=None):
                                _p(avg, ctypes.c_float))
     assert rc == 0
     return avg[:n], routs, words, tables
+
+
+def quant_error(cfg: Config, worker, step, g, r=None, b0=0, b1=None):
+    """(sum of expected squared rounding error, sum of u^2, realised sum of (Q(u)-u)^2)."""
+    g = _f32(g)
+    b1 = num_buckets(cfg) if b1 is None else b1
+    out = np.zeros(3, dtype=np.float64)
+    rp = _p(_f32(r), ctypes.c_float) if r is not None else None
+    rc = lib().or_quant_error(ctypes.byref(cfg.c()), worker, step, b0, b1, _p(g, ctypes.c_float), rp,
+                              _p(out, ctypes.c_double))
+    assert rc == 0
+    return out

@@ -274,7 +274,8 @@ double or_orq_select(const float *u, int n, int s, int *idx_out)
 }
 
 static void orq_bucket(const or_config *cfg, int worker, uint64_t step, int64_t base,
-                       const float *u, int n, uint8_t *code, float *q, float *table)
+                       const float *u, int n, uint8_t *code, float *q, float *table,
+                       float *blo, float *bhi, float *bp)
 {
     int s = cfg->levels;
     or_gridinfo gi;
@@ -284,6 +285,11 @@ static void orq_bucket(const or_config *cfg, int worker, uint64_t step, int64_t 
         for (int i = 0; i < n; ++i) {
             code[i] = 0;
             q[i] = gi.mn;
+            if (bp) {
+                blo[i] = gi.mn;
+                bhi[i] = gi.mn;
+                bp[i] = 0.0f;
+            }
         }
         return;
     }
@@ -306,6 +312,11 @@ static void orq_bucket(const or_config *cfg, int worker, uint64_t step, int64_t 
         int c = k + (U < p ? 1 : 0);
         code[i] = (uint8_t)c;
         q[i] = table[c];
+        if (bp) {
+            blo[i] = a;
+            bhi[i] = b;
+            bp[i] = p;
+        }
     }
     free(pos);
     free(cell);
@@ -323,7 +334,8 @@ static float qsgd_ratio(int code, int s)
 }
 
 static void qsgd_bucket(const or_config *cfg, int worker, uint64_t step, int64_t base,
-                        const float *u, int n, uint8_t *code, float *q, float *table)
+                        const float *u, int n, uint8_t *code, float *q, float *table,
+                        float *blo, float *bhi, float *bp)
 {
     int s = cfg->levels;
     float m = 0.0f;
@@ -345,6 +357,11 @@ static void qsgd_bucket(const or_config *cfg, int worker, uint64_t step, int64_t
         int c = k + (U < p ? 1 : 0);
         code[i] = (uint8_t)c;
         q[i] = m * qsgd_ratio(c, s);
+        if (bp) {
+            blo[i] = m * qsgd_ratio(k, s);
+            bhi[i] = m * qsgd_ratio(k + 1, s);
+            bp[i] = sat01(p);
+        }
     }
 }
 
@@ -411,7 +428,8 @@ void or_bingrad_b_fit(const float *u, int n, float *a_out, float *b_out, float *
     free(srt);
 }
 
-static void bingrad_b_bucket(const float *u, int n, uint8_t *code, float *q, float *table)
+static void bingrad_b_bucket(const float *u, int n, uint8_t *code, float *q, float *table,
+                             float *blo, float *bhi, float *bp)
 {
     float a, b, thr;
     int split;
@@ -422,6 +440,11 @@ static void bingrad_b_bucket(const float *u, int n, uint8_t *code, float *q, flo
         int c = (split > 0 && u[i] >= thr) ? 1 : 0;
         code[i] = (uint8_t)c;
         q[i] = c ? b : a;
+        if (bp) {
+            blo[i] = a;
+            bhi[i] = b;
+            bp[i] = (float)c;
+        }
     }
 }
 
@@ -478,7 +501,8 @@ void or_bingrad_pb_fit(const float *u, int n, int *A, int *B, float *ga, float *
 }
 
 static void bingrad_pb_bucket(const or_config *cfg, int worker, uint64_t step, int64_t base,
-                              const float *u, int n, uint8_t *code, float *q, float *table)
+                              const float *u, int n, uint8_t *code, float *q, float *table,
+                              float *blo, float *bhi, float *bp)
 {
     or_gridinfo gi;
     if (!grid_setup(u, n, OR_PB_FBITS, &gi)) {
@@ -487,6 +511,11 @@ static void bingrad_pb_bucket(const or_config *cfg, int worker, uint64_t step, i
         for (int i = 0; i < n; ++i) {
             code[i] = 0;
             q[i] = gi.mn;
+            if (bp) {
+                blo[i] = gi.mn;
+                bhi[i] = gi.mn;
+                bp[i] = 0.0f;
+            }
         }
         return;
     }
@@ -501,17 +530,25 @@ static void bingrad_pb_bucket(const or_config *cfg, int worker, uint64_t step, i
     int32_t pa = (int32_t)A << OR_PB_FBITS, pbv = (int32_t)B << OR_PB_FBITS;
     for (int i = 0; i < n; ++i) {
         int c;
+        float p;
         if (pos[i] < pa) {
             c = 0;
+            p = 0.0f;
         } else if (pos[i] >= pbv) {
             c = 1;
+            p = 1.0f;
         } else {
-            float p = sat01((u[i] - a) * rinv);
+            p = sat01((u[i] - a) * rinv);
             float U = or_uniform(cfg->seed, step, (uint32_t)worker, base + i);
             c = U < p ? 1 : 0;
         }
         code[i] = (uint8_t)c;
         q[i] = c ? b : a;
+        if (bp) {
+            blo[i] = a;
+            bhi[i] = b;
+            bp[i] = p;
+        }
     }
     free(pos);
 }
@@ -594,8 +631,11 @@ float or_dequant(const or_config *cfg, const float *table, int code)
 /* ------------------------------------------------------------------------------------------ */
 /* One bucket of one worker.                                                                   */
 /* ------------------------------------------------------------------------------------------ */
-int or_encode_bucket(const or_config *cfg, int worker, uint64_t step, int64_t bucket,
-                     const float *v, int n, uint8_t *code, float *q, float *table)
+static int bucket_len(const or_config *cfg, int64_t bucket);
+
+static int encode_bucket_ex(const or_config *cfg, int worker, uint64_t step, int64_t bucket,
+                            const float *v, int n, uint8_t *code, float *q, float *table,
+                            float *u_out, float *blo, float *bhi, float *bp)
 {
     if (n <= 0) return 0;
     int64_t base = bucket * (int64_t)cfg->bucket;
@@ -611,23 +651,79 @@ int or_encode_bucket(const or_config *cfg, int worker, uint64_t step, int64_t bu
     switch (cfg->scheme) {
     case OR_QSGD:
     case OR_TERNGRAD:
-        qsgd_bucket(cfg, worker, step, base, u, n, code, q, table);
+        qsgd_bucket(cfg, worker, step, base, u, n, code, q, table, blo, bhi, bp);
         break;
     case OR_BINGRAD_B:
-        bingrad_b_bucket(u, n, code, q, table);
+        bingrad_b_bucket(u, n, code, q, table, blo, bhi, bp);
         break;
     case OR_BINGRAD_PB:
-        bingrad_pb_bucket(cfg, worker, step, base, u, n, code, q, table);
+        bingrad_pb_bucket(cfg, worker, step, base, u, n, code, q, table, blo, bhi, bp);
         break;
     case OR_ORQ:
-        orq_bucket(cfg, worker, step, base, u, n, code, q, table);
+        orq_bucket(cfg, worker, step, base, u, n, code, q, table, blo, bhi, bp);
         break;
     default:
         free(u);
         return 1;
     }
+    if (u_out) memcpy(u_out, u, sizeof(float) * (size_t)n);
     free(u);
     return 0;
+}
+
+int or_encode_bucket(const or_config *cfg, int worker, uint64_t step, int64_t bucket,
+                     const float *v, int n, uint8_t *code, float *q, float *table)
+{
+    return encode_bucket_ex(cfg, worker, step, bucket, v, n, code, q, table, NULL, NULL, NULL, NULL);
+}
+
+/*
+ * Quantization error of one worker's vector over the buckets [b0, b1): out[0] = sum of the
+ * expected squared rounding error p (b - u)^2 + (1 - p) (a - u)^2 of every element (u the
+ * value quantized, [a, b] its bracket, p its probability of rounding up; for unbiased rounding
+ * this is the variance (b - u)(u - a) that ORQ minimises), out[1] = sum of u^2, out[2] = sum of
+ * the realised (Q(u) - u)^2 for this step's draws.  binary64, elements in index order.
+ */
+int or_quant_error(const or_config *cfg, int worker, uint64_t step, int64_t b0, int64_t b1,
+                   const float *g, const float *r, double *out)
+{
+    int d = cfg->bucket;
+    float *v = (float *)malloc(sizeof(float) * (size_t)d);
+    float *u = (float *)malloc(sizeof(float) * (size_t)d);
+    float *q = (float *)malloc(sizeof(float) * (size_t)d);
+    float *blo = (float *)malloc(sizeof(float) * (size_t)d);
+    float *bhi = (float *)malloc(sizeof(float) * (size_t)d);
+    float *bp = (float *)malloc(sizeof(float) * (size_t)d);
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    float table[16];
+    double e = 0.0, uu = 0.0, qq = 0.0;
+    int rc = 0;
+    for (int64_t bk = b0; bk < b1 && rc == 0; ++bk) {
+        int n = bucket_len(cfg, bk);
+        int64_t base = bk * d;
+        for (int i = 0; i < n; ++i) v[i] = (cfg->error_feedback && r) ? g[base + i] + r[base + i] : g[base + i];
+        rc = encode_bucket_ex(cfg, worker, step, bk, v, n, code, q, table, u, blo, bhi, bp);
+        for (int i = 0; i < n; ++i) {
+            double P = (double)sat01(bp[i]);
+            double dh = (double)bhi[i] - (double)u[i];
+            double dl = (double)blo[i] - (double)u[i];
+            double dq = (double)q[i] - (double)u[i];
+            e += P * dh * dh + (1.0 - P) * dl * dl;
+            uu += (double)u[i] * (double)u[i];
+            qq += dq * dq;
+        }
+    }
+    out[0] = e;
+    out[1] = uu;
+    out[2] = qq;
+    free(v);
+    free(u);
+    free(q);
+    free(blo);
+    free(bhi);
+    free(bp);
+    free(code);
+    return rc;
 }
 
 /* ------------------------------------------------------------------------------------------ */

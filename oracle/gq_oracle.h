@@ -72,6 +72,11 @@ void or_message_layout(const or_config *cfg, int64_t *bytes, int64_t *codes_off,
 int or_encode_bucket(const or_config *cfg, int worker, uint64_t step, int64_t bucket,
                      const float *v, int n, uint8_t *code, float *q, float *table);
 
+/* Quantization error over buckets [b0, b1) of one worker: out[0] = sum of the expected
+ * squared rounding error, out[1] = sum of u^2, out[2] = realised sum of (Q(u)-u)^2. */
+int or_quant_error(const or_config *cfg, int worker, uint64_t step, int64_t b0, int64_t b1,
+                   const float *g, const float *r, double *out);
+
 /* Pack n codes of one bucket into d*b/32 words (padding codes are 0). */
 void or_pack_bucket(const or_config *cfg, const uint8_t *code, int n, uint32_t *words);
 /* Inverse of or_pack_bucket for the first n codes. */

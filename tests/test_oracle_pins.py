@@ -490,3 +490,59 @@ def test_tie_rules():
     # give the least expected squared error (663, found by exhaustive search); the smaller wins.
     A, B, ga, gb = O.bingrad_pb_fit(np.array([0.0, 8.0, 32.0, 63.0], dtype=np.float32))
     assert (A, B, ga, gb) == (9, 51, 9.0, 51.0)
+
+
+# ------------------------------------------------------------------------------------------
+# Quantization error (expected and realised), the quantity the bucket sweep reports
+# ------------------------------------------------------------------------------------------
+def test_quant_error_matches_brackets_and_monte_carlo():
+    rng = np.random.default_rng(21)
+    n, d = 3 * 128 + 50, 128
+    g = (rng.laplace(0, 1e-3, n)).astype(np.float32)
+    for sch, s in [(O.ORQ, 5), (O.ORQ, 3), (O.QSGD, 5), (O.TERNGRAD, 3)]:
+        cfg = O.Config(sch, s, d, 1, 0, 0.0, 8, n)
+        e, uu, qq = O.quant_error(cfg, 0, 0, g)
+        assert abs(uu - float(np.sum(g.astype(np.float64) ** 2))) <= 1e-12 * uu
+        # expected error = sum (b-u)(u-a) over the brackets of the message's levels
+        msg = O.encode(cfg, 0, 0, g)
+        _, _, loff = O.message_layout(cfg)
+        L = O.table_len(sch, s)
+        tabs = msg[loff:].view(np.float32)
+        ref = 0.0
+        for bk in range(O.num_buckets(cfg)):
+            x = g[bk * d:(bk + 1) * d].astype(np.float64)
+            t = tabs[bk * L:(bk + 1) * L]
+            lv = [float(t[0]) * (2 * k - (s - 1)) / (s - 1) for k in range(s)] if sch in (O.QSGD, O.TERNGRAD) \
+                else [float(v) for v in t]
+            a, b = _bracket_moments(lv, x)
+            ref += float(np.sum(np.maximum((b - x) * (x - a), 0.0)))
+        assert abs(e - ref) <= 1e-6 * ref
+        # the realised error averages to the expected one
+        reps = np.array([O.quant_error(cfg, 0, t, g)[2] for t in range(300)])
+        assert abs(reps.mean() - e) < 5 * reps.std() / np.sqrt(len(reps)) + 1e-3 * e
+
+
+def test_quant_error_deterministic_schemes():
+    rng = np.random.default_rng(22)
+    n, d = 600, 128
+    g = (rng.standard_t(3, n) * 1e-3).astype(np.float32)
+    cfg = O.Config(O.BINGRAD_B, 2, d, 1, 0, 0.0, 1, n)
+    e, uu, qq = O.quant_error(cfg, 0, 0, g)
+    assert e == qq
+    sse = 0.0
+    for bk in range(O.num_buckets(cfg)):
+        x = g[bk * d:(bk + 1) * d]
+        a, b, thr, split = O.bingrad_b_fit(x)
+        xx = x.astype(np.float64)
+        sse += float(np.sum(np.where(xx >= thr, (xx - b) ** 2, (xx - a) ** 2)))
+    assert abs(e - sse) <= 1e-9 * sse
+    cfg = O.Config(O.BINGRAD_PB, 2, d, 1, 0, 0.0, 1, n)
+    e, uu, qq = O.quant_error(cfg, 0, 0, g)
+    ref = 0.0
+    for bk in range(O.num_buckets(cfg)):
+        x = g[bk * d:(bk + 1) * d]
+        _, _, ga, gb = O.bingrad_pb_fit(x)
+        ref += _pb_error(x, ga, gb)
+    # the clamp regions are decided on 16-bit grid positions, the formula here on values:
+    # elements within a position step of a level may fall on either side
+    assert abs(e - ref) <= 1e-6 * ref
