@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="bucket-size sweep (1e8 elements, W = 8, no error feedback): throughput and "
+                         "normalised quantization variance per bucket size, one JSON line")
     return ap.parse_args()
 
 
@@ -421,10 +424,69 @@ def run_cpu_baseline(args, wl, g):
             "sample": "first %d buckets (d=%d) of each of the %d workers, one step" % (nbk, args.bucket, wl.workers)}
 
 
+def run_sweep(args):
+    """Fused-step throughput and normalised quantization variance sum (b-u)(u-a) / sum u^2 for
+    every bucket size of the sweep workload, for ORQ-5 and QSGD-5."""
+    import torch
+
+    import gradient_quantization_communication_b200.gq as G
+    from gradient_quantization_communication_b200 import synth
+
+    wl = synth.WORKLOADS["mixture100m"]
+    n = min(wl.n, args.elements) if args.elements else wl.n
+    W = wl.workers
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    g = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
+    for w in range(W):
+        synth.gradient("mixture100m", w, 0, n=n, out=g[w])
+    avg = torch.empty(n, dtype=torch.float32, device=dev)
+    out = torch.zeros(3, dtype=torch.float64, device=dev)
+    peak, _ = measured_hbm_peak()
+    rows = []
+    for scheme, levels, _clip in wl.schemes:
+        for d in wl.buckets_sweep:
+            cfg = G.gq_config(scheme, levels, d, W, False, 0.0, wl.rounding_seed, n)
+            with G.Plan(cfg) as plan:
+                msgs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)]
+                for t in range(args.warmup):
+                    G.gq_fused_step(plan.handle, t, g, None, msgs, avg)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                a.record()
+                for t in range(args.steps):
+                    G.gq_fused_step(plan.handle, args.warmup + t, g, None, msgs, avg)
+                b.record()
+                torch.cuda.synchronize()
+                ms = a.elapsed_time(b) / args.steps
+                e = uu = 0.0
+                for w in range(W):
+                    G.gq_quant_error(plan.handle, w, 0, g[w], None, out)
+                    o = out.cpu().tolist()
+                    e += o[0]
+                    uu += o[1]
+                sid = G.SCHEMES[scheme]
+                bpe = bytes_per_worker_elem(sid, levels, d, W, False, True)
+                if d > 512:  # encode per worker + decode over the messages
+                    bpe += ((levels - 1).bit_length() / 8.0 + 4.0 * (levels if sid == 4 else 1) / d)
+                rows.append({"scheme": "%s-%d" % (scheme, levels), "bucket": d, "ms_per_step": round(ms, 4),
+                             "elem_per_s": W * n / (ms / 1000.0), "bytes_per_worker_elem": round(bpe, 4),
+                             "pct_hbm_peak": round(100.0 * bpe * W * n / (ms / 1000.0) / 1e9 / peak, 2),
+                             "normalised_variance": e / uu})
+                del msgs
+    print(json.dumps({"metric": "bucket-size sweep: throughput and normalised quantization variance",
+                      "workload": "mixture100m: %d fp32 elements x W=%d, error feedback off" % (n, W),
+                      "steps": args.steps, "warmup": args.warmup, "data": "synthetic", "sweep": rows}))
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_gq(args)
 
 

@@ -17,6 +17,7 @@ struct gq_plan {
     size_t msg_bytes, codes_off, levels_off;
     int device;
     unsigned int *status;  // device word
+    double *err_scratch;   // gq_quant_error: per-bucket sums and first-pass rows
 };
 
 namespace {
@@ -155,9 +156,13 @@ gq_status_t gq_plan_create(const gq_config_t *cfg, gq_plan_t *out)
     pl->tail = c.n > 0 ? (int)(c.n - (pl->nb - 1) * c.bucket) : 0;
     layout(c, &pl->msg_bytes, &pl->codes_off, &pl->levels_off);
     pl->status = nullptr;
+    pl->err_scratch = nullptr;
+    const size_t err_bytes = (size_t)gq::err_scratch_doubles(pl->nb) * sizeof(double);
     if (cudaGetDevice(&pl->device) != cudaSuccess || cudaMalloc(&pl->status, sizeof(unsigned int)) != cudaSuccess ||
-        cudaMemset(pl->status, 0, sizeof(unsigned int)) != cudaSuccess) {
+        cudaMemset(pl->status, 0, sizeof(unsigned int)) != cudaSuccess ||
+        (err_bytes && cudaMalloc(&pl->err_scratch, err_bytes) != cudaSuccess)) {
         if (pl->status) cudaFree(pl->status);
+        if (pl->err_scratch) cudaFree(pl->err_scratch);
         delete pl;
         return GQ_ERR_CUDA;
     }
@@ -168,7 +173,11 @@ gq_status_t gq_plan_create(const gq_config_t *cfg, gq_plan_t *out)
 gq_status_t gq_plan_destroy(gq_plan_t plan)
 {
     if (!plan) return GQ_ERR_INVALID;
-    const cudaError_t e = cudaFree(plan->status);
+    cudaError_t e = cudaFree(plan->status);
+    if (plan->err_scratch) {
+        const cudaError_t e2 = cudaFree(plan->err_scratch);
+        if (e == cudaSuccess) e = e2;
+    }
     delete plan;
     return from_cuda(e);
 }
@@ -255,6 +264,27 @@ gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *gra
     for (int w = 0; w < W; ++w) p.msg[w] = static_cast<unsigned char *>(msgs[w]);
     p.avg = avg;
     return from_cuda(gq::launch_decode(p, s));
+}
+
+gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, const float *residual,
+                           double *out, void *stream)
+{
+    if (!plan || !out) return GQ_ERR_INVALID;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (plan->cfg.n == 0) return from_cuda(cudaMemsetAsync(out, 0, 3 * sizeof(double), s));
+    if (!grad || !aligned16(grad)) return GQ_ERR_INVALID;
+    if ((plan->cfg.error_feedback != 0) != (residual != nullptr)) return GQ_ERR_INVALID;
+    if (residual && !aligned16(residual)) return GQ_ERR_INVALID;
+    gq_status_t st = check_device(*plan);
+    if (st != GQ_OK) return st;
+    gq::KParams p = base_params(*plan, step);
+    p.worker0 = worker;
+    p.g[0] = grad;
+    p.r[0] = const_cast<float *>(residual);  // read only in this mode
+    double *part = plan->err_scratch;
+    cudaError_t e = plan->cfg.bucket <= 512 ? gq::launch_warp_err(p, part, s) : gq::launch_cta_err(p, part, s);
+    if (e != cudaSuccess) return GQ_ERR_CUDA;
+    return from_cuda(gq::launch_err_reduce(part, plan->nb, part + 3 * plan->nb, out, s));
 }
 
 gq_status_t gq_plan_status(gq_plan_t plan, void *stream)

@@ -25,6 +25,7 @@ struct alignas(16) CtaShared {
     float redf[2][kCtaWarps];
     long long redl[3][kCtaWarps];
     double redd[kCtaWarps];
+    double rede[3][kCtaWarps];
     int redi[kCtaWarps];
     unsigned long long cs1[64], cs2[64];  // block histogram: sum of positions, of squares
     unsigned int ccnt[64];                // block histogram: count
@@ -113,8 +114,9 @@ __device__ __forceinline__ void flush_hist(uint32_t *hist, CtaShared &sh, int la
     __syncwarp();
 }
 
-template <int SCHEME>
-__global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KParams p)
+// ERR: the error mode of gq_quant_error; nothing is written but part[3 * bucket + k].
+template <int SCHEME, bool ERR>
+__global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KParams p, double *part)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ CtaShared sh;
@@ -140,6 +142,7 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
     const uint32_t worker = p.worker0;
     const int nchunks = d >> 7;
 
+    ErrAcc ea{0.0, 0.0, 0.0};
     for (int64_t beta = blockIdx.x; beta < p.nb; beta += gridDim.x) {
         const int64_t base = beta * (int64_t)d;
         const int nvalid = (beta == p.nb - 1) ? p.tail : d;
@@ -530,7 +533,19 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
             float *rout = r ? r + base + 128 * ch : nullptr;
             uint32_t *cwc = cw ? cw + ch * 4 * p.bits : nullptr;
             float q[4];
-            if constexpr (SCHEME == GQ_QSGD) {
+            if constexpr (ERR) {
+                if constexpr (SCHEME == GQ_QSGD) {
+                    err_chunk<true, false>(p, rq, blk, worker, lane, valid, u4, pos4, ea);
+                } else if constexpr (SCHEME == GQ_ORQ) {
+                    if (constant) err_chunk<false, false>(p, RoundConst{mn}, blk, worker, lane, valid, u4, pos4, ea);
+                    else err_chunk<true, false>(p, ro, blk, worker, lane, valid, u4, pos4, ea);
+                } else if constexpr (SCHEME == GQ_BINGRAD_PB) {
+                    if (constant) err_chunk<false, false>(p, RoundConst{mn}, blk, worker, lane, valid, u4, pos4, ea);
+                    else err_chunk<true, false>(p, rp, blk, worker, lane, valid, u4, pos4, ea);
+                } else {
+                    err_chunk<false, false>(p, rb, blk, worker, lane, valid, u4, pos4, ea);
+                }
+            } else if constexpr (SCHEME == GQ_QSGD) {
                 round_chunk<true, false, 0>(p, rq, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             } else if constexpr (SCHEME == GQ_ORQ) {
                 if (constant)
@@ -546,6 +561,22 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                 round_chunk<false, false, 0>(p, rb, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             }
         }
+        if constexpr (ERR) {
+            // bucket sums: warps in a fixed butterfly, then warp 0 .. 7 in order
+            ea = warp_sum_err(ea);
+            if (lane == 0) {
+                sh.rede[0][wid] = ea.e;
+                sh.rede[1][wid] = ea.uu;
+                sh.rede[2][wid] = ea.qq;
+            }
+            __syncthreads();
+            if (tid < 3) {
+                double t = 0.0;
+                for (int k = 0; k < kCtaWarps; ++k) t = __dadd_rn(t, sh.rede[tid][k]);
+                part[3 * beta + tid] = t;
+            }
+            ea = ErrAcc{0.0, 0.0, 0.0};
+        }
         // ---- level table --------------------------------------------------------------------------
         if (msg && tid < p.L) {
             float lv;
@@ -559,10 +590,10 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
     }
 }
 
-template <int SCHEME>
-cudaError_t launch(const KParams &p, cudaStream_t stream)
+template <int SCHEME, bool ERR>
+cudaError_t launch(const KParams &p, double *part, cudaStream_t stream)
 {
-    auto kern = k_cta<SCHEME>;
+    auto kern = k_cta<SCHEME, ERR>;
     const size_t smem = (size_t)p.d * 4 + (SCHEME == GQ_ORQ ? (size_t)kCtaWarps * 64 * 32 * 4 : 0);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -574,21 +605,26 @@ cudaError_t launch(const KParams &p, cudaStream_t stream)
     const int64_t cap = (int64_t)sms * per_sm;
     const int grid = (int)(p.nb < cap ? p.nb : cap);
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kCtaThreads, smem, stream>>>(p);
+    kern<<<grid, kCtaThreads, smem, stream>>>(p, part);
     return cudaGetLastError();
+}
+
+template <bool ERR>
+cudaError_t dispatch(const KParams &p, double *part, cudaStream_t stream)
+{
+    switch (p.scheme) {
+    case GQ_QSGD:
+    case GQ_TERNGRAD: return launch<GQ_QSGD, ERR>(p, part, stream);
+    case GQ_BINGRAD_B: return launch<GQ_BINGRAD_B, ERR>(p, part, stream);
+    case GQ_BINGRAD_PB: return launch<GQ_BINGRAD_PB, ERR>(p, part, stream);
+    default: return launch<GQ_ORQ, ERR>(p, part, stream);
+    }
 }
 
 }  // namespace
 
-cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream)
-{
-    switch (p.scheme) {
-    case GQ_QSGD:
-    case GQ_TERNGRAD: return launch<GQ_QSGD>(p, stream);
-    case GQ_BINGRAD_B: return launch<GQ_BINGRAD_B>(p, stream);
-    case GQ_BINGRAD_PB: return launch<GQ_BINGRAD_PB>(p, stream);
-    default: return launch<GQ_ORQ>(p, stream);
-    }
-}
+cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream) { return dispatch<false>(p, nullptr, stream); }
+
+cudaError_t launch_cta_err(const KParams &p, double *part, cudaStream_t stream) { return dispatch<true>(p, part, stream); }
 
 }  // namespace gq

@@ -51,4 +51,12 @@ cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream);
 // Dequantize + aggregate for any d.
 cudaError_t launch_decode(const KParams &p, cudaStream_t stream);
 
+// gq_quant_error: per-bucket binary64 error sums into part[3 * bucket + k] (one worker, nothing
+// else written), then their fixed-order reduction into out[3].  The scratch holds
+// err_scratch_doubles(nb) doubles: the nb bucket rows followed by the rows of the first pass.
+cudaError_t launch_warp_err(const KParams &p, double *part, cudaStream_t stream);
+cudaError_t launch_cta_err(const KParams &p, double *part, cudaStream_t stream);
+int64_t err_scratch_doubles(int64_t nb);
+cudaError_t launch_err_reduce(const double *part, int64_t nb, double *tmp, double *out, cudaStream_t stream);
+
 }  // namespace gq

@@ -26,6 +26,14 @@ struct RoundQSGD {
         code = k + (up ? 1 : 0);
         q = up ? lp.y : lp.x;
     }
+    __device__ __forceinline__ void bracket(float u, int, float &lo, float &hi, float &pu) const
+    {
+        const float y = __fmul_rn(__fadd_rn(__fmul_rn(u, inv_m), 1.0f), h);
+        const int k = min(max(__float2int_rz(y), 0), kmax);
+        pu = __fsub_rn(y, (float)k);
+        lo = pair[k].x;
+        hi = pair[k].y;
+    }
 };
 
 // ORQ: the bracket of the value's grid cell (the cell is passed in place of the position),
@@ -41,6 +49,13 @@ struct RoundORQ {
         code = __float_as_int(b.w) + (up ? 1 : 0);
         q = up ? b.y : b.x;
     }
+    __device__ __forceinline__ void bracket(float u, int cell, float &lo, float &hi, float &pu) const
+    {
+        const float4 b = ctab[cell];
+        lo = b.x;
+        hi = b.y;
+        pu = __fmul_rn(__fsub_rn(u, b.x), b.z);
+    }
 };
 
 // Constant bucket: one level, code 0.
@@ -50,6 +65,12 @@ struct RoundConst {
     {
         code = 0;
         q = lv;
+    }
+    __device__ __forceinline__ void bracket(float, int, float &lo, float &hi, float &pu) const
+    {
+        lo = lv;
+        hi = lv;
+        pu = 0.0f;
     }
 };
 
@@ -62,6 +83,12 @@ struct RoundB {
         const bool up = split && u >= thr;
         code = up ? 1 : 0;
         q = up ? b : a;
+    }
+    __device__ __forceinline__ void bracket(float u, int, float &lo, float &hi, float &pu) const
+    {
+        lo = a;
+        hi = b;
+        pu = (split && u >= thr) ? 1.0f : 0.0f;
     }
 };
 
@@ -77,6 +104,14 @@ struct RoundPB {
         else up = unit_float(word) < __fmul_rn(__fsub_rn(u, a), rinv);
         code = up ? 1 : 0;
         q = up ? b : a;
+    }
+    __device__ __forceinline__ void bracket(float u, int pos, float &lo, float &hi, float &pu) const
+    {
+        lo = a;
+        hi = b;
+        if (pos < pa) pu = 0.0f;
+        else if (pos >= pb) pu = 1.0f;
+        else pu = __fmul_rn(__fsub_rn(u, a), rinv);
     }
 };
 
@@ -125,6 +160,48 @@ __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uin
             }
         }
     }
+}
+
+// Running binary64 sums of the quantization error (see gq_quant_error): expected squared
+// rounding error p (b-u)^2 + (1-p) (a-u)^2, u^2, realised (Q(u)-u)^2.
+struct ErrAcc {
+    double e, uu, qq;
+};
+
+template <bool RANDOM, bool ALLVALID, class R>
+__device__ __forceinline__ void err_chunk(const KParams &p, const R &rule, uint64_t blk, uint32_t worker, int lane,
+                                          uint32_t valid, const float (&u)[4], const int (&pos)[4], ErrAcc &ea)
+{
+    uint4 rnd = make_uint4(0u, 0u, 0u, 0u);
+    if (RANDOM) rnd = draws4(p, blk + (uint64_t)lane, worker);
+    const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        if (ALLVALID || ((valid >> c) & 1u)) {
+            float lo, hi, pu, q;
+            int code;
+            rule.bracket(u[c], pos[c], lo, hi, pu);
+            rule.round(u[c], pos[c], words[c], code, q);
+            const double P = (double)sat01(pu);
+            const double du = (double)u[c];
+            const double dh = __dsub_rn((double)hi, du), dl = __dsub_rn((double)lo, du), dq = __dsub_rn((double)q, du);
+            ea.e = __dadd_rn(ea.e, __dadd_rn(__dmul_rn(__dmul_rn(P, dh), dh), __dmul_rn(__dmul_rn(__dsub_rn(1.0, P), dl), dl)));
+            ea.uu = __dadd_rn(ea.uu, __dmul_rn(du, du));
+            ea.qq = __dadd_rn(ea.qq, __dmul_rn(dq, dq));
+        }
+    }
+}
+
+// Warp sum of an ErrAcc in a fixed butterfly order (every lane gets the same bits).
+__device__ __forceinline__ ErrAcc warp_sum_err(ErrAcc a)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a.e = __dadd_rn(a.e, __shfl_xor_sync(kFull, a.e, o));
+        a.uu = __dadd_rn(a.uu, __shfl_xor_sync(kFull, a.uu, o));
+        a.qq = __dadd_rn(a.qq, __shfl_xor_sync(kFull, a.qq, o));
+    }
+    return a;
 }
 
 }  // namespace gq

@@ -6,6 +6,9 @@ namespace gq {
 cudaError_t launch_warp_orq(const KParams &p, bool fused, cudaStream_t stream);
 cudaError_t launch_warp_qsgd(const KParams &p, bool fused, cudaStream_t stream);
 cudaError_t launch_warp_bingrad(const KParams &p, bool fused, cudaStream_t stream);
+cudaError_t launch_warp_err_orq(const KParams &p, double *part, cudaStream_t stream);
+cudaError_t launch_warp_err_qsgd(const KParams &p, double *part, cudaStream_t stream);
+cudaError_t launch_warp_err_bingrad(const KParams &p, double *part, cudaStream_t stream);
 
 cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream)
 {
@@ -15,6 +18,17 @@ cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream
     case GQ_BINGRAD_B:
     case GQ_BINGRAD_PB: return launch_warp_bingrad(p, fused, stream);
     default: return launch_warp_orq(p, fused, stream);
+    }
+}
+
+cudaError_t launch_warp_err(const KParams &p, double *part, cudaStream_t stream)
+{
+    switch (p.scheme) {
+    case GQ_QSGD:
+    case GQ_TERNGRAD: return launch_warp_err_qsgd(p, part, stream);
+    case GQ_BINGRAD_B:
+    case GQ_BINGRAD_PB: return launch_warp_err_bingrad(p, part, stream);
+    default: return launch_warp_err_orq(p, part, stream);
     }
 }
 

@@ -79,12 +79,26 @@ __device__ __forceinline__ int slot_elem(int t, int lane) { return 128 * (t >> 2
 // ---------------------------------------------------------------------------------------------
 // Round + pack + residual + accumulate for one worker-bucket, chunk by chunk.
 // ---------------------------------------------------------------------------------------------
+// BITS < 0 selects the error mode of gq_quant_error: nothing is written, the error terms of
+// the bucket's elements are added to *ea.
 template <int EPL, bool FUSED, bool RANDOM, bool TAIL, int BITS, class R>
 __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t beta, int w, int lane, uint32_t vmask,
                                      const float (&v)[EPL], const float (&u)[EPL], const int (&pos)[EPL],
-                                     float (&acc)[EPL])
+                                     float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
     const int64_t base = beta * (int64_t)(32 * EPL);
+    if constexpr (BITS < 0) {
+        const uint32_t worker = p.worker0 + (uint32_t)w;
+#pragma unroll
+        for (int m = 0; m < EPL / 4; ++m) {
+            const float uu[4] = {u[4 * m], u[4 * m + 1], u[4 * m + 2], u[4 * m + 3]};
+            const int pp[4] = {pos[4 * m], pos[4 * m + 1], pos[4 * m + 2], pos[4 * m + 3]};
+            const uint32_t valid = TAIL ? (vmask >> (4 * m)) & 0xfu : 0xfu;
+            err_chunk<RANDOM, !TAIL>(p, rule, (uint64_t)(base >> 2) + (uint64_t)(32 * m), worker, lane, valid, uu, pp,
+                                     *ea);
+        }
+        return;
+    }
     float *r = p.r[w];
     unsigned char *msg = p.msg[w];
     uint32_t *cw = msg ? reinterpret_cast<uint32_t *>(msg) + beta * p.codes_words : nullptr;
@@ -123,7 +137,7 @@ __device__ __forceinline__ void flag_nonfinite(const KParams &p, int lane)
 // ---------------------------------------------------------------------------------------------
 template <int EPL, bool FUSED, bool TAIL, int BITS>
 __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
-                         const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
+                         const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
     float m = 0.0f;
 #pragma unroll
@@ -145,13 +159,13 @@ __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int
     int pos[EPL];
 #pragma unroll
     for (int t = 0; t < EPL; ++t) pos[t] = 0;
-    emit<EPL, FUSED, true, TAIL, BITS>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
+    emit<EPL, FUSED, true, TAIL, BITS>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
     store_table(p, w, beta, lane, m);
 }
 
 template <int EPL, bool FUSED, bool TAIL, int BITS>
 __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
-                        const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
+                        const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
@@ -169,7 +183,7 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     if (!(mx > mn)) {  // constant bucket (or NaN): one level, code 0
 #pragma unroll
         for (int t = 0; t < EPL; ++t) pos[t] = 0;
-        emit<EPL, FUSED, false, TAIL, BITS>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc);
+        emit<EPL, FUSED, false, TAIL, BITS>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc, ea);
         store_table(p, w, beta, lane, mn);
         return;
     }
@@ -242,7 +256,7 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
         if (mtab && ((mask >> j) & 1ull)) mtab[__popcll(mask & ((1ull << j) - 1ull))] = grid_point(mn, mx, step, j);
     }
     __syncwarp();
-    emit<EPL, FUSED, true, TAIL, BITS>(p, RoundORQ{sm.ctab}, beta, w, lane, vmask, v, u, pos, acc);
+    emit<EPL, FUSED, true, TAIL, BITS>(p, RoundORQ{sm.ctab}, beta, w, lane, vmask, v, u, pos, acc, ea);
     __syncwarp();
 }
 
@@ -283,7 +297,7 @@ __device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
 
 template <int EPL, bool FUSED, bool TAIL, int BITS>
 __device__ void fit_bingrad_b(const KParams &p, FitB &, int64_t beta, int w, int lane, uint32_t vmask, bool check,
-                              int nvalid, const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
+                              int nvalid, const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
     float m = 0.0f;
 #pragma unroll
@@ -366,13 +380,13 @@ __device__ void fit_bingrad_b(const KParams &p, FitB &, int64_t beta, int w, int
             rule = RoundB{a, b, tv, true};
         }
     }
-    emit<EPL, FUSED, false, TAIL, BITS>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
+    emit<EPL, FUSED, false, TAIL, BITS>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
     store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
 }
 
 template <int EPL, bool FUSED, bool TAIL, int BITS>
 __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
-                               const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL])
+                               const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
@@ -390,7 +404,7 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
     if (!(mx > mn)) {
 #pragma unroll
         for (int t = 0; t < EPL; ++t) pos[t] = 0;
-        emit<EPL, FUSED, false, TAIL, BITS>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc);
+        emit<EPL, FUSED, false, TAIL, BITS>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc, ea);
         store_table(p, w, beta, lane, mn);
         return;
     }
@@ -478,7 +492,7 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
     rule.rinv = __frcp_rn(__fsub_rn(rule.b, rule.a));
     rule.pa = A << kPbFBits;
     rule.pb = B << kPbFBits;
-    emit<EPL, FUSED, true, TAIL, BITS>(p, rule, beta, w, lane, vmask, v, u, pos, acc);
+    emit<EPL, FUSED, true, TAIL, BITS>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
     store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
 }
 
@@ -487,7 +501,8 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
 // ---------------------------------------------------------------------------------------------
 template <int EPL, int SCHEME, bool FUSED, bool TAIL, int BITS>
 __device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME>::type &fit, int64_t beta, int w,
-                                        int lane, int nvalid, uint32_t vmask, const float (&v)[EPL], float (&acc)[EPL])
+                                        int lane, int nvalid, uint32_t vmask, const float (&v)[EPL], float (&acc)[EPL],
+                                        ErrAcc *ea = nullptr)
 {
     float u[EPL];
     bool check = true;  // the fit flags non-finite values unless the clip pass already did
@@ -527,13 +542,13 @@ __device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME
         for (int t = 0; t < EPL; ++t) u[t] = v[t];
     }
     if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD)
-        fit_qsgd<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, v, u, acc);
+        fit_qsgd<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
     else if constexpr (SCHEME == GQ_ORQ)
-        fit_orq<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, v, u, acc);
+        fit_orq<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
     else if constexpr (SCHEME == GQ_BINGRAD_B)
-        fit_bingrad_b<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, nvalid, v, u, acc);
+        fit_bingrad_b<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, nvalid, v, u, acc, ea);
     else
-        fit_bingrad_pb<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, v, u, acc);
+        fit_bingrad_pb<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -670,6 +685,95 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME, kW
         } else {
             ++w;
         }
+    }
+}
+
+// gq_quant_error: one warp per bucket, grid-stride, plain 16-byte loads; the bucket's three
+// error sums (fixed summation order) go to part[3 * bucket + k].
+template <int EPL, int SCHEME>
+__global__ void __launch_bounds__(kWarpsPerCta * 32) k_warp_err(const __grid_constant__ KParams p, double *part)
+{
+    using Fit = typename FitFor<SCHEME>::type;
+    constexpr int D = 32 * EPL;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    Fit &fit = reinterpret_cast<Fit *>(smem_raw)[wib];
+    init_fit<SCHEME>(fit, lane);
+    __syncwarp();
+    const float *g = p.g[0];
+    const float *r = p.r[0];
+    float acc[EPL];
+    for (int64_t beta = (int64_t)blockIdx.x * kWarpsPerCta + wib; beta < p.nb; beta += (int64_t)gridDim.x * kWarpsPerCta) {
+        const int nvalid = beta == p.nb - 1 ? p.tail : D;
+        const float *gb = g + beta * D;
+        const float *rb = r ? r + beta * D : nullptr;
+        float v[EPL];
+        ErrAcc ea{0.0, 0.0, 0.0};
+        if (nvalid == D) {
+#pragma unroll
+            for (int m = 0; m < EPL / 4; ++m) {
+                float4 x = __ldg(reinterpret_cast<const float4 *>(gb + 128 * m + 4 * lane));
+                if (rb) {
+                    const float4 y = __ldg(reinterpret_cast<const float4 *>(rb + 128 * m + 4 * lane));
+                    x = make_float4(__fadd_rn(x.x, y.x), __fadd_rn(x.y, y.y), __fadd_rn(x.z, y.z), __fadd_rn(x.w, y.w));
+                }
+                v[4 * m + 0] = x.x;
+                v[4 * m + 1] = x.y;
+                v[4 * m + 2] = x.z;
+                v[4 * m + 3] = x.w;
+            }
+            process<EPL, SCHEME, false, false, -1>(p, fit, beta, 0, lane, D, 0xffffffffu, v, acc, &ea);
+        } else {
+            uint32_t vmask = 0;
+#pragma unroll
+            for (int t = 0; t < EPL; ++t) {
+                const int e = slot_elem(t, lane);
+                float x = 0.0f;
+                if (e < nvalid) {
+                    vmask |= 1u << t;
+                    x = gb[e];
+                    if (rb) x = __fadd_rn(x, rb[e]);
+                }
+                v[t] = x;
+            }
+            process<EPL, SCHEME, false, true, -1>(p, fit, beta, 0, lane, nvalid, vmask, v, acc, &ea);
+        }
+        ea = warp_sum_err(ea);
+        if (lane == 0) {
+            part[3 * beta + 0] = ea.e;
+            part[3 * beta + 1] = ea.uu;
+            part[3 * beta + 2] = ea.qq;
+        }
+        __syncwarp();
+    }
+}
+
+template <int EPL, int SCHEME>
+cudaError_t launch_err(const KParams &p, double *part, cudaStream_t stream)
+{
+    using Fit = typename FitFor<SCHEME>::type;
+    auto kern = k_warp_err<EPL, SCHEME>;
+    const size_t smem = sizeof(Fit) * kWarpsPerCta;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarpsPerCta * 32, smem);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t need = (p.nb + kWarpsPerCta - 1) / kWarpsPerCta;
+    const int64_t cap = (int64_t)sms * per_sm;
+    kern<<<(int)(need < cap ? need : cap), kWarpsPerCta * 32, smem, stream>>>(p, part);
+    return cudaGetLastError();
+}
+
+template <int SCHEME>
+cudaError_t warp_dispatch_err(const KParams &p, double *part, cudaStream_t stream)
+{
+    switch (p.d) {
+    case 128: return launch_err<4, SCHEME>(p, part, stream);
+    case 256: return launch_err<8, SCHEME>(p, part, stream);
+    default: return launch_err<16, SCHEME>(p, part, stream);
     }
 }
 

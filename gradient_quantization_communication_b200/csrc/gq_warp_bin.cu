@@ -9,4 +9,10 @@ cudaError_t launch_warp_bingrad(const KParams &p, bool fused, cudaStream_t strea
                                     : warp_dispatch<GQ_BINGRAD_PB>(p, fused, stream);
 }
 
+cudaError_t launch_warp_err_bingrad(const KParams &p, double *part, cudaStream_t stream)
+{
+    return p.scheme == GQ_BINGRAD_B ? warp_dispatch_err<GQ_BINGRAD_B>(p, part, stream)
+                                    : warp_dispatch_err<GQ_BINGRAD_PB>(p, part, stream);
+}
+
 }  // namespace gq

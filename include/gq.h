@@ -109,9 +109,9 @@ GQ_API gq_status_t gq_config_check(const gq_config_t *cfg);
  */
 GQ_API gq_status_t gq_message_layout(const gq_config_t *cfg, size_t *bytes, size_t *codes_off, size_t *levels_off);
 
-/* Create a plan: validates cfg, selects kernels and allocates the plan's 4-byte device status
- * word on the current device (the only device allocation the library makes).  The plan must
- * be used on that device only. */
+/* Create a plan: validates cfg, selects kernels and allocates on the current device the plan's
+ * 4-byte status word and the scratch of gq_quant_error (the only device allocations the library
+ * makes).  The plan must be used on that device only. */
 GQ_API gq_status_t gq_plan_create(const gq_config_t *cfg, gq_plan_t *out);
 /* Free the plan (synchronous; the caller must make sure no work of the plan is pending). */
 GQ_API gq_status_t gq_plan_destroy(gq_plan_t plan);
@@ -150,6 +150,22 @@ GQ_API gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs,
  */
 GQ_API gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *grads, float *const *residuals,
                           void *const *msgs, float *avg, void *stream);
+
+/*
+ * Quantization error of one worker's gradient, for measuring how much a fit loses (the
+ * expected quantization variance the review's ORQ minimises, section "Proposed method").  The
+ * fit and the rounding are those of gq_encode (same worker, step and draws); nothing but `out`
+ * is written and the residual is only read.
+ *   out   device, 3 doubles: out[0] = sum over elements of the expected squared rounding error
+ *         p (b - u)^2 + (1 - p) (a - u)^2 given the fitted levels (u the value quantized after
+ *         clipping, [a, b] its bracket, p its probability of rounding up; (b - u)(u - a) for
+ *         unbiased rounding), out[1] = sum of u^2, out[2] = sum of (Q(u) - u)^2 for this
+ *         step's draws.  Binary64; each bucket's sums are reduced in a fixed order, so the
+ *         result does not depend on the launch shape.
+ * Uses the plan's error scratch of 24 * (ceil(n/d) + ceil(ceil(n/d) / 4096)) bytes.
+ */
+GQ_API gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad,
+                                  const float *residual, double *out, void *stream);
 
 /* Synchronize `stream`, then report and clear the plan's status flags: GQ_ERR_NONFINITE if
  * a non-finite input was seen since the last call, GQ_ERR_CUDA if the stream failed. */
