@@ -51,12 +51,14 @@ def lib():
         L.gq_fused_step.argtypes = [vp, ctypes.c_uint64, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                     ctypes.POINTER(vp), vp, vp]
         L.gq_quant_error.argtypes = [vp, ctypes.c_uint32, ctypes.c_uint64, vp, vp, vp, vp]
+        L.gq_quant_error_noalloc.argtypes = [cfgp, ctypes.c_uint32, ctypes.c_uint64, vp, vp, vp, vp]
         L.gq_plan_status.argtypes = [vp, vp]
         L.gq_status_string.argtypes = [ctypes.c_int]
         L.gq_status_string.restype = ctypes.c_char_p
         L.gq_version.restype = ctypes.c_char_p
         for f in ("gq_config_check", "gq_message_layout", "gq_plan_create", "gq_plan_destroy", "gq_encode",
-                  "gq_decode_accumulate", "gq_fused_step", "gq_quant_error", "gq_plan_status"):
+                  "gq_decode_accumulate", "gq_fused_step", "gq_quant_error", "gq_quant_error_noalloc",
+                  "gq_plan_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -140,6 +142,11 @@ def gq_fused_step(plan, step, grads, residuals, msgs, avg, stream=None):
 def gq_quant_error(plan, worker, step, grad, residual, out, stream=None):
     _check(lib().gq_quant_error(plan, worker, step, _ptr(grad), _ptr(residual), _ptr(out), _stream(stream)),
            "gq_quant_error")
+
+
+def gq_quant_error_noalloc(cfg, worker, step, grad, residual, out, stream=None):
+    _check(lib().gq_quant_error_noalloc(ctypes.byref(cfg), worker, step, _ptr(grad), _ptr(residual), _ptr(out),
+                                        _stream(stream)), "gq_quant_error_noalloc")
 
 
 def gq_plan_status(plan, stream=None):

@@ -167,6 +167,29 @@ GQ_API gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *con
 GQ_API gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad,
                                   const float *residual, double *out, void *stream);
 
+/*
+ * Allocation-free variant of gq_quant_error.  There is no counterpart in the paper: this entry
+ * point exists for callers that cannot call cudaMalloc -- code running inside a framework's
+ * caching allocator or memory pool (which must not be re-entered), processes whose device
+ * memory is reserved up front, plugins that are handed buffers but no allocator.  Such callers
+ * cannot create a plan (gq_plan_create allocates), so this call takes the configuration and
+ * computes exactly what gq_quant_error computes for it (cfg->workers is ignored).
+ * Its scratch is a file-scope device array of the library, GQ_NOALLOC_SCRATCH_BYTES (about
+ * 384 KB), held on every device that loads the library until the process exits.  Hence:
+ *   - the input may span at most GQ_NOALLOC_MAX_BUCKETS buckets (ceil(n/d) <= 16384); larger
+ *     inputs return GQ_ERR_UNSUPPORTED before anything is enqueued;
+ *   - every call on a device shares that scratch and leaves its contents behind; calls whose
+ *     work overlaps on the GPU (different streams or host threads) race;
+ *   - non-finite input is not reported (there is no plan status word to read it from);
+ *   - the first call on each device looks up the scratch address (cudaGetSymbolAddress);
+ *     make that first call before any stream capture.
+ * Allocates nothing, on the device or on the host.
+ */
+#define GQ_NOALLOC_MAX_BUCKETS 16384
+#define GQ_NOALLOC_SCRATCH_BYTES (256 + 24 * (GQ_NOALLOC_MAX_BUCKETS + (GQ_NOALLOC_MAX_BUCKETS + 4095) / 4096))
+GQ_API gq_status_t gq_quant_error_noalloc(const gq_config_t *cfg, uint32_t worker, uint64_t step, const float *grad,
+                                          const float *residual, double *out, void *stream);
+
 /* Synchronize `stream`, then report and clear the plan's status flags: GQ_ERR_NONFINITE if
  * a non-finite input was seen since the last call, GQ_ERR_CUDA if the stream failed. */
 GQ_API gq_status_t gq_plan_status(gq_plan_t plan, void *stream);
