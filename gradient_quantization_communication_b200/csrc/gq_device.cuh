@@ -109,6 +109,20 @@ __device__ __forceinline__ float fmin_nan(float a, float b)
     return r;
 }
 
+// Three-operand forms (one instruction each on sm_100).
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float fmin3_nan(float a, float b, float c)
+{
+    float r;
+    asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Round to nearest even, float64 -> int64.
 __device__ __forceinline__ long long fixed_point(float x, double scale)
 {
@@ -226,22 +240,29 @@ __device__ __forceinline__ unsigned long long orq_delta(int A, int C, int B, int
 }
 
 // Incremental form: lane l owns candidates C = l and l + 32 with their current neighbours and
-// Delta in registers; after a level L is added only the candidates of the bracket it split
-// are re-evaluated (skipped warp-wide when no lane has one).
+// ranking key (Delta << 6 | 63 - C: the largest key has the largest Delta, ties to the smallest
+// C; 0 for an index that is chosen or never a candidate) in registers; after a level L is added
+// only the candidates of the bracket it split are re-evaluated (skipped warp-wide when no lane
+// has one).
+template <class T>
+__device__ __forceinline__ unsigned long long orq_key(int A, int C, int B, int P0A, int P0C, int P0B, T P1A, T P1C,
+                                                      T P1B)
+{
+    return (orq_delta(A, C, B, P0A, P0C, P0B, P1A, P1C, P1B) << 6) | (unsigned long long)(63 - C);
+}
+
 template <class T>
 __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T *P1, int s, int lane)
 {
     unsigned long long mask = 1ull | (1ull << 63);
     int A[2], B[2], P0A[2], P0B[2], P0C[2];
     T P1A[2], P1B[2], P1C[2];
-    unsigned long long delta[2];
-    bool live[2];
+    unsigned long long key[2];
     const int P0lo = P0[0], P0hi = P0[63];
     const T P1lo = P1[0], P1hi = P1[63];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int C = lane + 32 * h;
-        live[h] = C >= 1 && C <= 62;
         A[h] = 0;
         B[h] = 63;
         P0A[h] = P0lo;
@@ -250,15 +271,10 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T 
         P1B[h] = P1hi;
         P0C[h] = P0[C];
         P1C[h] = P1[C];
-        delta[h] = orq_delta(0, C, 63, P0lo, P0C[h], P0hi, P1lo, P1C[h], P1hi);
+        key[h] = (C >= 1 && C <= 62) ? orq_key(0, C, 63, P0lo, P0C[h], P0hi, P1lo, P1C[h], P1hi) : 0ull;
     }
     for (int round = 0; round < s - 2; ++round) {
-        unsigned long long best = 0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const unsigned long long key = (delta[h] << 6) | (unsigned long long)(63 - lane - 32 * h);
-            if (live[h]) best = key > best ? key : best;
-        }
+        const unsigned long long best = key[0] > key[1] ? key[0] : key[1];
         // warp argmax of the 64-bit key: high words first, then low words among the lanes that tie
         const unsigned hi = __reduce_max_sync(kFull, (unsigned)(best >> 32));
         const unsigned lo = __reduce_max_sync(kFull, (unsigned)(best >> 32) == hi ? (unsigned)best : 0u);
@@ -270,8 +286,8 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T 
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int C = lane + 32 * h;
-            if (C == L) live[h] = false;
-            const bool split = live[h] && A[h] < L && L < B[h];
+            if (C == L) key[h] = 0ull;
+            const bool split = key[h] != 0ull && A[h] < L && L < B[h];
             if (__any_sync(kFull, split)) {
                 if (split) {
                     if (L < C) {
@@ -283,7 +299,7 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T 
                         P0B[h] = P0L;
                         P1B[h] = P1L;
                     }
-                    delta[h] = orq_delta(A[h], C, B[h], P0A[h], P0C[h], P0B[h], P1A[h], P1C[h], P1B[h]);
+                    key[h] = orq_key(A[h], C, B[h], P0A[h], P0C[h], P0B[h], P1A[h], P1C[h], P1B[h]);
                 }
             }
         }

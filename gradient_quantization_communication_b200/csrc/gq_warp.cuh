@@ -43,10 +43,15 @@ struct alignas(16) StageBuf {
     float r[32 * EPL];
 };
 
+// ORQ histogram word of one (cell, column): count << kHistCountShift | sum of 16-bit fractions.
+// A column collects at most 4 lanes x 16 values = 64 entries, so the fraction sum stays below
+// 64 * 2^16 = 2^22 and the count (<= 64) fits above it.
+constexpr int kHistCountShift = 22;
 struct alignas(16) FitORQ {
-    uint32_t hcnt[64 * kHistCols];  // [cell][column]: element counts
-    uint32_t hsum[64 * kHistCols];  // [cell][column]: sums of 16-bit fractions
-    float4 ctab[64];                // cell -> {lower, upper, 1/(upper-lower), bracket}
+    uint32_t hist[64 * kHistCols];  // [cell][column]; cell 63 holds the values at the top grid point
+    float4 ctab[64];                // cell -> {lower, upper, 1/(upper-lower), bracket}; 63 repeats 62
+    float4 btab[GQ_MAX_LEVELS];     // bracket k -> {level k, level k+1, 1/difference, k}
+    float lev[GQ_MAX_LEVELS];       // chosen levels in increasing order
     uint32_t P1[64];                // sum of positions over cells < k (< 2^31 for d <= 512)
     int P0[64];                     // count over cells < k
 };
@@ -132,6 +137,41 @@ __device__ __forceinline__ void flag_nonfinite(const KParams &p, int lane)
     if (lane == 0) atomicOr(p.status, kStatusNonFinite);
 }
 
+// ORQ tables from the chosen grid indices (mask, s bits): the level table of the message, the
+// bracket table (one entry per pair of adjacent levels) and the per-cell bracket table the
+// rounding pass reads (cell j lies in bracket k = #{chosen indices <= j} - 1; cell 63, the top
+// grid point, in bracket s - 2 like cell 62).
+__device__ __forceinline__ void build_orq_tables(const KParams &p, FitORQ &sm, int w, int64_t beta, int lane,
+                                                 unsigned long long mask, float mn, float mx, float step)
+{
+    const uint32_t mlo = (uint32_t)mask, mhi = (uint32_t)(mask >> 32);
+    const uint32_t lt = (1u << lane) - 1u, le = lt | (1u << lane);
+    const int nlo = __popc(mlo);
+    unsigned char *msg = p.msg[w];
+    float *mtab = msg ? reinterpret_cast<float *>(msg + p.levels_off) + beta * p.L : nullptr;
+    if ((mlo >> lane) & 1u) {
+        const float lv = grid_point(mn, mx, step, lane);
+        const int rank = __popc(mlo & lt);
+        sm.lev[rank] = lv;
+        if (mtab) mtab[rank] = lv;
+    }
+    if ((mhi >> lane) & 1u) {
+        const float lv = grid_point(mn, mx, step, lane + 32);
+        const int rank = nlo + __popc(mhi & lt);
+        sm.lev[rank] = lv;
+        if (mtab) mtab[rank] = lv;
+    }
+    __syncwarp();
+    if (lane < p.s - 1) {
+        const float lo = sm.lev[lane], hi = sm.lev[lane + 1];
+        sm.btab[lane] = make_float4(lo, hi, __frcp_rn(__fsub_rn(hi, lo)), __int_as_float(lane));
+    }
+    __syncwarp();
+    sm.ctab[lane] = sm.btab[__popc(mlo & le) - 1];
+    sm.ctab[lane + 32] = sm.btab[min(nlo + __popc(mhi & le) - 1, p.s - 2)];
+    __syncwarp();
+}
+
 // ---------------------------------------------------------------------------------------------
 // Per-scheme fits (u: the values to quantize; v: the error-fed values the residual refers to)
 // ---------------------------------------------------------------------------------------------
@@ -168,12 +208,22 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
                         const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
     float mn = INFINITY, mx = -INFINITY;
+    if (TAIL) {
 #pragma unroll
-    for (int t = 0; t < EPL; ++t)
-        if (!TAIL || ((vmask >> t) & 1u)) {
-            mn = fmin_nan(mn, u[t]);
-            mx = fmax_nan(mx, u[t]);
+        for (int t = 0; t < EPL; ++t)
+            if ((vmask >> t) & 1u) {
+                mn = fmin_nan(mn, u[t]);
+                mx = fmax_nan(mx, u[t]);
+            }
+    } else {
+        mn = fmin3_nan(u[0], u[1], u[2]);
+        mx = fmax3_nan(u[0], u[1], u[2]);
+#pragma unroll
+        for (int t = 3; t < EPL; t += 2) {
+            mn = t + 1 < EPL ? fmin3_nan(mn, u[t], u[t + 1]) : fmin_nan(mn, u[t]);
+            mx = t + 1 < EPL ? fmax3_nan(mx, u[t], u[t + 1]) : fmax_nan(mx, u[t]);
         }
+    }
     mn = warp_redux_min(mn);
     mx = warp_redux_max(mx);
     if (check && !(mn >= -FLT_MAX && mx <= FLT_MAX)) flag_nonfinite(p, lane);
@@ -190,47 +240,57 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     const float range = __fsub_rn(mx, mn);
     const float step = __fdiv_rn(range, 63.0f);
     const float scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kOrqFBits));
-    // histogram: 8 columns per cell, lane l adds into column l % 8 with shared atomics; the
-    // rounding pass needs only the cell of each value, so the cells are what is kept
+    // histogram: 8 columns per cell, lane l adds into column l % 8 with one shared atomic per
+    // value (count and fraction packed); the rounding pass needs only the cell of each value.
+    // A valid value lies in [mn, mx], so its product below is >= 0 (or NaN, which converts to
+    // 0); it exceeds 63 * 2^16 only when 63 / range overflows to +inf (a range below 63 / FLT_MAX),
+    // hence the upper clamp.  The cell is the position's integer part, 63 for the top grid point.
     const int col = lane & (kHistCols - 1);
 #pragma unroll
     for (int t = 0; t < EPL; ++t) {
-        // every valid value is finite and >= mn here, so the position is >= 0 without a clamp
         int ps = min(__float2int_rz(__fmul_rn(__fsub_rn(u[t], mn), scale)), 63 << kOrqFBits);
-        if (TAIL) ps = max(ps, 0);
-        const int cell = min(ps >> kOrqFBits, kTopCell);
+        if (TAIL) ps = max(ps, 0);  // the invalid slots hold anything
+        const int cell = ps >> kOrqFBits;
         pos[t] = cell;
-        if (!TAIL || ((vmask >> t) & 1u)) {
-            atomicAdd(&sm.hcnt[cell * kHistCols + col], 1u);
-            atomicAdd(&sm.hsum[cell * kHistCols + col], (uint32_t)(ps - (cell << kOrqFBits)));
-        }
+        if (!TAIL || ((vmask >> t) & 1u))
+            atomicAdd(&sm.hist[cell * kHistCols + col], (uint32_t)(ps & 0xffff) | (1u << kHistCountShift));
     }
     __syncwarp();
-    // lane l reduces cells 2l and 2l+1 (16 consecutive words per array), clearing them; the
-    // four 16-byte reads are rotated by l/2 so that a quarter-warp touches 8 distinct bank groups
-    uint32_t c0 = 0, c1 = 0, f0 = 0, f1 = 0;
+    // lane l reduces cells 2l and 2l+1 (16 consecutive words), clearing them; the four 16-byte
+    // reads are rotated by l/2 so that a quarter-warp touches 8 distinct bank groups
+    uint32_t t0 = 0, t1 = 0, c0 = 0, c1 = 0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int q4 = (k + (lane >> 1)) & 3;
-        uint4 *pc = reinterpret_cast<uint4 *>(sm.hcnt + lane * 16) + q4;
-        uint4 *pf = reinterpret_cast<uint4 *>(sm.hsum + lane * 16) + q4;
-        const uint4 xc = *pc, xf = *pf;
-        *pc = make_uint4(0u, 0u, 0u, 0u);
-        *pf = make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t sc = xc.x + xc.y + xc.z + xc.w;
-        const uint32_t sf = xf.x + xf.y + xf.z + xf.w;
+        uint4 *ph = reinterpret_cast<uint4 *>(sm.hist + lane * 16) + q4;
+        const uint4 x = *ph;
+        *ph = make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t st = x.x + x.y + x.z + x.w;
+        const uint32_t sc = (x.x >> kHistCountShift) + (x.y >> kHistCountShift) + (x.z >> kHistCountShift) +
+                            (x.w >> kHistCountShift);
         if (q4 < 2) {
+            t0 += st;
             c0 += sc;
-            f0 += sf;
         } else {
+            t1 += st;
             c1 += sc;
-            f1 += sf;
         }
     }
-    // sums of positions of the two cells; one exclusive prefix over the cell pairs of the packed
-    // (sum << 16 | count): counts stay below 2^16 and sums below 2^31 for d <= 512
-    const uint32_t s0 = c0 * ((uint32_t)(2 * lane) << kOrqFBits) + f0;
-    const uint32_t s1 = c1 * ((uint32_t)(2 * lane + 1) << kOrqFBits) + f1;
+    // per cell: total < 2^32 (count <= 512 at bit 22 plus fractions < 2^25), fraction sum = total
+    // minus the counts' share
+    const uint32_t f0 = t0 - (c0 << kHistCountShift), f1 = t1 - (c1 << kHistCountShift);
+    // sums of positions of the two cells; the top grid point (cell 63) belongs to cell 62 with
+    // fraction 2^16, i.e. position 63 * 2^16, which is what s1 holds for lane 31
+    uint32_t s0 = c0 * ((uint32_t)(2 * lane) << kOrqFBits) + f0;
+    uint32_t s1 = c1 * ((uint32_t)(2 * lane + 1) << kOrqFBits) + f1;
+    if (lane == 31) {
+        c0 += c1;
+        s0 += s1;
+        c1 = 0u;
+        s1 = 0u;
+    }
+    // one exclusive prefix over the cell pairs of the packed (sum << 16 | count): counts stay
+    // below 2^16 and sums below 2^31 for d <= 512
     const unsigned long long own = ((unsigned long long)(s0 + s1) << 16) | (c0 + c1);
     const unsigned long long ex = warp_inclusive_scan(own, lane) - own;
     const int ec = (int)(ex & 0xffffu);
@@ -239,23 +299,7 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     reinterpret_cast<uint2 *>(sm.P1)[lane] = make_uint2(es, es + s0);
     __syncwarp();
     const unsigned long long mask = orq_greedy(sm.P0, sm.P1, p.s, lane);
-    // one table entry per cell, built in registers: the chosen grid indices around the cell
-    // give its bracket's ends; the lanes owning a chosen index write that level to the message
-    unsigned char *msg = p.msg[w];
-    float *mtab = msg ? reinterpret_cast<float *>(msg + p.levels_off) + beta * p.L : nullptr;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int j = lane + 32 * h;
-        if (j <= kTopCell) {
-            const unsigned long long upto = mask & ((2ull << j) - 1ull);  // chosen indices <= j
-            const int A = 63 - __clzll((long long)upto);
-            const int B = __ffsll((long long)(mask & ~((2ull << j) - 1ull))) - 1;
-            const float lo = grid_point(mn, mx, step, A), hi = grid_point(mn, mx, step, B);
-            sm.ctab[j] = make_float4(lo, hi, __frcp_rn(__fsub_rn(hi, lo)), __int_as_float(__popcll(upto) - 1));
-        }
-        if (mtab && ((mask >> j) & 1ull)) mtab[__popcll(mask & ((1ull << j) - 1ull))] = grid_point(mn, mx, step, j);
-    }
-    __syncwarp();
+    build_orq_tables(p, sm, w, beta, lane, mask, mn, mx, step);
     emit<EPL, FUSED, true, TAIL, BITS>(p, RoundORQ{sm.ctab}, beta, w, lane, vmask, v, u, pos, acc, ea);
     __syncwarp();
 }
@@ -569,10 +613,7 @@ template <int SCHEME, class Fit>
 __device__ __forceinline__ void init_fit(Fit &fit, int lane)
 {
     if constexpr (SCHEME == GQ_ORQ) {
-        for (int i = lane; i < 64 * kHistCols; i += 32) {
-            fit.hcnt[i] = 0u;
-            fit.hsum[i] = 0u;
-        }
+        for (int i = lane; i < 64 * kHistCols; i += 32) fit.hist[i] = 0u;
     }
     if constexpr (SCHEME == GQ_BINGRAD_PB) {
         for (int i = lane; i < 64; i += 32) {
