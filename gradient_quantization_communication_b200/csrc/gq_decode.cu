@@ -1,10 +1,9 @@
 // gq_decode.cu -- Dequantize + Aggregate: avg[i] = (sum_w level_w(code_w[i])) * (1/W).
 //
-// One warp owns a tile of 512 consecutive elements (four 128-element chunks of the packed
-// layout), for any bucket size.  Per worker and chunk the warp reads the b uint4 words of the
-// chunk (the same 16 bytes for all lanes: one broadcast transaction each) and the bucket's
-// level table; lane l pulls bit l of each word, which gives the codes of its elements
-// 128m + 4l + c, and looks the level up with a register shuffle (lane k holds level k).  The
+// One warp owns a tile of 512 consecutive elements (four 128-element chunks), for any bucket
+// size.  Per worker and chunk lane l reads the one or two words holding the codes of its
+// elements 128m + 4l + c (codes are packed densely, b bits each, in element order) and looks
+// the levels up with a register shuffle (lane k holds level k of the bucket).  The
 // sum runs in worker order in registers; the average is written once, with 16-byte stores.
 #include "gq_device.cuh"
 
@@ -45,17 +44,15 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
                 } else if (lane < p.L) {
                     lv = __ldg(tables + bk * p.L + lane);
                 }
-                uint32_t code0 = 0, code1 = 0, code2 = 0, code3 = 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (j < p.bits) {
-                        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(cw) + j);
-                        code0 |= ((x.x >> lane) & 1u) << j;
-                        code1 |= ((x.y >> lane) & 1u) << j;
-                        code2 |= ((x.z >> lane) & 1u) << j;
-                        code3 |= ((x.w >> lane) & 1u) << j;
-                    }
-                }
+                // lane l's four codes: the 4b-bit field at bit 4b*l of the chunk (it crosses a
+                // word boundary only for b = 3)
+                const int b = p.bits;
+                const int bitoff = 4 * b * lane, wi = bitoff >> 5, sh = bitoff & 31;
+                uint32_t x = __ldg(cw + wi) >> sh;
+                if (sh + 4 * b > 32) x |= __ldg(cw + wi + 1) << (32 - sh);
+                const uint32_t cmask = (1u << b) - 1u;
+                const uint32_t code0 = x & cmask, code1 = (x >> b) & cmask, code2 = (x >> (2 * b)) & cmask,
+                               code3 = (x >> (3 * b)) & cmask;
                 acc[4 * m + 0] = __fadd_rn(acc[4 * m + 0], __shfl_sync(kFull, lv, (int)code0));
                 acc[4 * m + 1] = __fadd_rn(acc[4 * m + 1], __shfl_sync(kFull, lv, (int)code1));
                 acc[4 * m + 2] = __fadd_rn(acc[4 * m + 2], __shfl_sync(kFull, lv, (int)code2));

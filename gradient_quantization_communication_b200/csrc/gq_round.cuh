@@ -115,12 +115,45 @@ struct RoundPB {
     }
 };
 
+// Dense packing of one 128-element chunk: the code of element e occupies bits [b*e, b*e + b)
+// of the chunk's 4b words (least significant bit first).  Lane l's four codes form the 4b-bit
+// field at bit 4b*l; pairs, quads and octets of lanes merge their fields with shuffles (the
+// fields do not overlap, so the merges are additions, done by the integer multiply-add unit),
+// and lane 8g stores the b words of octet g.  Every lane of the warp must take part.
+// BITS: bits per code when known at compile time, 0 to read it from p.bits.
+template <int BITS>
+__device__ __forceinline__ void pack_chunk(const KParams &p, int lane, const int (&code)[4], uint32_t *cw)
+{
+    const int b = BITS > 0 ? BITS : p.bits;  // (BITS < 0 only in never-run instantiations)
+    const uint32_t f1 = 1u << b, f2 = 1u << (2 * b), f3 = 1u << (3 * b);
+    const uint32_t y = (uint32_t)code[0] + (uint32_t)code[1] * f1 + (uint32_t)code[2] * f2 + (uint32_t)code[3] * f3;
+    const uint32_t z = y + __shfl_down_sync(kFull, y, 1) * (1u << (4 * b));  // 8b bits
+    const uint32_t z2 = __shfl_down_sync(kFull, z, 2);
+    const unsigned long long v = (unsigned long long)z2 * (1ull << (8 * b)) + z;  // 16b bits
+    const unsigned long long v2 = __shfl_down_sync(kFull, v, 4);
+    if ((lane & 7) == 0) {
+        uint32_t *o = cw + b * (lane >> 3);
+        if (b == 1) {
+            __stcs(o, (uint32_t)v + (uint32_t)v2 * 65536u);
+        } else if (b == 2) {
+            __stcs(reinterpret_cast<uint2 *>(o), make_uint2((uint32_t)v, (uint32_t)v2));
+        } else if (b == 3) {
+            __stcs(o, (uint32_t)v);
+            __stcs(o + 1, (uint32_t)(v >> 32) + (uint32_t)v2 * 65536u);
+            __stcs(o + 2, (uint32_t)(v2 >> 16));
+        } else {
+            __stcs(reinterpret_cast<uint4 *>(o), make_uint4((uint32_t)v, (uint32_t)(v >> 32), (uint32_t)v2,
+                                                            (uint32_t)(v2 >> 32)));
+        }
+    }
+}
+
 // One 128-element chunk of a bucket: lane l holds elements 4l .. 4l+3 of the chunk
 // (v: error-fed values, u: clipped values, pos: grid positions; valid: 4-bit mask, ignored
 // when ALLVALID).
 //   blk   global element index of the chunk's first element, divided by 4
 //   rout  residual of the chunk's first element (NULL: no residual), 16-byte aligned
-//   cw    packed words of the chunk (b uint4: plane j = words 4j..4j+3), NULL: no message
+//   cw    packed words of the chunk (4b words, 16-byte aligned), NULL: no message
 // Returns the dequantized values in q.
 // BITS: bits per code when known at compile time, 0 to read it from p.bits.
 template <bool RANDOM, bool ALLVALID, int BITS, class R>
@@ -147,19 +180,7 @@ __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uin
                 if ((valid >> c) & 1u) rout[4 * lane + c] = __fsub_rn(v[c], q[c]);
         }
     }
-    if (cw) {
-        // bit j of the code of element 4l + c -> bit l of word 4j + c of the chunk
-#pragma unroll
-        for (int j = 0; j < (BITS ? BITS : 4); ++j) {
-            if (BITS || j < p.bits) {
-                const uint32_t w0 = __ballot_sync(kFull, (code[0] >> j) & 1);
-                const uint32_t w1 = __ballot_sync(kFull, (code[1] >> j) & 1);
-                const uint32_t w2 = __ballot_sync(kFull, (code[2] >> j) & 1);
-                const uint32_t w3 = __ballot_sync(kFull, (code[3] >> j) & 1);
-                if (lane == 0) __stcs(reinterpret_cast<uint4 *>(cw) + j, make_uint4(w0, w1, w2, w3));
-            }
-        }
-    }
+    if (cw) pack_chunk<BITS>(p, lane, code, cw);
 }
 
 // Running binary64 sums of the quantization error (see gq_quant_error): expected squared

@@ -102,9 +102,9 @@ GQ_API gq_status_t gq_config_check(const gq_config_t *cfg);
  * buckets of d*b/32 uint32 words each.  *levels_off: offset (16-byte aligned) of the level
  * tables, ceil(n/d) tables of L float32 each (L = 1 for QSGD/TernGrad: the scale m; 2 for
  * BinGrad-b/pb: the two levels; s for ORQ: the ascending levels).
- * Packing inside a bucket: chunk m holds elements 128m .. 128m+127; element 128m + 4l + c
- * (l = 0..31, c = 0..3) stores bit j of its code (the index of its level) at bit l of word
- * (m*b + j)*4 + c.  Padding elements of the last bucket have code 0.
+ * Packing inside a bucket: dense, in element order, least significant bit first: bit j of the
+ * code (the index of its level) of element e is bit (b*e + j) % 32 of word (b*e + j) / 32 of
+ * the bucket's words.  Padding elements of the last bucket have code 0.
  * Any output pointer may be NULL.
  */
 GQ_API gq_status_t gq_message_layout(const gq_config_t *cfg, size_t *bytes, size_t *codes_off, size_t *levels_off);

@@ -594,29 +594,31 @@ void or_message_layout(const or_config *cfg, int64_t *bytes, int64_t *codes_off,
 }
 
 /*
- * Bit-plane packing of one bucket (b bits per code).  The bucket is cut into chunks of 128
- * elements; in chunk m, element e = 128m + 4l + c (l = 0..31, c = 0..3) puts bit j of its
- * code at bit l of word (m*b + j)*4 + c.  Codes of padding elements (e >= n) are 0.
+ * Dense packing of one bucket (b bits per code): the code of element e occupies bits
+ * b*e .. b*e + b - 1 of the bucket's d*b/32 words, read as one little-endian bit string (bit k
+ * is bit k % 32 of word k / 32).  Codes of padding elements (e >= n) are 0.
  */
 void or_pack_bucket(const or_config *cfg, const uint8_t *code, int n, uint32_t *words)
 {
     int b = or_bits(cfg->levels);
     int d = cfg->bucket;
     memset(words, 0, sizeof(uint32_t) * (size_t)(d * b / 32));
-    for (int e = 0; e < n; ++e) {
-        int m = e / 128, l = (e % 128) / 4, c = e % 4;
-        for (int j = 0; j < b; ++j)
-            if ((code[e] >> j) & 1) words[(m * b + j) * 4 + c] |= 1u << l;
-    }
+    for (int e = 0; e < n; ++e)
+        for (int j = 0; j < b; ++j) {
+            int64_t k = (int64_t)b * e + j;
+            if ((code[e] >> j) & 1) words[k / 32] |= 1u << (k % 32);
+        }
 }
 
 void or_unpack_bucket(const or_config *cfg, const uint32_t *words, int n, uint8_t *code)
 {
     int b = or_bits(cfg->levels);
     for (int e = 0; e < n; ++e) {
-        int m = e / 128, l = (e % 128) / 4, c = e % 4;
         int v = 0;
-        for (int j = 0; j < b; ++j) v |= (int)((words[(m * b + j) * 4 + c] >> l) & 1u) << j;
+        for (int j = 0; j < b; ++j) {
+            int64_t k = (int64_t)b * e + j;
+            v |= (int)((words[k / 32] >> (k % 32)) & 1u) << j;
+        }
         code[e] = (uint8_t)v;
     }
 }

@@ -413,6 +413,22 @@ def test_pack_roundtrip(levels):
                 assert np.array_equal(O.unpack_bucket(cfg, words, d)[n:], np.zeros(d - n, np.uint8))
 
 
+@pytest.mark.parametrize("levels", [2, 3, 5, 9, 16])
+def test_pack_is_dense_little_endian(levels):
+    """Packing layout: element e's code is bits b*e .. b*e+b-1 of the bucket's little-endian
+    bit string (here built as one Python integer, independently of the C loop)."""
+    rng = np.random.default_rng(100 + levels)
+    b = O.bits(levels)
+    for d, n in ((128, 128), (512, 512), (512, 301), (1024, 1000)):
+        cfg = O.Config(O.ORQ, levels, d, 1, 1, 0.0, 0, n)
+        code = rng.integers(0, levels, n).astype(np.uint8)
+        stream = 0
+        for e in range(n):
+            stream |= int(code[e]) << (b * e)
+        expect = np.array([(stream >> (32 * k)) & 0xffffffff for k in range(d * b // 32)], dtype=np.uint32)
+        assert np.array_equal(O.pack_bucket(cfg, code), expect)
+
+
 def test_error_feedback_telescopes():
     """[P3] error feedback: nothing is lost, only delayed: sum_t Q_t = sum_t g_t + r_0 - r_T."""
     rng = np.random.default_rng(18)
