@@ -221,42 +221,45 @@ __device__ __forceinline__ float clip_threshold_from_sums(long long sx, long lon
 // (x in units of 2^-16 cell).  Each round takes the largest Delta, ties to the smallest C.
 // Returns the 64-bit mask of chosen grid indices.
 // ---------------------------------------------------------------------------------------------
-// Buckets of up to 512 values: every prefix sum is below 512 * 63 * 2^16 < 2^31, so both
-// partial sums are exact in 32 bits and Delta takes two wide multiply-adds.
-__device__ __forceinline__ unsigned long long orq_delta(int A, int C, int B, int P0A, int P0C, int P0B, uint32_t P1A,
-                                                        uint32_t P1C, uint32_t P1B)
+// One side of Delta: the sum over the values between grid indices K and C (either order) of
+// their distance to K, in units of 2^-16 cell,
+//   side(K, C) = (P1[C] - P1[K]) - K * 2^16 * (P0[C] - P0[K]),
+// so that Delta(C) = (B-C) * side(A, C) + (C-A) * side(B, C).  The true value is non-negative;
+// with 32-bit prefix sums (buckets of up to 512 values: every prefix sum is below
+// 512 * 63 * 2^16 < 2^31) it is below 2^31 and exact in wrap-around arithmetic.
+__device__ __forceinline__ uint32_t orq_side(int K, int P0K, int P0C, uint32_t P1K, uint32_t P1C)
 {
-    const uint32_t lows = (P1C - P1A) - (uint32_t)(A << kOrqFBits) * (uint32_t)(P0C - P0A);
-    const uint32_t highs = (uint32_t)(B << kOrqFBits) * (uint32_t)(P0B - P0C) - (P1B - P1C);
-    return (unsigned long long)(uint32_t)(B - C) * lows + (unsigned long long)(uint32_t)(C - A) * highs;
+    return (P1C - P1K) - (uint32_t)(K << kOrqFBits) * (uint32_t)(P0C - P0K);
 }
-// Larger buckets: 64-bit prefix sums.
-__device__ __forceinline__ unsigned long long orq_delta(int A, int C, int B, int P0A, int P0C, int P0B, long long P1A,
-                                                        long long P1C, long long P1B)
+__device__ __forceinline__ long long orq_side(int K, int P0K, int P0C, long long P1K, long long P1C)
 {
-    const long long lows = (P1C - P1A) - (long long)(A << kOrqFBits) * (P0C - P0A);
-    const long long highs = (long long)(B << kOrqFBits) * (P0B - P0C) - (P1B - P1C);
-    return (unsigned long long)((long long)(B - C) * lows + (long long)(C - A) * highs);
+    return (P1C - P1K) - (long long)(K << kOrqFBits) * (long long)(P0C - P0K);
 }
-
-// Incremental form: lane l owns candidates C = l and l + 32 with their current neighbours and
-// ranking key (Delta << 6 | 63 - C: the largest key has the largest Delta, ties to the smallest
-// C; 0 for an index that is chosen or never a candidate) in registers; after a level L is added
-// only the candidates of the bracket it split are re-evaluated (skipped warp-wide when no lane
-// has one).
-template <class T>
-__device__ __forceinline__ unsigned long long orq_key(int A, int C, int B, int P0A, int P0C, int P0B, T P1A, T P1C,
-                                                      T P1B)
+// Ranking key of candidate C: Delta << 6 | 63 - C (the largest key has the largest Delta, ties
+// to the smallest C).
+__device__ __forceinline__ unsigned long long orq_key(int A, int C, int B, uint32_t lows, uint32_t highs)
 {
-    return (orq_delta(A, C, B, P0A, P0C, P0B, P1A, P1C, P1B) << 6) | (unsigned long long)(63 - C);
+    const unsigned long long delta =
+        (unsigned long long)(uint32_t)(B - C) * lows + (unsigned long long)(uint32_t)(C - A) * highs;
+    return (delta << 6) | (unsigned long long)(63 - C);
+}
+__device__ __forceinline__ unsigned long long orq_key(int A, int C, int B, long long lows, long long highs)
+{
+    const unsigned long long delta = (unsigned long long)((long long)(B - C) * lows + (long long)(C - A) * highs);
+    return (delta << 6) | (unsigned long long)(63 - C);
 }
 
+// Incremental form: lane l owns candidates C = l and l + 32 with their current neighbours
+// A < C < B, the two sides side(A, C), side(B, C) and the ranking key in registers (key 0 for
+// an index that is chosen or never a candidate).  Adding level L to the bracket (A, B) of a
+// candidate changes one neighbour and one side: for L < C the lower one, for L > C the upper
+// one, and both are side(L, C).
 template <class T>
 __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T *P1, int s, int lane)
 {
     unsigned long long mask = 1ull | (1ull << 63);
-    int A[2], B[2], P0A[2], P0B[2], P0C[2];
-    T P1A[2], P1B[2], P1C[2];
+    int A[2], B[2], P0C[2];
+    T P1C[2], lows[2], highs[2];
     unsigned long long key[2];
     const int P0lo = P0[0], P0hi = P0[63];
     const T P1lo = P1[0], P1hi = P1[63];
@@ -265,13 +268,11 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T 
         const int C = lane + 32 * h;
         A[h] = 0;
         B[h] = 63;
-        P0A[h] = P0lo;
-        P1A[h] = P1lo;
-        P0B[h] = P0hi;
-        P1B[h] = P1hi;
         P0C[h] = P0[C];
         P1C[h] = P1[C];
-        key[h] = (C >= 1 && C <= 62) ? orq_key(0, C, 63, P0lo, P0C[h], P0hi, P1lo, P1C[h], P1hi) : 0ull;
+        lows[h] = orq_side(0, P0lo, P0C[h], P1lo, P1C[h]);
+        highs[h] = orq_side(63, P0hi, P0C[h], P1hi, P1C[h]);
+        key[h] = (C >= 1 && C <= 62) ? orq_key(0, C, 63, lows[h], highs[h]) : 0ull;
     }
     for (int round = 0; round < s - 2; ++round) {
         const unsigned long long best = key[0] > key[1] ? key[0] : key[1];
@@ -286,21 +287,17 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T 
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int C = lane + 32 * h;
-            if (C == L) key[h] = 0ull;
-            const bool split = key[h] != 0ull && A[h] < L && L < B[h];
-            if (__any_sync(kFull, split)) {
-                if (split) {
-                    if (L < C) {
-                        A[h] = L;
-                        P0A[h] = P0L;
-                        P1A[h] = P1L;
-                    } else {
-                        B[h] = L;
-                        P0B[h] = P0L;
-                        P1B[h] = P1L;
-                    }
-                    key[h] = orq_key(A[h], C, B[h], P0A[h], P0C[h], P0B[h], P1A[h], P1C[h], P1B[h]);
+            // the chosen index itself lies in the split bracket too: its key drops to 0
+            if (key[h] != 0ull && A[h] < L && L < B[h]) {
+                const T x = orq_side(L, P0L, P0C[h], P1L, P1C[h]);
+                if (L < C) {
+                    A[h] = L;
+                    lows[h] = x;
+                } else {
+                    B[h] = L;
+                    highs[h] = x;
                 }
+                key[h] = C == L ? 0ull : orq_key(A[h], C, B[h], lows[h], highs[h]);
             }
         }
     }
