@@ -86,6 +86,20 @@ __device__ __forceinline__ double pow2d(int e)
     return __longlong_as_double((long long)(1023 + e) << 52);
 }
 
+// 2^e as a float, e in [-126, 127].
+__device__ __forceinline__ float pow2f(int e)
+{
+    return __uint_as_float((uint32_t)(127 + e) << 23);
+}
+
+// Reciprocal within 1 ulp (hardware approximation; positive normal inputs).
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // Saturate to [0, 1]; NaN and -0 become +0.
 __device__ __forceinline__ float sat01(float x)
 {

@@ -304,31 +304,31 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     __syncwarp();
 }
 
-// Bitonic sort of the 32*EPL keys, position i = lane*EPL + r.
+// Bitonic sort of the 32*EPL keys, position i = lane*EPL + r, ascending.  Every compare-
+// exchange is one min and one max: the direction of a merge of blocks of k keys, and for
+// distances j >= EPL the side of the partner lane, depend only on the lane once k >= EPL, so
+// they are taken once per stage instead of once per key.
 template <int EPL>
 __device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
 {
     constexpr int N = 32 * EPL;
 #pragma unroll
     for (int k = 2; k <= N; k <<= 1) {
+        const bool lane_up = ((lane * EPL) & k) == 0;  // blocks of k ascending (k >= EPL)
 #pragma unroll
         for (int j = k >> 1; j > 0; j >>= 1) {
             if (j >= EPL) {
-                const int lm = j / EPL;
+                const bool take_min = (((lane * EPL) & j) == 0) == lane_up;
 #pragma unroll
                 for (int r = 0; r < EPL; ++r) {
-                    const int i = lane * EPL + r;
-                    const float o = __shfl_xor_sync(kFull, key[r], lm);
-                    const bool up = (i & k) == 0;
-                    const bool lower = (i & j) == 0;
-                    key[r] = (lower == up) ? fminf(key[r], o) : fmaxf(key[r], o);
+                    const float o = __shfl_xor_sync(kFull, key[r], j / EPL);
+                    key[r] = take_min ? fminf(key[r], o) : fmaxf(key[r], o);
                 }
             } else {
 #pragma unroll
                 for (int r = 0; r < EPL; ++r) {
                     if ((r & j) == 0) {
-                        const int i = lane * EPL + r;
-                        const bool up = (i & k) == 0;
+                        const bool up = k >= EPL ? lane_up : (r & k) == 0;
                         const float a = key[r], b = key[r ^ j];
                         key[r] = up ? fminf(a, b) : fmaxf(a, b);
                         key[r ^ j] = up ? fmaxf(a, b) : fminf(a, b);
@@ -359,27 +359,51 @@ __device__ void fit_bingrad_b(const KParams &p, FitB &, int64_t beta, int w, int
         for (int t = 0; t < EPL; ++t) key[t] = (!TAIL || ((vmask >> t) & 1u)) ? u[t] : INFINITY;
         warp_bitonic_sort<EPL>(key, lane);
         const int e = 46 - fexpo(m);
-        const double sc = pow2d(e);
+        // fixed point round(x * 2^e) in binary32: the scaling by 2^e (as 2^(e/2) * 2^(e - e/2),
+        // both representable for e in [-81, 195]) is exact, except for products that fall below
+        // 2^-126, which round to 0 either way
+        const float s1 = pow2f(e >> 1), s2 = pow2f(e - (e >> 1));
         // inclusive prefix of the fixed-point values inside the lane, then across lanes
         long long pre[EPL];
         long long run = 0;
 #pragma unroll
         for (int r = 0; r < EPL; ++r) {
             const int i = lane * EPL + r;
-            run += (!TAIL || i < nvalid) ? fixed_point(key[r], sc) : 0ll;
+            run += (!TAIL || i < nvalid) ? __float2ll_rn(__fmul_rn(__fmul_rn(key[r], s1), s2)) : 0ll;
             pre[r] = run;
         }
         const long long incl = warp_inclusive_scan(run, lane);
         const long long lane_excl = incl - run;
         const long long total = __shfl_sync(kFull, incl, 31);
         const float prev_last = __shfl_up_sync(kFull, key[EPL - 1], 1);
-        double best_j = -1.0;
-        int best_i = 0x7fffffff;
+        // Screening: a binary32 estimate of J for every admissible split (two conversions of
+        // exact integers, two squares, two reciprocals within 1 ulp, two products and a sum:
+        // within 8 * 2^-24 of J), then the fp64 J only for the splits whose estimate reaches
+        // M (1 - 2^-18), M the largest estimate: every split whose fp64 J is the largest is
+        // among them, so the choice (ties to the smallest split) is the exhaustive one.
+        float est[EPL];
+        float emax = 0.0f;
 #pragma unroll
         for (int r = 0; r < EPL; ++r) {
             const int i = lane * EPL + r;  // split: positions < i on the left
             const float prev = r > 0 ? key[r - 1] : prev_last;
+            est[r] = -1.0f;
             if (i >= 1 && i < nvalid && prev < key[r]) {
+                const long long Sl = lane_excl + (r > 0 ? pre[r - 1] : 0ll);
+                const float l = __ll2float_rn(Sl), rr = __ll2float_rn(total - Sl);
+                est[r] = __fadd_rn(__fmul_rn(__fmul_rn(l, l), rcp_approx((float)i)),
+                                   __fmul_rn(__fmul_rn(rr, rr), rcp_approx((float)(nvalid - i))));
+                emax = fmaxf(emax, est[r]);
+            }
+        }
+        // the estimates are >= +0, so their bit patterns order like unsigned integers
+        const float thr = __fmul_rn(__uint_as_float(__reduce_max_sync(kFull, __float_as_uint(emax))), 1.0f - 0x1p-18f);
+        double best_j = -1.0;
+        int best_i = 0x7fffffff;
+#pragma unroll
+        for (int r = 0; r < EPL; ++r) {
+            if (est[r] >= thr) {
+                const int i = lane * EPL + r;
                 const long long Sl = lane_excl + (r > 0 ? pre[r - 1] : 0ll);
                 const double l = __ll2double_rn(Sl);
                 const double rr = __ll2double_rn(total - Sl);
@@ -603,10 +627,20 @@ __device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME
 #ifndef GQ_WARP_MIN_BLOCKS
 #define GQ_WARP_MIN_BLOCKS 4
 #endif
+// BinGrad keeps the sorted slice and its prefix sums (BinGrad-b) or the pair search state
+// (BinGrad-pb) in registers: 3 and 4 CTAs per SM are the most that compile without spills.
+#ifndef GQ_BINB_MIN_BLOCKS
+#define GQ_BINB_MIN_BLOCKS 3
+#endif
+#ifndef GQ_BINPB_MIN_BLOCKS
+#define GQ_BINPB_MIN_BLOCKS 4
+#endif
 template <int EPL, int SCHEME, int WARPS>
 constexpr int min_blocks()
 {
-    return (SCHEME == GQ_BINGRAD_B || SCHEME == GQ_BINGRAD_PB) ? 2 : GQ_WARP_MIN_BLOCKS * 4 / WARPS;
+    return SCHEME == GQ_BINGRAD_B    ? GQ_BINB_MIN_BLOCKS
+           : SCHEME == GQ_BINGRAD_PB ? GQ_BINPB_MIN_BLOCKS
+                                     : GQ_WARP_MIN_BLOCKS * 4 / WARPS;
 }
 
 template <int SCHEME, class Fit>
