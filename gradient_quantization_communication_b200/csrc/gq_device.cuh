@@ -264,10 +264,10 @@ __device__ __forceinline__ unsigned long long orq_key(int A, int C, int B, long 
 }
 
 // Incremental form: lane l owns candidates C = l and l + 32 with their current neighbours
-// A < C < B, the two sides side(A, C), side(B, C) and the ranking key in registers (key 0 for
-// an index that is chosen or never a candidate).  Adding level L to the bracket (A, B) of a
-// candidate changes one neighbour and one side: for L < C the lower one, for L > C the upper
-// one, and both are side(L, C).
+// A < C < B, the two sides side(A, C), side(B, C) and the ranking key in registers.  Adding level
+// L to the bracket (A, B) of a candidate changes one neighbour and one side: for L < C the lower
+// one, for L > C the upper one, and both are side(L, C).  An index that is chosen (or never a
+// candidate: 0 and 63) gets key 0 and the empty bracket A = B = C, which no later level splits.
 template <class T>
 __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T *P1, int s, int lane)
 {
@@ -280,13 +280,14 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T 
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int C = lane + 32 * h;
-        A[h] = 0;
-        B[h] = 63;
+        const bool cand = C >= 1 && C <= 62;
+        A[h] = cand ? 0 : C;
+        B[h] = cand ? 63 : C;
         P0C[h] = P0[C];
         P1C[h] = P1[C];
         lows[h] = orq_side(0, P0lo, P0C[h], P1lo, P1C[h]);
         highs[h] = orq_side(63, P0hi, P0C[h], P1hi, P1C[h]);
-        key[h] = (C >= 1 && C <= 62) ? orq_key(0, C, 63, lows[h], highs[h]) : 0ull;
+        key[h] = cand ? orq_key(0, C, 63, lows[h], highs[h]) : 0ull;
     }
     for (int round = 0; round < s - 2; ++round) {
         const unsigned long long best = key[0] > key[1] ? key[0] : key[1];
@@ -301,17 +302,22 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T 
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int C = lane + 32 * h;
-            // the chosen index itself lies in the split bracket too: its key drops to 0
-            if (key[h] != 0ull && A[h] < L && L < B[h]) {
-                const T x = orq_side(L, P0L, P0C[h], P1L, P1C[h]);
-                if (L < C) {
-                    A[h] = L;
-                    lows[h] = x;
+            if (A[h] < L && L < B[h]) {
+                if (C == L) {  // the chosen index: key 0, empty bracket
+                    A[h] = C;
+                    B[h] = C;
+                    key[h] = 0ull;
                 } else {
-                    B[h] = L;
-                    highs[h] = x;
+                    const T x = orq_side(L, P0L, P0C[h], P1L, P1C[h]);
+                    if (L < C) {
+                        A[h] = L;
+                        lows[h] = x;
+                    } else {
+                        B[h] = L;
+                        highs[h] = x;
+                    }
+                    key[h] = orq_key(A[h], C, B[h], lows[h], highs[h]);
                 }
-                key[h] = C == L ? 0ull : orq_key(A[h], C, B[h], lows[h], highs[h]);
             }
         }
     }

@@ -156,7 +156,8 @@ __device__ __forceinline__ void pack_chunk(const KParams &p, int lane, const int
 //   cw    packed words of the chunk (4b words, 16-byte aligned), NULL: no message
 // Returns the dequantized values in q.
 // BITS: bits per code when known at compile time, 0 to read it from p.bits.
-template <bool RANDOM, bool ALLVALID, int BITS, class R>
+// IO: bit 0 set if rout is known non-NULL, bit 1 if cw is (no run-time test then).
+template <bool RANDOM, bool ALLVALID, int BITS, int IO = 0, class R>
 __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uint64_t blk, uint32_t worker, int lane,
                                             uint32_t valid, const float (&v)[4], const float (&u)[4],
                                             const int (&pos)[4], float *rout, uint32_t *cw, float (&q)[4])
@@ -170,7 +171,7 @@ __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uin
         rule.round(u[c], pos[c], words[c], code[c], q[c]);
         if (!ALLVALID && !((valid >> c) & 1u)) code[c] = 0;
     }
-    if (rout) {
+    if ((IO & 1) || rout) {
         if (ALLVALID || valid == 0xfu) {
             __stcs(reinterpret_cast<float4 *>(rout + 4 * lane),
                    make_float4(__fsub_rn(v[0], q[0]), __fsub_rn(v[1], q[1]), __fsub_rn(v[2], q[2]), __fsub_rn(v[3], q[3])));
@@ -180,7 +181,7 @@ __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uin
                 if ((valid >> c) & 1u) rout[4 * lane + c] = __fsub_rn(v[c], q[c]);
         }
     }
-    if (cw) pack_chunk<BITS>(p, lane, code, cw);
+    if ((IO & 2) || cw) pack_chunk<BITS>(p, lane, code, cw);
 }
 
 // Running binary64 sums of the quantization error (see gq_quant_error): expected squared

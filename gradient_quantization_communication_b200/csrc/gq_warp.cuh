@@ -86,7 +86,7 @@ __device__ __forceinline__ int slot_elem(int t, int lane) { return 128 * (t >> 2
 // ---------------------------------------------------------------------------------------------
 // BITS < 0 selects the error mode of gq_quant_error: nothing is written, the error terms of
 // the bucket's elements are added to *ea.
-template <int EPL, bool FUSED, bool RANDOM, bool TAIL, int BITS, class R>
+template <int EPL, bool FUSED, bool RANDOM, bool TAIL, int BITS, int IO = 0, class R>
 __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t beta, int w, int lane, uint32_t vmask,
                                      const float (&v)[EPL], const float (&u)[EPL], const int (&pos)[EPL],
                                      float (&acc)[EPL], ErrAcc *ea = nullptr)
@@ -104,9 +104,11 @@ __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t be
         }
         return;
     }
+    constexpr bool kHasR = (IO & 1) != 0, kHasMsg = (IO & 2) != 0;
+    constexpr int kCodeWords = 4 * (BITS > 0 ? BITS : 0);  // words per chunk when b is known
     float *r = p.r[w];
     unsigned char *msg = p.msg[w];
-    uint32_t *cw = msg ? reinterpret_cast<uint32_t *>(msg) + beta * p.codes_words : nullptr;
+    uint32_t *cw = (kHasMsg || msg) ? reinterpret_cast<uint32_t *>(msg) + beta * p.codes_words : nullptr;
     const uint32_t worker = p.worker0 + (uint32_t)w;
 #pragma unroll
     for (int m = 0; m < EPL / 4; ++m) {
@@ -115,8 +117,9 @@ __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t be
         const int pp[4] = {pos[4 * m], pos[4 * m + 1], pos[4 * m + 2], pos[4 * m + 3]};
         const uint32_t valid = TAIL ? (vmask >> (4 * m)) & 0xfu : 0xfu;
         float q[4];
-        round_chunk<RANDOM, !TAIL, BITS>(p, rule, (uint64_t)(base >> 2) + (uint64_t)(32 * m), worker, lane, valid, vv, uu,
-                                   pp, r ? r + base + 128 * m : nullptr, cw ? cw + m * 4 * p.bits : nullptr, q);
+        round_chunk<RANDOM, !TAIL, BITS, IO>(p, rule, (uint64_t)(base >> 2) + (uint64_t)(32 * m), worker, lane, valid,
+                                             vv, uu, pp, (kHasR || r) ? r + base + 128 * m : nullptr,
+                                             (kHasMsg || cw) ? cw + m * (kCodeWords ? kCodeWords : 4 * p.bits) : nullptr, q);
         if (FUSED) {
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -175,7 +178,7 @@ __device__ __forceinline__ void build_orq_tables(const KParams &p, FitORQ &sm, i
 // ---------------------------------------------------------------------------------------------
 // Per-scheme fits (u: the values to quantize; v: the error-fed values the residual refers to)
 // ---------------------------------------------------------------------------------------------
-template <int EPL, bool FUSED, bool TAIL, int BITS>
+template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0>
 __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                          const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
@@ -199,11 +202,11 @@ __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int
     int pos[EPL];
 #pragma unroll
     for (int t = 0; t < EPL; ++t) pos[t] = 0;
-    emit<EPL, FUSED, true, TAIL, BITS>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
+    emit<EPL, FUSED, true, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
     store_table(p, w, beta, lane, m);
 }
 
-template <int EPL, bool FUSED, bool TAIL, int BITS>
+template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0>
 __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                         const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
@@ -233,7 +236,7 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     if (!(mx > mn)) {  // constant bucket (or NaN): one level, code 0
 #pragma unroll
         for (int t = 0; t < EPL; ++t) pos[t] = 0;
-        emit<EPL, FUSED, false, TAIL, BITS>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc, ea);
+        emit<EPL, FUSED, false, TAIL, BITS, IO>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc, ea);
         store_table(p, w, beta, lane, mn);
         return;
     }
@@ -300,7 +303,7 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     __syncwarp();
     const unsigned long long mask = orq_greedy(sm.P0, sm.P1, p.s, lane);
     build_orq_tables(p, sm, w, beta, lane, mask, mn, mx, step);
-    emit<EPL, FUSED, true, TAIL, BITS>(p, RoundORQ{sm.ctab}, beta, w, lane, vmask, v, u, pos, acc, ea);
+    emit<EPL, FUSED, true, TAIL, BITS, IO>(p, RoundORQ{sm.ctab}, beta, w, lane, vmask, v, u, pos, acc, ea);
     __syncwarp();
 }
 
@@ -339,7 +342,7 @@ __device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
     }
 }
 
-template <int EPL, bool FUSED, bool TAIL, int BITS>
+template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0>
 __device__ void fit_bingrad_b(const KParams &p, FitB &, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                               int nvalid, const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
@@ -448,11 +451,11 @@ __device__ void fit_bingrad_b(const KParams &p, FitB &, int64_t beta, int w, int
             rule = RoundB{a, b, tv, true};
         }
     }
-    emit<EPL, FUSED, false, TAIL, BITS>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
+    emit<EPL, FUSED, false, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
     store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
 }
 
-template <int EPL, bool FUSED, bool TAIL, int BITS>
+template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0>
 __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                                const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
@@ -472,7 +475,7 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
     if (!(mx > mn)) {
 #pragma unroll
         for (int t = 0; t < EPL; ++t) pos[t] = 0;
-        emit<EPL, FUSED, false, TAIL, BITS>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc, ea);
+        emit<EPL, FUSED, false, TAIL, BITS, IO>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc, ea);
         store_table(p, w, beta, lane, mn);
         return;
     }
@@ -560,14 +563,14 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
     rule.rinv = __frcp_rn(__fsub_rn(rule.b, rule.a));
     rule.pa = A << kPbFBits;
     rule.pb = B << kPbFBits;
-    emit<EPL, FUSED, true, TAIL, BITS>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
+    emit<EPL, FUSED, true, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
     store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
 }
 
 // ---------------------------------------------------------------------------------------------
 // One item: clip, fit, round, write
 // ---------------------------------------------------------------------------------------------
-template <int EPL, int SCHEME, bool FUSED, bool TAIL, int BITS>
+template <int EPL, int SCHEME, bool FUSED, bool TAIL, int BITS, int IO = 0>
 __device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME>::type &fit, int64_t beta, int w,
                                         int lane, int nvalid, uint32_t vmask, const float (&v)[EPL], float (&acc)[EPL],
                                         ErrAcc *ea = nullptr)
@@ -610,13 +613,13 @@ __device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME
         for (int t = 0; t < EPL; ++t) u[t] = v[t];
     }
     if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD)
-        fit_qsgd<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
+        fit_qsgd<EPL, FUSED, TAIL, BITS, IO>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
     else if constexpr (SCHEME == GQ_ORQ)
-        fit_orq<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
+        fit_orq<EPL, FUSED, TAIL, BITS, IO>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
     else if constexpr (SCHEME == GQ_BINGRAD_B)
-        fit_bingrad_b<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, nvalid, v, u, acc, ea);
+        fit_bingrad_b<EPL, FUSED, TAIL, BITS, IO>(p, fit, beta, w, lane, vmask, check, nvalid, v, u, acc, ea);
     else
-        fit_bingrad_pb<EPL, FUSED, TAIL, BITS>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
+        fit_bingrad_pb<EPL, FUSED, TAIL, BITS, IO>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -667,7 +670,9 @@ __device__ __forceinline__ void store_avg4(float *ab, int m, int lane, const flo
 
 // Full buckets 0 .. nfull-1: every warp walks its items (bucket, worker), bulk copies one item
 // ahead.
-template <int EPL, int SCHEME, bool FUSED, int BITS>
+// IO = 3: every worker has a residual and a message buffer (known at compile time, so the
+// rounding pass is straight-line code); IO = 0: checked at run time.
+template <int EPL, int SCHEME, bool FUSED, int BITS, int IO>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME, kWarpsPerCta>()))
     k_warp(const __grid_constant__ KParams p, int64_t nfull)
 {
@@ -690,7 +695,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME, kW
     if (first >= nfull) return;
     const int W = p.W;
     const int64_t nitems = ((nfull - 1 - first) / stride + 1) * W;
-    const bool ef = p.r[0] != nullptr;
+    const bool ef = (IO & 1) || p.r[0] != nullptr;
     const unsigned tx = ef ? 2 * kBytes : kBytes;
     auto issue = [&](int64_t beta, int w, int k) {  // lane 0
         fence_proxy_async();
@@ -749,7 +754,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME, kW
 #pragma unroll
             for (int t = 0; t < EPL; ++t) acc[t] = 0.0f;
         }
-        process<EPL, SCHEME, FUSED, false, BITS>(p, sm.fit, beta, w, lane, D, 0xffffffffu, v, acc);
+        process<EPL, SCHEME, FUSED, false, BITS, IO>(p, sm.fit, beta, w, lane, D, 0xffffffffu, v, acc);
         if (FUSED && last_w) {
 #pragma unroll
             for (int m = 0; m < EPL / 4; ++m) store_avg4(p.avg + beta * D, m, lane, acc + 4 * m, p.inv_w);
@@ -910,7 +915,9 @@ cudaError_t launch_one(const KParams &p, cudaStream_t stream)
     constexpr int D = 32 * EPL;
     const int64_t nfull = p.tail == D ? p.nb : p.nb - 1;
     if (nfull > 0) {
-        auto kern = k_warp<EPL, SCHEME, FUSED, BITS>;
+        bool all_io = true;
+        for (int w = 0; w < p.W; ++w) all_io = all_io && p.r[w] != nullptr && p.msg[w] != nullptr;
+        auto kern = all_io ? k_warp<EPL, SCHEME, FUSED, BITS, 3> : k_warp<EPL, SCHEME, FUSED, BITS, 0>;
         const size_t smem = sizeof(WarpSmem<EPL, SCHEME>) * kWarpsPerCta;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
