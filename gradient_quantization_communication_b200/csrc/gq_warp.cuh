@@ -307,21 +307,43 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     __syncwarp();
 }
 
-// Bitonic sort of the 32*EPL keys, position i = lane*EPL + r, ascending.  Every compare-
-// exchange is one min and one max: the direction of a merge of blocks of k keys, and for
-// distances j >= EPL the side of the partner lane, depend only on the lane once k >= EPL, so
-// they are taken once per stage instead of once per key.
+// Bitonic sort of the 32*EPL keys, position i = lane*EPL + r, ascending, in the form whose
+// comparators all put the minimum at the lower index: each merge of blocks of k keys starts by
+// comparing i with its mirror i ^ (k-1), then i with i ^ j for j = k/4 .. 1.  Inside a lane a
+// compare-exchange is one min and one max; across lanes (partner lane l ^ m) the lower lane keeps
+// the minimum, a choice that depends on the lane only.
 template <int EPL>
 __device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
 {
     constexpr int N = 32 * EPL;
 #pragma unroll
     for (int k = 2; k <= N; k <<= 1) {
-        const bool lane_up = ((lane * EPL) & k) == 0;  // blocks of k ascending (k >= EPL)
+        if (k <= EPL) {
 #pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int r = 0; r < EPL; ++r) {
+                const int q = r ^ (k - 1);
+                if (q > r) {
+                    const float a = key[r], b = key[q];
+                    key[r] = fminf(a, b);
+                    key[q] = fmaxf(a, b);
+                }
+            }
+        } else {
+            // partner of (lane, r) is (lane ^ m, EPL-1-r); pairs (r, EPL-1-r) are updated together
+            const int m = k / EPL - 1;
+            const bool take_min = (lane & ((k / EPL) >> 1)) == 0;
+#pragma unroll
+            for (int r = 0; r < EPL / 2; ++r) {
+                const float o1 = __shfl_xor_sync(kFull, key[EPL - 1 - r], m);
+                const float o2 = __shfl_xor_sync(kFull, key[r], m);
+                key[r] = take_min ? fminf(key[r], o1) : fmaxf(key[r], o1);
+                key[EPL - 1 - r] = take_min ? fminf(key[EPL - 1 - r], o2) : fmaxf(key[EPL - 1 - r], o2);
+            }
+        }
+#pragma unroll
+        for (int j = k >> 2; j > 0; j >>= 1) {
             if (j >= EPL) {
-                const bool take_min = (((lane * EPL) & j) == 0) == lane_up;
+                const bool take_min = (lane & (j / EPL)) == 0;
 #pragma unroll
                 for (int r = 0; r < EPL; ++r) {
                     const float o = __shfl_xor_sync(kFull, key[r], j / EPL);
@@ -331,10 +353,9 @@ __device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
 #pragma unroll
                 for (int r = 0; r < EPL; ++r) {
                     if ((r & j) == 0) {
-                        const bool up = k >= EPL ? lane_up : (r & k) == 0;
                         const float a = key[r], b = key[r ^ j];
-                        key[r] = up ? fminf(a, b) : fmaxf(a, b);
-                        key[r ^ j] = up ? fmaxf(a, b) : fminf(a, b);
+                        key[r] = fminf(a, b);
+                        key[r ^ j] = fmaxf(a, b);
                     }
                 }
             }
@@ -529,17 +550,21 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
         sm.de[K] = (long long)(k * uQ0 - uQ1);
     }
     __syncwarp();
-    // exhaustive search over A < B, ties to the smallest (A, B)
+    // exhaustive search over A < B, ties to the smallest (A, B).  Lane l takes B = l (A < l) and
+    // B = 63 - l (A < 63 - l): 63 pairs on every lane, one uniform loop.  With ga, de kept
+    // pre-multiplied by 2^16, E = al[A] + be[B] + A * ga16[B] + B * de16[A] (mod 2^64, exact).
     long long best_e = 0x7fffffffffffffffll;
     int best_ab = 0x7fffffff;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int B = lane + 32 * h;
-        const unsigned long long bb = (unsigned long long)B << kPbFBits;
-        const unsigned long long beB = sm.be[B], gaB = sm.ga[B];
-        for (int A = 0; A < B; ++A) {
-            const unsigned long long aa = (unsigned long long)A << kPbFBits;
-            const long long e = (long long)((unsigned long long)sm.al[A] + beB + aa * gaB + bb * (unsigned long long)sm.de[A]);
+    {
+        const int B0 = lane, B1 = 63 - lane;
+        const unsigned long long be0 = sm.be[B0], ga0 = (unsigned long long)sm.ga[B0] << kPbFBits;
+        const unsigned long long be1 = sm.be[B1], ga1 = (unsigned long long)sm.ga[B1] << kPbFBits;
+        for (int i = 0; i < 63; ++i) {
+            const bool first = i < B0;
+            const int A = first ? i : i - B0, B = first ? B0 : B1;
+            const unsigned long long beB = first ? be0 : be1, gaB = first ? ga0 : ga1;
+            const long long e = (long long)((unsigned long long)sm.al[A] + beB + (unsigned long long)A * gaB +
+                                            (unsigned long long)B * ((unsigned long long)sm.de[A] << kPbFBits));
             const int ab = A * 64 + B;
             if (e < best_e || (e == best_e && ab < best_ab)) {
                 best_e = e;
