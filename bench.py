@@ -416,25 +416,27 @@ def run_e2e(args, G, plan, W, n, g, r, msgs, avg, dev, stream, world):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, dev)
     del host_g, host_avg
     return {"value": world * W * n * args.e2e_steps / (ms / 1000.0), "unit": UNIT,
             "h2d_bytes_per_step": 4 * W * n, "d2h_bytes_per_step": 4 * n, "steps": args.e2e_steps}
 
 
 def run_cpu_baseline(args, wl, g):
+    """The oracle on all host cores, on the first buckets of every worker: a probe of 8 buckets
+    per thread calibrates the rate, then a sample sized to about args.cpu_seconds of CPU work
+    (at most 2 GB of host copies) is timed once."""
     threads = cpu_threads()
-    max_buckets = 64 * threads * 16
-    nelem = min(wl.n, max_buckets * args.bucket)
-    gs_host = [x[:nelem].cpu().numpy() for x in g]
-    nbk, _ = calibrated_buckets(wl, args, gs_host, threads, args.cpu_seconds)
-    nbk = min(nbk, nelem // args.bucket)
+    d = args.bucket
+    probe = min(8 * threads, wl.n // d)
+    gs_probe = [x[:probe * d].cpu().numpy() for x in g]
+    _, dt = oracle_sample_rate(wl, args, gs_probe, probe, threads)
+    nbk = int(args.cpu_seconds / (dt / probe))
+    nbk = max(probe, min(nbk, wl.n // d, (2 << 30) // (4 * d * wl.workers)))
+    gs_host = [x[:nbk * d].cpu().numpy() for x in g]
     rate, dt = oracle_sample_rate(wl, args, gs_host, nbk, threads)
     return {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "seconds": round(dt, 2),
-            "sample": "first %d buckets (d=%d) of each of the %d workers, one step" % (nbk, args.bucket, wl.workers)}
+            "sample": "first %d buckets (d=%d) of each of the %d workers, one step" % (nbk, d, wl.workers)}
 
 
 def run_sweep(args):
