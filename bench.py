@@ -2,7 +2,7 @@
 """Throughput of the bucketed gradient-quantization step on B200.
 
 One step = one pass of the whole hot path over one batch: for each of W simulated workers,
-error feedback (v = g + r), per-bucket level fit, Philox stochastic rounding, bit-plane packing
+error feedback (v = g + r), per-bucket level fit, Philox stochastic rounding, dense bit packing
 into the worker's message, residual update, and the decode + average of the W dequantized
 gradients (gq_fused_step, messages written).
 

@@ -1,6 +1,7 @@
 // gq_round.cuh -- per-element rounding rules of the five schemes and the 128-element chunk
 // step shared by the register path (d <= 512) and the shared-memory path (d >= 1024):
-// draw, round, dequantize, write the residual, bit-plane pack with warp ballots.
+// draw, round, dequantize, write the residual, pack the codes densely (shuffles and integer
+// multiply-adds).
 //
 // Every stochastic rule compares U (in [0, 1)) with the unsaturated probability p: U < p has
 // the same truth value as U < clamp(p, 0, 1) for every p, NaN included, so no clamp is needed.

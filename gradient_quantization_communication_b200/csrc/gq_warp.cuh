@@ -16,9 +16,10 @@
 //
 // Level fits per bucket:
 //   QSGD / TernGrad : m = max|u|, s uniform levels on [-m, m]
-//   ORQ             : shared-memory histogram of 22-bit fixed-point grid positions (8 columns
-//                     per cell, shared atomics), exact int64 prefix sums, s-2 greedy rounds
-//   BinGrad-b       : warp bitonic sort, exact int64 prefix sums, argmax of J(k)
+//   ORQ             : shared-memory histogram of grid positions with 16 fraction bits (8
+//                     columns per cell, one packed shared atomic per value), exact prefix
+//                     sums, s-2 incremental greedy rounds, per-bracket reciprocal table
+//   BinGrad-b       : warp bitonic sort, exact int64 prefix sums, screened argmax of J(k)
 //   BinGrad-pb      : shared-memory moments of 16-bit positions, exact search of all pairs
 // The last bucket, when ragged, is handled by a one-warp launch of the same code with guarded
 // plain loads, so the main kernel carries no tail logic.
@@ -971,7 +972,7 @@ cudaError_t launch_one(const KParams &p, cudaStream_t stream)
     return cudaSuccess;
 }
 
-// The code width is a template parameter of the main kernel (unrolled bit-plane packing).
+// The code width is a template parameter of the main kernel (packing with constant shifts).
 template <int SCHEME, int EPL, bool FUSED>
 cudaError_t dispatch_bits(const KParams &p, cudaStream_t stream)
 {
