@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--unfused", action="store_true",
+                    help="the unfused path: gq_encode per worker, then gq_decode_accumulate; per-kernel "
+                         "rooflines, one JSON line")
     ap.add_argument("--sweep", action="store_true",
                     help="bucket-size sweep (1e8 elements, W = 8, no error feedback): throughput and "
                          "normalised quantization variance per bucket size, one JSON line")
@@ -439,6 +442,91 @@ def run_cpu_baseline(args, wl, g):
             "sample": "first %d buckets (d=%d) of each of the %d workers, one step" % (nbk, d, wl.workers)}
 
 
+def run_unfused(args):
+    """The step as its separate calls: gq_encode for each worker (fit, round, pack, residual; the
+    message written to HBM), then gq_decode_accumulate over the W messages.  Each launch is
+    timed with events on the launching stream; the line gives the step's throughput and, per
+    kernel kind, the algorithmic bytes per launch over the mean launch time."""
+    import torch
+
+    import gradient_quantization_communication_b200.gq as G
+    from gradient_quantization_communication_b200 import synth
+
+    wl = synth.WORKLOADS[args.workload]
+    if args.elements:
+        wl = dataclasses.replace(wl, n=min(wl.n, args.elements))
+    W, n, d, ef = wl.workers, wl.n, args.bucket, wl.error_feedback
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    sid = G.SCHEMES[args.scheme]
+    cfg = G.gq_config(sid, args.levels, d, W, ef, args.clip, wl.rounding_seed, n)
+    plan = G.Plan(cfg)
+    stream = torch.cuda.current_stream()
+    g = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
+    for w in range(W):
+        synth.gradient(args.workload, w, 0, out=g[w])
+    r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)] if ef else None
+    msgs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)]
+    avg = torch.empty(n, dtype=torch.float32, device=dev)
+
+    def step(t, evs=None):
+        for w in range(W):
+            if evs is not None:
+                evs[w][0].record(stream)
+            G.gq_encode(plan.handle, w, t, g[w], r[w] if ef else None, msgs[w], stream)
+            if evs is not None:
+                evs[w][1].record(stream)
+        if evs is not None:
+            evs[W][0].record(stream)
+        G.gq_decode_accumulate(plan.handle, msgs, avg, stream)
+        if evs is not None:
+            evs[W][1].record(stream)
+
+    for t in range(args.warmup):
+        step(t)
+    torch.cuda.synchronize()
+    if G.gq_plan_status(plan.handle, stream) != G.GQ_OK:
+        raise RuntimeError("non-finite input in the benchmark workload")
+    sampler = ClockSampler(pci_bus_id(dev))
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(W + 1)]
+           for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(args.warmup + k, evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    enc_ms = statistics.mean(a.elapsed_time(b) for e in evs for a, b in e[:W])
+    dec_ms = statistics.mean(e[W][0].elapsed_time(e[W][1]) for e in evs)
+    plan.close()
+    bits = (args.levels - 1).bit_length()
+    L = 1 if sid in (0, 1) else (2 if sid in (2, 3) else args.levels)
+    msg_b = bits / 8.0 + 4.0 * L / d
+    enc_b = 4.0 + (8.0 if ef else 0.0) + msg_b          # per element of one worker
+    dec_b = W * msg_b + 4.0                             # per element of the average
+    peak, peak_kind = measured_hbm_peak()
+
+    def roof(bytes_per_launch, launch_ms):
+        a = bytes_per_launch / (launch_ms / 1000.0) / 1e9
+        return {"bound": "hbm", "achieved": round(a, 1), "peak": peak, "unit": "GB/s", "frac": round(a / peak, 4),
+                "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bytes_per_launch, "ms_per_launch": launch_ms}
+
+    print(json.dumps({
+        "metric": "unfused step: gq_encode x W + gq_decode_accumulate, worker-elements/s", "value": W * n / (ms / 1000.0),
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "f32", "data": "synthetic", "config": workload_config(args, wl),
+        "encode": roof(enc_b * n, enc_ms), "decode": roof(dec_b * n, dec_ms),
+        "bytes": {"encode_per_worker_elem": enc_b, "decode_per_elem": dec_b},
+        "gpu_launches": (W + 1) * args.steps, "clocks": clocks}))
+    return 0
+
+
 def run_sweep(args):
     """Fused-step throughput and normalised quantization variance sum (b-u)(u-a) / sum u^2 for
     every bucket size of the sweep workload, for ORQ-5 and QSGD-5."""
@@ -502,6 +590,8 @@ def main():
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.unfused:
+        return run_unfused(args)
     return run_gq(args)
 
 
