@@ -300,7 +300,7 @@ def run_gq(args):
     stream = torch.cuda.current_stream()
     g = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
     for w in range(W):
-        synth.gradient(args.workload, w, 0, out=g[w])
+        synth.gradient(args.workload, w, 0, n=n, out=g[w])
     r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)] if ef else None
     write_msgs = not args.no_msgs or d > 512
     msgs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)] if write_msgs else None
@@ -464,7 +464,7 @@ def run_unfused(args):
     stream = torch.cuda.current_stream()
     g = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
     for w in range(W):
-        synth.gradient(args.workload, w, 0, out=g[w])
+        synth.gradient(args.workload, w, 0, n=n, out=g[w])
     r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)] if ef else None
     msgs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)]
     avg = torch.empty(n, dtype=torch.float32, device=dev)

@@ -141,6 +141,8 @@ def gradient(workload: str, worker: int, step: int, n: int = None, device="cpu",
     n = wl.n if n is None else int(n)
     if out is None:
         out = torch.empty(n, dtype=torch.float32, device=device)
+    elif out.numel() != n:
+        raise ValueError("out holds %d elements, the request is for %d" % (out.numel(), n))
     device = out.device
     if workload == "gauss64k":
         seed = wl.seeds[worker] if worker < len(wl.seeds) else mix_seed(1, worker, step)
