@@ -5,8 +5,9 @@
 // rounds, packs and writes the residual chunk by chunk (warp k takes the 128-element chunks
 // k, k+8, ...).  Fits:
 //   QSGD / TernGrad : block max of |u|
-//   ORQ             : lane-private histograms per warp, flushed every 16 values per lane into
-//                     a block histogram (shared atomics); warp 0 runs the greedy
+//   ORQ             : per warp, the packed 8-column histogram of the register path (one shared
+//                     atomic per value), reduced every 512 values into the warp's cell totals;
+//                     warp 0 sums the warps' totals and runs the greedy
 //   BinGrad-pb      : block moments per cell (shared atomics), all 2016 pairs searched by
 //                     the 256 threads
 //   BinGrad-b       : block bitonic sort of u in place, exact int64 block scan, argmax of
@@ -86,31 +87,46 @@ __device__ long long block_sum(long long x, CtaShared &sh, int slot)
     return y;
 }
 
-// --- ORQ: lane-private histogram of one warp -> block histogram --------------------------------
-__device__ __forceinline__ void flush_hist(uint32_t *hist, CtaShared &sh, int lane)
+// --- ORQ: per-warp histogram -------------------------------------------------------------------
+// wh[0 .. 511]: [cell][column] words count << 22 | sum of 16-bit fractions (a column sees at most
+// 64 values between reductions); wh[512 .. 575]: the warp's cell counts; wh[576 .. 639]: the
+// warp's cell fraction sums (cell 63, the top grid point, is folded into cell 62 with fraction
+// 2^16).
+constexpr int kWarpHistWords = 64 * 8 + 64 + 64;
+constexpr int kCtaHistShift = 22;
+
+__device__ __forceinline__ void reduce_warp_hist(uint32_t *wh, int lane)
 {
     __syncwarp();
-    uint32_t ca = 0, fa = 0, cb = 0, fb = 0;
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k) {
-        const int col = (lane + k) & 31;
-        const uint32_t xa = hist[lane * 32 + col];
-        const uint32_t xb = hist[(lane + 32) * 32 + col];
-        hist[lane * 32 + col] = 0u;
-        hist[(lane + 32) * 32 + col] = 0u;
-        ca += xa >> 27;
-        fa += xa & 0x7ffffffu;
-        cb += xb >> 27;
-        fb += xb & 0x7ffffffu;
+    uint32_t t0 = 0, t1 = 0, c0 = 0, c1 = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int q4 = (k + (lane >> 1)) & 3;
+        uint4 *ph = reinterpret_cast<uint4 *>(wh + lane * 16) + q4;
+        const uint4 x = *ph;
+        *ph = make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t st = x.x + x.y + x.z + x.w;
+        const uint32_t sc = (x.x >> kCtaHistShift) + (x.y >> kCtaHistShift) + (x.z >> kCtaHistShift) +
+                            (x.w >> kCtaHistShift);
+        if (q4 < 2) {
+            t0 += st;
+            c0 += sc;
+        } else {
+            t1 += st;
+            c1 += sc;
+        }
     }
-    if (ca) {
-        atomicAdd(&sh.ccnt[lane], ca);
-        atomicAdd(&sh.cs1[lane], (unsigned long long)ca * ((unsigned long long)lane << kOrqFBits) + fa);
+    uint32_t f0 = t0 - (c0 << kCtaHistShift), f1 = t1 - (c1 << kCtaHistShift);
+    if (lane == 31) {  // cell 63 -> cell 62, fraction 2^16 each
+        c0 += c1;
+        f0 += c1 << kOrqFBits;
+        c1 = 0u;
+        f1 = 0u;
     }
-    if (cb) {
-        atomicAdd(&sh.ccnt[lane + 32], cb);
-        atomicAdd(&sh.cs1[lane + 32], (unsigned long long)cb * ((unsigned long long)(lane + 32) << kOrqFBits) + fb);
-    }
+    wh[512 + 2 * lane] += c0;
+    wh[512 + 2 * lane + 1] += c1;
+    wh[576 + 2 * lane] += f0;
+    wh[576 + 2 * lane + 1] += f1;
     __syncwarp();
 }
 
@@ -122,12 +138,12 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
     __shared__ CtaShared sh;
     const int d = p.d;
     float *vs = reinterpret_cast<float *>(smem_raw);                      // d floats
-    uint32_t *hist_all = reinterpret_cast<uint32_t *>(smem_raw + (size_t)d * 4);  // ORQ: 8 x 64 x 32
+    uint32_t *hist_all = reinterpret_cast<uint32_t *>(smem_raw + (size_t)d * 4);  // ORQ: 8 warps' histograms
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    uint32_t *hist = hist_all + wid * 64 * 32;
+    uint32_t *wh = hist_all + wid * kWarpHistWords;
 
     if constexpr (SCHEME == GQ_ORQ) {
-        for (int i = lane; i < 64 * 32; i += 32) hist[i] = 0u;
+        for (int i = lane; i < kWarpHistWords; i += 32) wh[i] = 0u;
     }
     for (int i = tid; i < 64; i += kCtaThreads) {
         sh.ccnt[i] = 0u;
@@ -242,7 +258,9 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                 const float step = __fdiv_rn(range, 63.0f);
                 if constexpr (SCHEME == GQ_ORQ) {
                     scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kOrqFBits));
-                    // warp k: chunks k, k+8, ...; flush every 4 chunks (16 values per lane)
+                    // warp k: chunks k, k+8, ...; its histogram is reduced every 4 chunks (16
+                    // values per lane, 64 per column)
+                    const int col = lane & 7;
                     int pending = 0;
                     for (int ch = wid; ch < nchunks; ch += kCtaWarps) {
                         const float4 x = reinterpret_cast<const float4 *>(vs)[ch * 32 + lane];
@@ -252,18 +270,34 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                             const int e = ch * 128 + 4 * lane + c;
                             if (e < nvalid) {
                                 const int ps = grid_pos<kOrqFBits>(clipped(xs[c]), mn, scale);
-                                const int cell = min(ps >> kOrqFBits, kTopCell);
-                                hist[cell * 32 + lane] += (1u << 27) + (uint32_t)(ps - (cell << kOrqFBits));
+                                atomicAdd(&wh[(ps >> kOrqFBits) * 8 + col], (uint32_t)(ps & 0xffff) | (1u << kCtaHistShift));
                             }
                         }
                         if (++pending == 4) {
-                            flush_hist(hist, sh, lane);
+                            reduce_warp_hist(wh, lane);
                             pending = 0;
                         }
                     }
-                    if (pending) flush_hist(hist, sh, lane);
+                    if (pending) reduce_warp_hist(wh, lane);
                     __syncthreads();
                     if (wid == 0) {
+                        // the warps' cell totals -> block histogram (count, sum of positions)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int j = lane + 32 * h;
+                            uint32_t cnt = 0u;
+                            unsigned long long fr = 0ull;
+                            for (int w = 0; w < kCtaWarps; ++w) {
+                                uint32_t *ow = hist_all + w * kWarpHistWords;
+                                cnt += ow[512 + j];
+                                fr += ow[576 + j];
+                                ow[512 + j] = 0u;
+                                ow[576 + j] = 0u;
+                            }
+                            sh.ccnt[j] = cnt;
+                            sh.cs1[j] = (unsigned long long)cnt * ((unsigned long long)j << kOrqFBits) + fr;
+                        }
+                        __syncwarp();
                         const long long c0 = sh.ccnt[lane], c1 = sh.ccnt[lane + 32];
                         const long long s0 = (long long)sh.cs1[lane], s1 = (long long)sh.cs1[lane + 32];
                         const long long ic0 = warp_inclusive_scan(c0, lane), ic1 = warp_inclusive_scan(c1, lane);
@@ -594,7 +628,7 @@ template <int SCHEME, bool ERR>
 cudaError_t launch(const KParams &p, double *part, cudaStream_t stream)
 {
     auto kern = k_cta<SCHEME, ERR>;
-    const size_t smem = (size_t)p.d * 4 + (SCHEME == GQ_ORQ ? (size_t)kCtaWarps * 64 * 32 * 4 : 0);
+    const size_t smem = (size_t)p.d * 4 + (SCHEME == GQ_ORQ ? (size_t)kCtaWarps * kWarpHistWords * 4 : 0);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
