@@ -61,10 +61,11 @@ __device__ __forceinline__ uint4 draws4(const KParams &p, uint64_t blk, uint32_t
     return philox_rounds_2_to_10(y0, (uint32_t)p.step_m1, y2, (uint32_t)p0, p.rk0 + 1, p.rk1 + 1);
 }
 
-// Uniform in [0, 1) at 24-bit resolution from one Philox output word.
+// Uniform in [0, 1) from one Philox output word: the word converted to binary32 rounding toward
+// zero, times 2^-32 (exact).  P(U < p) = ceil(p * 2^32) * 2^-32: exactly p for binary32 p >= 2^-9.
 __device__ __forceinline__ float unit_float(uint32_t word)
 {
-    return __fmul_rn(__uint2float_rn(word >> 8), 0x1p-24f);
+    return __fmul_rn(__uint2float_rz(word), 0x1p-32f);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -250,12 +251,12 @@ __device__ __forceinline__ long long orq_side(int K, int P0K, int P0C, long long
     return (P1C - P1K) - (long long)(K << kOrqFBits) * (long long)(P0C - P0K);
 }
 // Ranking key of candidate C: Delta << 6 | 63 - C (the largest key has the largest Delta, ties
-// to the smallest C).
+// to the smallest C).  With 32-bit sides the shift rides on the small factors: (B-C)*64 and
+// (C-A)*64 are below 2^12, so two 32 x 32 -> 64 multiply-adds give the key exactly (< 2^59).
 __device__ __forceinline__ unsigned long long orq_key(int A, int C, int B, uint32_t lows, uint32_t highs)
 {
-    const unsigned long long delta =
-        (unsigned long long)(uint32_t)(B - C) * lows + (unsigned long long)(uint32_t)(C - A) * highs;
-    return (delta << 6) | (unsigned long long)(63 - C);
+    return (unsigned long long)((uint32_t)(B - C) << 6) * lows +
+           ((unsigned long long)((uint32_t)(C - A) << 6) * highs + (unsigned long long)(63 - C));
 }
 __device__ __forceinline__ unsigned long long orq_key(int A, int C, int B, long long lows, long long highs)
 {
@@ -301,24 +302,19 @@ __device__ __forceinline__ unsigned long long orq_greedy(const int *P0, const T 
         const T P1L = P1[L];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
+            // branch-free: the split bracket's candidates take L as one neighbour and side(L, C)
+            // as that side; the chosen index itself gets key 0 and the empty bracket
             const int C = lane + 32 * h;
-            if (A[h] < L && L < B[h]) {
-                if (C == L) {  // the chosen index: key 0, empty bracket
-                    A[h] = C;
-                    B[h] = C;
-                    key[h] = 0ull;
-                } else {
-                    const T x = orq_side(L, P0L, P0C[h], P1L, P1C[h]);
-                    if (L < C) {
-                        A[h] = L;
-                        lows[h] = x;
-                    } else {
-                        B[h] = L;
-                        highs[h] = x;
-                    }
-                    key[h] = orq_key(A[h], C, B[h], lows[h], highs[h]);
-                }
-            }
+            const bool split = A[h] < L && L < B[h];
+            const bool self = C == L;
+            const bool below = L < C;
+            const T x = orq_side(L, P0L, P0C[h], P1L, P1C[h]);
+            A[h] = split ? (self ? C : (below ? L : A[h])) : A[h];
+            B[h] = split ? (self ? C : (below ? B[h] : L)) : B[h];
+            lows[h] = (split && below) ? x : lows[h];
+            highs[h] = (split && !below && !self) ? x : highs[h];
+            const unsigned long long nk = orq_key(A[h], C, B[h], lows[h], highs[h]);
+            key[h] = split ? (self ? 0ull : nk) : key[h];
         }
     }
     return mask;

@@ -144,7 +144,8 @@ __device__ __forceinline__ void flag_nonfinite(const KParams &p, int lane)
 // ORQ tables from the chosen grid indices (mask, s bits): the level table of the message, the
 // bracket table (one entry per pair of adjacent levels) and the per-cell bracket table the
 // rounding pass reads (cell j lies in bracket k = #{chosen indices <= j} - 1; cell 63, the top
-// grid point, in bracket s - 2 like cell 62).
+// grid point, in bracket s - 2 like cell 62).  IO bit 1: the message buffer is known present.
+template <int IO>
 __device__ __forceinline__ void build_orq_tables(const KParams &p, FitORQ &sm, int w, int64_t beta, int lane,
                                                  unsigned long long mask, float mn, float mx, float step)
 {
@@ -152,18 +153,17 @@ __device__ __forceinline__ void build_orq_tables(const KParams &p, FitORQ &sm, i
     const uint32_t lt = (1u << lane) - 1u, le = lt | (1u << lane);
     const int nlo = __popc(mlo);
     unsigned char *msg = p.msg[w];
-    float *mtab = msg ? reinterpret_cast<float *>(msg + p.levels_off) + beta * p.L : nullptr;
-    if ((mlo >> lane) & 1u) {
-        const float lv = grid_point(mn, mx, step, lane);
-        const int rank = __popc(mlo & lt);
-        sm.lev[rank] = lv;
-        if (mtab) mtab[rank] = lv;
-    }
-    if ((mhi >> lane) & 1u) {
-        const float lv = grid_point(mn, mx, step, lane + 32);
-        const int rank = nlo + __popc(mhi & lt);
-        sm.lev[rank] = lv;
-        if (mtab) mtab[rank] = lv;
+    float *mtab = ((IO & 2) || msg) ? reinterpret_cast<float *>(msg + p.levels_off) + beta * p.L : nullptr;
+    // lanes own grid indices lane and lane + 32; a chosen one stores its level at its rank
+    const bool ch0 = (mlo >> lane) & 1u, ch1 = (mhi >> lane) & 1u;
+    const int r0 = __popc(mlo & lt), r1 = nlo + __popc(mhi & lt);
+    const float lv0 = __fadd_rn(mn, __fmul_rn((float)lane, step));
+    const float lv1 = lane == 31 ? mx : __fadd_rn(mn, __fmul_rn((float)(lane + 32), step));
+    if (ch0) sm.lev[r0] = lv0;
+    if (ch1) sm.lev[r1] = lv1;
+    if ((IO & 2) || mtab) {
+        if (ch0) mtab[r0] = lv0;
+        if (ch1) mtab[r1] = lv1;
     }
     __syncwarp();
     if (lane < p.s - 1) {
@@ -303,7 +303,7 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     reinterpret_cast<uint2 *>(sm.P1)[lane] = make_uint2(es, es + s0);
     __syncwarp();
     const unsigned long long mask = orq_greedy(sm.P0, sm.P1, p.s, lane);
-    build_orq_tables(p, sm, w, beta, lane, mask, mn, mx, step);
+    build_orq_tables<IO>(p, sm, w, beta, lane, mask, mn, mx, step);
     emit<EPL, FUSED, true, TAIL, BITS, IO>(p, RoundORQ{sm.ctab}, beta, w, lane, vmask, v, u, pos, acc, ea);
     __syncwarp();
 }
