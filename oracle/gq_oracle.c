@@ -66,8 +66,19 @@ void or_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out
  * only ask for random rounding; the draw is keyed on (seed, step, worker, global element
  * index) so that it is reproducible and independent of the launch shape.  Reading: key =
  * (seed low word, seed high word), counter = (i/4 low word, i/4 high word, step low word,
- * worker); element i takes output word i mod 4; U = (word >> 8) * 2^-24.
+ * worker); element i takes output word i mod 4; U = rz(word) * 2^-32, rz(word) the largest
+ * binary32 value not above the word (its 24 leading significant bits).  Then
+ * P(U < p) = ceil(p * 2^32) * 2^-32 for every p in [0, 1]: exactly p for every binary32 p
+ * >= 2^-9, within 2^-32 below that, which is what keeps the rounding unbiased ([P3]).
  */
+static float uniform_from_word(uint32_t word)
+{
+    int len = 0;
+    for (uint32_t t = word; t; t >>= 1) ++len;
+    if (len > 24) word &= ~((1u << (len - 24)) - 1u); /* keep the 24 leading significant bits */
+    return (float)word * 0x1p-32f;                     /* exact: at most 24 significant bits */
+}
+
 float or_uniform(uint64_t seed, uint64_t step, uint32_t worker, int64_t i)
 {
     uint64_t blk = (uint64_t)i >> 2;
@@ -76,7 +87,7 @@ float or_uniform(uint64_t seed, uint64_t step, uint32_t worker, int64_t i)
     uint32_t out[4];
     or_philox4x32_10(ctr, key, out);
     uint32_t word = out[(uint64_t)i & 3u];
-    return (float)(word >> 8) * 0x1p-24f;
+    return uniform_from_word(word);
 }
 
 /* floor(log2(m)) for finite m > 0, read from the binary32 encoding. */

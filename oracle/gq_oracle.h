@@ -41,7 +41,8 @@ typedef struct {
 
 /* Philox4x32-10 block function (Salmon, Moraes, Dror, Shaw, SC'11). */
 void or_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
-/* The uniform in [0,1) drawn for global element index i (24-bit resolution). */
+/* The uniform in [0,1) drawn for global element index i: the Philox word rounded toward zero to
+ * binary32, times 2^-32. */
 float or_uniform(uint64_t seed, uint64_t step, uint32_t worker, int64_t i);
 
 /* floor(log2(m)) for finite m > 0, subnormals included. */

@@ -36,7 +36,7 @@ MUTATIONS = [
     ("grid_step", "gi->step = range / 63.0f;", "gi->step = range / 64.0f;"),
     ("average_scale", "float inv_w = 1.0f / (float)nmsgs;", "float inv_w = 1.0f / (float)(nmsgs + 1);"),
     ("residual_sign", "r[base + i] = v[i] - q[i];", "r[base + i] = q[i] - v[i];"),
-    ("uniform_bits", "return (float)(word >> 8) * 0x1p-24f;", "return (float)(word >> 9) * 0x1p-24f;"),
+    ("uniform_bits", "if (len > 24) word &= ~((1u << (len - 24)) - 1u);", "if (len > 23) word &= ~((1u << (len - 23)) - 1u);"),
     ("pack_padding", "memset(words, 0, sizeof(uint32_t) * (size_t)(d * b / 32));",
      "memset(words, 0xff, sizeof(uint32_t) * (size_t)(d * b / 32));"),
     ("pack_bit_order", "if ((code[e] >> j) & 1) words[k / 32] |= 1u << (k % 32);",

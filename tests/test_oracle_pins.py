@@ -34,7 +34,7 @@ def test_philox_known_answers():
 
 
 def test_uniform_statistics():
-    # 2^16 draws: mean 1/2, chi-square over 64 bins, 24-bit resolution
+    # 2^16 draws: mean 1/2, chi-square over 64 bins, round-toward-zero conversion of the word
     n = 1 << 16
     u = np.array([O.uniform(7, 3, 1, i) for i in range(n)], dtype=np.float64)
     assert u.min() >= 0.0 and u.max() < 1.0
@@ -42,7 +42,15 @@ def test_uniform_statistics():
     h, _ = np.histogram(u, bins=64, range=(0, 1))
     chi2 = ((h - n / 64) ** 2 / (n / 64)).sum()
     assert chi2 < 63 + 6 * math.sqrt(2 * 63)
-    assert np.all(np.round(u * 2 ** 24) == u * 2 ** 24)
+    # U * 2^32 is the binary32 value just at or below the generator's word (round toward zero)
+    words = []
+    for b in range(n // 4):
+        words.extend(int(x) for x in O.philox([b, 0, 3, 1], [7, 0]))
+    w = np.array(words[:n], dtype=np.float64)
+    x = (u * 2.0 ** 32).astype(np.float32)
+    assert np.all(x.astype(np.float64) == u * 2.0 ** 32)
+    assert np.all(x.astype(np.float64) <= w)
+    assert np.all(np.nextafter(x, np.float32(np.inf)).astype(np.float64) > w)
     # distinct workers / steps give distinct streams
     a = [O.uniform(7, 3, 1, i) for i in range(64)]
     b = [O.uniform(7, 3, 2, i) for i in range(64)]
