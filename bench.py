@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--unfused", action="store_true",
                     help="the unfused path: gq_encode per worker, then gq_decode_accumulate; per-kernel "
                          "rooflines, one JSON line")
