@@ -6,6 +6,8 @@
 #include <cstring>
 #include <new>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "gq_internal.h"
 
 struct gq_plan {
@@ -121,6 +123,13 @@ gq_status_t check_device(const gq_plan &pl)
 
 gq_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GQ_OK : GQ_ERR_CUDA; }
 
+// NVTX range around an entry point (free when no profiler is attached): shows the call on the
+// host timeline next to the kernels it enqueues.
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+};
+
 }  // namespace
 
 extern "C" {
@@ -185,6 +194,7 @@ gq_status_t gq_plan_destroy(gq_plan_t plan)
 gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, float *residual, void *msg,
                       void *stream)
 {
+    Range range("gq_encode");
     if (!plan) return GQ_ERR_INVALID;
     if (plan->cfg.n == 0) return GQ_OK;  // nothing to read or write: pointers may be NULL
     if (!grad || !msg || !aligned16(grad) || !aligned16(msg)) return GQ_ERR_INVALID;
@@ -204,6 +214,7 @@ gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const floa
 
 gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs, int nmsgs, float *avg, void *stream)
 {
+    Range range("gq_decode_accumulate");
     if (!plan || nmsgs < 1 || nmsgs > GQ_MAX_WORKERS) return GQ_ERR_INVALID;
     if (plan->cfg.n == 0) return GQ_OK;  // nothing to read or write: pointers may be NULL
     if (!msgs || !avg || !aligned16(avg)) return GQ_ERR_INVALID;
@@ -222,6 +233,7 @@ gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs, int nm
 gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *grads, float *const *residuals,
                           void *const *msgs, float *avg, void *stream)
 {
+    Range range("gq_fused_step");
     if (!plan) return GQ_ERR_INVALID;
     if (plan->cfg.n == 0) return GQ_OK;  // nothing to read or write: pointers may be NULL
     if (!grads || !avg || !aligned16(avg)) return GQ_ERR_INVALID;
@@ -269,6 +281,7 @@ gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *gra
 gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, const float *residual,
                            double *out, void *stream)
 {
+    Range range("gq_quant_error");
     if (!plan || !out) return GQ_ERR_INVALID;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (plan->cfg.n == 0) return from_cuda(cudaMemsetAsync(out, 0, 3 * sizeof(double), s));
@@ -287,6 +300,15 @@ gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step, const
     return from_cuda(gq::launch_err_reduce(part, plan->nb, part + 3 * plan->nb, out, s));
 }
 
+gq_status_t gq_selftest_bounded_wait(gq_plan_t plan, int64_t limit_ns, void *stream)
+{
+    if (!plan) return GQ_ERR_INVALID;
+    const gq_status_t st = check_device(*plan);
+    if (st != GQ_OK) return st;
+    const int64_t lim = limit_ns < 1000000 ? 1000000 : (limit_ns > 1000000000 ? 1000000000 : limit_ns);
+    return from_cuda(gq::launch_wait_selftest(plan->status, (unsigned long long)lim, static_cast<cudaStream_t>(stream)));
+}
+
 gq_status_t gq_plan_status(gq_plan_t plan, void *stream)
 {
     if (!plan) return GQ_ERR_INVALID;
@@ -295,7 +317,7 @@ gq_status_t gq_plan_status(gq_plan_t plan, void *stream)
     if (cudaMemcpyAsync(&flags, plan->status, sizeof flags, cudaMemcpyDeviceToHost, s) != cudaSuccess) return GQ_ERR_CUDA;
     if (cudaMemsetAsync(plan->status, 0, sizeof(unsigned int), s) != cudaSuccess) return GQ_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return GQ_ERR_CUDA;
-    if (flags & gq::kStatusTimeout) return GQ_ERR_CUDA;
+    if (flags & gq::kStatusTimeout) return GQ_ERR_TIMEOUT;
     if (flags & gq::kStatusNonFinite) return GQ_ERR_NONFINITE;
     return GQ_OK;
 }
@@ -309,6 +331,7 @@ const char *gq_status_string(gq_status_t status)
     case GQ_ERR_CUDA: return "CUDA error";
     case GQ_ERR_NONFINITE: return "non-finite input value";
     case GQ_ERR_NOMEM: return "out of host memory";
+    case GQ_ERR_TIMEOUT: return "a bounded wait for a bulk copy timed out";
     }
     return "unknown status";
 }

@@ -390,13 +390,14 @@ __device__ __forceinline__ unsigned long long global_ns()
 }
 
 // Warp-uniform bounded wait for the phase `parity` of `bar`; false if it timed out.
-__device__ __forceinline__ bool mbar_wait_warp(unsigned long long *bar, unsigned parity)
+__device__ __forceinline__ bool mbar_wait_warp(unsigned long long *bar, unsigned parity,
+                                               unsigned long long limit_ns = kWaitLimitNs)
 {
     if (__all_sync(kFull, mbar_try_wait(bar, parity))) return true;
     const unsigned long long t0 = global_ns();
     for (;;) {
         if (__all_sync(kFull, mbar_try_wait(bar, parity))) return true;
-        const bool late = global_ns() - t0 > kWaitLimitNs;
+        const bool late = global_ns() - t0 > limit_ns;
         if (__any_sync(kFull, late)) return false;
     }
 }

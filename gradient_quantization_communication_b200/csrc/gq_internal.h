@@ -58,5 +58,8 @@ cudaError_t launch_warp_err(const KParams &p, double *part, cudaStream_t stream)
 cudaError_t launch_cta_err(const KParams &p, double *part, cudaStream_t stream);
 int64_t err_scratch_doubles(int64_t nb);
 cudaError_t launch_err_reduce(const double *part, int64_t nb, double *tmp, double *out, cudaStream_t stream);
+// One warp waiting, with the kernels' bounded wait, on a barrier that nothing completes; raises
+// kStatusTimeout in *status after limit_ns.
+cudaError_t launch_wait_selftest(unsigned int *status, unsigned long long limit_ns, cudaStream_t stream);
 
 }  // namespace gq

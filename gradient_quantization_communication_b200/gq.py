@@ -11,7 +11,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgq.so")
 
 GQ_QSGD, GQ_TERNGRAD, GQ_BINGRAD_B, GQ_BINGRAD_PB, GQ_ORQ = 0, 1, 2, 3, 4
-GQ_OK, GQ_ERR_INVALID, GQ_ERR_UNSUPPORTED, GQ_ERR_CUDA, GQ_ERR_NONFINITE, GQ_ERR_NOMEM = 0, 1, 2, 3, 4, 5
+GQ_OK, GQ_ERR_INVALID, GQ_ERR_UNSUPPORTED, GQ_ERR_CUDA, GQ_ERR_NONFINITE, GQ_ERR_NOMEM, GQ_ERR_TIMEOUT = 0, 1, 2, 3, 4, 5, 6
 GQ_MAX_WORKERS = 64
 SCHEMES = {"qsgd": GQ_QSGD, "terngrad": GQ_TERNGRAD, "bingrad_b": GQ_BINGRAD_B,
            "bingrad_pb": GQ_BINGRAD_PB, "orq": GQ_ORQ}
@@ -53,12 +53,13 @@ def lib():
         L.gq_quant_error.argtypes = [vp, ctypes.c_uint32, ctypes.c_uint64, vp, vp, vp, vp]
         L.gq_quant_error_noalloc.argtypes = [cfgp, ctypes.c_uint32, ctypes.c_uint64, vp, vp, vp, vp]
         L.gq_plan_status.argtypes = [vp, vp]
+        L.gq_selftest_bounded_wait.argtypes = [vp, ctypes.c_int64, vp]
         L.gq_status_string.argtypes = [ctypes.c_int]
         L.gq_status_string.restype = ctypes.c_char_p
         L.gq_version.restype = ctypes.c_char_p
         for f in ("gq_config_check", "gq_message_layout", "gq_plan_create", "gq_plan_destroy", "gq_encode",
                   "gq_decode_accumulate", "gq_fused_step", "gq_quant_error", "gq_quant_error_noalloc",
-                  "gq_plan_status"):
+                  "gq_plan_status", "gq_selftest_bounded_wait"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -151,6 +152,10 @@ def gq_quant_error_noalloc(cfg, worker, step, grad, residual, out, stream=None):
 
 def gq_plan_status(plan, stream=None):
     return lib().gq_plan_status(plan, _stream(stream))
+
+
+def gq_selftest_bounded_wait(plan, limit_ns, stream=None):
+    _check(lib().gq_selftest_bounded_wait(plan, int(limit_ns), _stream(stream)), "gq_selftest_bounded_wait")
 
 
 def gq_status_string(status):

@@ -62,7 +62,8 @@ typedef enum {
     GQ_ERR_UNSUPPORTED = 2, /* a valid combination this build does not implement */
     GQ_ERR_CUDA = 3,        /* a CUDA call failed (launch, allocation of the plan's status word) */
     GQ_ERR_NONFINITE = 4,   /* gq_plan_status: some input value was NaN or infinite */
-    GQ_ERR_NOMEM = 5        /* host allocation failed */
+    GQ_ERR_NOMEM = 5,       /* host allocation failed */
+    GQ_ERR_TIMEOUT = 6      /* gq_plan_status: a kernel's bounded wait for a bulk copy gave up */
 } gq_status_t;
 
 /*
@@ -190,9 +191,19 @@ GQ_API gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step
 GQ_API gq_status_t gq_quant_error_noalloc(const gq_config_t *cfg, uint32_t worker, uint64_t step, const float *grad,
                                           const float *residual, double *out, void *stream);
 
-/* Synchronize `stream`, then report and clear the plan's status flags: GQ_ERR_NONFINITE if
- * a non-finite input was seen since the last call, GQ_ERR_CUDA if the stream failed. */
+/* Synchronize `stream`, then report and clear the plan's status flags: GQ_ERR_TIMEOUT if a
+ * kernel's bounded wait for a bulk copy gave up (the kernel then stopped early; its outputs are
+ * incomplete), else GQ_ERR_NONFINITE if a non-finite input was seen since the last call;
+ * GQ_ERR_CUDA if the stream failed. */
 GQ_API gq_status_t gq_plan_status(gq_plan_t plan, void *stream);
+
+/* Self-test of the failure path, no counterpart in the pages: every wait of the kernels for a
+ * bulk copy is bounded in time and, when it gives up, raises the plan's timeout flag instead of
+ * hanging.  This call enqueues one warp that waits, with the same bounded wait, on a barrier
+ * that nothing completes; after limit_ns nanoseconds (clamped to [1e6, 1e9]) it raises the flag
+ * and exits.  gq_plan_status then returns GQ_ERR_TIMEOUT, and the plan and the context stay
+ * usable.  Returns GQ_ERR_INVALID for a NULL plan, GQ_ERR_CUDA if the launch fails. */
+GQ_API gq_status_t gq_selftest_bounded_wait(gq_plan_t plan, int64_t limit_ns, void *stream);
 
 /* Static description of a status code. */
 GQ_API const char *gq_status_string(gq_status_t status);
