@@ -165,12 +165,6 @@ __device__ __forceinline__ float warp_max_nan(float x)
     for (int o = 16; o > 0; o >>= 1) x = fmax_nan(x, __shfl_xor_sync(kFull, x, o));
     return x;
 }
-__device__ __forceinline__ float warp_min_nan(float x)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fmin_nan(x, __shfl_xor_sync(kFull, x, o));
-    return x;
-}
 // Order-preserving map of binary32 onto int32 (NaN of either sign lands beyond +-inf, so a
 // NaN anywhere surfaces in the max or the min): lets a single REDUX find a float min / max.
 __device__ __forceinline__ int float_key(float f)
@@ -190,15 +184,6 @@ __device__ __forceinline__ long long warp_sum(long long x)
 {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
-    return x;
-}
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long y = __shfl_xor_sync(kFull, x, o);
-        x = y > x ? y : x;
-    }
     return x;
 }
 // Inclusive prefix sum over lanes.
