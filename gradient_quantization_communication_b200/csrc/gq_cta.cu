@@ -23,7 +23,7 @@ constexpr int kCtaWarps = 8;
 constexpr int kCtaThreads = kCtaWarps * 32;
 
 struct alignas(16) CtaShared {
-    float redf[2][kCtaWarps];
+    float redf[3][kCtaWarps];
     long long redl[3][kCtaWarps];
     double redd[kCtaWarps];
     double rede[3][kCtaWarps];
@@ -64,17 +64,6 @@ __device__ float block_min(float x, CtaShared &sh, int slot)
     __syncthreads();
     return y;
 }
-__device__ float block_max_nan(float x, CtaShared &sh, int slot)
-{
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    x = warp_max_nan(x);
-    if (lane == 0) sh.redf[slot][wid] = x;
-    __syncthreads();
-    float y = sh.redf[slot][lane & (kCtaWarps - 1)];
-    y = warp_max_nan(y);
-    __syncthreads();
-    return y;
-}
 __device__ long long block_sum(long long x, CtaShared &sh, int slot)
 {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -85,6 +74,25 @@ __device__ long long block_sum(long long x, CtaShared &sh, int slot)
     y = warp_sum(y);
     __syncthreads();
     return y;
+}
+
+// The three staging statistics in one exchange: NaN-propagating max |v|, min v and max v.
+__device__ void block_stats(float &am, float &lo, float &hi, CtaShared &sh)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    am = warp_redux_max_abs(am);
+    lo = warp_redux_min(lo);
+    hi = warp_redux_max(hi);
+    if (lane == 0) {
+        sh.redf[0][wid] = am;
+        sh.redf[1][wid] = lo;
+        sh.redf[2][wid] = hi;
+    }
+    __syncthreads();
+    am = warp_redux_max_abs(sh.redf[0][lane & (kCtaWarps - 1)]);
+    lo = warp_redux_min(sh.redf[1][lane & (kCtaWarps - 1)]);
+    hi = warp_redux_max(sh.redf[2][lane & (kCtaWarps - 1)]);
+    __syncthreads();
 }
 
 // --- ORQ: per-warp histogram -------------------------------------------------------------------
@@ -162,8 +170,8 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
     for (int64_t beta = blockIdx.x; beta < p.nb; beta += gridDim.x) {
         const int64_t base = beta * (int64_t)d;
         const int nvalid = (beta == p.nb - 1) ? p.tail : d;
-        // ---- stage v = g + r in shared memory; NaN-propagating max |v| --------------------------
-        float am = 0.0f;
+        // ---- stage v = g + r in shared memory; NaN-propagating max |v|, min v, max v ------------
+        float am = 0.0f, vlo = INFINITY, vhi = -INFINITY;
         for (int i4 = tid; i4 < (d >> 2); i4 += kCtaThreads) {
             const int e = 4 * i4;
             float4 x;
@@ -177,6 +185,8 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                     x.w = __fadd_rn(x.w, y.w);
                 }
                 am = fmax_nan(am, fmax_nan(fmax_nan(fabsf(x.x), fabsf(x.y)), fmax_nan(fabsf(x.z), fabsf(x.w))));
+                vlo = fmin3_nan(vlo, fmin3_nan(x.x, x.y, x.z), x.w);
+                vhi = fmax3_nan(vhi, fmax3_nan(x.x, x.y, x.z), x.w);
             } else {
                 float t[4];
 #pragma unroll
@@ -186,13 +196,15 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                         t[c] = g[base + e + c];
                         if (r) t[c] = __fadd_rn(t[c], r[base + e + c]);
                         am = fmax_nan(am, fabsf(t[c]));
+                        vlo = fmin_nan(vlo, t[c]);
+                        vhi = fmax_nan(vhi, t[c]);
                     }
                 }
                 x = make_float4(t[0], t[1], t[2], t[3]);
             }
             reinterpret_cast<float4 *>(vs)[i4] = x;
         }
-        am = block_max_nan(am, sh, 0);
+        block_stats(am, vlo, vhi, sh);
         if (!(am <= FLT_MAX) && tid == 0) atomicOr(p.status, kStatusNonFinite);
 
         // ---- clip threshold ---------------------------------------------------------------------
@@ -228,9 +240,12 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
         bool constant = false;
         float mn = 0.0f, mx = 0.0f, scale = 0.0f;
         if constexpr (SCHEME == GQ_QSGD) {
-            float m = 0.0f;
-            for (int i = tid; i < nvalid; i += kCtaThreads) m = fmaxf(m, fabsf(clipped(vs[i])));
-            m = block_max(m, sh, 0);
+            float m = am;  // without clipping u = v
+            if (clip) {
+                m = 0.0f;
+                for (int i = tid; i < nvalid; i += kCtaThreads) m = fmaxf(m, fabsf(clipped(vs[i])));
+                m = block_max(m, sh, 0);
+            }
             const int s = p.s;
             if (wid == 0) {
                 const float lv = lane < s ? __fmul_rn(m, p.qratio[lane]) : 0.0f;
@@ -244,14 +259,20 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
             rq.kmax = s - 2;
             rq.pair = sh.pair;
         } else if constexpr (SCHEME == GQ_ORQ || SCHEME == GQ_BINGRAD_PB) {
-            float lo = INFINITY, hi = -INFINITY;
-            for (int i = tid; i < nvalid; i += kCtaThreads) {
-                const float x = clipped(vs[i]);
-                lo = fminf(lo, x);
-                hi = fmaxf(hi, x);
+            float lo = vlo, hi = vhi;  // without clipping u = v
+            if (clip) {
+                lo = INFINITY;
+                hi = -INFINITY;
+                for (int i = tid; i < nvalid; i += kCtaThreads) {
+                    const float x = clipped(vs[i]);
+                    lo = fminf(lo, x);
+                    hi = fmaxf(hi, x);
+                }
+                lo = block_min(lo, sh, 0);
+                hi = block_max(hi, sh, 1);
             }
-            mn = __fadd_rn(block_min(lo, sh, 0), 0.0f);
-            mx = __fadd_rn(block_max(hi, sh, 1), 0.0f);
+            mn = __fadd_rn(lo, 0.0f);
+            mx = __fadd_rn(hi, 0.0f);
             constant = !(mx > mn);
             if (!constant) {
                 const float range = __fsub_rn(mx, mn);
@@ -426,9 +447,12 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                 }
             }
         } else {  // BinGrad-b
-            float m = 0.0f;
-            for (int i = tid; i < nvalid; i += kCtaThreads) m = fmaxf(m, fabsf(clipped(vs[i])));
-            m = block_max(m, sh, 0);
+            float m = am;  // without clipping u = v
+            if (clip) {
+                m = 0.0f;
+                for (int i = tid; i < nvalid; i += kCtaThreads) m = fmaxf(m, fabsf(clipped(vs[i])));
+                m = block_max(m, sh, 0);
+            }
             if (m > 0.0f) {
                 // sort u in place (padding = +inf)
                 for (int i = tid; i < d; i += kCtaThreads) vs[i] = i < nvalid ? clipped(vs[i]) : INFINITY;

@@ -159,12 +159,6 @@ __device__ __forceinline__ float warp_min(float x)
     for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(kFull, x, o));
     return x;
 }
-__device__ __forceinline__ float warp_max_nan(float x)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fmax_nan(x, __shfl_xor_sync(kFull, x, o));
-    return x;
-}
 // Order-preserving map of binary32 onto int32 (NaN of either sign lands beyond +-inf, so a
 // NaN anywhere surfaces in the max or the min): lets a single REDUX find a float min / max.
 __device__ __forceinline__ int float_key(float f)
