@@ -305,7 +305,9 @@ def run_gq(args):
     write_msgs = not args.no_msgs or d > 512
     msgs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)] if write_msgs else None
     avg = torch.empty(n, dtype=torch.float32, device=dev)
-    launches_per_step = 1 if d <= 512 else W + 1
+    # d <= 512: the fused kernel over the full buckets, plus one launch for a ragged last bucket;
+    # d > 512: one encode per worker, then the decode
+    launches_per_step = ((1 if n >= d else 0) + (1 if n % d else 0)) if d <= 512 else W + 1
 
     def step(t):
         G.gq_fused_step(plan.handle, t, g, r, msgs, avg, stream)
