@@ -383,30 +383,62 @@ def run_gq(args):
     return 0
 
 
+def all_ranks_min(x, device):
+    """The smallest of the ranks' values (every rank gets it); the value itself when alone."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return t.item()
+
+
+def e2e_host_mode(W, n, avail, local_world):
+    """Pinned host buffers the e2e leg can afford: 2 = one per worker plus the average,
+    1 = one gradient buffer copied into every worker's device gradient plus the average (the same
+    bytes cross PCIe every step), 0 = none.  The local ranks share the host's memory."""
+    if avail is None:
+        return 2
+    budget = avail / (1.5 * max(1, local_world))
+    if 4 * (W + 1) * n <= budget:
+        return 2
+    if 8 * n <= budget:
+        return 1
+    return 0
+
+
 def run_e2e(args, G, plan, W, n, g, r, msgs, avg, dev, stream, world):
     """The same step through the C ABI with the gradients in pinned host memory: every step
-    copies the W gradients host -> device, runs gq_fused_step and reads the average back."""
+    copies the W gradients host -> device, runs gq_fused_step and reads the average back.  All
+    ranks take the same decisions (and so the same collective calls) whatever their memory."""
     import torch
-    need = 4 * (W + 1) * n
     try:
         with open("/proc/meminfo") as f:
             avail = 1024 * int(next(ln for ln in f if ln.startswith("MemAvailable")).split()[1])
     except Exception:
         avail = None
-    if avail is not None and avail < 1.5 * need:
-        return {"value": None, "unit": UNIT, "error": "host memory: %d GB available, %d GB of pinned buffers needed"
-                % (avail >> 30, need >> 30)}
+    local_world = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+    mode = int(all_ranks_min(e2e_host_mode(W, n, avail, local_world), dev))
+    if mode == 0:
+        return {"value": None, "unit": UNIT, "error": "host memory: %s GB available for %d local ranks"
+                % ("?" if avail is None else avail >> 30, local_world)}
+    host_g, host_avg = [], None
     try:
-        host_g = [torch.empty(n, dtype=torch.float32, pin_memory=True) for _ in range(W)]
+        host_g = [torch.empty(n, dtype=torch.float32, pin_memory=True) for _ in range(W if mode == 2 else 1)]
         host_avg = torch.empty(n, dtype=torch.float32, pin_memory=True)
-    except Exception as e:  # host memory
-        return {"value": None, "unit": UNIT, "error": "pinned host allocation failed: %s" % str(e)[:80]}
-    for w in range(W):
-        host_g[w].copy_(g[w])
+        ok = 1
+    except Exception:
+        ok = 0
+    if all_ranks_min(ok, dev) < 1:
+        del host_g, host_avg
+        return {"value": None, "unit": UNIT, "error": "pinned host allocation failed on some rank"}
+    for i, hg in enumerate(host_g):
+        hg.copy_(g[i])
 
     def step(t):
         for w in range(W):
-            g[w].copy_(host_g[w], non_blocking=True)
+            g[w].copy_(host_g[w if mode == 2 else 0], non_blocking=True)
         G.gq_fused_step(plan.handle, 1000 + t, g, r, msgs, avg, stream)
         host_avg.copy_(avg, non_blocking=True)
 
@@ -424,7 +456,9 @@ def run_e2e(args, G, plan, W, n, g, r, msgs, avg, dev, stream, world):
         ms = max_over_ranks(ms, dev)
     del host_g, host_avg
     return {"value": world * W * n * args.e2e_steps / (ms / 1000.0), "unit": UNIT,
-            "h2d_bytes_per_step": 4 * W * n, "d2h_bytes_per_step": 4 * n, "steps": args.e2e_steps}
+            "h2d_bytes_per_step": 4 * W * n, "d2h_bytes_per_step": 4 * n, "steps": args.e2e_steps,
+            "host_gradients": "one pinned buffer per worker" if mode == 2 else
+            "one pinned buffer copied into every worker's gradient (host memory shared by %d ranks)" % local_world}
 
 
 def run_cpu_baseline(args, wl, g):

@@ -35,8 +35,10 @@ def _rank_main(rank, world, port, out):
     try:
         elapsed = bench.max_over_ranks(100.0 + 25.0 * rank, torch.device("cpu"))
         value = bench.job_value(world, 8, 1000, 10, elapsed)
+        # the e2e leg's host-buffer mode: every rank takes the smallest mode any rank can afford
+        mode = bench.all_ranks_min(2 - rank, torch.device("cpu"))
         with open(os.path.join(out, "rank%d.json" % rank), "w") as f:
-            json.dump({"elapsed": elapsed, "value": value}, f)
+            json.dump({"elapsed": elapsed, "value": value, "mode": mode}, f)
     finally:
         dist.destroy_process_group()
 
@@ -48,6 +50,16 @@ def test_max_over_ranks_and_job_value(tmp_path):
     for g in got:
         assert g["elapsed"] == 125.0  # the slower rank's time, on every rank
         assert abs(g["value"] - world * 8 * 1000 * 10 / 0.125) < 1e-6
+        assert g["mode"] == 1  # both ranks agree on the mode the poorer rank can afford
+
+
+def test_e2e_host_mode():
+    import bench
+    W, n = 8, 10 ** 9
+    assert bench.e2e_host_mode(W, n, None, 1) == 2
+    assert bench.e2e_host_mode(W, n, 196 << 30, 1) == 2  # 36 GB of pinned buffers for one rank
+    assert bench.e2e_host_mode(W, n, 196 << 30, 8) == 1  # eight ranks share the host: 8 GB each
+    assert bench.e2e_host_mode(W, n, 20 << 30, 8) == 0
 
 
 def test_reference_arm_two_ranks():
