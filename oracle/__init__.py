@@ -77,6 +77,12 @@ def lib():
         L.or_fused_step.argtypes = [P(_Cfg), ctypes.c_uint64, i64, i64, P(f32p), P(f32p), P(u8p), f32p]
         L.or_quant_error.argtypes = [P(_Cfg), ctypes.c_int, ctypes.c_uint64, i64, i64, f32p, f32p,
                                      P(ctypes.c_double)]
+        L.or_entropy_groups.argtypes = [ctypes.c_int, i32p, i32p]
+        L.or_entropy_words.argtypes = [P(_Cfg)]
+        L.or_entropy_words.restype = i64
+        L.or_entropy_layout.argtypes = [P(_Cfg), P(i64), P(i64), P(i64)]
+        L.or_entropy_pack.argtypes = [P(_Cfg), u8p, u8p]
+        L.or_entropy_unpack.argtypes = [P(_Cfg), u8p, u8p]
         L.or_fused_bucket.argtypes = [P(_Cfg), ctypes.c_uint64, i64, ctypes.c_int, P(f32p), P(f32p), P(f32p),
                                       P(u32p), P(f32p), f32p]
         _lib = L
@@ -276,4 +282,39 @@ def quant_error(cfg: Config, worker, step, g, r=None, b0=0, b1=None):
     rc = lib().or_quant_error(ctypes.byref(cfg.c()), worker, step, b0, b1, _p(g, ctypes.c_float), rp,
                               _p(out, ctypes.c_double))
     assert rc == 0
+    return out
+
+
+def entropy_groups(levels):
+    """(g, B): g codes of `levels` levels per B-bit group, or None if base-s packing has no
+    grouping for that level count."""
+    g, B = ctypes.c_int(), ctypes.c_int()
+    if not lib().or_entropy_groups(levels, ctypes.byref(g), ctypes.byref(B)):
+        return None
+    return g.value, B.value
+
+
+def entropy_words(cfg: Config):
+    return lib().or_entropy_words(ctypes.byref(cfg.c()))
+
+
+def entropy_layout(cfg: Config):
+    b, c, l = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    lib().or_entropy_layout(ctypes.byref(cfg.c()), ctypes.byref(b), ctypes.byref(c), ctypes.byref(l))
+    return b.value, c.value, l.value
+
+
+def entropy_pack(cfg: Config, msg):
+    """Dense message -> base-s message."""
+    msg = np.ascontiguousarray(msg, dtype=np.uint8)
+    out = np.zeros(entropy_layout(cfg)[0], dtype=np.uint8)
+    lib().or_entropy_pack(ctypes.byref(cfg.c()), _p(msg, ctypes.c_uint8), _p(out, ctypes.c_uint8))
+    return out
+
+
+def entropy_unpack(cfg: Config, emsg):
+    """Base-s message -> dense message."""
+    emsg = np.ascontiguousarray(emsg, dtype=np.uint8)
+    out = np.zeros(message_layout(cfg)[0], dtype=np.uint8)
+    lib().or_entropy_unpack(ctypes.byref(cfg.c()), _p(emsg, ctypes.c_uint8), _p(out, ctypes.c_uint8))
     return out

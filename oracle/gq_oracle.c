@@ -19,7 +19,9 @@
  *   - BinGrad-pb's pair against brute force over all grid pairs, and the ordering of
  *     quantization errors BinGrad-b <= BinGrad-pb stated in [P2] "Key findings";
  *   - QSGD/TernGrad against hand-computed closed forms;
- *   - packing against a bit-by-bit unpacker; error feedback against its telescoping sum.
+ *   - packing against a bit-by-bit unpacker; error feedback against its telescoping sum;
+ *   - base-s packing against a big-integer construction of the digit stream, the round trip,
+ *     and its bits per code against log2(s) (the compression ratios of [P2] "Key findings").
  * Parity of BinGrad-pb with the paper's own (unpublished on the pages) definition is unpinned:
  * only this reading of it is pinned.
  */
@@ -876,4 +878,110 @@ int or_fused_step(const or_config *cfg, uint64_t step, int64_t b0, int64_t b1,
         rc = or_fused_bucket(cfg, step, bk, n, gb, ef ? rb : NULL, ef ? ro : NULL, wb, tb, avg + base);
     }
     return rc;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Base-s packing of the codes (grouped digits).  [P2] "Key findings" quotes compression     */
+/* ratios of 20.2 (3 levels) and 10.1 (9 levels), which are 32 / log2(s): a code of s          */
+/* levels carries log2(s) bits, which b = ceil(log2 s) bits waste for s = 3, 5, 9.  Reading:    */
+/* g consecutive codes of a bucket form one base-s number V = sum_k code[g*i + k] * s^k (codes  */
+/* past the bucket's end count as 0), stored in B bits, with s^g <= 2^B:                      */
+/*   s = 3: g = 5, B = 8 (243 <= 256, 1.6 bits per code)                                      */
+/*   s = 5: g = 3, B = 7 (125 <= 128, 2.33 bits per code)                                     */
+/*   s = 9: g = 5, B = 16 (59049 <= 65536, 3.2 bits per code)                                 */
+/* The group values follow each other in a little-endian bit string, group i at bits          */
+/* B*i .. B*i + B - 1 of the bucket's ceil(ceil(d/g) * B / 32) words; the level tables are     */
+/* those of the dense message, after the codes region (16-byte aligned, as there).            */
+/* ------------------------------------------------------------------------------------------ */
+int or_entropy_groups(int levels, int *g, int *B)
+{
+    switch (levels) {
+    case 3: *g = 5; *B = 8; return 1;
+    case 5: *g = 3; *B = 7; return 1;
+    case 9: *g = 5; *B = 16; return 1;
+    default: return 0;
+    }
+}
+
+int64_t or_entropy_words(const or_config *cfg)
+{
+    int g, B;
+    if (!or_entropy_groups(cfg->levels, &g, &B)) return 0;
+    int64_t groups = (cfg->bucket + g - 1) / g;
+    return (groups * B + 31) / 32;
+}
+
+void or_entropy_layout(const or_config *cfg, int64_t *bytes, int64_t *codes_off, int64_t *levels_off)
+{
+    int64_t nb = or_num_buckets(cfg);
+    int64_t cbytes = nb * or_entropy_words(cfg) * 4;
+    int64_t lbytes = nb * or_table_len(cfg->scheme, cfg->levels) * 4;
+    cbytes = (cbytes + 15) / 16 * 16;
+    lbytes = (lbytes + 15) / 16 * 16;
+    *codes_off = 0;
+    *levels_off = cbytes;
+    *bytes = cbytes + lbytes;
+}
+
+/* Dense message -> base-s message (same buckets, same level tables). */
+void or_entropy_pack(const or_config *cfg, const uint8_t *msg, uint8_t *emsg)
+{
+    int g, B;
+    if (!or_entropy_groups(cfg->levels, &g, &B)) return;
+    int d = cfg->bucket, s = cfg->levels;
+    int64_t nb = or_num_buckets(cfg), dw = (int64_t)d * or_bits(s) / 32, ew = or_entropy_words(cfg);
+    int64_t bytes, coff, loff, ebytes, ecoff, eloff;
+    or_message_layout(cfg, &bytes, &coff, &loff);
+    or_entropy_layout(cfg, &ebytes, &ecoff, &eloff);
+    memset(emsg, 0, (size_t)ebytes);
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    for (int64_t bk = 0; bk < nb; ++bk) {
+        or_unpack_bucket(cfg, (const uint32_t *)(msg + coff) + bk * dw, d, code);
+        uint32_t *out = (uint32_t *)(emsg + ecoff) + bk * ew;
+        for (int64_t i = 0; g * i < d; ++i) {
+            uint32_t v = 0;
+            for (int k = g - 1; k >= 0; --k) {
+                int64_t e = g * i + k;
+                v = v * (uint32_t)s + (e < d ? code[e] : 0u);
+            }
+            for (int j = 0; j < B; ++j) {
+                int64_t bit = B * i + j;
+                if ((v >> j) & 1u) out[bit / 32] |= 1u << (bit % 32);
+            }
+        }
+    }
+    free(code);
+    memcpy(emsg + eloff, msg + loff, (size_t)(nb * or_table_len(cfg->scheme, s) * 4));
+}
+
+/* Base-s message -> dense message. */
+void or_entropy_unpack(const or_config *cfg, const uint8_t *emsg, uint8_t *msg)
+{
+    int g, B;
+    if (!or_entropy_groups(cfg->levels, &g, &B)) return;
+    int d = cfg->bucket, s = cfg->levels;
+    int64_t nb = or_num_buckets(cfg), dw = (int64_t)d * or_bits(s) / 32, ew = or_entropy_words(cfg);
+    int64_t bytes, coff, loff, ebytes, ecoff, eloff;
+    or_message_layout(cfg, &bytes, &coff, &loff);
+    or_entropy_layout(cfg, &ebytes, &ecoff, &eloff);
+    memset(msg, 0, (size_t)bytes);
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    for (int64_t bk = 0; bk < nb; ++bk) {
+        const uint32_t *in = (const uint32_t *)(emsg + ecoff) + bk * ew;
+        for (int64_t i = 0; g * i < d; ++i) {
+            uint32_t v = 0;
+            for (int j = 0; j < B; ++j) {
+                int64_t bit = B * i + j;
+                v |= ((in[bit / 32] >> (bit % 32)) & 1u) << j;
+            }
+            for (int k = 0; k < g; ++k) {
+                int64_t e = g * i + k;
+                if (e < d) code[e] = (uint8_t)(v % (uint32_t)s);
+                v /= (uint32_t)s;
+            }
+        }
+        or_pack_bucket(cfg, code, d, (uint32_t *)(msg + coff) + bk * dw);
+    }
+    free(code);
+    memcpy(msg + loff, emsg + eloff, (size_t)(nb * or_table_len(cfg->scheme, s) * 4));
 }

@@ -82,6 +82,13 @@ int or_quant_error(const or_config *cfg, int worker, uint64_t step, int64_t b0, 
 void or_pack_bucket(const or_config *cfg, const uint8_t *code, int n, uint32_t *words);
 /* Inverse of or_pack_bucket for the first n codes. */
 void or_unpack_bucket(const or_config *cfg, const uint32_t *words, int n, uint8_t *code);
+/* Base-s packing of the codes: group size g and bits B per group for `levels` (0 if none),
+ * code words per bucket, message layout, and the conversions dense <-> base-s message. */
+int or_entropy_groups(int levels, int *g, int *B);
+int64_t or_entropy_words(const or_config *cfg);
+void or_entropy_layout(const or_config *cfg, int64_t *bytes, int64_t *codes_off, int64_t *levels_off);
+void or_entropy_pack(const or_config *cfg, const uint8_t *msg, uint8_t *emsg);
+void or_entropy_unpack(const or_config *cfg, const uint8_t *emsg, uint8_t *msg);
 /* Dequantize one code with a bucket's level table. */
 float or_dequant(const or_config *cfg, const float *table, int code);
 

@@ -44,6 +44,9 @@ MUTATIONS = [
     ("bingrad_b_tie_rule", "if (best < 0 || j > best_j) {", "if (best < 0 || j >= best_j) {"),
     ("bingrad_pb_tie_rule", "if (bestA < 0 || e < best_e) {", "if (bestA < 0 || e <= best_e) {"),
     ("quant_error_term", "e += P * dh * dh + (1.0 - P) * dl * dl;", "e += P * dh * dh + P * dl * dl;"),
+    ("entropy_digit_order", "for (int k = g - 1; k >= 0; --k) {", "for (int k = 0; k < g; ++k) {"),
+    ("entropy_group_bits", "case 9: *g = 5; *B = 16; return 1;", "case 9: *g = 5; *B = 17; return 1;"),
+    ("entropy_unpack_radix", "v /= (uint32_t)s;", "v /= (uint32_t)(s + 1);"),
 ]
 
 

@@ -570,3 +570,90 @@ def test_quant_error_deterministic_schemes():
     # the clamp regions are decided on 16-bit grid positions, the formula here on values:
     # elements within a position step of a level may fall on either side
     assert abs(e - ref) <= 1e-6 * ref
+
+
+# ------------------------------------------------------------------------------------------
+# Base-s packing of the codes ([P2] "Key findings": compression ratios 20.2 for 3 levels and
+# 10.1 for 9 levels, i.e. 32 / log2(s) bits)
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("levels", [3, 5, 9])
+def test_entropy_groups_near_log2(levels):
+    """g codes of s levels fit B bits (s^g <= 2^B, B minimal), and B/g is within 1 % of the
+    entropy bound log2(s): the ratio 32*g/B is within 1 % of the pages' 32 / log2(s)."""
+    g, B = O.entropy_groups(levels)
+    assert levels ** g <= 2 ** B < 2 * levels ** g
+    assert abs(B / g - math.log2(levels)) / math.log2(levels) < 0.01
+    if levels == 3:
+        assert abs(32 * g / B - 20.2) / 20.2 < 0.01
+    if levels == 9:
+        assert abs(32 * g / B - 10.1) / 10.1 < 0.01
+    assert O.entropy_groups(4) is None and O.entropy_groups(2) is None and O.entropy_groups(16) is None
+
+
+@pytest.mark.parametrize("levels", [3, 5, 9])
+def test_entropy_sizes(levels):
+    """Words per bucket ceil(ceil(d/g)*B/32) and the layout's 16-byte-aligned regions."""
+    g, B = O.entropy_groups(levels)
+    for d, n in ((128, 1000), (512, 512 * 3 + 7), (2048, 2048)):
+        cfg = O.Config(O.ORQ, levels, d, 1, 1, 0.0, 0, n)
+        ew = -(-(-(-d // g)) * B // 32)
+        assert O.entropy_words(cfg) == ew
+        nb = -(-n // d)
+        tl = O.table_len(O.ORQ, levels)
+        nbytes, coff, loff = O.entropy_layout(cfg)
+        assert coff == 0 and loff == -(-nb * ew * 4 // 16) * 16
+        assert nbytes == loff + -(-nb * tl * 4 // 16) * 16
+    # d = 512: 26, 38 and 52 words against 32, 48 and 64 of the dense message
+    assert O.entropy_words(O.Config(O.ORQ, levels, 512, 1, 1, 0.0, 0, 512)) == {3: 26, 5: 38, 9: 52}[levels]
+
+
+def _encoded_msg(scheme, levels, d, n, seed):
+    rng = np.random.default_rng(seed)
+    cfg = O.Config(scheme, levels, d, 1, 0, 0.0, seed, n)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    return cfg, O.encode(cfg, 0, 0, g)
+
+
+@pytest.mark.parametrize("scheme,levels", [(O.ORQ, 3), (O.ORQ, 5), (O.ORQ, 9), (O.QSGD, 5),
+                                           (O.TERNGRAD, 3), (O.QSGD, 9)])
+def test_entropy_is_base_s_stream(scheme, levels):
+    """Each bucket's words hold the little-endian bit string sum_i V_i 2^(B i), with
+    V_i = sum_k code[g i + k] s^k (built here as one Python integer from the dense codes), and
+    the level tables are copied unchanged."""
+    g, B = O.entropy_groups(levels)
+    for d, n in ((128, 128 * 5 + 3), (512, 512 * 2 + 301)):
+        cfg, msg = _encoded_msg(scheme, levels, d, n, 31 + d + levels)
+        emsg = O.entropy_pack(cfg, msg)
+        _, coff, loff = O.message_layout(cfg)
+        _, ecoff, eloff = O.entropy_layout(cfg)
+        dw, ew = d * O.bits(levels) // 32, O.entropy_words(cfg)
+        words = msg[coff:].view(np.uint32)
+        ewords = emsg[ecoff:].view(np.uint32)
+        for bk in range(O.num_buckets(cfg)):
+            code = O.unpack_bucket(cfg, words[bk * dw:(bk + 1) * dw], d)
+            stream = 0
+            for i in range(-(-d // g)):
+                v = sum(int(code[g * i + k]) * levels ** k for k in range(g) if g * i + k < d)
+                stream |= v << (B * i)
+            expect = [(stream >> (32 * k)) & 0xffffffff for k in range(ew)]
+            assert [int(x) for x in ewords[bk * ew:(bk + 1) * ew]] == expect
+        tl = O.num_buckets(cfg) * O.table_len(scheme, levels) * 4
+        assert np.array_equal(emsg[eloff:eloff + tl], msg[loff:loff + tl])
+
+
+@pytest.mark.parametrize("levels", [3, 5, 9])
+def test_entropy_roundtrip(levels):
+    """unpack(pack(m)) == m for encoded messages, ragged last bucket included; every group
+    value is below s^g."""
+    g, B = O.entropy_groups(levels)
+    for scheme in (O.ORQ, O.QSGD):
+        for d, n in ((128, 1), (128, 127), (512, 4096), (1024, 1024 * 2 + 1)):
+            cfg, msg = _encoded_msg(scheme, levels, d, n, 7 * d + n)
+            emsg = O.entropy_pack(cfg, msg)
+            assert np.array_equal(O.entropy_unpack(cfg, emsg), msg)
+            ew = O.entropy_words(cfg)
+            ewords = emsg.view(np.uint32)
+            for bk in range(O.num_buckets(cfg)):
+                stream = sum(int(w) << (32 * k) for k, w in enumerate(ewords[bk * ew:(bk + 1) * ew]))
+                for i in range(-(-d // g)):
+                    assert (stream >> (B * i)) & ((1 << B) - 1) < levels ** g
