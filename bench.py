@@ -98,10 +98,17 @@ def job_value(world, workers, n, steps, elapsed_ms):
     return world * workers * n * steps / (elapsed_ms / 1000.0)
 
 
+# The sources the fused warp-per-bucket kernel (d <= 512) is compiled and launched from: its
+# code, its instantiation, its launch configuration and the plan it reads.  A stored traffic
+# figure stands only while these are byte-identical to what was captured.
+FUSED_KERNEL_SOURCES = ("gq_api.cu", "gq_device.cuh", "gq_internal.h", "gq_round.cuh", "gq_warp.cu",
+                        "gq_warp.cuh", "gq_warp_orq.cu")
+
+
 def source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gradient_quantization_communication_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in FUSED_KERNEL_SOURCES:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
