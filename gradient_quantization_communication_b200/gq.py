@@ -54,12 +54,16 @@ def lib():
         L.gq_quant_error_noalloc.argtypes = [cfgp, ctypes.c_uint32, ctypes.c_uint64, vp, vp, vp, vp]
         L.gq_plan_status.argtypes = [vp, vp]
         L.gq_selftest_bounded_wait.argtypes = [vp, ctypes.c_int64, vp]
+        L.gq_entropy_layout.argtypes = [cfgp, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.gq_entropy_pack.argtypes = [cfgp, vp, vp, vp]
+        L.gq_entropy_unpack.argtypes = [cfgp, vp, vp, vp]
         L.gq_status_string.argtypes = [ctypes.c_int]
         L.gq_status_string.restype = ctypes.c_char_p
         L.gq_version.restype = ctypes.c_char_p
         for f in ("gq_config_check", "gq_message_layout", "gq_plan_create", "gq_plan_destroy", "gq_encode",
                   "gq_decode_accumulate", "gq_fused_step", "gq_quant_error", "gq_quant_error_noalloc",
-                  "gq_plan_status", "gq_selftest_bounded_wait"):
+                  "gq_plan_status", "gq_selftest_bounded_wait", "gq_entropy_layout", "gq_entropy_pack",
+                  "gq_entropy_unpack"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -156,6 +160,21 @@ def gq_plan_status(plan, stream=None):
 
 def gq_selftest_bounded_wait(plan, limit_ns, stream=None):
     _check(lib().gq_selftest_bounded_wait(plan, int(limit_ns), _stream(stream)), "gq_selftest_bounded_wait")
+
+
+def gq_entropy_layout(cfg):
+    b, c, l = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().gq_entropy_layout(ctypes.byref(cfg), ctypes.byref(b), ctypes.byref(c), ctypes.byref(l)),
+           "gq_entropy_layout")
+    return b.value, c.value, l.value
+
+
+def gq_entropy_pack(cfg, msg, emsg, stream=None):
+    _check(lib().gq_entropy_pack(ctypes.byref(cfg), _ptr(msg), _ptr(emsg), _stream(stream)), "gq_entropy_pack")
+
+
+def gq_entropy_unpack(cfg, emsg, msg, stream=None):
+    _check(lib().gq_entropy_unpack(ctypes.byref(cfg), _ptr(emsg), _ptr(msg), _stream(stream)), "gq_entropy_unpack")
 
 
 def gq_status_string(status):

@@ -99,3 +99,59 @@ def test_plan_create_without_device_fails_cleanly():
     with pytest.raises(G.GQError) as ei:
         G.gq_plan_create(G.gq_config("orq", 5, 512, 1, True, 0.0, 0, 100))
     assert ei.value.status == G.GQ_ERR_CUDA
+
+
+@pytest.mark.parametrize("scheme,levels", [(0, 5), (1, 0), (1, 3), (4, 3), (4, 5), (4, 9), (0, 9), (0, 3)])
+@pytest.mark.parametrize("d", [128, 512, 4096, 32768])
+@pytest.mark.parametrize("n", [0, 1, 127, 1000, 11689512, 10 ** 9])
+def test_entropy_layout_matches_oracle(scheme, levels, d, n):
+    mine = G.gq_entropy_layout(G.gq_config(scheme, levels, d, 1, True, 0.0, 0, n))
+    ref = O.entropy_layout(O.Config(scheme, levels or 3, d, 1, 1, 0.0, 0, n))
+    assert mine == ref
+    assert mine[2] % 16 == 0 and mine[0] % 16 == 0
+
+
+@pytest.mark.parametrize("scheme,levels", [(0, 2), (0, 4), (4, 16), (2, 0), (3, 2), (4, 7)])
+def test_entropy_unsupported_levels(scheme, levels):
+    cfg = G.gq_config(scheme, levels, 512, 1, True, 0.0, 0, 1000)
+    for call in (lambda: G.gq_entropy_layout(cfg), lambda: G.gq_entropy_pack(cfg, 0, 0, stream=0),
+                 lambda: G.gq_entropy_unpack(cfg, 0, 0, stream=0)):
+        with pytest.raises(G.GQError) as ei:
+            call()
+        assert ei.value.status == G.GQ_ERR_UNSUPPORTED
+
+
+def test_entropy_argument_checks_without_device():
+    """Argument errors are found on the host before anything touches a device."""
+    cfg = G.gq_config("orq", 5, 512, 1, True, 0.0, 0, 5000)
+    nbytes, _, _ = G.gq_message_layout(cfg)
+    ebytes, _, _ = G.gq_entropy_layout(cfg)
+    base = 1 << 40  # never dereferenced: every case below fails its checks first
+    cases = [(0, base), (base, 0), (base + 4, base + (1 << 30)), (base, base + (1 << 30) + 8),
+             (base, base + 16),                      # overlapping
+             (base + ebytes - 16, base)]             # overlapping the other way
+    for a, b in cases:
+        for call in (G.gq_entropy_pack, G.gq_entropy_unpack):
+            with pytest.raises(G.GQError) as ei:
+                call(cfg, a, b, stream=0)
+            assert ei.value.status == G.GQ_ERR_INVALID, (call.__name__, a, b)
+    bad = G.gq_config("orq", 5, 384, 1, True, 0.0, 0, 5000)
+    with pytest.raises(G.GQError) as ei:
+        G.gq_entropy_pack(bad, base, base + (1 << 30), stream=0)
+    assert ei.value.status == G.GQ_ERR_INVALID
+    # n = 0: a no-op, NULL pointers allowed
+    G.gq_entropy_pack(G.gq_config("orq", 5, 512, 1, True, 0.0, 0, 0), 0, 0, stream=0)
+    G.gq_entropy_unpack(G.gq_config("orq", 5, 512, 1, True, 0.0, 0, 0), 0, 0, stream=0)
+    assert ebytes < nbytes
+
+
+@pytest.mark.parametrize("scheme,levels,ratio", [(1, 3, 32 * 512 / (26 * 32 + 32)),      # TernGrad
+                                                 (4, 3, 32 * 512 / (26 * 32 + 3 * 32)),  # ORQ-3
+                                                 (0, 9, 32 * 512 / (52 * 32 + 32)),      # QSGD-9
+                                                 (4, 9, 32 * 512 / (52 * 32 + 9 * 32))])  # ORQ-9
+def test_entropy_compression_ratio_d512(scheme, levels, ratio):
+    """Base-s messages at d = 512: 26 words (s = 3) or 52 words (s = 9) of codes per bucket plus
+    the level table; without the table the ratios are 32 * 512 / 832 = 19.7 and 9.85."""
+    n = 512 * 1000
+    nbytes, _, _ = G.gq_entropy_layout(G.gq_config(scheme, levels, 512, 1, True, 0.0, 0, n))
+    assert abs(32 * n / (8 * nbytes) - ratio) < 1e-9

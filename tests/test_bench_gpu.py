@@ -52,3 +52,14 @@ def test_unfused_and_sweep_lines():
     assert {r["bucket"] for r in rows} == {128, 512, 2048, 8192, 32768}
     for r in rows:
         assert r["elem_per_s"] > 0 and 0 < r["normalised_variance"] < 10
+
+
+@pytest.mark.gpu
+def test_entropy_line():
+    j = _run("--entropy", "--elements", "5120000", "--steps", "2", "--warmup", "3")
+    assert j["value"] > 0 and j["pack"]["frac"] > 0 and j["unpack"]["frac"] > 0
+    assert j["round_trip"] == "exact" and j["gpu_launches"] == 2 * 8 * 2
+    c = j["compression"]
+    # ORQ-5, d = 512: 38 words of codes per bucket against 48, plus the 5-float table
+    assert abs(c["base_s_bits_per_elem"] - (38 * 32 + 5 * 32) / 512) < 1e-9
+    assert abs(c["dense_bits_per_elem"] - (48 * 32 + 5 * 32) / 512) < 1e-9
