@@ -9,41 +9,32 @@
 // other in the bucket's bit string, least significant bit first.
 //
 // Kernel: one CTA per tile of T consecutive buckets (grid-stride over tiles).
-//   1. The tile's source words are one contiguous span: 16-byte vector loads of its aligned
-//      superset into shared memory (the codes region is padded to 16 bytes, so the superset
-//      stays inside the message).
-//   2. One thread per run of m groups (m * max(source, destination) bits <= 32): it reads the
-//      run's source bits as one funnel shift of two shared words, converts each group (digits
-//      of s <-> b-bit fields) and stores the run's destination bits as one shared word.
-//   3. One thread per destination word: it ORs the two or three runs that overlap the word's
-//      32 bits and stores it (coalesced).  The level tables are copied unchanged.
-// Memory-bound: every byte of both messages is read or written once.
+//   1. The tile's source words are one contiguous span: 16-byte asynchronous copies (cp.async)
+//      of its aligned superset into shared memory (the codes region is padded to 16 bytes, so
+//      the superset stays inside the message), issued one tile ahead into a second buffer.
+//   2. One thread per chunk (a run of groups that starts on a word in both bit strings, see
+//      gq_entropy.cuh): it reads the chunk's source words from shared memory (words past the
+//      bucket's end as 0), converts them in registers and stores its destination words to a
+//      second shared array.
+//   3. The tile's destination words are again one contiguous span: coalesced stores.  The level
+//      tables are copied unchanged.
+// Memory-bound by design: every byte of both messages is read or written once.
 #include <algorithm>
 #include <cstdint>
 
 #include <nvtx3/nvToolsExt.h>
 
+#include "gq_entropy.cuh"
 #include "gq_internal.h"
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTileBytes = 24576;  // shared memory target of one tile (several CTAs per SM)
+using gq::entropy::Base;
+using gq::entropy::Chunk;
 
-template <int S>
-struct Base;
-template <>
-struct Base<3> {
-    static constexpr int g = 5, B = 8, b = 2;
-};
-template <>
-struct Base<5> {
-    static constexpr int g = 3, B = 7, b = 3;
-};
-template <>
-struct Base<9> {
-    static constexpr int g = 5, B = 16, b = 4;
-};
+constexpr int kThreads = 256;
+constexpr int kTileBytes = 24576;  // shared memory target of one CTA (8 CTAs of 256 threads per SM)
+constexpr int kTabRegs = 4;        // level-table floats per thread and tile: T * L <= 4 * kThreads
 
 bool groups_for(int s, int *g, int *B, int *b)
 {
@@ -62,128 +53,134 @@ struct EParams {
     float *tdst;          // destination level tables
     int64_t nb;           // buckets
     int64_t tiles;        // ceil(nb / T)
-    int d;                // bucket size
-    int G;                // groups per bucket, ceil(d / g)
-    int runs;             // runs of m groups per bucket, ceil(G / m)
+    int chunks;           // chunks per bucket
     int sw, dw;           // source / destination words per bucket
     int T;                // buckets per tile
     int L;                // floats per level table
-    // ceil(2^32 / divisor): j / divisor = umulhi(j, magic) exactly for j < 2^32 / divisor; the
-    // indexes j stay below T * max(runs, dw), a few thousand (divisors are at most 10923)
-    uint32_t runs_magic;  // divisor runs
-    uint32_t dw_magic;    // divisor dw
+    // ceil(2^32 / chunks): j / chunks = umulhi(j, magic) exactly for j < 2^32 / chunks; the
+    // indexes j stay below T * chunks, a few thousand
+    uint32_t chunks_magic;
+    int stage_words;      // words of one source buffer in shared memory (a multiple of 4)
     int pad_words;        // zero words after the last bucket's destination words (to 16 bytes)
     int pad_floats;       // zero floats after the last destination level table (to 16 bytes)
 };
 
-__device__ __forceinline__ uint32_t low_mask(int bits) { return bits >= 32 ? 0xffffffffu : (1u << bits) - 1u; }
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// waits until at most N of this thread's committed groups are still in flight (the hardware
+// completes every issued copy; nothing here spins)
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
-// Run of M groups: source bits x (M groups of kSrc bits) -> destination bits (M groups of kDst).
-template <int S, bool PACK>
-struct Run {
-    using C = Base<S>;
-    static constexpr int kSrc = PACK ? C::b * C::g : C::B;  // source bits per group
-    static constexpr int kDst = PACK ? C::B : C::b * C::g;  // destination bits per group
-    static constexpr int M = 32 / (kSrc > kDst ? kSrc : kDst);
-    static constexpr int kRunSrc = M * kSrc;
-    static constexpr int kRunDst = M * kDst;
-    static constexpr int kOverlap = 31 / kRunDst + 2;  // most runs one 32-bit word can overlap
-
-    __device__ __forceinline__ static uint32_t convert(uint32_t x)
-    {
-        uint32_t out = 0;
-#pragma unroll
-        for (int k = 0; k < M; ++k) {
-            const uint32_t grp = x >> (kSrc * k);
-            uint32_t y = 0;
-            if (PACK) {
-                // Horner over the g b-bit codes, highest digit first
-#pragma unroll
-                for (int j = C::g - 1; j >= 0; --j) y = y * (uint32_t)S + ((grp >> (C::b * j)) & ((1u << C::b) - 1u));
-                y &= (1u << C::B) - 1u;
-            } else {
-                uint32_t v = grp & ((1u << C::B) - 1u);
-#pragma unroll
-                for (int j = 0; j < C::g; ++j) {
-                    const uint32_t q = v / (uint32_t)S;
-                    y |= ((v - q * (uint32_t)S) & ((1u << C::b) - 1u)) << (C::b * j);
-                    v = q;
-                }
-            }
-            out |= y << (kDst * k);
-        }
-        return out;
-    }
+// Source words of tile `tile`: buckets [b0, b0 + nt), words [w0, w1) of the source codes,
+// copied through their 16-byte aligned superset [a0, a1) (inside the padded codes region).
+struct TileSpan {
+    int64_t b0, a0;
+    int nt, lead, nvec;
 };
+__device__ __forceinline__ TileSpan tile_span(const EParams &p, int64_t tile)
+{
+    TileSpan t;
+    t.b0 = tile * p.T;
+    t.nt = (int)min((int64_t)p.T, p.nb - t.b0);
+    const int64_t w0 = t.b0 * p.sw, w1 = (t.b0 + t.nt) * p.sw;
+    t.a0 = w0 & ~int64_t(3);
+    t.lead = (int)(w0 - t.a0);
+    t.nvec = (int)((((w1 + 3) & ~int64_t(3)) - t.a0) >> 2);
+    return t;
+}
+
+__device__ __forceinline__ void stage_tile(const EParams &p, const TileSpan &t, uint32_t *buf)
+{
+    for (int v = threadIdx.x; v < t.nvec; v += kThreads) cp_async16(buf + 4 * v, p.src + t.a0 + 4 * v);
+}
 
 template <int S, bool PACK>
 __global__ void __launch_bounds__(kThreads) k_entropy(const __grid_constant__ EParams p)
 {
-    using R = Run<S, PACK>;
-    using C = Base<S>;
+    using K = Chunk<S, PACK>;
     extern __shared__ __align__(16) uint32_t sm[];
-    const int stage_words = p.T * p.sw + 8;
-    uint32_t *runs = sm + stage_words;
+    // [source buffer 0 | source buffer 1 | destination words], each 16-byte aligned: the next
+    // tile's source words are copied in (cp.async) while this tile is converted
+    uint32_t *out = sm + 2 * p.stage_words;
 
     if (blockIdx.x == 0) {
         if ((int)threadIdx.x < p.pad_words) p.dst[p.nb * p.dw + threadIdx.x] = 0u;
         if ((int)threadIdx.x < p.pad_floats) p.tdst[p.nb * p.L + threadIdx.x] = 0.0f;
     }
 
-    for (int64_t tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
-        const int64_t b0 = tile * p.T;
-        const int nt = (int)min((int64_t)p.T, p.nb - b0);
-        // 1. stage the source words [w0, w1) through their 16-byte aligned superset [a0, a1)
-        const int64_t w0 = b0 * p.sw, w1 = (b0 + nt) * p.sw;
-        const int64_t a0 = w0 & ~int64_t(3), a1 = (w1 + 3) & ~int64_t(3);
-        const int lead = (int)(w0 - a0);
-        const uint4 *src4 = reinterpret_cast<const uint4 *>(p.src + a0);
-        uint4 *sm4 = reinterpret_cast<uint4 *>(sm);
-        for (int v = threadIdx.x; v < (int)((a1 - a0) >> 2); v += kThreads) sm4[v] = __ldg(src4 + v);
-        __syncthreads();
-
-        // 2. runs of M groups
-        const uint32_t *stage = sm + lead;
-        for (int j = threadIdx.x; j < nt * p.runs; j += kThreads) {
-            const int bk = (int)__umulhi((uint32_t)j, p.runs_magic);
-            const int t = j - bk * p.runs;
-            const uint32_t *w = stage + bk * p.sw;
-            const int o = R::kRunSrc * t;
-            const int q = o >> 5;
-            const uint32_t lo = w[q];
-            const uint32_t hi = q + 1 < p.sw ? w[q + 1] : 0u;
-            uint32_t x = __funnelshift_r(lo, hi, o & 31) & low_mask(R::kRunSrc);
-            if (PACK) {
-                // codes past the bucket's end (the last run only) count as 0
-                const int valid = p.d - C::g * R::M * t;
-                if (valid < C::g * R::M) x &= (1u << (C::b * valid)) - 1u;
-            }
-            runs[j] = R::convert(x);
-        }
-        __syncthreads();
-
-        // 3. destination words, each the OR of the runs overlapping its 32 bits
-        for (int j = threadIdx.x; j < nt * p.dw; j += kThreads) {
-            const int bk = (int)__umulhi((uint32_t)j, p.dw_magic);
-            const int wb = j - bk * p.dw;
-            const uint32_t *r = runs + bk * p.runs;
-            const int lo_bit = 32 * wb;
-            const int i0 = lo_bit / R::kRunDst;
-            const int i1 = min((lo_bit + 31) / R::kRunDst, p.runs - 1);
-            uint32_t word = 0;
+    int64_t tile = blockIdx.x;
+    if (tile < p.tiles) stage_tile(p, tile_span(p, tile), sm);
+    cp_async_commit();
+    for (int it = 0; tile < p.tiles; tile += gridDim.x, ++it) {
+        const TileSpan t = tile_span(p, tile);
+        const int64_t next = tile + gridDim.x;
+        if (next < p.tiles) stage_tile(p, tile_span(p, next), sm + ((it & 1) ? 0 : p.stage_words));
+        cp_async_commit();
+        // this tile's level tables into registers; their latency overlaps the conversion
+        float tv[kTabRegs];
 #pragma unroll
-            for (int k = 0; k < R::kOverlap; ++k) {
-                const int i = i0 + k;
-                if (i <= i1) {
-                    const int sh = R::kRunDst * i - lo_bit;
-                    word |= sh >= 0 ? (r[i] << sh) : (r[i] >> -sh);
-                }
-            }
-            p.dst[b0 * p.dw + j] = word;
+        for (int k = 0; k < kTabRegs; ++k) {
+            const int j = threadIdx.x + k * kThreads;
+            tv[k] = j < t.nt * p.L ? p.tsrc[t.b0 * p.L + j] : 0.0f;
         }
-        for (int j = threadIdx.x; j < nt * p.L; j += kThreads) p.tdst[b0 * p.L + j] = p.tsrc[b0 * p.L + j];
-        __syncthreads();  // the next tile reuses the shared arrays
+        cp_async_wait<1>();  // this tile's copies (all but the group just committed)
+        __syncthreads();
+
+        // one chunk per thread.  The destination words start at `o` + 0, placed so that o and
+        // the tile's first destination word in global memory agree modulo 16 bytes.
+        const uint32_t *stage = sm + ((it & 1) ? p.stage_words : 0) + t.lead;
+        const int off = (int)((t.b0 * p.dw) & 3);
+        uint32_t *o = out + off;
+        for (int j = threadIdx.x; j < t.nt * p.chunks; j += kThreads) {
+            const int bk = (int)__umulhi((uint32_t)j, p.chunks_magic);
+            const int c = j - bk * p.chunks;
+            const int s0 = c * K::kSrcWords, d0 = c * K::kDstWords;
+            const uint32_t *w = stage + bk * p.sw + s0;
+            uint32_t *ow = o + bk * p.dw + d0;
+            // words past the bucket's end (its last chunk only) read as 0 and are not written;
+            // one predicated path for all chunks, so that the lanes of a warp do not diverge
+            uint32_t in[K::kSrcWords], res[K::kDstWords];
+#pragma unroll
+            for (int k = 0; k < K::kSrcWords; ++k) in[k] = s0 + k < p.sw ? w[k] : 0u;
+            gq::entropy::convert_chunk<S, PACK>(in, res);
+#pragma unroll
+            for (int k = 0; k < K::kDstWords; ++k)
+                if (d0 + k < p.dw) ow[k] = res[k];
+        }
+        __syncthreads();
+
+        // the tile's destination words (one contiguous span: scalar head and tail, 16-byte
+        // body) and level tables
+        uint32_t *dst = p.dst + t.b0 * p.dw;
+        const int nw = t.nt * p.dw;
+        const int head = min((4 - off) & 3, nw);
+        const int nvec = (nw - head) >> 2;
+        const int tail0 = head + 4 * nvec;
+        if ((int)threadIdx.x < head) dst[threadIdx.x] = o[threadIdx.x];
+        {
+            const uint4 *o4 = reinterpret_cast<const uint4 *>(o + head);
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + head);
+            for (int j = threadIdx.x; j < nvec; j += kThreads) d4[j] = o4[j];
+        }
+        if ((int)threadIdx.x < nw - tail0) dst[tail0 + threadIdx.x] = o[tail0 + threadIdx.x];
+#pragma unroll
+        for (int k = 0; k < kTabRegs; ++k) {
+            const int j = threadIdx.x + k * kThreads;
+            if (j < t.nt * p.L) p.tdst[t.b0 * p.L + j] = tv[k];
+        }
+        // the next iteration's first __syncthreads orders these reads of `out` before its writes,
+        // and this iteration's second one ordered the reads of this tile's buffer before the
+        // copies into it that the next iteration issues
     }
+    cp_async_wait<0>();
 }
 
 struct Layouts {
@@ -231,29 +228,44 @@ gq_status_t layouts(const gq_config_t *cfg, Layouts *out)
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <int S, bool PACK>
-cudaError_t launch(EParams p, cudaStream_t stream)
+cudaError_t launch(EParams p, int d, cudaStream_t stream)
 {
-    using R = Run<S, PACK>;
-    const int G = (p.d + Base<S>::g - 1) / Base<S>::g;
-    p.G = G;
-    p.runs = (G + R::M - 1) / R::M;
-    const int per_bucket = p.sw + p.runs;  // shared words per bucket
-    p.T = (int)std::max<int64_t>(1, std::min<int64_t>(p.nb, (kTileBytes / 4 - 8) / per_bucket));
+    using C = Base<S>;
+    const int G = (d + C::g - 1) / C::g;
+    p.chunks = (G + C::CG - 1) / C::CG;
+    const int per_bucket = 2 * p.sw + p.dw;  // shared words per bucket
+    int64_t T = std::min<int64_t>(p.nb, (kTileBytes / 4 - 28) / per_bucket);
+    T = std::min<int64_t>(T, kTabRegs * kThreads / p.L);
+    // whole passes of the CTA's threads over the tile's chunks (no near-empty last pass)
+    if (T * p.chunks >= kThreads) T = (T * p.chunks / kThreads) * kThreads / p.chunks;
+    p.T = (int)std::max<int64_t>(1, T);
     p.tiles = (p.nb + p.T - 1) / p.T;
-    p.runs_magic = (uint32_t)(((uint64_t(1) << 32) + p.runs - 1) / p.runs);
-    p.dw_magic = (uint32_t)(((uint64_t(1) << 32) + p.dw - 1) / p.dw);
-    const size_t smem = (size_t)4 * ((size_t)p.T * p.sw + 8 + (size_t)p.T * p.runs);
+    p.chunks_magic = (uint32_t)(((uint64_t(1) << 32) + p.chunks - 1) / p.chunks);
+    // [2 x (source words of a tile + up to 3 + 3 of alignment) | up to 3 + destination words
+    // of a tile]
+    p.stage_words = (p.T * p.sw + 8 + 3) & ~3;
+    const size_t smem = (size_t)4 * (2 * (size_t)p.stage_words + 3 + (size_t)p.T * p.dw);
     auto kern = k_entropy<S, PACK>;
     if (smem > 48 * 1024) {
         const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    int dev = 0, sms = 0, per_sm = 0;
+    // the whole unified L1 as shared memory: eight CTAs of ~23 KB per SM (the kernel reads
+    // global memory only through the asynchronous copies and the level tables)
+    static bool carveout_set = false;  // a repeated set is harmless, so no lock
+    if (!carveout_set) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                                   (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        carveout_set = true;
+    }
+    // grid-stride over tiles: at most as many CTAs as fit on the device at full occupancy
+    // (2048 threads per SM); with less shared memory per SM some wait for a free slot
+    int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
     if (e != cudaSuccess) return e;
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(p.tiles, (int64_t)sms * std::max(per_sm, 1)));
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(p.tiles, (int64_t)sms * (2048 / kThreads)));
     kern<<<(unsigned)grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
@@ -277,7 +289,6 @@ gq_status_t convert(const gq_config_t *cfg, const void *in, void *out, void *str
                                              (pack ? l.dense_levels_off : l.base_levels_off));
     p.tdst = reinterpret_cast<float *>(static_cast<unsigned char *>(out) + (pack ? l.base_levels_off : l.dense_levels_off));
     p.nb = l.nb;
-    p.d = cfg->bucket;
     p.sw = pack ? l.dense_words : l.base_words;
     p.dw = pack ? l.base_words : l.dense_words;
     p.L = l.L;
@@ -288,9 +299,9 @@ gq_status_t convert(const gq_config_t *cfg, const void *in, void *out, void *str
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaErrorInvalidValue;
     switch (l.s) {
-    case 3: e = pack ? launch<3, true>(p, s) : launch<3, false>(p, s); break;
-    case 5: e = pack ? launch<5, true>(p, s) : launch<5, false>(p, s); break;
-    case 9: e = pack ? launch<9, true>(p, s) : launch<9, false>(p, s); break;
+    case 3: e = pack ? launch<3, true>(p, cfg->bucket, s) : launch<3, false>(p, cfg->bucket, s); break;
+    case 5: e = pack ? launch<5, true>(p, cfg->bucket, s) : launch<5, false>(p, cfg->bucket, s); break;
+    case 9: e = pack ? launch<9, true>(p, cfg->bucket, s) : launch<9, false>(p, cfg->bucket, s); break;
     default: break;
     }
     return e == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
