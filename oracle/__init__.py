@@ -11,9 +11,9 @@ import numpy as np
 
 from . import build as _build
 
-QSGD, TERNGRAD, BINGRAD_B, BINGRAD_PB, ORQ = 0, 1, 2, 3, 4
+QSGD, TERNGRAD, BINGRAD_B, BINGRAD_PB, ORQ, QSGD_NEAREST, SIGNSGD = 0, 1, 2, 3, 4, 5, 6
 SCHEMES = {"qsgd": QSGD, "terngrad": TERNGRAD, "bingrad_b": BINGRAD_B,
-           "bingrad_pb": BINGRAD_PB, "orq": ORQ}
+           "bingrad_pb": BINGRAD_PB, "orq": ORQ, "qsgd_nearest": QSGD_NEAREST, "signsgd": SIGNSGD}
 
 
 class _Cfg(ctypes.Structure):
@@ -57,6 +57,8 @@ def lib():
         L.or_clip_threshold.argtypes = [f32p, ctypes.c_int, ctypes.c_float]
         L.or_clip_threshold.restype = ctypes.c_float
         L.or_grid.argtypes = [f32p, ctypes.c_int, f32p]
+        L.or_sign_scale.argtypes = [f32p, ctypes.c_int]
+        L.or_sign_scale.restype = ctypes.c_float
         L.or_orq_select.argtypes = [f32p, ctypes.c_int, ctypes.c_int, i32p]
         L.or_orq_select.restype = ctypes.c_double
         L.or_bingrad_b_fit.argtypes = [f32p, ctypes.c_int, f32p, f32p, f32p, i32p]
@@ -117,6 +119,11 @@ def fexpo(m):
 def clip_threshold(v, c):
     v = _f32(v)
     return lib().or_clip_threshold(_p(v, ctypes.c_float), len(v), c)
+
+
+def sign_scale(u):
+    u = _f32(u)
+    return lib().or_sign_scale(_p(u, ctypes.c_float), len(u))
 
 
 def grid(u):

@@ -21,12 +21,15 @@
  *   - QSGD/TernGrad against hand-computed closed forms;
  *   - packing against a bit-by-bit unpacker; error feedback against its telescoping sum;
  *   - base-s packing against a big-integer construction of the digit stream, the round trip,
- *     and its bits per code against log2(s) (the compression ratios of [P2] "Key findings").
+ *     and its bits per code against log2(s) (the compression ratios of [P2] "Key findings");
+ *   - nearest-level QSGD against brute force over the levels and its tie rule; the scaled sign
+ *     against the exact rational mean of |u|, its sign rule and its error-feedback sum.
  * Parity of BinGrad-pb with the paper's own (unpublished on the pages) definition is unpinned:
  * only this reading of it is pinned.
  */
 #include "gq_oracle.h"
 
+#include <float.h>
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -346,9 +349,15 @@ static float qsgd_ratio(int code, int s)
     return (float)(2 * code - (s - 1)) / (float)(s - 1);
 }
 
+/*
+ * nearest = 1: deterministic rounding ([P3] "Deterministic vs stochastic rounding": every value
+ * goes to its nearest representable level; simple, but biased).  Same levels and message as
+ * QSGD.  Reading: nearest in the binary32 position y below, ties (y - k = 1/2) to the upper
+ * level; no random draw.
+ */
 static void qsgd_bucket(const or_config *cfg, int worker, uint64_t step, int64_t base,
                         const float *u, int n, uint8_t *code, float *q, float *table,
-                        float *blo, float *bhi, float *bp)
+                        float *blo, float *bhi, float *bp, int nearest)
 {
     int s = cfg->levels;
     float m = 0.0f;
@@ -366,14 +375,64 @@ static void qsgd_bucket(const or_config *cfg, int worker, uint64_t step, int64_t
         int k = 0;
         if (y > 0.0f) k = (y >= (float)(s - 2)) ? s - 2 : (int)y;
         float p = y - (float)k;
-        float U = or_uniform(cfg->seed, step, (uint32_t)worker, base + i);
-        int c = k + (U < p ? 1 : 0);
+        int up;
+        if (nearest) {
+            up = p >= 0.5f;
+        } else {
+            float U = or_uniform(cfg->seed, step, (uint32_t)worker, base + i);
+            up = U < p;
+        }
+        int c = k + up;
         code[i] = (uint8_t)c;
         q[i] = m * qsgd_ratio(c, s);
         if (bp) {
             blo[i] = m * qsgd_ratio(k, s);
             bhi[i] = m * qsgd_ratio(k + 1, s);
-            bp[i] = sat01(p);
+            bp[i] = nearest ? (float)up : sat01(p);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Scaled sign.  [P3] "Ternary and binary quantization": SignSGD transmits only the signs of   */
+/* the gradient (32x compression) and needs error feedback.  The pages fix no scale.  Reading: */
+/* per bucket the two levels are -m1 and +m1, m1 the mean of |u| (for fixed signs the scale    */
+/* that minimises the squared error), code 1 for u >= 0 (zeros of either sign go up).  m1 is   */
+/* computed from an exact integer sum of |u| in fixed point with 45 fraction bits below the    */
+/* bucket's largest magnitude (each term below 2^46, so the sum of up to 2^17 terms is exact  */
+/* in int64), so that it does not depend on summation order:                                  */
+/*   m1 = binary32(((binary64) S * 2^-E) / n),  S = sum of round(|u| * 2^E),  E = 45 - e,     */
+/* e = floor(log2 max|u|).  The level table holds {-m1, +m1}.                                  */
+/* ------------------------------------------------------------------------------------------ */
+float or_sign_scale(const float *u, int n)
+{
+    float m0 = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(u[i]);
+        if (a > m0) m0 = a;
+    }
+    if (!(m0 > 0.0f) || n <= 0) return m0 > 0.0f ? m0 : 0.0f;  /* zero bucket: 0; NaN/inf: unspecified */
+    if (!(m0 <= FLT_MAX)) return m0;
+    int E = 45 - or_fexpo(m0);
+    int64_t S = 0;
+    for (int i = 0; i < n; ++i) S += llrint(ldexp(fabs((double)u[i]), E));
+    return (float)(ldexp((double)S, -E) / (double)n);
+}
+
+static void sign_bucket(const float *u, int n, uint8_t *code, float *q, float *table,
+                        float *blo, float *bhi, float *bp)
+{
+    float m1 = or_sign_scale(u, n);
+    table[0] = -m1;
+    table[1] = m1;
+    for (int i = 0; i < n; ++i) {
+        int up = u[i] >= 0.0f;
+        code[i] = (uint8_t)up;
+        q[i] = up ? m1 : -m1;
+        if (bp) {
+            blo[i] = -m1;
+            bhi[i] = m1;
+            bp[i] = (float)up;
         }
     }
 }
@@ -578,8 +637,8 @@ int or_bits(int levels)
 
 int or_table_len(int scheme, int levels)
 {
-    if (scheme == OR_QSGD || scheme == OR_TERNGRAD) return 1;
-    if (scheme == OR_BINGRAD_B || scheme == OR_BINGRAD_PB) return 2;
+    if (scheme == OR_QSGD || scheme == OR_TERNGRAD || scheme == OR_QSGD_NEAREST) return 1;
+    if (scheme == OR_BINGRAD_B || scheme == OR_BINGRAD_PB || scheme == OR_SIGNSGD) return 2;
     return levels;
 }
 
@@ -638,7 +697,7 @@ void or_unpack_bucket(const or_config *cfg, const uint32_t *words, int n, uint8_
 
 float or_dequant(const or_config *cfg, const float *table, int code)
 {
-    if (cfg->scheme == OR_QSGD || cfg->scheme == OR_TERNGRAD)
+    if (cfg->scheme == OR_QSGD || cfg->scheme == OR_TERNGRAD || cfg->scheme == OR_QSGD_NEAREST)
         return table[0] * qsgd_ratio(code, cfg->levels);
     return table[code];
 }
@@ -666,7 +725,13 @@ static int encode_bucket_ex(const or_config *cfg, int worker, uint64_t step, int
     switch (cfg->scheme) {
     case OR_QSGD:
     case OR_TERNGRAD:
-        qsgd_bucket(cfg, worker, step, base, u, n, code, q, table, blo, bhi, bp);
+        qsgd_bucket(cfg, worker, step, base, u, n, code, q, table, blo, bhi, bp, 0);
+        break;
+    case OR_QSGD_NEAREST:
+        qsgd_bucket(cfg, worker, step, base, u, n, code, q, table, blo, bhi, bp, 1);
+        break;
+    case OR_SIGNSGD:
+        sign_bucket(u, n, code, q, table, blo, bhi, bp);
         break;
     case OR_BINGRAD_B:
         bingrad_b_bucket(u, n, code, q, table, blo, bhi, bp);

@@ -26,7 +26,9 @@
 extern "C" {
 #endif
 
-enum { OR_QSGD = 0, OR_TERNGRAD = 1, OR_BINGRAD_B = 2, OR_BINGRAD_PB = 3, OR_ORQ = 4 };
+enum { OR_QSGD = 0, OR_TERNGRAD = 1, OR_BINGRAD_B = 2, OR_BINGRAD_PB = 3, OR_ORQ = 4,
+       OR_QSGD_NEAREST = 5, /* QSGD levels, deterministic rounding to the nearest level */
+       OR_SIGNSGD = 6 };    /* scaled sign: levels -m1, +m1, m1 the mean |u| of the bucket */
 
 typedef struct {
     int32_t scheme;          /* OR_* */
@@ -50,6 +52,8 @@ int or_fexpo(float m);
 
 /* Per-bucket clipping threshold T = c * sigma (0 if the bucket is all zero). */
 float or_clip_threshold(const float *v, int n, float c);
+/* Scale m1 of the scaled-sign scheme: the mean of |u| from exact fixed-point sums. */
+float or_sign_scale(const float *u, int n);
 
 /* 64-point candidate grid and fixed-point positions; returns 0 for a constant bucket. */
 int or_grid(const float *u, int n, float grid[64]);

@@ -47,6 +47,11 @@ MUTATIONS = [
     ("entropy_digit_order", "for (int k = g - 1; k >= 0; --k) {", "for (int k = 0; k < g; ++k) {"),
     ("entropy_group_bits", "case 9: *g = 5; *B = 16; return 1;", "case 9: *g = 5; *B = 17; return 1;"),
     ("entropy_unpack_radix", "v /= (uint32_t)s;", "v /= (uint32_t)(s + 1);"),
+    ("qsgd_nearest_tie", "up = p >= 0.5f;", "up = p > 0.5f;"),
+    ("sign_zero_up", "int up = u[i] >= 0.0f;", "int up = u[i] > 0.0f;"),
+    ("sign_mean_divisor", "return (float)(ldexp((double)S, -E) / (double)n);",
+     "return (float)(ldexp((double)S, -E) / (double)(n + 1));"),
+    ("sign_table_order", "table[0] = -m1;", "table[0] = m1;"),
 ]
 
 

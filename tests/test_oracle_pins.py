@@ -657,3 +657,92 @@ def test_entropy_roundtrip(levels):
                 stream = sum(int(w) << (32 * k) for k, w in enumerate(ewords[bk * ew:(bk + 1) * ew]))
                 for i in range(-(-d // g)):
                     assert (stream >> (B * i)) & ((1 << B) - 1) < levels ** g
+
+
+# ------------------------------------------------------------------------------------------
+# Biased baselines ([P3] "Deterministic vs stochastic rounding", "Ternary and binary
+# quantization"): QSGD levels with rounding to the nearest level, and the scaled sign
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("levels", [2, 3, 5, 9, 15, 16])
+def test_qsgd_nearest_is_nearest_level(levels):
+    """Every value goes to a nearest QSGD level (brute force over the levels, up to the
+    rounding of the binary32 position); no randomness: seed, step and worker do not matter."""
+    rng = np.random.default_rng(70 + levels)
+    v = (rng.standard_normal(512) * 1e-3).astype(np.float32)
+    outs = []
+    for seed, step, worker in ((0, 0, 0), (5, 9, 3)):
+        cfg = O.Config(O.QSGD_NEAREST, levels, 512, 1, 0, 0.0, seed, 512)
+        code, q, table = O.encode_bucket(cfg, worker, step, 0, v)
+        outs.append(code.copy())
+        m = float(table[0])
+        assert m == float(np.abs(v).max())
+        lv = np.array([m * (2 * k - (levels - 1)) / (levels - 1) for k in range(levels)])
+        dist = np.abs(lv[None, :] - v.astype(np.float64)[:, None])
+        best = dist.min(axis=1)
+        got = np.abs(q.astype(np.float64) - v)
+        assert np.all(got <= best + 1e-6 * m)
+        assert np.array_equal(q, np.array([O.dequant(cfg, table, int(c)) for c in code], dtype=np.float32))
+        # the same bracket as stochastic QSGD: the code is k or k + 1
+        ks = np.clip(np.trunc((v / np.float32(m) + 1) * (levels - 1) / 2), 0, levels - 2)
+        assert np.all((code == ks) | (code == ks + 1))
+    assert np.array_equal(outs[0], outs[1])
+
+
+def test_qsgd_nearest_ties_go_up():
+    """Values exactly half-way between two levels (position y = k + 1/2) take the upper one."""
+    v = np.zeros(512, dtype=np.float32)
+    v[0] = 1.0                          # m = 1; s = 5: levels -1, -0.5, 0, 0.5, 1, h = 2
+    v[1], v[2], v[3], v[4] = 0.25, -0.75, 0.75, -0.25   # y = 2.5, 0.5, 3.5, 1.5
+    cfg = O.Config(O.QSGD_NEAREST, 5, 512, 1, 0, 0.0, 0, 512)
+    code, q, _ = O.encode_bucket(cfg, 0, 0, 0, v)
+    assert list(code[:5]) == [4, 3, 1, 4, 2]
+    assert list(q[1:5]) == [0.5, -0.5, 1.0, 0.0]
+
+
+def test_sign_scale_is_mean_abs():
+    """m1 is the binary32 value nearest the exact mean of |u| (checked with rationals), to
+    within one ulp (the fixed-point sum carries 45 fraction bits below the largest magnitude)."""
+    rng = np.random.default_rng(80)
+    for n, scale in ((512, 1e-3), (300, 1e-30), (128, 3e5), (1, 1.0)):
+        u = (rng.standard_normal(n) * scale).astype(np.float32)
+        exact = sum(Fraction(float(abs(x))) for x in u) / n
+        m1 = O.sign_scale(u)
+        assert abs(Fraction(float(m1)) - exact) <= Fraction(float(np.spacing(np.float32(m1))))
+    assert O.sign_scale(np.zeros(64, np.float32)) == 0.0
+
+
+def test_signsgd_codes_and_levels():
+    """Code 1 for u >= 0 (both zeros included), levels {-m1, +m1}; m1 minimises the squared
+    error among scales of the same signs (checked against neighbouring binary32 scales)."""
+    rng = np.random.default_rng(81)
+    v = (rng.standard_normal(512) * 1e-3).astype(np.float32)
+    v[3], v[4] = 0.0, -0.0
+    cfg = O.Config(O.SIGNSGD, 2, 512, 1, 0, 0.0, 0, 512)
+    code, q, table = O.encode_bucket(cfg, 0, 0, 0, v)
+    m1 = O.sign_scale(v)
+    assert list(table) == [-m1, m1]
+    assert np.array_equal(code, (v >= 0).astype(np.uint8)) and code[3] == 1 and code[4] == 1
+    assert np.array_equal(q, np.where(v >= 0, m1, -m1).astype(np.float32))
+    sgn = np.where(v >= 0, 1.0, -1.0)
+    sse = lambda a: float(np.sum((v.astype(np.float64) - a * sgn) ** 2))
+    assert sse(m1) <= sse(np.nextafter(np.float32(m1), np.float32(1))) and \
+        sse(m1) <= sse(np.nextafter(np.float32(m1), np.float32(0)))
+    # an all-zero bucket quantizes to zeros
+    code, q, table = O.encode_bucket(cfg, 0, 0, 0, np.zeros(512, np.float32))
+    assert np.all(code == 1) and np.all(q == 0.0) and list(table) == [0.0, 0.0]
+
+
+def test_signsgd_error_feedback_telescopes():
+    """With error feedback the scaled sign loses nothing: sum_t Q_t = sum_t g_t - r_T."""
+    rng = np.random.default_rng(82)
+    n, d, T = 1000, 128, 8
+    cfg = O.Config(O.SIGNSGD, 2, d, 1, 1, 0.0, 0, n)
+    r = np.zeros(n, dtype=np.float32)
+    gsum = np.zeros(n)
+    qsum = np.zeros(n)
+    for t in range(T):
+        g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+        gsum += g
+        msg = O.encode(cfg, 0, t, g, r)
+        qsum += O.decode_accumulate(cfg, [msg]).astype(np.float64)
+    assert np.allclose(qsum, gsum - r, atol=1e-8)
