@@ -76,11 +76,17 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def table_len(scheme_id, levels):
+    """Floats per level table: the scale for QSGD / TernGrad / QSGD-nearest, two levels for
+    BinGrad-b / BinGrad-pb / SignSGD, s levels for ORQ."""
+    return 1 if scheme_id in (0, 1, 5) else (2 if scheme_id in (2, 3, 6) else levels)
+
+
 def bytes_per_worker_elem(scheme_id, levels, d, W, ef, msgs):
     """Algorithmic HBM bytes per worker-element of the fused step: read g (and r), write r',
     the message (b/8 bits + level table share) and the worker's share of the average."""
     bits = (levels - 1).bit_length()
-    L = 1 if scheme_id in (0, 1) else (2 if scheme_id in (2, 3) else levels)
+    L = table_len(scheme_id, levels)
     b = 4.0 + (8.0 if ef else 0.0) + 4.0 / W
     if msgs:
         b += bits / 8.0 + 4.0 * L / d
@@ -552,7 +558,7 @@ def run_unfused(args):
     dec_ms = statistics.mean(e[W][0].elapsed_time(e[W][1]) for e in evs)
     plan.close()
     bits = (args.levels - 1).bit_length()
-    L = 1 if sid in (0, 1) else (2 if sid in (2, 3) else args.levels)
+    L = table_len(sid, args.levels)
     msg_b = bits / 8.0 + 4.0 * L / d
     enc_b = 4.0 + (8.0 if ef else 0.0) + msg_b          # per element of one worker
     dec_b = W * msg_b + 4.0                             # per element of the average
@@ -648,7 +654,7 @@ def run_entropy(args):
     # algorithmic bytes per launch: the dense message read and the base-s message written (or
     # the reverse), codes and level tables, without the padding
     bits = (args.levels - 1).bit_length()
-    L = 1 if sid in (0, 1) else (2 if sid in (2, 3) else args.levels)
+    L = table_len(sid, args.levels)
     nb = (n + d - 1) // d
     gsz, B = {3: (5, 8), 5: (3, 7), 9: (5, 16)}[args.levels]
     ew = (-(-d // gsz) * B + 31) // 32

@@ -35,8 +35,8 @@ int bits_for(int s)
 
 int table_len(int scheme, int s)
 {
-    if (scheme == GQ_QSGD || scheme == GQ_TERNGRAD) return 1;
-    if (scheme == GQ_BINGRAD_B || scheme == GQ_BINGRAD_PB) return 2;
+    if (scheme == GQ_QSGD || scheme == GQ_TERNGRAD || scheme == GQ_QSGD_NEAREST) return 1;
+    if (scheme == GQ_BINGRAD_B || scheme == GQ_BINGRAD_PB || scheme == GQ_SIGNSGD) return 2;
     return s;
 }
 
@@ -48,6 +48,7 @@ gq_status_t normalise(const gq_config_t *in, gq_config_t *out)
     switch (c.scheme) {
     case GQ_QSGD:
     case GQ_ORQ:
+    case GQ_QSGD_NEAREST:
         if (c.levels < 2 || c.levels > GQ_MAX_LEVELS) return GQ_ERR_INVALID;
         break;
     case GQ_TERNGRAD:
@@ -56,6 +57,7 @@ gq_status_t normalise(const gq_config_t *in, gq_config_t *out)
         break;
     case GQ_BINGRAD_B:
     case GQ_BINGRAD_PB:
+    case GQ_SIGNSGD:
         if (c.levels == 0) c.levels = 2;
         if (c.levels != 2) return GQ_ERR_INVALID;
         break;
@@ -66,6 +68,8 @@ gq_status_t normalise(const gq_config_t *in, gq_config_t *out)
     if (c.error_feedback != 0 && c.error_feedback != 1) return GQ_ERR_INVALID;
     if (!(c.clip_sigma >= 0.0f) || !std::isfinite(c.clip_sigma)) return GQ_ERR_INVALID;
     if (c.n < 0 || c.n >= (int64_t(1) << 40)) return GQ_ERR_INVALID;
+    // the biased baselines are built for the register path only
+    if ((c.scheme == GQ_QSGD_NEAREST || c.scheme == GQ_SIGNSGD) && c.bucket > 512) return GQ_ERR_UNSUPPORTED;
     *out = c;
     return GQ_OK;
 }

@@ -128,7 +128,8 @@ cudaError_t launch_bits(const KParams &p, cudaStream_t stream)
 
 cudaError_t launch_decode(const KParams &p, cudaStream_t stream)
 {
-    return (p.scheme == GQ_QSGD || p.scheme == GQ_TERNGRAD) ? launch_bits<true>(p, stream) : launch_bits<false>(p, stream);
+    const bool qsgd = p.scheme == GQ_QSGD || p.scheme == GQ_TERNGRAD || p.scheme == GQ_QSGD_NEAREST;
+    return qsgd ? launch_bits<true>(p, stream) : launch_bits<false>(p, stream);
 }
 
 }  // namespace gq

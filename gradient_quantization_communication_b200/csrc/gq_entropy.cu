@@ -193,8 +193,8 @@ struct Layouts {
 
 int table_len(int scheme, int s)
 {
-    if (scheme == GQ_QSGD || scheme == GQ_TERNGRAD) return 1;
-    if (scheme == GQ_BINGRAD_B || scheme == GQ_BINGRAD_PB) return 2;
+    if (scheme == GQ_QSGD || scheme == GQ_TERNGRAD || scheme == GQ_QSGD_NEAREST) return 1;
+    if (scheme == GQ_BINGRAD_B || scheme == GQ_BINGRAD_PB || scheme == GQ_SIGNSGD) return 2;
     return s;
 }
 
@@ -206,7 +206,8 @@ gq_status_t layouts(const gq_config_t *cfg, Layouts *out)
     const gq_status_t st = gq_config_check(&c);
     if (st != GQ_OK) return st;
     if (c.scheme == GQ_TERNGRAD && c.levels == 0) c.levels = 3;
-    if ((c.scheme == GQ_BINGRAD_B || c.scheme == GQ_BINGRAD_PB) && c.levels == 0) c.levels = 2;
+    if ((c.scheme == GQ_BINGRAD_B || c.scheme == GQ_BINGRAD_PB || c.scheme == GQ_SIGNSGD) && c.levels == 0)
+        c.levels = 2;
     Layouts l;
     if (!groups_for(c.levels, &l.g, &l.B, &l.b)) return GQ_ERR_UNSUPPORTED;
     size_t coff = 0;

@@ -60,7 +60,8 @@ extern "C" GQ_API gq_status_t gq_quant_error_noalloc(const gq_config_t *cfg, uin
     if (!out) return GQ_ERR_INVALID;
     gq_config_t c = *cfg;
     if (c.scheme == GQ_TERNGRAD && c.levels == 0) c.levels = 3;
-    if ((c.scheme == GQ_BINGRAD_B || c.scheme == GQ_BINGRAD_PB) && c.levels == 0) c.levels = 2;
+    if ((c.scheme == GQ_BINGRAD_B || c.scheme == GQ_BINGRAD_PB || c.scheme == GQ_SIGNSGD) && c.levels == 0)
+        c.levels = 2;
     const int64_t nb = (c.n + c.bucket - 1) / c.bucket;
     if (nb > kMaxBuckets) return GQ_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -87,8 +88,9 @@ extern "C" GQ_API gq_status_t gq_quant_error_noalloc(const gq_config_t *cfg, uin
     p.scheme = c.scheme;
     p.s = c.levels;
     p.bits = bits;
-    p.L = (c.scheme == GQ_QSGD || c.scheme == GQ_TERNGRAD) ? 1
-          : (c.scheme == GQ_BINGRAD_B || c.scheme == GQ_BINGRAD_PB) ? 2 : c.levels;
+    p.L = (c.scheme == GQ_QSGD || c.scheme == GQ_TERNGRAD || c.scheme == GQ_QSGD_NEAREST) ? 1
+          : (c.scheme == GQ_BINGRAD_B || c.scheme == GQ_BINGRAD_PB || c.scheme == GQ_SIGNSGD) ? 2
+                                                                                               : c.levels;
     p.d = c.bucket;
     p.W = 1;
     p.n = c.n;

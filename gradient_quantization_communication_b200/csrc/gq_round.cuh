@@ -13,7 +13,9 @@ namespace gq {
 
 // QSGD / TernGrad: position y = (u/m + 1) * (s-1)/2 in level units, bracket k = trunc(y)
 // clamped to [0, s-2], up with probability y - k.  pair[k] = {level k, level k+1}.
-struct RoundQSGD {
+// NEAREST (QSGD-nearest): up iff y - k >= 1/2, no draw; the bracket's probability is then 0 or 1.
+template <bool NEAREST>
+struct RoundQSGDT {
     float inv_m, h;
     int kmax;
     const float2 *pair;
@@ -22,7 +24,7 @@ struct RoundQSGD {
         const float y = __fmul_rn(__fadd_rn(__fmul_rn(u, inv_m), 1.0f), h);
         const int k = min(max(__float2int_rz(y), 0), kmax);
         const float pu = __fsub_rn(y, (float)k);
-        const bool up = unit_float(word) < pu;
+        const bool up = NEAREST ? pu >= 0.5f : unit_float(word) < pu;
         const float2 lp = pair[k];
         code = k + (up ? 1 : 0);
         q = up ? lp.y : lp.x;
@@ -32,8 +34,27 @@ struct RoundQSGD {
         const float y = __fmul_rn(__fadd_rn(__fmul_rn(u, inv_m), 1.0f), h);
         const int k = min(max(__float2int_rz(y), 0), kmax);
         pu = __fsub_rn(y, (float)k);
+        if (NEAREST) pu = pu >= 0.5f ? 1.0f : 0.0f;
         lo = pair[k].x;
         hi = pair[k].y;
+    }
+};
+using RoundQSGD = RoundQSGDT<false>;
+
+// Scaled sign: code 1 (level +m1) for u >= 0, both zeros included; code 0 (level -m1) below.
+struct RoundSign {
+    float m1;
+    __device__ __forceinline__ void round(float u, int, uint32_t, int &code, float &q) const
+    {
+        const bool up = u >= 0.0f;
+        code = up ? 1 : 0;
+        q = up ? m1 : -m1;
+    }
+    __device__ __forceinline__ void bracket(float u, int, float &lo, float &hi, float &pu) const
+    {
+        lo = -m1;
+        hi = m1;
+        pu = u >= 0.0f ? 1.0f : 0.0f;
     }
 };
 

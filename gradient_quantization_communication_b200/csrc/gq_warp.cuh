@@ -21,6 +21,8 @@
 //                     sums, s-2 incremental greedy rounds, per-bracket reciprocal table
 //   BinGrad-b       : warp bitonic sort, exact int64 prefix sums, screened argmax of J(k)
 //   BinGrad-pb      : shared-memory moments of 16-bit positions, exact search of all pairs
+//   QSGD-nearest    : the QSGD levels, rounding to the nearest level (no draws)
+//   SignSGD         : m1 = mean |u| from an exact fixed-point warp sum, levels -m1 and +m1
 // The last bucket, when ragged, is handled by a one-warp launch of the same code with guarded
 // plain loads, so the main kernel carries no tail logic.
 #pragma once
@@ -179,7 +181,7 @@ __device__ __forceinline__ void build_orq_tables(const KParams &p, FitORQ &sm, i
 // ---------------------------------------------------------------------------------------------
 // Per-scheme fits (u: the values to quantize; v: the error-fed values the residual refers to)
 // ---------------------------------------------------------------------------------------------
-template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0>
+template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0, bool NEAREST = false>
 __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                          const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
@@ -195,7 +197,7 @@ __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int
     __syncwarp();
     if (lane < s - 1) sm.pair[lane] = make_float2(lv, lv_next);
     __syncwarp();
-    RoundQSGD rule;
+    RoundQSGDT<NEAREST> rule;
     rule.inv_m = m > 0.0f ? __frcp_rn(m) : 0.0f;
     rule.h = __fmul_rn((float)(s - 1), 0.5f);
     rule.kmax = s - 2;
@@ -203,8 +205,40 @@ __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int
     int pos[EPL];
 #pragma unroll
     for (int t = 0; t < EPL; ++t) pos[t] = 0;
-    emit<EPL, FUSED, true, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
+    emit<EPL, FUSED, !NEAREST, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
     store_table(p, w, beta, lane, m);
+}
+
+// Scaled sign: m1 = mean |u| of the valid elements from an exact int64 sum of
+// round(|u| * 2^E), E = 45 - floor(log2 max|u|) (every term below 2^46, at most 512 of them),
+// m1 = fp32((S * 2^-E) / n) in binary64; table {-m1, +m1}.
+template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0>
+__device__ void fit_sign(const KParams &p, int64_t beta, int w, int lane, uint32_t vmask, bool check, int nvalid,
+                         const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
+{
+    float m = 0.0f;
+#pragma unroll
+    for (int t = 0; t < EPL; ++t)
+        if (!TAIL || ((vmask >> t) & 1u)) m = fmax_nan(m, fabsf(u[t]));
+    m = warp_redux_max_abs(m);
+    if (check && !(m <= FLT_MAX)) flag_nonfinite(p, lane);
+    RoundSign rule;
+    rule.m1 = m > 0.0f ? m : 0.0f;  // zero bucket: 0; non-finite: unspecified (flagged)
+    if (m > 0.0f && m <= FLT_MAX) {
+        const int E = 45 - fexpo(m);
+        const double sc = pow2d(E);
+        long long S = 0;
+#pragma unroll
+        for (int t = 0; t < EPL; ++t)
+            if (!TAIL || ((vmask >> t) & 1u)) S += fixed_point(fabsf(u[t]), sc);
+        S = warp_sum(S);
+        rule.m1 = __double2float_rn(__ddiv_rn(__dmul_rn(__ll2double_rn(S), pow2d(-E)), (double)nvalid));
+    }
+    int pos[EPL];
+#pragma unroll
+    for (int t = 0; t < EPL; ++t) pos[t] = 0;
+    emit<EPL, FUSED, false, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
+    store_table(p, w, beta, lane, lane == 0 ? -rule.m1 : rule.m1);
 }
 
 template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0>
@@ -640,6 +674,10 @@ __device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME
     }
     if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD)
         fit_qsgd<EPL, FUSED, TAIL, BITS, IO>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
+    else if constexpr (SCHEME == GQ_QSGD_NEAREST)
+        fit_qsgd<EPL, FUSED, TAIL, BITS, IO, true>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
+    else if constexpr (SCHEME == GQ_SIGNSGD)
+        fit_sign<EPL, FUSED, TAIL, BITS, IO>(p, beta, w, lane, vmask, check, nvalid, v, u, acc, ea);
     else if constexpr (SCHEME == GQ_ORQ)
         fit_orq<EPL, FUSED, TAIL, BITS, IO>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
     else if constexpr (SCHEME == GQ_BINGRAD_B)

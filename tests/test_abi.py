@@ -155,3 +155,27 @@ def test_entropy_compression_ratio_d512(scheme, levels, ratio):
     n = 512 * 1000
     nbytes, _, _ = G.gq_entropy_layout(G.gq_config(scheme, levels, 512, 1, True, 0.0, 0, n))
     assert abs(32 * n / (8 * nbytes) - ratio) < 1e-9
+
+
+
+@pytest.mark.parametrize("scheme,levels", [(5, 2), (5, 3), (5, 15), (5, 16), (6, 2), (6, 0)])
+@pytest.mark.parametrize("d", [128, 256, 512])
+@pytest.mark.parametrize("n", [0, 1, 1000, 10 ** 9])
+def test_biased_layout_matches_oracle(scheme, levels, d, n):
+    mine = G.gq_message_layout(G.gq_config(scheme, levels, d, 1, True, 0.0, 0, n))
+    ref = O.message_layout(O.Config(scheme, levels or 2, d, 1, 1, 0.0, 0, n))
+    assert mine == ref
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(scheme="qsgd_nearest", levels=5, bucket=1024), "GQ_ERR_UNSUPPORTED"),
+    (dict(scheme="signsgd", levels=2, bucket=2048), "GQ_ERR_UNSUPPORTED"),
+    (dict(scheme="signsgd", levels=3, bucket=512), "GQ_ERR_INVALID"),
+    (dict(scheme="qsgd_nearest", levels=17, bucket=512), "GQ_ERR_INVALID"),
+    (dict(scheme="qsgd_nearest", levels=1, bucket=512), "GQ_ERR_INVALID"),
+    (dict(scheme="signsgd", levels=0, bucket=512), "GQ_OK"),
+    (dict(scheme="qsgd_nearest", levels=16, bucket=128), "GQ_OK"),
+])
+def test_biased_config_check(kw, status):
+    cfg = G.gq_config(kw["scheme"], kw["levels"], kw["bucket"], 1, True, 0.0, 0, 1000)
+    assert G.gq_config_check(cfg) == getattr(G, status)
