@@ -11,9 +11,9 @@ import numpy as np
 
 from . import build as _build
 
-QSGD, TERNGRAD, BINGRAD_B, BINGRAD_PB, ORQ, QSGD_NEAREST, SIGNSGD = 0, 1, 2, 3, 4, 5, 6
-SCHEMES = {"qsgd": QSGD, "terngrad": TERNGRAD, "bingrad_b": BINGRAD_B,
-           "bingrad_pb": BINGRAD_PB, "orq": ORQ, "qsgd_nearest": QSGD_NEAREST, "signsgd": SIGNSGD}
+QSGD, TERNGRAD, BINGRAD_B, BINGRAD_PB, ORQ, QSGD_NEAREST, SIGNSGD, QSGD_L2 = 0, 1, 2, 3, 4, 5, 6, 7
+SCHEMES = {"qsgd": QSGD, "terngrad": TERNGRAD, "bingrad_b": BINGRAD_B, "bingrad_pb": BINGRAD_PB, "orq": ORQ,
+           "qsgd_nearest": QSGD_NEAREST, "signsgd": SIGNSGD, "qsgd_l2": QSGD_L2}
 
 
 class _Cfg(ctypes.Structure):
@@ -59,6 +59,13 @@ def lib():
         L.or_grid.argtypes = [f32p, ctypes.c_int, f32p]
         L.or_sign_scale.argtypes = [f32p, ctypes.c_int]
         L.or_sign_scale.restype = ctypes.c_float
+        L.or_l2_scale.argtypes = [f32p, ctypes.c_int]
+        L.or_l2_scale.restype = ctypes.c_float
+        L.or_elias_layout.argtypes = [P(_Cfg), P(i64), P(i64), P(i64), P(i64)]
+        L.or_elias_pack.argtypes = [P(_Cfg), u8p, u8p]
+        L.or_elias_pack.restype = i64
+        L.or_elias_unpack.argtypes = [P(_Cfg), u8p, u8p]
+        L.or_elias_gamma_len.argtypes = [ctypes.c_uint32]
         L.or_orq_select.argtypes = [f32p, ctypes.c_int, ctypes.c_int, i32p]
         L.or_orq_select.restype = ctypes.c_double
         L.or_bingrad_b_fit.argtypes = [f32p, ctypes.c_int, f32p, f32p, f32p, i32p]
@@ -124,6 +131,11 @@ def clip_threshold(v, c):
 def sign_scale(u):
     u = _f32(u)
     return lib().or_sign_scale(_p(u, ctypes.c_float), len(u))
+
+
+def l2_scale(u):
+    u = _f32(u)
+    return lib().or_l2_scale(_p(u, ctypes.c_float), len(u))
 
 
 def grid(u):
@@ -325,3 +337,30 @@ def entropy_unpack(cfg: Config, emsg):
     out = np.zeros(message_layout(cfg)[0], dtype=np.uint8)
     lib().or_entropy_unpack(ctypes.byref(cfg.c()), _p(emsg, ctypes.c_uint8), _p(out, ctypes.c_uint8))
     return out
+
+
+def elias_layout(cfg: Config):
+    """(capacity bytes, offsets_off, tables_off, stream_off), or None if unsupported."""
+    v = [ctypes.c_int64() for _ in range(4)]
+    if not lib().or_elias_layout(ctypes.byref(cfg.c()), *[ctypes.byref(x) for x in v]):
+        return None
+    return tuple(x.value for x in v)
+
+
+def elias_pack(cfg: Config, msg):
+    """Dense message -> (Elias message buffer of the capacity size, bytes used)."""
+    msg = np.ascontiguousarray(msg, dtype=np.uint8)
+    out = np.zeros(elias_layout(cfg)[0], dtype=np.uint8)
+    used = lib().or_elias_pack(ctypes.byref(cfg.c()), _p(msg, ctypes.c_uint8), _p(out, ctypes.c_uint8))
+    return out, used
+
+
+def elias_unpack(cfg: Config, emsg):
+    emsg = np.ascontiguousarray(emsg, dtype=np.uint8)
+    out = np.zeros(message_layout(cfg)[0], dtype=np.uint8)
+    assert lib().or_elias_unpack(ctypes.byref(cfg.c()), _p(emsg, ctypes.c_uint8), _p(out, ctypes.c_uint8))
+    return out
+
+
+def elias_gamma_len(x):
+    return lib().or_elias_gamma_len(x)

@@ -23,7 +23,10 @@
  *   - base-s packing against a big-integer construction of the digit stream, the round trip,
  *     and its bits per code against log2(s) (the compression ratios of [P2] "Key findings");
  *   - nearest-level QSGD against brute force over the levels and its tie rule; the scaled sign
- *     against the exact rational mean of |u|, its sign rule and its error-feedback sum.
+ *     against the exact rational mean of |u|, its sign rule and its error-feedback sum;
+ *   - QSGD-l2's scale against the exact norm and its unbiasedness; Elias gamma against the
+ *     published codeword table, the stream against a bit string built from it, the offsets,
+ *     the round trip and the expected length.
  * Parity of BinGrad-pb with the paper's own (unpublished on the pages) definition is unpinned:
  * only this reading of it is pinned.
  */
@@ -355,6 +358,8 @@ static float qsgd_ratio(int code, int s)
  * QSGD.  Reading: nearest in the binary32 position y below, ties (y - k = 1/2) to the upper
  * level; no random draw.
  */
+static float or_l2_scale_fwd(const float *u, int n);
+
 static void qsgd_bucket(const or_config *cfg, int worker, uint64_t step, int64_t base,
                         const float *u, int n, uint8_t *code, float *q, float *table,
                         float *blo, float *bhi, float *bp, int nearest)
@@ -365,6 +370,7 @@ static void qsgd_bucket(const or_config *cfg, int worker, uint64_t step, int64_t
         float a = fabsf(u[i]);
         if (a > m) m = a;
     }
+    if (cfg->scheme == OR_QSGD_L2) m = or_l2_scale_fwd(u, n);
     table[0] = m;
     float inv_m = m > 0.0f ? 1.0f / m : 0.0f;
     float h = (float)(s - 1) * 0.5f;
@@ -417,6 +423,33 @@ float or_sign_scale(const float *u, int n)
     int64_t S = 0;
     for (int i = 0; i < n; ++i) S += llrint(ldexp(fabs((double)u[i]), E));
     return (float)(ldexp((double)S, -E) / (double)n);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* QSGD as originally published (Alistarh et al., "QSGD: Communication-Efficient SGD via      */
+/* Gradient Quantization and Encoding", NIPS 2017) scales by the l2 norm of the vector; [P3]   */
+/* "QSGD" describes it as the generalisation of stochastic quantization whose codes are then    */
+/* Elias-coded.  Reading: per bucket, m = ||u||_2 replaces max |u| in QSGD's levels and         */
+/* rounding (every |u| <= m, so every value lies inside the level range), computed from the    */
+/* same exact fixed-point sums as the clip's sigma (20 fraction bits below the largest          */
+/* magnitude): m = binary32(sqrt((binary64) SXX) * 2^-e).                                       */
+/* ------------------------------------------------------------------------------------------ */
+float or_l2_scale(const float *u, int n)
+{
+    float m0 = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(u[i]);
+        if (a > m0) m0 = a;
+    }
+    if (!(m0 > 0.0f) || n <= 0) return 0.0f;
+    if (!(m0 <= FLT_MAX)) return m0;
+    int e = 20 - or_fexpo(m0);
+    int64_t sxx = 0;
+    for (int i = 0; i < n; ++i) {
+        int64_t x = llrint(ldexp((double)u[i], e));
+        sxx += x * x;
+    }
+    return (float)ldexp(sqrt((double)sxx), -e);
 }
 
 static void sign_bucket(const float *u, int n, uint8_t *code, float *q, float *table,
@@ -637,7 +670,7 @@ int or_bits(int levels)
 
 int or_table_len(int scheme, int levels)
 {
-    if (scheme == OR_QSGD || scheme == OR_TERNGRAD || scheme == OR_QSGD_NEAREST) return 1;
+    if (scheme == OR_QSGD || scheme == OR_TERNGRAD || scheme == OR_QSGD_NEAREST || scheme == OR_QSGD_L2) return 1;
     if (scheme == OR_BINGRAD_B || scheme == OR_BINGRAD_PB || scheme == OR_SIGNSGD) return 2;
     return levels;
 }
@@ -697,7 +730,8 @@ void or_unpack_bucket(const or_config *cfg, const uint32_t *words, int n, uint8_
 
 float or_dequant(const or_config *cfg, const float *table, int code)
 {
-    if (cfg->scheme == OR_QSGD || cfg->scheme == OR_TERNGRAD || cfg->scheme == OR_QSGD_NEAREST)
+    if (cfg->scheme == OR_QSGD || cfg->scheme == OR_TERNGRAD || cfg->scheme == OR_QSGD_NEAREST ||
+        cfg->scheme == OR_QSGD_L2)
         return table[0] * qsgd_ratio(code, cfg->levels);
     return table[code];
 }
@@ -729,6 +763,9 @@ static int encode_bucket_ex(const or_config *cfg, int worker, uint64_t step, int
         break;
     case OR_QSGD_NEAREST:
         qsgd_bucket(cfg, worker, step, base, u, n, code, q, table, blo, bhi, bp, 1);
+        break;
+    case OR_QSGD_L2:
+        qsgd_bucket(cfg, worker, step, base, u, n, code, q, table, blo, bhi, bp, 0);
         break;
     case OR_SIGNSGD:
         sign_bucket(u, n, code, q, table, blo, bhi, bp);
@@ -1049,4 +1086,126 @@ void or_entropy_unpack(const or_config *cfg, const uint8_t *emsg, uint8_t *msg)
     }
     free(code);
     memcpy(msg + loff, emsg + eloff, (size_t)(nb * or_table_len(cfg->scheme, s) * 4));
+}
+
+static float or_l2_scale_fwd(const float *u, int n) { return or_l2_scale(u, n); }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Elias integer coding.  [P3] "QSGD": the quantized values are encoded with Elias integer     */
+/* coding for further lossless compression.  Elias gamma (P. Elias, "Universal codeword sets   */
+/* and representations of the integers", IEEE Trans. Inf. Theory 21(2), 1975): an integer     */
+/* x >= 1 with N = floor(log2 x) is written as N zero bits followed by the N + 1 bits of x,    */
+/* most significant first.  Reading, for the QSGD family with an odd number of levels s (a    */
+/* zero level, z0 = (s-1)/2): code c becomes the signed level z = c - z0, zigzag-mapped to     */
+/* x = 2z + 1 (z >= 0) or -2z (z < 0), so that the zero level costs one bit.                   */
+/* Message: [8 bytes: T, the stream's bit count][8 zero bytes][ceil(n/d) uint64: the first     */
+/* stream bit of each bucket, padded to 16 bytes][the level tables, as in the dense message,   */
+/* padded to 16 bytes][the stream: the valid codes of every bucket in element order, bit k of  */
+/* the stream is bit k % 32 of word k / 32, the bits after T zero, padded to 16 bytes].        */
+/* ------------------------------------------------------------------------------------------ */
+int or_elias_gamma_len(uint32_t x)
+{
+    int N = 0;
+    while ((x >> (N + 1)) != 0u) ++N;
+    return 2 * N + 1;
+}
+
+static int elias_supported(const or_config *cfg)
+{
+    int s = cfg->levels;
+    int qs = cfg->scheme == OR_QSGD || cfg->scheme == OR_TERNGRAD || cfg->scheme == OR_QSGD_NEAREST ||
+             cfg->scheme == OR_QSGD_L2;
+    return qs && (s % 2) == 1;
+}
+
+static uint32_t elias_symbol(int code, int s)
+{
+    int z = code - (s - 1) / 2;
+    return z >= 0 ? (uint32_t)(2 * z + 1) : (uint32_t)(-2 * z);
+}
+
+static int elias_code(uint32_t x, int s)
+{
+    int z = (x & 1u) ? (int)((x - 1u) / 2u) : -(int)(x / 2u);
+    return z + (s - 1) / 2;
+}
+
+int or_elias_layout(const or_config *cfg, int64_t *cap_bytes, int64_t *offsets_off, int64_t *tables_off,
+                    int64_t *stream_off)
+{
+    if (!elias_supported(cfg)) return 0;
+    int s = cfg->levels;
+    int64_t nb = or_num_buckets(cfg);
+    int L = or_table_len(cfg->scheme, s);
+    int maxbits = or_elias_gamma_len((uint32_t)s);   /* the largest symbol is s (z = z0) */
+    int64_t obytes = (nb * 8 + 15) / 16 * 16;
+    int64_t tbytes = (nb * L * 4 + 15) / 16 * 16;
+    int64_t sbytes = ((cfg->n * maxbits + 31) / 32 * 4 + 15) / 16 * 16;
+    *offsets_off = 16;
+    *tables_off = 16 + obytes;
+    *stream_off = 16 + obytes + tbytes;
+    *cap_bytes = *stream_off + sbytes;
+    return 1;
+}
+
+int64_t or_elias_pack(const or_config *cfg, const uint8_t *msg, uint8_t *emsg)
+{
+    int64_t cap, ooff, toff, soff;
+    if (!or_elias_layout(cfg, &cap, &ooff, &toff, &soff)) return -1;
+    int s = cfg->levels, d = cfg->bucket;
+    int64_t nb = or_num_buckets(cfg), dw = (int64_t)d * or_bits(s) / 32;
+    int L = or_table_len(cfg->scheme, s);
+    int64_t bytes, coff, loff;
+    or_message_layout(cfg, &bytes, &coff, &loff);
+    memset(emsg, 0, (size_t)cap);
+    uint64_t *offs = (uint64_t *)(emsg + ooff);
+    uint32_t *stream = (uint32_t *)(emsg + soff);
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    uint64_t k = 0;
+    for (int64_t bk = 0; bk < nb; ++bk) {
+        int n = bucket_len(cfg, bk);
+        offs[bk] = k;
+        or_unpack_bucket(cfg, (const uint32_t *)(msg + coff) + bk * dw, n, code);
+        for (int e = 0; e < n; ++e) {
+            uint32_t x = elias_symbol(code[e], s);
+            int len = or_elias_gamma_len(x), N = len / 2;
+            k += (uint64_t)N;                                  /* N zeros */
+            for (int j = N; j >= 0; --j, ++k)                  /* x, most significant bit first */
+                if ((x >> j) & 1u) stream[k / 32] |= 1u << (k % 32);
+        }
+    }
+    free(code);
+    memcpy(emsg, &k, sizeof k);
+    memcpy(emsg + toff, msg + loff, (size_t)(nb * L * 4));
+    return soff + ((int64_t)(k + 31) / 32 * 4 + 15) / 16 * 16;
+}
+
+int or_elias_unpack(const or_config *cfg, const uint8_t *emsg, uint8_t *msg)
+{
+    int64_t cap, ooff, toff, soff;
+    if (!or_elias_layout(cfg, &cap, &ooff, &toff, &soff)) return 0;
+    int s = cfg->levels, d = cfg->bucket;
+    int64_t nb = or_num_buckets(cfg), dw = (int64_t)d * or_bits(s) / 32;
+    int L = or_table_len(cfg->scheme, s);
+    int64_t bytes, coff, loff;
+    or_message_layout(cfg, &bytes, &coff, &loff);
+    memset(msg, 0, (size_t)bytes);
+    const uint64_t *offs = (const uint64_t *)(emsg + ooff);
+    const uint32_t *stream = (const uint32_t *)(emsg + soff);
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    for (int64_t bk = 0; bk < nb; ++bk) {
+        int n = bucket_len(cfg, bk);
+        uint64_t k = offs[bk];
+        for (int e = 0; e < n; ++e) {
+            int N = 0;
+            while (N < 31 && ((stream[k / 32] >> (k % 32)) & 1u) == 0u) { ++N; ++k; }
+            uint32_t x = 0;
+            for (int j = 0; j <= N; ++j, ++k) x = (x << 1) | ((stream[k / 32] >> (k % 32)) & 1u);
+            code[e] = (uint8_t)elias_code(x, s);
+        }
+        or_pack_bucket(cfg, code, n, (uint32_t *)(msg + coff) + bk * dw);
+    }
+    free(code);
+    memcpy(msg + loff, emsg + toff, (size_t)(nb * L * 4));
+    return 1;
 }

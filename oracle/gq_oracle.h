@@ -28,7 +28,8 @@ extern "C" {
 
 enum { OR_QSGD = 0, OR_TERNGRAD = 1, OR_BINGRAD_B = 2, OR_BINGRAD_PB = 3, OR_ORQ = 4,
        OR_QSGD_NEAREST = 5, /* QSGD levels, deterministic rounding to the nearest level */
-       OR_SIGNSGD = 6 };    /* scaled sign: levels -m1, +m1, m1 the mean |u| of the bucket */
+       OR_SIGNSGD = 6,      /* scaled sign: levels -m1, +m1, m1 the mean |u| of the bucket */
+       OR_QSGD_L2 = 7 };    /* QSGD levels scaled by the bucket's l2 norm instead of max |u| */
 
 typedef struct {
     int32_t scheme;          /* OR_* */
@@ -54,6 +55,8 @@ int or_fexpo(float m);
 float or_clip_threshold(const float *v, int n, float c);
 /* Scale m1 of the scaled-sign scheme: the mean of |u| from exact fixed-point sums. */
 float or_sign_scale(const float *u, int n);
+/* Scale of QSGD-l2: the l2 norm of u from exact fixed-point sums of squares. */
+float or_l2_scale(const float *u, int n);
 
 /* 64-point candidate grid and fixed-point positions; returns 0 for a constant bucket. */
 int or_grid(const float *u, int n, float grid[64]);
@@ -93,6 +96,13 @@ int64_t or_entropy_words(const or_config *cfg);
 void or_entropy_layout(const or_config *cfg, int64_t *bytes, int64_t *codes_off, int64_t *levels_off);
 void or_entropy_pack(const or_config *cfg, const uint8_t *msg, uint8_t *emsg);
 void or_entropy_unpack(const or_config *cfg, const uint8_t *emsg, uint8_t *msg);
+/* Elias-gamma coding of the codes of odd-s QSGD-family messages (0 if unsupported): layout of
+ * the largest message, the conversions (pack returns the bytes used), and one code's length. */
+int or_elias_layout(const or_config *cfg, int64_t *cap_bytes, int64_t *offsets_off, int64_t *tables_off,
+                    int64_t *stream_off);
+int64_t or_elias_pack(const or_config *cfg, const uint8_t *msg, uint8_t *emsg);
+int or_elias_unpack(const or_config *cfg, const uint8_t *emsg, uint8_t *msg);
+int or_elias_gamma_len(uint32_t x);
 /* Dequantize one code with a bucket's level table. */
 float or_dequant(const or_config *cfg, const float *table, int code);
 

@@ -52,6 +52,11 @@ MUTATIONS = [
     ("sign_mean_divisor", "return (float)(ldexp((double)S, -E) / (double)n);",
      "return (float)(ldexp((double)S, -E) / (double)(n + 1));"),
     ("sign_table_order", "table[0] = -m1;", "table[0] = m1;"),
+    ("elias_zigzag", "return z >= 0 ? (uint32_t)(2 * z + 1) : (uint32_t)(-2 * z);",
+     "return z >= 0 ? (uint32_t)(2 * z + 1) : (uint32_t)(-2 * z + 1);"),
+    ("elias_bit_order", "for (int j = N; j >= 0; --j, ++k)", "for (int j = 0; j <= N; ++j, ++k)"),
+    ("elias_offsets", "offs[bk] = k;", "offs[bk] = k + 1;"),
+    ("l2_sqrt", "return (float)ldexp(sqrt((double)sxx), -e);", "return (float)ldexp((double)sxx, -e);"),
 ]
 
 

@@ -746,3 +746,124 @@ def test_signsgd_error_feedback_telescopes():
         msg = O.encode(cfg, 0, t, g, r)
         qsum += O.decode_accumulate(cfg, [msg]).astype(np.float64)
     assert np.allclose(qsum, gsum - r, atol=1e-8)
+
+
+# ------------------------------------------------------------------------------------------
+# QSGD as published (l2 scaling) and Elias integer coding ([P3] "QSGD")
+# ------------------------------------------------------------------------------------------
+def test_l2_scale_is_norm():
+    """m = ||u||_2 from fixed-point sums with 20 fraction bits below max|u|: within 2^-15 of the
+    exact norm (checked with rationals), and never below max|u| by more than that."""
+    rng = np.random.default_rng(90)
+    for n, scale in ((512, 1e-3), (128, 1e-30), (300, 5e4), (1, 2.0)):
+        u = (rng.standard_normal(n) * scale).astype(np.float32)
+        exact = math.sqrt(float(sum(Fraction(float(x)) ** 2 for x in u)))
+        m = O.l2_scale(u)
+        assert abs(m - exact) <= 2 ** -15 * exact
+        assert m >= float(np.abs(u).max()) * (1 - 2 ** -15)
+    assert O.l2_scale(np.zeros(16, np.float32)) == 0.0
+
+
+def test_qsgd_l2_levels_and_unbiased():
+    """QSGD-l2 uses m = ||u||_2 as its scale: table m, levels m (2k - (s-1))/(s-1), and the
+    rounding is unbiased (Monte Carlo over 4000 steps)."""
+    rng = np.random.default_rng(91)
+    v = (rng.standard_normal(128) * 1e-3).astype(np.float32)
+    cfg = O.Config(O.QSGD_L2, 3, 128, 1, 0, 0.0, 5, 128)
+    _, _, table = O.encode_bucket(cfg, 0, 0, 0, v)
+    assert table[0] == O.l2_scale(v)
+    acc = np.zeros(128)
+    T = 4000
+    for t in range(T):
+        _, q, _ = O.encode_bucket(cfg, 0, t, 0, v)
+        acc += q
+    m = float(table[0])
+    # each element's variance is at most m^2 / 4 per step
+    assert np.all(np.abs(acc / T - v) <= 5 * (m / 2) / math.sqrt(T))
+
+
+def _gamma_table():
+    return {int(r[0]): r[1] for r in _rows("elias_gamma.txt")}
+
+
+def _elias_stream_bits(codes, s):
+    """Concatenated codewords of the codes' symbols, from the golden table (x <= 17)."""
+    tab = _gamma_table()
+    z0 = (s - 1) // 2
+    out = []
+    for c in codes:
+        z = int(c) - z0
+        x = 2 * z + 1 if z >= 0 else -2 * z
+        out.append(tab[x])
+    return "".join(out)
+
+
+def test_elias_gamma_lengths_match_table():
+    for x, w in _gamma_table().items():
+        assert O.elias_gamma_len(x) == len(w)
+
+
+@pytest.mark.parametrize("scheme,levels", [(O.QSGD, 5), (O.TERNGRAD, 3), (O.QSGD_NEAREST, 9),
+                                           (O.QSGD_L2, 3), (O.QSGD_L2, 15), (O.QSGD, 15)])
+def test_elias_stream_offsets_and_round_trip(scheme, levels):
+    """The stream is the codewords of every valid code in order (built here from the golden
+    table), the header holds T and each bucket's first bit, the level tables are copied, and
+    unpacking gives the dense message back."""
+    for d, n in ((128, 128 * 3 + 5), (512, 512 * 2)):
+        rng = np.random.default_rng(d + levels + scheme)
+        cfg = O.Config(scheme, levels, d, 1, 0, 0.0, 3, n)
+        g = (rng.laplace(0, 1e-3, n)).astype(np.float32)
+        msg = O.encode(cfg, 0, 1, g)
+        emsg, used = O.elias_pack(cfg, msg)
+        cap, ooff, toff, soff = O.elias_layout(cfg)
+        nb = O.num_buckets(cfg)
+        _, coff, loff = O.message_layout(cfg)
+        dw = d * O.bits(levels) // 32
+        words = msg[coff:].view(np.uint32)
+        bits, offs = "", []
+        for bk in range(nb):
+            nv = min(d, n - bk * d)
+            offs.append(len(bits))
+            bits += _elias_stream_bits(O.unpack_bucket(cfg, words[bk * dw:(bk + 1) * dw], nv), levels)
+        T = int(emsg[:8].view(np.uint64)[0])
+        assert T == len(bits)
+        assert list(emsg[ooff:ooff + 8 * nb].view(np.uint64)) == offs
+        stream = 0
+        for k, ch in enumerate(bits):
+            if ch == "1":
+                stream |= 1 << k
+        nwords = (T + 31) // 32
+        got = emsg[soff:soff + 4 * nwords].view(np.uint32)
+        assert [int(x) for x in got] == [(stream >> (32 * k)) & 0xffffffff for k in range(nwords)]
+        assert not emsg[soff + 4 * nwords:].any()
+        assert used == soff + -(-4 * nwords // 16) * 16
+        L = O.table_len(scheme, levels)
+        assert np.array_equal(emsg[toff:toff + 4 * L * nb], msg[loff:loff + 4 * L * nb])
+        assert np.array_equal(O.elias_unpack(cfg, emsg), msg)
+
+
+def test_elias_unsupported():
+    for scheme, levels in ((O.ORQ, 5), (O.QSGD, 4), (O.BINGRAD_B, 2), (O.SIGNSGD, 2), (O.QSGD_L2, 2)):
+        assert O.elias_layout(O.Config(scheme, levels, 512, 1, 0, 0.0, 0, 1000)) is None
+
+
+def test_elias_expected_length_qsgd_l2():
+    """QSGD-l2 with 3 levels: element i is non-zero with probability |u_i| / m, so its codeword
+    has 1 + 2 |u_i| / m bits on average; the realised stream length over 50 steps agrees within
+    five standard deviations."""
+    rng = np.random.default_rng(92)
+    d, n, steps = 512, 512 * 8, 50
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    cfg = O.Config(O.QSGD_L2, 3, d, 1, 0, 0.0, 11, n)
+    mean = var = 0.0
+    for bk in range(n // d):
+        u = g[bk * d:(bk + 1) * d]
+        p = np.abs(u.astype(np.float64)) / O.l2_scale(u)
+        mean += float(np.sum(1 + 2 * p))
+        var += float(np.sum(4 * p * (1 - p)))
+    total = 0
+    for t in range(steps):
+        emsg, _ = O.elias_pack(cfg, O.encode(cfg, 0, t, g))
+        total += int(emsg[:8].view(np.uint64)[0])
+    assert abs(total - steps * mean) <= 5 * math.sqrt(steps * var)
+    assert total / (steps * n) < 1.1   # about 1.06 bits per element against 2 for the dense codes
