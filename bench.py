@@ -77,9 +77,9 @@ def measured_hbm_peak():
 
 
 def table_len(scheme_id, levels):
-    """Floats per level table: the scale for QSGD / TernGrad / QSGD-nearest, two levels for
-    BinGrad-b / BinGrad-pb / SignSGD, s levels for ORQ."""
-    return 1 if scheme_id in (0, 1, 5) else (2 if scheme_id in (2, 3, 6) else levels)
+    """Floats per level table: the scale for the QSGD family (QSGD, TernGrad, QSGD-nearest,
+    QSGD-l2), two levels for BinGrad-b / BinGrad-pb / SignSGD, s levels for ORQ."""
+    return 1 if scheme_id in (0, 1, 5, 7) else (2 if scheme_id in (2, 3, 6) else levels)
 
 
 def bytes_per_worker_elem(scheme_id, levels, d, W, ef, msgs):

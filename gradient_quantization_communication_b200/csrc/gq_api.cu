@@ -35,7 +35,7 @@ int bits_for(int s)
 
 int table_len(int scheme, int s)
 {
-    if (scheme == GQ_QSGD || scheme == GQ_TERNGRAD || scheme == GQ_QSGD_NEAREST) return 1;
+    if (scheme == GQ_QSGD || scheme == GQ_TERNGRAD || scheme == GQ_QSGD_NEAREST || scheme == GQ_QSGD_L2) return 1;
     if (scheme == GQ_BINGRAD_B || scheme == GQ_BINGRAD_PB || scheme == GQ_SIGNSGD) return 2;
     return s;
 }
@@ -49,6 +49,7 @@ gq_status_t normalise(const gq_config_t *in, gq_config_t *out)
     case GQ_QSGD:
     case GQ_ORQ:
     case GQ_QSGD_NEAREST:
+    case GQ_QSGD_L2:
         if (c.levels < 2 || c.levels > GQ_MAX_LEVELS) return GQ_ERR_INVALID;
         break;
     case GQ_TERNGRAD:
@@ -69,7 +70,8 @@ gq_status_t normalise(const gq_config_t *in, gq_config_t *out)
     if (!(c.clip_sigma >= 0.0f) || !std::isfinite(c.clip_sigma)) return GQ_ERR_INVALID;
     if (c.n < 0 || c.n >= (int64_t(1) << 40)) return GQ_ERR_INVALID;
     // the biased baselines are built for the register path only
-    if ((c.scheme == GQ_QSGD_NEAREST || c.scheme == GQ_SIGNSGD) && c.bucket > 512) return GQ_ERR_UNSUPPORTED;
+    if ((c.scheme == GQ_QSGD_NEAREST || c.scheme == GQ_SIGNSGD || c.scheme == GQ_QSGD_L2) && c.bucket > 512)
+        return GQ_ERR_UNSUPPORTED;
     *out = c;
     return GQ_OK;
 }

@@ -128,7 +128,8 @@ cudaError_t launch_bits(const KParams &p, cudaStream_t stream)
 
 cudaError_t launch_decode(const KParams &p, cudaStream_t stream)
 {
-    const bool qsgd = p.scheme == GQ_QSGD || p.scheme == GQ_TERNGRAD || p.scheme == GQ_QSGD_NEAREST;
+    const bool qsgd =
+        p.scheme == GQ_QSGD || p.scheme == GQ_TERNGRAD || p.scheme == GQ_QSGD_NEAREST || p.scheme == GQ_QSGD_L2;
     return qsgd ? launch_bits<true>(p, stream) : launch_bits<false>(p, stream);
 }
 

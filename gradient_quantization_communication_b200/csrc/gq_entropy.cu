@@ -193,7 +193,7 @@ struct Layouts {
 
 int table_len(int scheme, int s)
 {
-    if (scheme == GQ_QSGD || scheme == GQ_TERNGRAD || scheme == GQ_QSGD_NEAREST) return 1;
+    if (scheme == GQ_QSGD || scheme == GQ_TERNGRAD || scheme == GQ_QSGD_NEAREST || scheme == GQ_QSGD_L2) return 1;
     if (scheme == GQ_BINGRAD_B || scheme == GQ_BINGRAD_PB || scheme == GQ_SIGNSGD) return 2;
     return s;
 }

@@ -88,7 +88,7 @@ extern "C" GQ_API gq_status_t gq_quant_error_noalloc(const gq_config_t *cfg, uin
     p.scheme = c.scheme;
     p.s = c.levels;
     p.bits = bits;
-    p.L = (c.scheme == GQ_QSGD || c.scheme == GQ_TERNGRAD || c.scheme == GQ_QSGD_NEAREST) ? 1
+    p.L = (c.scheme == GQ_QSGD || c.scheme == GQ_TERNGRAD || c.scheme == GQ_QSGD_NEAREST || c.scheme == GQ_QSGD_L2) ? 1
           : (c.scheme == GQ_BINGRAD_B || c.scheme == GQ_BINGRAD_PB || c.scheme == GQ_SIGNSGD) ? 2
                                                                                                : c.levels;
     p.d = c.bucket;

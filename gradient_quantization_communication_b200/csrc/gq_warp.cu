@@ -9,8 +9,8 @@ cudaError_t launch_warp_bingrad(const KParams &p, bool fused, cudaStream_t strea
 cudaError_t launch_warp_err_orq(const KParams &p, double *part, cudaStream_t stream);
 cudaError_t launch_warp_err_qsgd(const KParams &p, double *part, cudaStream_t stream);
 cudaError_t launch_warp_err_bingrad(const KParams &p, double *part, cudaStream_t stream);
-cudaError_t launch_warp_biased(const KParams &p, bool fused, cudaStream_t stream);
-cudaError_t launch_warp_err_biased(const KParams &p, double *part, cudaStream_t stream);
+cudaError_t launch_warp_extra(const KParams &p, bool fused, cudaStream_t stream);
+cudaError_t launch_warp_err_extra(const KParams &p, double *part, cudaStream_t stream);
 
 cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream)
 {
@@ -20,7 +20,8 @@ cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream
     case GQ_BINGRAD_B:
     case GQ_BINGRAD_PB: return launch_warp_bingrad(p, fused, stream);
     case GQ_QSGD_NEAREST:
-    case GQ_SIGNSGD: return launch_warp_biased(p, fused, stream);
+    case GQ_SIGNSGD:
+    case GQ_QSGD_L2: return launch_warp_extra(p, fused, stream);
     default: return launch_warp_orq(p, fused, stream);
     }
 }
@@ -33,7 +34,8 @@ cudaError_t launch_warp_err(const KParams &p, double *part, cudaStream_t stream)
     case GQ_BINGRAD_B:
     case GQ_BINGRAD_PB: return launch_warp_err_bingrad(p, part, stream);
     case GQ_QSGD_NEAREST:
-    case GQ_SIGNSGD: return launch_warp_err_biased(p, part, stream);
+    case GQ_SIGNSGD:
+    case GQ_QSGD_L2: return launch_warp_err_extra(p, part, stream);
     default: return launch_warp_err_orq(p, part, stream);
     }
 }

@@ -22,6 +22,7 @@
 //   BinGrad-b       : warp bitonic sort, exact int64 prefix sums, screened argmax of J(k)
 //   BinGrad-pb      : shared-memory moments of 16-bit positions, exact search of all pairs
 //   QSGD-nearest    : the QSGD levels, rounding to the nearest level (no draws)
+//   QSGD-l2         : the QSGD levels scaled by ||u||_2 (exact fixed-point sum of squares)
 //   SignSGD         : m1 = mean |u| from an exact fixed-point warp sum, levels -m1 and +m1
 // The last bucket, when ragged, is handled by a one-warp launch of the same code with guarded
 // plain loads, so the main kernel carries no tail logic.
@@ -181,7 +182,10 @@ __device__ __forceinline__ void build_orq_tables(const KParams &p, FitORQ &sm, i
 // ---------------------------------------------------------------------------------------------
 // Per-scheme fits (u: the values to quantize; v: the error-fed values the residual refers to)
 // ---------------------------------------------------------------------------------------------
-template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0, bool NEAREST = false>
+// L2: the scale is ||u||_2 instead of max|u|, from the exact int64 sum of the squares of
+// round(u * 2^e), e = 20 - floor(log2 max|u|) (the clip's fixed point):
+// m = fp32(sqrt(SXX) * 2^-e) in binary64.
+template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0, bool NEAREST = false, bool L2 = false>
 __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                          const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
@@ -191,6 +195,23 @@ __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int
         if (!TAIL || ((vmask >> t) & 1u)) m = fmax_nan(m, fabsf(u[t]));
     m = warp_redux_max_abs(m);
     if (check && !(m <= FLT_MAX)) flag_nonfinite(p, lane);
+    if constexpr (L2) {
+        if (m > 0.0f && m <= FLT_MAX) {
+            const int e = 20 - fexpo(m);
+            const double sc = pow2d(e);
+            long long sxx = 0;
+#pragma unroll
+            for (int t = 0; t < EPL; ++t)
+                if (!TAIL || ((vmask >> t) & 1u)) {
+                    const long long X = fixed_point(u[t], sc);
+                    sxx += X * X;
+                }
+            sxx = warp_sum(sxx);
+            m = __double2float_rn(__dmul_rn(__dsqrt_rn(__ll2double_rn(sxx)), pow2d(-e)));
+        } else if (!(m > 0.0f)) {
+            m = 0.0f;  // zero bucket (NaN: unspecified, flagged)
+        }
+    }
     const int s = p.s;
     const float lv = lane < s ? __fmul_rn(m, p.qratio[lane]) : 0.0f;
     const float lv_next = __shfl_down_sync(kFull, lv, 1);
@@ -676,6 +697,8 @@ __device__ __forceinline__ void process(const KParams &p, typename FitFor<SCHEME
         fit_qsgd<EPL, FUSED, TAIL, BITS, IO>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
     else if constexpr (SCHEME == GQ_QSGD_NEAREST)
         fit_qsgd<EPL, FUSED, TAIL, BITS, IO, true>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
+    else if constexpr (SCHEME == GQ_QSGD_L2)
+        fit_qsgd<EPL, FUSED, TAIL, BITS, IO, false, true>(p, fit, beta, w, lane, vmask, check, v, u, acc, ea);
     else if constexpr (SCHEME == GQ_SIGNSGD)
         fit_sign<EPL, FUSED, TAIL, BITS, IO>(p, beta, w, lane, vmask, check, nvalid, v, u, acc, ea);
     else if constexpr (SCHEME == GQ_ORQ)

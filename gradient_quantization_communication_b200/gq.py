@@ -10,11 +10,12 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgq.so")
 
-GQ_QSGD, GQ_TERNGRAD, GQ_BINGRAD_B, GQ_BINGRAD_PB, GQ_ORQ, GQ_QSGD_NEAREST, GQ_SIGNSGD = 0, 1, 2, 3, 4, 5, 6
+GQ_QSGD, GQ_TERNGRAD, GQ_BINGRAD_B, GQ_BINGRAD_PB, GQ_ORQ, GQ_QSGD_NEAREST, GQ_SIGNSGD, GQ_QSGD_L2 = range(8)
 GQ_OK, GQ_ERR_INVALID, GQ_ERR_UNSUPPORTED, GQ_ERR_CUDA, GQ_ERR_NONFINITE, GQ_ERR_NOMEM, GQ_ERR_TIMEOUT = 0, 1, 2, 3, 4, 5, 6
 GQ_MAX_WORKERS = 64
 SCHEMES = {"qsgd": GQ_QSGD, "terngrad": GQ_TERNGRAD, "bingrad_b": GQ_BINGRAD_B,
-           "bingrad_pb": GQ_BINGRAD_PB, "orq": GQ_ORQ, "qsgd_nearest": GQ_QSGD_NEAREST, "signsgd": GQ_SIGNSGD}
+           "bingrad_pb": GQ_BINGRAD_PB, "orq": GQ_ORQ, "qsgd_nearest": GQ_QSGD_NEAREST, "signsgd": GQ_SIGNSGD,
+           "qsgd_l2": GQ_QSGD_L2}
 
 
 class gq_config_t(ctypes.Structure):

@@ -58,8 +58,11 @@ typedef enum {
      * and "Ternary and binary quantization"); buckets of d <= 512 only: */
     GQ_QSGD_NEAREST = 5, /* the QSGD-s levels and message, each value rounded to its nearest level (ties to the
                           * upper one), no randomness; s = 3 is deterministic TernGrad, s = 15 symmetric INT4 */
-    GQ_SIGNSGD = 6       /* scaled sign: levels -m1 and +m1, m1 = mean |u| of the bucket (exact fixed-point
+    GQ_SIGNSGD = 6,      /* scaled sign: levels -m1 and +m1, m1 = mean |u| of the bucket (exact fixed-point
                           * sum), code 1 for u >= 0; 1 bit per element */
+    /* QSGD as published (l2 scaling; the glossary's QSGD, whose codes are Elias-coded), d <= 512: */
+    GQ_QSGD_L2 = 7       /* the QSGD-s levels and stochastic rounding with m = ||u||_2 of the bucket (exact
+                          * fixed-point sum of squares) in place of max |u|; sparse codes for gq_elias_pack */
 } gq_scheme_t;
 
 typedef enum {
@@ -76,10 +79,10 @@ typedef enum {
  * Configuration of a plan.
  *   scheme         gq_scheme_t.
  *   levels         s.  QSGD: 2..16.  TernGrad: 3 (0 means 3).  BinGrad-b/pb: 2 (0 means 2).
- *                  ORQ: 2..16.  QSGD-nearest: 2..16.  SignSGD: 2 (0 means 2).  Codes take
+ *                  ORQ: 2..16.  QSGD-nearest, QSGD-l2: 2..16.  SignSGD: 2 (0 means 2).  Codes take
  *                  b = ceil(log2 s) bits (1..4).
  *   bucket         d, elements per bucket: a power of two in [128, 32768] (at most 512 for
- *                  QSGD-nearest and SignSGD: GQ_ERR_UNSUPPORTED above).  The vector is cut
+ *                  QSGD-nearest, SignSGD and QSGD-l2: GQ_ERR_UNSUPPORTED above).  The vector is cut
  *                  into ceil(n/d) buckets; the last one may hold fewer than d elements.
  *   workers        W in [1, 64] for gq_fused_step (gq_encode ignores it).
  *   error_feedback 1: v = g + r is quantized and r <- v - Q(v); 0: v = g, no residual.
@@ -109,7 +112,7 @@ GQ_API gq_status_t gq_config_check(const gq_config_t *cfg);
  * Layout of one worker's message, the bytes a worker would transmit (host computation, no
  * device needed).  *bytes: total size.  *codes_off: offset of the packed codes, ceil(n/d)
  * buckets of d*b/32 uint32 words each.  *levels_off: offset (16-byte aligned) of the level
- * tables, ceil(n/d) tables of L float32 each (L = 1 for QSGD/TernGrad/QSGD-nearest: the scale m;
+ * tables, ceil(n/d) tables of L float32 each (L = 1 for the QSGD family: the scale m;
  * 2 for BinGrad-b/pb and SignSGD: the two levels; s for ORQ: the ascending levels).
  * Packing inside a bucket: dense, in element order, least significant bit first: bit j of the
  * code (the index of its level) of element e is bit (b*e + j) % 32 of word (b*e + j) / 32 of

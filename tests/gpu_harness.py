@@ -6,7 +6,7 @@ import torch
 import gradient_quantization_communication_b200.gq as G
 import oracle as O
 
-SCHEME_ID = {"qsgd": 0, "terngrad": 1, "bingrad_b": 2, "bingrad_pb": 3, "orq": 4, "qsgd_nearest": 5, "signsgd": 6}
+SCHEME_ID = {"qsgd": 0, "terngrad": 1, "bingrad_b": 2, "bingrad_pb": 3, "orq": 4, "qsgd_nearest": 5, "signsgd": 6, "qsgd_l2": 7}
 
 
 def configs(scheme, levels, d, W, ef, clip, seed, n):

@@ -53,7 +53,7 @@ def test_version_and_status_strings():
     (dict(scheme="terngrad", levels=5), False),
     (dict(scheme="bingrad_b", levels=0), True),
     (dict(scheme="bingrad_pb", levels=3), False),
-    (dict(scheme=7, levels=3), False),
+    (dict(scheme=8, levels=3), False),
     (dict(scheme="orq", levels=5, bucket=64), False),
     (dict(scheme="orq", levels=5, bucket=384), False),
     (dict(scheme="orq", levels=5, bucket=65536), False),
@@ -158,7 +158,7 @@ def test_entropy_compression_ratio_d512(scheme, levels, ratio):
 
 
 
-@pytest.mark.parametrize("scheme,levels", [(5, 2), (5, 3), (5, 15), (5, 16), (6, 2), (6, 0)])
+@pytest.mark.parametrize("scheme,levels", [(5, 2), (5, 3), (5, 15), (5, 16), (6, 2), (6, 0), (7, 3), (7, 16)])
 @pytest.mark.parametrize("d", [128, 256, 512])
 @pytest.mark.parametrize("n", [0, 1, 1000, 10 ** 9])
 def test_biased_layout_matches_oracle(scheme, levels, d, n):
@@ -170,6 +170,8 @@ def test_biased_layout_matches_oracle(scheme, levels, d, n):
 @pytest.mark.parametrize("kw,status", [
     (dict(scheme="qsgd_nearest", levels=5, bucket=1024), "GQ_ERR_UNSUPPORTED"),
     (dict(scheme="signsgd", levels=2, bucket=2048), "GQ_ERR_UNSUPPORTED"),
+    (dict(scheme="qsgd_l2", levels=3, bucket=1024), "GQ_ERR_UNSUPPORTED"),
+    (dict(scheme="qsgd_l2", levels=3, bucket=512), "GQ_OK"),
     (dict(scheme="signsgd", levels=3, bucket=512), "GQ_ERR_INVALID"),
     (dict(scheme="qsgd_nearest", levels=17, bucket=512), "GQ_ERR_INVALID"),
     (dict(scheme="qsgd_nearest", levels=1, bucket=512), "GQ_ERR_INVALID"),
