@@ -62,6 +62,10 @@ def parse_args():
     ap.add_argument("--entropy", action="store_true",
                     help="base-s packing: gq_entropy_pack then gq_entropy_unpack of the W messages of one "
                          "step; per-kernel rooflines and the compression ratios, one JSON line")
+    ap.add_argument("--elias", action="store_true",
+                    help="Elias-gamma coding: gq_elias_pack then gq_elias_unpack of the W messages of one "
+                         "step (an odd-level QSGD-family scheme, e.g. --scheme qsgd_l2 --levels 3); "
+                         "per-call rooflines and the bits per element, one JSON line")
     return ap.parse_args()
 
 
@@ -680,6 +684,109 @@ def run_entropy(args):
     return 0
 
 
+def run_elias(args):
+    """Elias-gamma coding of the W messages of one fused step: a timed step is gq_elias_pack of
+    every worker's message (five launches) followed by gq_elias_unpack of every Elias message
+    (one launch), each call timed with events on the launching stream.  After timing, every
+    unpacked message must equal its dense message byte for byte."""
+    import numpy as np
+    import torch
+
+    import gradient_quantization_communication_b200.gq as G
+    from gradient_quantization_communication_b200 import synth
+
+    wl = synth.WORKLOADS[args.workload]
+    if args.elements:
+        wl = dataclasses.replace(wl, n=min(wl.n, args.elements))
+    W, n, d, ef = wl.workers, wl.n, args.bucket, wl.error_feedback
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    sid = G.SCHEMES[args.scheme]
+    cfg = G.gq_config(sid, args.levels, d, W, ef, args.clip, wl.rounding_seed, n)
+    stream = torch.cuda.current_stream()
+    plan = G.Plan(cfg)
+    msgs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)]
+    g = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
+    for w in range(W):
+        synth.gradient(args.workload, w, 0, n=n, out=g[w])
+    r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)] if ef else None
+    avg = torch.empty(n, dtype=torch.float32, device=dev)
+    G.gq_fused_step(plan.handle, 0, g, r, msgs, avg, stream)
+    if G.gq_plan_status(plan.handle, stream) != G.GQ_OK:
+        raise RuntimeError("non-finite input in the benchmark workload")
+    plan.close()
+    del g, r, avg
+    torch.cuda.empty_cache()
+    cap, _, _, _ = G.gq_elias_layout(cfg)
+    emsgs = [torch.empty(cap, dtype=torch.uint8, device=dev) for _ in range(W)]
+    backs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)]
+
+    def step(evs=None):
+        for w in range(W):
+            if evs is not None:
+                evs[w][0].record(stream)
+            G.gq_elias_pack(cfg, msgs[w], emsgs[w], stream)
+            if evs is not None:
+                evs[w][1].record(stream)
+        for w in range(W):
+            if evs is not None:
+                evs[W + w][0].record(stream)
+            G.gq_elias_unpack(cfg, emsgs[w], backs[w], stream)
+            if evs is not None:
+                evs[W + w][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(pci_bus_id(dev))
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2 * W)]
+           for _ in range(args.steps)]
+    sampler.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    for w in range(W):
+        if not torch.equal(backs[w], msgs[w]):
+            raise RuntimeError("Elias round trip differs for worker %d" % w)
+    ms = t0.elapsed_time(t1) / args.steps
+    pack_ms = statistics.mean(a.elapsed_time(b) for e in evs for a, b in e[:W])
+    unpack_ms = statistics.mean(a.elapsed_time(b) for e in evs for a, b in e[W:])
+    T = [int(e[:8].cpu().numpy().view(np.uint64)[0]) for e in emsgs]
+    used = [G.gq_elias_used_bytes(cfg, t) for t in T]
+    bits = (args.levels - 1).bit_length()
+    L = table_len(sid, args.levels)
+    nb = (n + d - 1) // d
+    dense_b = nb * (d * bits // 8 + 4 * L)
+    elias_b = statistics.mean(used)
+    # algorithmic bytes of one call: the dense message read and the Elias message written (or
+    # the reverse); pack also reads and writes the per-bucket counts once more for the scan
+    algo = dense_b + elias_b
+    peak, peak_kind = measured_hbm_peak()
+
+    def roof(bytes_per_call, call_ms):
+        a = bytes_per_call / (call_ms / 1000.0) / 1e9
+        return {"bound": "hbm", "achieved": round(a, 1), "peak": peak, "unit": "GB/s", "frac": round(a / peak, 4),
+                "peak_kind": peak_kind, "algorithmic_bytes_per_call": bytes_per_call, "ms_per_call": call_ms}
+
+    print(json.dumps({
+        "metric": "Elias-gamma pack + unpack of the W messages, worker-elements/s", "value": W * n / (ms / 1000.0),
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "u32", "data": "synthetic", "config": workload_config(args, wl),
+        "pack": roof(algo, pack_ms), "unpack": roof(algo, unpack_ms),
+        "compression": {"dense_bits_per_elem": 8.0 * dense_b / n, "stream_bits_per_elem": statistics.mean(T) / n,
+                        "elias_bits_per_elem": 8.0 * elias_b / n,
+                        "ratio_vs_fp32_dense": round(32.0 * n / (8.0 * dense_b), 3),
+                        "ratio_vs_fp32_elias": round(32.0 * n / (8.0 * elias_b), 3)},
+        "round_trip": "exact", "gpu_launches": 6 * W * args.steps, "clocks": clocks}))
+    return 0
+
+
 def run_sweep(args):
     """Fused-step throughput and normalised quantization variance sum (b-u)(u-a) / sum u^2 for
     every bucket size of the sweep workload, for ORQ-5 and QSGD-5."""
@@ -747,6 +854,8 @@ def main():
         return run_unfused(args)
     if args.entropy:
         return run_entropy(args)
+    if args.elias:
+        return run_elias(args)
     return run_gq(args)
 
 

@@ -58,13 +58,19 @@ def lib():
         L.gq_entropy_layout.argtypes = [cfgp, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)]
         L.gq_entropy_pack.argtypes = [cfgp, vp, vp, vp]
         L.gq_entropy_unpack.argtypes = [cfgp, vp, vp, vp]
+        L.gq_elias_layout.argtypes = [cfgp, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz),
+                                      ctypes.POINTER(sz)]
+        L.gq_elias_used_bytes.argtypes = [cfgp, ctypes.c_uint64, ctypes.POINTER(sz)]
+        L.gq_elias_pack.argtypes = [cfgp, vp, vp, vp]
+        L.gq_elias_unpack.argtypes = [cfgp, vp, vp, vp]
         L.gq_status_string.argtypes = [ctypes.c_int]
         L.gq_status_string.restype = ctypes.c_char_p
         L.gq_version.restype = ctypes.c_char_p
         for f in ("gq_config_check", "gq_message_layout", "gq_plan_create", "gq_plan_destroy", "gq_encode",
                   "gq_decode_accumulate", "gq_fused_step", "gq_quant_error", "gq_quant_error_noalloc",
                   "gq_plan_status", "gq_selftest_bounded_wait", "gq_entropy_layout", "gq_entropy_pack",
-                  "gq_entropy_unpack"):
+                  "gq_entropy_unpack", "gq_elias_layout", "gq_elias_used_bytes", "gq_elias_pack",
+                  "gq_elias_unpack"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -176,6 +182,27 @@ def gq_entropy_pack(cfg, msg, emsg, stream=None):
 
 def gq_entropy_unpack(cfg, emsg, msg, stream=None):
     _check(lib().gq_entropy_unpack(ctypes.byref(cfg), _ptr(emsg), _ptr(msg), _stream(stream)), "gq_entropy_unpack")
+
+
+def gq_elias_layout(cfg):
+    """(capacity bytes, offsets_off, tables_off, stream_off)."""
+    v = [ctypes.c_size_t() for _ in range(4)]
+    _check(lib().gq_elias_layout(ctypes.byref(cfg), *[ctypes.byref(x) for x in v]), "gq_elias_layout")
+    return tuple(x.value for x in v)
+
+
+def gq_elias_used_bytes(cfg, stream_bits):
+    b = ctypes.c_size_t()
+    _check(lib().gq_elias_used_bytes(ctypes.byref(cfg), int(stream_bits), ctypes.byref(b)), "gq_elias_used_bytes")
+    return b.value
+
+
+def gq_elias_pack(cfg, msg, emsg, stream=None):
+    _check(lib().gq_elias_pack(ctypes.byref(cfg), _ptr(msg), _ptr(emsg), _stream(stream)), "gq_elias_pack")
+
+
+def gq_elias_unpack(cfg, emsg, msg, stream=None):
+    _check(lib().gq_elias_unpack(ctypes.byref(cfg), _ptr(emsg), _ptr(msg), _stream(stream)), "gq_elias_unpack")
 
 
 def gq_status_string(status):

@@ -238,6 +238,45 @@ GQ_API gq_status_t gq_entropy_layout(const gq_config_t *cfg, size_t *bytes, size
 GQ_API gq_status_t gq_entropy_pack(const gq_config_t *cfg, const void *msg, void *emsg, void *stream);
 GQ_API gq_status_t gq_entropy_unpack(const gq_config_t *cfg, const void *emsg, void *msg, void *stream);
 
+/*
+ * Elias-gamma coding of a message's codes.  The glossary "Gradient Quantization" (section QSGD)
+ * says QSGD encodes its quantized values with Elias integer coding for further lossless
+ * compression.  Elias gamma (Elias, 1975) writes x >= 1 with N = floor(log2 x) as N zero bits
+ * followed by x's N + 1 bits, most significant first.  Supported: the QSGD family (QSGD,
+ * TernGrad, QSGD-nearest, QSGD-l2) with an odd number of levels s and d <= 512; anything else
+ * returns GQ_ERR_UNSUPPORTED.  Code c is sent as the signed level z = c - (s-1)/2, zigzag-mapped
+ * to x = 2z + 1 (z >= 0) or -2z (z < 0): the zero level costs one bit.
+ *
+ * Message, little-endian: [uint64 T: the stream's bit count][8 zero bytes][ceil(n/d) uint64:
+ * each bucket's first stream bit, padded to 16 bytes][the level tables, as in the dense message,
+ * padded to 16 bytes][the stream: every bucket's valid codes in element order, stream bit k is
+ * bit k % 32 of word k / 32, zero bits after T up to the next 16 bytes].  Its size depends on
+ * the data: gq_elias_used_bytes(T) of the gq_elias_layout capacity are written.
+ *
+ * gq_elias_layout: *cap_bytes the largest message (buffers are sized for it), and the offsets of
+ * the offsets region, the tables region and the stream.  Host computation; outputs may be NULL.
+ * gq_elias_used_bytes: bytes of a message whose stream holds `stream_bits` bits (T, read by the
+ * caller from the message's first 8 bytes).  GQ_ERR_INVALID if T exceeds the capacity.
+ */
+GQ_API gq_status_t gq_elias_layout(const gq_config_t *cfg, size_t *cap_bytes, size_t *offsets_off, size_t *tables_off,
+                                   size_t *stream_off);
+GQ_API gq_status_t gq_elias_used_bytes(const gq_config_t *cfg, uint64_t stream_bits, size_t *bytes);
+
+/*
+ * gq_elias_pack: dense message -> Elias message (five launches on `stream`; its level-table
+ * region serves as the scan's scratch before the tables are written).  gq_elias_unpack: the
+ * inverse (one launch).
+ *   msg   device, the dense message (gq_message_layout bytes): read by pack, written completely
+ *         by unpack.
+ *   emsg  device, gq_elias_layout capacity bytes: its first gq_elias_used_bytes(T) bytes are
+ *         written by pack (the rest is left as it was) and read by unpack.
+ * Both 16-byte aligned and not overlapping (GQ_ERR_INVALID otherwise).  Codes >= s in a dense
+ * message are encoded as s - 1; a damaged stream decodes to unspecified codes below 2^b, every
+ * read inside the capacity.  Stateless: no plan, no allocation.
+ */
+GQ_API gq_status_t gq_elias_pack(const gq_config_t *cfg, const void *msg, void *emsg, void *stream);
+GQ_API gq_status_t gq_elias_unpack(const gq_config_t *cfg, const void *emsg, void *msg, void *stream);
+
 /* Synchronize `stream`, then report and clear the plan's status flags: GQ_ERR_TIMEOUT if a
  * kernel's bounded wait for a bulk copy gave up (the kernel then stopped early; its outputs are
  * incomplete), else GQ_ERR_NONFINITE if a non-finite input was seen since the last call;

@@ -181,3 +181,42 @@ def test_biased_layout_matches_oracle(scheme, levels, d, n):
 def test_biased_config_check(kw, status):
     cfg = G.gq_config(kw["scheme"], kw["levels"], kw["bucket"], 1, True, 0.0, 0, 1000)
     assert G.gq_config_check(cfg) == getattr(G, status)
+
+
+@pytest.mark.parametrize("scheme,levels", [(0, 3), (0, 5), (1, 0), (5, 9), (7, 3), (7, 15)])
+@pytest.mark.parametrize("d", [128, 256, 512])
+@pytest.mark.parametrize("n", [0, 1, 1000, 10 ** 9])
+def test_elias_layout_matches_oracle(scheme, levels, d, n):
+    cfg = G.gq_config(scheme, levels, d, 1, True, 0.0, 0, n)
+    mine = G.gq_elias_layout(cfg)
+    ref = O.elias_layout(O.Config(scheme, levels or 3, d, 1, 1, 0.0, 0, n))
+    assert mine == ref
+    assert all(x % 16 == 0 for x in mine)
+    assert G.gq_elias_used_bytes(cfg, 0) == mine[3]
+    if n > 0:
+        assert G.gq_elias_used_bytes(cfg, 33) == mine[3] + 16
+
+
+@pytest.mark.parametrize("scheme,levels,d", [(4, 5, 512), (0, 4, 512), (0, 5, 1024), (2, 0, 512), (6, 2, 512),
+                                             (7, 2, 256)])
+def test_elias_unsupported(scheme, levels, d):
+    cfg = G.gq_config(scheme, levels, d, 1, True, 0.0, 0, 1000)
+    for call in (lambda: G.gq_elias_layout(cfg), lambda: G.gq_elias_pack(cfg, 0, 0, stream=0),
+                 lambda: G.gq_elias_unpack(cfg, 0, 0, stream=0)):
+        with pytest.raises(G.GQError) as ei:
+            call()
+        assert ei.value.status == G.GQ_ERR_UNSUPPORTED
+
+
+def test_elias_argument_checks_without_device():
+    cfg = G.gq_config("qsgd_l2", 3, 512, 1, True, 0.0, 0, 5000)
+    cap = G.gq_elias_layout(cfg)[0]
+    base = 1 << 40  # never dereferenced: every case fails its checks first
+    for a, b in [(0, base), (base, 0), (base + 8, base + (1 << 30)), (base, base + 16), (base + 16, base)]:
+        for call in (G.gq_elias_pack, G.gq_elias_unpack):
+            with pytest.raises(G.GQError) as ei:
+                call(cfg, a, b, stream=0)
+            assert ei.value.status == G.GQ_ERR_INVALID
+    with pytest.raises(G.GQError):
+        G.gq_elias_used_bytes(cfg, 8 * cap)
+    G.gq_elias_pack(G.gq_config("qsgd_l2", 3, 512, 1, True, 0.0, 0, 0), 0, 0, stream=0)

@@ -63,3 +63,13 @@ def test_entropy_line():
     # ORQ-5, d = 512: 38 words of codes per bucket against 48, plus the 5-float table
     assert abs(c["base_s_bits_per_elem"] - (38 * 32 + 5 * 32) / 512) < 1e-9
     assert abs(c["dense_bits_per_elem"] - (48 * 32 + 5 * 32) / 512) < 1e-9
+
+
+@pytest.mark.gpu
+def test_elias_line():
+    j = _run("--elias", "--scheme", "qsgd_l2", "--levels", "3", "--elements", "5120000", "--steps", "2",
+             "--warmup", "3")
+    assert j["value"] > 0 and j["pack"]["frac"] > 0 and j["unpack"]["frac"] > 0
+    assert j["round_trip"] == "exact" and j["gpu_launches"] == 6 * 8 * 2
+    c = j["compression"]
+    assert 1.0 <= c["stream_bits_per_elem"] < 1.3 and c["dense_bits_per_elem"] == (32 * 32 + 32) / 512
