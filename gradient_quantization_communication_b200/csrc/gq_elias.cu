@@ -28,8 +28,9 @@
 //      contiguous run of elements, the run's words built in a 64-bit register), then stores
 //      the words that lie wholly inside the bucket's bit range and ORs the two shared ones
 //      (atomicOr on words zeroed by steps 3 and 4); the level table is copied.
-// Unpack: k_decode, one thread per bucket, reads its codewords from its first bit and writes
-// the bucket's dense words; the level tables are copied.
+// Unpack: k_decode, one thread per bucket, reads its codewords from its first bit (one table
+// lookup on the next 7 bits per codeword) and writes the bucket's dense words; the level tables
+// are copied.  Count and encode take each code's codeword and length from 16-entry tables.
 //
 // Robustness: codes >= s in a dense message are encoded as s - 1, so the stream never exceeds
 // the capacity; a damaged stream decodes to unspecified codes below 2^b, with every read inside
@@ -59,11 +60,21 @@ struct ElParams {
     uint32_t *stream;
     int64_t nb, ntiles, cap_words;
     int d, s, b, L, dw, tail, z0;
+    // per code c (0..15, codes >= s taken as s - 1): its codeword in stream order (the N zero
+    // bits, then x most significant bit first; at most 7 bits) and its length
+    unsigned long long cw_lo, cw_hi;  // 8 bits per code: codes 0..7, 8..15
+    unsigned long long len_tab;       // 4 bits per code
+    // decoding: the next 7 stream bits -> code | length << 4 (one byte each)
+    unsigned char dec[128];
 };
 
 __device__ __forceinline__ int bucket_valid(const ElParams &p, int64_t bk) { return bk == p.nb - 1 ? p.tail : p.d; }
 
-__device__ __forceinline__ uint32_t symbol(int c, int z0) { return c >= z0 ? 2u * (c - z0) + 1u : 2u * (z0 - c); }
+__device__ __forceinline__ int code_len(const ElParams &p, int c) { return (int)((p.len_tab >> (4 * c)) & 15u); }
+__device__ __forceinline__ uint32_t code_word(const ElParams &p, int c)
+{
+    return (uint32_t)(((c < 8 ? p.cw_lo : p.cw_hi) >> (8 * (c & 7))) & 0xFFu);
+}
 
 // A lane's run of d/32 consecutive codes (at most 64 bits) in a window of three dense words
 // starting at word q0 = floor(b * e0 / 32); words past the bucket's end read as 0.
@@ -80,28 +91,32 @@ __device__ __forceinline__ Run load_run(const ElParams &p, const uint32_t *bw, i
     r.base = bit & 31;
     return r;
 }
-// code j of the run (codes >= s read as s - 1)
-__device__ __forceinline__ int run_code(const ElParams &p, const Run &r, int j)
+// code j of the run (the raw b bits; the tables map codes >= s to s - 1)
+template <int B>
+__device__ __forceinline__ int run_code(const Run &r, int j)
 {
-    const int bit = r.base + p.b * j;
+    const int bit = r.base + B * j;
     const uint64_t two = bit < 32 ? ((uint64_t)r.w[1] << 32) | r.w[0] : ((uint64_t)r.w[2] << 32) | r.w[1];
-    const uint32_t c = (uint32_t)(two >> (bit & 31)) & ((1u << p.b) - 1u);
-    return min((int)c, p.s - 1);
+    return (int)((uint32_t)(two >> (bit & 31)) & ((1u << B) - 1u));
 }
 
-__device__ __forceinline__ int gamma_len(uint32_t x) { return 2 * (31 - __clz(x)) + 1; }
-
 // ---- 1. counts ----------------------------------------------------------------------------
+template <int B>
 __global__ void __launch_bounds__(kWarpThreads) k_count(const __grid_constant__ ElParams p)
 {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * (kWarpThreads / 32);
-    for (int64_t bk = (int64_t)blockIdx.x * (kWarpThreads / 32) + (threadIdx.x >> 5); bk < p.nb; bk += nwarps) {
-        const int n = bucket_valid(p, bk);
-        const int per_lane = p.d / 32, e0 = lane * per_lane, cnt = min(per_lane, n - e0);
-        const Run r = load_run(p, p.dense + bk * p.dw, e0);
+    const int per_lane = p.d / 32, e0 = lane * per_lane;
+    int64_t bk = (int64_t)blockIdx.x * (kWarpThreads / 32) + (threadIdx.x >> 5);
+    Run nr{};
+    if (bk < p.nb) nr = load_run(p, p.dense + bk * p.dw, e0);
+    for (; bk < p.nb; bk += nwarps) {
+        const Run r = nr;
+        const int64_t nx = bk + nwarps;
+        if (nx < p.nb) nr = load_run(p, p.dense + nx * p.dw, e0);  // one bucket ahead
+        const int cnt = min(per_lane, bucket_valid(p, bk) - e0);
         int bits = 0;
-        for (int j = 0; j < cnt; ++j) bits += gamma_len(symbol(run_code(p, r, j), p.z0));
+        for (int j = 0; j < cnt; ++j) bits += code_len(p, run_code<B>(r, j));
         bits = __reduce_add_sync(kFull, (unsigned)bits);
         if (lane == 0) p.offs[bk] = (uint64_t)bits;
     }
@@ -206,6 +221,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_apply(const __grid_consta
 }
 
 // ---- 5. encode ----------------------------------------------------------------------------
+template <int B>
 __global__ void __launch_bounds__(kWarpThreads) k_encode(const __grid_constant__ ElParams p, int pad_floats)
 {
     __shared__ uint32_t stage_all[kWarpThreads / 32][kMaxStageWords];
@@ -215,12 +231,32 @@ __global__ void __launch_bounds__(kWarpThreads) k_encode(const __grid_constant__
     uint32_t *st = stage_all[wid];
     const int64_t nwarps = (int64_t)gridDim.x * (kWarpThreads / 32);
     const int per_lane = p.d / 32;
-    for (int64_t bk = (int64_t)blockIdx.x * (kWarpThreads / 32) + wid; bk < p.nb; bk += nwarps) {
+    const int e0 = lane * per_lane;
+    // software pipeline: the next bucket's code window, first bit and table entry are loaded
+    // before this bucket is written, so the warp waits on one round trip per bucket, not three
+    int64_t bk = (int64_t)blockIdx.x * (kWarpThreads / 32) + wid;
+    Run nr{};
+    uint64_t noff = 0;
+    float ntab = 0.0f;
+    if (bk < p.nb) {
+        nr = load_run(p, p.dense + bk * p.dw, e0);
+        noff = p.offs[bk];
+        if (lane < p.L) ntab = p.dtab[bk * p.L + lane];
+    }
+    for (; bk < p.nb; bk += nwarps) {
+        const Run rr = nr;
+        const uint64_t off = noff;
+        const float tab = ntab;
+        const int64_t nx = bk + nwarps;
+        if (nx < p.nb) {
+            nr = load_run(p, p.dense + nx * p.dw, e0);
+            noff = p.offs[nx];
+            if (lane < p.L) ntab = p.dtab[nx * p.L + lane];
+        }
         const int n = bucket_valid(p, bk);
-        const int e0 = lane * per_lane, cnt = min(per_lane, n - e0);
-        const Run rr = load_run(p, p.dense + bk * p.dw, e0);
+        const int cnt = min(per_lane, n - e0);
         int bits = 0;
-        for (int j = 0; j < cnt; ++j) bits += gamma_len(symbol(run_code(p, rr, j), p.z0));
+        for (int j = 0; j < cnt; ++j) bits += code_len(p, run_code<B>(rr, j));
         int incl = bits;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -228,7 +264,6 @@ __global__ void __launch_bounds__(kWarpThreads) k_encode(const __grid_constant__
             if (lane >= o) incl += y;
         }
         const int total = __shfl_sync(kFull, incl, 31);
-        const uint64_t off = p.offs[bk];
         const int base = (int)(off & 31u);
         const int nw = (base + total + 31) >> 5;
         for (int j = lane; j < nw; j += 32) st[j] = 0u;
@@ -239,11 +274,9 @@ __global__ void __launch_bounds__(kWarpThreads) k_encode(const __grid_constant__
             uint64_t acc = 0;
             bool first = true;
             for (int j = 0; j < cnt; ++j) {
-                const uint32_t x = symbol(run_code(p, rr, j), p.z0);
-                const int N = 31 - __clz(x);
-                const uint32_t cw = __brev(x) >> (31 - N);  // x's N + 1 bits, most significant first
-                acc |= (uint64_t)cw << (accbits + N);
-                accbits += 2 * N + 1;
+                const int c = run_code<B>(rr, j);
+                acc |= (uint64_t)code_word(p, c) << accbits;
+                accbits += code_len(p, c);
                 if (accbits >= 32) {
                     if (first) atomicOr(&st[wi], (uint32_t)acc);
                     else st[wi] = (uint32_t)acc;
@@ -264,7 +297,7 @@ __global__ void __launch_bounds__(kWarpThreads) k_encode(const __grid_constant__
             if (whole) p.stream[gw] = st[j];
             else atomicOr(&p.stream[gw], st[j]);
         }
-        if (lane < p.L) p.etab[bk * p.L + lane] = p.dtab[bk * p.L + lane];
+        if (lane < p.L) p.etab[bk * p.L + lane] = tab;
         __syncwarp();  // the stage is reused by the next bucket
     }
 }
@@ -276,16 +309,19 @@ __device__ __forceinline__ uint32_t stream_word(const ElParams &p, int64_t q)
 }
 
 // One thread per bucket.  The thread reads its stream through a 64-bit bit buffer refilled a
-// word at a time, with the next word's load issued one refill ahead, so that the decode loop
-// waits on memory about once per 32 stream bits rather than once per codeword.
+// word at a time, with the next word's load issued one refill ahead, and decodes one codeword
+// per lookup: the next 7 stream bits index a 128-entry shared table (code, length).
+template <int B>
 __global__ void __launch_bounds__(256) k_decode(const __grid_constant__ ElParams p, float *dtab_out,
                                                 uint32_t *dense_out, int pad_floats)
 {
+    __shared__ unsigned char dec[128];
+    if (threadIdx.x < 128) dec[threadIdx.x] = p.dec[threadIdx.x];
+    __syncthreads();
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
     for (int64_t j = tid; j < p.nb * p.L; j += nthreads) dtab_out[j] = p.etab[j];
     if (tid < pad_floats) dtab_out[p.nb * p.L + tid] = 0.0f;
-    const int cmax = (1 << p.b) - 1;
     for (int64_t bk = tid; bk < p.nb; bk += nthreads) {
         const int n = bucket_valid(p, bk);
         uint32_t *out = dense_out + bk * p.dw;
@@ -299,22 +335,17 @@ __global__ void __launch_bounds__(256) k_decode(const __grid_constant__ ElParams
         uint64_t acc = 0;
         int accbits = 0, wi = 0;
         for (int e = 0; e < n; ++e) {
-            if (nbuf < 32) {  // refill: a codeword has at most 31 bits
+            if (nbuf < 32) {  // refill: a codeword has at most 7 bits
                 buf |= (uint64_t)next << nbuf;
                 nbuf += 32;
                 next = stream_word(p, ++q);
             }
-            const uint32_t lo = (uint32_t)buf;
-            const int N = min(lo ? __ffs(lo) - 1 : 15, 15);  // leading zero bits of the codeword
-            const uint32_t y = (uint32_t)(buf >> N) & ((2u << N) - 1u);
-            const int len = 2 * N + 1;
+            const unsigned t = dec[(uint32_t)buf & 127u];
+            const int len = (int)(t >> 4);
             buf >>= len;
             nbuf -= len;
-            const uint32_t x = __brev(y) >> (31 - N);
-            const int z = (x & 1u) ? (int)((x - 1u) >> 1) : -(int)(x >> 1);
-            const int c = min(max(z + p.z0, 0), cmax);
-            acc |= (uint64_t)c << accbits;
-            accbits += p.b;
+            acc |= (uint64_t)(t & 15u) << accbits;
+            accbits += B;
             if (accbits >= 32) {
                 out[wi++] = (uint32_t)acc;
                 acc >>= 32;
@@ -396,6 +427,38 @@ ElParams make_params(const gq_config_t *cfg, const ElLayout &l, const void *msg,
     p.dw = cfg->bucket * l.b / 32;
     p.tail = (int)(cfg->n - (l.nb - 1) * (int64_t)cfg->bucket);
     p.z0 = (l.s - 1) / 2;
+    // codeword tables: code c -> z = c - z0 -> x = 2z + 1 (z >= 0) or -2z (z < 0) -> N zero bits,
+    // then x's N + 1 bits most significant first (stream order: first bit in bit 0)
+    p.cw_lo = p.cw_hi = p.len_tab = 0ull;
+    for (int c = 0; c < 16; ++c) {
+        const int cc = std::min(c, l.s - 1);
+        const int z = cc - p.z0;
+        const uint32_t x = z >= 0 ? (uint32_t)(2 * z + 1) : (uint32_t)(-2 * z);
+        int N = 0;
+        while ((x >> (N + 1)) != 0u) ++N;
+        uint32_t v = 0;
+        for (int j = 0; j <= N; ++j)  // bit N - j of x goes to stream position N + j
+            if ((x >> (N - j)) & 1u) v |= 1u << (N + j);
+        const unsigned long long vv = (unsigned long long)v << (8 * (c & 7));
+        if (c < 8) p.cw_lo |= vv;
+        else p.cw_hi |= vv;
+        p.len_tab |= (unsigned long long)(2 * N + 1) << (4 * c);
+    }
+    // decoding table over the next 7 stream bits (a codeword here has at most 7 bits); a bit
+    // pattern that starts no valid codeword decodes to code s - 1 and consumes 7 bits
+    for (int t = 0; t < 128; ++t) {
+        int N = 0;
+        while (N < 7 && !((t >> N) & 1)) ++N;
+        int code = l.s - 1, len = 7;
+        if (2 * N + 1 <= 7) {
+            uint32_t x = 0;
+            for (int j = 0; j <= N; ++j) x = (x << 1) | (uint32_t)((t >> (N + j)) & 1);
+            const int z = (x & 1u) ? (int)((x - 1u) / 2u) : -(int)(x / 2u);
+            code = std::min(std::max(z + p.z0, 0), (1 << l.b) - 1);
+            len = 2 * N + 1;
+        }
+        p.dec[t] = (unsigned char)(code | (len << 4));
+    }
     return p;
 }
 
@@ -454,12 +517,14 @@ gq_status_t gq_elias_pack(const gq_config_t *cfg, const void *msg, void *emsg, v
     const ElParams p = make_params(cfg, l, msg, emsg);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int g = warp_grid(l.nb);
-    k_count<<<g, kWarpThreads, 0, s>>>(p);
+    auto count = l.b == 2 ? k_count<2> : l.b == 3 ? k_count<3> : k_count<4>;
+    auto encode = l.b == 2 ? k_encode<2> : l.b == 3 ? k_encode<3> : k_encode<4>;
+    count<<<g, kWarpThreads, 0, s>>>(p);
     k_tile_sums<<<(unsigned)p.ntiles, kScanThreads, 0, s>>>(p);
     k_scan_top<<<1, kScanThreads, 0, s>>>(p);
     k_scan_apply<<<(unsigned)p.ntiles, kScanThreads, 0, s>>>(p);
     const int64_t tab = l.nb * l.L;
-    k_encode<<<g, kWarpThreads, 0, s>>>(p, (int)(((tab + 3) & ~int64_t(3)) - tab));
+    encode<<<g, kWarpThreads, 0, s>>>(p, (int)(((tab + 3) & ~int64_t(3)) - tab));
     return cudaGetLastError() == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
 }
 
@@ -480,7 +545,8 @@ gq_status_t gq_elias_unpack(const gq_config_t *cfg, const void *emsg, void *msg,
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((l.nb + 255) / 256, (int64_t)sms * 8));
-    k_decode<<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+    auto decode = l.b == 2 ? k_decode<2> : l.b == 3 ? k_decode<3> : k_decode<4>;
+    decode<<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
         p, reinterpret_cast<float *>(m + l.dense_levels_off), reinterpret_cast<uint32_t *>(m), pad);
     return cudaGetLastError() == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
 }
