@@ -16,7 +16,9 @@
 // of word k / 32; the bits after T zero up to the next 16 bytes].
 //
 // Pack, five launches on the caller's stream:
-//   1. k_count: one warp per bucket writes its codeword bit count into its header slot.
+//   1. k_count: one warp per bucket writes its codeword bit count into its header slot (each
+//      lane over a contiguous run of codes held in a three-word register window, the next
+//      bucket's window loaded one bucket ahead).
 //   2. k_tile_sums: one CTA per tile of 4096 buckets sums the counts into scratch, which is
 //      the message's level-table region (written last, by step 5).
 //   3. k_scan_top: one CTA turns the tile sums into exclusive prefix sums, writes T, and zeroes
