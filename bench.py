@@ -15,6 +15,13 @@ on: 71 GB resident in HBM, far larger than L2.  Metric: gradient worker-elements
 --impl reference times the CPU oracle (plain C, all host cores) on bounded samples of the same
 workload.  With N > 1 (torchrun) every rank runs an independent replica on its GPU: the path
 has no exchange between GPUs.
+
+Other one-line modes (one GPU):
+  --unfused   gq_encode per worker and gq_decode_accumulate, each against its own bytes
+  --sweep     bucket sizes 128 .. 32768: throughput and normalised quantization variance
+  --entropy   base-s packing of the W messages (gq_entropy_pack / gq_entropy_unpack)
+  --elias     Elias-gamma coding of the W messages (gq_elias_pack / gq_elias_unpack), for an
+              odd-level QSGD-family scheme such as --scheme qsgd_l2 --levels 3
 """
 import argparse
 import concurrent.futures as cf
