@@ -867,3 +867,30 @@ def test_elias_expected_length_qsgd_l2():
         total += int(emsg[:8].view(np.uint64)[0])
     assert abs(total - steps * mean) <= 5 * math.sqrt(steps * var)
     assert total / (steps * n) < 1.1   # about 1.06 bits per element against 2 for the dense codes
+
+
+@pytest.mark.parametrize("scheme,levels", [(O.ORQ, 5), (O.QSGD, 3), (O.BINGRAD_B, 2), (O.SIGNSGD, 2)])
+def test_fused_bucket_is_a_slice_of_the_step(scheme, levels):
+    """The per-bucket step (used to check sampled buckets of large workloads) gives, for every
+    bucket, exactly the slice of the whole-vector step: the average, the new residuals, the
+    packed words and the level tables; with error feedback over two steps."""
+    rng = np.random.default_rng(95 + scheme)
+    d, n, W = 128, 128 * 3 + 50, 3
+    cfg = O.Config(scheme, levels, d, W, 1, 0.0, 8, n)
+    rs = [np.zeros(n, np.float32) for _ in range(W)]
+    r_b = {b: [np.zeros(min(d, n - b * d), np.float32) for _ in range(W)] for b in range(O.num_buckets(cfg))}
+    words = d * O.bits(levels) // 32
+    L = O.table_len(scheme, levels)
+    _, coff, loff = O.message_layout(cfg)
+    for t in range(2):
+        gs = [(rng.laplace(0, 1e-3, n)).astype(np.float32) for _ in range(W)]
+        avg, msgs = O.fused_step(cfg, t, gs, rs)
+        for b in range(O.num_buckets(cfg)):
+            lo, hi = b * d, min(n, (b + 1) * d)
+            a_b, r_new, w_b, t_b = O.fused_bucket(cfg, t, b, [g[lo:hi] for g in gs], r_b[b])
+            assert np.array_equal(a_b.view(np.uint32), avg[lo:hi].view(np.uint32))
+            for w in range(W):
+                assert np.array_equal(r_new[w].view(np.uint32), rs[w][lo:hi].view(np.uint32))
+                assert np.array_equal(w_b[w], msgs[w][coff + 4 * words * b:coff + 4 * words * (b + 1)].view(np.uint32))
+                assert np.array_equal(t_b[w].view(np.uint32), msgs[w][loff + 4 * L * b:loff + 4 * L * (b + 1)].view(np.uint32))
+            r_b[b] = r_new
