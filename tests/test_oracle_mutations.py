@@ -57,6 +57,8 @@ MUTATIONS = [
     ("elias_bit_order", "for (int j = N; j >= 0; --j, ++k)", "for (int j = 0; j <= N; ++j, ++k)"),
     ("elias_offsets", "offs[bk] = k;", "offs[bk] = k + 1;"),
     ("l2_sqrt", "return (float)ldexp(sqrt((double)sxx), -e);", "return (float)ldexp((double)sxx, -e);"),
+    ("fused_bucket_sum", "for (int i = 0; i < n; ++i) acc[i] = acc[i] + q[i];",
+     "for (int i = 0; i < n; ++i) acc[i] = acc[i] + v[i];"),
 ]
 
 

@@ -873,7 +873,10 @@ def test_elias_expected_length_qsgd_l2():
 def test_fused_bucket_is_a_slice_of_the_step(scheme, levels):
     """The per-bucket step (used to check sampled buckets of large workloads) gives, for every
     bucket, exactly the slice of the whole-vector step: the average, the new residuals, the
-    packed words and the level tables; with error feedback over two steps."""
+    packed words and the level tables; with error feedback over two steps.  (The whole-vector
+    step is built from the per-bucket one; its arithmetic is pinned separately against encode
+    followed by decode, which share no code with it.  This checks the per-bucket interface:
+    slicing, the ragged last bucket and the residual chain.)"""
     rng = np.random.default_rng(95 + scheme)
     d, n, W = 128, 128 * 3 + 50, 3
     cfg = O.Config(scheme, levels, d, W, 1, 0.0, 8, n)
