@@ -493,6 +493,10 @@ def test_message_sizes_and_compression():
     for s, bits, ratio in rows[:2]:
         assert round(32 / math.log2(int(s)), 1) == float(ratio)
     assert O.bits(3) == 2 and O.bits(5) == 3 and O.bits(9) == 4 and O.bits(2) == 1
+    # the glossary's TernGrad (16x) and SignSGD (32x) figures are the codes alone: 2 and 1 bits
+    for s, bits, ratio in rows[3:5]:
+        assert O.bits(int(s)) == int(bits) and 32 // O.bits(int(s)) == int(ratio)
+    assert O.bits(O.table_len(O.SIGNSGD, 2)) == 1 and O.table_len(O.SIGNSGD, 2) == 2
     n = 512 * 1000
     cfg = O.Config(O.ORQ, 5, 512, 1, 1, 0.0, 0, n)
     nbytes, coff, loff = O.message_layout(cfg)
@@ -583,10 +587,9 @@ def test_entropy_groups_near_log2(levels):
     g, B = O.entropy_groups(levels)
     assert levels ** g <= 2 ** B < 2 * levels ** g
     assert abs(B / g - math.log2(levels)) / math.log2(levels) < 0.01
-    if levels == 3:
-        assert abs(32 * g / B - 20.2) / 20.2 < 0.01
-    if levels == 9:
-        assert abs(32 * g / B - 10.1) / 10.1 < 0.01
+    printed = {int(r[0]): float(r[2]) for r in _rows("compression_ratios.txt")[:2]}  # 3 -> 20.2, 9 -> 10.1
+    if levels in printed:
+        assert abs(32 * g / B - printed[levels]) / printed[levels] < 0.01
     assert O.entropy_groups(4) is None and O.entropy_groups(2) is None and O.entropy_groups(16) is None
 
 
