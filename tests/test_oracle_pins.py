@@ -496,7 +496,7 @@ def test_message_sizes_and_compression():
     # the glossary's TernGrad (16x) and SignSGD (32x) figures are the codes alone: 2 and 1 bits
     for s, bits, ratio in rows[3:5]:
         assert O.bits(int(s)) == int(bits) and 32 // O.bits(int(s)) == int(ratio)
-    assert O.bits(O.table_len(O.SIGNSGD, 2)) == 1 and O.table_len(O.SIGNSGD, 2) == 2
+    assert O.table_len(O.SIGNSGD, 2) == 2 and O.table_len(O.QSGD_NEAREST, 3) == 1
     n = 512 * 1000
     cfg = O.Config(O.ORQ, 5, 512, 1, 1, 0.0, 0, n)
     nbytes, coff, loff = O.message_layout(cfg)
