@@ -39,6 +39,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "gradient elems/s (encode+pack+decode+sum), ORQ-5 d=512; % of HBM peak"
+
+
+def metric_name(args):
+    """The headline metric's name for the default configuration (ORQ-5, d = 512); the same
+    metric for another scheme, level count or bucket size names that configuration."""
+    if (args.scheme, args.levels, args.bucket) == ("orq", 5, 512):
+        return METRIC
+    return "gradient elems/s (encode+pack+decode+sum), %s-%d d=%d; %% of HBM peak" % (
+        args.scheme, args.levels, args.bucket)
 UNIT = "elem/s"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -276,7 +285,7 @@ def run_reference(args):
     value = wl.workers * nbk * args.bucket * args.steps / total
     sample = "first %d buckets (d=%d) of each of the %d workers per step" % (nbk, args.bucket, wl.workers)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric_name(args), "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(args, wl),
@@ -395,7 +404,7 @@ def run_gq(args):
     plan.close()
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": metric_name(args), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(args, wl),
             "hbm_gbs_achieved": round(bpe * W * n * world / (ms_per_step / 1000.0) / 1e9 / world, 1),
