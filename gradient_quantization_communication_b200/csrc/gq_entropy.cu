@@ -20,6 +20,7 @@
 //      tables are copied unchanged.
 // Memory-bound by design: every byte of both messages is read or written once.
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 
 #include <nvtx3/nvToolsExt.h>
@@ -253,12 +254,12 @@ cudaError_t launch(EParams p, int d, cudaStream_t stream)
     }
     // the whole unified L1 as shared memory: eight CTAs of ~23 KB per SM (the kernel reads
     // global memory only through the asynchronous copies and the level tables)
-    static bool carveout_set = false;  // a repeated set is harmless, so no lock
-    if (!carveout_set) {
+    static std::atomic<bool> carveout_set{false};  // a repeated set is harmless, so no lock
+    if (!carveout_set.load(std::memory_order_relaxed)) {
         const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                                    (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
-        carveout_set = true;
+        carveout_set.store(true, std::memory_order_relaxed);
     }
     // grid-stride over tiles: at most as many CTAs as fit on the device at full occupancy
     // (2048 threads per SM); with less shared memory per SM some wait for a free slot
