@@ -50,6 +50,7 @@ def metric_name(args):
         args.scheme, args.levels, args.bucket)
 UNIT = "elem/s"
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e specification, shown beside the measured-peak fraction
 
 
 def parse_args():
@@ -409,6 +410,8 @@ def run_gq(args):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(args, wl),
             "hbm_gbs_achieved": round(bpe * W * n * world / (ms_per_step / 1000.0) / 1e9 / world, 1),
             "pct_hbm_peak": round(100.0 * bpe * W * n / (ms_per_step / 1000.0) / 1e9 / peak, 2),
+            "pct_hbm_spec": round(100.0 * bpe * W * n / (ms_per_step / 1000.0) / 1e9 / SPEC_HBM_GBS, 2),
+            "elem_per_s_per_worker": value / (W * world),
             "bytes_per_worker_elem": bpe,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
@@ -510,8 +513,12 @@ def run_cpu_baseline(args, wl, g):
     nbk = max(probe, min(nbk, wl.n // d, (2 << 30) // (4 * d * wl.workers)))
     gs_host = [x[:nbk * d].cpu().numpy() for x in g]
     rate, dt = oracle_sample_rate(wl, args, gs_host, nbk, threads)
+    # the same oracle on one thread, over the probe's buckets
+    rate1, dt1 = oracle_sample_rate(wl, args, gs_probe, probe, 1)
     return {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "seconds": round(dt, 2),
-            "sample": "first %d buckets (d=%d) of each of the %d workers, one step" % (nbk, d, wl.workers)}
+            "sample": "first %d buckets (d=%d) of each of the %d workers, one step" % (nbk, d, wl.workers),
+            "single_thread": {"value": rate1, "seconds": round(dt1, 2),
+                              "sample": "first %d buckets of each worker" % probe}}
 
 
 def run_unfused(args):
