@@ -387,11 +387,16 @@ def run_gq(args):
     achieved = bpe * W * n / (per_launch_ms / 1000.0) / 1e9 if d <= 512 else None
     kernel_key = "fused_%s%d_d%d_w%d" % (args.scheme, args.levels, d, W)
     traffic = traffic_record(kernel_key)
+    # the stored figure is per launch of the captured configuration; it stands for this run only
+    # when the workload, error feedback, message writes and clip match, scaled by the elements
+    if traffic and (traffic.get("workload"), traffic.get("error_feedback"), traffic.get("messages_written"),
+                    traffic.get("clip")) != (args.workload, bool(ef), bool(write_msgs), float(args.clip)):
+        traffic = None
     roofline = None
     if achieved is not None:
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                    "traffic": traffic["bytes_per_launch"] if traffic else None,
+                    "traffic": traffic["bytes_per_launch"] * n / traffic["elements"] if traffic else None,
                     "algorithmic_bytes_per_launch": bpe * W * n, "kernel": kernel_key}
 
     e2e = None
