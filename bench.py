@@ -311,6 +311,41 @@ def workload_config(args, wl):
 # ---------------------------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------------------------
+def fused_roofline(args, d, W, n, ef, write_msgs, bpe, achieved, peak, peak_kind):
+    """The roofline object of the fused kernel's line (None above d = 512, where the step is two
+    kernels).  The stored DRAM traffic is per launch of the captured configuration: it stands for
+    this run only when the workload, error feedback, message writes and clip match, scaled by the
+    elements processed."""
+    if achieved is None:
+        return None
+    kernel_key = "fused_%s%d_d%d_w%d" % (args.scheme, args.levels, d, W)
+    traffic = traffic_record(kernel_key)
+    if traffic and (traffic.get("workload"), traffic.get("error_feedback"), traffic.get("messages_written"),
+                    traffic.get("clip")) != (args.workload, bool(ef), bool(write_msgs), float(args.clip)):
+        traffic = None
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+            "traffic": traffic["bytes_per_launch"] * n / traffic["elements"] if traffic else None,
+            "algorithmic_bytes_per_launch": bpe * W * n, "kernel": kernel_key}
+
+
+def default_line(args, wl, value, world, W, n, ms_per_step, bpe, peak, roofline, cpu, e2e, gpu_launches, clocks):
+    """The default run's JSON line (rank 0)."""
+    gbs = bpe * W * n / (ms_per_step / 1000.0) / 1e9  # one rank's bytes over the step time
+    return {
+        "metric": metric_name(args), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(args, wl),
+        "hbm_gbs_achieved": round(gbs, 1),
+        "pct_hbm_peak": round(100.0 * gbs / peak, 2),
+        "pct_hbm_spec": round(100.0 * gbs / SPEC_HBM_GBS, 2),
+        "elem_per_s_per_worker": value / (W * world),
+        "bytes_per_worker_elem": bpe,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": gpu_launches, "clocks": clocks,
+    }
+
+
 def run_gq(args):
     import torch
     import torch.distributed as dist
@@ -385,19 +420,7 @@ def run_gq(args):
     bpe = bytes_per_worker_elem(sid, args.levels, d, W, ef, write_msgs)
     peak, peak_kind = measured_hbm_peak()
     achieved = bpe * W * n / (per_launch_ms / 1000.0) / 1e9 if d <= 512 else None
-    kernel_key = "fused_%s%d_d%d_w%d" % (args.scheme, args.levels, d, W)
-    traffic = traffic_record(kernel_key)
-    # the stored figure is per launch of the captured configuration; it stands for this run only
-    # when the workload, error feedback, message writes and clip match, scaled by the elements
-    if traffic and (traffic.get("workload"), traffic.get("error_feedback"), traffic.get("messages_written"),
-                    traffic.get("clip")) != (args.workload, bool(ef), bool(write_msgs), float(args.clip)):
-        traffic = None
-    roofline = None
-    if achieved is not None:
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                    "traffic": traffic["bytes_per_launch"] * n / traffic["elements"] if traffic else None,
-                    "algorithmic_bytes_per_launch": bpe * W * n, "kernel": kernel_key}
+    roofline = fused_roofline(args, d, W, n, ef, write_msgs, bpe, achieved, peak, peak_kind)
 
     e2e = None
     if not args.no_e2e:
@@ -409,18 +432,8 @@ def run_gq(args):
 
     plan.close()
     if rank == 0:
-        line = {
-            "metric": metric_name(args), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(args, wl),
-            "hbm_gbs_achieved": round(bpe * W * n * world / (ms_per_step / 1000.0) / 1e9 / world, 1),
-            "pct_hbm_peak": round(100.0 * bpe * W * n / (ms_per_step / 1000.0) / 1e9 / peak, 2),
-            "pct_hbm_spec": round(100.0 * bpe * W * n / (ms_per_step / 1000.0) / 1e9 / SPEC_HBM_GBS, 2),
-            "elem_per_s_per_worker": value / (W * world),
-            "bytes_per_worker_elem": bpe,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
-        }
+        line = default_line(args, wl, value, world, W, n, ms_per_step, bpe, peak, roofline, cpu, e2e,
+                            launches_per_step * args.steps, clocks)
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()

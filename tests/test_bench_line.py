@@ -1,0 +1,74 @@
+"""The benchmark's JSON line and roofline object, built on the CPU from given timings (the
+GPU run feeds the same functions): every contract field, the metric's name, and the stored
+DRAM traffic applied only to its captured configuration, scaled by the element count."""
+import sys
+
+import pytest
+
+import bench
+from gradient_quantization_communication_b200 import synth
+
+
+def _args(*argv):
+    old = sys.argv
+    sys.argv = ["bench.py", *argv]
+    try:
+        return bench.parse_args()
+    finally:
+        sys.argv = old
+
+
+def test_default_line_fields():
+    args = _args()
+    wl = synth.WORKLOADS[args.workload]
+    W, n = wl.workers, wl.n
+    bpe = bench.bytes_per_worker_elem(4, 5, 512, W, True, True)
+    assert abs(bpe - 12.914) < 1e-3
+    ms = 26.0
+    peak = 6541.1
+    achieved = bpe * W * n / (ms / 1000) / 1e9
+    roof = bench.fused_roofline(args, 512, W, n, True, True, bpe, achieved, peak, "measured")
+    value = W * n / (ms / 1000)
+    line = bench.default_line(args, wl, value, 1, W, n, ms, bpe, peak, roof, None, None, 5, {})
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "roofline", "cpu_baseline", "e2e", "gpu_launches", "clocks"):
+        assert k in line, k
+    assert line["metric"] == bench.METRIC and line["config"]["workload"].startswith("blocks1b")
+    assert line["pct_hbm_peak"] == pytest.approx(100 * achieved / peak, abs=0.01)
+    assert line["pct_hbm_spec"] == pytest.approx(100 * achieved / 8000.0, abs=0.01)
+    assert line["elem_per_s_per_worker"] == pytest.approx(n / (ms / 1000))
+    r = line["roofline"]
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["frac"] == pytest.approx(achieved / peak, abs=1e-4)
+    assert r["algorithmic_bytes_per_launch"] == pytest.approx(bpe * W * n)
+    rec = bench.traffic_record("fused_orq5_d512_w8")
+    if rec is None:  # the kernel's sources changed since the capture: the line must say null
+        assert r["traffic"] is None
+    else:
+        assert r["traffic"] == pytest.approx(rec["bytes_per_launch"])
+        # DRAM traffic within 2 % of the algorithmic bytes: nothing is read twice
+        assert abs(r["traffic"] / r["algorithmic_bytes_per_launch"] - 1) < 0.02
+
+
+def test_traffic_scaled_and_matched():
+    args = _args("--elements", "5120000")
+    n, W = 5120000, 8
+    bpe = bench.bytes_per_worker_elem(4, 5, 512, W, True, True)
+    r = bench.fused_roofline(args, 512, W, n, True, True, bpe, 4000.0, 6541.1, "measured")
+    rec = bench.traffic_record("fused_orq5_d512_w8")
+    if rec is not None:
+        assert r["traffic"] == pytest.approx(rec["bytes_per_launch"] * n / 1e9)
+    # other configurations have no stored figure
+    assert bench.fused_roofline(args, 512, W, n, False, True, bpe, 4000.0, 6541.1, "measured")["traffic"] is None
+    assert bench.fused_roofline(args, 512, W, n, True, False, bpe, 4000.0, 6541.1, "measured")["traffic"] is None
+    a2 = _args("--workload", "mixture100m")
+    assert bench.fused_roofline(a2, 512, W, n, True, True, bpe, 4000.0, 6541.1, "measured")["traffic"] is None
+    a3 = _args("--scheme", "qsgd")
+    assert bench.fused_roofline(a3, 512, W, n, True, True, bpe, 4000.0, 6541.1, "measured")["traffic"] is None
+    # no roofline object above d = 512 (two kernels per step)
+    assert bench.fused_roofline(args, 2048, W, n, True, True, bpe, None, 6541.1, "measured") is None
+
+
+def test_metric_name_follows_the_configuration():
+    assert bench.metric_name(_args()) == bench.METRIC
+    assert "signsgd-2 d=512" in bench.metric_name(_args("--scheme", "signsgd", "--levels", "2"))
+    assert "orq-5 d=2048" in bench.metric_name(_args("--bucket", "2048"))
