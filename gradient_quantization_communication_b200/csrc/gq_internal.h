@@ -54,10 +54,12 @@ cudaError_t launch_decode(const KParams &p, cudaStream_t stream);
 // gq_quant_error: per-bucket binary64 error sums into part[3 * bucket + k] (one worker, nothing
 // else written), then their fixed-order reduction into out[3].  The scratch holds
 // err_scratch_doubles(nb) doubles: the nb bucket rows followed by the rows of the first pass.
+// With a status word, the reduction writes NaN to out[0..2] when any of its bits is set.
 cudaError_t launch_warp_err(const KParams &p, double *part, cudaStream_t stream);
 cudaError_t launch_cta_err(const KParams &p, double *part, cudaStream_t stream);
 int64_t err_scratch_doubles(int64_t nb);
-cudaError_t launch_err_reduce(const double *part, int64_t nb, double *tmp, double *out, cudaStream_t stream);
+cudaError_t launch_err_reduce(const double *part, int64_t nb, double *tmp, double *out, cudaStream_t stream,
+                              const unsigned int *status = nullptr);
 // One warp waiting, with the kernels' bounded wait, on a barrier that nothing completes; raises
 // kStatusTimeout in *status after limit_ns.
 cudaError_t launch_wait_selftest(unsigned int *status, unsigned long long limit_ns, cudaStream_t stream);

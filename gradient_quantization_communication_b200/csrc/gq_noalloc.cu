@@ -11,8 +11,18 @@
 //
 // The scratch is shared by every call on a device and keeps the last call's contents.  What
 // must start at zero (the status word the kernels OR into) is cleared at the start of every
-// call; the per-bucket rows are always fully written before they are read.  Two calls whose
-// work overlaps on the GPU (different streams, or different host threads) race on the array.
+// call; the per-bucket rows are fully written before they are read unless a kernel stops
+// early (a bounded wait that gave up), and then the status word is set and the reduction
+// writes NaN to all three outputs instead of summing rows left by an earlier call.  Two calls
+// whose work overlaps on the GPU (different streams, or different host threads) race on the
+// array.
+//
+// In host code the array's name is a host-side stand-in, never a device address: the address
+// is looked up with cudaGetSymbolAddress with the device current.  The lookup is cached per
+// device together with the identity of the context it was made in (cuCtxGetId, reached through
+// cudaGetDriverEntryPoint, so the library needs no link to the driver library); a call made in
+// another context of that device (after cudaDeviceReset, say) looks the address up again.
+#include <cuda.h>
 #include <cstring>
 #include <mutex>
 
@@ -29,21 +39,57 @@ constexpr size_t kScratchBytes = kStatusBytes + sizeof(double) * 3 * (kMaxBucket
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-unsigned char *g_scratch_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+struct ScratchEntry {
+    unsigned long long ctx_id;  // context the address belongs to (0: none looked up yet)
+    unsigned char *ptr;         // device address of g_noalloc_scratch in that context
+};
+ScratchEntry g_scratch[kMaxDevices];
 std::mutex g_setup_mutex;
 
-// Device address of the scratch array on the current device (looked up once per device: in
-// host code the array's name is only a host-side stand-in, never a device address).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+// Identity of the calling thread's current context (unique for the life of the process).
+gq_status_t current_context_id(unsigned long long *id)
+{
+    if (!g_ctx_get_current || !g_ctx_get_id) {
+        void *f1 = nullptr, *f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess || !f1)
+            return GQ_ERR_CUDA;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess || !f2)
+            return GQ_ERR_CUDA;
+        g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+        g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+    CUcontext ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || !ctx) return GQ_ERR_CUDA;
+    return g_ctx_get_id(ctx, id) == CUDA_SUCCESS ? GQ_OK : GQ_ERR_CUDA;
+}
+
+// Device address of the scratch array on the current device.  In host code the array's name is
+// only a host-side stand-in, never a device address, so it is looked up with
+// cudaGetSymbolAddress, once per device and context: the first call on a device (and the first
+// after that device's context was replaced) does the lookup and must come before any stream
+// capture; later calls reuse it.
 gq_status_t scratch_address(int dev, unsigned char **out)
 {
     if (dev < 0 || dev >= kMaxDevices) return GQ_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
+    unsigned long long id = 0;
+    const gq_status_t st = current_context_id(&id);
+    if (st != GQ_OK) return st;
+    if (g_scratch[dev].ctx_id != id || !g_scratch[dev].ptr) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQ_ERR_CUDA;
-        g_scratch_ptr[dev] = static_cast<unsigned char *>(p);
+        g_scratch[dev].ptr = static_cast<unsigned char *>(p);
+        g_scratch[dev].ctx_id = id;
     }
-    *out = g_scratch_ptr[dev];
+    *out = g_scratch[dev].ptr;
     return GQ_OK;
 }
 
@@ -55,10 +101,11 @@ extern "C" GQ_API gq_status_t gq_quant_error_noalloc(const gq_config_t *cfg, uin
                                                      const float *grad, const float *residual, double *out,
                                                      void *stream)
 {
-    const gq_status_t st = gq_config_check(cfg);
-    if (st != GQ_OK) return st;
-    if (!out) return GQ_ERR_INVALID;
+    if (!cfg || !out) return GQ_ERR_INVALID;
     gq_config_t c = *cfg;
+    c.workers = 1;  // one worker's gradient: the configured worker count plays no part
+    const gq_status_t st = gq_config_check(&c);
+    if (st != GQ_OK) return st;
     if (c.scheme == GQ_TERNGRAD && c.levels == 0) c.levels = 3;
     if ((c.scheme == GQ_BINGRAD_B || c.scheme == GQ_BINGRAD_PB || c.scheme == GQ_SIGNSGD) && c.levels == 0)
         c.levels = 2;
@@ -115,5 +162,7 @@ extern "C" GQ_API gq_status_t gq_quant_error_noalloc(const gq_config_t *cfg, uin
     p.status = status;
     cudaError_t e = c.bucket <= 512 ? gq::launch_warp_err(p, part, s) : gq::launch_cta_err(p, part, s);
     if (e != cudaSuccess) return GQ_ERR_CUDA;
-    return gq::launch_err_reduce(part, nb, part + 3 * nb, out, s) == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
+    // the reduction reads the status word: a kernel that stopped early (or saw a non-finite
+    // value) makes all three outputs NaN
+    return gq::launch_err_reduce(part, nb, part + 3 * nb, out, s, status) == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
 }

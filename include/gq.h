@@ -185,16 +185,21 @@ GQ_API gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step
  * caching allocator or memory pool (which must not be re-entered), processes whose device
  * memory is reserved up front, plugins that are handed buffers but no allocator.  Such callers
  * cannot create a plan (gq_plan_create allocates), so this call takes the configuration and
- * computes exactly what gq_quant_error computes for it (cfg->workers is ignored).
+ * computes exactly what gq_quant_error computes for it, bit for bit (cfg->workers is ignored:
+ * any value is accepted, the call covers one worker's gradient).
  * Its scratch is a file-scope device array of the library, GQ_NOALLOC_SCRATCH_BYTES (about
  * 384 KB), held on every device that loads the library until the process exits.  Hence:
  *   - the input may span at most GQ_NOALLOC_MAX_BUCKETS buckets (ceil(n/d) <= 16384); larger
  *     inputs return GQ_ERR_UNSUPPORTED before anything is enqueued;
  *   - every call on a device shares that scratch and leaves its contents behind; calls whose
  *     work overlaps on the GPU (different streams or host threads) race;
- *   - non-finite input is not reported (there is no plan status word to read it from);
- *   - the first call on each device looks up the scratch address (cudaGetSymbolAddress);
- *     make that first call before any stream capture.
+ *   - there is no plan status word to query: when a kernel of the call sees a non-finite value,
+ *     or a bounded wait of its kernels gives up (the kernel then stops early), all three
+ *     outputs are NaN;
+ *   - the first call on each device looks up the scratch's device address
+ *     (cudaGetSymbolAddress) and caches it with the identity of the device's current context;
+ *     make that first call, and the first call after the context was replaced (for instance by
+ *     cudaDeviceReset), before any stream capture.
  * Allocates nothing, on the device or on the host.
  */
 #define GQ_NOALLOC_MAX_BUCKETS 16384

@@ -3,9 +3,9 @@
 It serves callers that cannot call cudaMalloc (code inside a caching allocator or memory pool,
 processes with device memory reserved up front, plugins given buffers but no allocator): it
 takes a configuration instead of a plan and keeps its scratch in a static device array of the
-library.  Its results must equal those of gq_quant_error, call after call, even though every
-call reuses the same scratch.  This file is collected last so that a failure here cannot stop a
-run before the other tests.
+library.  Its results must equal those of gq_quant_error bit for bit, call after call, even
+though every call reuses the same scratch.  This file is collected last so that a failure here
+cannot stop a run before the other tests.
 """
 import numpy as np
 import pytest
@@ -38,7 +38,40 @@ def test_noalloc_matches_planned_call_twice(scheme, levels, d):
         G.gq_quant_error_noalloc(cfg, call, call + 5, g, r, out_free)
         torch.cuda.synchronize()
         a, b = out_plan.cpu().numpy(), out_free.cpu().numpy()
-        assert np.all(np.abs(a - b) <= 1e-12 * np.abs(a)), (call, a, b)
+        # same kernels, same fixed reduction order: the same bits
+        assert np.array_equal(a.view(np.uint64), b.view(np.uint64)), (call, a, b)
+
+
+@pytest.mark.parametrize("workers", [0, 1, 100])
+def test_noalloc_ignores_the_worker_count(workers):
+    d, n = 512, 9 * 512 + 3
+    g, r = _inputs(n, seed=7)
+    ref = torch.zeros(3, dtype=torch.float64, device="cuda")
+    out = torch.zeros(3, dtype=torch.float64, device="cuda")
+    G.gq_quant_error_noalloc(G.gq_config("orq", 5, d, 1, True, 0.0, 3, n), 2, 1, g, r, ref)
+    G.gq_quant_error_noalloc(G.gq_config("orq", 5, d, workers, True, 0.0, 3, n), 2, 1, g, r, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(ref.cpu().numpy().view(np.uint64), out.cpu().numpy().view(np.uint64))
+
+
+def test_noalloc_reports_a_raised_status_as_nan_then_recovers():
+    """A status bit raised by the call's kernels (here: a non-finite input) turns all three
+    outputs into NaN; the next call clears the word and is exact again."""
+    d, n = 256, 20 * 256
+    cfg = G.gq_config("qsgd", 5, d, 1, False, 0.0, 11, n)
+    g, _ = _inputs(n, seed=5)
+    bad = g.clone()
+    bad[3 * d + 17] = float("nan")
+    out = torch.zeros(3, dtype=torch.float64, device="cuda")
+    G.gq_quant_error_noalloc(cfg, 0, 0, bad, None, out)
+    torch.cuda.synchronize()
+    assert np.all(np.isnan(out.cpu().numpy()))
+    ref = torch.zeros(3, dtype=torch.float64, device="cuda")
+    with G.Plan(cfg) as plan:
+        G.gq_quant_error(plan.handle, 0, 0, g, None, ref)
+    G.gq_quant_error_noalloc(cfg, 0, 0, g, None, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(ref.cpu().numpy().view(np.uint64), out.cpu().numpy().view(np.uint64))
 
 
 def test_noalloc_rejects_inputs_beyond_its_scratch():
