@@ -16,8 +16,10 @@
  *   - stochastic rounding against the 0.7 example of [P3] and Monte Carlo mean / variance;
  *   - ORQ's greedy against an independent naive greedy on the raw values;
  *   - BinGrad-b's split against brute force over all thresholds;
- *   - BinGrad-pb's pair against brute force over all grid pairs, and the ordering of
- *     quantization errors BinGrad-b <= BinGrad-pb stated in [P2] "Key findings";
+ *   - BinGrad-pb's pair against brute force over the admissible grid pairs, its range against
+ *     BinGrad-b's ("wider range", [P2] "Proposed method"), its per-value bias against BinGrad-b's
+ *     error, and the ordering of quantization errors BinGrad-b <= BinGrad-pb stated in [P2]
+ *     "Key findings";
  *   - QSGD/TernGrad against hand-computed closed forms;
  *   - packing against a bit-by-bit unpacker; error feedback against its telescoping sum;
  *   - base-s packing against a big-integer construction of the digit stream, the round trip,
@@ -27,8 +29,8 @@
  *   - QSGD-l2's scale against the exact norm and its unbiasedness; Elias gamma against the
  *     published codeword table, the stream against a bit string built from it, the offsets,
  *     the round trip and the expected length.
- * Parity of BinGrad-pb with the paper's own (unpublished on the pages) definition is unpinned:
- * only this reading of it is pinned.
+ * The pages state BinGrad-pb's properties (wider range, less bias, larger error than BinGrad-b)
+ * but not its formula: the reading below is pinned to those properties.
  */
 #include "gq_oracle.h"
 
@@ -554,20 +556,41 @@ static void bingrad_b_bucket(const float *u, int n, uint8_t *code, float *q, flo
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* BinGrad-pb.  [P2]: the binary variant that trades some variance for less bias by a wider   */
-/* range, with a larger quantization error than BinGrad-b.  Reading ("partially biased"):     */
-/* two levels (g_A, g_B) from the 64-point grid; values between them are rounded             */
-/* stochastically (unbiased), values outside are clamped to the nearer level (biased).  The    */
-/* pair minimises the expected squared error                                                  */
-/*   sum_{x<a} (a-x)^2 + sum_{a<=x<b} (b-x)(x-a) + sum_{x>=b} (x-b)^2                         */
-/* in fixed point with 16 fraction bits per cell (exact int128), ties to the smallest (A, B).  */
+/* BinGrad-pb.  [P2] "Proposed method": the binary variant that, unlike BinGrad-b, reduces bias */
+/* through a wider range; [P2] "Key findings": its quantization error is larger than           */
+/* BinGrad-b's.  Reading ("partially biased"): two levels (g_A, g_B) from the 64-point grid,    */
+/* at least as far apart as BinGrad-b's levels (a_b, b_b) on the same bucket: g_A <= a_b and    */
+/* g_B >= b_b (A at most the largest grid index whose point is <= a_b, 0 when there is none; B  */
+/* at least the smallest whose point is >= b_b, 63 when there is none).  Values between the     */
+/* levels are rounded stochastically (unbiased), values outside are clamped to the nearer       */
+/* level (biased).  Among the admissible pairs the one that minimises the expected squared      */
+/* error                                                                                        */
+/*   sum_{x<a} (a-x)^2 + sum_{a<=x<b} (b-x)(x-a) + sum_{x>=b} (x-b)^2                           */
+/* is taken, in fixed point with 16 fraction bits per cell (exact int128), ties to the smallest */
+/* (A, B).  The range condition makes the span at least BinGrad-b's and every clamped value's   */
+/* bias at most its BinGrad-b error; the expected error is never below BinGrad-b's, since       */
+/* (b-x)(x-a) >= min(x-a, b-x)^2 for every x between the levels.                                */
 /* ------------------------------------------------------------------------------------------ */
-static void pb_select_pos(const int32_t *pos, int n, int *A_out, int *B_out)
+static void pb_limits(const or_gridinfo *gi, const float *u, int n, int *Amax, int *Bmin)
+{
+    float a, b, thr;
+    int split;
+    or_bingrad_b_fit(u, n, &a, &b, &thr, &split);
+    int am = 0, bm = OR_GRIDPTS - 1;
+    for (int j = 0; j < OR_GRIDPTS; ++j)
+        if (gi->grid[j] <= a) am = j;
+    for (int j = OR_GRIDPTS - 1; j >= 0; --j)
+        if (gi->grid[j] >= b) bm = j;
+    *Amax = am;
+    *Bmin = bm;
+}
+
+static void pb_select_pos(const int32_t *pos, int n, int Amax, int Bmin, int *A_out, int *B_out)
 {
     int bestA = -1, bestB = -1;
     __int128 best_e = 0;
-    for (int A = 0; A < OR_GRIDPTS - 1; ++A) {
-        for (int B = A + 1; B < OR_GRIDPTS; ++B) {
+    for (int A = 0; A <= Amax && A < OR_GRIDPTS - 1; ++A) {
+        for (int B = (Bmin > A + 1 ? Bmin : A + 1); B < OR_GRIDPTS; ++B) {
             int64_t a = (int64_t)A << OR_PB_FBITS, b = (int64_t)B << OR_PB_FBITS;
             __int128 e = 0;
             for (int i = 0; i < n; ++i) {
@@ -599,7 +622,9 @@ void or_bingrad_pb_fit(const float *u, int n, int *A, int *B, float *ga, float *
     }
     int32_t *pos = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
     for (int i = 0; i < n; ++i) pos[i] = grid_pos(&gi, u[i], OR_PB_FBITS);
-    pb_select_pos(pos, n, A, B);
+    int Amax, Bmin;
+    pb_limits(&gi, u, n, &Amax, &Bmin);
+    pb_select_pos(pos, n, Amax, Bmin, A, B);
     *ga = gi.grid[*A];
     *gb = gi.grid[*B];
     free(pos);
@@ -626,8 +651,9 @@ static void bingrad_pb_bucket(const or_config *cfg, int worker, uint64_t step, i
     }
     int32_t *pos = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
     for (int i = 0; i < n; ++i) pos[i] = grid_pos(&gi, u[i], OR_PB_FBITS);
-    int A, B;
-    pb_select_pos(pos, n, &A, &B);
+    int A, B, Amax, Bmin;
+    pb_limits(&gi, u, n, &Amax, &Bmin);
+    pb_select_pos(pos, n, Amax, Bmin, &A, &B);
     float a = gi.grid[A], b = gi.grid[B];
     table[0] = a;
     table[1] = b;

@@ -43,6 +43,8 @@ MUTATIONS = [
      "if ((code[e] >> j) & 1) words[k / 32] |= 1u << (31 - k % 32);"),
     ("bingrad_b_tie_rule", "if (best < 0 || j > best_j) {", "if (best < 0 || j >= best_j) {"),
     ("bingrad_pb_tie_rule", "if (bestA < 0 || e < best_e) {", "if (bestA < 0 || e <= best_e) {"),
+    ("bingrad_pb_lower_limit", "*Amax = am;", "*Amax = OR_GRIDPTS - 2;"),
+    ("bingrad_pb_upper_limit", "if (gi->grid[j] >= b) bm = j;", "if (gi->grid[j] >= a) bm = j;"),
     ("quant_error_term", "e += P * dh * dh + (1.0 - P) * dl * dl;", "e += P * dh * dh + P * dl * dl;"),
     ("entropy_digit_order", "for (int k = g - 1; k >= 0; --k) {", "for (int k = 0; k < g; ++k) {"),
     ("entropy_group_bits", "case 9: *g = 5; *B = 16; return 1;", "case 9: *g = 5; *B = 17; return 1;"),

@@ -295,7 +295,8 @@ def test_bingrad_b_codes_deterministic():
 
 
 # ------------------------------------------------------------------------------------------
-# BinGrad-pb: brute force over every grid pair, and the b <= pb ordering of [P2]
+# BinGrad-pb: the properties [P2] states (a wider range and less bias than BinGrad-b, a larger
+# error), and brute force over the admissible grid pairs
 # ------------------------------------------------------------------------------------------
 def _pb_error(x, a, b):
     x = np.asarray(x, dtype=np.float64)
@@ -303,19 +304,107 @@ def _pb_error(x, a, b):
     return float(e.sum())
 
 
+def _grid32(u):
+    """The 64-point grid in binary32: min + j * ((max - min) / 63), the last point max."""
+    mn, mx = np.float32(u.min()), np.float32(u.max())
+    step = np.float32(mx - mn) / np.float32(63.0)
+    g = np.array([np.float32(mn + np.float32(j) * step) for j in range(64)], dtype=np.float32)
+    g[63] = mx
+    return g
+
+
+def _pb_buckets(seed, count, n=512):
+    rng = np.random.default_rng(seed)
+    draws = [rng.standard_normal, lambda k: rng.laplace(0, 1, k), lambda k: rng.standard_t(3, k),
+             lambda k: rng.uniform(-1, 1, k)]
+    return [(draws[t % 4](n) * 1e-3).astype(np.float32) for t in range(count)]
+
+
 def test_bingrad_pb_brute_force():
+    """The pair minimises the expected squared error over every grid pair at least as wide as
+    BinGrad-b's levels (brute force on the values in binary64)."""
     rng = np.random.default_rng(13)
-    for t in range(8):
-        n = int(rng.integers(8, 40))
-        u = (rng.standard_t(3, n) * 1e-3).astype(np.float32)
+    for t in range(24):
+        n = int(rng.integers(8, 160))
+        u = (rng.standard_t(3, n) if t % 2 else rng.laplace(0, 1, n)) * 1e-3
+        u = u.astype(np.float32)
         A, B, ga, gb = O.bingrad_pb_fit(u)
+        a_b, b_b, _, _ = O.bingrad_b_fit(u)
+        grid = _grid32(u)
         x = u.astype(np.float64)
-        mn, mx = x.min(), x.max()
-        grid = mn + np.arange(64) * (mx - mn) / 63.0
-        grid[63] = mx
-        best = min(_pb_error(x, grid[i], grid[j]) for i in range(63) for j in range(i + 1, 64))
-        assert 0 <= A < B <= 63
-        assert _pb_error(x, grid[A], grid[B]) <= best * (1 + 1e-4) + 1e-30
+        ok = [(i, j) for i in range(63) for j in range(i + 1, 64)
+              if (grid[i] <= a_b or i == 0) and (grid[j] >= b_b or j == 63)]
+        best = min(_pb_error(x, float(grid[i]), float(grid[j])) for i, j in ok)
+        assert (A, B) in ok
+        assert (ga, gb) == (grid[A], grid[B])
+        assert _pb_error(x, ga, gb) <= best * (1 + 1e-4) + 1e-30
+
+
+# Integer buckets on which the best admissible pair lies inside the admissible corner (found
+# by a search over random integer buckets); the expected pairs are computed below.
+_PB_INNER = [[0, 2, 3, 30, 52, 53, 63], [0, 1, 29, 63], [0, 31, 50, 63], [0, 7, 14, 35, 61, 61, 63],
+             [0, 34, 62, 63], [0, 33, 57, 63], [0, 3, 30, 48, 63], [0, 1, 31, 57, 62, 63], [0, 11, 32, 63],
+             [0, 1, 29, 62, 62, 63], [0, 11, 13, 33, 56, 62, 63], [0, 2, 29, 59, 61, 63], [0, 12, 12, 33, 59, 63],
+             [0, 2, 9, 30, 57, 59, 63], [0, 3, 30, 56, 58, 63], [0, 11, 33, 57, 61, 63], [0, 1, 5, 32, 62, 63],
+             [0, 7, 31, 63], [0, 2, 4, 33, 60, 63], [0, 1, 33, 60, 63], [0, 1, 1, 5, 28, 53, 63],
+             [0, 33, 61, 63], [0, 10, 33, 60, 63], [0, 1, 3, 33, 62, 63], [0, 15, 33, 61, 63],
+             [0, 2, 30, 61, 63], [0, 5, 32, 58, 63], [0, 1, 1, 29, 63], [0, 32, 59, 63], [0, 15, 33, 63],
+             [0, 8, 8, 34, 62, 63], [0, 4, 6, 30, 51, 53, 57, 59, 63], [0, 6, 33, 62, 63], [0, 4, 29, 63],
+             [0, 4, 30, 60, 63], [0, 31, 52, 63], [0, 3, 32, 59, 63], [0, 11, 13, 32, 63]]
+
+
+def test_bingrad_pb_exact_on_the_integer_grid():
+    """Small buckets of integers with minimum 0 and maximum 63: the grid is 0..63 exactly and the
+    positions are exact, so the pair must equal an exact-integer brute force over the
+    admissible pairs (ties to the smallest (A, B))."""
+    from fractions import Fraction
+    rng = np.random.default_rng(16)
+    cases = _PB_INNER + [[0, 63] + rng.integers(1, 63, int(rng.integers(1, 7))).tolist() for _ in range(150)]
+    inner = 0
+    for x in cases:
+        xs = sorted(x)
+        n = len(xs)
+        best = None
+        for k in range(1, n):  # BinGrad-b's split, exactly
+            if xs[k - 1] < xs[k]:
+                J = Fraction(sum(xs[:k])) ** 2 / k + Fraction(sum(xs[k:])) ** 2 / (n - k)
+                if best is None or J > best[0]:
+                    best = (J, k)
+        k = best[1]
+        a_b, b_b = Fraction(sum(xs[:k]), k), Fraction(sum(xs[k:]), n - k)
+        amax = max(j for j in range(64) if j <= a_b)
+        bmin = min(j for j in range(64) if j >= b_b)
+
+        def err(A, B):
+            return sum((A - v) ** 2 if v < A else (v - B) ** 2 if v >= B else (B - v) * (v - A) for v in x)
+        pair = min(((err(A, B), A, B) for A in range(amax + 1) for B in range(max(A + 1, bmin), 64)))
+        inner += (pair[1], pair[2]) != (amax, bmin)
+        A, B, ga, gb = O.bingrad_pb_fit(np.array(x, dtype=np.float32))
+        assert (A, B) == (pair[1], pair[2]), (x, (A, B), pair)
+        assert (ga, gb) == (float(A), float(B))
+    assert inner >= len(_PB_INNER)
+
+
+def test_bingrad_pb_wider_range_than_b():
+    """[P2] Proposed method: BinGrad-pb reduces bias with a wider range than BinGrad-b."""
+    for u in _pb_buckets(31, 200):
+        a, b, _, _ = O.bingrad_b_fit(u)
+        _, _, ga, gb = O.bingrad_pb_fit(u)
+        assert ga <= a and gb >= b
+        assert gb - ga >= b - a
+
+
+def test_bingrad_pb_less_bias_than_b():
+    """[P2] Proposed method: BinGrad-pb reduces bias.  Its expected value differs from a value only
+    where the value is clamped, and by less than BinGrad-b's deterministic error there."""
+    for u in _pb_buckets(32, 120):
+        a, b, thr, _ = O.bingrad_b_fit(u)
+        _, _, ga, gb = O.bingrad_pb_fit(u)
+        x = u.astype(np.float64)
+        bias_pb = np.where(x < ga, ga - x, np.where(x > gb, x - gb, 0.0))
+        err_b = np.abs(np.where(x >= thr, b, a) - x)
+        assert np.all(bias_pb <= err_b * (1 + 1e-6) + 1e-12)
+        assert bias_pb.sum() < err_b.sum()
 
 
 def test_bingrad_b_error_below_pb():
@@ -514,10 +603,12 @@ def test_tie_rules():
     # the smaller split wins.
     a, b, thr, split = O.bingrad_b_fit(np.array([1.0, -1.0, 0.0], dtype=np.float32))
     assert (split, thr, a, b) == (1, 0.0, -1.0, 0.5)
-    # BinGrad-pb on the integer grid 0..63 (min 0, max 63): the pairs (9, 51) and (9, 52) both
-    # give the least expected squared error (663, found by exhaustive search); the smaller wins.
-    A, B, ga, gb = O.bingrad_pb_fit(np.array([0.0, 8.0, 32.0, 63.0], dtype=np.float32))
-    assert (A, B, ga, gb) == (9, 51, 9.0, 51.0)
+    # BinGrad-pb on the integer grid 0..63 (min 0, max 63) for {0, 1, 30, 63}: BinGrad-b's levels
+    # are 1/2 and 93/2, so A <= 0 and B >= 47; the pairs (0, 47) and (0, 48) both give the least
+    # expected squared error, 812 (0 + 46 + 17 * 30 + 16^2 = 0 + 47 + 18 * 30 + 15^2); the
+    # smaller wins.
+    A, B, ga, gb = O.bingrad_pb_fit(np.array([0.0, 1.0, 30.0, 63.0], dtype=np.float32))
+    assert (A, B, ga, gb) == (0, 47, 0.0, 47.0)
 
 
 # ------------------------------------------------------------------------------------------
