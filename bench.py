@@ -374,12 +374,12 @@ def run_gq(args):
     for w in range(W):
         synth.gradient(args.workload, w, 0, n=n, out=g[w])
     r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)] if ef else None
-    write_msgs = not args.no_msgs or d > 512
+    write_msgs = not args.no_msgs
     msgs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)] if write_msgs else None
     avg = torch.empty(n, dtype=torch.float32, device=dev)
     # d <= 512: the fused kernel over the full buckets, plus one launch for a ragged last bucket;
-    # d > 512: one encode per worker, then the decode
-    launches_per_step = ((1 if n >= d else 0) + (1 if n % d else 0)) if d <= 512 else W + 1
+    # d > 512: one fused launch of the large-bucket kernel
+    launches_per_step = ((1 if n >= d else 0) + (1 if n % d else 0)) if d <= 512 else 1
 
     def step(t):
         G.gq_fused_step(plan.handle, t, g, r, msgs, avg, stream)
@@ -872,8 +872,6 @@ def run_sweep(args):
                     uu += o[1]
                 sid = G.SCHEMES[scheme]
                 bpe = bytes_per_worker_elem(sid, levels, d, W, False, True)
-                if d > 512:  # encode per worker + decode over the messages
-                    bpe += ((levels - 1).bit_length() / 8.0 + 4.0 * (levels if sid == 4 else 1) / d)
                 rows.append({"scheme": "%s-%d" % (scheme, levels), "bucket": d, "ms_per_step": round(ms, 4),
                              "elem_per_s": W * n / (ms / 1000.0), "bytes_per_worker_elem": round(bpe, 4),
                              "pct_hbm_peak": round(100.0 * bpe * W * n / (ms / 1000.0) / 1e9 / peak, 2),

@@ -251,37 +251,20 @@ gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *gra
         if (ef && (!residuals[w] || !aligned16(residuals[w]))) return GQ_ERR_INVALID;
         if (msgs && (!msgs[w] || !aligned16(msgs[w]))) return GQ_ERR_INVALID;
     }
-    if (!msgs && plan->cfg.bucket > 512) return GQ_ERR_INVALID;
     gq_status_t st = check_device(*plan);
     if (st != GQ_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     gq::KParams p = base_params(*plan, step);
-    if (plan->cfg.bucket <= 512) {
-        p.W = W;
-        p.inv_w = 1.0f / (float)W;
-        for (int w = 0; w < W; ++w) {
-            p.g[w] = grads[w];
-            p.r[w] = ef ? residuals[w] : nullptr;
-            p.msg[w] = msgs ? static_cast<unsigned char *>(msgs[w]) : nullptr;
-        }
-        p.avg = avg;
-        return from_cuda(gq::launch_warp_encode(p, true, s));
-    }
-    // large buckets: quantize each worker into its message, then decode + aggregate
-    for (int w = 0; w < W; ++w) {
-        gq::KParams q = p;
-        q.worker0 = (uint32_t)w;
-        q.g[0] = grads[w];
-        q.r[0] = ef ? residuals[w] : nullptr;
-        q.msg[0] = static_cast<unsigned char *>(msgs[w]);
-        const cudaError_t e = gq::launch_cta_encode(q, s);
-        if (e != cudaSuccess) return GQ_ERR_CUDA;
-    }
     p.W = W;
     p.inv_w = 1.0f / (float)W;
-    for (int w = 0; w < W; ++w) p.msg[w] = static_cast<unsigned char *>(msgs[w]);
+    for (int w = 0; w < W; ++w) {
+        p.g[w] = grads[w];
+        p.r[w] = ef ? residuals[w] : nullptr;
+        p.msg[w] = msgs ? static_cast<unsigned char *>(msgs[w]) : nullptr;
+    }
     p.avg = avg;
-    return from_cuda(gq::launch_decode(p, s));
+    if (plan->cfg.bucket <= 512) return from_cuda(gq::launch_warp_encode(p, true, s));
+    return from_cuda(gq::launch_cta_encode(p, s));
 }
 
 gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, const float *residual,

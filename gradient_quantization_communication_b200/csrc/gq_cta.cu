@@ -1,17 +1,24 @@
-// gq_cta.cu -- quantization of large buckets (d = 1024 .. 32768): one CTA per bucket.
+// gq_cta.cu -- quantization of large buckets (d = 1024 .. 32768): one CTA per bucket index.
 //
-// The CTA (8 warps) stages the bucket's error-fed values v = g + r in shared memory (16-byte
-// coalesced loads), reduces the bucket statistics across its warps, fits the levels and then
-// rounds, packs and writes the residual chunk by chunk (warp k takes the 128-element chunks
-// k, k+8, ...).  Fits:
+// The CTA (NW warps: 8, or 16 for d >= 16384) walks the items (bucket, worker) of its bucket
+// index in worker order; W = 1 for gq_encode and gq_quant_error.  For each item it stages
+// v = g + r in shared memory (16-byte coalesced evict-first loads; the next item's g and r are
+// brought into L2 by bulk prefetches while this one is processed), reduces the bucket
+// statistics across its warps, fits the levels and then rounds, packs and writes the residual
+// chunk by chunk (warp k takes the 128-element chunks k, k + NW, ...).  In the fused step the
+// dequantized values are added, in worker order, to a running sum kept on chip: in shared
+// memory when it fits beside the staged bucket (d <= 8192), else in the average's own slice,
+// which stays in L2 while the CTA works on the bucket; the last worker writes the average.
+// Fits:
 //   QSGD / TernGrad : block max of |u|
 //   ORQ             : per warp, the packed 8-column histogram of the register path (one shared
 //                     atomic per value), reduced every 512 values into the warp's cell totals;
 //                     warp 0 sums the warps' totals and runs the greedy
-//   BinGrad-pb      : block moments per cell (shared atomics), all 2016 pairs searched by
-//                     the 256 threads
 //   BinGrad-b       : block bitonic sort of u in place, exact int64 block scan, argmax of
 //                     J(k); the final pass re-reads g and r because the sort overwrote v
+//   BinGrad-pb      : BinGrad-b's levels first (as above: the final pass re-reads g and r),
+//                     which bound the pair from inside; block moments per cell (shared
+//                     atomics), the admissible pairs among all 2016 searched by the threads
 // The per-element rules and the chunk step are those of the register path (gq_round.cuh), so
 // both paths produce identical codes.
 #include "gq_round.cuh"
@@ -19,15 +26,13 @@
 namespace gq {
 namespace {
 
-constexpr int kCtaWarps = 8;
-constexpr int kCtaThreads = kCtaWarps * 32;
-
+template <int NW>
 struct alignas(16) CtaShared {
-    float redf[3][kCtaWarps];
-    long long redl[3][kCtaWarps];
-    double redd[kCtaWarps];
-    double rede[3][kCtaWarps];
-    int redi[kCtaWarps];
+    float redf[3][NW];
+    long long redl[3][NW];
+    double redd[NW];
+    double rede[3][NW];
+    int redi[NW];
     unsigned long long cs1[64], cs2[64];  // block histogram: sum of positions, of squares
     unsigned int ccnt[64];                // block histogram: count
     long long P1[64];
@@ -42,42 +47,46 @@ struct alignas(16) CtaShared {
 };
 
 // --- block reductions (every thread receives the result) -------------------------------------
-__device__ float block_max(float x, CtaShared &sh, int slot)
+template <int NW>
+__device__ float block_max(float x, CtaShared<NW> &sh, int slot)
 {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     x = warp_max(x);
     if (lane == 0) sh.redf[slot][wid] = x;
     __syncthreads();
-    float y = sh.redf[slot][lane & (kCtaWarps - 1)];
+    float y = sh.redf[slot][lane & (NW - 1)];
     y = warp_max(y);
     __syncthreads();
     return y;
 }
-__device__ float block_min(float x, CtaShared &sh, int slot)
+template <int NW>
+__device__ float block_min(float x, CtaShared<NW> &sh, int slot)
 {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     x = warp_min(x);
     if (lane == 0) sh.redf[slot][wid] = x;
     __syncthreads();
-    float y = sh.redf[slot][lane & (kCtaWarps - 1)];
+    float y = sh.redf[slot][lane & (NW - 1)];
     y = warp_min(y);
     __syncthreads();
     return y;
 }
-__device__ long long block_sum(long long x, CtaShared &sh, int slot)
+template <int NW>
+__device__ long long block_sum(long long x, CtaShared<NW> &sh, int slot)
 {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     x = warp_sum(x);
     if (lane == 0) sh.redl[slot][wid] = x;
     __syncthreads();
-    long long y = lane < kCtaWarps ? sh.redl[slot][lane] : 0ll;
+    long long y = lane < NW ? sh.redl[slot][lane] : 0ll;
     y = warp_sum(y);
     __syncthreads();
     return y;
 }
 
 // The three staging statistics in one exchange: NaN-propagating max |v|, min v and max v.
-__device__ void block_stats(float &am, float &lo, float &hi, CtaShared &sh)
+template <int NW>
+__device__ void block_stats(float &am, float &lo, float &hi, CtaShared<NW> &sh)
 {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     am = warp_redux_max_abs(am);
@@ -89,9 +98,9 @@ __device__ void block_stats(float &am, float &lo, float &hi, CtaShared &sh)
         sh.redf[2][wid] = hi;
     }
     __syncthreads();
-    am = warp_redux_max_abs(sh.redf[0][lane & (kCtaWarps - 1)]);
-    lo = warp_redux_min(sh.redf[1][lane & (kCtaWarps - 1)]);
-    hi = warp_redux_max(sh.redf[2][lane & (kCtaWarps - 1)]);
+    am = warp_redux_max_abs(sh.redf[0][lane & (NW - 1)]);
+    lo = warp_redux_min(sh.redf[1][lane & (NW - 1)]);
+    hi = warp_redux_max(sh.redf[2][lane & (NW - 1)]);
     __syncthreads();
 }
 
@@ -138,15 +147,142 @@ __device__ __forceinline__ void reduce_warp_hist(uint32_t *wh, int lane)
     __syncwarp();
 }
 
-// ERR: the error mode of gq_quant_error; nothing is written but part[3 * bucket + k].
-template <int SCHEME, bool ERR>
-__global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KParams p, double *part)
+// BinGrad-b's levels of the staged bucket (m = max|u| > 0): sorts the clipped values in place
+// (padding +inf; the staged values are lost), exact int64 block scan of their fixed-point
+// values, argmax of J(k) ties to the smallest k.  {a, b, split value, split found}.  Also used by
+// BinGrad-pb, whose levels must be at least as far apart.
+template <int NW, class Clip>
+__device__ RoundB cta_bingrad_b_levels(float *vs, int d, int nvalid, float m, const Clip &clipped, CtaShared<NW> &sh)
 {
+    constexpr int kCtaThreads = NW * 32;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    RoundB rb{0.0f, 0.0f, 0.0f, false};
+    // sort u in place (padding = +inf)
+    for (int i = tid; i < d; i += kCtaThreads) vs[i] = i < nvalid ? clipped(vs[i]) : INFINITY;
+    __syncthreads();
+    for (int k = 2; k <= d; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < d; i += kCtaThreads) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const float a = vs[i], b = vs[ixj];
+                    const bool up = (i & k) == 0;
+                    if ((a > b) == up) {
+                        vs[i] = b;
+                        vs[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    // exact prefix sums of the fixed-point values: thread t owns positions [t*seg, (t+1)*seg)
+    const int e2 = 46 - fexpo(m);
+    const double sc = pow2d(e2);
+    const int seg = d / kCtaThreads;
+    long long run = 0;
+    for (int i = tid * seg; i < tid * seg + seg; ++i) run += (i < nvalid) ? fixed_point(vs[i], sc) : 0ll;
+    const long long incl = warp_inclusive_scan(run, lane);
+    if (lane == 31) sh.redl[0][wid] = incl;
+    __syncthreads();
+    long long wpre = 0, total = 0;
+    for (int k = 0; k < NW; ++k) {
+        const long long t = sh.redl[0][k];
+        if (k < wid) wpre += t;
+        total += t;
+    }
+    __syncthreads();
+    long long S = wpre + incl - run;  // sum of positions before tid*seg
+    double best_j = -1.0;
+    int best_i = 0x7fffffff;
+    long long best_s = 0;
+    for (int i = tid * seg; i < tid * seg + seg; ++i) {
+        if (i >= 1 && i < nvalid && vs[i - 1] < vs[i]) {
+            const double l = __ll2double_rn(S);
+            const double rr = __ll2double_rn(total - S);
+            const double J = __dadd_rn(__ddiv_rn(__dmul_rn(l, l), (double)i),
+                                       __ddiv_rn(__dmul_rn(rr, rr), (double)(nvalid - i)));
+            if (J > best_j) {
+                best_j = J;
+                best_i = i;
+                best_s = S;
+            }
+        }
+        if (i < nvalid) S += fixed_point(vs[i], sc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double oj = __shfl_xor_sync(kFull, best_j, o);
+        const int oi = __shfl_xor_sync(kFull, best_i, o);
+        const long long os = __shfl_xor_sync(kFull, best_s, o);
+        if (oj > best_j || (oj == best_j && oi < best_i)) {
+            best_j = oj;
+            best_i = oi;
+            best_s = os;
+        }
+    }
+    if (lane == 0) {
+        sh.redd[wid] = best_j;
+        sh.redi[wid] = best_i;
+        sh.redl[1][wid] = best_s;
+    }
+    __syncthreads();
+    best_j = sh.redd[lane & (NW - 1)];
+    best_i = sh.redi[lane & (NW - 1)];
+    best_s = sh.redl[1][lane & (NW - 1)];
+#pragma unroll
+    for (int o = NW / 2; o > 0; o >>= 1) {
+        const double oj = __shfl_xor_sync(kFull, best_j, o);
+        const int oi = __shfl_xor_sync(kFull, best_i, o);
+        const long long os = __shfl_xor_sync(kFull, best_s, o);
+        if (oj > best_j || (oj == best_j && oi < best_i)) {
+            best_j = oj;
+            best_i = oi;
+            best_s = os;
+        }
+    }
+    if (best_i == 0x7fffffff) {
+        const float v0 = __fadd_rn(vs[0], 0.0f);
+        rb = RoundB{v0, v0, v0, false};
+    } else {
+        const double inv_sc = pow2d(-e2);
+        const float a = __double2float_rn(__dmul_rn(__ddiv_rn(__ll2double_rn(best_s), (double)best_i), inv_sc));
+        const float b = __double2float_rn(
+            __dmul_rn(__ddiv_rn(__ll2double_rn(total - best_s), (double)(nvalid - best_i)), inv_sc));
+        rb = RoundB{a, b, vs[best_i], true};
+    }
+    __syncthreads();
+    return rb;
+}
+
+// Largest bucket whose running sum of the fused step stays in shared memory beside the staged
+// bucket; larger ones keep it in the average's slice of global memory (L2-resident).
+constexpr int kAccSmemMax = 8192;
+
+// Bulk prefetch of [p, p + bytes) into L2 (bytes a multiple of 16, p 16-byte aligned), in
+// pieces of at most 32 KB.
+__device__ __forceinline__ void prefetch_l2(const void *p, unsigned bytes)
+{
+    const char *c = static_cast<const char *>(p);
+    for (unsigned off = 0; off < bytes; off += 32768u) {
+        const unsigned len = bytes - off < 32768u ? bytes - off : 32768u;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(c + off), "r"(len) : "memory");
+    }
+}
+
+// ERR: the error mode of gq_quant_error; nothing is written but part[3 * bucket + k].
+template <int SCHEME, bool ERR, int NW>
+__global__ void __launch_bounds__(NW * 32) k_cta(const __grid_constant__ KParams p, double *part)
+{
+    constexpr int kCtaWarps = NW, kCtaThreads = NW * 32;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    __shared__ CtaShared sh;
+    __shared__ CtaShared<NW> sh;
     const int d = p.d;
-    float *vs = reinterpret_cast<float *>(smem_raw);                      // d floats
-    uint32_t *hist_all = reinterpret_cast<uint32_t *>(smem_raw + (size_t)d * 4);  // ORQ: 8 warps' histograms
+    const bool fused = !ERR && p.avg != nullptr;
+    const bool acc_smem = fused && d <= kAccSmemMax;
+    float *vs = reinterpret_cast<float *>(smem_raw);  // d floats
+    float *accs = acc_smem ? vs + d : nullptr;         // the running sum (d floats) when it fits
+    uint32_t *hist_all = reinterpret_cast<uint32_t *>(smem_raw + (size_t)d * 4 * (acc_smem ? 2 : 1));  // ORQ
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     uint32_t *wh = hist_all + wid * kWarpHistWords;
 
@@ -160,16 +296,32 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
     }
     __syncthreads();
 
-    const float *g = p.g[0];
-    float *r = p.r[0];
-    unsigned char *msg = p.msg[0];
-    const uint32_t worker = p.worker0;
     const int nchunks = d >> 7;
+    const int W = p.W;
 
     ErrAcc ea{0.0, 0.0, 0.0};
     for (int64_t beta = blockIdx.x; beta < p.nb; beta += gridDim.x) {
-        const int64_t base = beta * (int64_t)d;
-        const int nvalid = (beta == p.nb - 1) ? p.tail : d;
+      const int64_t base = beta * (int64_t)d;
+      const int nvalid = (beta == p.nb - 1) ? p.tail : d;
+      for (int w = 0; w < W; ++w) {
+        const float *g = p.g[w];
+        float *r = p.r[w];
+        unsigned char *msg = p.msg[w];
+        const uint32_t worker = p.worker0 + (uint32_t)w;
+        if (tid == 0) {
+            // the next item's g and r into L2 while this one is processed
+            const bool same = w + 1 < W;
+            const int64_t nbeta = same ? beta : beta + gridDim.x;
+            const int nw = same ? w + 1 : 0;
+            if (nbeta < p.nb) {
+                const int nv = nbeta == p.nb - 1 ? p.tail : d;
+                const unsigned bytes = (unsigned)(nv * 4) & ~15u;
+                if (bytes) {
+                    prefetch_l2(p.g[nw] + nbeta * d, bytes);
+                    if (p.r[nw]) prefetch_l2(p.r[nw] + nbeta * d, bytes);
+                }
+            }
+        }
         // ---- stage v = g + r in shared memory; NaN-propagating max |v|, min v, max v ------------
         float am = 0.0f, vlo = INFINITY, vhi = -INFINITY;
         for (int i4 = tid; i4 < (d >> 2); i4 += kCtaThreads) {
@@ -354,6 +506,21 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                     __syncthreads();
                 } else {
                     scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kPbFBits));
+                    // BinGrad-b's levels bound the pair from inside: A <= Amax, the largest grid
+                    // index whose point is <= a_b (0 if none), B >= Bmin, the smallest whose point
+                    // is >= b_b (63 if none).  The sort leaves the clipped values permuted in vs,
+                    // which the histogram below does not mind; the final pass re-reads g and r.
+                    const RoundB bl = cta_bingrad_b_levels<NW>(vs, d, nvalid, fmaxf(fabsf(mn), fabsf(mx)), clipped, sh);
+                    int Amax, Bmin;
+                    {
+                        const float g0 = grid_point(mn, mx, step, lane), g1 = grid_point(mn, mx, step, lane + 32);
+                        const unsigned long long le = (unsigned long long)__ballot_sync(kFull, g0 <= bl.a) |
+                                                      ((unsigned long long)__ballot_sync(kFull, g1 <= bl.a) << 32);
+                        const unsigned long long ge = (unsigned long long)__ballot_sync(kFull, g0 >= bl.b) |
+                                                      ((unsigned long long)__ballot_sync(kFull, g1 >= bl.b) << 32);
+                        Amax = le ? 63 - __clzll(le) : 0;
+                        Bmin = ge ? __ffsll(ge) - 1 : 63;
+                    }
                     for (int i = tid; i < nvalid; i += kCtaThreads) {
                         const int ps = grid_pos<kPbFBits>(clipped(vs[i]), mn, scale);
                         const int cell = min(ps >> kPbFBits, kTopCell);
@@ -397,17 +564,19 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                         }
                     }
                     __syncthreads();
-                    // thread (B = tid % 64, group tid / 64) searches A in [16*group, 16*group + 16) below B
+                    // thread (B = tid % 64, group tid / 64) searches A in [kSpan*group, kSpan*(group + 1)) below B
+                    constexpr int kSpan = 128 / NW;  // A values per thread: NW / 2 groups of 64 threads
                     const int B = tid & 63, grp = tid >> 6;
                     const unsigned long long bb = (unsigned long long)B << kPbFBits;
                     const unsigned long long beB = sh.be[B], gaB = sh.ga[B];
                     long long best_e = 0x7fffffffffffffffll;
                     int best_ab = 0x7fffffff;
-                    for (int A = 16 * grp; A < 16 * grp + 16 && A < B; ++A) {
+                    for (int A = kSpan * grp; A < kSpan * grp + kSpan && A < B; ++A) {
                         const unsigned long long aa = (unsigned long long)A << kPbFBits;
                         const long long e = (long long)((unsigned long long)sh.al[A] + beB + aa * gaB + bb * (unsigned long long)sh.de[A]);
                         const int ab = A * 64 + B;
-                        if (e < best_e || (e == best_e && ab < best_ab)) {
+                        const bool admissible = A <= Amax && B >= Bmin;
+                        if (admissible && (e < best_e || (e == best_e && ab < best_ab))) {
                             best_e = e;
                             best_ab = ab;
                         }
@@ -426,10 +595,10 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                         sh.redi[wid] = best_ab;
                     }
                     __syncthreads();
-                    best_e = sh.redl[0][lane & 7];
-                    best_ab = sh.redi[lane & 7];
+                    best_e = sh.redl[0][lane & (NW - 1)];
+                    best_ab = sh.redi[lane & (NW - 1)];
 #pragma unroll
-                    for (int o = 4; o > 0; o >>= 1) {
+                    for (int o = NW / 2; o > 0; o >>= 1) {
                         const long long oe = __shfl_xor_sync(kFull, best_e, o);
                         const int oab = __shfl_xor_sync(kFull, best_ab, o);
                         if (oe < best_e || (oe == best_e && oab < best_ab)) {
@@ -453,103 +622,7 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                 for (int i = tid; i < nvalid; i += kCtaThreads) m = fmaxf(m, fabsf(clipped(vs[i])));
                 m = block_max(m, sh, 0);
             }
-            if (m > 0.0f) {
-                // sort u in place (padding = +inf)
-                for (int i = tid; i < d; i += kCtaThreads) vs[i] = i < nvalid ? clipped(vs[i]) : INFINITY;
-                __syncthreads();
-                for (int k = 2; k <= d; k <<= 1) {
-                    for (int j = k >> 1; j > 0; j >>= 1) {
-                        for (int i = tid; i < d; i += kCtaThreads) {
-                            const int ixj = i ^ j;
-                            if (ixj > i) {
-                                const float a = vs[i], b = vs[ixj];
-                                const bool up = (i & k) == 0;
-                                if ((a > b) == up) {
-                                    vs[i] = b;
-                                    vs[ixj] = a;
-                                }
-                            }
-                        }
-                        __syncthreads();
-                    }
-                }
-                // exact prefix sums of the fixed-point values: thread t owns positions [t*seg, (t+1)*seg)
-                const int e2 = 46 - fexpo(m);
-                const double sc = pow2d(e2);
-                const int seg = d / kCtaThreads;
-                long long run = 0;
-                for (int i = tid * seg; i < tid * seg + seg; ++i) run += (i < nvalid) ? fixed_point(vs[i], sc) : 0ll;
-                const long long incl = warp_inclusive_scan(run, lane);
-                if (lane == 31) sh.redl[0][wid] = incl;
-                __syncthreads();
-                long long wpre = 0, total = 0;
-                for (int k = 0; k < kCtaWarps; ++k) {
-                    const long long t = sh.redl[0][k];
-                    if (k < wid) wpre += t;
-                    total += t;
-                }
-                __syncthreads();
-                long long S = wpre + incl - run;  // sum of positions before tid*seg
-                double best_j = -1.0;
-                int best_i = 0x7fffffff;
-                long long best_s = 0;
-                for (int i = tid * seg; i < tid * seg + seg; ++i) {
-                    if (i >= 1 && i < nvalid && vs[i - 1] < vs[i]) {
-                        const double l = __ll2double_rn(S);
-                        const double rr = __ll2double_rn(total - S);
-                        const double J = __dadd_rn(__ddiv_rn(__dmul_rn(l, l), (double)i),
-                                                   __ddiv_rn(__dmul_rn(rr, rr), (double)(nvalid - i)));
-                        if (J > best_j) {
-                            best_j = J;
-                            best_i = i;
-                            best_s = S;
-                        }
-                    }
-                    if (i < nvalid) S += fixed_point(vs[i], sc);
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const double oj = __shfl_xor_sync(kFull, best_j, o);
-                    const int oi = __shfl_xor_sync(kFull, best_i, o);
-                    const long long os = __shfl_xor_sync(kFull, best_s, o);
-                    if (oj > best_j || (oj == best_j && oi < best_i)) {
-                        best_j = oj;
-                        best_i = oi;
-                        best_s = os;
-                    }
-                }
-                if (lane == 0) {
-                    sh.redd[wid] = best_j;
-                    sh.redi[wid] = best_i;
-                    sh.redl[1][wid] = best_s;
-                }
-                __syncthreads();
-                best_j = sh.redd[lane & 7];
-                best_i = sh.redi[lane & 7];
-                best_s = sh.redl[1][lane & 7];
-#pragma unroll
-                for (int o = 4; o > 0; o >>= 1) {
-                    const double oj = __shfl_xor_sync(kFull, best_j, o);
-                    const int oi = __shfl_xor_sync(kFull, best_i, o);
-                    const long long os = __shfl_xor_sync(kFull, best_s, o);
-                    if (oj > best_j || (oj == best_j && oi < best_i)) {
-                        best_j = oj;
-                        best_i = oi;
-                        best_s = os;
-                    }
-                }
-                if (best_i == 0x7fffffff) {
-                    const float v0 = __fadd_rn(vs[0], 0.0f);
-                    rb = RoundB{v0, v0, v0, false};
-                } else {
-                    const double inv_sc = pow2d(-e2);
-                    const float a = __double2float_rn(__dmul_rn(__ddiv_rn(__ll2double_rn(best_s), (double)best_i), inv_sc));
-                    const float b = __double2float_rn(
-                        __dmul_rn(__ddiv_rn(__ll2double_rn(total - best_s), (double)(nvalid - best_i)), inv_sc));
-                    rb = RoundB{a, b, vs[best_i], true};
-                }
-                __syncthreads();
-            }
+            if (m > 0.0f) rb = cta_bingrad_b_levels<NW>(vs, d, nvalid, m, clipped, sh);
         }
 
         // ---- round, pack, write residual and message ---------------------------------------------
@@ -557,7 +630,7 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
         for (int ch = wid; ch < nchunks; ch += kCtaWarps) {
             const int e0 = ch * 128 + 4 * lane;
             float v4[4];
-            if constexpr (SCHEME == GQ_BINGRAD_B) {
+            if constexpr (SCHEME == GQ_BINGRAD_B || SCHEME == GQ_BINGRAD_PB) {
                 // the sort overwrote the staged values: read g (+ r) again
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -603,20 +676,47 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
                 } else {
                     err_chunk<false, false>(p, rb, blk, worker, lane, valid, u4, pos4, ea);
                 }
-            } else if constexpr (SCHEME == GQ_QSGD) {
-                round_chunk<true, false, 0>(p, rq, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
-            } else if constexpr (SCHEME == GQ_ORQ) {
-                if (constant)
-                    round_chunk<false, false, 0>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
-                else
-                    round_chunk<true, false, 0>(p, ro, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
-            } else if constexpr (SCHEME == GQ_BINGRAD_PB) {
-                if (constant)
-                    round_chunk<false, false, 0>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
-                else
-                    round_chunk<true, false, 0>(p, rp, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
             } else {
-                round_chunk<false, false, 0>(p, rb, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                if constexpr (SCHEME == GQ_QSGD) {
+                    round_chunk<true, false, 0>(p, rq, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                } else if constexpr (SCHEME == GQ_ORQ) {
+                    if (constant)
+                        round_chunk<false, false, 0>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    else
+                        round_chunk<true, false, 0>(p, ro, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                } else if constexpr (SCHEME == GQ_BINGRAD_PB) {
+                    if (constant)
+                        round_chunk<false, false, 0>(p, RoundConst{mn}, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                    else
+                        round_chunk<true, false, 0>(p, rp, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                } else {
+                    round_chunk<false, false, 0>(p, rb, blk, worker, lane, valid, v4, u4, pos4, rout, cwc, q);
+                }
+                if (fused) {
+                    // running sum in worker order from +0; the last worker writes the average.  The
+                    // element's sum is read and written by this thread only.
+                    float *ab = (acc_smem ? accs : p.avg + base) + e0;
+                    float *out = p.avg + base + e0;
+                    const bool last = w == W - 1;
+                    if (valid == 0xfu) {
+                        float4 a = w == 0 ? make_float4(0.0f, 0.0f, 0.0f, 0.0f) : *reinterpret_cast<const float4 *>(ab);
+                        a = make_float4(__fadd_rn(a.x, q[0]), __fadd_rn(a.y, q[1]), __fadd_rn(a.z, q[2]), __fadd_rn(a.w, q[3]));
+                        if (last)
+                            __stcs(reinterpret_cast<float4 *>(out), make_float4(__fmul_rn(a.x, p.inv_w), __fmul_rn(a.y, p.inv_w),
+                                                                                __fmul_rn(a.z, p.inv_w), __fmul_rn(a.w, p.inv_w)));
+                        else
+                            *reinterpret_cast<float4 *>(ab) = a;
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            if ((valid >> c) & 1u) {
+                                const float a = __fadd_rn(w == 0 ? 0.0f : ab[c], q[c]);
+                                if (last) out[c] = __fmul_rn(a, p.inv_w);
+                                else ab[c] = a;
+                            }
+                        }
+                    }
+                }
             }
         }
         if constexpr (ERR) {
@@ -645,26 +745,36 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta(const __grid_constant__ KPa
             reinterpret_cast<float *>(msg + p.levels_off)[beta * p.L + tid] = lv;
         }
         __syncthreads();
+      }
     }
 }
 
-template <int SCHEME, bool ERR>
+template <int SCHEME, bool ERR, int NW>
 cudaError_t launch(const KParams &p, double *part, cudaStream_t stream)
 {
-    auto kern = k_cta<SCHEME, ERR>;
-    const size_t smem = (size_t)p.d * 4 + (SCHEME == GQ_ORQ ? (size_t)kCtaWarps * kWarpHistWords * 4 : 0);
+    auto kern = k_cta<SCHEME, ERR, NW>;
+    const bool acc_smem = !ERR && p.avg != nullptr && p.d <= kAccSmemMax;
+    const size_t smem = (size_t)p.d * 4 * (acc_smem ? 2 : 1) +
+                        (SCHEME == GQ_ORQ ? (size_t)NW * kWarpHistWords * 4 : 0);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCtaThreads, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NW * 32, smem);
     if (per_sm < 1) per_sm = 1;
     const int64_t cap = (int64_t)sms * per_sm;
     const int grid = (int)(p.nb < cap ? p.nb : cap);
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kCtaThreads, smem, stream>>>(p, part);
+    kern<<<grid, NW * 32, smem, stream>>>(p, part);
     return cudaGetLastError();
+}
+
+// 8 warps per CTA, 16 for the largest buckets (one CTA fits per SM there).
+template <int SCHEME, bool ERR>
+cudaError_t launch_nw(const KParams &p, double *part, cudaStream_t stream)
+{
+    return p.d >= 16384 ? launch<SCHEME, ERR, 16>(p, part, stream) : launch<SCHEME, ERR, 8>(p, part, stream);
 }
 
 template <bool ERR>
@@ -672,10 +782,10 @@ cudaError_t dispatch(const KParams &p, double *part, cudaStream_t stream)
 {
     switch (p.scheme) {
     case GQ_QSGD:
-    case GQ_TERNGRAD: return launch<GQ_QSGD, ERR>(p, part, stream);
-    case GQ_BINGRAD_B: return launch<GQ_BINGRAD_B, ERR>(p, part, stream);
-    case GQ_BINGRAD_PB: return launch<GQ_BINGRAD_PB, ERR>(p, part, stream);
-    default: return launch<GQ_ORQ, ERR>(p, part, stream);
+    case GQ_TERNGRAD: return launch_nw<GQ_QSGD, ERR>(p, part, stream);
+    case GQ_BINGRAD_B: return launch_nw<GQ_BINGRAD_B, ERR>(p, part, stream);
+    case GQ_BINGRAD_PB: return launch_nw<GQ_BINGRAD_PB, ERR>(p, part, stream);
+    default: return launch_nw<GQ_ORQ, ERR>(p, part, stream);
     }
 }
 

@@ -46,7 +46,8 @@ constexpr unsigned kStatusTimeout = 2u;  // a bounded wait on a bulk copy gave u
 // The ragged last bucket (when n is not a multiple of d) goes to a one-warp launch of the same
 // code with guarded loads, so the main kernel carries no tail logic.
 cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream);
-// Shared-memory path (d = 1024 .. 32768): one CTA per bucket, one worker per launch.
+// Shared-memory path (d = 1024 .. 32768): one CTA per bucket index walking the p.W workers;
+// with p.avg set, the average of the dequantized values is accumulated on chip and written.
 cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream);
 // Dequantize + aggregate for any d.
 cudaError_t launch_decode(const KParams &p, cudaStream_t stream);

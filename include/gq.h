@@ -153,11 +153,13 @@ GQ_API gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs,
 /*
  * The whole step for the plan's W workers: worker w (w = 0..W-1, Philox worker index w) is
  * quantized as by gq_encode and the mean of the W dequantized gradients is written to avg,
- * as by gq_decode_accumulate; for d <= 512 the dequantized values never leave the chip.
+ * as by gq_decode_accumulate; the dequantized values never leave the chip (for d <= 512 they
+ * are summed in registers; for larger buckets one CTA walks a bucket's W workers and keeps the
+ * running sum in shared memory, or, above d = 8192, in avg's own slice while it stays in L2).
  *   grads      host array of W device pointers (n float32 each).
  *   residuals  host array of W device pointers (in/out), or NULL iff error_feedback is 0.
  *   msgs       host array of W device pointers receiving the messages, or NULL not to write
- *              messages (allowed for d <= 512 only; larger buckets go through the messages).
+ *              messages.
  *   avg        device, n float32, overwritten.
  */
 GQ_API gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *grads, float *const *residuals,

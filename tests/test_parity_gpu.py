@@ -124,6 +124,27 @@ def test_fused_without_messages_matches():
         assert all(np.array_equal(x, y) for x, y in zip(gr, orr))
 
 
+@pytest.mark.parametrize("scheme,levels", [("orq", 5), ("qsgd", 5), ("bingrad_b", 2), ("bingrad_pb", 2)])
+@pytest.mark.parametrize("d", [1024, 8192, 16384, 32768])
+def test_large_buckets_fused_without_messages(scheme, levels, d):
+    """One CTA walks the W workers of a bucket and keeps the running sum on chip: in shared
+    memory up to d = 8192, in the average's own slice (L2) above; with and without messages
+    the average and residuals equal the oracle's, including a ragged last bucket."""
+    W = 5
+    nbk = 1 if (scheme == "bingrad_pb" and d >= 8192) else 2
+    n = nbk * d + (77 if d < 32768 else -300)
+    cg, co = configs(scheme, levels, d, W, True, 0.0, 21, n)
+    g = _grads(n, W, 2, seed=d + 7 * levels, dist="t3")
+    o = run_oracle_fused(co, 2, g)
+    for with_msgs in (False, True):
+        a = run_gpu_fused(cg, 2, g, with_msgs=with_msgs)
+        if with_msgs:
+            compare_steps(a, o, co, "%s-%d d=%d" % (scheme, levels, d))
+        for (ga, gr, _), (oa, orr, _) in zip(a, o):
+            assert np.array_equal(ga.view(np.uint32), oa.view(np.uint32))
+            assert all(np.array_equal(x, y) for x, y in zip(gr, orr))
+
+
 def test_many_workers():
     n, W = 3 * 512 + 11, 64
     cg, co = configs("orq", 5, 512, W, True, 0.0, 2, n)
@@ -172,11 +193,8 @@ def test_invalid_arguments_rejected():
         assert ei.value.status == G.GQ_ERR_INVALID
         with pytest.raises(G.GQError):         # misaligned gradient
             G.gq_encode(plan.handle, 0, 0, g.data_ptr() + 4, g, msg)
-        with pytest.raises(G.GQError):         # no messages for a fused step with d > 512 is
-            cg2, _ = configs("orq", 5, 2048, 2, True, 0.0, 1, 4096)      # checked per plan
-            with G.Plan(cg2) as p2:
-                x = torch.zeros(4096, device="cuda")
-                G.gq_fused_step(p2.handle, 0, [x, x], [x.clone(), x.clone()], None, x.clone())
+        with pytest.raises(G.GQError):         # misaligned average
+            G.gq_fused_step(plan.handle, 0, [g, g], [g.clone(), g.clone()], None, g.data_ptr() + 4)
 
 
 def test_deterministic_repeat():
@@ -211,3 +229,44 @@ def test_checkpoint_resume_is_bit_identical():
             G.gq_fused_step(plan.handle, t, [torch.from_numpy(x).cuda() for x in g[t]], r, None, avg)
             assert np.array_equal(avg.cpu().numpy().view(np.uint32), full[t][0].view(np.uint32))
         assert all(np.array_equal(x.cpu().numpy(), y) for x, y in zip(r, full[3][1]))
+
+
+def _bingrad_buckets(kind, d, rng):
+    """Buckets that stress BinGrad's split search: duplicates, gaps, heavy tails, huge dynamic
+    range, narrow all-positive ranges (where the grid cannot separate the values) and
+    distributions whose best split is far from the middle."""
+    if kind == "integers":
+        return rng.integers(-3, 4, d).astype(np.float32)
+    if kind == "bimodal":
+        x = np.concatenate([rng.normal(-1.0, 0.01, d // 2), rng.normal(2.0, 0.01, d - d // 2)])
+        return (rng.permutation(x) * 1e-3).astype(np.float32)
+    if kind == "cauchy":
+        return (rng.standard_cauchy(d) * 1e-4).astype(np.float32)
+    if kind == "dynamic":
+        return (np.sign(rng.standard_normal(d)) * 10.0 ** rng.uniform(-30, 0, d)).astype(np.float32)
+    if kind == "narrow":
+        return (1.0 + rng.standard_normal(d) * 1e-6).astype(np.float32)
+    if kind == "skewed":
+        return (rng.exponential(1.0, d) ** 3 * 1e-3).astype(np.float32)
+    if kind == "uniform":
+        return rng.uniform(-1e-3, 1e-3, d).astype(np.float32)
+    if kind == "fewvalues":
+        return rng.choice(np.array([-2e-3, -1e-3, 5e-4, 3e-3], np.float32), d)
+    raise KeyError(kind)
+
+
+@pytest.mark.parametrize("kind", ["integers", "bimodal", "cauchy", "dynamic", "narrow", "skewed", "uniform",
+                                  "fewvalues"])
+@pytest.mark.parametrize("scheme", ["bingrad_b", "bingrad_pb"])
+@pytest.mark.parametrize("d", [128, 512])
+def test_bingrad_split_search_stress(kind, scheme, d):
+    """The register path's split search sorts only the grid cells that can hold the best split
+    (falling back to a full sort when they hold too many values); every choice must still be
+    the exhaustive one, bit for bit."""
+    rng = np.random.default_rng(sum(map(ord, kind)) + d)
+    W, nbk = 2, 12
+    g = [[np.concatenate([_bingrad_buckets(kind, d, rng) for _ in range(nbk)] + [_bingrad_buckets(kind, 77, rng)])
+          for _ in range(W)]]
+    n = g[0][0].size
+    cg, co = configs(scheme, 2, d, W, True, 0.0, 13, n)
+    compare_steps(run_gpu_fused(cg, 1, g), run_oracle_fused(co, 1, g), co, "%s %s d=%d" % (scheme, kind, d))
