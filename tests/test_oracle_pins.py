@@ -171,8 +171,13 @@ def _naive_orq(u, s):
 
 @pytest.mark.parametrize("s", [2, 3, 5, 9])
 def test_orq_matches_naive_greedy(s):
+    """The fixed-point greedy (positions with 16 fraction bits per grid cell, exact integer
+    objective) against an independent greedy on the raw values in float64.  Every pick must be
+    as good as the real-valued one to 1e-9 relative; on normal and Laplace buckets the picks
+    must be the same levels.  (Measured on 300 buckets of d = 512 per workload distribution and
+    s = 3, 5, 9: the picks differ only on Student-t buckets with outliers, where candidates tie
+    exactly -- the real-valued variances differ by at most 1.1e-13 relative.)"""
     rng = np.random.default_rng(s)
-    same = 0
     trials = 12
     for t in range(trials):
         n = int(rng.integers(40, 300))
@@ -189,9 +194,9 @@ def test_orq_matches_naive_greedy(s):
         assert sorted(idx.tolist()) == idx.tolist()
         assert idx[0] == 0 and idx[-1] == 63
         mine = total(list(idx))
-        assert mine <= tot * (1 + 1e-5) + 1e-30
-        same += list(idx) == lv
-    assert same >= trials - 1
+        assert mine <= tot * (1 + 1e-9) + 1e-30
+        if dist < 2:
+            assert list(idx) == lv, (t, list(idx), lv)
 
 
 def test_orq_greedy_nested_and_monotone():
@@ -494,7 +499,7 @@ def test_clip_threshold_is_c_sigma():
     assert table[-1] <= T and table[0] >= -T and np.abs(q).max() <= T
 
 
-@pytest.mark.parametrize("levels", [2, 3, 4, 5, 9, 16])
+@pytest.mark.parametrize("levels", [2, 3, 4, 5, 9, 16, 255])
 def test_pack_roundtrip(levels):
     rng = np.random.default_rng(levels)
     for d in (128, 512, 2048):
@@ -510,10 +515,11 @@ def test_pack_roundtrip(levels):
                 assert np.array_equal(O.unpack_bucket(cfg, words, d)[n:], np.zeros(d - n, np.uint8))
 
 
-@pytest.mark.parametrize("levels", [2, 3, 5, 9, 16])
+@pytest.mark.parametrize("levels", [2, 3, 5, 9, 16, 255])
 def test_pack_is_dense_little_endian(levels):
     """Packing layout: element e's code is bits b*e .. b*e+b-1 of the bucket's little-endian
-    bit string (here built as one Python integer, independently of the C loop)."""
+    bit string (here built as one Python integer, independently of the C loop); 255 levels
+    give the byte codes of INT8."""
     rng = np.random.default_rng(100 + levels)
     b = O.bits(levels)
     for d, n in ((128, 128), (512, 512), (512, 301), (1024, 1000)):
@@ -757,7 +763,7 @@ def test_entropy_roundtrip(levels):
 # Biased baselines ([P3] "Deterministic vs stochastic rounding", "Ternary and binary
 # quantization"): QSGD levels with rounding to the nearest level, and the scaled sign
 # ------------------------------------------------------------------------------------------
-@pytest.mark.parametrize("levels", [2, 3, 5, 9, 15, 16])
+@pytest.mark.parametrize("levels", [2, 3, 5, 9, 15, 16, 129, 255, 256])
 def test_qsgd_nearest_is_nearest_level(levels):
     """Every value goes to a nearest QSGD level (brute force over the levels, up to the
     rounding of the binary32 position); no randomness: seed, step and worker do not matter."""
@@ -780,6 +786,28 @@ def test_qsgd_nearest_is_nearest_level(levels):
         ks = np.clip(np.trunc((v / np.float32(m) + 1) * (levels - 1) / 2), 0, levels - 2)
         assert np.all((code == ks) | (code == ks + 1))
     assert np.array_equal(outs[0], outs[1])
+
+
+def test_int8_levels_are_symmetric_integers():
+    """[P3] core mechanism: INT8 maps each value to an 8-bit integer with a scale, for a 4x
+    compression.  Reading: QSGD with 255 levels, m * (2k - 254) / 254 = m * (k - 127) / 127,
+    i.e. the integers -127 .. 127 times m / 127 (zero included), nearest rounding; 8-bit codes."""
+    rng = np.random.default_rng(255)
+    v = (rng.laplace(0, 1e-3, 512)).astype(np.float32)
+    cfg = O.Config(O.QSGD_NEAREST, 255, 512, 1, 0, 0.0, 0, 512)
+    assert O.bits(255) == 8
+    code, q, table = O.encode_bucket(cfg, 0, 0, 0, v)
+    m = float(table[0])
+    for c in np.unique(code):
+        lvl = O.dequant(cfg, table, int(c))
+        assert abs(lvl - m * (int(c) - 127) / 127) <= 2 ** -23 * m
+    assert O.dequant(cfg, table, 127) == 0.0
+    x = v.astype(np.float64) / m * 127          # nearest integer in -127 .. 127
+    near = np.rint(x)
+    off = np.abs(x - near) < 0.5 - 1e-3         # away from half-way points
+    assert np.array_equal(code[off].astype(int) - 127, near[off].astype(int))
+    total, _, _ = O.message_layout(O.Config(O.QSGD_NEAREST, 255, 512, 1, 0, 0.0, 0, 512 * 64))
+    assert 32 * 512 * 64 / (8 * total) > 3.9       # about 4x over fp32 with the scale table
 
 
 def test_qsgd_nearest_ties_go_up():
