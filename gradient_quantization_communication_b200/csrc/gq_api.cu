@@ -46,11 +46,15 @@ gq_status_t normalise(const gq_config_t *in, gq_config_t *out)
     if (!in) return GQ_ERR_INVALID;
     gq_config_t c = *in;
     switch (c.scheme) {
-    case GQ_QSGD:
     case GQ_ORQ:
+        if (c.levels < 2 || c.levels > GQ_MAX_LEVELS) return GQ_ERR_INVALID;
+        break;
+    case GQ_QSGD:
     case GQ_QSGD_NEAREST:
     case GQ_QSGD_L2:
-        if (c.levels < 2 || c.levels > GQ_MAX_LEVELS) return GQ_ERR_INVALID;
+        // 2 .. 16 levels take 1 .. 4-bit codes; 129 .. 256 levels take 8-bit codes
+        if (c.levels < 2 || (c.levels > GQ_MAX_LEVELS && c.levels <= 128) || c.levels > GQ_MAX_QSGD_LEVELS)
+            return GQ_ERR_INVALID;
         break;
     case GQ_TERNGRAD:
         if (c.levels == 0) c.levels = 3;

@@ -39,7 +39,7 @@ struct alignas(16) CtaShared {
     int P0[64];
     long long al[64], be[64], ga[64], de[64];
     float4 ctab[64];
-    float2 pair[16];
+    float2 pair[GQ_MAX_QSGD_LEVELS];
     float lev[16];
     float rinv[16];
     float bcast_f[4];
@@ -399,11 +399,8 @@ __global__ void __launch_bounds__(NW * 32) k_cta(const __grid_constant__ KParams
                 m = block_max(m, sh, 0);
             }
             const int s = p.s;
-            if (wid == 0) {
-                const float lv = lane < s ? __fmul_rn(m, p.qratio[lane]) : 0.0f;
-                const float lv_next = __shfl_down_sync(kFull, lv, 1);
-                if (lane < s - 1) sh.pair[lane] = make_float2(lv, lv_next);
-            }
+            for (int k = tid; k < s - 1; k += kCtaThreads)
+                sh.pair[k] = make_float2(__fmul_rn(m, p.qratio[k]), __fmul_rn(m, p.qratio[k + 1]));
             if (tid == 0) sh.bcast_f[0] = m;
             __syncthreads();
             rq.inv_m = m > 0.0f ? __frcp_rn(m) : 0.0f;

@@ -7,7 +7,8 @@
 // are formed once per item; the chunks then sit at fixed offsets from them.  The level lookup
 // is a register shuffle within segments of 2^b lanes: every segment holds the bucket's level
 // table in its first L lanes, and a shuffle of width 2^b takes its source lane modulo 2^b, so
-// the code needs no masking.  The loads of a group of workers are issued together before any
+// the code needs no masking (8-bit codes of the QSGD family look their ratio up in a shared
+// table instead).  The loads of a group of workers are issued together before any
 // of them is used; the sum runs in worker order in registers and the average is written once,
 // with 16-byte stores.
 #include "gq_device.cuh"
@@ -33,6 +34,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
     const bool cross = sh + 4 * BITS > 32;  // the field crosses a word boundary (b = 3 only)
     const bool has_level = slot < p.L;
     const float qr = (QSGD && slot < p.s) ? p.qratio[slot] : 0.0f;
+    // 8-bit codes (QSGD family, 129 .. 256 levels): the level ratios in shared memory
+    __shared__ float qtab[BITS == 8 ? 256 : 1];
+    if (BITS == 8) {
+        for (int k = threadIdx.x; k < p.s; k += blockDim.x) qtab[k] = p.qratio[k];
+        __syncthreads();
+    }
     for (int64_t it = first; it < nitems; it += stride) {
         const int64_t e0 = it * (128 * CPI);
         const int64_t bk = e0 >> log2d;
@@ -67,7 +74,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
             }
 #pragma unroll
             for (int k = 0; k < kDecodeGroup; ++k) {
-                if (w0 + k < p.W) {
+                if (BITS == 8 && w0 + k < p.W) {
+#pragma unroll
+                    for (int c = 0; c < CPI; ++c)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            acc[c][e] = __fadd_rn(acc[c][e], __fmul_rn(lv[k], qtab[(x[k][c] >> (8 * e)) & 0xffu]));
+                } else if (w0 + k < p.W) {
                     const float level = QSGD ? __fmul_rn(lv[k], qr) : lv[k];
 #pragma unroll
                     for (int c = 0; c < CPI; ++c) {
@@ -132,7 +145,10 @@ cudaError_t launch_bits(const KParams &p, cudaStream_t stream)
     case 1: return launch_cpi<QSGD, 1>(p, stream);
     case 2: return launch_cpi<QSGD, 2>(p, stream);
     case 3: return launch_cpi<QSGD, 3>(p, stream);
-    default: return launch_cpi<QSGD, 4>(p, stream);
+    case 4: return launch_cpi<QSGD, 4>(p, stream);
+    default:
+        if constexpr (QSGD) return launch_cpi<QSGD, 8>(p, stream);  // 8-bit codes: QSGD family only
+        else return cudaErrorInvalidValue;
     }
 }
 

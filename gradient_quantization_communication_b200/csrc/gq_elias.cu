@@ -384,7 +384,7 @@ gq_status_t el_layout(const gq_config_t *cfg, ElLayout *out)
     if (c.scheme == GQ_TERNGRAD && c.levels == 0) c.levels = 3;
     const bool qs = c.scheme == GQ_QSGD || c.scheme == GQ_TERNGRAD || c.scheme == GQ_QSGD_NEAREST ||
                     c.scheme == GQ_QSGD_L2;
-    if (!qs || c.levels % 2 == 0 || c.bucket > 512) return GQ_ERR_UNSUPPORTED;
+    if (!qs || c.levels % 2 == 0 || c.levels > 15 || c.bucket > 512) return GQ_ERR_UNSUPPORTED;
     ElLayout l;
     l.s = c.levels;
     l.b = 0;

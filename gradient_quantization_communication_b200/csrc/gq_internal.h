@@ -28,7 +28,7 @@ struct KParams {
     unsigned long long step_m1;  // 0xCD9E8D57 * step_lo (Philox round-1 product of counter word 2)
     uint32_t worker0;    // Philox worker index of worker slot 0
     float inv_w;         // 1/W for the average
-    float qratio[GQ_MAX_LEVELS];  // QSGD level k = m * qratio[k], qratio[k] = (2k-(s-1))/(s-1)
+    float qratio[GQ_MAX_QSGD_LEVELS];  // QSGD level k = m * qratio[k], qratio[k] = (2k-(s-1))/(s-1)
     int64_t codes_words; // words of packed codes per bucket (d*b/32)
     int64_t levels_off;  // byte offset of the level tables inside a message
     const float *g[GQ_MAX_WORKERS];

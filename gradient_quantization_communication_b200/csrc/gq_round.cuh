@@ -141,12 +141,19 @@ struct RoundPB {
 // of the chunk's 4b words (least significant bit first).  Lane l's four codes form the 4b-bit
 // field at bit 4b*l; pairs, quads and octets of lanes merge their fields with shuffles (the
 // fields do not overlap, so the merges are additions, done by the integer multiply-add unit),
-// and lane 8g stores the b words of octet g.  Every lane of the warp must take part.
+// and lane 8g stores the b words of octet g.  8-bit codes are stored by every lane, one word
+// each.  Every lane of the warp must take part.
 // BITS: bits per code when known at compile time, 0 to read it from p.bits.
 template <int BITS>
 __device__ __forceinline__ void pack_chunk(const KParams &p, int lane, const int (&code)[4], uint32_t *cw)
 {
     const int b = BITS > 0 ? BITS : p.bits;  // (BITS < 0 only in never-run instantiations)
+    if (BITS == 8 || (BITS == 0 && b == 8)) {
+        // 8-bit codes: lane l's four codes are word l of the chunk
+        __stcs(cw + lane, (uint32_t)code[0] | ((uint32_t)code[1] << 8) | ((uint32_t)code[2] << 16) |
+                              ((uint32_t)code[3] << 24));
+        return;
+    }
     const uint32_t f1 = 1u << b, f2 = 1u << (2 * b), f3 = 1u << (3 * b);
     const uint32_t y = (uint32_t)code[0] + (uint32_t)code[1] * f1 + (uint32_t)code[2] * f2 + (uint32_t)code[3] * f3;
     const uint32_t z = y + __shfl_down_sync(kFull, y, 1) * (1u << (4 * b));  // 8b bits

@@ -63,7 +63,8 @@ struct alignas(16) FitORQ {
     int P0[64];                     // count over cells < k
 };
 struct alignas(16) FitQSGD {
-    float2 pair[16];  // {level k, level k+1}
+    float2 pair[GQ_MAX_QSGD_LEVELS];  // {level k, level k+1}
+    float qr[GQ_MAX_QSGD_LEVELS];     // the level ratios (2k - (s-1)) / (s-1), copied once
 };
 struct alignas(16) FitPB {
     FitB b;                             // BinGrad-b's split search, run first
@@ -214,10 +215,8 @@ __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int
         }
     }
     const int s = p.s;
-    const float lv = lane < s ? __fmul_rn(m, p.qratio[lane]) : 0.0f;
-    const float lv_next = __shfl_down_sync(kFull, lv, 1);
     __syncwarp();
-    if (lane < s - 1) sm.pair[lane] = make_float2(lv, lv_next);
+    for (int k = lane; k < s - 1; k += 32) sm.pair[k] = make_float2(__fmul_rn(m, sm.qr[k]), __fmul_rn(m, sm.qr[k + 1]));
     __syncwarp();
     RoundQSGDT<NEAREST> rule;
     rule.inv_m = m > 0.0f ? __frcp_rn(m) : 0.0f;
@@ -604,8 +603,11 @@ constexpr int min_blocks()
 }
 
 template <int SCHEME, class Fit>
-__device__ __forceinline__ void init_fit(Fit &fit, int lane)
+__device__ __forceinline__ void init_fit(const KParams &p, Fit &fit, int lane)
 {
+    if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD || SCHEME == GQ_QSGD_NEAREST || SCHEME == GQ_QSGD_L2) {
+        for (int k = lane; k < p.s; k += 32) fit.qr[k] = p.qratio[k];
+    }
     if constexpr (SCHEME == GQ_ORQ || SCHEME == GQ_BINGRAD_B) {
         for (int i = lane; i < 64 * kHistCols; i += 32) fit.hist[i] = 0u;
     }
@@ -641,7 +643,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, (min_blocks<EPL, SCHEME, kW
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
     Smem &sm = reinterpret_cast<Smem *>(smem_raw)[wib];
-    init_fit<SCHEME>(sm.fit, lane);
+    init_fit<SCHEME>(p, sm.fit, lane);
     if (lane == 0) {
         for (int k = 0; k < kStages; ++k) mbar_init(&sm.bar[k], 1);
         fence_barrier_init();
@@ -736,7 +738,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) k_warp_err(const __grid_con
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     Fit &fit = reinterpret_cast<Fit *>(smem_raw)[wib];
-    init_fit<SCHEME>(fit, lane);
+    init_fit<SCHEME>(p, fit, lane);
     __syncwarp();
     const float *g = p.g[0];
     const float *r = p.r[0];
@@ -828,7 +830,7 @@ __global__ void __launch_bounds__(512) k_warp_tail(const __grid_constant__ KPara
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     Fit &fit = reinterpret_cast<Fit *>(smem_raw)[wid];
     float *qbuf = reinterpret_cast<float *>(smem_raw + sizeof(Fit) * nwarps);  // [W][D]
-    init_fit<SCHEME>(fit, lane);
+    init_fit<SCHEME>(p, fit, lane);
     __syncwarp();
     const int64_t beta = p.nb - 1;
     const int nvalid = p.tail;
@@ -908,14 +910,22 @@ cudaError_t launch_one(const KParams &p, cudaStream_t stream)
 template <int SCHEME, int EPL, bool FUSED>
 cudaError_t dispatch_bits(const KParams &p, cudaStream_t stream)
 {
-    if constexpr (SCHEME == GQ_BINGRAD_B || SCHEME == GQ_BINGRAD_PB) {
+    if constexpr (SCHEME == GQ_BINGRAD_B || SCHEME == GQ_BINGRAD_PB || SCHEME == GQ_SIGNSGD) {
         return launch_one<EPL, SCHEME, FUSED, 1>(p, stream);
-    } else {
+    } else if constexpr (SCHEME == GQ_ORQ) {
         switch (p.bits) {
         case 1: return launch_one<EPL, SCHEME, FUSED, 1>(p, stream);
         case 2: return launch_one<EPL, SCHEME, FUSED, 2>(p, stream);
         case 3: return launch_one<EPL, SCHEME, FUSED, 3>(p, stream);
         default: return launch_one<EPL, SCHEME, FUSED, 4>(p, stream);
+        }
+    } else {
+        switch (p.bits) {
+        case 1: return launch_one<EPL, SCHEME, FUSED, 1>(p, stream);
+        case 2: return launch_one<EPL, SCHEME, FUSED, 2>(p, stream);
+        case 3: return launch_one<EPL, SCHEME, FUSED, 3>(p, stream);
+        case 4: return launch_one<EPL, SCHEME, FUSED, 4>(p, stream);
+        default: return launch_one<EPL, SCHEME, FUSED, 8>(p, stream);
         }
     }
 }

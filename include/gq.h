@@ -47,6 +47,9 @@ extern "C" {
 #define GQ_MIN_BUCKET 128
 #define GQ_MAX_BUCKET 32768
 #define GQ_MAX_LEVELS 16
+/* Largest level count of the QSGD family (QSGD, QSGD-nearest, QSGD-l2): 129 .. 256 levels take
+ * 8-bit codes (255 levels with nearest rounding is symmetric INT8). */
+#define GQ_MAX_QSGD_LEVELS 256
 
 typedef enum {
     GQ_QSGD = 0,       /* s uniform levels on [-m, m], m = max|u| of the bucket, stochastic rounding */

@@ -93,3 +93,38 @@ def test_no_randomness():
         cg, _ = configs("qsgd_nearest", 5, d, 1, False, 0.0, seed, n)
         outs.append(run_gpu_fused(cg, 1, g)[0][2][0])
     assert np.array_equal(outs[0], outs[1])
+
+
+# INT8: the QSGD family with 129 .. 256 levels and 8-bit codes (255 levels with nearest
+# rounding: the symmetric integers -127 .. 127 times m / 127)
+INT8 = [("qsgd_nearest", 255), ("qsgd", 255), ("qsgd_nearest", 256), ("qsgd", 129), ("qsgd_l2", 255)]
+
+
+@pytest.mark.parametrize("scheme,levels", INT8)
+@pytest.mark.parametrize("d", [128, 512, 2048])
+def test_int8_fused_and_unfused(scheme, levels, d):
+    if d > 512 and scheme != "qsgd":
+        pytest.skip("nearest rounding and l2 scaling run on the register path only (d <= 512)")
+    n, W, steps = 5 * d + 37, 3, 2
+    cg, co = configs(scheme, levels, d, W, True, 0.0, 42, n)
+    g = _grads(n, W, steps, seed=d + levels)
+    o = run_oracle_fused(co, steps, g)
+    compare_steps(run_gpu_fused(cg, steps, g), o, co, "%s-%d d=%d" % (scheme, levels, d))
+    compare_steps(run_gpu_fused(cg, steps, g, unfused=True), o, co, "unfused %s-%d d=%d" % (scheme, levels, d))
+
+
+@pytest.mark.parametrize("kind", ["zero", "constant", "spike", "subnormal"])
+def test_int8_special_buckets(kind):
+    d, W = 512, 2
+    parts = [synth.special_bucket(kind, d, seed=w).numpy() for w in range(W)]
+    rng = np.random.default_rng(1)
+    g = [[np.concatenate([parts[w], (rng.standard_normal(d + 40) * 1e-3).astype(np.float32)]) for w in range(W)]]
+    n = g[0][0].size
+    cg, co = configs("qsgd_nearest", 255, d, W, True, 0.0, 3, n)
+    compare_steps(run_gpu_fused(cg, 1, g), run_oracle_fused(co, 1, g), co, kind)
+
+
+def test_int8_level_counts_between_17_and_128_are_rejected():
+    for levels in (17, 64, 128, 257):
+        assert G.gq_config_check(G.gq_config("qsgd_nearest", levels, 512, 1, True, 0.0, 0, 1024)) == G.GQ_ERR_INVALID
+    assert G.gq_config_check(G.gq_config("orq", 255, 512, 1, True, 0.0, 0, 1024)) == G.GQ_ERR_INVALID
