@@ -94,6 +94,10 @@ def lib():
         L.or_entropy_unpack.argtypes = [P(_Cfg), u8p, u8p]
         L.or_fused_bucket.argtypes = [P(_Cfg), ctypes.c_uint64, i64, ctypes.c_int, P(f32p), P(f32p), P(f32p),
                                       P(u32p), P(f32p), f32p]
+        i64p = P(i64)
+        L.or_tg_layer_layout.argtypes = [P(_Cfg), ctypes.c_int, P(i64), P(i64), P(i64)]
+        L.or_tg_layer_encode.argtypes = [P(_Cfg), i64p, ctypes.c_int, ctypes.c_int, ctypes.c_uint64, f32p, f32p, u8p]
+        L.or_tg_layer_decode_accumulate.argtypes = [P(_Cfg), i64p, ctypes.c_int, P(u8p), ctypes.c_int, f32p]
         _lib = L
     return _lib
 
@@ -364,3 +368,39 @@ def elias_unpack(cfg: Config, emsg):
 
 def elias_gamma_len(x):
     return lib().or_elias_gamma_len(x)
+
+
+# ---------------------------------------------------------------------------------------------
+# TernGrad with one scale per parameter tensor (segments [off[t], off[t+1]))
+# ---------------------------------------------------------------------------------------------
+def _offsets(off):
+    off = np.ascontiguousarray(np.asarray(off, dtype=np.int64))
+    return off, len(off) - 1
+
+
+def tg_layer_layout(cfg: Config, nseg):
+    b, c, s = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    lib().or_tg_layer_layout(ctypes.byref(cfg.c()), nseg, ctypes.byref(b), ctypes.byref(c), ctypes.byref(s))
+    return b.value, c.value, s.value
+
+
+def tg_layer_encode(cfg: Config, off, worker, step, g, r=None):
+    """One worker's message; r (float32, in/out) is updated in place when error feedback is on."""
+    off, nseg = _offsets(off)
+    assert g.dtype == np.float32 and g.flags.c_contiguous
+    nbytes, _, _ = tg_layer_layout(cfg, nseg)
+    msg = np.zeros(nbytes, dtype=np.uint8)
+    rp = _p(r, ctypes.c_float) if r is not None else None
+    rc = lib().or_tg_layer_encode(ctypes.byref(cfg.c()), _p(off, ctypes.c_int64), nseg, worker, step,
+                                  _p(g, ctypes.c_float), rp, _p(msg, ctypes.c_uint8))
+    assert rc == 0
+    return msg
+
+
+def tg_layer_decode_accumulate(cfg: Config, off, msgs):
+    off, nseg = _offsets(off)
+    arr = (ctypes.POINTER(ctypes.c_uint8) * len(msgs))(*[_p(m, ctypes.c_uint8) for m in msgs])
+    avg = np.zeros(cfg.n, dtype=np.float32)
+    lib().or_tg_layer_decode_accumulate(ctypes.byref(cfg.c()), _p(off, ctypes.c_int64), nseg, arr, len(msgs),
+                                        _p(avg, ctypes.c_float))
+    return avg

@@ -1235,3 +1235,109 @@ int or_elias_unpack(const or_config *cfg, const uint8_t *emsg, uint8_t *msg)
     memcpy(msg + loff, emsg + toff, (size_t)(nb * L * 4));
     return 1;
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* TernGrad with one scale per parameter tensor.  [P3] "Ternary and binary quantization":     */
+/* TernGrad sends three levels {-m, 0, +m} with a single scaling factor per layer.  The        */
+/* gradient is the concatenation of nseg tensors; tensor t holds elements [off[t], off[t+1]).  */
+/* Reading: m_t = max |v| over the tensor's elements (v = g + r with error feedback, no clip);  */
+/* element i of tensor t is rounded between the two of {-m_t, 0, +m_t} around it exactly as    */
+/* TernGrad per bucket does (position y = (v / m_t + 1), bracket k = trunc(y) clamped to       */
+/* [0, 1], up with probability y - k against the element's Philox draw).  The message holds    */
+/* the 2-bit codes in the bucket layout of the dense message (bucket size d), then the nseg    */
+/* scales (float); both regions start on 16-byte boundaries.                                   */
+/* ------------------------------------------------------------------------------------------ */
+void or_tg_layer_layout(const or_config *cfg, int nseg, int64_t *bytes, int64_t *codes_off, int64_t *scales_off)
+{
+    int64_t nb = or_num_buckets(cfg);
+    int64_t cbytes = (nb * (int64_t)cfg->bucket * 2 / 32 * 4 + 15) / 16 * 16;
+    int64_t sbytes = ((int64_t)nseg * 4 + 15) / 16 * 16;
+    *codes_off = 0;
+    *scales_off = cbytes;
+    *bytes = cbytes + sbytes;
+}
+
+static int tg_segment_of(const int64_t *off, int nseg, int64_t i)
+{
+    int t = 0;
+    while (t + 1 < nseg && off[t + 1] <= i) ++t;
+    return t;
+}
+
+int or_tg_layer_encode(const or_config *cfg, const int64_t *off, int nseg, int worker, uint64_t step,
+                       const float *g, float *r, uint8_t *msg)
+{
+    int64_t n = cfg->n, bytes, coff, soff;
+    int d = cfg->bucket;
+    if (nseg < 1 || off[0] != 0 || off[nseg] != n) return 1;
+    or_tg_layer_layout(cfg, nseg, &bytes, &coff, &soff);
+    memset(msg, 0, (size_t)bytes);
+    float *v = (float *)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+    for (int64_t i = 0; i < n; ++i) v[i] = (cfg->error_feedback && r) ? g[i] + r[i] : g[i];
+    float *scales = (float *)(msg + soff);
+    for (int t = 0; t < nseg; ++t) {
+        float m = 0.0f;
+        for (int64_t i = off[t]; i < off[t + 1]; ++i) {
+            float a = fabsf(v[i]);
+            if (a > m) m = a;
+        }
+        scales[t] = m;
+    }
+    or_config c3 = *cfg;
+    c3.levels = 3;
+    int64_t nb = or_num_buckets(cfg);
+    int64_t words = (int64_t)d * 2 / 32;
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    for (int64_t bk = 0; bk < nb; ++bk) {
+        int64_t base = bk * d;
+        int nv = (int)((n - base) < d ? (n - base) : d);
+        for (int e = 0; e < nv; ++e) {
+            int64_t i = base + e;
+            float m = scales[tg_segment_of(off, nseg, i)];
+            float inv_m = m > 0.0f ? 1.0f / m : 0.0f;
+            float y = (v[i] * inv_m + 1.0f) * 1.0f;  /* h = (s - 1) / 2 = 1 */
+            int k = 0;
+            if (y > 0.0f) k = (y >= 1.0f) ? 1 : (int)y;
+            float p = y - (float)k;
+            float U = or_uniform(cfg->seed, step, (uint32_t)worker, i);
+            int c = k + (U < p ? 1 : 0);
+            code[e] = (uint8_t)c;
+            float q = m * qsgd_ratio(c, 3);
+            if (cfg->error_feedback && r) r[i] = v[i] - q;
+        }
+        or_pack_bucket(&c3, code, nv, (uint32_t *)(msg + coff) + bk * words);
+    }
+    free(code);
+    free(v);
+    return 0;
+}
+
+int or_tg_layer_decode_accumulate(const or_config *cfg, const int64_t *off, int nseg, const uint8_t *const *msgs,
+                                  int nmsgs, float *avg)
+{
+    int64_t n = cfg->n, bytes, coff, soff;
+    int d = cfg->bucket;
+    or_tg_layer_layout(cfg, nseg, &bytes, &coff, &soff);
+    or_config c3 = *cfg;
+    c3.levels = 3;
+    int64_t nb = or_num_buckets(cfg);
+    int64_t words = (int64_t)d * 2 / 32;
+    float inv_w = 1.0f / (float)nmsgs;
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    float *acc = (float *)malloc(sizeof(float) * (size_t)d);
+    for (int64_t bk = 0; bk < nb; ++bk) {
+        int64_t base = bk * d;
+        int nv = (int)((n - base) < d ? (n - base) : d);
+        for (int e = 0; e < nv; ++e) acc[e] = 0.0f;
+        for (int w = 0; w < nmsgs; ++w) {
+            const float *scales = (const float *)(msgs[w] + soff);
+            or_unpack_bucket(&c3, (const uint32_t *)(msgs[w] + coff) + bk * words, nv, code);
+            for (int e = 0; e < nv; ++e)
+                acc[e] = acc[e] + scales[tg_segment_of(off, nseg, base + e)] * qsgd_ratio(code[e], 3);
+        }
+        for (int e = 0; e < nv; ++e) avg[base + e] = acc[e] * inv_w;
+    }
+    free(code);
+    free(acc);
+    return 0;
+}

@@ -122,6 +122,15 @@ int or_fused_bucket(const or_config *cfg, uint64_t step, int64_t bucket, int n,
                     const float *const *g, const float *const *r_in, float *const *r_out,
                     uint32_t *const *words, float *const *tables, float *avg);
 
+/* TernGrad with one scale per parameter tensor (segments [off[t], off[t+1]), off[0] = 0,
+ * off[nseg] = n): message layout, encode of one worker (r in/out, NULL without error feedback),
+ * decode + average of nmsgs messages. */
+void or_tg_layer_layout(const or_config *cfg, int nseg, int64_t *bytes, int64_t *codes_off, int64_t *scales_off);
+int or_tg_layer_encode(const or_config *cfg, const int64_t *off, int nseg, int worker, uint64_t step,
+                       const float *g, float *r, uint8_t *msg);
+int or_tg_layer_decode_accumulate(const or_config *cfg, const int64_t *off, int nseg, const uint8_t *const *msgs,
+                                  int nmsgs, float *avg);
+
 #ifdef __cplusplus
 }
 #endif

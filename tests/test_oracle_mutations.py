@@ -59,6 +59,12 @@ MUTATIONS = [
     ("elias_bit_order", "for (int j = N; j >= 0; --j, ++k)", "for (int j = 0; j <= N; ++j, ++k)"),
     ("elias_offsets", "offs[bk] = k;", "offs[bk] = k + 1;"),
     ("l2_sqrt", "return (float)ldexp(sqrt((double)sxx), -e);", "return (float)ldexp((double)sxx, -e);"),
+    ("tg_layer_segment_edge", "while (t + 1 < nseg && off[t + 1] <= i) ++t;",
+     "while (t + 1 < nseg && off[t + 1] < i) ++t;"),
+    ("tg_layer_scale_range", "for (int64_t i = off[t]; i < off[t + 1]; ++i) {",
+     "for (int64_t i = off[t]; i + 1 < off[t + 1]; ++i) {"),
+    ("tg_layer_no_draw", "(uint32_t)worker, i);\n            int c = k + (U < p ? 1 : 0);",
+     "(uint32_t)worker, i);\n            int c = k + (p >= 0.5f ? 1 : 0);"),
     ("fused_bucket_sum", "for (int i = 0; i < n; ++i) acc[i] = acc[i] + q[i];",
      "for (int i = 0; i < n; ++i) acc[i] = acc[i] + v[i];"),
 ]

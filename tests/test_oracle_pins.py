@@ -1019,3 +1019,84 @@ def test_fused_bucket_is_a_slice_of_the_step(scheme, levels):
                 assert np.array_equal(w_b[w], msgs[w][coff + 4 * words * b:coff + 4 * words * (b + 1)].view(np.uint32))
                 assert np.array_equal(t_b[w].view(np.uint32), msgs[w][loff + 4 * L * b:loff + 4 * L * (b + 1)].view(np.uint32))
             r_b[b] = r_new
+
+
+# ------------------------------------------------------------------------------------------
+# TernGrad with one scale per parameter tensor ([P3] "Ternary and binary quantization")
+# ------------------------------------------------------------------------------------------
+def test_tg_layer_equals_terngrad_when_every_tensor_is_a_bucket():
+    """With the tensors cut exactly at the bucket boundaries (the last one ragged), one scale per
+    tensor is one scale per bucket: codes, scales, residuals and average equal TernGrad's."""
+    rng = np.random.default_rng(41)
+    for d, n in ((128, 5 * 128 + 9), (512, 3 * 512)):
+        off = list(range(0, n, d)) + [n]
+        cfg = O.Config(O.TERNGRAD, 3, d, 2, 1, 0.0, 7, n)
+        gs = [(rng.laplace(0, 1e-3, n)).astype(np.float32) for _ in range(2)]
+        ra = [np.zeros(n, np.float32) for _ in range(2)]
+        rb = [np.zeros(n, np.float32) for _ in range(2)]
+        ma = [O.tg_layer_encode(cfg, off, w, 3, gs[w], ra[w]) for w in range(2)]
+        mb = [O.encode(cfg, w, 3, gs[w], rb[w]) for w in range(2)]
+        _, _, soff = O.tg_layer_layout(cfg, len(off) - 1)
+        _, coff, loff = O.message_layout(cfg)
+        for w in range(2):
+            assert np.array_equal(ma[w][:soff], mb[w][:loff])  # the codes regions
+            nb = len(off) - 1
+            assert np.array_equal(ma[w][soff:soff + 4 * nb].view(np.float32), mb[w][loff:loff + 4 * nb].view(np.float32))
+            assert np.array_equal(ra[w], rb[w])
+        assert np.array_equal(O.tg_layer_decode_accumulate(cfg, off, ma), O.decode_accumulate(cfg, mb))
+
+
+def _tensor_offsets(rng, n, small=True):
+    sizes = []
+    while sum(sizes) < n:
+        sizes.append(int(rng.choice([64, 37, 1000, 2304, 9, 4096])) if small else 4096)
+    off = np.concatenate([[0], np.cumsum(sizes)])
+    off[-1] = n
+    return off[off <= n] if off[-2] < n else np.concatenate([off[off < n], [n]])
+
+
+def test_tg_layer_scales_levels_and_residual():
+    """Each tensor's scale is its largest |v|; every value is sent as -m, 0 or +m of its own
+    tensor, on a side of the value's bracket; the residual keeps v - Q(v)."""
+    rng = np.random.default_rng(42)
+    n, d = 12000, 512
+    off = _tensor_offsets(rng, n)
+    cfg = O.Config(O.TERNGRAD, 3, d, 1, 1, 0.0, 9, n)
+    g = (rng.laplace(0, 1, n) * 10.0 ** rng.uniform(-4, -2, n)).astype(np.float32)
+    for t in range(0, len(off) - 1, 2):  # every other tensor has its largest value last
+        g[off[t + 1] - 1] = np.float32((-1) ** t * 3.0 * np.abs(g[off[t]:off[t + 1]]).max())
+    r0 = (rng.standard_normal(n) * 1e-5).astype(np.float32)
+    r = r0.copy()
+    msg = O.tg_layer_encode(cfg, off, 0, 1, g, r)
+    nseg = len(off) - 1
+    _, _, soff = O.tg_layer_layout(cfg, nseg)
+    scales = msg[soff:soff + 4 * nseg].view(np.float32)
+    v = g + r0
+    q = O.tg_layer_decode_accumulate(cfg, off, [msg])   # one worker: the dequantized values
+    assert np.array_equal(r, v - q)
+    for t in range(nseg):
+        seg = slice(off[t], off[t + 1])
+        m = np.float32(np.abs(v[seg]).max())
+        assert scales[t] == m
+        assert np.all(np.isin(q[seg], np.array([-m, 0.0, m], dtype=np.float32)))
+        lo = np.where(v[seg] >= 0, 0.0, -m)
+        hi = np.where(v[seg] >= 0, m, 0.0)
+        assert np.all((q[seg] == lo) | (q[seg] == hi))
+
+
+def test_tg_layer_unbiased():
+    """Stochastic rounding keeps the expectation: the mean over steps tends to v (3 sigma)."""
+    rng = np.random.default_rng(43)
+    n, d, steps = 600, 128, 400
+    off = [0, 50, 250, 600]
+    cfg = O.Config(O.TERNGRAD, 3, d, 1, 0, 0.0, 3, n)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    qs = np.stack([O.tg_layer_decode_accumulate(cfg, off, [O.tg_layer_encode(cfg, off, 0, t, g)]) for t in range(steps)])
+    v = g.astype(np.float64)
+    m = np.concatenate([np.full(off[t + 1] - off[t], np.abs(v[off[t]:off[t + 1]]).max()) for t in range(3)])
+    var = np.abs(v) * (m - np.abs(v))            # (b - v)(v - a) for the bracket [0, m] or [-m, 0]
+    sure = var <= 1e-9 * m * m                   # at a level (each tensor's largest): no randomness
+    assert np.all(qs[:, sure] == np.float32(v[sure]))
+    z = (qs.mean(axis=0)[~sure] - v[~sure]) / np.sqrt(var[~sure] / steps)
+    assert np.mean(z ** 2) < 1.3
+    assert np.abs(z).max() < 5.5
