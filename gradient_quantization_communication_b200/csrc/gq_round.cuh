@@ -147,7 +147,8 @@ struct RoundPB {
 template <int BITS>
 __device__ __forceinline__ void pack_chunk(const KParams &p, int lane, const int (&code)[4], uint32_t *cw)
 {
-    const int b = BITS > 0 ? BITS : p.bits;  // (BITS < 0 only in never-run instantiations)
+    // (BITS < 0 only in never-run instantiations; BITS == 8 never reaches the shifts below)
+    const int b = BITS > 0 ? (BITS == 8 ? 1 : BITS) : p.bits;
     if (BITS == 8 || (BITS == 0 && b == 8)) {
         // 8-bit codes: lane l's four codes are word l of the chunk
         __stcs(cw + lane, (uint32_t)code[0] | ((uint32_t)code[1] << 8) | ((uint32_t)code[2] << 16) |

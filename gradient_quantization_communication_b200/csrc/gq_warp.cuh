@@ -19,8 +19,7 @@
 //   ORQ             : shared-memory histogram of grid positions with 16 fraction bits (8
 //                     columns per cell, one packed shared atomic per value), exact prefix
 //                     sums, s-2 incremental greedy rounds, per-bracket reciprocal table
-//   BinGrad-b       : histogram-pruned exact split search (gq_bingrad.cuh): only the values of
-//                     the grid cells that can hold the best split are ordered
+//   BinGrad-b       : warp bitonic sort, exact int64 prefix sums, screened argmax of J(k)
 //   BinGrad-pb      : BinGrad-b's levels (as above) bound the pair from inside; shared-memory
 //                     moments of 16-bit positions, exact search of the admissible pairs
 //   QSGD-nearest    : the QSGD levels, rounding to the nearest level (no draws)
@@ -30,7 +29,6 @@
 // plain loads, so the main kernel carries no tail logic.
 #pragma once
 
-#include "gq_bingrad.cuh"
 #include "gq_round.cuh"
 
 namespace gq {
@@ -67,10 +65,13 @@ struct alignas(16) FitQSGD {
     float qr[GQ_MAX_QSGD_LEVELS];     // the level ratios (2k - (s-1)) / (s-1), copied once
 };
 struct alignas(16) FitPB {
-    FitB b;                             // BinGrad-b's split search, run first
     unsigned long long s1[64], s2[64];  // per cell: sum of positions, of squared positions
     unsigned int cnt[64];               // per cell: count
     long long al[64], be[64], ga[64], de[64];
+};
+
+struct alignas(16) FitB {
+    int unused;
 };
 
 template <int S> struct FitFor { using type = FitQSGD; };
@@ -363,8 +364,165 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     __syncwarp();
 }
 
+// Bitonic sort of the 32*EPL keys, position i = lane*EPL + r, ascending, in the form whose
+// comparators all put the minimum at the lower index: each merge of blocks of k keys starts by
+// comparing i with its mirror i ^ (k-1), then i with i ^ j for j = k/4 .. 1.  Inside a lane a
+// compare-exchange is one min and one max; across lanes (partner lane l ^ m) the lower lane keeps
+// the minimum, a choice that depends on the lane only.
+template <int EPL>
+__device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
+{
+    constexpr int N = 32 * EPL;
+#pragma unroll
+    for (int k = 2; k <= N; k <<= 1) {
+        if (k <= EPL) {
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) {
+                const int q = r ^ (k - 1);
+                if (q > r) {
+                    const float a = key[r], b = key[q];
+                    key[r] = fminf(a, b);
+                    key[q] = fmaxf(a, b);
+                }
+            }
+        } else {
+            // partner of (lane, r) is (lane ^ m, EPL-1-r); pairs (r, EPL-1-r) are updated together
+            const int m = k / EPL - 1;
+            const bool take_min = (lane & ((k / EPL) >> 1)) == 0;
+#pragma unroll
+            for (int r = 0; r < EPL / 2; ++r) {
+                const float o1 = __shfl_xor_sync(kFull, key[EPL - 1 - r], m);
+                const float o2 = __shfl_xor_sync(kFull, key[r], m);
+                key[r] = take_min ? fminf(key[r], o1) : fmaxf(key[r], o1);
+                key[EPL - 1 - r] = take_min ? fminf(key[EPL - 1 - r], o2) : fmaxf(key[EPL - 1 - r], o2);
+            }
+        }
+#pragma unroll
+        for (int j = k >> 2; j > 0; j >>= 1) {
+            if (j >= EPL) {
+                const bool take_min = (lane & (j / EPL)) == 0;
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) {
+                    const float o = __shfl_xor_sync(kFull, key[r], j / EPL);
+                    key[r] = take_min ? fminf(key[r], o) : fmaxf(key[r], o);
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) {
+                    if ((r & j) == 0) {
+                        const float a = key[r], b = key[r ^ j];
+                        key[r] = fminf(a, b);
+                        key[r ^ j] = fmaxf(a, b);
+                    }
+                }
+            }
+        }
+    }
+}
+
+// BinGrad-b's levels of the bucket (m = max|u| over the valid values, already reduced): the
+// sorted values' exact fixed-point prefix sums and the screened argmax of J; {a, b, split value,
+// split found}.  Also used by BinGrad-pb, whose levels must be at least as far apart.
+template <int EPL, bool TAIL>
+__device__ __forceinline__ RoundB bingrad_b_levels(int lane, uint32_t vmask, int nvalid, float m, const float (&u)[EPL])
+{
+    RoundB rule{0.0f, 0.0f, 0.0f, false};
+    if (!(m > 0.0f)) return rule;
+    float key[EPL];
+#pragma unroll
+    for (int t = 0; t < EPL; ++t) key[t] = (!TAIL || ((vmask >> t) & 1u)) ? u[t] : INFINITY;
+    warp_bitonic_sort<EPL>(key, lane);
+    const int e = 46 - fexpo(m);
+    // fixed point round(x * 2^e) in binary32: the scaling by 2^e (as 2^(e/2) * 2^(e - e/2),
+    // both representable for e in [-81, 195]) is exact, except for products that fall below
+    // 2^-126, which round to 0 either way
+    const float s1 = pow2f(e >> 1), s2 = pow2f(e - (e >> 1));
+    // inclusive prefix of the fixed-point values inside the lane, then across lanes
+    long long pre[EPL];
+    long long run = 0;
+#pragma unroll
+    for (int r = 0; r < EPL; ++r) {
+        const int i = lane * EPL + r;
+        run += (!TAIL || i < nvalid) ? __float2ll_rn(__fmul_rn(__fmul_rn(key[r], s1), s2)) : 0ll;
+        pre[r] = run;
+    }
+    const long long incl = warp_inclusive_scan(run, lane);
+    const long long lane_excl = incl - run;
+    const long long total = __shfl_sync(kFull, incl, 31);
+    const float prev_last = __shfl_up_sync(kFull, key[EPL - 1], 1);
+    // Screening: a binary32 estimate of J for every admissible split (two conversions of
+    // exact integers, two squares, two reciprocals within 1 ulp, two products and a sum:
+    // within 8 * 2^-24 of J), then the fp64 J only for the splits whose estimate reaches
+    // M (1 - 2^-18), M the largest estimate: every split whose fp64 J is the largest is
+    // among them, so the choice (ties to the smallest split) is the exhaustive one.
+    float est[EPL];
+    float emax = 0.0f;
+#pragma unroll
+    for (int r = 0; r < EPL; ++r) {
+        const int i = lane * EPL + r;  // split: positions < i on the left
+        const float prev = r > 0 ? key[r - 1] : prev_last;
+        est[r] = -1.0f;
+        if (i >= 1 && i < nvalid && prev < key[r]) {
+            const long long Sl = lane_excl + (r > 0 ? pre[r - 1] : 0ll);
+            const float l = __ll2float_rn(Sl), rr = __ll2float_rn(total - Sl);
+            est[r] = __fadd_rn(__fmul_rn(__fmul_rn(l, l), rcp_approx((float)i)),
+                               __fmul_rn(__fmul_rn(rr, rr), rcp_approx((float)(nvalid - i))));
+            emax = fmaxf(emax, est[r]);
+        }
+    }
+    // the estimates are >= +0, so their bit patterns order like unsigned integers
+    const float thr = __fmul_rn(__uint_as_float(__reduce_max_sync(kFull, __float_as_uint(emax))), 1.0f - 0x1p-18f);
+    double best_j = -1.0;
+    int best_i = 0x7fffffff;
+#pragma unroll
+    for (int r = 0; r < EPL; ++r) {
+        if (est[r] >= thr) {
+            const int i = lane * EPL + r;
+            const long long Sl = lane_excl + (r > 0 ? pre[r - 1] : 0ll);
+            const double l = __ll2double_rn(Sl);
+            const double rr = __ll2double_rn(total - Sl);
+            const double J = __dadd_rn(__ddiv_rn(__dmul_rn(l, l), (double)i),
+                                       __ddiv_rn(__dmul_rn(rr, rr), (double)(nvalid - i)));
+            if (J > best_j) {
+                best_j = J;
+                best_i = i;
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double oj = __shfl_xor_sync(kFull, best_j, o);
+        const int oi = __shfl_xor_sync(kFull, best_i, o);
+        if (oj > best_j || (oj == best_j && oi < best_i)) {
+            best_j = oj;
+            best_i = oi;
+        }
+    }
+    if (best_i == 0x7fffffff) {
+        // every value equal: a single level, code 0
+        const float v0 = __fadd_rn(__shfl_sync(kFull, key[0], 0), 0.0f);
+        return RoundB{v0, v0, v0, false};
+    }
+    // owner lane publishes the threshold value and the left sum
+    float tv = 0.0f;
+    long long sl = 0;
+#pragma unroll
+    for (int r = 0; r < EPL; ++r)
+        if (lane * EPL + r == best_i) {
+            tv = key[r];
+            sl = lane_excl + (r > 0 ? pre[r - 1] : 0ll);
+        }
+    const int owner = best_i / EPL;
+    tv = __shfl_sync(kFull, tv, owner);
+    sl = __shfl_sync(kFull, sl, owner);
+    const double inv_sc = pow2d(-e);
+    const float a = __double2float_rn(__dmul_rn(__ddiv_rn(__ll2double_rn(sl), (double)best_i), inv_sc));
+    const float b = __double2float_rn(__dmul_rn(__ddiv_rn(__ll2double_rn(total - sl), (double)(nvalid - best_i)), inv_sc));
+    return RoundB{a, b, tv, true};
+}
+
 template <int EPL, bool FUSED, bool TAIL, int BITS, int IO = 0>
-__device__ void fit_bingrad_b(const KParams &p, FitB &sm, int64_t beta, int w, int lane, uint32_t vmask, bool check,
+__device__ void fit_bingrad_b(const KParams &p, FitB &, int64_t beta, int w, int lane, uint32_t vmask, bool check,
                               int nvalid, const float (&v)[EPL], const float (&u)[EPL], float (&acc)[EPL], ErrAcc *ea = nullptr)
 {
     float m = 0.0f;
@@ -376,9 +534,7 @@ __device__ void fit_bingrad_b(const KParams &p, FitB &sm, int64_t beta, int w, i
     int pos[EPL];
 #pragma unroll
     for (int t = 0; t < EPL; ++t) pos[t] = 0;
-    RoundB rule{0.0f, 0.0f, 0.0f, false};
-    if (m > 0.0f)
-        rule = bingrad_b_pruned<EPL, TAIL>(sm, lane, vmask, nvalid, m, u);
+    const RoundB rule = bingrad_b_levels<EPL, TAIL>(lane, vmask, nvalid, m, u);
     emit<EPL, FUSED, false, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
     store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
 }
@@ -417,8 +573,7 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
     // B >= Bmin, the smallest whose point is >= b_b (63 if none)
     int Amax, Bmin;
     {
-        const float m = fmaxf(fabsf(mn), fabsf(mx));
-        const RoundB bl = bingrad_b_pruned<EPL, TAIL>(sm.b, lane, vmask, nvalid, m, u);
+        const RoundB bl = bingrad_b_levels<EPL, TAIL>(lane, vmask, nvalid, fmaxf(fabsf(mn), fabsf(mx)), u);
         const float g0 = grid_point(mn, mx, step, lane), g1 = grid_point(mn, mx, step, lane + 32);
         const unsigned long long le = (unsigned long long)__ballot_sync(kFull, g0 <= bl.a) |
                                       ((unsigned long long)__ballot_sync(kFull, g1 <= bl.a) << 32);
@@ -608,11 +763,10 @@ __device__ __forceinline__ void init_fit(const KParams &p, Fit &fit, int lane)
     if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD || SCHEME == GQ_QSGD_NEAREST || SCHEME == GQ_QSGD_L2) {
         for (int k = lane; k < p.s; k += 32) fit.qr[k] = p.qratio[k];
     }
-    if constexpr (SCHEME == GQ_ORQ || SCHEME == GQ_BINGRAD_B) {
+    if constexpr (SCHEME == GQ_ORQ) {
         for (int i = lane; i < 64 * kHistCols; i += 32) fit.hist[i] = 0u;
     }
     if constexpr (SCHEME == GQ_BINGRAD_PB) {
-        for (int i = lane; i < 64 * kHistCols; i += 32) fit.b.hist[i] = 0u;
         for (int i = lane; i < 64; i += 32) {
             fit.cnt[i] = 0u;
             fit.s1[i] = 0ull;
