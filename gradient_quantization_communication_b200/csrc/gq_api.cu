@@ -20,6 +20,9 @@ struct gq_plan {
     int device;
     unsigned int *status;  // device word
     double *err_scratch;   // gq_quant_error: per-bucket sums and first-pass rows
+    int64_t *seg_off;      // GQ_TERNGRAD_LAYER: the tensors' offsets (device), NULL until set
+    int nseg;
+    unsigned int *seg_max; // GQ_TERNGRAD_LAYER: W x nseg scales (device scratch)
 };
 
 namespace {
@@ -66,6 +69,10 @@ gq_status_t normalise(const gq_config_t *in, gq_config_t *out)
         if (c.levels == 0) c.levels = 2;
         if (c.levels != 2) return GQ_ERR_INVALID;
         break;
+    case GQ_TERNGRAD_LAYER:
+        if (c.levels == 0) c.levels = 3;
+        if (c.levels != 3) return GQ_ERR_INVALID;
+        break;
     default: return GQ_ERR_INVALID;
     }
     if (c.bucket < GQ_MIN_BUCKET || c.bucket > GQ_MAX_BUCKET || (c.bucket & (c.bucket - 1)) != 0) return GQ_ERR_INVALID;
@@ -76,6 +83,7 @@ gq_status_t normalise(const gq_config_t *in, gq_config_t *out)
     // the biased baselines are built for the register path only
     if ((c.scheme == GQ_QSGD_NEAREST || c.scheme == GQ_SIGNSGD || c.scheme == GQ_QSGD_L2) && c.bucket > 512)
         return GQ_ERR_UNSUPPORTED;
+    if (c.scheme == GQ_TERNGRAD_LAYER && c.clip_sigma > 0.0f) return GQ_ERR_UNSUPPORTED;
     *out = c;
     return GQ_OK;
 }
@@ -121,6 +129,9 @@ gq::KParams base_params(const gq_plan &pl, uint64_t step)
     p.codes_words = (int64_t)pl.cfg.bucket * pl.bits / 32;
     p.levels_off = (int64_t)pl.levels_off;
     p.status = pl.status;
+    p.seg_off = pl.seg_off;
+    p.nseg = pl.nseg;
+    p.seg_max = pl.seg_max;
     return p;
 }
 
@@ -155,6 +166,7 @@ gq_status_t gq_message_layout(const gq_config_t *cfg, size_t *bytes, size_t *cod
     gq_config_t c;
     const gq_status_t st = normalise(cfg, &c);
     if (st != GQ_OK) return st;
+    if (c.scheme == GQ_TERNGRAD_LAYER) return GQ_ERR_UNSUPPORTED;  // sized by the tensors: gq_plan_message_layout
     layout(c, bytes, codes_off, levels_off);
     return GQ_OK;
 }
@@ -176,6 +188,10 @@ gq_status_t gq_plan_create(const gq_config_t *cfg, gq_plan_t *out)
     layout(c, &pl->msg_bytes, &pl->codes_off, &pl->levels_off);
     pl->status = nullptr;
     pl->err_scratch = nullptr;
+    pl->seg_off = nullptr;
+    pl->nseg = 0;
+    pl->seg_max = nullptr;
+    if (c.scheme == GQ_TERNGRAD_LAYER) pl->msg_bytes = pl->codes_off = pl->levels_off = 0;  // until the segments
     const size_t err_bytes = (size_t)gq::err_scratch_doubles(pl->nb) * sizeof(double);
     if (cudaGetDevice(&pl->device) != cudaSuccess || cudaMalloc(&pl->status, sizeof(unsigned int)) != cudaSuccess ||
         cudaMemset(pl->status, 0, sizeof(unsigned int)) != cudaSuccess ||
@@ -197,8 +213,31 @@ gq_status_t gq_plan_destroy(gq_plan_t plan)
         const cudaError_t e2 = cudaFree(plan->err_scratch);
         if (e == cudaSuccess) e = e2;
     }
+    if (plan->seg_off) {
+        const cudaError_t e2 = cudaFree(plan->seg_off);
+        if (e == cudaSuccess) e = e2;
+    }
+    if (plan->seg_max) {
+        const cudaError_t e2 = cudaFree(plan->seg_max);
+        if (e == cudaSuccess) e = e2;
+    }
     delete plan;
     return from_cuda(e);
+}
+
+// Buckets above 512: the group kernels take the full buckets of ORQ and QSGD / TernGrad without
+// clipping (the CTA kernel the ragged last one); everything else goes to the CTA kernel.
+static cudaError_t launch_large(const gq::KParams &p, bool fused, cudaStream_t s)
+{
+    const bool group = p.clip == 0.0f && (p.scheme == GQ_ORQ || p.scheme == GQ_QSGD || p.scheme == GQ_TERNGRAD);
+    if (!group) return gq::launch_cta_encode(p, s);
+    const int64_t nfull = p.tail == p.d ? p.nb : p.nb - 1;
+    if (nfull > 0) {
+        const cudaError_t e = p.scheme == GQ_ORQ ? gq::launch_group_orq(p, nfull, fused, s)
+                                                 : gq::launch_group_qsgd(p, nfull, fused, s);
+        if (e != cudaSuccess) return e;
+    }
+    return nfull < p.nb ? gq::launch_cta_encode(p, s, nfull) : cudaSuccess;
 }
 
 gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, float *residual, void *msg,
@@ -210,6 +249,7 @@ gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const floa
     if (!grad || !msg || !aligned16(grad) || !aligned16(msg)) return GQ_ERR_INVALID;
     if ((plan->cfg.error_feedback != 0) != (residual != nullptr)) return GQ_ERR_INVALID;
     if (residual && !aligned16(residual)) return GQ_ERR_INVALID;
+    if (plan->cfg.scheme == GQ_TERNGRAD_LAYER && !plan->seg_off) return GQ_ERR_INVALID;
     gq_status_t st = check_device(*plan);
     if (st != GQ_OK) return st;
     gq::KParams p = base_params(*plan, step);
@@ -218,8 +258,9 @@ gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const floa
     p.r[0] = residual;
     p.msg[0] = static_cast<unsigned char *>(msg);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (plan->cfg.scheme == GQ_TERNGRAD_LAYER) return from_cuda(gq::launch_layer_encode(p, s));
     if (plan->cfg.bucket <= 512) return from_cuda(gq::launch_warp_encode(p, false, s));
-    return from_cuda(gq::launch_cta_encode(p, s));
+    return from_cuda(launch_large(p, false, s));
 }
 
 gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs, int nmsgs, float *avg, void *stream)
@@ -230,6 +271,7 @@ gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs, int nm
     if (!msgs || !avg || !aligned16(avg)) return GQ_ERR_INVALID;
     for (int w = 0; w < nmsgs; ++w)
         if (!msgs[w] || !aligned16(msgs[w])) return GQ_ERR_INVALID;
+    if (plan->cfg.scheme == GQ_TERNGRAD_LAYER && !plan->seg_off) return GQ_ERR_INVALID;
     gq_status_t st = check_device(*plan);
     if (st != GQ_OK) return st;
     gq::KParams p = base_params(*plan, 0);
@@ -237,6 +279,7 @@ gq_status_t gq_decode_accumulate(gq_plan_t plan, const void *const *msgs, int nm
     p.inv_w = 1.0f / (float)nmsgs;
     for (int w = 0; w < nmsgs; ++w) p.msg[w] = static_cast<unsigned char *>(const_cast<void *>(msgs[w]));
     p.avg = avg;
+    if (plan->cfg.scheme == GQ_TERNGRAD_LAYER) return from_cuda(gq::launch_layer_decode(p, static_cast<cudaStream_t>(stream)));
     return from_cuda(gq::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -255,6 +298,7 @@ gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *gra
         if (ef && (!residuals[w] || !aligned16(residuals[w]))) return GQ_ERR_INVALID;
         if (msgs && (!msgs[w] || !aligned16(msgs[w]))) return GQ_ERR_INVALID;
     }
+    if (plan->cfg.scheme == GQ_TERNGRAD_LAYER && !plan->seg_off) return GQ_ERR_INVALID;
     gq_status_t st = check_device(*plan);
     if (st != GQ_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -267,8 +311,9 @@ gq_status_t gq_fused_step(gq_plan_t plan, uint64_t step, const float *const *gra
         p.msg[w] = msgs ? static_cast<unsigned char *>(msgs[w]) : nullptr;
     }
     p.avg = avg;
+    if (plan->cfg.scheme == GQ_TERNGRAD_LAYER) return from_cuda(gq::launch_layer_encode(p, s));
     if (plan->cfg.bucket <= 512) return from_cuda(gq::launch_warp_encode(p, true, s));
-    return from_cuda(gq::launch_cta_encode(p, s));
+    return from_cuda(launch_large(p, true, s));
 }
 
 gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, const float *residual,
@@ -276,6 +321,7 @@ gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step, const
 {
     Range range("gq_quant_error");
     if (!plan || !out) return GQ_ERR_INVALID;
+    if (plan->cfg.scheme == GQ_TERNGRAD_LAYER) return GQ_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (plan->cfg.n == 0) return from_cuda(cudaMemsetAsync(out, 0, 3 * sizeof(double), s));
     if (!grad || !aligned16(grad)) return GQ_ERR_INVALID;
@@ -291,6 +337,47 @@ gq_status_t gq_quant_error(gq_plan_t plan, uint32_t worker, uint64_t step, const
     cudaError_t e = plan->cfg.bucket <= 512 ? gq::launch_warp_err(p, part, s) : gq::launch_cta_err(p, part, s);
     if (e != cudaSuccess) return GQ_ERR_CUDA;
     return from_cuda(gq::launch_err_reduce(part, plan->nb, part + 3 * plan->nb, out, s));
+}
+
+gq_status_t gq_plan_set_segments(gq_plan_t plan, const int64_t *offsets, int nseg)
+{
+    if (!plan || !offsets || nseg < 1 || plan->cfg.scheme != GQ_TERNGRAD_LAYER) return GQ_ERR_INVALID;
+    if (offsets[0] != 0 || offsets[nseg] != plan->cfg.n) return GQ_ERR_INVALID;
+    for (int t = 0; t < nseg; ++t)
+        if (offsets[t + 1] < offsets[t]) return GQ_ERR_INVALID;
+    const gq_status_t st = check_device(*plan);
+    if (st != GQ_OK) return st;
+    if (plan->seg_off) cudaFree(plan->seg_off);
+    if (plan->seg_max) cudaFree(plan->seg_max);
+    plan->seg_off = nullptr;
+    plan->seg_max = nullptr;
+    plan->nseg = 0;
+    if (cudaMalloc(&plan->seg_off, sizeof(int64_t) * (size_t)(nseg + 1)) != cudaSuccess ||
+        cudaMalloc(&plan->seg_max, sizeof(unsigned int) * (size_t)nseg * plan->cfg.workers) != cudaSuccess ||
+        cudaMemcpy(plan->seg_off, offsets, sizeof(int64_t) * (size_t)(nseg + 1), cudaMemcpyHostToDevice) != cudaSuccess) {
+        if (plan->seg_off) cudaFree(plan->seg_off);
+        if (plan->seg_max) cudaFree(plan->seg_max);
+        plan->seg_off = nullptr;
+        plan->seg_max = nullptr;
+        return GQ_ERR_CUDA;
+    }
+    plan->nseg = nseg;
+    const int64_t cbytes = (plan->nb * (int64_t)plan->cfg.bucket * 2 / 8 + 15) / 16 * 16;
+    const int64_t sbytes = ((int64_t)nseg * 4 + 15) / 16 * 16;
+    plan->codes_off = 0;
+    plan->levels_off = (size_t)cbytes;
+    plan->msg_bytes = (size_t)(cbytes + sbytes);
+    return GQ_OK;
+}
+
+gq_status_t gq_plan_message_layout(gq_plan_t plan, size_t *bytes, size_t *codes_off, size_t *levels_off)
+{
+    if (!plan) return GQ_ERR_INVALID;
+    if (plan->cfg.scheme == GQ_TERNGRAD_LAYER && !plan->seg_off) return GQ_ERR_INVALID;
+    if (bytes) *bytes = plan->msg_bytes;
+    if (codes_off) *codes_off = plan->codes_off;
+    if (levels_off) *levels_off = plan->levels_off;
+    return GQ_OK;
 }
 
 gq_status_t gq_selftest_bounded_wait(gq_plan_t plan, int64_t limit_ns, void *stream)

@@ -206,6 +206,7 @@ gq_status_t layouts(const gq_config_t *cfg, Layouts *out)
     c.workers = 1;  // ignored here
     const gq_status_t st = gq_config_check(&c);
     if (st != GQ_OK) return st;
+    if (c.scheme == GQ_TERNGRAD_LAYER) return GQ_ERR_UNSUPPORTED;  // its message holds per-tensor scales
     if (c.scheme == GQ_TERNGRAD && c.levels == 0) c.levels = 3;
     if ((c.scheme == GQ_BINGRAD_B || c.scheme == GQ_BINGRAD_PB || c.scheme == GQ_SIGNSGD) && c.levels == 0)
         c.levels = 2;

@@ -1,0 +1,11 @@
+// gq_group_orq.cu -- instantiation of the group kernels for GQ_ORQ.
+#include "gq_group.cuh"
+
+namespace gq {
+
+cudaError_t launch_group_orq(const KParams &p, int64_t nfull, bool fused, cudaStream_t stream)
+{
+    return fused ? launch_group_fused<GQ_ORQ, true>(p, nfull, stream) : launch_group_fused<GQ_ORQ, false>(p, nfull, stream);
+}
+
+}  // namespace gq

@@ -36,6 +36,9 @@ struct KParams {
     unsigned char *msg[GQ_MAX_WORKERS];// NULL: do not write the message
     float *avg;                        // fused kernels only
     unsigned int *status;              // plan status word
+    const int64_t *seg_off;            // GQ_TERNGRAD_LAYER: nseg + 1 tensor offsets (device)
+    int nseg;
+    unsigned int *seg_max;             // GQ_TERNGRAD_LAYER: W x nseg scales (float bits, device scratch)
 };
 
 // Status bits raised by kernels.
@@ -48,9 +51,17 @@ constexpr unsigned kStatusTimeout = 2u;  // a bounded wait on a bulk copy gave u
 cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream);
 // Shared-memory path (d = 1024 .. 32768): one CTA per bucket index walking the p.W workers;
 // with p.avg set, the average of the dequantized values is accumulated on chip and written.
-cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream);
+cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream, int64_t first = 0);
+// d = 1024 .. 32768, ORQ or QSGD / TernGrad, no clipping: full buckets 0 .. nfull-1 spread over
+// groups of d / 512 warps (gq_group.cuh).
+cudaError_t launch_group_orq(const KParams &p, int64_t nfull, bool fused, cudaStream_t stream);
+cudaError_t launch_group_qsgd(const KParams &p, int64_t nfull, bool fused, cudaStream_t stream);
 // Dequantize + aggregate for any d.
 cudaError_t launch_decode(const KParams &p, cudaStream_t stream);
+// GQ_TERNGRAD_LAYER: the tensors' scales (into p.seg_max), then the encode of p.W workers (the
+// average too when p.avg is set); and the decode + average of p.W messages.
+cudaError_t launch_layer_encode(const KParams &p, cudaStream_t stream);
+cudaError_t launch_layer_decode(const KParams &p, cudaStream_t stream);
 
 // gq_quant_error: per-bucket binary64 error sums into part[3 * bucket + k] (one worker, nothing
 // else written), then their fixed-order reduction into out[3].  The scratch holds

@@ -55,7 +55,8 @@ typedef enum {
     GQ_QSGD = 0,       /* s uniform levels on [-m, m], m = max|u| of the bucket, stochastic rounding */
     GQ_TERNGRAD = 1,   /* QSGD with s = 3: levels {-m, 0, m} */
     GQ_BINGRAD_B = 2,  /* two levels at the side means of the SSE-optimal split, deterministic */
-    GQ_BINGRAD_PB = 3, /* two grid levels minimising expected squared error; stochastic inside, clamped outside */
+    GQ_BINGRAD_PB = 3, /* two grid levels at least as far apart as BinGrad-b's, minimising the expected squared
+                        * error among such pairs; stochastic inside, clamped outside */
     GQ_ORQ = 4,        /* s levels: {min, max} plus s-2 greedy picks from a 64-point grid, stochastic rounding */
     /* Biased baselines ("Gradient Quantization" glossary, "Deterministic vs stochastic rounding"
      * and "Ternary and binary quantization"); buckets of d <= 512 only: */
@@ -64,8 +65,11 @@ typedef enum {
     GQ_SIGNSGD = 6,      /* scaled sign: levels -m1 and +m1, m1 = mean |u| of the bucket (exact fixed-point
                           * sum), code 1 for u >= 0; 1 bit per element */
     /* QSGD as published (l2 scaling; the glossary's QSGD, whose codes are Elias-coded), d <= 512: */
-    GQ_QSGD_L2 = 7       /* the QSGD-s levels and stochastic rounding with m = ||u||_2 of the bucket (exact
+    GQ_QSGD_L2 = 7,      /* the QSGD-s levels and stochastic rounding with m = ||u||_2 of the bucket (exact
                           * fixed-point sum of squares) in place of max |u|; sparse codes for gq_elias_pack */
+    /* TernGrad with one scale per parameter tensor (the glossary's "single scaling factor per
+     * layer"); needs the tensors' offsets (gq_plan_set_segments); no clipping: */
+    GQ_TERNGRAD_LAYER = 8
 } gq_scheme_t;
 
 typedef enum {
@@ -286,6 +290,29 @@ GQ_API gq_status_t gq_elias_used_bytes(const gq_config_t *cfg, uint64_t stream_b
  */
 GQ_API gq_status_t gq_elias_pack(const gq_config_t *cfg, const void *msg, void *emsg, void *stream);
 GQ_API gq_status_t gq_elias_unpack(const gq_config_t *cfg, const void *emsg, void *msg, void *stream);
+
+/*
+ * TernGrad with one scale per parameter tensor (scheme GQ_TERNGRAD_LAYER, 3 levels).  The
+ * glossary "Gradient Quantization" (section Ternary and binary quantization) gives TernGrad a
+ * single scaling factor per layer; here the gradient is the concatenation of nseg tensors,
+ * tensor t holding elements [offsets[t], offsets[t+1]).  Per worker m_t = max |v| over tensor t
+ * (v = g + r), and each element is rounded between the two of {-m_t, 0, +m_t} around it exactly
+ * as GQ_TERNGRAD rounds it (same position, probability and Philox draw).
+ * Message: the 2-bit codes in the layout of the dense message (bucket after bucket), then the
+ * nseg scales (float32); both regions 16-byte aligned.  gq_message_layout cannot size it (it
+ * depends on nseg): use gq_plan_message_layout.
+ *
+ * gq_plan_set_segments: offsets is a HOST array of nseg + 1 non-decreasing offsets with
+ * offsets[0] = 0 and offsets[nseg] = n (empty tensors allowed); the plan copies it to device
+ * memory it owns (this call allocates, like gq_plan_create; a second call replaces the first).
+ * GQ_ERR_INVALID for another scheme or bad offsets.  gq_encode, gq_decode_accumulate and
+ * gq_fused_step on such a plan return GQ_ERR_INVALID until the segments are set; gq_quant_error
+ * returns GQ_ERR_UNSUPPORTED.
+ * gq_plan_message_layout: the plan's message size and region offsets (any scheme; for
+ * GQ_TERNGRAD_LAYER once the segments are set).
+ */
+GQ_API gq_status_t gq_plan_set_segments(gq_plan_t plan, const int64_t *offsets, int nseg);
+GQ_API gq_status_t gq_plan_message_layout(gq_plan_t plan, size_t *bytes, size_t *codes_off, size_t *levels_off);
 
 /* Synchronize `stream`, then report and clear the plan's status flags: GQ_ERR_TIMEOUT if a
  * kernel's bounded wait for a bulk copy gave up (the kernel then stopped early; its outputs are

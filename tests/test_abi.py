@@ -53,7 +53,10 @@ def test_version_and_status_strings():
     (dict(scheme="terngrad", levels=5), False),
     (dict(scheme="bingrad_b", levels=0), True),
     (dict(scheme="bingrad_pb", levels=3), False),
-    (dict(scheme=8, levels=3), False),
+    (dict(scheme=9, levels=3), False),
+    (dict(scheme="terngrad_layer", levels=3), True),
+    (dict(scheme="terngrad_layer", levels=0), True),
+    (dict(scheme="terngrad_layer", levels=5), False),
     (dict(scheme="orq", levels=5, bucket=64), False),
     (dict(scheme="orq", levels=5, bucket=384), False),
     (dict(scheme="orq", levels=5, bucket=65536), False),
@@ -165,6 +168,18 @@ def test_biased_layout_matches_oracle(scheme, levels, d, n):
     mine = G.gq_message_layout(G.gq_config(scheme, levels, d, 1, True, 0.0, 0, n))
     ref = O.message_layout(O.Config(scheme, levels or 2, d, 1, 1, 0.0, 0, n))
     assert mine == ref
+
+
+def test_terngrad_layer_host_checks():
+    """Per-tensor TernGrad: no clipping; its message is sized by the tensors, so the
+    configuration-only layouts (dense, base-s, Elias) refuse it."""
+    cfg = G.gq_config("terngrad_layer", 3, 512, 2, True, 0.0, 0, 1000)
+    assert G.gq_config_check(cfg) == G.GQ_OK
+    assert G.gq_config_check(G.gq_config("terngrad_layer", 3, 512, 2, True, 2.5, 0, 1000)) == G.GQ_ERR_UNSUPPORTED
+    for call in (lambda: G.gq_message_layout(cfg), lambda: G.gq_entropy_layout(cfg), lambda: G.gq_elias_layout(cfg)):
+        with pytest.raises(G.GQError) as ei:
+            call()
+        assert ei.value.status == G.GQ_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("kw,status", [

@@ -34,7 +34,10 @@ MUTATIONS = [
     ("bingrad_pb_inner_term", "else e += (__int128)(b - x) * (x - a);", "else e += (__int128)(b - x) * (b - x);"),
     ("clip_mean", "double var = (double)sxx / (double)n - mean * mean;", "double var = (double)sxx / (double)n;"),
     ("grid_step", "gi->step = range / 63.0f;", "gi->step = range / 64.0f;"),
-    ("average_scale", "float inv_w = 1.0f / (float)nmsgs;", "float inv_w = 1.0f / (float)(nmsgs + 1);"),
+    ("average_scale", "or_message_layout(cfg, &bytes, &coff, &loff);\n    float inv_w = 1.0f / (float)nmsgs;",
+     "or_message_layout(cfg, &bytes, &coff, &loff);\n    float inv_w = 1.0f / (float)(nmsgs + 1);"),
+    ("tg_layer_average_scale", "int64_t words = (int64_t)d * 2 / 32;\n    float inv_w = 1.0f / (float)nmsgs;",
+     "int64_t words = (int64_t)d * 2 / 32;\n    float inv_w = 1.0f / (float)(nmsgs + 1);"),
     ("residual_sign", "r[base + i] = v[i] - q[i];", "r[base + i] = q[i] - v[i];"),
     ("uniform_bits", "if (len > 24) word &= ~((1u << (len - 24)) - 1u);", "if (len > 23) word &= ~((1u << (len - 23)) - 1u);"),
     ("pack_padding", "memset(words, 0, sizeof(uint32_t) * (size_t)(d * b / 32));",
