@@ -225,19 +225,13 @@ gq_status_t gq_plan_destroy(gq_plan_t plan)
     return from_cuda(e);
 }
 
-// Buckets above 512: the group kernels take the full buckets of ORQ and QSGD / TernGrad without
-// clipping (the CTA kernel the ragged last one); everything else goes to the CTA kernel.
+// Buckets above 512: the group kernels take ORQ and QSGD / TernGrad without clipping; everything
+// else goes to the CTA kernel.
 static cudaError_t launch_large(const gq::KParams &p, bool fused, cudaStream_t s)
 {
     const bool group = p.clip == 0.0f && (p.scheme == GQ_ORQ || p.scheme == GQ_QSGD || p.scheme == GQ_TERNGRAD);
     if (!group) return gq::launch_cta_encode(p, s);
-    const int64_t nfull = p.tail == p.d ? p.nb : p.nb - 1;
-    if (nfull > 0) {
-        const cudaError_t e = p.scheme == GQ_ORQ ? gq::launch_group_orq(p, nfull, fused, s)
-                                                 : gq::launch_group_qsgd(p, nfull, fused, s);
-        if (e != cudaSuccess) return e;
-    }
-    return nfull < p.nb ? gq::launch_cta_encode(p, s, nfull) : cudaSuccess;
+    return p.scheme == GQ_ORQ ? gq::launch_group_orq(p, fused, s) : gq::launch_group_qsgd(p, fused, s);
 }
 
 gq_status_t gq_encode(gq_plan_t plan, uint32_t worker, uint64_t step, const float *grad, float *residual, void *msg,

@@ -11,9 +11,9 @@
 // Only what the fit needs crosses warps:
 //   QSGD / TernGrad : each warp's max |u| -> the group's max (one exchange);
 //   ORQ             : each warp's min and max -> the group's; then each warp's 64 cell counts
-//                     and sums of 16-bit grid positions -> the group's histogram.  Every warp
-//                     runs the same greedy on the same prefix sums and builds the same tables,
-//                     so no result has to be broadcast.
+//                     and sums of 16-bit grid positions -> the group's histogram, from which
+//                     the group's first warp (in a cluster, every CTA's first warp, on the same
+//                     totals) runs the greedy and builds the bracket table the others read.
 // Warp k of a group rounds elements 512k .. 512k+511 of the bucket, so it writes the codes,
 // residual and fused sum of a 512-element slice at the same global index with the per-element
 // rules, Philox counters and dense code layout of the other paths (the launcher passes
@@ -22,10 +22,13 @@
 // Each warp stages its slice of the next item with a 1-D bulk copy while it works on the
 // current one (as the register path does).  Every exchange slot is double-buffered by item
 // parity: a slot is rewritten two items later, after a barrier that every reader of its
-// previous contents has passed.  A copy that does not complete within the wait limit is
-// reported at the next exchange; the whole group then stops at the same point (after a last
-// cluster barrier, so that no CTA leaves while a peer may still read its shared memory).
-// The last bucket, when ragged, is quantized by the CTA path.
+// previous contents has passed.  Across CTAs the threads that wrote a slot fence it at cluster
+// scope and every thread then arrives at the cluster barrier without a release of its own.  A
+// copy that does not complete within the wait limit is reported at the next exchange; the whole
+// group then stops at the same point (after a last cluster barrier, so that no CTA leaves while
+// a peer may still read its shared memory).
+// The ragged last bucket is a second launch of the same kernel (TAIL): one group, guarded
+// plain loads, the invalid slots masked out of the statistics and the stores.
 #pragma once
 
 #include "gq_warp.cuh"
@@ -62,8 +65,6 @@ struct alignas(16) GroupXchg {
     uint4 cells[2][kGroupWarps][32];        // per warp and lane l: counts and position sums of cells 2l, 2l+1
     unsigned long long cta_s[2][32][2];     // clusters: the CTA's sums of cells 2l, 2l+1
     unsigned int cta_c[2][32][2];           // clusters: the CTA's counts
-    unsigned long long tot_s[2][32][2];     // clusters: the group's sums
-    unsigned int tot_c[2][32][2];           // clusters: the group's counts
 };
 
 // --- barriers and distributed shared memory ----------------------------------------------------
@@ -75,6 +76,13 @@ __device__ __forceinline__ void cluster_bar()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// Cluster barrier whose arrival orders nothing: the threads that wrote exchange slots fenced
+// them first (fence_cluster), the wait acquires.
+__device__ __forceinline__ void cluster_bar_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 // Address of the same shared-memory object in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t peer_addr(const void *p, uint32_t rank)
 {
@@ -137,8 +145,9 @@ __device__ __forceinline__ void group_orq_tables(const KParams &p, FitGroupORQ &
     __syncwarp();
 }
 
-template <int SCHEME, int G, bool FUSED>
-__global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_constant__ KParams p, int64_t nfull)
+// Buckets b0 .. b1-1 (TAIL: the ragged last bucket alone, b0 = nb - 1, b1 = nb).
+template <int SCHEME, int G, bool FUSED, bool TAIL>
+__global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_constant__ KParams p, int64_t b0, int64_t b1)
 {
     constexpr int C = G > kGroupWarps ? G / kGroupWarps : 1;    // CTAs per bucket
     constexpr int GPC = G < kGroupWarps ? kGroupWarps / G : 1;  // groups per CTA
@@ -153,13 +162,20 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
     const int gid = C > 1 ? 0 : wib / G;                                         // group within the CTA
     const uint32_t crank = C > 1 ? (uint32_t)(blockIdx.x % C) : 0u;             // CTA within the cluster
     const int rk = C > 1 ? (int)crank * kGroupWarps + wib : wib % G;           // warp within the group
-    const int64_t first = C > 1 ? (int64_t)(blockIdx.x / C) : (int64_t)blockIdx.x * GPC + gid;
+    const int64_t first = b0 + (C > 1 ? (int64_t)(blockIdx.x / C) : (int64_t)blockIdx.x * GPC + gid);
     const int64_t stride = C > 1 ? (int64_t)(gridDim.x / C) : (int64_t)gridDim.x * GPC;
     // the group's first exchange: named barrier of its warps, or the cluster's barrier
     auto sync_group = [&]() {
-        if constexpr (C > 1) cluster_bar();
+        if constexpr (C > 1) cluster_bar_relaxed();
         else named_bar(1 + gid, 32 * G);
     };
+    // TAIL: the valid slots of the warp's slice
+    uint32_t vmask = 0xffffffffu;
+    if constexpr (TAIL) {
+        vmask = 0u;
+#pragma unroll
+        for (int t = 0; t < EPL; ++t) vmask |= (rk * (32 * EPL) + slot_elem(t, lane) < p.tail ? 1u : 0u) << t;
+    }
 
     init_fit<SCHEME>(p, sm.fit, lane);
     if (lane == 0) {
@@ -167,9 +183,9 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
         fence_barrier_init();
     }
     __syncwarp();
-    if (first >= nfull) return;  // the whole group (or cluster) leaves together
+    if (first >= b1) return;  // the whole group (or cluster) leaves together
     const int W = p.W;
-    const int64_t nitems = ((nfull - 1 - first) / stride + 1) * W;
+    const int64_t nitems = ((b1 - 1 - first) / stride + 1) * W;
     const bool ef = p.r[0] != nullptr;
     const unsigned tx = ef ? 2 * kBytes : kBytes;
     auto issue = [&](int64_t beta, int w) {  // lane 0
@@ -179,7 +195,7 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
         bulk_load(sm.stage.g, p.g[w] + off, kBytes, &sm.bar);
         if (ef) bulk_load(sm.stage.r, p.r[w] + off, kBytes, &sm.bar);
     };
-    if (lane == 0) issue(first, 0);
+    if (!TAIL && lane == 0) issue(first, 0);
     int64_t pbeta = first;
     int pw = 1;
     if (pw == W) {
@@ -192,9 +208,23 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
     unsigned parity = 0;
     float acc[EPL];
     for (int64_t it = 0; it < nitems; ++it) {
-        const bool ok = mbar_wait_warp(&sm.bar, parity);
+        const bool ok = TAIL || mbar_wait_warp(&sm.bar, parity);
         float v[EPL];
-        if (ok) {
+        if constexpr (TAIL) {
+            const int64_t off = beta * D + (int64_t)rk * (32 * EPL);
+            const float *g = p.g[w] + off;
+            const float *r = ef ? p.r[w] + off : nullptr;
+#pragma unroll
+            for (int t = 0; t < EPL; ++t) {
+                const int e = slot_elem(t, lane);
+                float x = 0.0f;
+                if ((vmask >> t) & 1u) {
+                    x = g[e];
+                    if (r) x = __fadd_rn(x, r[e]);
+                }
+                v[t] = x;
+            }
+        } else if (ok) {
             parity ^= 1u;
 #pragma unroll
             for (int m = 0; m < EPL / 4; ++m) {
@@ -213,7 +243,7 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
             for (int t = 0; t < EPL; ++t) v[t] = 0.0f;
         }
         __syncwarp();
-        const bool issued = ok && it + 1 < nitems;
+        const bool issued = !TAIL && ok && it + 1 < nitems;
         if (issued && lane == 0) issue(pbeta, pw);
         if (++pw == W) {
             pw = 0;
@@ -230,25 +260,39 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
         // ---- first exchange: the group's statistics (and whether every copy arrived) -----------
         float s0, s1;
         if constexpr (SCHEME == GQ_ORQ) {
-            float mn = fmin3_nan(v[0], v[1], v[2]), mx = fmax3_nan(v[0], v[1], v[2]);
+            float mn = INFINITY, mx = -INFINITY;
+            if constexpr (TAIL) {
 #pragma unroll
-            for (int t = 3; t < EPL; t += 2) {
-                mn = t + 1 < EPL ? fmin3_nan(mn, v[t], v[t + 1]) : fmin_nan(mn, v[t]);
-                mx = t + 1 < EPL ? fmax3_nan(mx, v[t], v[t + 1]) : fmax_nan(mx, v[t]);
+                for (int t = 0; t < EPL; ++t)
+                    if ((vmask >> t) & 1u) {
+                        mn = fmin_nan(mn, v[t]);
+                        mx = fmax_nan(mx, v[t]);
+                    }
+            } else {
+                mn = fmin3_nan(v[0], v[1], v[2]);
+                mx = fmax3_nan(v[0], v[1], v[2]);
+#pragma unroll
+                for (int t = 3; t < EPL; t += 2) {
+                    mn = t + 1 < EPL ? fmin3_nan(mn, v[t], v[t + 1]) : fmin_nan(mn, v[t]);
+                    mx = t + 1 < EPL ? fmax3_nan(mx, v[t], v[t + 1]) : fmax_nan(mx, v[t]);
+                }
             }
             s0 = warp_redux_min(mn);
             s1 = warp_redux_max(mx);
         } else {
             float m = 0.0f;
 #pragma unroll
-            for (int t = 0; t < EPL; ++t) m = fmax_nan(m, fabsf(v[t]));
+            for (int t = 0; t < EPL; ++t)
+                if (!TAIL || ((vmask >> t) & 1u)) m = fmax_nan(m, fabsf(v[t]));
             s0 = warp_redux_max_abs(m);
             s1 = 0.0f;
         }
         if (lane == 0) {
             xg.stat[par][wib] = make_float2(s0, s1);
             xg.fail[par][wib] = ok ? 0 : 1;
+            if (C > 1) fence_cluster();
         }
+        __syncwarp();
         sync_group();
         float2 st = make_float2(SCHEME == GQ_ORQ ? INFINITY : 0.0f, -INFINITY);
         int failed = 0;
@@ -292,7 +336,7 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
             if (!(mx > mn)) {  // constant bucket (or NaN): one level, code 0 -- the whole group
 #pragma unroll
                 for (int t = 0; t < EPL; ++t) pos[t] = 0;
-                emit<EPL, FUSED, false, false, 0>(p, RoundConst{mn}, sigma, w, lane, 0xffffffffu, v, v, pos, acc);
+                emit<EPL, FUSED, false, TAIL, 0>(p, RoundConst{mn}, sigma, w, lane, vmask, v, v, pos, acc);
                 if (writer) store_table(p, w, beta, lane, mn);
             } else {
                 const float range = __fsub_rn(mx, mn);
@@ -302,10 +346,12 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
                 const int col = lane & (kHistCols - 1);
 #pragma unroll
                 for (int t = 0; t < EPL; ++t) {
-                    const int ps = min(__float2int_rz(__fmul_rn(__fsub_rn(v[t], mn), scale)), 63 << kOrqFBits);
+                    int ps = min(__float2int_rz(__fmul_rn(__fsub_rn(v[t], mn), scale)), 63 << kOrqFBits);
+                    if (TAIL) ps = max(ps, 0);  // the invalid slots hold 0, maybe outside [mn, mx]
                     const int cell = ps >> kOrqFBits;
                     pos[t] = cell;
-                    atomicAdd(&sm.fit.hist[cell * kHistCols + col], (uint32_t)(ps & 0xffff) | (1u << kHistCountShift));
+                    if (!TAIL || ((vmask >> t) & 1u))
+                        atomicAdd(&sm.fit.hist[cell * kHistCols + col], (uint32_t)(ps & 0xffff) | (1u << kHistCountShift));
                 }
                 __syncwarp();
                 uint32_t t0 = 0, t1 = 0, c0 = 0, c1 = 0;
@@ -336,37 +382,37 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
                     w1 = 0u;
                 }
                 // ---- second exchange: the group's histogram ---------------------------------
+                // The leader (group rank 0; in a cluster every CTA's warp 0) sums the cells, runs
+                // the greedy and builds the tables; the other warps wait for them at a barrier.
                 xg.cells[par][wib][lane] = make_uint4(c0, c1, w0, w1);
+                const int bar_id = C > 1 ? 1 : 1 + gid;
+                const int bar_n = 32 * (C > 1 ? kGroupWarps : G);
+                const int wfirst = C > 1 ? 0 : gid * G;  // the first warp of the group in this CTA
+                const bool leads = wib == wfirst;
+                Smem &lead = reinterpret_cast<Smem *>(smem_raw + sizeof(GroupXchg))[wfirst];
+                named_bar(bar_id, bar_n);
                 unsigned int C0 = 0u, C1 = 0u;
                 unsigned long long S0 = 0ull, S1 = 0ull;
-                if constexpr (C == 1) {
-                    named_bar(1 + gid, 32 * G);
+                if (leads) {
 #pragma unroll
-                    for (int j = 0; j < G; ++j) {
-                        const uint4 x = xg.cells[par][gid * G + j][lane];
+                    for (int j = 0; j < (C > 1 ? kGroupWarps : G); ++j) {
+                        const uint4 x = xg.cells[par][wfirst + j][lane];
                         C0 += x.x;
                         C1 += x.y;
                         S0 += x.z;
                         S1 += x.w;
                     }
-                } else {
-                    named_bar(1, 32 * kGroupWarps);
-                    if (wib == 0) {
-#pragma unroll
-                        for (int j = 0; j < kGroupWarps; ++j) {
-                            const uint4 x = xg.cells[par][j][lane];
-                            C0 += x.x;
-                            C1 += x.y;
-                            S0 += x.z;
-                            S1 += x.w;
-                        }
+                }
+                if constexpr (C > 1) {
+                    if (leads) {
                         xg.cta_c[par][lane][0] = C0;
                         xg.cta_c[par][lane][1] = C1;
                         xg.cta_s[par][lane][0] = S0;
                         xg.cta_s[par][lane][1] = S1;
+                        fence_cluster();
                     }
-                    cluster_bar();
-                    if (wib == 0) {
+                    cluster_bar_relaxed();
+                    if (leads) {
                         C0 = C1 = 0u;
                         S0 = S1 = 0ull;
 #pragma unroll
@@ -378,31 +424,25 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
                             S0 += s.x;
                             S1 += s.y;
                         }
-                        xg.tot_c[par][lane][0] = C0;
-                        xg.tot_c[par][lane][1] = C1;
-                        xg.tot_s[par][lane][0] = S0;
-                        xg.tot_s[par][lane][1] = S1;
                     }
-                    named_bar(1, 32 * kGroupWarps);
-                    C0 = xg.tot_c[par][lane][0];
-                    C1 = xg.tot_c[par][lane][1];
-                    S0 = xg.tot_s[par][lane][0];
-                    S1 = xg.tot_s[par][lane][1];
                 }
-                // exclusive prefix over the cell pairs of (sum << 16 | count): counts up to 32768
-                // and sums below 2^37 fit the packed 64-bit word
-                const unsigned long long own = ((S0 + S1) << 16) | (unsigned long long)(C0 + C1);
-                const unsigned long long ex = warp_inclusive_scan(own, lane) - own;
-                const int ec = (int)(ex & 0xffffull);
-                const long long es = (long long)(ex >> 16);
-                sm.fit.P0[2 * lane] = ec;
-                sm.fit.P0[2 * lane + 1] = ec + (int)C0;
-                sm.fit.P1[2 * lane] = es;
-                sm.fit.P1[2 * lane + 1] = es + (long long)S0;
-                __syncwarp();
-                const unsigned long long mask = orq_greedy(sm.fit.P0, sm.fit.P1, p.s, lane);
-                group_orq_tables(p, sm.fit, w, beta, lane, writer, mask, mn, mx, step);
-                emit<EPL, FUSED, true, false, 0>(p, RoundORQ{sm.fit.ctab}, sigma, w, lane, 0xffffffffu, v, v, pos, acc);
+                if (leads) {
+                    // exclusive prefix over the cell pairs of (sum << 16 | count): counts up to
+                    // 32768 and sums below 2^37 fit the packed 64-bit word
+                    const unsigned long long own = ((S0 + S1) << 16) | (unsigned long long)(C0 + C1);
+                    const unsigned long long ex = warp_inclusive_scan(own, lane) - own;
+                    const int ec = (int)(ex & 0xffffull);
+                    const long long es = (long long)(ex >> 16);
+                    sm.fit.P0[2 * lane] = ec;
+                    sm.fit.P0[2 * lane + 1] = ec + (int)C0;
+                    sm.fit.P1[2 * lane] = es;
+                    sm.fit.P1[2 * lane + 1] = es + (long long)S0;
+                    __syncwarp();
+                    const unsigned long long mask = orq_greedy(sm.fit.P0, sm.fit.P1, p.s, lane);
+                    group_orq_tables(p, sm.fit, w, beta, lane, writer, mask, mn, mx, step);
+                }
+                named_bar(bar_id, bar_n);
+                emit<EPL, FUSED, true, TAIL, 0>(p, RoundORQ{lead.fit.ctab}, sigma, w, lane, vmask, v, v, pos, acc);
                 __syncwarp();
             }
         } else {
@@ -420,15 +460,21 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
             int pos[EPL];
 #pragma unroll
             for (int t = 0; t < EPL; ++t) pos[t] = 0;
-            emit<EPL, FUSED, true, false, 0>(p, rule, sigma, w, lane, 0xffffffffu, v, v, pos, acc);
+            emit<EPL, FUSED, true, TAIL, 0>(p, rule, sigma, w, lane, vmask, v, v, pos, acc);
             if (writer) store_table(p, w, beta, lane, m);
             __syncwarp();
         }
 
         const bool last_w = w == W - 1;
         if (FUSED && last_w) {
+            if constexpr (TAIL) {
 #pragma unroll
-            for (int m = 0; m < EPL / 4; ++m) store_avg4(p.avg + sigma * (32 * EPL), m, lane, acc + 4 * m, p.inv_w);
+                for (int t = 0; t < EPL; ++t)
+                    if ((vmask >> t) & 1u) p.avg[sigma * (32 * EPL) + slot_elem(t, lane)] = __fmul_rn(acc[t], p.inv_w);
+            } else {
+#pragma unroll
+                for (int m = 0; m < EPL / 4; ++m) store_avg4(p.avg + sigma * (32 * EPL), m, lane, acc + 4 * m, p.inv_w);
+            }
         }
         if (last_w) {
             w = 0;
@@ -440,14 +486,15 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
     if constexpr (C > 1) cluster_bar();  // no CTA leaves while a peer may still read its slots
 }
 
-template <int SCHEME, int G, bool FUSED>
-cudaError_t launch_group_g(const KParams &p0, int64_t nfull, cudaStream_t stream)
+template <int SCHEME, int G, bool FUSED, bool TAIL>
+cudaError_t launch_group_g(const KParams &p0, int64_t b0, int64_t b1, cudaStream_t stream)
 {
     constexpr int C = G > kGroupWarps ? G / kGroupWarps : 1;
     constexpr int GPC = G < kGroupWarps ? kGroupWarps / G : 1;
     KParams p = p0;
     p.codes_words = (int64_t)(32 * kSliceEPL) * p.bits / 32;  // code words of one 512-element slice
-    auto kern = k_group<SCHEME, G, FUSED>;
+    auto kern = k_group<SCHEME, G, FUSED, TAIL>;
+    const int64_t nbk = b1 - b0;
     const size_t smem = sizeof(GroupXchg) + sizeof(GroupWarpSmem<SCHEME>) * kGroupWarps;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -472,34 +519,46 @@ cudaError_t launch_group_g(const KParams &p0, int64_t nfull, cudaStream_t stream
         e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
         if (e != cudaSuccess) return e;
         if (nclusters < 1) return cudaErrorInvalidConfiguration;
-        groups = nfull < nclusters ? nfull : nclusters;
+        groups = nbk < nclusters ? nbk : nclusters;
         cfg.gridDim = dim3((unsigned)(groups * C), 1, 1);
     } else {
         int per_sm = 0;
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGroupWarps * 32, smem);
         if (per_sm < 1) per_sm = 1;
         const int64_t cap = (int64_t)sms * per_sm * GPC;
-        groups = nfull < cap ? nfull : cap;
+        groups = nbk < cap ? nbk : cap;
         cfg.gridDim = dim3((unsigned)((groups + GPC - 1) / GPC), 1, 1);
         cfg.attrs = nullptr;
         cfg.numAttrs = 0;
     }
-    e = cudaLaunchKernelEx(&cfg, kern, p, nfull);
+    e = cudaLaunchKernelEx(&cfg, kern, p, b0, b1);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-template <int SCHEME, bool FUSED>
-cudaError_t launch_group_fused(const KParams &p, int64_t nfull, cudaStream_t stream)
+template <int SCHEME, bool FUSED, bool TAIL>
+cudaError_t launch_group_range(const KParams &p, int64_t b0, int64_t b1, cudaStream_t stream)
 {
     switch (p.d) {
-    case 1024: return launch_group_g<SCHEME, 2, FUSED>(p, nfull, stream);
-    case 2048: return launch_group_g<SCHEME, 4, FUSED>(p, nfull, stream);
-    case 4096: return launch_group_g<SCHEME, 8, FUSED>(p, nfull, stream);
-    case 8192: return launch_group_g<SCHEME, 16, FUSED>(p, nfull, stream);
-    case 16384: return launch_group_g<SCHEME, 32, FUSED>(p, nfull, stream);
-    default: return launch_group_g<SCHEME, 64, FUSED>(p, nfull, stream);
+    case 1024: return launch_group_g<SCHEME, 2, FUSED, TAIL>(p, b0, b1, stream);
+    case 2048: return launch_group_g<SCHEME, 4, FUSED, TAIL>(p, b0, b1, stream);
+    case 4096: return launch_group_g<SCHEME, 8, FUSED, TAIL>(p, b0, b1, stream);
+    case 8192: return launch_group_g<SCHEME, 16, FUSED, TAIL>(p, b0, b1, stream);
+    case 16384: return launch_group_g<SCHEME, 32, FUSED, TAIL>(p, b0, b1, stream);
+    default: return launch_group_g<SCHEME, 64, FUSED, TAIL>(p, b0, b1, stream);
     }
+}
+
+// Every bucket of p: the full ones, then the ragged last one (if any) in a one-group launch.
+template <int SCHEME, bool FUSED>
+cudaError_t launch_group_fused(const KParams &p, cudaStream_t stream)
+{
+    const int64_t nfull = p.tail == p.d ? p.nb : p.nb - 1;
+    if (nfull > 0) {
+        const cudaError_t e = launch_group_range<SCHEME, FUSED, false>(p, 0, nfull, stream);
+        if (e != cudaSuccess) return e;
+    }
+    return nfull < p.nb ? launch_group_range<SCHEME, FUSED, true>(p, nfull, p.nb, stream) : cudaSuccess;
 }
 
 }  // namespace

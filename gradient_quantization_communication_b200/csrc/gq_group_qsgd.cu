@@ -3,9 +3,9 @@
 
 namespace gq {
 
-cudaError_t launch_group_qsgd(const KParams &p, int64_t nfull, bool fused, cudaStream_t stream)
+cudaError_t launch_group_qsgd(const KParams &p, bool fused, cudaStream_t stream)
 {
-    return fused ? launch_group_fused<GQ_QSGD, true>(p, nfull, stream) : launch_group_fused<GQ_QSGD, false>(p, nfull, stream);
+    return fused ? launch_group_fused<GQ_QSGD, true>(p, stream) : launch_group_fused<GQ_QSGD, false>(p, stream);
 }
 
 }  // namespace gq

@@ -52,10 +52,10 @@ cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream
 // Shared-memory path (d = 1024 .. 32768): one CTA per bucket index walking the p.W workers;
 // with p.avg set, the average of the dequantized values is accumulated on chip and written.
 cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream, int64_t first = 0);
-// d = 1024 .. 32768, ORQ or QSGD / TernGrad, no clipping: full buckets 0 .. nfull-1 spread over
-// groups of d / 512 warps (gq_group.cuh).
-cudaError_t launch_group_orq(const KParams &p, int64_t nfull, bool fused, cudaStream_t stream);
-cudaError_t launch_group_qsgd(const KParams &p, int64_t nfull, bool fused, cudaStream_t stream);
+// d = 1024 .. 32768, ORQ or QSGD / TernGrad, no clipping: every bucket spread over a group of
+// d / 512 warps (gq_group.cuh); the ragged last one in a second, one-group launch.
+cudaError_t launch_group_orq(const KParams &p, bool fused, cudaStream_t stream);
+cudaError_t launch_group_qsgd(const KParams &p, bool fused, cudaStream_t stream);
 // Dequantize + aggregate for any d.
 cudaError_t launch_decode(const KParams &p, cudaStream_t stream);
 // GQ_TERNGRAD_LAYER: the tensors' scales (into p.seg_max), then the encode of p.W workers (the
