@@ -66,6 +66,8 @@ def parse_args():
     ap.add_argument("--clip", type=float, default=0.0)
     ap.add_argument("--elements", type=int, default=0, help="truncate the workload (profiling runs)")
     ap.add_argument("--no-msgs", action="store_true", help="do not write the messages")
+    ap.add_argument("--base-s", action="store_true",
+                    help="base-s messages (s = 3, 5, 9 levels) written by the encode and read by the decode")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -103,14 +105,26 @@ def table_len(scheme_id, levels):
     return 1 if scheme_id in (0, 1, 5, 7) else (2 if scheme_id in (2, 3, 6) else levels)
 
 
-def bytes_per_worker_elem(scheme_id, levels, d, W, ef, msgs):
-    """Algorithmic HBM bytes per worker-element of the fused step: read g (and r), write r',
-    the message (b/8 bits + level table share) and the worker's share of the average."""
-    bits = (levels - 1).bit_length()
+# base-s groups: s -> (g codes, B bits)
+BASE_S_GROUPS = {3: (5, 8), 5: (3, 7), 9: (5, 16)}
+
+
+def message_bytes_per_elem(scheme_id, levels, d, base_s=False):
+    """A message's bytes per element: the codes (b/8, or a bucket's base-s words over d) and the
+    level table's share."""
     L = table_len(scheme_id, levels)
+    if base_s:
+        g, B = BASE_S_GROUPS[levels]
+        return 4.0 * ((-(-d // g) * B + 31) // 32) / d + 4.0 * L / d
+    return (levels - 1).bit_length() / 8.0 + 4.0 * L / d
+
+
+def bytes_per_worker_elem(scheme_id, levels, d, W, ef, msgs, base_s=False):
+    """Algorithmic HBM bytes per worker-element of the fused step: read g (and r), write r',
+    the message and the worker's share of the average."""
     b = 4.0 + (8.0 if ef else 0.0) + 4.0 / W
     if msgs:
-        b += bits / 8.0 + 4.0 * L / d
+        b += message_bytes_per_elem(scheme_id, levels, d, base_s)
     return b
 
 
@@ -303,6 +317,7 @@ def workload_config(args, wl):
         "on" if wl.error_feedback else "off", (", clip %.1f sigma" % args.clip) if args.clip else ""),
         "elements": wl.n, "workers": wl.workers, "scheme": args.scheme, "levels": args.levels,
         "bucket": args.bucket, "messages_written": not args.no_msgs,
+        "message_format": "base-s" if getattr(args, "base_s", False) else "dense",
         "l2": ("inputs larger than L2 (working set %.1f GB, L2 126 MB): no flush needed" % (wl.n * wl.workers * 12 / 1e9)
                if wl.n * wl.workers * 12 > 4 * 126e6 else "working set within a few L2 sizes: timings include L2 reuse"),
         "gradients": "drawn once in HBM before timing; the residual evolves every step"}
@@ -318,7 +333,7 @@ def fused_roofline(args, d, W, n, ef, write_msgs, bpe, achieved, peak, peak_kind
     elements processed."""
     if achieved is None:
         return None
-    kernel_key = "fused_%s%d_d%d_w%d" % (args.scheme, args.levels, d, W)
+    kernel_key = "fused_%s%d_d%d_w%d%s" % (args.scheme, args.levels, d, W, "_bases" if getattr(args, "base_s", False) else "")
     traffic = traffic_record(kernel_key)
     if traffic and (traffic.get("workload"), traffic.get("error_feedback"), traffic.get("messages_written"),
                     traffic.get("clip")) != (args.workload, bool(ef), bool(write_msgs), float(args.clip)):
@@ -368,7 +383,7 @@ def run_gq(args):
     W, n, d, ef = wl.workers, wl.n, args.bucket, wl.error_feedback
     sid = G.SCHEMES[args.scheme]
     cfg = G.gq_config(sid, args.levels, d, W, ef, args.clip, wl.rounding_seed, n)
-    plan = G.Plan(cfg)
+    plan = G.Plan(cfg, fmt=G.GQ_FORMAT_BASE_S if args.base_s else G.GQ_FORMAT_DENSE)
     stream = torch.cuda.current_stream()
     g = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
     for w in range(W):
@@ -417,7 +432,7 @@ def run_gq(args):
     ms_per_step = elapsed_ms / args.steps
     value = job_value(world, W, n, args.steps, elapsed_ms)
 
-    bpe = bytes_per_worker_elem(sid, args.levels, d, W, ef, write_msgs)
+    bpe = bytes_per_worker_elem(sid, args.levels, d, W, ef, write_msgs, args.base_s)
     peak, peak_kind = measured_hbm_peak()
     achieved = bpe * W * n / (per_launch_ms / 1000.0) / 1e9 if d <= 512 else None
     roofline = fused_roofline(args, d, W, n, ef, write_msgs, bpe, achieved, peak, peak_kind)
@@ -557,7 +572,7 @@ def run_unfused(args):
     torch.cuda.set_device(dev)
     sid = G.SCHEMES[args.scheme]
     cfg = G.gq_config(sid, args.levels, d, W, ef, args.clip, wl.rounding_seed, n)
-    plan = G.Plan(cfg)
+    plan = G.Plan(cfg, fmt=G.GQ_FORMAT_BASE_S if args.base_s else G.GQ_FORMAT_DENSE)
     stream = torch.cuda.current_stream()
     g = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
     for w in range(W):
@@ -602,9 +617,7 @@ def run_unfused(args):
     enc_ms = statistics.mean(a.elapsed_time(b) for e in evs for a, b in e[:W])
     dec_ms = statistics.mean(e[W][0].elapsed_time(e[W][1]) for e in evs)
     plan.close()
-    bits = (args.levels - 1).bit_length()
-    L = table_len(sid, args.levels)
-    msg_b = bits / 8.0 + 4.0 * L / d
+    msg_b = message_bytes_per_elem(sid, args.levels, d, args.base_s)
     enc_b = 4.0 + (8.0 if ef else 0.0) + msg_b          # per element of one worker
     dec_b = W * msg_b + 4.0                             # per element of the average
     peak, peak_kind = measured_hbm_peak()

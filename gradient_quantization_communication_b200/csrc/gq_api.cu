@@ -23,6 +23,8 @@ struct gq_plan {
     int64_t *seg_off;      // GQ_TERNGRAD_LAYER: the tensors' offsets (device), NULL until set
     int nseg;
     unsigned int *seg_max; // GQ_TERNGRAD_LAYER: W x nseg scales (device scratch)
+    int fmt_s;             // base-s messages of s levels (GQ_FORMAT_BASE_S), 0 = dense
+    int64_t base_words;    // base-s words per bucket
 };
 
 namespace {
@@ -126,7 +128,8 @@ gq::KParams base_params(const gq_plan &pl, uint64_t step)
     p.inv_w = 1.0f;
     for (int k = 0; k < pl.cfg.levels; ++k)
         p.qratio[k] = (float)(2 * k - (pl.cfg.levels - 1)) / (float)(pl.cfg.levels - 1);
-    p.codes_words = (int64_t)pl.cfg.bucket * pl.bits / 32;
+    p.codes_words = pl.fmt_s ? pl.base_words : (int64_t)pl.cfg.bucket * pl.bits / 32;
+    p.fmt_s = pl.fmt_s;
     p.levels_off = (int64_t)pl.levels_off;
     p.status = pl.status;
     p.seg_off = pl.seg_off;
@@ -191,6 +194,8 @@ gq_status_t gq_plan_create(const gq_config_t *cfg, gq_plan_t *out)
     pl->seg_off = nullptr;
     pl->nseg = 0;
     pl->seg_max = nullptr;
+    pl->fmt_s = 0;
+    pl->base_words = 0;
     if (c.scheme == GQ_TERNGRAD_LAYER) pl->msg_bytes = pl->codes_off = pl->levels_off = 0;  // until the segments
     const size_t err_bytes = (size_t)gq::err_scratch_doubles(pl->nb) * sizeof(double);
     if (cudaGetDevice(&pl->device) != cudaSuccess || cudaMalloc(&pl->status, sizeof(unsigned int)) != cudaSuccess ||
@@ -361,6 +366,34 @@ gq_status_t gq_plan_set_segments(gq_plan_t plan, const int64_t *offsets, int nse
     plan->codes_off = 0;
     plan->levels_off = (size_t)cbytes;
     plan->msg_bytes = (size_t)(cbytes + sbytes);
+    return GQ_OK;
+}
+
+gq_status_t gq_plan_set_format(gq_plan_t plan, int format)
+{
+    if (!plan) return GQ_ERR_INVALID;
+    if (plan->cfg.scheme == GQ_TERNGRAD_LAYER)  // its message is dense and sized by the tensors
+        return format == GQ_FORMAT_DENSE ? GQ_OK : (format == GQ_FORMAT_BASE_S ? GQ_ERR_UNSUPPORTED : GQ_ERR_INVALID);
+    if (format == GQ_FORMAT_DENSE) {
+        plan->fmt_s = 0;
+        plan->base_words = 0;
+        layout(plan->cfg, &plan->msg_bytes, &plan->codes_off, &plan->levels_off);
+        return GQ_OK;
+    }
+    if (format != GQ_FORMAT_BASE_S) return GQ_ERR_INVALID;
+    const gq_config_t &c = plan->cfg;
+    const bool family = c.scheme == GQ_ORQ || c.scheme == GQ_QSGD || c.scheme == GQ_TERNGRAD ||
+                        c.scheme == GQ_QSGD_NEAREST || c.scheme == GQ_QSGD_L2;
+    if (!family || c.bucket > 512 || (c.levels != 3 && c.levels != 5 && c.levels != 9)) return GQ_ERR_UNSUPPORTED;
+    size_t bytes = 0, coff = 0, loff = 0;
+    const gq_status_t st = gq_entropy_layout(&c, &bytes, &coff, &loff);
+    if (st != GQ_OK) return st;
+    const int g = c.levels == 5 ? 3 : 5, B = c.levels == 3 ? 8 : c.levels == 5 ? 7 : 16;
+    plan->fmt_s = c.levels;
+    plan->base_words = (((int64_t)c.bucket + g - 1) / g * B + 31) / 32;
+    plan->msg_bytes = bytes;
+    plan->codes_off = coff;
+    plan->levels_off = loff;
     return GQ_OK;
 }
 

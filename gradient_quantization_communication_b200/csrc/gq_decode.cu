@@ -11,6 +11,7 @@
 // table instead).  The loads of a group of workers are issued together before any
 // of them is used; the sum runs in worker order in registers and the average is written once,
 // with 16-byte stores.
+#include "gq_bases.cuh"
 #include "gq_device.cuh"
 
 namespace gq {
@@ -109,6 +110,63 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
     }
 }
 
+// Base-s messages (s = 3, 5, 9; d <= 512): the same items and sum, with each lane's four codes
+// of a chunk taken from the one or two base-s groups that hold them (base_codes4).
+template <bool QSGD, int S, int CPI>
+__global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base(const __grid_constant__ KParams p)
+{
+    constexpr int BITS = S == 3 ? 2 : S == 5 ? 3 : 4;  // the level lookup's segment: 2^b lanes
+    constexpr int kWidth = 1 << BITS;
+    const int lane = threadIdx.x & 31;
+    const int slot = lane & (kWidth - 1);
+    const int64_t nitems = (p.n + 128 * CPI - 1) / (128 * CPI);
+    const int64_t first = (int64_t)blockIdx.x * kDecodeWarps + (threadIdx.x >> 5);
+    const int64_t stride = (int64_t)gridDim.x * kDecodeWarps;
+    const int log2d = 31 - __clz(p.d);
+    const int nw = (int)p.codes_words;
+    const bool has_level = slot < p.L;
+    const float qr = (QSGD && slot < p.s) ? p.qratio[slot] : 0.0f;
+    for (int64_t it = first; it < nitems; it += stride) {
+        const int64_t e0 = it * (128 * CPI);
+        const int64_t bk = e0 >> log2d;
+        const int eb = (int)(e0 & (p.d - 1)) + 4 * lane;  // this lane's first element in the bucket
+        const int64_t tbase = QSGD ? bk : bk * p.L + slot;
+        int nlive = (int)((p.n - e0 + 127) >> 7);
+        nlive = nlive < CPI ? nlive : CPI;
+        float acc[CPI][4];
+#pragma unroll
+        for (int c = 0; c < CPI; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
+        for (int w = 0; w < p.W; ++w) {
+            const unsigned char *msg = p.msg[w];
+            const uint32_t *words = reinterpret_cast<const uint32_t *>(msg) + bk * p.codes_words;
+            float lv = 0.0f;
+            if (QSGD || has_level) lv = __ldg(reinterpret_cast<const float *>(msg + p.levels_off) + tbase);
+            const float level = QSGD ? __fmul_rn(lv, qr) : lv;
+#pragma unroll
+            for (int c = 0; c < CPI; ++c) {
+                int code[4] = {0, 0, 0, 0};
+                if (c < nlive) base_codes4<S>(words, nw, eb + 128 * c, code);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, code[e], kWidth));
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < CPI; ++c) {
+            const int64_t e = e0 + 128 * c + 4 * lane;
+            if (e + 3 < p.n) {
+                __stcs(reinterpret_cast<float4 *>(p.avg + e),
+                       make_float4(__fmul_rn(acc[c][0], p.inv_w), __fmul_rn(acc[c][1], p.inv_w),
+                                   __fmul_rn(acc[c][2], p.inv_w), __fmul_rn(acc[c][3], p.inv_w)));
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (e + q < p.n) p.avg[e + q] = __fmul_rn(acc[c][q], p.inv_w);
+            }
+        }
+    }
+}
+
 template <bool QSGD, int BITS, int CPI>
 cudaError_t launch(const KParams &p, cudaStream_t stream)
 {
@@ -138,6 +196,45 @@ cudaError_t launch_cpi(const KParams &p, cudaStream_t stream)
     }
 }
 
+template <bool QSGD, int S, int CPI>
+cudaError_t launch_base(const KParams &p, cudaStream_t stream)
+{
+    auto kern = k_decode_base<QSGD, S, CPI>;
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecodeWarps * 32, 0);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t nitems = (p.n + 128 * CPI - 1) / (128 * CPI);
+    const int64_t need = (nitems + kDecodeWarps - 1) / kDecodeWarps;
+    const int64_t cap = (int64_t)sms * per_sm;
+    const int grid = (int)(need < cap ? need : cap);
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, kDecodeWarps * 32, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <bool QSGD, int S>
+cudaError_t launch_base_cpi(const KParams &p, cudaStream_t stream)
+{
+    switch (p.d) {
+    case 128: return launch_base<QSGD, S, 1>(p, stream);
+    case 256: return launch_base<QSGD, S, 2>(p, stream);
+    default: return launch_base<QSGD, S, 4>(p, stream);
+    }
+}
+
+template <bool QSGD>
+cudaError_t launch_base_s(const KParams &p, cudaStream_t stream)
+{
+    switch (p.fmt_s) {
+    case 3: return launch_base_cpi<QSGD, 3>(p, stream);
+    case 5: return launch_base_cpi<QSGD, 5>(p, stream);
+    case 9: return launch_base_cpi<QSGD, 9>(p, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 template <bool QSGD>
 cudaError_t launch_bits(const KParams &p, cudaStream_t stream)
 {
@@ -158,6 +255,7 @@ cudaError_t launch_decode(const KParams &p, cudaStream_t stream)
 {
     const bool qsgd =
         p.scheme == GQ_QSGD || p.scheme == GQ_TERNGRAD || p.scheme == GQ_QSGD_NEAREST || p.scheme == GQ_QSGD_L2;
+    if (p.fmt_s != 0) return qsgd ? launch_base_s<true>(p, stream) : launch_base_s<false>(p, stream);
     return qsgd ? launch_bits<true>(p, stream) : launch_bits<false>(p, stream);
 }
 

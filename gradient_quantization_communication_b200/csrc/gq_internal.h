@@ -36,6 +36,8 @@ struct KParams {
     unsigned char *msg[GQ_MAX_WORKERS];// NULL: do not write the message
     float *avg;                        // fused kernels only
     unsigned int *status;              // plan status word
+    int fmt_s;                         // base-s messages of s levels (3, 5, 9), 0 = dense; codes_words
+                                       // then counts the bucket's base-s words
     const int64_t *seg_off;            // GQ_TERNGRAD_LAYER: nseg + 1 tensor offsets (device)
     int nseg;
     unsigned int *seg_max;             // GQ_TERNGRAD_LAYER: W x nseg scales (float bits, device scratch)

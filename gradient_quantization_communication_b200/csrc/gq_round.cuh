@@ -186,7 +186,9 @@ __device__ __forceinline__ void pack_chunk(const KParams &p, int lane, const int
 //   cw    packed words of the chunk (4b words, 16-byte aligned), NULL: no message
 // Returns the dequantized values in q.
 // BITS: bits per code when known at compile time, 0 to read it from p.bits.
-// IO: bit 0 set if rout is known non-NULL, bit 1 if cw is (no run-time test then).
+// IO: bit 0 set if rout is known non-NULL, bit 1 if cw is (no run-time test then); IO >= 4
+// (base-s messages): cw is the chunk's 32 words of codes as bytes in shared memory, element
+// order, instead of its packed words.
 template <bool RANDOM, bool ALLVALID, int BITS, int IO = 0, class R>
 __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uint64_t blk, uint32_t worker, int lane,
                                             uint32_t valid, const float (&v)[4], const float (&u)[4],
@@ -211,7 +213,12 @@ __device__ __forceinline__ void round_chunk(const KParams &p, const R &rule, uin
                 if ((valid >> c) & 1u) rout[4 * lane + c] = __fsub_rn(v[c], q[c]);
         }
     }
-    if ((IO & 2) || cw) pack_chunk<BITS>(p, lane, code, cw);
+    if constexpr (IO >= 4) {
+        if ((IO & 2) || cw)
+            cw[lane] = (uint32_t)code[0] | ((uint32_t)code[1] << 8) | ((uint32_t)code[2] << 16) | ((uint32_t)code[3] << 24);
+    } else {
+        if ((IO & 2) || cw) pack_chunk<BITS>(p, lane, code, cw);
+    }
 }
 
 // Running binary64 sums of the quantization error (see gq_quant_error): expected squared

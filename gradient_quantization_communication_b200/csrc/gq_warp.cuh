@@ -29,6 +29,7 @@
 // plain loads, so the main kernel carries no tail logic.
 #pragma once
 
+#include "gq_bases.cuh"
 #include "gq_round.cuh"
 
 namespace gq {
@@ -52,6 +53,9 @@ struct alignas(16) StageBuf {
 // A column collects at most 4 lanes x 16 values = 64 entries, so the fraction sum stays below
 // 64 * 2^16 = 2^22 and the count (<= 64) fits above it.
 constexpr int kHistCountShift = 22;
+// Words of a bucket's codes as bytes (base-s messages): 512 bytes and 32 bytes of zeros past
+// them for the last group's missing codes.
+constexpr int kCodeBytesWords = 512 / 4 + 8;
 struct alignas(16) FitORQ {
     uint32_t hist[64 * kHistCols];  // [cell][column]; cell 63 holds the values at the top grid point
     float4 ctab[64];                // cell -> {lower, upper, 1/(upper-lower), bracket}; 63 repeats 62
@@ -59,10 +63,12 @@ struct alignas(16) FitORQ {
     float lev[GQ_MAX_LEVELS];       // chosen levels in increasing order
     uint32_t P1[64];                // sum of positions over cells < k (< 2^31 for d <= 512)
     int P0[64];                     // count over cells < k
+    uint32_t codes[kCodeBytesWords];  // base-s messages: the bucket's codes as bytes (0 past d)
 };
 struct alignas(16) FitQSGD {
     float2 pair[GQ_MAX_QSGD_LEVELS];  // {level k, level k+1}
     float qr[GQ_MAX_QSGD_LEVELS];     // the level ratios (2k - (s-1)) / (s-1), copied once
+    uint32_t codes[kCodeBytesWords];  // base-s messages: the bucket's codes as bytes (0 past d)
 };
 struct alignas(16) FitPB {
     unsigned long long s1[64], s2[64];  // per cell: sum of positions, of squared positions
@@ -93,10 +99,12 @@ __device__ __forceinline__ int slot_elem(int t, int lane) { return 128 * (t >> 2
 // ---------------------------------------------------------------------------------------------
 // BITS < 0 selects the error mode of gq_quant_error: nothing is written, the error terms of
 // the bucket's elements are added to *ea.
+// IO >> 2 = s selects base-s messages: the codes go to `codes` (the warp's shared bytes) chunk by
+// chunk and the bucket's base-s words are built from them after the last chunk.
 template <int EPL, bool FUSED, bool RANDOM, bool TAIL, int BITS, int IO = 0, class R>
 __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t beta, int w, int lane, uint32_t vmask,
                                      const float (&v)[EPL], const float (&u)[EPL], const int (&pos)[EPL],
-                                     float (&acc)[EPL], ErrAcc *ea = nullptr)
+                                     float (&acc)[EPL], ErrAcc *ea = nullptr, uint32_t *codes = nullptr)
 {
     const int64_t base = beta * (int64_t)(32 * EPL);
     if constexpr (BITS < 0) {
@@ -112,10 +120,12 @@ __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t be
         return;
     }
     constexpr bool kHasR = (IO & 1) != 0, kHasMsg = (IO & 2) != 0;
-    constexpr int kCodeWords = 4 * (BITS > 0 ? BITS : 0);  // words per chunk when b is known
+    constexpr int kBaseS = IO >> 2;
+    constexpr int kCodeWords = kBaseS ? 32 : 4 * (BITS > 0 ? BITS : 0);  // words per chunk when known
     float *r = p.r[w];
     unsigned char *msg = p.msg[w];
-    uint32_t *cw = (kHasMsg || msg) ? reinterpret_cast<uint32_t *>(msg) + beta * p.codes_words : nullptr;
+    uint32_t *out = (kHasMsg || msg) ? reinterpret_cast<uint32_t *>(msg) + beta * p.codes_words : nullptr;
+    uint32_t *cw = kBaseS ? ((kHasMsg || msg) ? codes : nullptr) : out;
     const uint32_t worker = p.worker0 + (uint32_t)w;
 #pragma unroll
     for (int m = 0; m < EPL / 4; ++m) {
@@ -131,6 +141,15 @@ __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t be
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 if (!TAIL || ((valid >> c) & 1u)) acc[4 * m + c] = __fadd_rn(acc[4 * m + c], q[c]);
+        }
+    }
+    if constexpr (kBaseS != 0) {
+        if (kHasMsg || out) {
+            __syncwarp();
+            constexpr int G = (32 * EPL + BaseS<kBaseS>::g - 1) / BaseS<kBaseS>::g;
+            const unsigned char *c8 = reinterpret_cast<const unsigned char *>(codes);
+            for (int k = lane; k < p.codes_words; k += 32) __stcs(out + k, base_word<kBaseS>(c8, k, G));
+            __syncwarp();
         }
     }
 }
@@ -227,7 +246,7 @@ __device__ void fit_qsgd(const KParams &p, FitQSGD &sm, int64_t beta, int w, int
     int pos[EPL];
 #pragma unroll
     for (int t = 0; t < EPL; ++t) pos[t] = 0;
-    emit<EPL, FUSED, !NEAREST, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
+    emit<EPL, FUSED, !NEAREST, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea, sm.codes);
     store_table(p, w, beta, lane, m);
 }
 
@@ -293,7 +312,7 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     if (!(mx > mn)) {  // constant bucket (or NaN): one level, code 0
 #pragma unroll
         for (int t = 0; t < EPL; ++t) pos[t] = 0;
-        emit<EPL, FUSED, false, TAIL, BITS, IO>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc, ea);
+        emit<EPL, FUSED, false, TAIL, BITS, IO>(p, RoundConst{mn}, beta, w, lane, vmask, v, u, pos, acc, ea, sm.codes);
         store_table(p, w, beta, lane, mn);
         return;
     }
@@ -360,7 +379,7 @@ __device__ void fit_orq(const KParams &p, FitORQ &sm, int64_t beta, int w, int l
     __syncwarp();
     const unsigned long long mask = orq_greedy(sm.P0, sm.P1, p.s, lane);
     build_orq_tables<IO>(p, sm, w, beta, lane, mask, mn, mx, step);
-    emit<EPL, FUSED, true, TAIL, BITS, IO>(p, RoundORQ{sm.ctab}, beta, w, lane, vmask, v, u, pos, acc, ea);
+    emit<EPL, FUSED, true, TAIL, BITS, IO>(p, RoundORQ{sm.ctab}, beta, w, lane, vmask, v, u, pos, acc, ea, sm.codes);
     __syncwarp();
 }
 
@@ -762,9 +781,11 @@ __device__ __forceinline__ void init_fit(const KParams &p, Fit &fit, int lane)
 {
     if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD || SCHEME == GQ_QSGD_NEAREST || SCHEME == GQ_QSGD_L2) {
         for (int k = lane; k < p.s; k += 32) fit.qr[k] = p.qratio[k];
+        for (int i = lane; i < kCodeBytesWords; i += 32) fit.codes[i] = 0u;
     }
     if constexpr (SCHEME == GQ_ORQ) {
         for (int i = lane; i < 64 * kHistCols; i += 32) fit.hist[i] = 0u;
+        for (int i = lane; i < kCodeBytesWords; i += 32) fit.codes[i] = 0u;
     }
     if constexpr (SCHEME == GQ_BINGRAD_PB) {
         for (int i = lane; i < 64; i += 32) {
@@ -975,7 +996,7 @@ cudaError_t warp_dispatch_err(const KParams &p, double *part, cudaStream_t strea
 // (warp k takes workers k, k + nwarps, ...).  Each warp's dequantized values are parked in
 // shared memory (qbuf[w][e]) and summed afterwards in worker order, which gives the same bits
 // as the register sum of the main kernel: every partial sum starts from +0.
-template <int EPL, int SCHEME, bool FUSED>
+template <int EPL, int SCHEME, bool FUSED, int IO = 0>
 __global__ void __launch_bounds__(512) k_warp_tail(const __grid_constant__ KParams p)
 {
     using Fit = typename FitFor<SCHEME>::type;
@@ -1006,7 +1027,7 @@ __global__ void __launch_bounds__(512) k_warp_tail(const __grid_constant__ KPara
             v[t] = x;
             acc[t] = 0.0f;
         }
-        process<EPL, SCHEME, FUSED, true, 0>(p, fit, beta, w, lane, nvalid, vmask, v, acc);
+        process<EPL, SCHEME, FUSED, true, 0, IO>(p, fit, beta, w, lane, nvalid, vmask, v, acc);
         if (FUSED) {
 #pragma unroll
             for (int t = 0; t < EPL; ++t) qbuf[w * D + slot_elem(t, lane)] = acc[t];
@@ -1023,15 +1044,29 @@ __global__ void __launch_bounds__(512) k_warp_tail(const __grid_constant__ KPara
     }
 }
 
+// The base-s level count a code width can carry (s = 3, 5, 9 for b = 2, 3, 4), 0 for none.
+template <int SCHEME, int BITS>
+constexpr int base_s_for()
+{
+    if constexpr (SCHEME == GQ_ORQ || SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD || SCHEME == GQ_QSGD_NEAREST ||
+                  SCHEME == GQ_QSGD_L2)
+        return BITS == 2 ? 3 : BITS == 3 ? 5 : BITS == 4 ? 9 : 0;
+    return 0;
+}
+
 template <int EPL, int SCHEME, bool FUSED, int BITS>
 cudaError_t launch_one(const KParams &p, cudaStream_t stream)
 {
     constexpr int D = 32 * EPL;
+    constexpr int SB = base_s_for<SCHEME, BITS>();
+    const bool bases = SB != 0 && p.fmt_s == SB;  // base-s messages (the plan checked s)
+    if (p.fmt_s != 0 && !bases) return cudaErrorInvalidValue;
     const int64_t nfull = p.tail == D ? p.nb : p.nb - 1;
     if (nfull > 0) {
         bool all_io = true;
         for (int w = 0; w < p.W; ++w) all_io = all_io && p.r[w] != nullptr && p.msg[w] != nullptr;
-        auto kern = all_io ? k_warp<EPL, SCHEME, FUSED, BITS, 3> : k_warp<EPL, SCHEME, FUSED, BITS, 0>;
+        auto kern = bases ? (all_io ? k_warp<EPL, SCHEME, FUSED, BITS, 3 | (SB << 2)> : k_warp<EPL, SCHEME, FUSED, BITS, (SB << 2)>)
+                          : (all_io ? k_warp<EPL, SCHEME, FUSED, BITS, 3> : k_warp<EPL, SCHEME, FUSED, BITS, 0>);
         const size_t smem = sizeof(WarpSmem<EPL, SCHEME>) * kWarpsPerCta;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -1049,7 +1084,7 @@ cudaError_t launch_one(const KParams &p, cudaStream_t stream)
     }
     if (nfull < p.nb) {
         using Fit = typename FitFor<SCHEME>::type;
-        auto tail = k_warp_tail<EPL, SCHEME, FUSED>;
+        auto tail = bases ? k_warp_tail<EPL, SCHEME, FUSED, (SB << 2)> : k_warp_tail<EPL, SCHEME, FUSED, 0>;
         const int nwarps = p.W < 16 ? p.W : 16;
         const size_t smem = sizeof(Fit) * nwarps + (FUSED ? (size_t)p.W * D * 4 : 0);
         cudaError_t e = cudaFuncSetAttribute(tail, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

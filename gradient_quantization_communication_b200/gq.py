@@ -13,6 +13,7 @@ LIB_PATH = os.path.join(_HERE, "libgq.so")
 GQ_QSGD, GQ_TERNGRAD, GQ_BINGRAD_B, GQ_BINGRAD_PB, GQ_ORQ, GQ_QSGD_NEAREST, GQ_SIGNSGD, GQ_QSGD_L2, GQ_TERNGRAD_LAYER = range(9)
 GQ_OK, GQ_ERR_INVALID, GQ_ERR_UNSUPPORTED, GQ_ERR_CUDA, GQ_ERR_NONFINITE, GQ_ERR_NOMEM, GQ_ERR_TIMEOUT = 0, 1, 2, 3, 4, 5, 6
 GQ_MAX_WORKERS = 64
+GQ_FORMAT_DENSE, GQ_FORMAT_BASE_S = 0, 1
 SCHEMES = {"qsgd": GQ_QSGD, "terngrad": GQ_TERNGRAD, "bingrad_b": GQ_BINGRAD_B,
            "bingrad_pb": GQ_BINGRAD_PB, "orq": GQ_ORQ, "qsgd_nearest": GQ_QSGD_NEAREST, "signsgd": GQ_SIGNSGD,
            "qsgd_l2": GQ_QSGD_L2, "terngrad_layer": GQ_TERNGRAD_LAYER}
@@ -55,6 +56,7 @@ def lib():
         L.gq_quant_error_noalloc.argtypes = [cfgp, ctypes.c_uint32, ctypes.c_uint64, vp, vp, vp, vp]
         L.gq_plan_status.argtypes = [vp, vp]
         L.gq_plan_set_segments.argtypes = [vp, ctypes.POINTER(ctypes.c_int64), ctypes.c_int]
+        L.gq_plan_set_format.argtypes = [vp, ctypes.c_int]
         L.gq_plan_message_layout.argtypes = [vp, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)]
         L.gq_selftest_bounded_wait.argtypes = [vp, ctypes.c_int64, vp]
         L.gq_entropy_layout.argtypes = [cfgp, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)]
@@ -70,7 +72,8 @@ def lib():
         L.gq_version.restype = ctypes.c_char_p
         for f in ("gq_config_check", "gq_message_layout", "gq_plan_create", "gq_plan_destroy", "gq_encode",
                   "gq_decode_accumulate", "gq_fused_step", "gq_quant_error", "gq_quant_error_noalloc",
-                  "gq_plan_status", "gq_plan_set_segments", "gq_plan_message_layout", "gq_selftest_bounded_wait", "gq_entropy_layout", "gq_entropy_pack",
+                  "gq_plan_status", "gq_plan_set_segments", "gq_plan_message_layout", "gq_plan_set_format",
+                  "gq_selftest_bounded_wait", "gq_entropy_layout", "gq_entropy_pack",
                   "gq_entropy_unpack", "gq_elias_layout", "gq_elias_used_bytes", "gq_elias_pack",
                   "gq_elias_unpack"):
             getattr(L, f).restype = ctypes.c_int
@@ -168,6 +171,10 @@ def gq_plan_set_segments(plan, offsets):
     _check(lib().gq_plan_set_segments(plan, arr, len(offsets) - 1), "gq_plan_set_segments")
 
 
+def gq_plan_set_format(plan, fmt):
+    _check(lib().gq_plan_set_format(plan, int(fmt)), "gq_plan_set_format")
+
+
 def gq_plan_message_layout(plan):
     b, c, l = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
     _check(lib().gq_plan_message_layout(plan, ctypes.byref(b), ctypes.byref(c), ctypes.byref(l)),
@@ -230,12 +237,15 @@ def gq_version():
 class Plan:
     """Owner of a gq_plan_t (destroyed on close / exit of a ``with`` block)."""
 
-    def __init__(self, cfg, segments=None):
-        """segments: the tensors' offsets (nseg + 1 values) for GQ_TERNGRAD_LAYER."""
+    def __init__(self, cfg, segments=None, fmt=GQ_FORMAT_DENSE):
+        """segments: the tensors' offsets (nseg + 1 values) for GQ_TERNGRAD_LAYER; fmt: the
+        message format (GQ_FORMAT_BASE_S: base-s messages written and read directly)."""
         self.cfg = cfg
         self.handle = gq_plan_create(cfg)
         if segments is not None:
             gq_plan_set_segments(self.handle, segments)
+        if fmt != GQ_FORMAT_DENSE:
+            gq_plan_set_format(self.handle, fmt)
         if cfg.scheme == GQ_TERNGRAD_LAYER and segments is None:
             self.msg_bytes = self.codes_off = self.levels_off = None
         else:

@@ -314,6 +314,22 @@ GQ_API gq_status_t gq_elias_unpack(const gq_config_t *cfg, const void *emsg, voi
 GQ_API gq_status_t gq_plan_set_segments(gq_plan_t plan, const int64_t *offsets, int nseg);
 GQ_API gq_status_t gq_plan_message_layout(gq_plan_t plan, size_t *bytes, size_t *codes_off, size_t *levels_off);
 
+/*
+ * The format of a plan's messages.  The review "[Paper Review] Optimal Gradient Quantization
+ * Condition for Communication-Efficient Distributed Training" ("Key findings") quotes compression
+ * ratios of 32 / log2(s); GQ_FORMAT_BASE_S is the message of gq_entropy_pack (g codes per B-bit
+ * base-s number, the level tables unchanged), written by gq_encode / gq_fused_step and read by
+ * gq_decode_accumulate directly, so that no dense message exists.  s = 3, 5 or 9 levels; ORQ and
+ * the QSGD family (QSGD, TernGrad, QSGD-nearest, QSGD-l2); d <= 512.
+ * gq_plan_set_format: GQ_FORMAT_DENSE (the default) or GQ_FORMAT_BASE_S; afterwards
+ * gq_plan_message_layout gives the message size and offsets (gq_entropy_layout's for base-s).
+ * GQ_ERR_UNSUPPORTED for a plan base-s does not cover, GQ_ERR_INVALID for an unknown format.
+ * Host only; no allocation.  gq_message_layout keeps describing the dense message.
+ */
+#define GQ_FORMAT_DENSE 0
+#define GQ_FORMAT_BASE_S 1
+GQ_API gq_status_t gq_plan_set_format(gq_plan_t plan, int format);
+
 /* Synchronize `stream`, then report and clear the plan's status flags: GQ_ERR_TIMEOUT if a
  * kernel's bounded wait for a bulk copy gave up (the kernel then stopped early; its outputs are
  * incomplete), else GQ_ERR_NONFINITE if a non-finite input was seen since the last call;

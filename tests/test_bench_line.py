@@ -72,3 +72,22 @@ def test_metric_name_follows_the_configuration():
     assert bench.metric_name(_args()) == bench.METRIC
     assert "signsgd-2 d=512" in bench.metric_name(_args("--scheme", "signsgd", "--levels", "2"))
     assert "orq-5 d=2048" in bench.metric_name(_args("--bucket", "2048"))
+
+
+@pytest.mark.parametrize("scheme,levels", [(4, 3), (4, 5), (4, 9), (0, 5), (1, 3)])
+@pytest.mark.parametrize("d", [128, 256, 512])
+def test_message_bytes_match_the_oracle_layouts(scheme, levels, d):
+    """The bench's message bytes per element, dense and base-s, times the elements of whole
+    buckets equal the oracle's message sizes without their 16-byte padding."""
+    import oracle as O
+    nb = 1000
+    co = O.Config(scheme, levels, d, 1, 1, 0.0, 0, nb * d)
+    L = O.table_len(scheme, levels)
+    dense = bench.message_bytes_per_elem(scheme, levels, d) * d * nb
+    assert dense == nb * d * ((levels - 1).bit_length()) / 8 + 4 * L * nb
+    assert O.message_layout(co)[0] - dense < 32
+    bases = bench.message_bytes_per_elem(scheme, levels, d, base_s=True) * d * nb
+    assert abs(bases - (nb * O.entropy_words(co) * 4 + 4 * L * nb)) < 1e-6
+    assert 0 <= O.entropy_layout(co)[0] - bases < 32
+    args = _args("--base-s", "--levels", str(levels))
+    assert args.base_s
