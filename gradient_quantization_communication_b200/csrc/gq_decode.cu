@@ -126,6 +126,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base(const __grid_
     const int nw = (int)p.codes_words;
     const bool has_level = slot < p.L;
     const float qr = (QSGD && slot < p.s) ? p.qratio[slot] : 0.0f;
+    __shared__ DigitTab<S> tab;
+    build_digit_tab<S>(tab);
+    __syncthreads();
     for (int64_t it = first; it < nitems; it += stride) {
         const int64_t e0 = it * (128 * CPI);
         const int64_t bk = e0 >> log2d;
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base(const __grid_
 #pragma unroll
             for (int c = 0; c < CPI; ++c) {
                 int code[4] = {0, 0, 0, 0};
-                if (c < nlive) base_codes4<S>(words, nw, eb + 128 * c, code);
+                if (c < nlive) base_codes4<S>(tab, words, nw, eb + 128 * c, code);
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, code[e], kWidth));

@@ -53,9 +53,10 @@ struct alignas(16) StageBuf {
 // A column collects at most 4 lanes x 16 values = 64 entries, so the fraction sum stays below
 // 64 * 2^16 = 2^22 and the count (<= 64) fits above it.
 constexpr int kHistCountShift = 22;
-// Words of a bucket's codes as bytes (base-s messages): 512 bytes and 32 bytes of zeros past
-// them for the last group's missing codes.
+// Base-s messages: the bucket's codes as bytes (512 bytes and 32 bytes of zeros past them for
+// the last group's missing codes), then the word buffer of its base-s words (at most 52).
 constexpr int kCodeBytesWords = 512 / 4 + 8;
+constexpr int kBaseOutWords = 56;
 struct alignas(16) FitORQ {
     uint32_t hist[64 * kHistCols];  // [cell][column]; cell 63 holds the values at the top grid point
     float4 ctab[64];                // cell -> {lower, upper, 1/(upper-lower), bracket}; 63 repeats 62
@@ -63,12 +64,12 @@ struct alignas(16) FitORQ {
     float lev[GQ_MAX_LEVELS];       // chosen levels in increasing order
     uint32_t P1[64];                // sum of positions over cells < k (< 2^31 for d <= 512)
     int P0[64];                     // count over cells < k
-    uint32_t codes[kCodeBytesWords];  // base-s messages: the bucket's codes as bytes (0 past d)
+    uint32_t codes[kCodeBytesWords + kBaseOutWords];  // base-s messages: codes as bytes, output words
 };
 struct alignas(16) FitQSGD {
     float2 pair[GQ_MAX_QSGD_LEVELS];  // {level k, level k+1}
     float qr[GQ_MAX_QSGD_LEVELS];     // the level ratios (2k - (s-1)) / (s-1), copied once
-    uint32_t codes[kCodeBytesWords];  // base-s messages: the bucket's codes as bytes (0 past d)
+    uint32_t codes[kCodeBytesWords + kBaseOutWords];  // base-s messages: codes as bytes, output words
 };
 struct alignas(16) FitPB {
     unsigned long long s1[64], s2[64];  // per cell: sum of positions, of squared positions
@@ -146,10 +147,7 @@ __device__ __forceinline__ void emit(const KParams &p, const R &rule, int64_t be
     if constexpr (kBaseS != 0) {
         if (kHasMsg || out) {
             __syncwarp();
-            constexpr int G = (32 * EPL + BaseS<kBaseS>::g - 1) / BaseS<kBaseS>::g;
-            const unsigned char *c8 = reinterpret_cast<const unsigned char *>(codes);
-            for (int k = lane; k < p.codes_words; k += 32) __stcs(out + k, base_word<kBaseS>(c8, k, G));
-            __syncwarp();
+            base_s_store<kBaseS, 32 * EPL>(codes, codes + kCodeBytesWords, out, (int)p.codes_words, lane);
         }
     }
 }
@@ -781,11 +779,11 @@ __device__ __forceinline__ void init_fit(const KParams &p, Fit &fit, int lane)
 {
     if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD || SCHEME == GQ_QSGD_NEAREST || SCHEME == GQ_QSGD_L2) {
         for (int k = lane; k < p.s; k += 32) fit.qr[k] = p.qratio[k];
-        for (int i = lane; i < kCodeBytesWords; i += 32) fit.codes[i] = 0u;
+        for (int i = lane; i < kCodeBytesWords + kBaseOutWords; i += 32) fit.codes[i] = 0u;
     }
     if constexpr (SCHEME == GQ_ORQ) {
         for (int i = lane; i < 64 * kHistCols; i += 32) fit.hist[i] = 0u;
-        for (int i = lane; i < kCodeBytesWords; i += 32) fit.codes[i] = 0u;
+        for (int i = lane; i < kCodeBytesWords + kBaseOutWords; i += 32) fit.codes[i] = 0u;
     }
     if constexpr (SCHEME == GQ_BINGRAD_PB) {
         for (int i = lane; i < 64; i += 32) {
