@@ -16,9 +16,9 @@
 // of word k / 32; the bits after T zero up to the next 16 bytes].
 //
 // Pack, five launches on the caller's stream:
-//   1. k_count: one warp per bucket writes its codeword bit count into its header slot (each
-//      lane over a contiguous run of codes held in a three-word register window, the next
-//      bucket's window loaded one bucket ahead).
+//   1. k_count: one thread per bucket writes its codeword bit count into its header slot; a warp
+//      copies its 32 buckets' dense words into shared rows with coalesced loads first, and each
+//      thread walks its row G codes per table lookup.
 //   2. k_tile_sums: one CTA per tile of 4096 buckets sums the counts into scratch, which is
 //      the message's level-table region (written last, by step 5).
 //   3. k_scan_top: one CTA turns the tile sums into exclusive prefix sums, writes T, and zeroes
@@ -26,13 +26,15 @@
 //      end.
 //   4. k_scan_apply: one CTA per tile writes each bucket's first bit and zeroes the stream word
 //      that a bucket shares with its predecessor.
-//   5. k_encode: one warp per bucket assembles its codewords in shared memory (each lane a
-//      contiguous run of elements, the run's words built in a 64-bit register), then stores
-//      the words that lie wholly inside the bucket's bit range and ORs the two shared ones
-//      (atomicOr on words zeroed by steps 3 and 4); the level table is copied.
-// Unpack: k_decode, one thread per bucket, reads its codewords from its first bit (one table
-// lookup on the next 7 bits per codeword) and writes the bucket's dense words; the level tables
-// are copied.  Count and encode take each code's codeword and length from 16-entry tables.
+//   5. k_encode: one thread per bucket (rows as in step 1) appends its codewords, G codes per
+//      table lookup, to a 64-bit bit buffer aligned to its first stream bit and stores each full
+//      word; the words it shares with its neighbours (the first and the last, when the bucket
+//      starts or ends inside a word) go by atomicOr onto words zeroed by steps 3 and 4; the level
+//      table is copied.
+// Unpack: k_decode, one thread per bucket, reads its codewords from its first bit (one lookup of
+// the next 8 bits decodes every codeword inside them) into the warp's shared rows, and the warp
+// writes 32 buckets' dense words at a time; the level tables are copied.  Count and encode take
+// the codewords and lengths of 2 or 4 codes at once from 256-entry tables.
 //
 // Robustness: codes >= s in a dense message are encoded as s - 1, so the stream never exceeds
 // the capacity; a damaged stream decodes to unspecified codes below 2^b, with every read inside
@@ -47,10 +49,8 @@
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kWarpThreads = 256;  // 8 warps per CTA for the per-bucket kernels
 constexpr int kTile = 4096;        // buckets per scan tile
 constexpr int kScanThreads = 1024; // 4 buckets per thread
-constexpr int kMaxStageWords = 512 * 7 / 32 + 4;  // d <= 512, at most 7 bits per code (s <= 15)
 
 struct ElParams {
     const uint32_t *dense;  // dense codes region
@@ -68,7 +68,17 @@ struct ElParams {
     unsigned long long len_tab;       // 4 bits per code
     // decoding: the next 7 stream bits -> code | length << 4 (one byte each)
     unsigned char dec[128];
+    // G = 8 / b codes (2 for b = 3) as one table index of G * b bits -> their codewords in stream
+    // order (bits 0 .. 23) | total length << 24
+    uint32_t enc[256];
+    // the next 8 stream bits -> the codewords that lie wholly inside them, decoded: their codes
+    // packed b bits each (bits 0 .. 31) | count << 32 | bits consumed << 40
+    unsigned long long dec8[256];
 };
+
+// codes per table index of the group tables
+template <int B>
+__host__ __device__ constexpr int group_codes() { return B == 3 ? 2 : 8 / B; }
 
 __device__ __forceinline__ int bucket_valid(const ElParams &p, int64_t bk) { return bk == p.nb - 1 ? p.tail : p.d; }
 
@@ -78,49 +88,94 @@ __device__ __forceinline__ uint32_t code_word(const ElParams &p, int c)
     return (uint32_t)(((c < 8 ? p.cw_lo : p.cw_hi) >> (8 * (c & 7))) & 0xFFu);
 }
 
-// A lane's run of d/32 consecutive codes (at most 64 bits) in a window of three dense words
-// starting at word q0 = floor(b * e0 / 32); words past the bucket's end read as 0.
-struct Run {
-    uint32_t w[3];
-    int base;  // bit offset of code e0 inside the window
-};
-__device__ __forceinline__ Run load_run(const ElParams &p, const uint32_t *bw, int e0)
-{
-    Run r;
-    const int bit = p.b * e0, q0 = bit >> 5;
-#pragma unroll
-    for (int k = 0; k < 3; ++k) r.w[k] = q0 + k < p.dw ? bw[q0 + k] : 0u;
-    r.base = bit & 31;
-    return r;
-}
-// code j of the run (the raw b bits; the tables map codes >= s to s - 1)
+// ---- 1. counts ----------------------------------------------------------------------------
+// One thread per bucket, a warp per 32 consecutive buckets: the warp copies the 32 buckets'
+// dense words (one contiguous span) into its shared rows with coalesced loads, then each thread
+// walks its row by table index (G codes at a time).
+constexpr int kBktWarps = 4;  // warps per CTA of the thread-per-bucket kernels
+
+// Group k (G codes, G * B bits) of a row of dense words.
 template <int B>
-__device__ __forceinline__ int run_code(const Run &r, int j)
+__device__ __forceinline__ uint32_t row_group(const uint32_t *row, int k)
 {
-    const int bit = r.base + B * j;
-    const uint64_t two = bit < 32 ? ((uint64_t)r.w[1] << 32) | r.w[0] : ((uint64_t)r.w[2] << 32) | r.w[1];
-    return (int)((uint32_t)(two >> (bit & 31)) & ((1u << B) - 1u));
+    constexpr int G = group_codes<B>(), NB = G * B;
+    if constexpr (NB == 8) {
+        return (row[k >> 2] >> (8 * (k & 3))) & 0xFFu;
+    } else {
+        const int bit = NB * k, w = bit >> 5, sh = bit & 31;
+        const uint32_t lo = row[w] >> sh;
+        const uint32_t hi = sh + NB > 32 ? row[w + 1] << (32 - sh) : 0u;
+        return (lo | hi) & ((1u << NB) - 1u);
+    }
+}
+// Code j of a row of dense words.
+template <int B>
+__device__ __forceinline__ int row_code(const uint32_t *row, int j)
+{
+    const int bit = B * j, w = bit >> 5, sh = bit & 31;
+    uint32_t x = row[w] >> sh;
+    if (sh + B > 32) x |= row[w + 1] << (32 - sh);
+    return (int)(x & ((1u << B) - 1u));
 }
 
-// ---- 1. counts ----------------------------------------------------------------------------
-template <int B>
-__global__ void __launch_bounds__(kWarpThreads) k_count(const __grid_constant__ ElParams p)
+// The warp's 32 buckets from bk0 into rows [32][dw + 1] (the pad word stays 0).  The buckets'
+// words are one contiguous span (dw is a multiple of 4): 16-byte loads, eight in flight per lane
+// before any is stored.
+__device__ __forceinline__ void load_rows(const ElParams &p, uint32_t *rows, int64_t bk0, int lane)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t nwarps = (int64_t)gridDim.x * (kWarpThreads / 32);
-    const int per_lane = p.d / 32, e0 = lane * per_lane;
-    int64_t bk = (int64_t)blockIdx.x * (kWarpThreads / 32) + (threadIdx.x >> 5);
-    Run nr{};
-    if (bk < p.nb) nr = load_run(p, p.dense + bk * p.dw, e0);
-    for (; bk < p.nb; bk += nwarps) {
-        const Run r = nr;
-        const int64_t nx = bk + nwarps;
-        if (nx < p.nb) nr = load_run(p, p.dense + nx * p.dw, e0);  // one bucket ahead
-        const int cnt = min(per_lane, bucket_valid(p, bk) - e0);
-        int bits = 0;
-        for (int j = 0; j < cnt; ++j) bits += code_len(p, run_code<B>(r, j));
-        bits = __reduce_add_sync(kFull, (unsigned)bits);
-        if (lane == 0) p.offs[bk] = (uint64_t)bits;
+    const int dw = p.dw, rs = p.dw + 1;
+    const int nrows = (int)min((int64_t)32, p.nb - bk0);
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.dense + bk0 * dw);
+    const int nq = nrows * dw / 4;
+    for (int i0 = 0; i0 < nq; i0 += 8 * 32) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + 32 * u + lane;
+            if (i < nq) v[u] = __ldg(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + 32 * u + lane;
+            if (i < nq) {
+                const int w = 4 * i, r = w / dw, c = w - r * dw;
+                uint32_t *d = rows + r * rs + c;
+                d[0] = v[u].x;
+                d[1] = v[u].y;
+                d[2] = v[u].z;
+                d[3] = v[u].w;
+            }
+        }
+    }
+    if (lane < nrows) rows[lane * rs + dw] = 0u;
+}
+
+template <int B>
+__global__ void __launch_bounds__(kBktWarps * 32) k_count(const __grid_constant__ ElParams p)
+{
+    constexpr int G = group_codes<B>();
+    __shared__ uint32_t enc[256];
+    extern __shared__ uint32_t rows_all[];  // [warps][32][dw + 1]
+    for (int i = threadIdx.x; i < (1 << (G * B)); i += blockDim.x) enc[i] = p.enc[i];
+    __syncthreads();
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int rs = p.dw + 1;
+    uint32_t *rows = rows_all + wid * 32 * rs;
+    const uint32_t *row = rows + lane * rs;
+    const int64_t nwarps = (int64_t)gridDim.x * kBktWarps;
+    for (int64_t bk0 = ((int64_t)blockIdx.x * kBktWarps + wid) * 32; bk0 < p.nb; bk0 += nwarps * 32) {
+        load_rows(p, rows, bk0, lane);
+        __syncwarp();
+        const int64_t bk = bk0 + lane;
+        if (bk < p.nb) {
+            const int n = bucket_valid(p, bk);
+            const int ng = n / G;
+            int bits = 0;
+            for (int k = 0; k < ng; ++k) bits += (int)(enc[row_group<B>(row, k)] >> 24);
+            for (int j = ng * G; j < n; ++j) bits += code_len(p, row_code<B>(row, j));
+            p.offs[bk] = (uint64_t)bits;
+        }
+        __syncwarp();
     }
 }
 
@@ -223,84 +278,64 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_apply(const __grid_consta
 }
 
 // ---- 5. encode ----------------------------------------------------------------------------
+// One thread per bucket (rows as in the count): the thread appends its codewords, G codes per
+// table lookup, to a 64-bit bit buffer that starts at its bucket's first stream bit and stores
+// each full word.  The first word is shared with the previous bucket when the bucket starts
+// inside a word, the last with the next one when it ends inside one: those go by atomicOr onto
+// the words the scan zeroed; every other word belongs to this bucket alone.
 template <int B>
-__global__ void __launch_bounds__(kWarpThreads) k_encode(const __grid_constant__ ElParams p, int pad_floats)
+__global__ void __launch_bounds__(kBktWarps * 32) k_encode(const __grid_constant__ ElParams p, int pad_floats)
 {
-    __shared__ uint32_t stage_all[kWarpThreads / 32][kMaxStageWords];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    constexpr int G = group_codes<B>();
+    __shared__ uint32_t enc[256];
+    extern __shared__ uint32_t rows_all[];
+    for (int i = threadIdx.x; i < (1 << (G * B)); i += blockDim.x) enc[i] = p.enc[i];
+    __syncthreads();
     // padding of the level-table region (it held the scan's tile sums)
     if (blockIdx.x == 0 && (int)threadIdx.x < pad_floats) p.etab[p.nb * p.L + threadIdx.x] = 0.0f;
-    uint32_t *st = stage_all[wid];
-    const int64_t nwarps = (int64_t)gridDim.x * (kWarpThreads / 32);
-    const int per_lane = p.d / 32;
-    const int e0 = lane * per_lane;
-    // software pipeline: the next bucket's code window, first bit and table entry are loaded
-    // before this bucket is written, so the warp waits on one round trip per bucket, not three
-    int64_t bk = (int64_t)blockIdx.x * (kWarpThreads / 32) + wid;
-    Run nr{};
-    uint64_t noff = 0;
-    float ntab = 0.0f;
-    if (bk < p.nb) {
-        nr = load_run(p, p.dense + bk * p.dw, e0);
-        noff = p.offs[bk];
-        if (lane < p.L) ntab = p.dtab[bk * p.L + lane];
-    }
-    for (; bk < p.nb; bk += nwarps) {
-        const Run rr = nr;
-        const uint64_t off = noff;
-        const float tab = ntab;
-        const int64_t nx = bk + nwarps;
-        if (nx < p.nb) {
-            nr = load_run(p, p.dense + nx * p.dw, e0);
-            noff = p.offs[nx];
-            if (lane < p.L) ntab = p.dtab[nx * p.L + lane];
-        }
-        const int n = bucket_valid(p, bk);
-        const int cnt = min(per_lane, n - e0);
-        int bits = 0;
-        for (int j = 0; j < cnt; ++j) bits += code_len(p, run_code<B>(rr, j));
-        int incl = bits;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += y;
-        }
-        const int total = __shfl_sync(kFull, incl, 31);
-        const int base = (int)(off & 31u);
-        const int nw = (base + total + 31) >> 5;
-        for (int j = lane; j < nw; j += 32) st[j] = 0u;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int rs = p.dw + 1;
+    uint32_t *rows = rows_all + wid * 32 * rs;
+    const uint32_t *row = rows + lane * rs;
+    const int64_t nwarps = (int64_t)gridDim.x * kBktWarps;
+    for (int64_t bk0 = ((int64_t)blockIdx.x * kBktWarps + wid) * 32; bk0 < p.nb; bk0 += nwarps * 32) {
+        load_rows(p, rows, bk0, lane);
         __syncwarp();
-        if (bits > 0) {
-            const int pos = base + incl - bits;  // this lane's first bit in the stage
-            int wi = pos >> 5, accbits = pos & 31;
+        const int64_t bk = bk0 + lane;
+        if (bk < p.nb) {
+            const int n = bucket_valid(p, bk);
+            const int ng = n / G;
+            const uint64_t off = p.offs[bk];
+            uint32_t *wp = p.stream + (off >> 5);
+            int accbits = (int)(off & 31u);
+            bool shared_first = accbits != 0;
             uint64_t acc = 0;
-            bool first = true;
-            for (int j = 0; j < cnt; ++j) {
-                const int c = run_code<B>(rr, j);
+            auto flush = [&]() {
+                if (shared_first) atomicOr(wp, (uint32_t)acc);
+                else *wp = (uint32_t)acc;
+                shared_first = false;
+                ++wp;
+                acc >>= 32;
+                accbits -= 32;
+            };
+            for (int k = 0; k < ng; ++k) {
+                const uint32_t e = enc[row_group<B>(row, k)];
+                acc |= (uint64_t)(e & 0xFFFFFFu) << accbits;
+                accbits += (int)(e >> 24);
+                if (accbits >= 32) flush();
+            }
+            for (int j = ng * G; j < n; ++j) {
+                const int c = row_code<B>(row, j);
                 acc |= (uint64_t)code_word(p, c) << accbits;
                 accbits += code_len(p, c);
-                if (accbits >= 32) {
-                    if (first) atomicOr(&st[wi], (uint32_t)acc);
-                    else st[wi] = (uint32_t)acc;
-                    first = false;
-                    ++wi;
-                    acc >>= 32;
-                    accbits -= 32;
-                }
+                if (accbits >= 32) flush();
             }
-            if (accbits > 0) atomicOr(&st[wi], (uint32_t)acc);  // may be shared with the next lane
+            if (accbits > 0) atomicOr(wp, (uint32_t)acc);  // may be shared with the next bucket
+            if (p.L > 0) {
+                for (int k = 0; k < p.L; ++k) p.etab[bk * p.L + k] = p.dtab[bk * p.L + k];
+            }
         }
         __syncwarp();
-        const int64_t w0 = (int64_t)(off >> 5);
-        const uint64_t end = off + (uint64_t)total;
-        for (int j = lane; j < nw; j += 32) {
-            const int64_t gw = w0 + j;
-            const bool whole = (uint64_t)gw * 32 >= off && (uint64_t)gw * 32 + 32 <= end;
-            if (whole) p.stream[gw] = st[j];
-            else atomicOr(&p.stream[gw], st[j]);
-        }
-        if (lane < p.L) p.etab[bk * p.L + lane] = tab;
-        __syncwarp();  // the stage is reused by the next bucket
     }
 }
 
@@ -310,52 +345,131 @@ __device__ __forceinline__ uint32_t stream_word(const ElParams &p, int64_t q)
     return q < p.cap_words ? __ldg(p.stream + q) : 0u;
 }
 
-// One thread per bucket.  The thread reads its stream through a 64-bit bit buffer refilled a
-// word at a time, with the next word's load issued one refill ahead, and decodes one codeword
-// per lookup: the next 7 stream bits index a 128-entry shared table (code, length).
+// One thread per bucket, a warp per 32 consecutive buckets.  The thread reads its stream through
+// a 64-bit bit buffer refilled a word at a time, with the next word's load issued one refill
+// ahead.  While at least 8 codes remain, one lookup of the next 8 stream bits decodes every
+// codeword that lies wholly inside them (dec8); the rest go one codeword per lookup of the next
+// 7 bits (dec).  The thread builds its bucket's dense words in its row of the warp's shared
+// buffer (rows of dw + 1 words, so that the lanes' stores hit distinct banks); the warp then
+// writes the 32 buckets' words, which are contiguous in the dense message, row by row with
+// coalesced stores.
+constexpr int kDecodeWarps = 4;
+constexpr int kStreamStage = 1024;  // stream words a warp stages for its 32 buckets (4 KB)
+
+// The codes of one bucket from its first stream bit: rd(q) reads stream word q.
+template <int B, class Rd>
+__device__ __forceinline__ void decode_bucket(const unsigned char *dec, const unsigned long long *dec8, uint64_t start,
+                                              int n, int dw, uint32_t *out, const Rd &rd)
+{
+    int64_t q = (int64_t)(start >> 5);
+    const int sh = (int)(start & 31u);
+    uint64_t buf = ((uint64_t)rd(q) | ((uint64_t)rd(q + 1) << 32)) >> sh;
+    int nbuf = 64 - sh;
+    q += 2;
+    uint32_t next = rd(q);
+    uint64_t acc = 0;
+    int accbits = 0, wi = 0;
+    int e = 0;
+    for (; e + 8 <= n;) {
+        if (nbuf < 32) {
+            buf |= (uint64_t)next << nbuf;
+            nbuf += 32;
+            next = rd(++q);
+        }
+        const unsigned long long t = dec8[(uint32_t)buf & 255u];
+        const int cnt = (int)((t >> 32) & 15u), len = (int)((t >> 40) & 15u);
+        buf >>= len;
+        nbuf -= len;
+        acc |= (t & 0xFFFFFFFFull) << accbits;
+        accbits += B * cnt;
+        e += cnt;
+        if (accbits >= 32) {
+            out[wi++] = (uint32_t)acc;
+            acc >>= 32;
+            accbits -= 32;
+        }
+    }
+    for (; e < n; ++e) {
+        if (nbuf < 32) {  // refill: a codeword has at most 7 bits
+            buf |= (uint64_t)next << nbuf;
+            nbuf += 32;
+            next = rd(++q);
+        }
+        const unsigned t = dec[(uint32_t)buf & 127u];
+        const int len = (int)(t >> 4);
+        buf >>= len;
+        nbuf -= len;
+        acc |= (uint64_t)(t & 15u) << accbits;
+        accbits += B;
+        if (accbits >= 32) {
+            out[wi++] = (uint32_t)acc;
+            acc >>= 32;
+            accbits -= 32;
+        }
+    }
+    if (accbits > 0) out[wi++] = (uint32_t)acc;
+    for (; wi < dw; ++wi) out[wi] = 0u;  // padding codes of a ragged last bucket
+}
+
+// One thread per bucket, a warp per 32 consecutive buckets.  Their stream bits are one span:
+// when it fits in kStreamStage words the warp first copies it into shared memory with coalesced
+// loads, else the threads read global memory.  A thread reads its codewords through a 64-bit
+// bit buffer; while at least 8 codes remain, one lookup of the next 8 stream bits decodes every
+// codeword that lies wholly inside them (dec8), the rest go one codeword per lookup of the next
+// 7 bits (dec).  The thread builds its bucket's dense words in its row of the warp's shared
+// buffer (rows of dw + 1 words, so that the lanes' stores hit distinct banks); the warp then
+// writes the 32 buckets' words, which are contiguous in the dense message, row by row with
+// coalesced stores.
 template <int B>
-__global__ void __launch_bounds__(256) k_decode(const __grid_constant__ ElParams p, float *dtab_out,
-                                                uint32_t *dense_out, int pad_floats)
+__global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_constant__ ElParams p, float *dtab_out,
+                                                              uint32_t *dense_out, int pad_floats)
 {
     __shared__ unsigned char dec[128];
+    __shared__ unsigned long long dec8[256];
+    __shared__ uint32_t stage_all[kDecodeWarps][kStreamStage];
+    extern __shared__ uint32_t rows_all[];  // [warps][32][dw + 1]
     if (threadIdx.x < 128) dec[threadIdx.x] = p.dec[threadIdx.x];
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) dec8[i] = p.dec8[i];
     __syncthreads();
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int dw = p.dw, rs = p.dw + 1;
+    uint32_t *rows = rows_all + wid * 32 * rs;
+    uint32_t *out = rows + lane * rs;
+    uint32_t *stage = stage_all[wid];
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
     for (int64_t j = tid; j < p.nb * p.L; j += nthreads) dtab_out[j] = p.etab[j];
     if (tid < pad_floats) dtab_out[p.nb * p.L + tid] = 0.0f;
-    for (int64_t bk = tid; bk < p.nb; bk += nthreads) {
-        const int n = bucket_valid(p, bk);
-        uint32_t *out = dense_out + bk * p.dw;
-        const uint64_t start = p.offs[bk];
-        int64_t q = (int64_t)(start >> 5);
-        const int sh = (int)(start & 31u);
-        uint64_t buf = ((uint64_t)stream_word(p, q) | ((uint64_t)stream_word(p, q + 1) << 32)) >> sh;
-        int nbuf = 64 - sh;
-        q += 2;
-        uint32_t next = stream_word(p, q);
-        uint64_t acc = 0;
-        int accbits = 0, wi = 0;
-        for (int e = 0; e < n; ++e) {
-            if (nbuf < 32) {  // refill: a codeword has at most 7 bits
-                buf |= (uint64_t)next << nbuf;
-                nbuf += 32;
-                next = stream_word(p, ++q);
-            }
-            const unsigned t = dec[(uint32_t)buf & 127u];
-            const int len = (int)(t >> 4);
-            buf >>= len;
-            nbuf -= len;
-            acc |= (uint64_t)(t & 15u) << accbits;
-            accbits += B;
-            if (accbits >= 32) {
-                out[wi++] = (uint32_t)acc;
-                acc >>= 32;
-                accbits -= 32;
+    const int64_t nwarps = (int64_t)gridDim.x * kDecodeWarps;
+    for (int64_t bk0 = ((int64_t)blockIdx.x * kDecodeWarps + wid) * 32; bk0 < p.nb; bk0 += nwarps * 32) {
+        const int nrows = (int)min((int64_t)32, p.nb - bk0);
+        // the span of stream words the 32 decoders read: from the first bucket's first word to
+        // the word after the last bucket's end, plus the two a bit buffer reads ahead
+        const uint64_t s0 = p.offs[bk0];
+        const uint64_t s1 = bk0 + nrows < p.nb ? p.offs[bk0 + nrows] : p.hdr[0];
+        const int64_t w0 = (int64_t)(s0 >> 5);
+        const int64_t w1 = min((int64_t)((s1 + 31) >> 5) + 4, p.cap_words);
+        const bool staged = w1 - w0 <= kStreamStage;
+        if (staged) {
+            for (int64_t i = w0 + lane; i < w1; i += 32) stage[i - w0] = __ldg(p.stream + i);
+        }
+        __syncwarp();
+        const int64_t bk = bk0 + lane;
+        if (bk < p.nb) {
+            const int n = bucket_valid(p, bk);
+            const uint64_t start = p.offs[bk];
+            if (staged) {
+                decode_bucket<B>(dec, dec8, start, n, dw, out,
+                                 [&](int64_t q) { return q < w1 ? stage[q - w0] : 0u; });
+            } else {
+                decode_bucket<B>(dec, dec8, start, n, dw, out, [&](int64_t q) { return stream_word(p, q); });
             }
         }
-        if (accbits > 0) out[wi++] = (uint32_t)acc;
-        for (; wi < p.dw; ++wi) out[wi] = 0u;  // padding codes of a ragged last bucket
+        __syncwarp();
+        uint32_t *dst = dense_out + bk0 * dw;
+        for (int r = 0; r < nrows; ++r)
+            for (int j = lane; j < dw; j += 32) dst[r * dw + j] = rows[r * rs + j];
+        __syncwarp();
     }
 }
 
@@ -461,16 +575,53 @@ ElParams make_params(const gq_config_t *cfg, const ElLayout &l, const void *msg,
         }
         p.dec[t] = (unsigned char)(code | (len << 4));
     }
+    // group encoding table: G codes of one index, their codewords one after the other
+    const int G = l.b == 3 ? 2 : 8 / l.b;
+    for (int idx = 0; idx < 256; ++idx) {
+        uint32_t bitsv = 0;
+        int len = 0;
+        if (idx < (1 << (G * l.b))) {
+            for (int k = 0; k < G; ++k) {
+                const int c = (idx >> (l.b * k)) & ((1 << l.b) - 1);
+                const uint32_t cw = (uint32_t)(((c < 8 ? p.cw_lo : p.cw_hi) >> (8 * (c & 7))) & 0xFFu);
+                bitsv |= cw << len;
+                len += (int)((p.len_tab >> (4 * c)) & 15u);
+            }
+        }
+        p.enc[idx] = bitsv | ((uint32_t)len << 24);
+    }
+    // multi-codeword decoding table over 8 stream bits: decode as the single table does while the
+    // next codeword lies wholly inside the 8 bits (the first one always does: a codeword has at
+    // most 7 bits, and a pattern that starts none takes 7)
+    for (int t = 0; t < 256; ++t) {
+        int pos = 0, cnt = 0;
+        unsigned long long codes = 0;
+        while (pos < 8) {
+            const int u = (t >> pos) & 127;  // the next 7 bits (zeros past the window)
+            const int c = p.dec[u] & 15, len = p.dec[u] >> 4;
+            if (pos + len > 8) break;
+            // the single table saw zeros past bit 8: accept its answer only if the codeword's
+            // bits all lie inside the window
+            codes |= (unsigned long long)c << (l.b * cnt);
+            ++cnt;
+            pos += len;
+        }
+        p.dec8[t] = codes | ((unsigned long long)cnt << 32) | ((unsigned long long)pos << 40);
+    }
     return p;
 }
 
-int warp_grid(int64_t nb)
+// Grid of a thread-per-bucket kernel (warps of 32 buckets, kBktWarps per CTA): the resident CTAs
+// or fewer; -1 if the shared memory cannot be granted.
+int bucket_grid(const void *kern, int64_t nb, size_t smem)
 {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        sms = 148;
-    const int64_t want = (nb + kWarpThreads / 32 - 1) / (kWarpThreads / 32);
-    return (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * (2048 / kWarpThreads)));
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return -1;
+    int dev = 0, sms = 148, per_sm = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBktWarps * 32, smem);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t want = (nb + 32 * kBktWarps - 1) / (32 * kBktWarps);
+    return (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * per_sm));
 }
 
 struct Range {
@@ -518,15 +669,18 @@ gq_status_t gq_elias_pack(const gq_config_t *cfg, const void *msg, void *emsg, v
     if (i0 < o0 + l.cap && o0 < i0 + l.dense_bytes) return GQ_ERR_INVALID;
     const ElParams p = make_params(cfg, l, msg, emsg);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int g = warp_grid(l.nb);
     auto count = l.b == 2 ? k_count<2> : l.b == 3 ? k_count<3> : k_count<4>;
     auto encode = l.b == 2 ? k_encode<2> : l.b == 3 ? k_encode<3> : k_encode<4>;
-    count<<<g, kWarpThreads, 0, s>>>(p);
+    const size_t smem = sizeof(uint32_t) * kBktWarps * 32 * (size_t)(p.dw + 1);
+    const int gc = bucket_grid(reinterpret_cast<const void *>(count), l.nb, smem);
+    const int ge = bucket_grid(reinterpret_cast<const void *>(encode), l.nb, smem);
+    if (gc < 0 || ge < 0) return GQ_ERR_CUDA;
+    count<<<gc, kBktWarps * 32, smem, s>>>(p);
     k_tile_sums<<<(unsigned)p.ntiles, kScanThreads, 0, s>>>(p);
     k_scan_top<<<1, kScanThreads, 0, s>>>(p);
     k_scan_apply<<<(unsigned)p.ntiles, kScanThreads, 0, s>>>(p);
     const int64_t tab = l.nb * l.L;
-    encode<<<g, kWarpThreads, 0, s>>>(p, (int)(((tab + 3) & ~int64_t(3)) - tab));
+    encode<<<ge, kBktWarps * 32, smem, s>>>(p, (int)(((tab + 3) & ~int64_t(3)) - tab));
     return cudaGetLastError() == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
 }
 
@@ -546,9 +700,16 @@ gq_status_t gq_elias_unpack(const gq_config_t *cfg, const void *emsg, void *msg,
     const int pad = (int)(((tab + 3) & ~int64_t(3)) - tab);
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((l.nb + 255) / 256, (int64_t)sms * 8));
     auto decode = l.b == 2 ? k_decode<2> : l.b == 3 ? k_decode<3> : k_decode<4>;
-    decode<<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+    const size_t smem = sizeof(uint32_t) * kDecodeWarps * 32 * (size_t)(p.dw + 1);
+    if (cudaFuncSetAttribute(decode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GQ_ERR_CUDA;
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode, kDecodeWarps * 32, smem);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t want = (l.nb + 32 * kDecodeWarps - 1) / (32 * kDecodeWarps);
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * per_sm));
+    decode<<<(unsigned)grid, kDecodeWarps * 32, smem, static_cast<cudaStream_t>(stream)>>>(
         p, reinterpret_cast<float *>(m + l.dense_levels_off), reinterpret_cast<uint32_t *>(m), pad);
     return cudaGetLastError() == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
 }
