@@ -4,8 +4,9 @@
 //
 // Included by gq_group_orq.cu and gq_group_qsgd.cu (one scheme each, compiled in parallel).
 //
-// CTAs of 8 warps.  For G <= 8 a CTA holds 8 / G groups, each synchronised by its own named
-// barrier.  For G > 8 a bucket takes a cluster of C = G / 8 CTAs (d = 8192: 2, 16384: 4,
+// CTAs of NW warps: 4 for d <= 2048, 8 above.  Up to NW warps a CTA holds NW / G groups, each
+// synchronised by its own named barrier (d = 1024: two per CTA of 4, 2048: one, 4096: one per CTA
+// of 8).  For G > 8 a bucket takes a cluster of C = G / 8 CTAs (d = 8192: 2, 16384: 4,
 // 32768: 8), synchronised by cluster barriers, and the statistics cross CTAs through
 // distributed shared memory (plain loads of the peer CTA's shared memory; no multicast).
 // Only what the fit needs crosses warps:
@@ -36,7 +37,10 @@
 namespace gq {
 namespace {
 
-constexpr int kGroupWarps = 8;  // warps per CTA
+// Warps per CTA: 4 for G <= 4 (one or two groups per CTA; more CTAs per SM hide the groups'
+// barrier waits better, measured 5 % faster at d = 2048), 8 above (clusters of G / 8 CTAs; with 4
+// the clusters of d = 32768 would take 16 CTAs, measured 20-30 % slower).
+template <int G> constexpr int group_cta_warps() { return G <= 4 ? 4 : 8; }
 constexpr int kSliceEPL = 16;   // values per lane: a warp holds 512 values
 
 struct alignas(16) FitGroupORQ {
@@ -60,10 +64,11 @@ struct alignas(16) GroupWarpSmem {
 };
 
 // The CTA's exchange slots, [item parity][...].
+template <int NW>
 struct alignas(16) GroupXchg {
-    float2 stat[2][kGroupWarps];            // per warp: {min, max} (ORQ) or {max |u|, 0} (QSGD)
-    int fail[2][kGroupWarps];               // per warp: its copy timed out
-    uint4 cells[2][kGroupWarps][32];        // per warp and lane l: counts and position sums of cells 2l, 2l+1
+    float2 stat[2][NW];            // per warp: {min, max} (ORQ) or {max |u|, 0} (QSGD)
+    int fail[2][NW];               // per warp: its copy timed out
+    uint4 cells[2][NW][32];        // per warp and lane l: counts and position sums of cells 2l, 2l+1
     unsigned long long cta_s[2][32][2];     // clusters: the CTA's sums of cells 2l, 2l+1
     unsigned int cta_c[2][32][2];           // clusters: the CTA's counts
 };
@@ -147,9 +152,10 @@ __device__ __forceinline__ void group_orq_tables(const KParams &p, FitGroupORQ &
 }
 
 // Buckets b0 .. b1-1 (TAIL: the ragged last bucket alone, b0 = nb - 1, b1 = nb).
-template <int SCHEME, int G, bool FUSED, bool TAIL>
-__global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_constant__ KParams p, int64_t b0, int64_t b1)
+template <int SCHEME, int G, int NW, bool FUSED, bool TAIL>
+__global__ void __launch_bounds__(NW * 32, 16 / NW) k_group(const __grid_constant__ KParams p, int64_t b0, int64_t b1)
 {
+    constexpr int kGroupWarps = NW;
     constexpr int C = G > kGroupWarps ? G / kGroupWarps : 1;    // CTAs per bucket
     constexpr int GPC = G < kGroupWarps ? kGroupWarps / G : 1;  // groups per CTA
     constexpr int EPL = kSliceEPL;
@@ -157,9 +163,9 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
     constexpr unsigned kBytes = 32 * EPL * 4;
     using Smem = GroupWarpSmem<SCHEME>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    GroupXchg &xg = *reinterpret_cast<GroupXchg *>(smem_raw);
+    GroupXchg<NW> &xg = *reinterpret_cast<GroupXchg<NW> *>(smem_raw);
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    Smem &sm = reinterpret_cast<Smem *>(smem_raw + sizeof(GroupXchg))[wib];
+    Smem &sm = reinterpret_cast<Smem *>(smem_raw + sizeof(GroupXchg<NW>))[wib];
     const int gid = C > 1 ? 0 : wib / G;                                         // group within the CTA
     const uint32_t crank = C > 1 ? (uint32_t)(blockIdx.x % C) : 0u;             // CTA within the cluster
     const int rk = C > 1 ? (int)crank * kGroupWarps + wib : wib % G;           // warp within the group
@@ -390,7 +396,7 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
                 const int bar_n = 32 * (C > 1 ? kGroupWarps : G);
                 const int wfirst = C > 1 ? 0 : gid * G;  // the first warp of the group in this CTA
                 const bool leads = wib == wfirst;
-                Smem &lead = reinterpret_cast<Smem *>(smem_raw + sizeof(GroupXchg))[wfirst];
+                Smem &lead = reinterpret_cast<Smem *>(smem_raw + sizeof(GroupXchg<NW>))[wfirst];
                 named_bar(bar_id, bar_n);
                 unsigned int C0 = 0u, C1 = 0u;
                 unsigned long long S0 = 0ull, S1 = 0ull;
@@ -490,13 +496,14 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 2) k_group(const __grid_cons
 template <int SCHEME, int G, bool FUSED, bool TAIL>
 cudaError_t launch_group_g(const KParams &p0, int64_t b0, int64_t b1, cudaStream_t stream)
 {
+    constexpr int kGroupWarps = group_cta_warps<G>();
     constexpr int C = G > kGroupWarps ? G / kGroupWarps : 1;
     constexpr int GPC = G < kGroupWarps ? kGroupWarps / G : 1;
     KParams p = p0;
     p.codes_words = (int64_t)(32 * kSliceEPL) * p.bits / 32;  // code words of one 512-element slice
-    auto kern = k_group<SCHEME, G, FUSED, TAIL>;
+    auto kern = k_group<SCHEME, G, kGroupWarps, FUSED, TAIL>;
     const int64_t nbk = b1 - b0;
-    const size_t smem = sizeof(GroupXchg) + sizeof(GroupWarpSmem<SCHEME>) * kGroupWarps;
+    const size_t smem = sizeof(GroupXchg<kGroupWarps>) + sizeof(GroupWarpSmem<SCHEME>) * kGroupWarps;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
