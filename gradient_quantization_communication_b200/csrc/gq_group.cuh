@@ -4,11 +4,11 @@
 //
 // Included by gq_group_orq.cu and gq_group_qsgd.cu (one scheme each, compiled in parallel).
 //
-// CTAs of NW warps: 4 for d <= 2048, 8 above.  Up to NW warps a CTA holds NW / G groups, each
-// synchronised by its own named barrier (d = 1024: two per CTA of 4, 2048: one, 4096: one per CTA
-// of 8).  For G > 8 a bucket takes a cluster of C = G / 8 CTAs (d = 8192: 2, 16384: 4,
-// 32768: 8), synchronised by cluster barriers, and the statistics cross CTAs through
-// distributed shared memory (plain loads of the peer CTA's shared memory; no multicast).
+// CTAs of NW warps: 4 for d <= 2048, 8 for 4096, 16 above.  Up to NW warps a CTA holds NW / G
+// groups, each synchronised by its own named barrier (d = 1024: two per CTA of 4; 2048, 4096 and
+// 8192: one).  For G > NW a bucket takes a cluster of C = G / NW CTAs (d = 16384: 2, 32768: 4),
+// synchronised by cluster barriers, and the statistics cross CTAs through distributed shared
+// memory (plain loads of the peer CTA's shared memory; no multicast).
 // Only what the fit needs crosses warps:
 //   QSGD / TernGrad : each warp's max |u| -> the group's max (one exchange);
 //   ORQ             : each warp's min and max -> the group's; then each warp's 64 cell counts
@@ -38,9 +38,10 @@ namespace gq {
 namespace {
 
 // Warps per CTA: 4 for G <= 4 (one or two groups per CTA; more CTAs per SM hide the groups'
-// barrier waits better, measured 5 % faster at d = 2048), 8 above (clusters of G / 8 CTAs; with 4
-// the clusters of d = 32768 would take 16 CTAs, measured 20-30 % slower).
-template <int G> constexpr int group_cta_warps() { return G <= 4 ? 4 : 8; }
+// barrier waits better: 5 % faster at d = 2048 than 8), 8 for G = 8, and 16 from G = 16 on (one
+// CTA per SM and per d = 8192 bucket, clusters of 2 and 4 CTAs for 16384 and 32768: 20 % faster
+// at d = 8192 than clusters of two 8-warp CTAs, 3-5 % at 32768).
+template <int G> constexpr int group_cta_warps() { return G <= 4 ? 4 : (G >= 16 ? 16 : 8); }
 constexpr int kSliceEPL = 16;   // values per lane: a warp holds 512 values
 
 struct alignas(16) FitGroupORQ {
