@@ -272,7 +272,7 @@ __device__ __forceinline__ void prefetch_l2(const void *p, unsigned bytes)
 
 // ERR: the error mode of gq_quant_error; nothing is written but part[3 * bucket + k].
 template <int SCHEME, bool ERR, int NW>
-__global__ void __launch_bounds__(NW * 32) k_cta(const __grid_constant__ KParams p, double *part, int64_t first)
+__global__ void __launch_bounds__(NW * 32) k_cta(const __grid_constant__ KParams p, double *part)
 {
     constexpr int kCtaWarps = NW, kCtaThreads = NW * 32;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(NW * 32) k_cta(const __grid_constant__ KParams
     const int W = p.W;
 
     ErrAcc ea{0.0, 0.0, 0.0};
-    for (int64_t beta = first + blockIdx.x; beta < p.nb; beta += gridDim.x) {
+    for (int64_t beta = blockIdx.x; beta < p.nb; beta += gridDim.x) {
       const int64_t base = beta * (int64_t)d;
       const int nvalid = (beta == p.nb - 1) ? p.tail : d;
       for (int w = 0; w < W; ++w) {
@@ -747,7 +747,7 @@ __global__ void __launch_bounds__(NW * 32) k_cta(const __grid_constant__ KParams
 }
 
 template <int SCHEME, bool ERR, int NW>
-cudaError_t launch(const KParams &p, double *part, int64_t first, cudaStream_t stream)
+cudaError_t launch(const KParams &p, double *part, cudaStream_t stream)
 {
     auto kern = k_cta<SCHEME, ERR, NW>;
     const bool acc_smem = !ERR && p.avg != nullptr && p.d <= kAccSmemMax;
@@ -761,36 +761,35 @@ cudaError_t launch(const KParams &p, double *part, int64_t first, cudaStream_t s
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NW * 32, smem);
     if (per_sm < 1) per_sm = 1;
     const int64_t cap = (int64_t)sms * per_sm;
-    const int64_t items = p.nb - first;
-    const int grid = (int)(items < cap ? items : cap);
+    const int grid = (int)(p.nb < cap ? p.nb : cap);
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, NW * 32, smem, stream>>>(p, part, first);
+    kern<<<grid, NW * 32, smem, stream>>>(p, part);
     return cudaGetLastError();
 }
 
 // 8 warps per CTA, 16 for the largest buckets (one CTA fits per SM there).
 template <int SCHEME, bool ERR>
-cudaError_t launch_nw(const KParams &p, double *part, int64_t first, cudaStream_t stream)
+cudaError_t launch_nw(const KParams &p, double *part, cudaStream_t stream)
 {
-    return p.d >= 16384 ? launch<SCHEME, ERR, 16>(p, part, first, stream) : launch<SCHEME, ERR, 8>(p, part, first, stream);
+    return p.d >= 16384 ? launch<SCHEME, ERR, 16>(p, part, stream) : launch<SCHEME, ERR, 8>(p, part, stream);
 }
 
 template <bool ERR>
-cudaError_t dispatch(const KParams &p, double *part, int64_t first, cudaStream_t stream)
+cudaError_t dispatch(const KParams &p, double *part, cudaStream_t stream)
 {
     switch (p.scheme) {
     case GQ_QSGD:
-    case GQ_TERNGRAD: return launch_nw<GQ_QSGD, ERR>(p, part, first, stream);
-    case GQ_BINGRAD_B: return launch_nw<GQ_BINGRAD_B, ERR>(p, part, first, stream);
-    case GQ_BINGRAD_PB: return launch_nw<GQ_BINGRAD_PB, ERR>(p, part, first, stream);
-    default: return launch_nw<GQ_ORQ, ERR>(p, part, first, stream);
+    case GQ_TERNGRAD: return launch_nw<GQ_QSGD, ERR>(p, part, stream);
+    case GQ_BINGRAD_B: return launch_nw<GQ_BINGRAD_B, ERR>(p, part, stream);
+    case GQ_BINGRAD_PB: return launch_nw<GQ_BINGRAD_PB, ERR>(p, part, stream);
+    default: return launch_nw<GQ_ORQ, ERR>(p, part, stream);
     }
 }
 
 }  // namespace
 
-cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream, int64_t first) { return dispatch<false>(p, nullptr, first, stream); }
+cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream) { return dispatch<false>(p, nullptr, stream); }
 
-cudaError_t launch_cta_err(const KParams &p, double *part, cudaStream_t stream) { return dispatch<true>(p, part, 0, stream); }
+cudaError_t launch_cta_err(const KParams &p, double *part, cudaStream_t stream) { return dispatch<true>(p, part, stream); }
 
 }  // namespace gq

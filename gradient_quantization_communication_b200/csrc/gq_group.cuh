@@ -51,7 +51,6 @@ struct alignas(16) FitGroupORQ {
     float lev[GQ_MAX_LEVELS];
     long long P1[64];  // the group's prefix sums of positions (up to 32768 * 63 * 2^16 < 2^37)
     int P0[64];
-    uint32_t codes[kCodeBytesWords + kBaseOutWords];  // (the register path's base-s messages only)
 };
 
 template <int SCHEME> struct GroupFitFor { using type = FitQSGD; };

@@ -53,7 +53,7 @@ constexpr unsigned kStatusTimeout = 2u;  // a bounded wait on a bulk copy gave u
 cudaError_t launch_warp_encode(const KParams &p, bool fused, cudaStream_t stream);
 // Shared-memory path (d = 1024 .. 32768): one CTA per bucket index walking the p.W workers;
 // with p.avg set, the average of the dequantized values is accumulated on chip and written.
-cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream, int64_t first = 0);
+cudaError_t launch_cta_encode(const KParams &p, cudaStream_t stream);
 // d = 1024 .. 32768, ORQ or QSGD / TernGrad, no clipping: every bucket spread over a group of
 // d / 512 warps (gq_group.cuh); the ragged last one in a second, one-group launch.
 cudaError_t launch_group_orq(const KParams &p, bool fused, cudaStream_t stream);

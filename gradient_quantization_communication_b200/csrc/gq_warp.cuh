@@ -774,15 +774,20 @@ constexpr int min_blocks()
                                      : GQ_WARP_MIN_BLOCKS * 4 / WARPS;
 }
 
+// Fits with a byte buffer of codes (base-s messages) have it cleared once.
+template <class F, class = void> struct HasCodes { static constexpr bool value = false; };
+template <class F> struct HasCodes<F, decltype((void)sizeof(((F *)nullptr)->codes))> { static constexpr bool value = true; };
+
 template <int SCHEME, class Fit>
 __device__ __forceinline__ void init_fit(const KParams &p, Fit &fit, int lane)
 {
     if constexpr (SCHEME == GQ_QSGD || SCHEME == GQ_TERNGRAD || SCHEME == GQ_QSGD_NEAREST || SCHEME == GQ_QSGD_L2) {
         for (int k = lane; k < p.s; k += 32) fit.qr[k] = p.qratio[k];
-        for (int i = lane; i < kCodeBytesWords + kBaseOutWords; i += 32) fit.codes[i] = 0u;
     }
     if constexpr (SCHEME == GQ_ORQ) {
         for (int i = lane; i < 64 * kHistCols; i += 32) fit.hist[i] = 0u;
+    }
+    if constexpr (HasCodes<Fit>::value) {
         for (int i = lane; i < kCodeBytesWords + kBaseOutWords; i += 32) fit.codes[i] = 0u;
     }
     if constexpr (SCHEME == GQ_BINGRAD_PB) {
