@@ -18,11 +18,14 @@ namespace gq {
 namespace {
 
 constexpr int kDecodeWarps = 4;
-constexpr int kDecodeGroup = 4;  // workers whose loads are in flight together
 
-template <bool QSGD, int BITS, int CPI>
+// WK: the worker count when known at compile time (2, 4 or 8: the loops unroll with no guards,
+// and up to 8 workers' loads are in flight together), 0 for any other count (4 at a time).
+template <bool QSGD, int BITS, int CPI, int WK = 0>
 __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_constant__ KParams p)
 {
+    constexpr int kDecodeGroup = WK > 0 ? (WK < 8 ? WK : 8) : 4;  // workers whose loads are in flight together
+    const int W = WK > 0 ? WK : p.W;
     constexpr int kWidth = 1 << BITS;
     constexpr int kChunkWords = 4 * BITS;  // words of one chunk's codes
     const int lane = threadIdx.x & 31;
@@ -52,7 +55,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
         float acc[CPI][4];
 #pragma unroll
         for (int c = 0; c < CPI; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
-        for (int w0 = 0; w0 < p.W; w0 += kDecodeGroup) {
+        for (int w0 = 0; w0 < W; w0 += kDecodeGroup) {
             uint32_t x[kDecodeGroup][CPI], y[kDecodeGroup][CPI];
             float lv[kDecodeGroup];
 #pragma unroll
@@ -60,7 +63,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
                 lv[k] = 0.0f;
 #pragma unroll
                 for (int c = 0; c < CPI; ++c) x[k][c] = y[k][c] = 0u;
-                if (w0 + k < p.W) {
+                if (w0 + k < W) {
                     const unsigned char *msg = p.msg[w0 + k];
                     const uint32_t *cw = reinterpret_cast<const uint32_t *>(msg) + wbase;
 #pragma unroll
@@ -75,13 +78,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
             }
 #pragma unroll
             for (int k = 0; k < kDecodeGroup; ++k) {
-                if (BITS == 8 && w0 + k < p.W) {
+                if (BITS == 8 && w0 + k < W) {
 #pragma unroll
                     for (int c = 0; c < CPI; ++c)
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
                             acc[c][e] = __fadd_rn(acc[c][e], __fmul_rn(lv[k], qtab[(x[k][c] >> (8 * e)) & 0xffu]));
-                } else if (w0 + k < p.W) {
+                } else if (w0 + k < W) {
                     const float level = QSGD ? __fmul_rn(lv[k], qr) : lv[k];
 #pragma unroll
                     for (int c = 0; c < CPI; ++c) {
@@ -173,7 +176,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base(const __grid_
 template <bool QSGD, int BITS, int CPI>
 cudaError_t launch(const KParams &p, cudaStream_t stream)
 {
-    auto kern = k_decode<QSGD, BITS, CPI>;
+    auto kern = p.W == 8   ? k_decode<QSGD, BITS, CPI, 8>
+                : p.W == 4 ? k_decode<QSGD, BITS, CPI, 4>
+                : p.W == 2 ? k_decode<QSGD, BITS, CPI, 2>
+                           : k_decode<QSGD, BITS, CPI>;
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
