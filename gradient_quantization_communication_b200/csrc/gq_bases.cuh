@@ -12,8 +12,8 @@
 // order, one 32-bit word per lane and chunk) instead of packing them; after the bucket's last
 // chunk each lane forms the values of every 32nd group and puts them in place (base_s_store).
 // Reader: the four codes of a lane (elements 4l .. 4l+3 of a chunk) lie in at most two groups,
-// whose 2B <= 32 bits one 64-bit window of two words holds; their digits come from a shared
-// table (base_codes4).
+// whose 2B <= 32 bits one 64-bit window of two words holds (base_pos); their digits come from a
+// shared table (base_codes4).
 #pragma once
 
 #include "gq_entropy.cuh"
@@ -125,23 +125,31 @@ __device__ __forceinline__ uint32_t group_digits(const DigitTab<S> &t, uint32_t 
     else return t.lo[V];
 }
 
-// The codes of elements e, e+1, e+2, e+3 of a bucket (e a multiple of 4, e + 3 < d) from its
-// base-s words (nw of them): at most two groups hold them.
+// Where the codes of elements e .. e+3 of a bucket (e a multiple of 4, e + 3 < d) lie in its
+// base-s words: at most two groups hold them, in words wi and wi + 1 from bit sh; element e is
+// digit k0 of the first.
+struct BasePos {
+    int wi, sh, k0;
+};
 template <int S>
-__device__ __forceinline__ void base_codes4(const DigitTab<S> &t, const uint32_t *words, int nw, int e, int (&code)[4])
+__device__ __forceinline__ BasePos base_pos(int e)
 {
     constexpr int g = BaseS<S>::g, B = BaseS<S>::B;
-    const int j0 = e / g;
-    const int bit = B * j0, wi = bit >> 5, sh = bit & 31;
-    const uint32_t lo = __ldg(words + wi);
-    const uint32_t hi = wi + 1 < nw ? __ldg(words + wi + 1) : 0u;
-    const unsigned long long two = ((unsigned long long)hi << 32 | lo) >> sh;
+    const int j0 = e / g, bit = B * j0;
+    return BasePos{bit >> 5, bit & 31, e - j0 * g};
+}
+// The four codes from the two words (lo, hi) at that place.
+template <int S>
+__device__ __forceinline__ void base_codes4(const DigitTab<S> &t, uint32_t lo, uint32_t hi, const BasePos &ps,
+                                            int (&code)[4])
+{
+    constexpr int g = BaseS<S>::g, B = BaseS<S>::B;
+    const unsigned long long two = ((unsigned long long)hi << 32 | lo) >> ps.sh;
     constexpr uint32_t mask = (1u << B) - 1u;
-    // the digits of both groups, 4 bits each, group j0's first: element e + q is digit k0 + q
+    // the digits of both groups, 4 bits each, the first group's first: element e + q is digit k0 + q
     const unsigned long long dg = (unsigned long long)group_digits<S>(t, (uint32_t)two & mask) |
                                   ((unsigned long long)group_digits<S>(t, (uint32_t)(two >> B) & mask) << (4 * g));
-    const int k0 = e - j0 * g;
-    const uint32_t run = (uint32_t)(dg >> (4 * k0));
+    const uint32_t run = (uint32_t)(dg >> (4 * ps.k0));
 #pragma unroll
     for (int q = 0; q < 4; ++q) code[q] = (int)((run >> (4 * q)) & 0xfu);
 }

@@ -114,7 +114,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
 }
 
 // Base-s messages (s = 3, 5, 9; d <= 512): the same items and sum, with each lane's four codes
-// of a chunk taken from the one or two base-s groups that hold them (base_codes4).
+// of a chunk taken from the one or two base-s groups that hold them (base_codes4); the code words
+// of kBaseGroup workers are loaded before any is decoded.
+constexpr int kBaseGroup = 4;
 template <bool QSGD, int S, int CPI>
 __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base(const __grid_constant__ KParams p)
 {
@@ -140,21 +142,47 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base(const __grid_
         int nlive = (int)((p.n - e0 + 127) >> 7);
         nlive = nlive < CPI ? nlive : CPI;
         float acc[CPI][4];
+        BasePos ps[CPI];
 #pragma unroll
-        for (int c = 0; c < CPI; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
-        for (int w = 0; w < p.W; ++w) {
-            const unsigned char *msg = p.msg[w];
-            const uint32_t *words = reinterpret_cast<const uint32_t *>(msg) + bk * p.codes_words;
-            float lv = 0.0f;
-            if (QSGD || has_level) lv = __ldg(reinterpret_cast<const float *>(msg + p.levels_off) + tbase);
-            const float level = QSGD ? __fmul_rn(lv, qr) : lv;
+        for (int c = 0; c < CPI; ++c) {
+            acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
+            ps[c] = base_pos<S>(eb + 128 * c);
+        }
+        // the loads of a group of workers go out before any is used
+        for (int w0 = 0; w0 < p.W; w0 += kBaseGroup) {
+            uint32_t lo[kBaseGroup][CPI], hi[kBaseGroup][CPI];
+            float lv[kBaseGroup];
 #pragma unroll
-            for (int c = 0; c < CPI; ++c) {
-                int code[4] = {0, 0, 0, 0};
-                if (c < nlive) base_codes4<S>(tab, words, nw, eb + 128 * c, code);
+            for (int k = 0; k < kBaseGroup; ++k) {
+                lv[k] = 0.0f;
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, code[e], kWidth));
+                for (int c = 0; c < CPI; ++c) lo[k][c] = hi[k][c] = 0u;
+                if (w0 + k < p.W) {
+                    const unsigned char *msg = p.msg[w0 + k];
+                    const uint32_t *words = reinterpret_cast<const uint32_t *>(msg) + bk * p.codes_words;
+#pragma unroll
+                    for (int c = 0; c < CPI; ++c) {
+                        if (c < nlive) {
+                            lo[k][c] = __ldg(words + ps[c].wi);
+                            if (ps[c].wi + 1 < nw) hi[k][c] = __ldg(words + ps[c].wi + 1);
+                        }
+                    }
+                    if (QSGD || has_level) lv[k] = __ldg(reinterpret_cast<const float *>(msg + p.levels_off) + tbase);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kBaseGroup; ++k) {
+                if (w0 + k < p.W) {
+                    const float level = QSGD ? __fmul_rn(lv[k], qr) : lv[k];
+#pragma unroll
+                    for (int c = 0; c < CPI; ++c) {
+                        int code[4];
+                        base_codes4<S>(tab, lo[k][c], hi[k][c], ps[c], code);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, code[e], kWidth));
+                    }
+                }
             }
         }
 #pragma unroll
