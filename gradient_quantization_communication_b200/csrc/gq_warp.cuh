@@ -72,9 +72,11 @@ struct alignas(16) FitQSGD {
     uint32_t codes[kCodeBytesWords + kBaseOutWords];  // base-s messages: codes as bytes, output words
 };
 struct alignas(16) FitPB {
-    unsigned long long s1[64], s2[64];  // per cell: sum of positions, of squared positions
-    unsigned int cnt[64];               // per cell: count
-    long long al[64], be[64], ga[64], de[64];
+    unsigned long long q2[64];  // at a cell's first value in sorted order: sum of squared positions before it
+    unsigned int q1[64];        // ... sum of positions before it (< 2^31 for d <= 512)
+    int q0[64];                 // ... 1 + count before it; 0 for an empty cell
+    long long al[64], be[64];   // per-index terms of E(A, B)
+    unsigned long long ga16[64], de16[64];  // ... pre-multiplied by 2^16
 };
 
 struct alignas(16) FitB {
@@ -440,12 +442,14 @@ __device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
 // BinGrad-b's levels of the bucket (m = max|u| over the valid values, already reduced): the
 // sorted values' exact fixed-point prefix sums and the screened argmax of J; {a, b, split value,
 // split found}.  Also used by BinGrad-pb, whose levels must be at least as far apart.
+// The sorted values are left in key (position lane*EPL + r, the invalid ones last as +inf) when
+// m > 0.
 template <int EPL, bool TAIL>
-__device__ __forceinline__ RoundB bingrad_b_levels(int lane, uint32_t vmask, int nvalid, float m, const float (&u)[EPL])
+__device__ __forceinline__ RoundB bingrad_b_levels(int lane, uint32_t vmask, int nvalid, float m, const float (&u)[EPL],
+                                                   float (&key)[EPL])
 {
     RoundB rule{0.0f, 0.0f, 0.0f, false};
     if (!(m > 0.0f)) return rule;
-    float key[EPL];
 #pragma unroll
     for (int t = 0; t < EPL; ++t) key[t] = (!TAIL || ((vmask >> t) & 1u)) ? u[t] : INFINITY;
     warp_bitonic_sort<EPL>(key, lane);
@@ -551,7 +555,8 @@ __device__ void fit_bingrad_b(const KParams &p, FitB &, int64_t beta, int w, int
     int pos[EPL];
 #pragma unroll
     for (int t = 0; t < EPL; ++t) pos[t] = 0;
-    const RoundB rule = bingrad_b_levels<EPL, TAIL>(lane, vmask, nvalid, m, u);
+    float key[EPL];
+    const RoundB rule = bingrad_b_levels<EPL, TAIL>(lane, vmask, nvalid, m, u, key);
     emit<EPL, FUSED, false, TAIL, BITS, IO>(p, rule, beta, w, lane, vmask, v, u, pos, acc, ea);
     store_table(p, w, beta, lane, lane == 0 ? rule.a : rule.b);
 }
@@ -587,10 +592,12 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
     const float step = __fdiv_rn(range, 63.0f);
     const float scale = __fmul_rn(__fdiv_rn(63.0f, range), (float)(1 << kPbFBits));
     // the admissible pairs: A <= Amax, the largest grid index whose point is <= a_b (0 if none);
-    // B >= Bmin, the smallest whose point is >= b_b (63 if none)
+    // B >= Bmin, the smallest whose point is >= b_b (63 if none).  mx > mn makes max|u| > 0, so
+    // the level search sorts the values into key.
     int Amax, Bmin;
+    float key[EPL];
     {
-        const RoundB bl = bingrad_b_levels<EPL, TAIL>(lane, vmask, nvalid, fmaxf(fabsf(mn), fabsf(mx)), u);
+        const RoundB bl = bingrad_b_levels<EPL, TAIL>(lane, vmask, nvalid, fmaxf(fabsf(mn), fabsf(mx)), u, key);
         const float g0 = grid_point(mn, mx, step, lane), g1 = grid_point(mn, mx, step, lane + 32);
         const unsigned long long le = (unsigned long long)__ballot_sync(kFull, g0 <= bl.a) |
                                       ((unsigned long long)__ballot_sync(kFull, g1 <= bl.a) << 32);
@@ -600,72 +607,111 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
         Bmin = ge ? __ffsll(ge) - 1 : 63;
     }
 #pragma unroll
-    for (int t = 0; t < EPL; ++t) {
-        pos[t] = grid_pos<kPbFBits>(u[t], mn, scale);
-        if (!TAIL || ((vmask >> t) & 1u)) {
-            const int cell = min(pos[t] >> kPbFBits, kTopCell);
-            const unsigned long long x = (unsigned long long)pos[t];
-            atomicAdd(&sm.cnt[cell], 1u);
-            atomicAdd(&sm.s1[cell], x);
-            atomicAdd(&sm.s2[cell], x * x);
+    for (int t = 0; t < EPL; ++t) pos[t] = grid_pos<kPbFBits>(u[t], mn, scale);
+    // Q0, Q1, Q2 (count, sum of positions, of squared positions over the cells < k) from the
+    // sorted values: the position is monotone in the value, so the cells are too, and Q(k) is the
+    // prefix before the first value whose cell is >= k.  Each nonempty cell records the prefix at
+    // its first value; no two values add into one shared counter.
+    unsigned long long tx_all, ty_all;
+    {
+        int cell[EPL];
+        unsigned int x1[EPL];
+        unsigned long long x2[EPL];
+        unsigned int run1 = 0u;  // at most 512 * 63 * 2^16 < 2^32
+        unsigned long long run2 = 0ull;
+#pragma unroll
+        for (int r = 0; r < EPL; ++r) {
+            const bool valid = !TAIL || lane * EPL + r < nvalid;
+            const int ps = grid_pos<kPbFBits>(key[r], mn, scale);
+            cell[r] = valid ? min(ps >> kPbFBits, kTopCell) : 64;
+            x1[r] = run1;
+            x2[r] = run2;
+            if (valid) {
+                run1 += (unsigned int)ps;
+                run2 += (unsigned long long)ps * (unsigned long long)ps;
+            }
+        }
+        const unsigned int in1 = warp_inclusive_scan(run1, lane);
+        const unsigned long long in2 = warp_inclusive_scan(run2, lane);
+        tx_all = __shfl_sync(kFull, in1, 31);
+        ty_all = __shfl_sync(kFull, in2, 31);
+        const unsigned int ex1 = in1 - run1;
+        const unsigned long long ex2 = in2 - run2;
+        const int prev_cell = __shfl_up_sync(kFull, cell[EPL - 1], 1);
+#pragma unroll
+        for (int r = 0; r < EPL; ++r) {
+            const int cp = r > 0 ? cell[r - 1] : (lane > 0 ? prev_cell : -1);
+            if (cell[r] != cp && cell[r] < 64) {
+                sm.q0[cell[r]] = lane * EPL + r + 1;
+                sm.q1[cell[r]] = ex1 + x1[r];
+                sm.q2[cell[r]] = ex2 + x2[r];
+            }
         }
     }
     __syncwarp();
-    // prefix sums Q0, Q1, Q2 over cells < k, then the per-index terms of
-    // E(A,B) = al[A] + be[B] + a*ga[B] + b*de[A]   (a = A*2^16, b = B*2^16)
-    const long long c0 = sm.cnt[lane], c1 = sm.cnt[lane + 32];
-    const long long x0 = (long long)sm.s1[lane], x1 = (long long)sm.s1[lane + 32];
-    const long long y0 = (long long)sm.s2[lane], y1 = (long long)sm.s2[lane + 32];
-    __syncwarp();
-    sm.cnt[lane] = 0u;
-    sm.cnt[lane + 32] = 0u;
-    sm.s1[lane] = 0ull;
-    sm.s1[lane + 32] = 0ull;
-    sm.s2[lane] = 0ull;
-    sm.s2[lane + 32] = 0ull;
-    const long long ic0 = warp_inclusive_scan(c0, lane), ic1 = warp_inclusive_scan(c1, lane);
-    const long long ix0 = warp_inclusive_scan(x0, lane), ix1 = warp_inclusive_scan(x1, lane);
-    const long long iy0 = warp_inclusive_scan(y0, lane), iy1 = warp_inclusive_scan(y1, lane);
-    const long long tc = __shfl_sync(kFull, ic0, 31), tx = __shfl_sync(kFull, ix0, 31), ty = __shfl_sync(kFull, iy0, 31);
-    const long long tc_all = __shfl_sync(kFull, tc + ic1, 31);
-    const long long tx_all = __shfl_sync(kFull, tx + ix1, 31);
-    const long long ty_all = __shfl_sync(kFull, ty + iy1, 31);
+    // the per-index terms of E(A,B) = al[A] + be[B] + a*ga[B] + b*de[A]   (a = A*2^16, b = B*2^16)
+    {
+        const unsigned long long tc_all = (unsigned long long)(TAIL ? nvalid : 32 * EPL);
+        const unsigned long long nonempty = (unsigned long long)__ballot_sync(kFull, sm.q0[lane] != 0) |
+                                            ((unsigned long long)__ballot_sync(kFull, sm.q0[lane + 32] != 0) << 32);
+        unsigned long long uQ0[2], uQ1[2], uQ2[2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int K = lane + 32 * h;
-        const long long Q0 = h ? tc + ic1 - c1 : ic0 - c0;
-        const long long Q1 = h ? tx + ix1 - x1 : ix0 - x0;
-        const long long Q2 = h ? ty + iy1 - y1 : iy0 - y0;
-        const unsigned long long k = (unsigned long long)K << kPbFBits;
-        // modular 64-bit arithmetic: every E(A,B) fits in int64, so wrapped partial terms cancel
-        const unsigned long long uQ0 = Q0, uQ1 = Q1, uQ2 = Q2;
-        sm.al[K] = (long long)(k * k * uQ0 - 3ull * k * uQ1 + 2ull * uQ2);
-        sm.be[K] = (long long)(3ull * k * uQ1 - 2ull * uQ2 + (unsigned long long)ty_all - 2ull * k * (unsigned long long)tx_all +
-                               k * k * ((unsigned long long)tc_all - uQ0));
-        sm.ga[K] = (long long)(uQ1 - k * uQ0);
-        sm.de[K] = (long long)(k * uQ0 - uQ1);
+        for (int h = 0; h < 2; ++h) {
+            const unsigned long long later = nonempty & (~0ull << (lane + 32 * h));
+            if (later) {
+                const int c = __ffsll(later) - 1;
+                uQ0[h] = (unsigned long long)(sm.q0[c] - 1);
+                uQ1[h] = sm.q1[c];
+                uQ2[h] = sm.q2[c];
+            } else {
+                uQ0[h] = tc_all;
+                uQ1[h] = tx_all;
+                uQ2[h] = ty_all;
+            }
+        }
+        __syncwarp();
+        sm.q0[lane] = 0;
+        sm.q0[lane + 32] = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int K = lane + 32 * h;
+            const unsigned long long k = (unsigned long long)K << kPbFBits;
+            // modular 64-bit arithmetic: every E(A,B) fits in int64, so wrapped partial terms cancel
+            sm.al[K] = (long long)(k * k * uQ0[h] - 3ull * k * uQ1[h] + 2ull * uQ2[h]);
+            sm.be[K] = (long long)(3ull * k * uQ1[h] - 2ull * uQ2[h] + ty_all - 2ull * k * tx_all + k * k * (tc_all - uQ0[h]));
+            sm.ga16[K] = (uQ1[h] - k * uQ0[h]) << kPbFBits;
+            sm.de16[K] = (k * uQ0[h] - uQ1[h]) << kPbFBits;
+        }
     }
     __syncwarp();
-    // exhaustive search over A < B, ties to the smallest (A, B).  Lane l takes B = l (A < l) and
-    // B = 63 - l (A < 63 - l): 63 pairs on every lane, one uniform loop.  With ga, de kept
-    // pre-multiplied by 2^16, E = al[A] + be[B] + A * ga16[B] + B * de16[A] (mod 2^64, exact).
+    // exhaustive search over the admissible pairs (A <= Amax, B >= Bmin, A < B), ties to the
+    // smallest (A, B).  The nB = 64 - Bmin columns B are spread over the lanes, P lanes to a column
+    // for nB <= 16 (lane l: column l / P, A = l % P, l % P + P, ...), and a lane walks its column's A
+    // up to Amax.  With ga, de pre-multiplied by 2^16, E = al[A] + be[B] + A * ga16[B] + B * de16[A]
+    // (mod 2^64, exact).
     long long best_e = 0x7fffffffffffffffll;
     int best_ab = 0x7fffffff;
     {
-        const int B0 = lane, B1 = 63 - lane;
-        const unsigned long long be0 = sm.be[B0], ga0 = (unsigned long long)sm.ga[B0] << kPbFBits;
-        const unsigned long long be1 = sm.be[B1], ga1 = (unsigned long long)sm.ga[B1] << kPbFBits;
-        for (int i = 0; i < 63; ++i) {
-            const bool first = i < B0;
-            const int A = first ? i : i - B0, B = first ? B0 : B1;
-            const unsigned long long beB = first ? be0 : be1, gaB = first ? ga0 : ga1;
-            const long long e = (long long)((unsigned long long)sm.al[A] + beB + (unsigned long long)A * gaB +
-                                            (unsigned long long)B * ((unsigned long long)sm.de[A] << kPbFBits));
-            const int ab = A * 64 + B;
-            const bool admissible = A <= Amax && B >= Bmin;
-            if (admissible && (e < best_e || (e == best_e && ab < best_ab))) {
-                best_e = e;
-                best_ab = ab;
+        const int nB = 64 - Bmin;
+        const int lp = nB > 16 ? 0 : 5 - (32 - __clz(nB - 1));  // log2 P
+        const int P = 1 << lp, sub = lane & (P - 1), col = lane >> lp;
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+            const int B = Bmin + col + 32 * pass;
+            if (B > 63) break;
+            const unsigned long long beB = (unsigned long long)sm.be[B], gaB = sm.ga16[B];
+            const unsigned long long dg = (unsigned long long)P * gaB;
+            unsigned long long ag = (unsigned long long)sub * gaB;
+#pragma unroll 2
+            for (int A = sub; A <= Amax; A += P) {
+                const long long e =
+                    (long long)((unsigned long long)sm.al[A] + beB + ag + (unsigned long long)(unsigned)B * sm.de16[A]);
+                ag += dg;
+                const int ab = A * 64 + B;
+                if (A < B && (e < best_e || (e == best_e && ab < best_ab))) {
+                    best_e = e;
+                    best_ab = ab;
+                }
             }
         }
     }
@@ -791,11 +837,7 @@ __device__ __forceinline__ void init_fit(const KParams &p, Fit &fit, int lane)
         for (int i = lane; i < kCodeBytesWords + kBaseOutWords; i += 32) fit.codes[i] = 0u;
     }
     if constexpr (SCHEME == GQ_BINGRAD_PB) {
-        for (int i = lane; i < 64; i += 32) {
-            fit.cnt[i] = 0u;
-            fit.s1[i] = 0ull;
-            fit.s2[i] = 0ull;
-        }
+        for (int i = lane; i < 64; i += 32) fit.q0[i] = 0;
     }
 }
 
