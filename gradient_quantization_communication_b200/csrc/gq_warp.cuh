@@ -684,35 +684,48 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
         }
     }
     __syncwarp();
-    // exhaustive search over the admissible pairs (A <= Amax, B >= Bmin, A < B), ties to the
-    // smallest (A, B).  The nB = 64 - Bmin columns B are spread over the lanes, P lanes to a column
-    // for nB <= 16 (lane l: column l / P, A = l % P, l % P + P, ...), and a lane walks its column's A
-    // up to Amax.  With ga, de pre-multiplied by 2^16, E = al[A] + be[B] + A * ga16[B] + B * de16[A]
-    // (mod 2^64, exact).
+    // The least E over the admissible pairs (A <= Amax, B >= Bmin, A < B), ties to the smallest
+    // (A, B), column by column: lane l takes B = Bmin + l and Bmin + l + 32.  With ga, de
+    // pre-multiplied by 2^16, E = al[A] + be[B] + A * ga16[B] + B * de16[A] (mod 2^64; the exact
+    // E fits in int64).  For a fixed b, E is convex in a: a value x contributes (x - a)(b - x),
+    // of slope -(b - x) <= 0, while a <= x and (a - x)^2, of slope 2(a - x) >= 0, past it, and
+    // nothing that depends on a when x > b.  So along a column the differences
+    // E(A+1, B) - E(A, B) never decrease, and the smallest minimiser over A in [0, Ahi] is the
+    // first A whose difference is >= 0 (Ahi if none): found from the last difference, else by
+    // bisection.  The column minima then go to the warp's reduction.
     long long best_e = 0x7fffffffffffffffll;
     int best_ab = 0x7fffffff;
-    {
-        const int nB = 64 - Bmin;
-        const int lp = nB > 16 ? 0 : 5 - (32 - __clz(nB - 1));  // log2 P
-        const int P = 1 << lp, sub = lane & (P - 1), col = lane >> lp;
 #pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-            const int B = Bmin + col + 32 * pass;
-            if (B > 63) break;
-            const unsigned long long beB = (unsigned long long)sm.be[B], gaB = sm.ga16[B];
-            const unsigned long long dg = (unsigned long long)P * gaB;
-            unsigned long long ag = (unsigned long long)sub * gaB;
-#pragma unroll 2
-            for (int A = sub; A <= Amax; A += P) {
-                const long long e =
-                    (long long)((unsigned long long)sm.al[A] + beB + ag + (unsigned long long)(unsigned)B * sm.de16[A]);
-                ag += dg;
-                const int ab = A * 64 + B;
-                if (A < B && (e < best_e || (e == best_e && ab < best_ab))) {
-                    best_e = e;
-                    best_ab = ab;
+    for (int pass = 0; pass < 2; ++pass) {
+        const int B = Bmin + lane + 32 * pass;
+        const int Ahi = min(Amax, B - 1);
+        if (B > 63) break;
+        if (Ahi < 0) continue;  // B = 0
+        const unsigned long long beB = (unsigned long long)sm.be[B], gaB = sm.ga16[B];
+        auto E = [&](int A) {
+            return (long long)((unsigned long long)sm.al[A] + beB + (unsigned long long)(unsigned)A * gaB +
+                               (unsigned long long)(unsigned)B * sm.de16[A]);
+        };
+        int As = Ahi;
+        long long es = E(Ahi);
+        if (Ahi > 0) {
+            const long long eb = E(Ahi - 1);
+            if (!(es < eb)) {
+                // the difference at Ahi - 1 is >= 0: the first such A lies in [0, Ahi - 1]
+                int lo = 0, hi = Ahi - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (E(mid + 1) - E(mid) >= 0) hi = mid;
+                    else lo = mid + 1;
                 }
+                As = lo;
+                es = lo == Ahi - 1 ? eb : E(lo);
             }
+        }
+        const int ab = As * 64 + B;
+        if (es < best_e || (es == best_e && ab < best_ab)) {
+            best_e = es;
+            best_ab = ab;
         }
     }
 #pragma unroll
