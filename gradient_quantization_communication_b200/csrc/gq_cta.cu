@@ -561,21 +561,23 @@ __global__ void __launch_bounds__(NW * 32) k_cta(const __grid_constant__ KParams
                         }
                     }
                     __syncthreads();
-                    // thread (B = tid % 64, group tid / 64) searches A in [kSpan*group, kSpan*(group + 1)) below B
-                    constexpr int kSpan = 128 / NW;  // A values per thread: NW / 2 groups of 64 threads
-                    const int B = tid & 63, grp = tid >> 6;
-                    const unsigned long long bb = (unsigned long long)B << kPbFBits;
-                    const unsigned long long beB = sh.be[B], gaB = sh.ga[B];
+                    // thread B < 64 finds column B's least E over A <= min(Amax, B - 1)
+                    // (pb_column_argmin; E exact mod 2^64), ties to the smallest (A, B)
                     long long best_e = 0x7fffffffffffffffll;
                     int best_ab = 0x7fffffff;
-                    for (int A = kSpan * grp; A < kSpan * grp + kSpan && A < B; ++A) {
-                        const unsigned long long aa = (unsigned long long)A << kPbFBits;
-                        const long long e = (long long)((unsigned long long)sh.al[A] + beB + aa * gaB + bb * (unsigned long long)sh.de[A]);
-                        const int ab = A * 64 + B;
-                        const bool admissible = A <= Amax && B >= Bmin;
-                        if (admissible && (e < best_e || (e == best_e && ab < best_ab))) {
-                            best_e = e;
-                            best_ab = ab;
+                    {
+                        const int B = tid;
+                        const int Ahi = min(Amax, B - 1);
+                        if (B < 64 && B >= Bmin && Ahi >= 0) {
+                            const unsigned long long beB = sh.be[B], gaB = (unsigned long long)sh.ga[B] << kPbFBits;
+                            const unsigned long long bb = (unsigned long long)B << kPbFBits;
+                            auto E = [&](int A) {
+                                return (long long)((unsigned long long)sh.al[A] + beB + (unsigned long long)(unsigned)A * gaB +
+                                                   bb * (unsigned long long)sh.de[A]);
+                            };
+                            long long es;
+                            best_ab = pb_column_argmin(E, Ahi, es) * 64 + B;
+                            best_e = es;
                         }
                     }
 #pragma unroll

@@ -305,6 +305,30 @@ __device__ __forceinline__ float grid_point(float mn, float mx, float step, int 
     return j == 63 ? mx : __fadd_rn(mn, __fmul_rn((float)j, step));
 }
 
+// BinGrad-pb, one column of the pair search: the smallest minimiser over A in [0, Ahi] (Ahi >= 0)
+// of E(A) = E(A, B) for a fixed B, and its value in es.  E(a, b) is convex in a for a fixed b: a
+// value x contributes (x - a)(b - x), of slope -(b - x) <= 0, while a <= x, and (a - x)^2, of
+// slope 2(a - x) >= 0, past it (nothing that depends on a when x > b).  So the differences
+// E(A+1) - E(A) never decrease and the first A whose difference is >= 0 (Ahi if none) is the
+// answer: the last difference decides whether it is Ahi, else a bisection finds it.  E is exact
+// (int64), so the choice is the one an exhaustive scan with ties to the smallest A makes.
+template <class EF>
+__device__ __forceinline__ int pb_column_argmin(const EF &E, int Ahi, long long &es)
+{
+    es = E(Ahi);
+    if (Ahi == 0) return 0;
+    const long long eb = E(Ahi - 1);
+    if (es < eb) return Ahi;
+    int lo = 0, hi = Ahi - 1;  // the difference at hi is >= 0
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (E(mid + 1) - E(mid) >= 0) hi = mid;
+        else lo = mid + 1;
+    }
+    es = lo == Ahi - 1 ? eb : E(lo);
+    return lo;
+}
+
 // Fixed-point grid position, floor((u - mn) * scale) clamped to [0, 63 * 2^F].
 template <int F>
 __device__ __forceinline__ int grid_pos(float u, float mn, float scale)

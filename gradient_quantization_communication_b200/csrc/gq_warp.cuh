@@ -685,14 +685,9 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
     }
     __syncwarp();
     // The least E over the admissible pairs (A <= Amax, B >= Bmin, A < B), ties to the smallest
-    // (A, B), column by column: lane l takes B = Bmin + l and Bmin + l + 32.  With ga, de
-    // pre-multiplied by 2^16, E = al[A] + be[B] + A * ga16[B] + B * de16[A] (mod 2^64; the exact
-    // E fits in int64).  For a fixed b, E is convex in a: a value x contributes (x - a)(b - x),
-    // of slope -(b - x) <= 0, while a <= x and (a - x)^2, of slope 2(a - x) >= 0, past it, and
-    // nothing that depends on a when x > b.  So along a column the differences
-    // E(A+1, B) - E(A, B) never decrease, and the smallest minimiser over A in [0, Ahi] is the
-    // first A whose difference is >= 0 (Ahi if none): found from the last difference, else by
-    // bisection.  The column minima then go to the warp's reduction.
+    // (A, B), column by column (pb_column_argmin): lane l takes B = Bmin + l and Bmin + l + 32.
+    // With ga, de pre-multiplied by 2^16, E = al[A] + be[B] + A * ga16[B] + B * de16[A]
+    // (mod 2^64; the exact E fits in int64).  The column minima then go to the warp's reduction.
     long long best_e = 0x7fffffffffffffffll;
     int best_ab = 0x7fffffff;
 #pragma unroll 1
@@ -706,23 +701,8 @@ __device__ void fit_bingrad_pb(const KParams &p, FitPB &sm, int64_t beta, int w,
             return (long long)((unsigned long long)sm.al[A] + beB + (unsigned long long)(unsigned)A * gaB +
                                (unsigned long long)(unsigned)B * sm.de16[A]);
         };
-        int As = Ahi;
-        long long es = E(Ahi);
-        if (Ahi > 0) {
-            const long long eb = E(Ahi - 1);
-            if (!(es < eb)) {
-                // the difference at Ahi - 1 is >= 0: the first such A lies in [0, Ahi - 1]
-                int lo = 0, hi = Ahi - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (E(mid + 1) - E(mid) >= 0) hi = mid;
-                    else lo = mid + 1;
-                }
-                As = lo;
-                es = lo == Ahi - 1 ? eb : E(lo);
-            }
-        }
-        const int ab = As * 64 + B;
+        long long es;
+        const int ab = pb_column_argmin(E, Ahi, es) * 64 + B;
         if (es < best_e || (es == best_e && ab < best_ab)) {
             best_e = es;
             best_ab = ab;
