@@ -22,6 +22,8 @@ Other one-line modes (one GPU):
   --entropy   base-s packing of the W messages (gq_entropy_pack / gq_entropy_unpack)
   --elias     Elias-gamma coding of the W messages (gq_elias_pack / gq_elias_unpack), for an
               odd-level QSGD-family scheme such as --scheme qsgd_l2 --levels 3
+  --exchange  the data-parallel exchange (exchange.Exchange): one worker per rank under
+              torchrun, gq_encode + NCCL all-gather of the packed messages + gq_decode_accumulate
 """
 import argparse
 import concurrent.futures as cf
@@ -81,6 +83,9 @@ def parse_args():
     ap.add_argument("--entropy", action="store_true",
                     help="base-s packing: gq_entropy_pack then gq_entropy_unpack of the W messages of one "
                          "step; per-kernel rooflines and the compression ratios, one JSON line")
+    ap.add_argument("--exchange", action="store_true",
+                    help="the quantized all-gather exchange, one worker per rank (W = the number of ranks): "
+                         "per-phase times (encode, all-gather, decode), one JSON line from rank 0")
     ap.add_argument("--elias", action="store_true",
                     help="Elias-gamma coding: gq_elias_pack then gq_elias_unpack of the W messages of one "
                          "step (an odd-level QSGD-family scheme, e.g. --scheme qsgd_l2 --levels 3); "
@@ -637,6 +642,117 @@ def run_unfused(args):
     return 0
 
 
+# Measured peer copy between two B200s of this machine over NVLink, one direction (900 nominal).
+PEER_LINK_GBS = 770.0
+
+
+def run_exchange(args):
+    """The data-parallel exchange of exchange.Exchange, one worker per rank: rank w quantizes its
+    own gradient (worker index w) with gq_encode, the W packed messages are all-gathered over NCCL
+    and every rank decodes and averages them with gq_decode_accumulate.  Each phase is timed with
+    events on the launching stream (the all-gather's completion is ordered onto it); the step
+    time is the slowest rank's.  Per-worker elements: the workload's n; W = the number of ranks.
+    With one rank the all-gather is a copy on the GPU and no byte crosses a link."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import gradient_quantization_communication_b200.gq as G
+    from gradient_quantization_communication_b200 import synth
+    from gradient_quantization_communication_b200.exchange import Exchange
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world == 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(_free_port()))
+        os.environ.setdefault("RANK", "0")
+        os.environ.setdefault("WORLD_SIZE", "1")
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    wl = synth.WORKLOADS[args.workload]
+    if args.elements:
+        wl = dataclasses.replace(wl, n=min(wl.n, args.elements))
+    n, d, ef, W = wl.n, args.bucket, wl.error_feedback, world
+    sid = G.SCHEMES[args.scheme]
+    cfg = G.gq_config(sid, args.levels, d, W, ef, args.clip, wl.rounding_seed, n)
+    ex = Exchange(cfg, device=dev)
+    g = torch.empty(n, dtype=torch.float32, device=dev)
+    synth.gradient(args.workload, rank, 0, n=n, out=g)
+    r = torch.zeros(n, dtype=torch.float32, device=dev) if ef else None
+    avg = torch.empty(n, dtype=torch.float32, device=dev)
+    for t in range(args.warmup):
+        ex.step(t, g, r, avg)
+    torch.cuda.synchronize()
+    if G.gq_plan_status(ex.plan.handle) != G.GQ_OK:
+        raise RuntimeError("non-finite input in the benchmark workload")
+    sampler = ClockSampler(pci_bus_id(dev)) if rank == 0 else None
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for k in range(args.steps):
+        ex.step(args.warmup + k, g, r, avg, events=evs[k])
+    t1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), dev)
+    phase = [max_over_ranks(statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs), dev) for i in range(3)]
+    msg_bytes = ex.msg_bytes
+    ex.close()
+    dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    ms = elapsed_ms / args.steps
+    msg_b = message_bytes_per_elem(sid, args.levels, d)
+    enc_b = 4.0 + (8.0 if ef else 0.0) + msg_b  # per element of this rank's worker
+    dec_b = W * msg_b + 4.0                     # per element of the average
+    peak, peak_kind = measured_hbm_peak()
+
+    def roof(bytes_per_call, call_ms):
+        a = bytes_per_call / (call_ms / 1000.0) / 1e9
+        return {"bound": "hbm", "achieved": round(a, 1), "peak": peak, "unit": "GB/s", "frac": round(a / peak, 4),
+                "peak_kind": peak_kind, "algorithmic_bytes_per_call": bytes_per_call, "ms_per_call": call_ms}
+
+    recv = (W - 1) * msg_bytes  # bytes that reach each rank over the links
+    link = {"bound": "nvlink", "ms_per_call": phase[1], "bytes_received_per_rank": recv,
+            "achieved": round(recv / (phase[1] / 1000.0) / 1e9, 1) if recv else None, "peak": PEER_LINK_GBS,
+            "unit": "GB/s", "frac": round(recv / (phase[1] / 1000.0) / 1e9 / PEER_LINK_GBS, 4) if recv else None,
+            "peak_kind": "measured peer copy, one direction"}
+    config = workload_config(args, wl)
+    config.update({"workload": "%s: %d fp32 elements per worker x W=%d workers (one per rank), %s-%d, d=%d, "
+                               "error feedback %s" % (args.workload, n, W, args.scheme, args.levels, d,
+                                                      "on" if ef else "off"),
+                   "workers": W, "elements_per_worker": n,
+                   "parallelism": "one worker per rank, all-gather of the packed messages"})
+    tail = 1 if n % d else 0
+    print(json.dumps({
+        "metric": "quantized exchange step (encode + all-gather + decode), worker-elements/s",
+        "value": W * n / (ms / 1000.0), "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": config,
+        "encode": roof(enc_b * n, phase[0]), "allgather": link, "decode": roof(dec_b * n, phase[2]),
+        "bytes": {"encode_per_elem": enc_b, "decode_per_elem": dec_b, "message": msg_bytes},
+        "gpu_launches": ((1 if n >= d else 0) + tail + 1) * args.steps, "clocks": clocks}))
+    return 0
+
+
+def _free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
 def run_entropy(args):
     """Base-s packing of the W messages of one fused step: a timed step is gq_entropy_pack of
     every worker's message followed by gq_entropy_unpack of every base-s message (each launch
@@ -908,6 +1024,8 @@ def main():
         return run_entropy(args)
     if args.elias:
         return run_elias(args)
+    if args.exchange:
+        return run_exchange(args)
     return run_gq(args)
 
 

@@ -77,11 +77,22 @@ class Exchange:
         b = self.msg_bytes
         return [self.buf.gathered[w * b:(w + 1) * b] for w in range(self.world)]
 
-    def step(self, step, grad, residual, avg):
-        """Quantize this rank's gradient, exchange the messages, write the average to avg."""
+    def step(self, step, grad, residual, avg, events=None):
+        """Quantize this rank's gradient, exchange the messages, write the average to avg.
+        events: optional four CUDA events, recorded on the current stream before the encode,
+        after it, after the all-gather (whose completion the current stream waits for) and after
+        the decode."""
+        if events is not None:
+            events[0].record()
         self._encode(step, self.rank, grad, residual, self.buf.msg)
+        if events is not None:
+            events[1].record()
         dist.all_gather_into_tensor(self.buf.gathered, self.buf.msg, group=self.group)
+        if events is not None:
+            events[2].record()
         self._decode(self.messages(), avg)
+        if events is not None:
+            events[3].record()
 
     def close(self):
         if self.plan is not None:

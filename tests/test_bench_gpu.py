@@ -73,3 +73,14 @@ def test_elias_line():
     assert j["round_trip"] == "exact" and j["gpu_launches"] == 6 * 8 * 2
     c = j["compression"]
     assert 1.0 <= c["stream_bits_per_elem"] < 1.3 and c["dense_bits_per_elem"] == (32 * 32 + 32) / 512
+
+
+@pytest.mark.gpu
+def test_exchange_line():
+    """One rank: the all-gather is a copy on the GPU, no byte crosses a link."""
+    j = _run("--exchange", "--elements", "5120000", "--steps", "2", "--warmup", "3")
+    assert j["n_gpus"] == 1 and j["config"]["workers"] == 1 and j["value"] > 0
+    assert j["encode"]["frac"] > 0 and j["decode"]["frac"] > 0
+    assert j["allgather"]["bytes_received_per_rank"] == 0 and j["allgather"]["ms_per_call"] > 0
+    assert j["gpu_launches"] == 2 * 2
+
