@@ -270,3 +270,33 @@ def test_bingrad_split_search_stress(kind, scheme, d):
     n = g[0][0].size
     cg, co = configs(scheme, 2, d, W, True, 0.0, 13, n)
     compare_steps(run_gpu_fused(cg, 1, g), run_oracle_fused(co, 1, g), co, "%s %s d=%d" % (scheme, kind, d))
+
+
+@pytest.mark.parametrize("d", [128, 512])
+def test_bingrad_pb_interior_optima(d):
+    """Buckets whose best admissible pair lies strictly inside the admissible range (A below the
+    largest admissible lower index, or B above the smallest admissible upper one): integer values
+    0 .. 63 on the exact grid, from the oracle pins' interior cases repeated to the bucket size.
+    There the kernel's per-column search cannot stop at the range's corner: along a column it
+    must find an interior minimum (the bisection), and the pair must still be the exhaustive
+    scan's, bit for bit."""
+    import oracle as O
+    from test_oracle_pins import _PB_INNER, _grid32
+    rng = np.random.default_rng(77 + d)
+    buckets, inner = [], 0
+    for lst in _PB_INNER:
+        u = np.resize(np.array(lst, np.float32), d)
+        rng.shuffle(u)
+        buckets.append(u)
+        A, B, _, _ = O.bingrad_pb_fit(u)
+        a_b, b_b = O.bingrad_b_fit(u)[:2]
+        grid = _grid32(u)
+        amax = max([j for j in range(64) if grid[j] <= a_b], default=0)
+        bmin = min([j for j in range(64) if grid[j] >= b_b], default=63)
+        inner += A < amax or B > bmin
+    assert inner >= 20, inner
+    W = 2
+    g = [[np.concatenate([buckets[(i + 5 * w) % len(buckets)] for i in range(len(buckets))]) for w in range(W)]]
+    n = g[0][0].size
+    cg, co = configs("bingrad_pb", 2, d, W, True, 0.0, 21, n)
+    compare_steps(run_gpu_fused(cg, 1, g), run_oracle_fused(co, 1, g), co, "bingrad_pb interior d=%d" % d)
