@@ -272,7 +272,7 @@ def test_bingrad_split_search_stress(kind, scheme, d):
     compare_steps(run_gpu_fused(cg, 1, g), run_oracle_fused(co, 1, g), co, "%s %s d=%d" % (scheme, kind, d))
 
 
-@pytest.mark.parametrize("d", [128, 512])
+@pytest.mark.parametrize("d", [128, 512, 2048])
 def test_bingrad_pb_interior_optima(d):
     """Buckets whose best admissible pair lies strictly inside the admissible range (A below the
     largest admissible lower index, or B above the smallest admissible upper one): integer values
