@@ -487,8 +487,9 @@ def e2e_host_mode(W, n, avail, local_world):
 
 def run_e2e(args, G, plan, W, n, g, r, msgs, avg, dev, stream, world):
     """The same step through the C ABI with the gradients in pinned host memory: every step
-    copies the W gradients host -> device, runs gq_fused_step and reads the average back.  All
-    ranks take the same decisions (and so the same collective calls) whatever their memory."""
+    copies the W gradients host -> device, runs gq_fused_step and reads the average back, the
+    steps pipelined when the device holds a second set of gradients and averages.  All ranks take
+    the same decisions (and so the same collective calls) whatever their memory."""
     import torch
     try:
         with open("/proc/meminfo") as f:
@@ -512,30 +513,69 @@ def run_e2e(args, G, plan, W, n, g, r, msgs, avg, dev, stream, world):
         return {"value": None, "unit": UNIT, "error": "pinned host allocation failed on some rank"}
     for i, hg in enumerate(host_g):
         hg.copy_(g[i])
+    # Pipelined across steps when a second set of device gradients and a second average fit: step
+    # t's copy in (its own stream) fills the set step t - 1 is not reading, overlapping that
+    # step's kernel, and step t - 1's average goes out on a third stream while step t's inputs
+    # come in (PCIe carries both directions at once).  Every step still copies all of its inputs
+    # in and its average out inside the timed region.
+    try:
+        g2 = [torch.empty_like(x) for x in g]
+        avg2 = torch.empty_like(avg)
+        ok = 1
+    except Exception:
+        g2, avg2, ok = None, None, 0
+    pipelined = all_ranks_min(ok, dev) >= 1
+    if not pipelined:
+        g2, avg2 = None, None
+        torch.cuda.empty_cache()
+    gsets, avgs = ([g, g2], [avg, avg2]) if pipelined else ([g], [avg])
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    nb = len(gsets)
+    read_done = [torch.cuda.Event() for _ in range(nb)]  # the kernel that read gradient set k
+    out_done = [torch.cuda.Event() for _ in range(nb)]   # the copy out of average k
+    for k in range(nb):
+        read_done[k].record(stream)
+        out_done[k].record(stream)
 
     def step(t):
-        for w in range(W):
-            g[w].copy_(host_g[w if mode == 2 else 0], non_blocking=True)
-        G.gq_fused_step(plan.handle, 1000 + t, g, r, msgs, avg, stream)
-        host_avg.copy_(avg, non_blocking=True)
+        k = t % nb
+        s_in.wait_event(read_done[k])
+        with torch.cuda.stream(s_in):
+            for w in range(W):
+                gsets[k][w].copy_(host_g[w if mode == 2 else 0], non_blocking=True)
+        stream.wait_stream(s_in)
+        stream.wait_event(out_done[k])
+        G.gq_fused_step(plan.handle, 1000 + t, gsets[k], r, msgs, avgs[k], stream)
+        read_done[k].record(stream)
+        s_out.wait_event(read_done[k])
+        with torch.cuda.stream(s_out):
+            host_avg.copy_(avgs[k], non_blocking=True)
+        out_done[k].record(s_out)
 
     step(0)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
     for t in range(args.e2e_steps):
         step(1 + t)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     if world > 1:
         ms = max_over_ranks(ms, dev)
+    del g2, avg2
     del host_g, host_avg
     return {"value": world * W * n * args.e2e_steps / (ms / 1000.0), "unit": UNIT,
             "h2d_bytes_per_step": 4 * W * n, "d2h_bytes_per_step": 4 * n, "steps": args.e2e_steps,
             "host_gradients": "one pinned buffer per worker" if mode == 2 else
-            "one pinned buffer copied into every worker's gradient (host memory shared by %d ranks)" % local_world}
+            "one pinned buffer copied into every worker's gradient (host memory shared by %d ranks)" % local_world,
+            "pipelined": ("copies in, kernel and copy out of consecutive steps overlap (two device gradient sets)"
+                          if pipelined else "one device gradient set: copy in, kernel, copy out in sequence")}
 
 
 def run_cpu_baseline(args, wl, g):
