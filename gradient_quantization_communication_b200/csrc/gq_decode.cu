@@ -113,6 +113,139 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
     }
 }
 
+// The same decode and sum for a worker count known at compile time (2, 4 or 8), with each item's
+// code words staged in the warp's shared memory: one 1-D bulk copy (no multicast) per worker and
+// item, one item ahead on a two-stage mbarrier pipeline, so that the lanes read their code words
+// from shared memory instead of waiting on global loads.  The level tables (a few floats per
+// worker and bucket, not 16-byte aligned) are loaded into registers one item ahead.  An item's
+// copy spans its CPI chunks of the bucket's codes, which exist in full even when the vector ends
+// inside them; the message and every chunk start on 16 bytes.  Every wait is bounded: a copy that
+// does not land in time sets kStatusTimeout, the warp waits (bounded) for its other copy in
+// flight and stops.
+template <bool QSGD, int BITS, int CPI, int WK>
+struct DecodeStage {
+    static constexpr int kChunkWords = BITS == 8 ? 32 : 4 * BITS;
+    static constexpr int kItemWords = CPI * kChunkWords;
+    uint32_t w[2][WK][kItemWords];
+    unsigned long long bar[2];
+};
+
+template <bool QSGD, int BITS, int CPI, int WK>
+__global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_staged(const __grid_constant__ KParams p)
+{
+    using Stage = DecodeStage<QSGD, BITS, CPI, WK>;
+    constexpr int kWidth = BITS == 8 ? 32 : 1 << BITS;
+    constexpr int kChunkWords = Stage::kChunkWords;
+    constexpr int kItemWords = Stage::kItemWords;
+    constexpr unsigned kItemBytes = kItemWords * 4u;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    Stage &sm = reinterpret_cast<Stage *>(smem_raw)[wib];
+    const int slot = lane & (kWidth - 1);
+    const int64_t nitems = (p.n + 128 * CPI - 1) / (128 * CPI);
+    const int64_t first = (int64_t)blockIdx.x * kDecodeWarps + wib;
+    const int64_t stride = (int64_t)gridDim.x * kDecodeWarps;
+    const int log2d = 31 - __clz(p.d);
+    const int bitoff = 4 * (BITS == 8 ? 8 : BITS) * lane, wi = bitoff >> 5, sh = bitoff & 31;
+    const bool cross = BITS == 3 && sh + 12 > 32;  // the field crosses a word boundary (b = 3 only)
+    const bool has_level = slot < p.L;
+    const float qr = (QSGD && slot < p.s) ? p.qratio[slot] : 0.0f;
+    __shared__ float qtab[BITS == 8 ? 256 : 1];
+    if (BITS == 8) {
+        for (int k = threadIdx.x; k < p.s; k += blockDim.x) qtab[k] = p.qratio[k];
+        __syncthreads();
+    }
+    if (first >= nitems) return;
+    if (lane == 0) {
+        mbar_init(&sm.bar[0], 1);
+        mbar_init(&sm.bar[1], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    auto issue = [&](int64_t it, int k) {  // lane 0: the item's code words of every worker
+        const int64_t e0 = it * (128 * CPI);
+        const int64_t off = (e0 >> log2d) * p.codes_words + (int64_t)((e0 & (p.d - 1)) >> 7) * kChunkWords;
+        fence_proxy_async();
+        mbar_arrive_expect_tx(&sm.bar[k], WK * kItemBytes);
+#pragma unroll
+        for (int w = 0; w < WK; ++w)
+            bulk_load(sm.w[k][w], reinterpret_cast<const uint32_t *>(p.msg[w]) + off, kItemBytes, &sm.bar[k]);
+    };
+    auto levels = [&](int64_t it, float (&lv)[WK]) {
+        const int64_t bk = (it * (128 * CPI)) >> log2d;
+        const int64_t tbase = QSGD ? bk : bk * p.L + slot;
+#pragma unroll
+        for (int w = 0; w < WK; ++w)
+            lv[w] = (QSGD || has_level) ? __ldg(reinterpret_cast<const float *>(p.msg[w] + p.levels_off) + tbase) : 0.0f;
+    };
+    if (lane == 0) issue(first, 0);
+    float lv[WK];
+    levels(first, lv);
+    unsigned parity = 0;  // bit k: phase parity awaited next on stage k
+    int k = 0;
+    for (int64_t it = first; it < nitems; it += stride) {
+        const int64_t nxt = it + stride;
+        if (lane == 0 && nxt < nitems) issue(nxt, k ^ 1);
+        if (!mbar_wait_warp(&sm.bar[k], (parity >> k) & 1u)) {
+            // report it, give both copies still in flight one more bounded wait so that none can
+            // land after the warp has left, and stop
+            if (lane == 0) atomicOr(p.status, kStatusTimeout);
+            mbar_wait_warp(&sm.bar[k], (parity >> k) & 1u);
+            if (nxt < nitems) mbar_wait_warp(&sm.bar[k ^ 1], (parity >> (k ^ 1)) & 1u);
+            return;
+        }
+        parity ^= 1u << k;
+        float lvn[WK];
+        if (nxt < nitems) levels(nxt, lvn);
+        const int64_t e0 = it * (128 * CPI);
+        int nlive = (int)((p.n - e0 + 127) >> 7);
+        nlive = nlive < CPI ? nlive : CPI;
+        float acc[CPI][4];
+#pragma unroll
+        for (int c = 0; c < CPI; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
+#pragma unroll
+        for (int w = 0; w < WK; ++w) {
+            const uint32_t *cw = sm.w[k][w];
+            if (BITS == 8) {
+#pragma unroll
+                for (int c = 0; c < CPI; ++c) {
+                    const uint32_t x = cw[c * kChunkWords + lane];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        acc[c][e] = __fadd_rn(acc[c][e], __fmul_rn(lv[w], qtab[(x >> (8 * e)) & 0xffu]));
+                }
+            } else {
+                const float level = QSGD ? __fmul_rn(lv[w], qr) : lv[w];
+#pragma unroll
+                for (int c = 0; c < CPI; ++c) {
+                    uint32_t f = cw[c * kChunkWords + wi] >> sh;
+                    if (cross) f |= cw[c * kChunkWords + wi + 1] << (32 - sh);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, (int)(f >> (BITS * e)), kWidth));
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < CPI; ++c) {
+            const int64_t e = e0 + 128 * c + 4 * lane;
+            if (c < nlive && e + 3 < p.n) {
+                __stcs(reinterpret_cast<float4 *>(p.avg + e),
+                       make_float4(__fmul_rn(acc[c][0], p.inv_w), __fmul_rn(acc[c][1], p.inv_w),
+                                   __fmul_rn(acc[c][2], p.inv_w), __fmul_rn(acc[c][3], p.inv_w)));
+            } else if (c < nlive) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (e + q < p.n) p.avg[e + q] = __fmul_rn(acc[c][q], p.inv_w);
+            }
+        }
+        __syncwarp();  // every lane has read stage k before it is filled again
+#pragma unroll
+        for (int w = 0; w < WK; ++w) lv[w] = lvn[w];
+        k ^= 1;
+    }
+}
+
 // Base-s messages (s = 3, 5, 9; d <= 512): the same items and sum, with each lane's four codes
 // of a chunk taken from the one or two base-s groups that hold them (base_codes4); the code words
 // of kBaseGroup workers are loaded before any is decoded.
@@ -201,25 +334,39 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base(const __grid_
     }
 }
 
-template <bool QSGD, int BITS, int CPI>
-cudaError_t launch(const KParams &p, cudaStream_t stream)
+template <class K>
+cudaError_t launch_items(K kern, const KParams &p, int cpi, size_t smem, cudaStream_t stream)
 {
-    auto kern = p.W == 8   ? k_decode<QSGD, BITS, CPI, 8>
-                : p.W == 4 ? k_decode<QSGD, BITS, CPI, 4>
-                : p.W == 2 ? k_decode<QSGD, BITS, CPI, 2>
-                           : k_decode<QSGD, BITS, CPI>;
+    if (smem > 0 && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return cudaGetLastError();
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecodeWarps * 32, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecodeWarps * 32, smem);
     if (per_sm < 1) per_sm = 1;
-    const int64_t nitems = (p.n + 128 * CPI - 1) / (128 * CPI);
+    const int64_t nitems = (p.n + 128 * cpi - 1) / (128 * cpi);
     const int64_t need = (nitems + kDecodeWarps - 1) / kDecodeWarps;
     const int64_t cap = (int64_t)sms * per_sm;
     const int grid = (int)(need < cap ? need : cap);
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kDecodeWarps * 32, 0, stream>>>(p);
+    kern<<<grid, kDecodeWarps * 32, smem, stream>>>(p);
     return cudaGetLastError();
+}
+
+template <bool QSGD, int BITS, int CPI, int WK>
+cudaError_t launch_staged(const KParams &p, cudaStream_t stream)
+{
+    return launch_items(k_decode_staged<QSGD, BITS, CPI, WK>, p, CPI,
+                        sizeof(DecodeStage<QSGD, BITS, CPI, WK>) * kDecodeWarps, stream);
+}
+
+template <bool QSGD, int BITS, int CPI>
+cudaError_t launch(const KParams &p, cudaStream_t stream)
+{
+    if (p.W == 8) return launch_staged<QSGD, BITS, CPI, 8>(p, stream);
+    if (p.W == 4) return launch_staged<QSGD, BITS, CPI, 4>(p, stream);
+    if (p.W == 2) return launch_staged<QSGD, BITS, CPI, 2>(p, stream);
+    return launch_items(k_decode<QSGD, BITS, CPI>, p, CPI, 0, stream);
 }
 
 // Chunks per item: a whole bucket for d = 128, 256, four chunks of it for larger buckets.
