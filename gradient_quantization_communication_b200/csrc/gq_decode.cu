@@ -8,9 +8,10 @@
 // is a register shuffle within segments of 2^b lanes: every segment holds the bucket's level
 // table in its first L lanes, and a shuffle of width 2^b takes its source lane modulo 2^b, so
 // the code needs no masking (8-bit codes of the QSGD family look their ratio up in a shared
-// table instead).  The loads of a group of workers are issued together before any
-// of them is used; the sum runs in worker order in registers and the average is written once,
-// with 16-byte stores.
+// table instead).  For 1, 2, 4 and 8 workers the item's code words of every worker come into
+// shared memory by bulk copies one item ahead (k_decode_staged); for other counts the loads of a
+// group of workers are issued together before any of them is used (k_decode).  The sum runs in
+// worker order in registers and the average is written once, with 16-byte stores.
 #include "gq_bases.cuh"
 #include "gq_device.cuh"
 
@@ -19,13 +20,13 @@ namespace {
 
 constexpr int kDecodeWarps = 4;
 
-// WK: the worker count when known at compile time (2, 4 or 8: the loops unroll with no guards,
-// and up to 8 workers' loads are in flight together), 0 for any other count (4 at a time).
-template <bool QSGD, int BITS, int CPI, int WK = 0>
+// Any worker count (the counts 1, 2, 4 and 8 go to k_decode_staged below): the loads of four
+// workers are issued before any of them is used.
+template <bool QSGD, int BITS, int CPI>
 __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_constant__ KParams p)
 {
-    constexpr int kDecodeGroup = WK > 0 ? (WK < 8 ? WK : 8) : 4;  // workers whose loads are in flight together
-    const int W = WK > 0 ? WK : p.W;
+    constexpr int kDecodeGroup = 4;  // workers whose loads are in flight together
+    const int W = p.W;
     constexpr int kWidth = 1 << BITS;
     constexpr int kChunkWords = 4 * BITS;  // words of one chunk's codes
     const int lane = threadIdx.x & 31;
@@ -113,7 +114,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
     }
 }
 
-// The same decode and sum for a worker count known at compile time (2, 4 or 8), with each item's
+// The same decode and sum for a worker count known at compile time (1, 2, 4 or 8), with each item's
 // code words staged in the warp's shared memory: one 1-D bulk copy (no multicast) per worker and
 // item, one item ahead on a two-stage mbarrier pipeline, so that the lanes read their code words
 // from shared memory instead of waiting on global loads.  The level tables (a few floats per
@@ -366,6 +367,7 @@ cudaError_t launch(const KParams &p, cudaStream_t stream)
     if (p.W == 8) return launch_staged<QSGD, BITS, CPI, 8>(p, stream);
     if (p.W == 4) return launch_staged<QSGD, BITS, CPI, 4>(p, stream);
     if (p.W == 2) return launch_staged<QSGD, BITS, CPI, 2>(p, stream);
+    if (p.W == 1) return launch_staged<QSGD, BITS, CPI, 1>(p, stream);
     return launch_items(k_decode<QSGD, BITS, CPI>, p, CPI, 0, stream);
 }
 
