@@ -335,6 +335,134 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base(const __grid_
     }
 }
 
+// Base-s words staged like the dense ones (1, 2, 4 or 8 workers, d <= 512 so that an item is a
+// bucket).  A bucket's nw words start on any word, so each worker's copy takes the 16-byte units
+// that hold them, at most nw + 6 words (the codes region ends on 16 bytes), and the lanes index
+// from the bucket's offset in them.  A lane's second word is read only inside the bucket, as in
+// k_decode_base.
+template <int S, int CPI>
+struct BaseStageDims {
+    static constexpr int kWords = ((CPI * 128 + BaseS<S>::g - 1) / BaseS<S>::g * BaseS<S>::B + 31) / 32;
+    static constexpr int kStageWords = (kWords + 6 + 3) & ~3;
+};
+template <int S, int CPI, int WK>
+struct BaseDecodeStage {
+    uint32_t w[2][WK][BaseStageDims<S, CPI>::kStageWords];
+    unsigned long long bar[2];
+};
+
+template <bool QSGD, int S, int CPI, int WK>
+__global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base_staged(const __grid_constant__ KParams p)
+{
+    using Stage = BaseDecodeStage<S, CPI, WK>;
+    constexpr int BITS = S == 3 ? 2 : S == 5 ? 3 : 4;  // the level lookup's segment: 2^b lanes
+    constexpr int kWidth = 1 << BITS;
+    constexpr int nw = BaseStageDims<S, CPI>::kWords;  // the bucket's words (the host checked p.codes_words)
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    Stage &sm = reinterpret_cast<Stage *>(smem_raw)[wib];
+    const int slot = lane & (kWidth - 1);
+    const int64_t nitems = (p.n + 128 * CPI - 1) / (128 * CPI);
+    const int64_t first = (int64_t)blockIdx.x * kDecodeWarps + wib;
+    const int64_t stride = (int64_t)gridDim.x * kDecodeWarps;
+    const bool has_level = slot < p.L;
+    const float qr = (QSGD && slot < p.s) ? p.qratio[slot] : 0.0f;
+    __shared__ DigitTab<S> tab;
+    build_digit_tab<S>(tab);
+    __syncthreads();
+    if (first >= nitems) return;
+    if (lane == 0) {
+        mbar_init(&sm.bar[0], 1);
+        mbar_init(&sm.bar[1], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    BasePos ps[CPI];
+#pragma unroll
+    for (int c = 0; c < CPI; ++c) ps[c] = base_pos<S>(4 * lane + 128 * c);
+    auto span = [&](int64_t it, int64_t &a0, int &off, int &words) {
+        const int64_t sw = it * nw;  // item = bucket
+        a0 = sw & ~int64_t(3);
+        off = (int)(sw - a0);
+        words = (int)(((sw + nw + 3) & ~int64_t(3)) - a0);
+    };
+    auto issue = [&](int64_t it, int k) {  // lane 0
+        int64_t a0;
+        int off, words;
+        span(it, a0, off, words);
+        fence_proxy_async();
+        mbar_arrive_expect_tx(&sm.bar[k], (unsigned)(WK * words * 4));
+#pragma unroll
+        for (int w = 0; w < WK; ++w)
+            bulk_load(sm.w[k][w], reinterpret_cast<const uint32_t *>(p.msg[w]) + a0, (unsigned)(words * 4), &sm.bar[k]);
+    };
+    auto levels = [&](int64_t it, float (&lv)[WK]) {
+        const int64_t tbase = QSGD ? it : it * p.L + slot;
+#pragma unroll
+        for (int w = 0; w < WK; ++w)
+            lv[w] = (QSGD || has_level) ? __ldg(reinterpret_cast<const float *>(p.msg[w] + p.levels_off) + tbase) : 0.0f;
+    };
+    if (lane == 0) issue(first, 0);
+    float lv[WK];
+    levels(first, lv);
+    unsigned parity = 0;
+    int k = 0;
+    for (int64_t it = first; it < nitems; it += stride) {
+        const int64_t nxt = it + stride;
+        if (lane == 0 && nxt < nitems) issue(nxt, k ^ 1);
+        if (!mbar_wait_warp(&sm.bar[k], (parity >> k) & 1u)) {
+            if (lane == 0) atomicOr(p.status, kStatusTimeout);
+            mbar_wait_warp(&sm.bar[k], (parity >> k) & 1u);
+            if (nxt < nitems) mbar_wait_warp(&sm.bar[k ^ 1], (parity >> (k ^ 1)) & 1u);
+            return;
+        }
+        parity ^= 1u << k;
+        float lvn[WK];
+        if (nxt < nitems) levels(nxt, lvn);
+        const int64_t e0 = it * (128 * CPI);
+        int nlive = (int)((p.n - e0 + 127) >> 7);
+        nlive = nlive < CPI ? nlive : CPI;
+        int64_t a0;
+        int off, words;
+        span(it, a0, off, words);
+        float acc[CPI][4];
+#pragma unroll
+        for (int c = 0; c < CPI; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
+#pragma unroll
+        for (int w = 0; w < WK; ++w) {
+            const uint32_t *bw = sm.w[k][w] + off;
+            const float level = QSGD ? __fmul_rn(lv[w], qr) : lv[w];
+#pragma unroll
+            for (int c = 0; c < CPI; ++c) {
+                const uint32_t lo = bw[ps[c].wi];
+                const uint32_t hi = ps[c].wi + 1 < nw ? bw[ps[c].wi + 1] : 0u;
+                int code[4];
+                base_codes4<S>(tab, lo, hi, ps[c], code);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, code[e], kWidth));
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < CPI; ++c) {
+            const int64_t e = e0 + 128 * c + 4 * lane;
+            if (c < nlive && e + 3 < p.n) {
+                __stcs(reinterpret_cast<float4 *>(p.avg + e),
+                       make_float4(__fmul_rn(acc[c][0], p.inv_w), __fmul_rn(acc[c][1], p.inv_w),
+                                   __fmul_rn(acc[c][2], p.inv_w), __fmul_rn(acc[c][3], p.inv_w)));
+            } else if (c < nlive) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (e + q < p.n) p.avg[e + q] = __fmul_rn(acc[c][q], p.inv_w);
+            }
+        }
+        __syncwarp();  // every lane has read stage k before it is filled again
+#pragma unroll
+        for (int w = 0; w < WK; ++w) lv[w] = lvn[w];
+        k ^= 1;
+    }
+}
+
 template <class K>
 cudaError_t launch_items(K kern, const KParams &p, int cpi, size_t smem, cudaStream_t stream)
 {
@@ -385,6 +513,15 @@ cudaError_t launch_cpi(const KParams &p, cudaStream_t stream)
 template <bool QSGD, int S, int CPI>
 cudaError_t launch_base(const KParams &p, cudaStream_t stream)
 {
+    if (p.codes_words == BaseStageDims<S, CPI>::kWords && CPI * 128 == p.d) {
+        switch (p.W) {
+        case 8: return launch_items(k_decode_base_staged<QSGD, S, CPI, 8>, p, CPI, sizeof(BaseDecodeStage<S, CPI, 8>) * kDecodeWarps, stream);
+        case 4: return launch_items(k_decode_base_staged<QSGD, S, CPI, 4>, p, CPI, sizeof(BaseDecodeStage<S, CPI, 4>) * kDecodeWarps, stream);
+        case 2: return launch_items(k_decode_base_staged<QSGD, S, CPI, 2>, p, CPI, sizeof(BaseDecodeStage<S, CPI, 2>) * kDecodeWarps, stream);
+        case 1: return launch_items(k_decode_base_staged<QSGD, S, CPI, 1>, p, CPI, sizeof(BaseDecodeStage<S, CPI, 1>) * kDecodeWarps, stream);
+        default: break;
+        }
+    }
     auto kern = k_decode_base<QSGD, S, CPI>;
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
