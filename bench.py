@@ -24,6 +24,9 @@ Other one-line modes (one GPU):
               odd-level QSGD-family scheme such as --scheme qsgd_l2 --levels 3
   --exchange  the data-parallel exchange (exchange.Exchange): one worker per rank under
               torchrun, gq_encode + NCCL all-gather of the packed messages + gq_decode_accumulate
+  --scheme terngrad_layer --workload resnet50
+              TernGrad with one scale per parameter tensor (two passes: the tensors' maxima,
+              then the rounding)
 """
 import argparse
 import concurrent.futures as cf
@@ -682,6 +685,74 @@ def run_unfused(args):
     return 0
 
 
+def run_layer(args):
+    """TernGrad with one scale per parameter tensor (--scheme terngrad_layer) on a workload with
+    tensor structure (resnet18 / resnet50: their parameter tensors; blocks1b: its 1e6-element
+    blocks).  The fused step is two launches: the per-tensor maxima of |g + r| (a pass over g and
+    r), then the rounding, residual, message and average (a second pass).  Both passes belong to
+    the method: an element's scale depends on its whole tensor, which is far larger than the
+    chip's memory for most tensors, so the algorithmic bytes count g and r twice."""
+    import torch
+
+    import gradient_quantization_communication_b200.gq as G
+    from gradient_quantization_communication_b200 import synth
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    if args.elements:
+        wl = dataclasses.replace(wl, n=min(wl.n, args.elements))
+    W, n, d, ef = wl.workers, wl.n, args.bucket, wl.error_feedback
+    off = synth.tensor_offsets(args.workload, n)
+    nseg = len(off) - 1
+    cfg = G.gq_config(G.SCHEMES["terngrad_layer"], 3, d, W, ef, 0.0, wl.rounding_seed, n)
+    plan = G.Plan(cfg, segments=off)
+    stream = torch.cuda.current_stream()
+    g = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
+    for w in range(W):
+        synth.gradient(args.workload, w, 0, n=n, out=g[w])
+    r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)] if ef else None
+    msgs = [torch.empty(plan.msg_bytes, dtype=torch.uint8, device=dev) for _ in range(W)]
+    avg = torch.empty(n, dtype=torch.float32, device=dev)
+    for t in range(args.warmup):
+        G.gq_fused_step(plan.handle, t, g, r, msgs, avg, stream)
+    torch.cuda.synchronize()
+    if G.gq_plan_status(plan.handle, stream) != G.GQ_OK:
+        raise RuntimeError("non-finite input in the benchmark workload")
+    sampler = ClockSampler(pci_bus_id(dev))
+    sampler.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        G.gq_fused_step(plan.handle, args.warmup + k, g, r, msgs, avg, stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    msg_bytes = plan.msg_bytes
+    plan.close()
+    rw = 8.0 if ef else 4.0  # g (and r) per element and pass
+    bpe = 2.0 * rw + (4.0 if ef else 0.0) + msg_bytes / n + 4.0 / W
+    peak, peak_kind = measured_hbm_peak()
+    achieved = bpe * W * n / (ms / 1000.0) / 1e9
+    config = workload_config(args, wl)
+    config.update({"scheme": "terngrad_layer", "levels": 3, "tensors": nseg,
+                   "workload": "%s: %d fp32 elements in %d tensors x W=%d workers, terngrad_layer (one scale per "
+                               "tensor), error feedback %s" % (args.workload, n, nseg, W, "on" if ef else "off")})
+    print(json.dumps({
+        "metric": "TernGrad with one scale per tensor, fused step, worker-elements/s", "value": W * n / (ms / 1000.0),
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "f32", "data": "synthetic", "config": config,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "traffic": None,
+                     "algorithmic_bytes_per_worker_elem": bpe,
+                     "note": "both passes over g and r counted: the per-tensor scale needs the whole tensor first"},
+        "gpu_launches": 2 * args.steps, "clocks": clocks}))
+    return 0
+
+
 # Measured peer copy between two B200s of this pool over NVLink, one direction (900 nominal).
 PEER_LINK_GBS = 770.0
 
@@ -1066,6 +1137,8 @@ def main():
         return run_elias(args)
     if args.exchange:
         return run_exchange(args)
+    if args.scheme == "terngrad_layer":
+        return run_layer(args)
     return run_gq(args)
 
 

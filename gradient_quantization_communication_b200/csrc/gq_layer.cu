@@ -10,17 +10,21 @@
 // The message is the dense message's codes region (2-bit codes, bucket after bucket: since a
 // bucket is a whole number of 128-element chunks, chunk c's codes are words 8c .. 8c+7) followed
 // by the nseg scales.  Three kernels:
-//   k_layer_max     grid (chunks, W): every warp's 512-element slice, |v| per element, one
-//                   atomicMax (float bits, NaN above +inf) per lane and tensor it touches into
-//                   the plan's scale scratch, zeroed before;
-//   k_layer_encode  a warp per 128-element chunk, grid-stride: per worker v, the tensor's scale,
-//                   the rounding, the residual, the packed codes; the W dequantized values are
-//                   summed in registers in worker order and the average written once (fused);
-//                   the scales are copied into each message, and the codes of the last bucket's
-//                   chunks past n are written as zeros;
-//   k_layer_decode  a warp per chunk: the W messages' codes and scales, summed in worker order.
-// A lane finds the tensor of its first element by binary search over the offsets and walks
-// forward over the boundaries inside its four elements.
+//   k_layer_max     grid (x, W): every warp a contiguous run of 512-element slices, |v| per
+//                   element, a running maximum per lane and tensor, published by atomicMax
+//                   (float bits, NaN above +inf) into the plan's scale scratch, zeroed before;
+//                   the lanes that end on one tensor reduce first, so that a tensor's word sees
+//                   about one atomic per warp;
+//   k_layer_encode  every warp a contiguous run of 128-element chunks: per worker v, the
+//                   tensor's scale (its reciprocal once per chunk when the lane's four elements
+//                   share a tensor), the rounding, the residual, the packed codes; the W
+//                   dequantized values are summed in registers in worker order and the average
+//                   written once (fused); the scales are copied into each message, and the codes
+//                   of the last bucket's chunks past n are written as zeros;
+//   k_layer_decode  the same runs of chunks: the W messages' codes and scales, summed in worker
+//                   order.
+// A lane finds the tensor of its first element once by binary search over the offsets; its
+// elements rise, so after that it only walks forward over the tensor boundaries it reaches.
 #include "gq_round.cuh"
 
 namespace gq {
@@ -40,21 +44,14 @@ __device__ __forceinline__ int segment_of(const int64_t *off, int nseg, int64_t 
     return lo;
 }
 
-// The tensors of four consecutive elements i0 .. i0 + 3 (seg[c] for element i0 + c).
-__device__ __forceinline__ void segments4(const int64_t *off, int nseg, int64_t i0, int (&seg)[4])
-{
-    int t = segment_of(off, nseg, i0);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        while (t + 1 < nseg && __ldg(off + t + 1) <= i0 + c) ++t;
-        seg[c] = t;
-    }
-}
-
 __device__ __forceinline__ float scale_of(const unsigned int *bits, int t) { return __uint_as_float(bits[t]); }
 
-// Largest |v| per worker and tensor: grid.y = worker; each warp a slice of 512 elements
-// (lane l: elements 4l .. 4l+3 of each of four 128-element chunks).
+// Largest |v| per worker and tensor: grid.y = worker; each warp a contiguous run of slices of
+// 512 elements (lane l: elements 4l .. 4l+3 of each of four 128-element chunks), so that a lane's
+// elements rise and it keeps one running maximum per tensor across slices.  A lane publishes its
+// maximum (atomicMax on the bits: |v| >= 0 orders like its bits, NaN above everything) when its
+// tensor changes; at the end the warp first reduces the maxima of the lanes that share a tensor,
+// so that a tensor's word sees about one atomic per warp instead of one per lane and slice.
 __global__ void __launch_bounds__(kLayerWarps * 32) k_layer_max(const __grid_constant__ KParams p)
 {
     const int lane = threadIdx.x & 31;
@@ -63,10 +60,16 @@ __global__ void __launch_bounds__(kLayerWarps * 32) k_layer_max(const __grid_con
     const float *r = p.r[w];
     unsigned int *smax = p.seg_max + (int64_t)w * p.nseg;
     const int64_t nslices = (p.n + 511) / 512;
-    for (int64_t sl = (int64_t)blockIdx.x * kLayerWarps + (threadIdx.x >> 5); sl < nslices;
-         sl += (int64_t)gridDim.x * kLayerWarps) {
-        int cur = -1;
-        float run = 0.0f;
+    const int64_t nwarps = (int64_t)gridDim.x * kLayerWarps;
+    const int64_t per = (nslices + nwarps - 1) / nwarps;
+    const int64_t s0 = ((int64_t)blockIdx.x * kLayerWarps + (threadIdx.x >> 5)) * per;
+    const int64_t s1 = s0 + per < nslices ? s0 + per : nslices;
+    int cur = -1;
+    float run = 0.0f;
+    // the lane's tensor and the next tensor's first element, advanced as its elements rise
+    int t = s0 < s1 ? segment_of(p.seg_off, p.nseg, min(s0 * 512 + 4 * lane, p.n - 1)) : 0;
+    int64_t nextb = t + 1 < p.nseg ? __ldg(p.seg_off + t + 1) : INT64_MAX;
+    for (int64_t sl = s0; sl < s1; ++sl) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int64_t i0 = sl * 512 + 128 * j + 4 * lane;
@@ -83,20 +86,28 @@ __global__ void __launch_bounds__(kLayerWarps * 32) k_layer_max(const __grid_con
 #pragma unroll
                 for (int c = 0; c < 4; ++c) v[c] = i0 + c < p.n ? (r ? __fadd_rn(g[i0 + c], r[i0 + c]) : g[i0 + c]) : 0.0f;
             }
-            int seg[4];
-            segments4(p.seg_off, p.nseg, i0, seg);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 if (i0 + c >= p.n) break;
-                if (seg[c] != cur) {
+                while (i0 + c >= nextb) {  // empty tensors are passed over
+                    ++t;
+                    nextb = t + 1 < p.nseg ? __ldg(p.seg_off + t + 1) : INT64_MAX;
+                }
+                if (t != cur) {
                     if (cur >= 0) atomicMax(smax + cur, __float_as_uint(run));
-                    cur = seg[c];
+                    cur = t;
                     run = 0.0f;
                 }
                 run = fmax_nan(run, fabsf(v[c]));
             }
         }
-        if (cur >= 0) atomicMax(smax + cur, __float_as_uint(run));
+    }
+    const int c0 = __shfl_sync(kFull, cur, 0);
+    if (__all_sync(kFull, cur == c0)) {
+        const unsigned m = __reduce_max_sync(kFull, __float_as_uint(run));
+        if (lane == 0 && c0 >= 0) atomicMax(smax + c0, m);
+    } else if (cur >= 0) {
+        atomicMax(smax + cur, __float_as_uint(run));
     }
 }
 
@@ -115,14 +126,29 @@ __global__ void __launch_bounds__(kLayerWarps * 32) k_layer_encode(const __grid_
             for (int64_t t = gtid; t < pad; t += (int64_t)gridDim.x * blockDim.x)
                 tab[t] = t < p.nseg ? scale_of(p.seg_max + (int64_t)w * p.nseg, (int)t) : 0.0f;
         }
-    for (int64_t ch = (int64_t)blockIdx.x * kLayerWarps + (threadIdx.x >> 5); ch < nchunks;
-         ch += (int64_t)gridDim.x * kLayerWarps) {
+    // each warp a contiguous run of chunks, so that a lane's elements rise and its tensor index
+    // only advances (no search per chunk)
+    const int64_t nwarps = (int64_t)gridDim.x * kLayerWarps;
+    const int64_t per = (nchunks + nwarps - 1) / nwarps;
+    const int64_t c0 = ((int64_t)blockIdx.x * kLayerWarps + (threadIdx.x >> 5)) * per;
+    const int64_t c1 = c0 + per < nchunks ? c0 + per : nchunks;
+    int t = c0 < c1 ? segment_of(p.seg_off, p.nseg, min(c0 * 128 + 4 * lane, p.n - 1)) : 0;
+    int64_t nextb = t + 1 < p.nseg ? __ldg(p.seg_off + t + 1) : INT64_MAX;
+    for (int64_t ch = c0; ch < c1; ++ch) {
         const int64_t i0 = ch * 128 + 4 * lane;
         uint32_t valid = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) valid |= (i0 + c < p.n ? 1u : 0u) << c;
-        int seg[4] = {0, 0, 0, 0};
-        if (valid) segments4(p.seg_off, p.nseg, i0, seg);
+        int seg[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            while (i0 + c >= nextb && i0 + c < p.n) {  // empty tensors are passed over
+                ++t;
+                nextb = t + 1 < p.nseg ? __ldg(p.seg_off + t + 1) : INT64_MAX;
+            }
+            seg[c] = t;
+        }
+        const bool one_seg = seg[0] == seg[3];  // the common case: one scale for the lane's four
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for (int w = 0; w < p.W; ++w) {
             const float *g = p.g[w];
@@ -145,10 +171,12 @@ __global__ void __launch_bounds__(kLayerWarps * 32) k_layer_encode(const __grid_
             const unsigned int *smax = p.seg_max + (int64_t)w * p.nseg;
             int code[4];
             float q[4];
+            const float m0 = scale_of(smax, seg[0]);
+            const float inv_m0 = m0 > 0.0f ? __frcp_rn(m0) : 0.0f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const float m = scale_of(smax, seg[c]);
-                const float inv_m = m > 0.0f ? __frcp_rn(m) : 0.0f;
+                const float m = one_seg ? m0 : scale_of(smax, seg[c]);
+                const float inv_m = one_seg ? inv_m0 : (m > 0.0f ? __frcp_rn(m) : 0.0f);
                 const float y = __fadd_rn(__fmul_rn(v[c], inv_m), 1.0f);  // (v / m + 1) * (s - 1) / 2, s = 3
                 const int k = min(max(__float2int_rz(y), 0), 1);
                 const float pu = __fsub_rn(y, (float)k);
@@ -200,12 +228,25 @@ __global__ void __launch_bounds__(kLayerWarps * 32) k_layer_decode(const __grid_
 {
     const int lane = threadIdx.x & 31;
     const int64_t nchunks = (p.n + 127) / 128;
-    for (int64_t ch = (int64_t)blockIdx.x * kLayerWarps + (threadIdx.x >> 5); ch < nchunks;
-         ch += (int64_t)gridDim.x * kLayerWarps) {
+    // contiguous runs of chunks per warp: the lane's tensor index only advances
+    const int64_t nwarps = (int64_t)gridDim.x * kLayerWarps;
+    const int64_t per = (nchunks + nwarps - 1) / nwarps;
+    const int64_t c0 = ((int64_t)blockIdx.x * kLayerWarps + (threadIdx.x >> 5)) * per;
+    const int64_t c1 = c0 + per < nchunks ? c0 + per : nchunks;
+    int t = c0 < c1 ? segment_of(p.seg_off, p.nseg, min(c0 * 128 + 4 * lane, p.n - 1)) : 0;
+    int64_t nextb = t + 1 < p.nseg ? __ldg(p.seg_off + t + 1) : INT64_MAX;
+    for (int64_t ch = c0; ch < c1; ++ch) {
         const int64_t i0 = ch * 128 + 4 * lane;
         if (i0 >= p.n) continue;
         int seg[4];
-        segments4(p.seg_off, p.nseg, i0, seg);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            while (i0 + c >= nextb && i0 + c < p.n) {  // empty tensors are passed over
+                ++t;
+                nextb = t + 1 < p.nseg ? __ldg(p.seg_off + t + 1) : INT64_MAX;
+            }
+            seg[c] = t;
+        }
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for (int w = 0; w < p.W; ++w) {
             const unsigned char *msg = p.msg[w];

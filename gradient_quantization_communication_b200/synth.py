@@ -129,6 +129,26 @@ WORKLOADS = {
 }
 
 
+def tensor_offsets(workload: str, n: int = None) -> List[int]:
+    """The parameter tensors of a workload with tensor structure, as offsets into its gradient
+    (nseg + 1 values from 0 to n): resnet18 / resnet50, their parameter tensors in order;
+    blocks1b, its 1e6-element blocks.  ``n`` truncates the vector (the last tensor is cut)."""
+    wl = WORKLOADS[workload]
+    n = wl.n if n is None else int(n)
+    if workload in ("resnet18", "resnet50"):
+        sizes = resnet_param_sizes(18 if workload == "resnet18" else 50)
+    elif workload == "blocks1b":
+        sizes = [1_000_000] * ((n + 999_999) // 1_000_000)
+    else:
+        raise KeyError("%s has no tensor structure" % workload)
+    off = [0]
+    for sz in sizes:
+        if off[-1] >= n:
+            break
+        off.append(min(n, off[-1] + sz))
+    return off
+
+
 def gradient(workload: str, worker: int, step: int, n: int = None, device="cpu",
              out: torch.Tensor = None) -> torch.Tensor:
     """Worker ``worker``'s fp32 gradient at ``step`` for ``workload``.

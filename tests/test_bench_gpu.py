@@ -84,3 +84,12 @@ def test_exchange_line():
     assert j["allgather"]["bytes_received_per_rank"] == 0 and j["allgather"]["ms_per_call"] > 0
     assert j["gpu_launches"] == 2 * 2
 
+
+
+@pytest.mark.gpu
+def test_terngrad_layer_line():
+    j = _run("--scheme", "terngrad_layer", "--workload", "resnet18", "--elements", "3000000", "--steps", "2",
+             "--warmup", "3")
+    assert j["value"] > 0 and j["config"]["tensors"] >= 2 and j["gpu_launches"] == 4
+    r = j["roofline"]
+    assert r["bound"] == "hbm" and 0 < r["frac"] < 2 and r["algorithmic_bytes_per_worker_elem"] > 20

@@ -91,3 +91,17 @@ def test_message_bytes_match_the_oracle_layouts(scheme, levels, d):
     assert 0 <= O.entropy_layout(co)[0] - bases < 32
     args = _args("--base-s", "--levels", str(levels))
     assert args.base_s
+
+
+def test_tensor_offsets():
+    """The per-tensor TernGrad bench's tensors: the parameter tensors of the resnet workloads and
+    the 1e6-element blocks of blocks1b, as offsets from 0 to n, cut at a truncated n."""
+    off = synth.tensor_offsets("resnet50")
+    assert len(off) - 1 == 161 and off[0] == 0 and off[-1] == synth.WORKLOADS["resnet50"].n
+    assert all(b > a for a, b in zip(off, off[1:]))
+    assert [b - a for a, b in zip(off, off[1:])] == synth.resnet_param_sizes(50)
+    assert synth.tensor_offsets("blocks1b", 2_500_000) == [0, 1_000_000, 2_000_000, 2_500_000]
+    cut = synth.tensor_offsets("resnet18", 100_000)
+    assert cut[-1] == 100_000 and all(b > a for a, b in zip(cut, cut[1:]))
+    with pytest.raises(KeyError):
+        synth.tensor_offsets("mixture100m")

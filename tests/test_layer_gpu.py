@@ -97,3 +97,14 @@ def test_segments_required_and_checked():
         G.gq_plan_set_segments(plan.handle, [0, 400, n])
         assert G.gq_plan_message_layout(plan.handle)[0] == O.tg_layer_layout(
             O.Config(G.GQ_TERNGRAD_LAYER, 3, 128, 1, 0, 0.0, 1, n), 2)[0]
+
+
+def test_long_vector_many_tensors():
+    """More chunks than the grid has warps, so that every warp walks a run of chunks and slices
+    across many tensor boundaries (random sizes from 0 to 40000, so boundaries fall inside a
+    lane's four elements, across chunk edges, and empty tensors follow each other)."""
+    rng = np.random.default_rng(21)
+    n = 3_000_000 + 13
+    sizes = rng.integers(0, 40000, 400)
+    sizes[rng.integers(0, 400, 40)] = 0
+    _run(n, 512, 2, 1, _offsets(n, sizes.tolist()), True, seed=22)
