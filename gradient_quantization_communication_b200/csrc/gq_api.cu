@@ -4,7 +4,9 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
+#include <vector>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -26,6 +28,49 @@ struct gq_plan {
     int fmt_s;             // base-s messages of s levels (GQ_FORMAT_BASE_S), 0 = dense
     int64_t base_words;    // base-s words per bucket
 };
+
+namespace gq {
+
+cudaError_t kernel_occupancy(const void *kern, int threads, size_t smem, int *per_sm, int *sms)
+{
+    struct Entry {
+        const void *kern;
+        int threads, device;
+        size_t smem;
+        int per_sm, sms;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const Entry &x : cache)
+            if (x.kern == kern && x.threads == threads && x.smem == smem && x.device == dev) {
+                *per_sm = x.per_sm;
+                *sms = x.sms;
+                return cudaSuccess;
+            }
+    }
+    if (smem > 0) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    int n_sm = 0, per = 0;
+    e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (per < 1) per = 1;
+    *per_sm = per;
+    *sms = n_sm;
+    std::lock_guard<std::mutex> lock(mu);
+    cache.push_back(Entry{kern, threads, dev, smem, per, n_sm});
+    return cudaSuccess;
+}
+
+}  // namespace gq
 
 namespace {
 

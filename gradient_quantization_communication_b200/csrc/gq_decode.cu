@@ -466,13 +466,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base_staged(const 
 template <class K>
 cudaError_t launch_items(K kern, const KParams &p, int cpi, size_t smem, cudaStream_t stream)
 {
-    if (smem > 0 && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return cudaGetLastError();
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecodeWarps * 32, smem);
-    if (per_sm < 1) per_sm = 1;
+    int sms = 0, per_sm = 0;
+    const cudaError_t e = kernel_occupancy(reinterpret_cast<const void *>(kern), kDecodeWarps * 32, smem, &per_sm, &sms);
+    if (e != cudaSuccess) return e;
     const int64_t nitems = (p.n + 128 * cpi - 1) / (128 * cpi);
     const int64_t need = (nitems + kDecodeWarps - 1) / kDecodeWarps;
     const int64_t cap = (int64_t)sms * per_sm;

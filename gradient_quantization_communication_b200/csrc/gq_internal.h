@@ -74,6 +74,12 @@ cudaError_t launch_cta_err(const KParams &p, double *part, cudaStream_t stream);
 int64_t err_scratch_doubles(int64_t nb);
 cudaError_t launch_err_reduce(const double *part, int64_t nb, double *tmp, double *out, cudaStream_t stream,
                               const unsigned int *status = nullptr);
+// Resident CTAs per SM of kernel `kern` at `threads` threads and `smem` bytes of dynamic shared
+// memory on the current device (at least 1), and the device's SM count; the kernel's dynamic
+// shared memory limit is raised to `smem` first.  Cached per kernel, block shape and device: the
+// queries cost microseconds each, more than the launch of a small step.
+cudaError_t kernel_occupancy(const void *kern, int threads, size_t smem, int *per_sm, int *sms);
+
 // One warp waiting, with the kernels' bounded wait, on a barrier that nothing completes; raises
 // kStatusTimeout in *status after limit_ns.
 cudaError_t launch_wait_selftest(unsigned int *status, unsigned long long limit_ns, cudaStream_t stream);

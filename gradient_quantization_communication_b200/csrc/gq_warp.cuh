@@ -1106,13 +1106,9 @@ cudaError_t launch_one(const KParams &p, cudaStream_t stream)
         auto kern = bases ? (all_io ? k_warp<EPL, SCHEME, FUSED, BITS, 3 | (SB << 2)> : k_warp<EPL, SCHEME, FUSED, BITS, (SB << 2)>)
                           : (all_io ? k_warp<EPL, SCHEME, FUSED, BITS, 3> : k_warp<EPL, SCHEME, FUSED, BITS, 0>);
         const size_t smem = sizeof(WarpSmem<EPL, SCHEME>) * kWarpsPerCta;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        int sms = 0, per_sm = 0;
+        cudaError_t e = kernel_occupancy(reinterpret_cast<const void *>(kern), kWarpsPerCta * 32, smem, &per_sm, &sms);
         if (e != cudaSuccess) return e;
-        int dev = 0, sms = 0, per_sm = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarpsPerCta * 32, smem);
-        if (per_sm < 1) per_sm = 1;
         const int64_t need = (nfull + kWarpsPerCta - 1) / kWarpsPerCta;
         const int64_t cap = (int64_t)sms * per_sm;
         const int grid = (int)(need < cap ? need : cap);
@@ -1125,7 +1121,8 @@ cudaError_t launch_one(const KParams &p, cudaStream_t stream)
         auto tail = bases ? k_warp_tail<EPL, SCHEME, FUSED, (SB << 2)> : k_warp_tail<EPL, SCHEME, FUSED, 0>;
         const int nwarps = p.W < 16 ? p.W : 16;
         const size_t smem = sizeof(Fit) * nwarps + (FUSED ? (size_t)p.W * D * 4 : 0);
-        cudaError_t e = cudaFuncSetAttribute(tail, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        int sms = 0, per_sm = 0;
+        cudaError_t e = kernel_occupancy(reinterpret_cast<const void *>(tail), 32 * nwarps, smem, &per_sm, &sms);
         if (e != cudaSuccess) return e;
         tail<<<1, 32 * nwarps, smem, stream>>>(p);
         return cudaGetLastError();
