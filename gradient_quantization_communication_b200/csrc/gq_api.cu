@@ -33,30 +33,42 @@ namespace gq {
 
 cudaError_t kernel_occupancy(const void *kern, int threads, size_t smem, int *per_sm, int *sms)
 {
-    struct Entry {
+    // The dynamic shared memory limit is the kernel's own state on the device, shared by every
+    // launch of it: it is raised to the largest size asked for so far and never lowered, so that
+    // a cached answer for a larger size stays launchable after a smaller one.
+    struct Occ {
         const void *kern;
         int threads, device;
         size_t smem;
         int per_sm, sms;
     };
+    struct Limit {
+        const void *kern;
+        int device;
+        size_t smem;
+    };
     static std::mutex mu;
-    static std::vector<Entry> cache;
+    static std::vector<Occ> occ;
+    static std::vector<Limit> limits;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        for (const Entry &x : cache)
-            if (x.kern == kern && x.threads == threads && x.smem == smem && x.device == dev) {
-                *per_sm = x.per_sm;
-                *sms = x.sms;
-                return cudaSuccess;
-            }
-    }
-    if (smem > 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    Limit *lim = nullptr;
+    for (Limit &x : limits)
+        if (x.kern == kern && x.device == dev) lim = &x;
+    if (smem > 0 && (!lim || lim->smem < smem)) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
+        if (lim) lim->smem = smem;
+        else limits.push_back(Limit{kern, dev, smem});
     }
+    for (const Occ &x : occ)
+        if (x.kern == kern && x.threads == threads && x.smem == smem && x.device == dev) {
+            *per_sm = x.per_sm;
+            *sms = x.sms;
+            return cudaSuccess;
+        }
     int n_sm = 0, per = 0;
     e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
@@ -65,8 +77,7 @@ cudaError_t kernel_occupancy(const void *kern, int threads, size_t smem, int *pe
     if (per < 1) per = 1;
     *per_sm = per;
     *sms = n_sm;
-    std::lock_guard<std::mutex> lock(mu);
-    cache.push_back(Entry{kern, threads, dev, smem, per, n_sm});
+    occ.push_back(Occ{kern, threads, dev, smem, per, n_sm});
     return cudaSuccess;
 }
 

@@ -518,44 +518,91 @@ __global__ void __launch_bounds__(NW * 32) k_cta(const __grid_constant__ KParams
                         Amax = le ? 63 - __clzll(le) : 0;
                         Bmin = ge ? __ffsll(ge) - 1 : 63;
                     }
-                    for (int i = tid; i < nvalid; i += kCtaThreads) {
-                        const int ps = grid_pos<kPbFBits>(clipped(vs[i]), mn, scale);
-                        const int cell = min(ps >> kPbFBits, kTopCell);
-                        const unsigned long long x = (unsigned long long)ps;
-                        atomicAdd(&sh.ccnt[cell], 1u);
-                        atomicAdd(&sh.cs1[cell], x);
-                        atomicAdd(&sh.cs2[cell], x * x);
+                    // Q0, Q1, Q2 over the cells < k from the sorted values (the level search left them
+                    // sorted in vs, valid ones first): the position is monotone in the value, so the
+                    // cells are too, and Q(k) is the prefix before the first value whose cell is
+                    // >= k.  Thread t walks positions [t*seg, (t+1)*seg); each nonempty cell records
+                    // the prefix at its first value (count + 1 in ccnt, sums in cs1, cs2).
+                    {
+                        const int seg = d / kCtaThreads;
+                        unsigned long long r1 = 0ull, r2 = 0ull;
+                        for (int i = tid * seg; i < tid * seg + seg && i < nvalid; ++i) {
+                            const unsigned long long ps = (unsigned long long)grid_pos<kPbFBits>(vs[i], mn, scale);
+                            r1 += ps;
+                            r2 += ps * ps;
+                        }
+                        unsigned long long i1 = warp_inclusive_scan(r1, lane), i2 = warp_inclusive_scan(r2, lane);
+                        if (lane == 31) {
+                            sh.redl[0][wid] = (long long)i1;
+                            sh.redl[1][wid] = (long long)i2;
+                        }
+                        __syncthreads();
+                        unsigned long long w1 = 0ull, w2 = 0ull, t1 = 0ull, t2 = 0ull;
+                        for (int k = 0; k < NW; ++k) {
+                            const unsigned long long a1 = (unsigned long long)sh.redl[0][k], a2 = (unsigned long long)sh.redl[1][k];
+                            if (k < wid) {
+                                w1 += a1;
+                                w2 += a2;
+                            }
+                            t1 += a1;
+                            t2 += a2;
+                        }
+                        unsigned long long x1 = w1 + i1 - r1, x2 = w2 + i2 - r2;
+                        const int i0 = tid * seg;
+                        int prev = (i0 > 0 && i0 - 1 < nvalid)
+                                       ? min(grid_pos<kPbFBits>(vs[i0 - 1], mn, scale) >> kPbFBits, kTopCell)
+                                       : -1;
+                        for (int i = i0; i < i0 + seg && i < nvalid; ++i) {
+                            const int ps = grid_pos<kPbFBits>(vs[i], mn, scale);
+                            const int c = min(ps >> kPbFBits, kTopCell);
+                            if (c != prev) {
+                                sh.ccnt[c] = (unsigned int)(i + 1);
+                                sh.cs1[c] = x1;
+                                sh.cs2[c] = x2;
+                            }
+                            prev = c;
+                            x1 += (unsigned long long)ps;
+                            x2 += (unsigned long long)ps * (unsigned long long)ps;
+                        }
+                        if (tid == 0) {
+                            sh.bcast_l[0] = (long long)t1;
+                            sh.bcast_l[1] = (long long)t2;
+                        }
                     }
                     __syncthreads();
                     if (wid == 0) {
-                        const long long c0 = sh.ccnt[lane], c1 = sh.ccnt[lane + 32];
-                        const long long x0 = (long long)sh.cs1[lane], x1 = (long long)sh.cs1[lane + 32];
-                        const long long y0 = (long long)sh.cs2[lane], y1 = (long long)sh.cs2[lane + 32];
+                        const unsigned long long tc_all = (unsigned long long)nvalid;
+                        const unsigned long long tx_all = (unsigned long long)sh.bcast_l[0];
+                        const unsigned long long ty_all = (unsigned long long)sh.bcast_l[1];
+                        const unsigned long long nonempty =
+                            (unsigned long long)__ballot_sync(kFull, sh.ccnt[lane] != 0u) |
+                            ((unsigned long long)__ballot_sync(kFull, sh.ccnt[lane + 32] != 0u) << 32);
+                        unsigned long long Q0[2], Q1[2], Q2[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const unsigned long long later = nonempty & (~0ull << (lane + 32 * h));
+                            if (later) {
+                                const int c = __ffsll(later) - 1;
+                                Q0[h] = (unsigned long long)(sh.ccnt[c] - 1u);
+                                Q1[h] = sh.cs1[c];
+                                Q2[h] = sh.cs2[c];
+                            } else {
+                                Q0[h] = tc_all;
+                                Q1[h] = tx_all;
+                                Q2[h] = ty_all;
+                            }
+                        }
+                        __syncwarp();
                         sh.ccnt[lane] = 0u;
                         sh.ccnt[lane + 32] = 0u;
-                        sh.cs1[lane] = 0ull;
-                        sh.cs1[lane + 32] = 0ull;
-                        sh.cs2[lane] = 0ull;
-                        sh.cs2[lane + 32] = 0ull;
-                        const long long ic0 = warp_inclusive_scan(c0, lane), ic1 = warp_inclusive_scan(c1, lane);
-                        const long long ix0 = warp_inclusive_scan(x0, lane), ix1 = warp_inclusive_scan(x1, lane);
-                        const long long iy0 = warp_inclusive_scan(y0, lane), iy1 = warp_inclusive_scan(y1, lane);
-                        const long long tc = __shfl_sync(kFull, ic0, 31), tx = __shfl_sync(kFull, ix0, 31),
-                                        ty = __shfl_sync(kFull, iy0, 31);
-                        const long long tc_all = __shfl_sync(kFull, tc + ic1, 31);
-                        const long long tx_all = __shfl_sync(kFull, tx + ix1, 31);
-                        const long long ty_all = __shfl_sync(kFull, ty + iy1, 31);
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             const int K = lane + 32 * h;
-                            const unsigned long long uQ0 = h ? tc + ic1 - c1 : ic0 - c0;
-                            const unsigned long long uQ1 = h ? tx + ix1 - x1 : ix0 - x0;
-                            const unsigned long long uQ2 = h ? ty + iy1 - y1 : iy0 - y0;
+                            const unsigned long long uQ0 = Q0[h], uQ1 = Q1[h], uQ2 = Q2[h];
                             const unsigned long long k = (unsigned long long)K << kPbFBits;
                             sh.al[K] = (long long)(k * k * uQ0 - 3ull * k * uQ1 + 2ull * uQ2);
-                            sh.be[K] = (long long)(3ull * k * uQ1 - 2ull * uQ2 + (unsigned long long)ty_all -
-                                                   2ull * k * (unsigned long long)tx_all +
-                                                   k * k * ((unsigned long long)tc_all - uQ0));
+                            sh.be[K] = (long long)(3ull * k * uQ1 - 2ull * uQ2 + ty_all - 2ull * k * tx_all +
+                                                   k * k * (tc_all - uQ0));
                             sh.ga[K] = (long long)(uQ1 - k * uQ0);
                             sh.de[K] = (long long)(k * uQ0 - uQ1);
                         }
