@@ -157,24 +157,65 @@ __device__ RoundB cta_bingrad_b_levels(float *vs, int d, int nvalid, float m, co
     constexpr int kCtaThreads = NW * 32;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     RoundB rb{0.0f, 0.0f, 0.0f, false};
-    // sort u in place (padding = +inf)
+    // sort u in place (padding = +inf), by the register path's network (every comparator puts
+    // the minimum at the lower index): the warps sort runs of 512 keys in registers; each merge of
+    // blocks of k >= 1024 keys then takes its mirror stage (i against i ^ (k-1)) and its
+    // half-cleaners down to distance 512 in shared memory, and the stages below 512, which stay
+    // inside a run, in registers again
+    constexpr int kRun = 512;
     for (int i = tid; i < d; i += kCtaThreads) vs[i] = i < nvalid ? clipped(vs[i]) : INFINITY;
     __syncthreads();
-    for (int k = 2; k <= d; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
+    const int nruns = d / kRun;
+    auto run_io = [&](int run, float (&key)[16], bool load) {
+        float4 *q = reinterpret_cast<float4 *>(vs + run * kRun + 16 * lane);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            if (load) {
+                const float4 x = q[v];
+                key[4 * v] = x.x;
+                key[4 * v + 1] = x.y;
+                key[4 * v + 2] = x.z;
+                key[4 * v + 3] = x.w;
+            } else {
+                q[v] = make_float4(key[4 * v], key[4 * v + 1], key[4 * v + 2], key[4 * v + 3]);
+            }
+        }
+    };
+    for (int run = wid; run < nruns; run += NW) {
+        float key[16];
+        run_io(run, key, true);
+        warp_bitonic_sort<16>(key, lane);
+        run_io(run, key, false);
+    }
+    __syncthreads();
+    for (int k = 2 * kRun; k <= d; k <<= 1) {
+        for (int i = tid; i < d; i += kCtaThreads) {  // mirror stage
+            const int ixj = i ^ (k - 1);
+            if (ixj > i) {
+                const float a = vs[i], b = vs[ixj];
+                vs[i] = fminf(a, b);
+                vs[ixj] = fmaxf(a, b);
+            }
+        }
+        __syncthreads();
+        for (int j = k >> 2; j >= kRun; j >>= 1) {
             for (int i = tid; i < d; i += kCtaThreads) {
                 const int ixj = i ^ j;
                 if (ixj > i) {
                     const float a = vs[i], b = vs[ixj];
-                    const bool up = (i & k) == 0;
-                    if ((a > b) == up) {
-                        vs[i] = b;
-                        vs[ixj] = a;
-                    }
+                    vs[i] = fminf(a, b);
+                    vs[ixj] = fmaxf(a, b);
                 }
             }
             __syncthreads();
         }
+        for (int run = wid; run < nruns; run += NW) {
+            float key[16];
+            run_io(run, key, true);
+            warp_halfclean<16, kRun / 2>(key, lane);
+            run_io(run, key, false);
+        }
+        __syncthreads();
     }
     // exact prefix sums of the fixed-point values: thread t owns positions [t*seg, (t+1)*seg)
     const int e2 = 46 - fexpo(m);
@@ -192,23 +233,48 @@ __device__ RoundB cta_bingrad_b_levels(float *vs, int d, int nvalid, float m, co
         total += t;
     }
     __syncthreads();
-    long long S = wpre + incl - run;  // sum of positions before tid*seg
+    const long long S0 = wpre + incl - run;  // sum of positions before tid*seg
+    // Screening, as in the register path: a binary32 estimate of J for every admissible split
+    // (within 8 * 2^-24 of J), then the fp64 J only for the splits whose estimate reaches
+    // M (1 - 2^-18), M the block's largest estimate; every split whose fp64 J is the largest is
+    // among them, so the choice (ties to the smallest split) is the exhaustive one.
+    float emax = 0.0f;
+    {
+        long long S = S0;
+        for (int i = tid * seg; i < tid * seg + seg; ++i) {
+            if (i >= 1 && i < nvalid && vs[i - 1] < vs[i]) {
+                const float l = __ll2float_rn(S), rr = __ll2float_rn(total - S);
+                emax = fmaxf(emax, __fadd_rn(__fmul_rn(__fmul_rn(l, l), rcp_approx((float)i)),
+                                             __fmul_rn(__fmul_rn(rr, rr), rcp_approx((float)(nvalid - i)))));
+            }
+            if (i < nvalid) S += fixed_point(vs[i], sc);
+        }
+    }
+    const float thr = __fmul_rn(block_max(emax, sh, 2), 1.0f - 0x1p-18f);
     double best_j = -1.0;
     int best_i = 0x7fffffff;
     long long best_s = 0;
-    for (int i = tid * seg; i < tid * seg + seg; ++i) {
-        if (i >= 1 && i < nvalid && vs[i - 1] < vs[i]) {
-            const double l = __ll2double_rn(S);
-            const double rr = __ll2double_rn(total - S);
-            const double J = __dadd_rn(__ddiv_rn(__dmul_rn(l, l), (double)i),
-                                       __ddiv_rn(__dmul_rn(rr, rr), (double)(nvalid - i)));
-            if (J > best_j) {
-                best_j = J;
-                best_i = i;
-                best_s = S;
+    {
+        long long S = S0;
+        for (int i = tid * seg; i < tid * seg + seg; ++i) {
+            if (i >= 1 && i < nvalid && vs[i - 1] < vs[i]) {
+                const float l = __ll2float_rn(S), rr = __ll2float_rn(total - S);
+                const float est = __fadd_rn(__fmul_rn(__fmul_rn(l, l), rcp_approx((float)i)),
+                                            __fmul_rn(__fmul_rn(rr, rr), rcp_approx((float)(nvalid - i))));
+                if (est >= thr) {
+                    const double ld = __ll2double_rn(S);
+                    const double rd = __ll2double_rn(total - S);
+                    const double J = __dadd_rn(__ddiv_rn(__dmul_rn(ld, ld), (double)i),
+                                               __ddiv_rn(__dmul_rn(rd, rd), (double)(nvalid - i)));
+                    if (J > best_j) {
+                        best_j = J;
+                        best_i = i;
+                        best_s = S;
+                    }
+                }
             }
+            if (i < nvalid) S += fixed_point(vs[i], sc);
         }
-        if (i < nvalid) S += fixed_point(vs[i], sc);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {

@@ -305,6 +305,90 @@ __device__ __forceinline__ float grid_point(float mn, float mx, float step, int 
     return j == 63 ? mx : __fadd_rn(mn, __fmul_rn((float)j, step));
 }
 
+// Bitonic sort of the 32*EPL keys, position i = lane*EPL + r, ascending, in the form whose
+// comparators all put the minimum at the lower index: each merge of blocks of k keys starts by
+// comparing i with its mirror i ^ (k-1), then i with i ^ j for j = k/4 .. 1.  Inside a lane a
+// compare-exchange is one min and one max; across lanes (partner lane l ^ m) the lower lane keeps
+// the minimum, a choice that depends on the lane only.
+template <int EPL>
+__device__ __forceinline__ void warp_bitonic_sort(float (&key)[EPL], int lane)
+{
+    constexpr int N = 32 * EPL;
+#pragma unroll
+    for (int k = 2; k <= N; k <<= 1) {
+        if (k <= EPL) {
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) {
+                const int q = r ^ (k - 1);
+                if (q > r) {
+                    const float a = key[r], b = key[q];
+                    key[r] = fminf(a, b);
+                    key[q] = fmaxf(a, b);
+                }
+            }
+        } else {
+            // partner of (lane, r) is (lane ^ m, EPL-1-r); pairs (r, EPL-1-r) are updated together
+            const int m = k / EPL - 1;
+            const bool take_min = (lane & ((k / EPL) >> 1)) == 0;
+#pragma unroll
+            for (int r = 0; r < EPL / 2; ++r) {
+                const float o1 = __shfl_xor_sync(kFull, key[EPL - 1 - r], m);
+                const float o2 = __shfl_xor_sync(kFull, key[r], m);
+                key[r] = take_min ? fminf(key[r], o1) : fmaxf(key[r], o1);
+                key[EPL - 1 - r] = take_min ? fminf(key[EPL - 1 - r], o2) : fmaxf(key[EPL - 1 - r], o2);
+            }
+        }
+#pragma unroll
+        for (int j = k >> 2; j > 0; j >>= 1) {
+            if (j >= EPL) {
+                const bool take_min = (lane & (j / EPL)) == 0;
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) {
+                    const float o = __shfl_xor_sync(kFull, key[r], j / EPL);
+                    key[r] = take_min ? fminf(key[r], o) : fmaxf(key[r], o);
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) {
+                    if ((r & j) == 0) {
+                        const float a = key[r], b = key[r ^ j];
+                        key[r] = fminf(a, b);
+                        key[r ^ j] = fmaxf(a, b);
+                    }
+                }
+            }
+        }
+    }
+}
+
+// The half-cleaner stages j = JTOP, JTOP/2, .., 1 of the same network on the 32*EPL keys
+// (position lane*EPL + r): i against i ^ j, the minimum at the lower index.  Applied to a block
+// whose two halves hold the outcome of a merge's first stages, it finishes the merge.
+template <int EPL, int JTOP>
+__device__ __forceinline__ void warp_halfclean(float (&key)[EPL], int lane)
+{
+#pragma unroll
+    for (int j = JTOP; j > 0; j >>= 1) {
+        if (j >= EPL) {
+            const bool take_min = (lane & (j / EPL)) == 0;
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) {
+                const float o = __shfl_xor_sync(kFull, key[r], j / EPL);
+                key[r] = take_min ? fminf(key[r], o) : fmaxf(key[r], o);
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) {
+                if ((r & j) == 0) {
+                    const float a = key[r], b = key[r ^ j];
+                    key[r] = fminf(a, b);
+                    key[r ^ j] = fmaxf(a, b);
+                }
+            }
+        }
+    }
+}
+
 // BinGrad-pb, one column of the pair search: the smallest minimiser over A in [0, Ahi] (Ahi >= 0)
 // of E(A) = E(A, B) for a fixed B, and its value in es.  E(a, b) is convex in a for a fixed b: a
 // value x contributes (x - a)(b - x), of slope -(b - x) <= 0, while a <= x, and (a - x)^2, of
