@@ -300,3 +300,15 @@ def test_bingrad_pb_interior_optima(d):
     n = g[0][0].size
     cg, co = configs("bingrad_pb", 2, d, W, True, 0.0, 21, n)
     compare_steps(run_gpu_fused(cg, 1, g), run_oracle_fused(co, 1, g), co, "bingrad_pb interior d=%d" % d)
+
+
+@pytest.mark.parametrize("W", [1, 4, 5, 8])
+@pytest.mark.parametrize("scheme,levels,d", [("orq", 5, 512), ("qsgd", 3, 128), ("qsgd", 255, 256), ("orq", 9, 2048)])
+def test_decode_worker_counts(W, scheme, levels, d):
+    """gq_decode_accumulate for 1, 4 and 8 messages (the staged decode, the count a template
+    argument) and for 5 (the generic one), 3-, 2-, 8- and 4-bit codes, against the oracle."""
+    n = 6 * d + 71
+    cg, co = configs(scheme, levels, d, W, True, 0.0, 91 + W, n)
+    g = _grads(n, W, 1, seed=7 * W + d)
+    compare_steps(run_gpu_fused(cg, 1, g, unfused=True), run_oracle_fused(co, 1, g), co,
+                  "decode W=%d %s-%d d=%d" % (W, scheme, levels, d))
