@@ -99,12 +99,14 @@ def test_segments_required_and_checked():
             O.Config(G.GQ_TERNGRAD_LAYER, 3, 128, 1, 0, 0.0, 1, n), 2)[0]
 
 
-def test_long_vector_many_tensors():
+@pytest.mark.parametrize("W,ef", [(2, True), (8, True), (1, False), (5, True)])
+def test_long_vector_many_tensors(W, ef):
     """More chunks than the grid has warps, so that every warp walks a run of chunks and slices
     across many tensor boundaries (random sizes from 0 to 40000, so boundaries fall inside a
-    lane's four elements, across chunk edges, and empty tensors follow each other)."""
+    lane's four elements, across chunk edges, and empty tensors follow each other); 1, 2 and 8
+    workers take the staged encode, 5 the generic one; a ragged last chunk."""
     rng = np.random.default_rng(21)
-    n = 3_000_000 + 13
+    n = 3_000_000 + 13 if W <= 2 else 1_000_000 + 77
     sizes = rng.integers(0, 40000, 400)
     sizes[rng.integers(0, 400, 40)] = 0
-    _run(n, 512, 2, 1, _offsets(n, sizes.tolist()), True, seed=22)
+    _run(n, 512, W, 1, _offsets(n, sizes.tolist()), ef, seed=22 + W)
