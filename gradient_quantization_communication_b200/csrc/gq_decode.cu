@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
 }
 
 // The same decode and sum for a worker count known at compile time (1, 2, 4 or 8), with each item's
-// code words staged in the warp's shared memory: one 1-D bulk copy (no multicast) per worker and
+// code words staged in the warp's shared memory: one 1-D bulk copy (into this CTA only) per worker and
 // item, one item ahead on a two-stage mbarrier pipeline, so that the lanes read their code words
 // from shared memory instead of waiting on global loads.  The level tables (a few floats per
 // worker and bucket, not 16-byte aligned) are loaded into registers one item ahead.  An item's

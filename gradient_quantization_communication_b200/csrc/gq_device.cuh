@@ -422,7 +422,7 @@ __device__ __forceinline__ int grid_pos(float u, float mn, float scale)
 }
 
 // ---------------------------------------------------------------------------------------------
-// Bulk asynchronous copies (TMA, no multicast) into shared memory, completed on an mbarrier.
+// Bulk asynchronous copies (TMA, 1-D, into this CTA only) into shared memory, completed on an mbarrier.
 // Every wait is bounded: after kWaitLimitNs of global time it gives up and reports failure.
 // ---------------------------------------------------------------------------------------------
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // one second

@@ -8,7 +8,7 @@
 // groups, each synchronised by its own named barrier (d = 1024: two per CTA of 4; 2048, 4096 and
 // 8192: one).  For G > NW a bucket takes a cluster of C = G / NW CTAs (d = 16384: 2, 32768: 4),
 // synchronised by cluster barriers, and the statistics cross CTAs through distributed shared
-// memory (plain loads of the peer CTA's shared memory; no multicast).
+// memory (plain loads of the peer CTA's shared memory).
 // Only what the fit needs crosses warps:
 //   QSGD / TernGrad : each warp's max |u| -> the group's max (one exchange);
 //   ORQ             : each warp's min and max -> the group's; then each warp's 64 cell counts

@@ -5,7 +5,7 @@
 //
 // One warp owns one bucket index at a time and walks its items (bucket, worker) in order.  The
 // g and r of each item (2 x d floats) are staged into the warp's shared memory by bulk
-// asynchronous copies (TMA, 1-D, no multicast) completed on an mbarrier: as soon as an item's
+// asynchronous copies (TMA, 1-D, into this CTA only) completed on an mbarrier: as soon as an item's
 // values are in registers the copy of the next item is issued into the same buffer, so the
 // copy engine keeps 4 KB per warp in flight during the whole fit and no registers are spent on
 // prefetching.  Lane l then holds EPL = d/32 values in registers, slot
