@@ -14,11 +14,13 @@
 //   ORQ             : per warp, the packed 8-column histogram of the register path (one shared
 //                     atomic per value), reduced every 512 values into the warp's cell totals;
 //                     warp 0 sums the warps' totals and runs the greedy
-//   BinGrad-b       : block bitonic sort of u in place, exact int64 block scan, argmax of
-//                     J(k); the final pass re-reads g and r because the sort overwrote v
+//   BinGrad-b       : sort of u in place (runs of 512 sorted by the warps in registers, then
+//                     merged: the stages of distance >= 512 in shared memory, the rest in
+//                     registers), exact int64 block scan, argmax of J(k) screened in binary32;
+//                     the final pass re-reads g and r because the sort overwrote v
 //   BinGrad-pb      : BinGrad-b's levels first (as above: the final pass re-reads g and r),
-//                     which bound the pair from inside; block moments per cell (shared
-//                     atomics), the admissible pairs among all 2016 searched by the threads
+//                     which bound the pair from inside; the cells' prefix moments read off the
+//                     sorted values; per column B the least E over the admissible A (convex in A)
 // The per-element rules and the chunk step are those of the register path (gq_round.cuh), so
 // both paths produce identical codes.
 #include "gq_round.cuh"
