@@ -20,8 +20,9 @@
 //                     columns per cell, one packed shared atomic per value), exact prefix
 //                     sums, s-2 incremental greedy rounds, per-bracket reciprocal table
 //   BinGrad-b       : warp bitonic sort, exact int64 prefix sums, screened argmax of J(k)
-//   BinGrad-pb      : BinGrad-b's levels (as above) bound the pair from inside; shared-memory
-//                     moments of 16-bit positions, exact search of the admissible pairs
+//   BinGrad-pb      : BinGrad-b's levels (as above) bound the pair from inside; the cells'
+//                     prefix moments of 16-bit positions read off the sorted values; per
+//                     column the least E over the admissible A (E is convex in A)
 //   QSGD-nearest    : the QSGD levels, rounding to the nearest level (no draws)
 //   QSGD-l2         : the QSGD levels scaled by ||u||_2 (exact fixed-point sum of squares)
 //   SignSGD         : m1 = mean |u| from an exact fixed-point warp sum, levels -m1 and +m1
