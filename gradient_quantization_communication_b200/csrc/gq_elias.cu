@@ -345,16 +345,10 @@ __device__ __forceinline__ uint32_t stream_word(const ElParams &p, int64_t q)
     return q < p.cap_words ? __ldg(p.stream + q) : 0u;
 }
 
-// One thread per bucket, a warp per 32 consecutive buckets.  The thread reads its stream through
-// a 64-bit bit buffer refilled a word at a time, with the next word's load issued one refill
-// ahead.  While at least 8 codes remain, one lookup of the next 8 stream bits decodes every
-// codeword that lies wholly inside them (dec8); the rest go one codeword per lookup of the next
-// 7 bits (dec).  The thread builds its bucket's dense words in its row of the warp's shared
-// buffer (rows of dw + 1 words, so that the lanes' stores hit distinct banks); the warp then
-// writes the 32 buckets' words, which are contiguous in the dense message, row by row with
-// coalesced stores.
-constexpr int kDecodeWarps = 4;
-constexpr int kStreamStage = 1024;  // stream words a warp stages for its 32 buckets (4 KB)
+// Decode CTAs: eight warps, each staging up to 2.5 KB of stream; with the 32 rows of dense
+// words this keeps 32 warps resident per SM at d = 512, 2-bit codes.
+constexpr int kDecodeWarps = 8;
+constexpr int kStreamStage = 640;  // stream words a warp stages for its 32 buckets
 
 // The codes of one bucket from its first stream bit: rd(q) reads stream word q.
 template <int B, class Rd>
