@@ -32,7 +32,7 @@
 //      starts or ends inside a word) go by atomicOr onto words zeroed by steps 3 and 4; the level
 //      table is copied.
 // Unpack: k_decode, one thread per bucket, reads its codewords from its first bit (one lookup of
-// the next 8 bits decodes every codeword inside them) into the warp's shared rows, and the warp
+// the next 10 bits decodes every codeword inside them) into the warp's shared rows, and the warp
 // writes 32 buckets' dense words at a time; the level tables are copied.  Count and encode take
 // the codewords and lengths of 2 or 4 codes at once from 256-entry tables.
 //
@@ -71,9 +71,6 @@ struct ElParams {
     // G = 8 / b codes (2 for b = 3) as one table index of G * b bits -> their codewords in stream
     // order (bits 0 .. 23) | total length << 24
     uint32_t enc[256];
-    // the next 8 stream bits -> the codewords that lie wholly inside them, decoded: their codes
-    // packed b bits each (bits 0 .. 31) | count << 32 | bits consumed << 40
-    unsigned long long dec8[256];
 };
 
 // codes per table index of the group tables
@@ -345,15 +342,43 @@ __device__ __forceinline__ uint32_t stream_word(const ElParams &p, int64_t q)
     return q < p.cap_words ? __ldg(p.stream + q) : 0u;
 }
 
-// Decode CTAs: eight warps, each staging up to 2.5 KB of stream; with the 32 rows of dense
-// words this keeps 32 warps resident per SM at d = 512, 2-bit codes.
+// Decode CTAs: eight warps, each staging up to 2.4 KB of stream; with the window table and the
+// 32 rows of dense words this keeps 32 warps resident per SM at d = 512, 2-bit codes.
 constexpr int kDecodeWarps = 8;
-constexpr int kStreamStage = 640;  // stream words a warp stages for its 32 buckets
+constexpr int kStreamStage = 600;  // stream words a warp stages for its 32 buckets
+// Multi-codeword lookups read the next kDecWin stream bits: the codewords that lie wholly inside
+// them, decoded, as one 32-bit entry (codes b bits each at bits 0 .. 23, count << 24, bits
+// consumed << 28).  At most 24 / b codes go in one entry.
+constexpr int kDecWin = 10;
+static_assert(3 * kDecWin <= 32, "three lookups per refill");
+
+// The window table from the single-codeword table dec (the next 7 bits -> code | length << 4):
+// decode as dec does while the next codeword lies wholly inside the window; the first one always
+// does (a codeword has at most 7 bits, and a pattern that starts none takes 7).  dec saw zeros
+// past the window, so its answer stands only for a codeword whose bits all lie inside.
+template <int B>
+__device__ __forceinline__ void build_window_table(const unsigned char *dec, uint32_t *decw)
+{
+    constexpr int cap = 24 / B;
+    for (int t = threadIdx.x; t < (1 << kDecWin); t += blockDim.x) {
+        int pos = 0, cnt = 0;
+        uint32_t codes = 0;
+        while (pos < kDecWin && cnt < cap) {
+            const unsigned e = dec[(t >> pos) & 127];
+            const int len = (int)(e >> 4);
+            if (pos + len > kDecWin) break;
+            codes |= (e & 15u) << (B * cnt);
+            ++cnt;
+            pos += len;
+        }
+        decw[t] = codes | ((uint32_t)cnt << 24) | ((uint32_t)pos << 28);
+    }
+}
 
 // The codes of one bucket from its first stream bit: rd(q) reads stream word q.
 template <int B, class Rd>
-__device__ __forceinline__ void decode_bucket(const unsigned char *dec, const unsigned long long *dec8, uint64_t start,
-                                              int n, int dw, uint32_t *out, const Rd &rd)
+__device__ __forceinline__ void decode_bucket(const unsigned char *dec, const uint32_t *decw, uint64_t start, int n,
+                                              int dw, uint32_t *out, const Rd &rd)
 {
     int64_t q = (int64_t)(start >> 5);
     const int sh = (int)(start & 31u);
@@ -364,17 +389,12 @@ __device__ __forceinline__ void decode_bucket(const unsigned char *dec, const un
     uint64_t acc = 0;
     int accbits = 0, wi = 0;
     int e = 0;
-    for (; e + 8 <= n;) {
-        if (nbuf < 32) {
-            buf |= (uint64_t)next << nbuf;
-            nbuf += 32;
-            next = rd(++q);
-        }
-        const unsigned long long t = dec8[(uint32_t)buf & 255u];
-        const int cnt = (int)((t >> 32) & 15u), len = (int)((t >> 40) & 15u);
+    const auto look = [&]() {
+        const uint32_t t = decw[(uint32_t)buf & ((1u << kDecWin) - 1u)];
+        const int cnt = (int)((t >> 24) & 15u), len = (int)(t >> 28);
         buf >>= len;
         nbuf -= len;
-        acc |= (t & 0xFFFFFFFFull) << accbits;
+        acc |= (uint64_t)(t & 0xFFFFFFu) << accbits;
         accbits += B * cnt;
         e += cnt;
         if (accbits >= 32) {
@@ -382,6 +402,25 @@ __device__ __forceinline__ void decode_bucket(const unsigned char *dec, const un
             acc >>= 32;
             accbits -= 32;
         }
+    };
+    // a refill leaves at least 32 bits in the buffer: three lookups of up to kDecWin bits each
+    for (; e + 3 * kDecWin <= n;) {
+        if (nbuf < 32) {
+            buf |= (uint64_t)next << nbuf;
+            nbuf += 32;
+            next = rd(++q);
+        }
+        look();
+        look();
+        look();
+    }
+    for (; e + kDecWin <= n;) {
+        if (nbuf < 32) {
+            buf |= (uint64_t)next << nbuf;
+            nbuf += 32;
+            next = rd(++q);
+        }
+        look();
     }
     for (; e < n; ++e) {
         if (nbuf < 32) {  // refill: a codeword has at most 7 bits
@@ -408,9 +447,9 @@ __device__ __forceinline__ void decode_bucket(const unsigned char *dec, const un
 // One thread per bucket, a warp per 32 consecutive buckets.  Their stream bits are one span:
 // when it fits in kStreamStage words the warp first copies it into shared memory with coalesced
 // loads, else the threads read global memory.  A thread reads its codewords through a 64-bit
-// bit buffer; while at least 8 codes remain, one lookup of the next 8 stream bits decodes every
-// codeword that lies wholly inside them (dec8), the rest go one codeword per lookup of the next
-// 7 bits (dec).  The thread builds its bucket's dense words in its row of the warp's shared
+// bit buffer; while at least kDecWin codes remain, one lookup of the next kDecWin stream bits
+// decodes every codeword that lies wholly inside them (decw, built by each CTA), the rest go one
+// codeword per lookup of the next 7 bits (dec).  The thread builds its bucket's dense words in its row of the warp's shared
 // buffer (rows of dw + 1 words, so that the lanes' stores hit distinct banks); the warp then
 // writes the 32 buckets' words, which are contiguous in the dense message, row by row with
 // coalesced stores.
@@ -419,11 +458,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
                                                               uint32_t *dense_out, int pad_floats)
 {
     __shared__ unsigned char dec[128];
-    __shared__ unsigned long long dec8[256];
+    __shared__ uint32_t decw[1 << kDecWin];
     __shared__ uint32_t stage_all[kDecodeWarps][kStreamStage];
     extern __shared__ uint32_t rows_all[];  // [warps][32][dw + 1]
     if (threadIdx.x < 128) dec[threadIdx.x] = p.dec[threadIdx.x];
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) dec8[i] = p.dec8[i];
+    __syncthreads();
+    build_window_table<B>(dec, decw);
     __syncthreads();
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int dw = p.dw, rs = p.dw + 1;
@@ -453,10 +493,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode(const __grid_const
             const int n = bucket_valid(p, bk);
             const uint64_t start = p.offs[bk];
             if (staged) {
-                decode_bucket<B>(dec, dec8, start, n, dw, out,
+                decode_bucket<B>(dec, decw, start, n, dw, out,
                                  [&](int64_t q) { return q < w1 ? stage[q - w0] : 0u; });
             } else {
-                decode_bucket<B>(dec, dec8, start, n, dw, out, [&](int64_t q) { return stream_word(p, q); });
+                decode_bucket<B>(dec, decw, start, n, dw, out, [&](int64_t q) { return stream_word(p, q); });
             }
         }
         __syncwarp();
@@ -583,24 +623,6 @@ ElParams make_params(const gq_config_t *cfg, const ElLayout &l, const void *msg,
             }
         }
         p.enc[idx] = bitsv | ((uint32_t)len << 24);
-    }
-    // multi-codeword decoding table over 8 stream bits: decode as the single table does while the
-    // next codeword lies wholly inside the 8 bits (the first one always does: a codeword has at
-    // most 7 bits, and a pattern that starts none takes 7)
-    for (int t = 0; t < 256; ++t) {
-        int pos = 0, cnt = 0;
-        unsigned long long codes = 0;
-        while (pos < 8) {
-            const int u = (t >> pos) & 127;  // the next 7 bits (zeros past the window)
-            const int c = p.dec[u] & 15, len = p.dec[u] >> 4;
-            if (pos + len > 8) break;
-            // the single table saw zeros past bit 8: accept its answer only if the codeword's
-            // bits all lie inside the window
-            codes |= (unsigned long long)c << (l.b * cnt);
-            ++cnt;
-            pos += len;
-        }
-        p.dec8[t] = codes | ((unsigned long long)cnt << 32) | ((unsigned long long)pos << 40);
     }
     return p;
 }
