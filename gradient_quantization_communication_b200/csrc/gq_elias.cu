@@ -167,8 +167,16 @@ __global__ void __launch_bounds__(kBktWarps * 32) k_count(const __grid_constant_
         if (bk < p.nb) {
             const int n = bucket_valid(p, bk);
             const int ng = n / G;
-            int bits = 0;
-            for (int k = 0; k < ng; ++k) bits += (int)(enc[row_group<B>(row, k)] >> 24);
+            int bits = 0, k = 0;
+            if constexpr (G * B == 8) {
+                // a row word holds four whole table indices
+                for (; k + 4 <= ng; k += 4) {
+                    const uint32_t x = row[k >> 2];
+                    bits += (int)((enc[x & 0xFFu] >> 24) + (enc[(x >> 8) & 0xFFu] >> 24) +
+                                  (enc[(x >> 16) & 0xFFu] >> 24) + (enc[x >> 24] >> 24));
+                }
+            }
+            for (; k < ng; ++k) bits += (int)(enc[row_group<B>(row, k)] >> 24);
             for (int j = ng * G; j < n; ++j) bits += code_len(p, row_code<B>(row, j));
             p.offs[bk] = (uint64_t)bits;
         }
@@ -315,10 +323,27 @@ __global__ void __launch_bounds__(kBktWarps * 32) k_encode(const __grid_constant
                 acc >>= 32;
                 accbits -= 32;
             };
-            for (int k = 0; k < ng; ++k) {
-                const uint32_t e = enc[row_group<B>(row, k)];
+            const auto put = [&](uint32_t e) {
                 acc |= (uint64_t)(e & 0xFFFFFFu) << accbits;
                 accbits += (int)(e >> 24);
+            };
+            int k = 0;
+            if constexpr (G * B == 8) {
+                // a row word holds four whole table indices; two groups take at most 28 bits
+                // (4 codewords of at most 3 bits, or 2 of at most 7), so one check after each pair
+                // keeps the buffer below 64 bits
+                for (; k + 4 <= ng; k += 4) {
+                    const uint32_t x = row[k >> 2];
+                    put(enc[x & 0xFFu]);
+                    put(enc[(x >> 8) & 0xFFu]);
+                    if (accbits >= 32) flush();
+                    put(enc[(x >> 16) & 0xFFu]);
+                    put(enc[x >> 24]);
+                    if (accbits >= 32) flush();
+                }
+            }
+            for (; k < ng; ++k) {
+                put(enc[row_group<B>(row, k)]);
                 if (accbits >= 32) flush();
             }
             for (int j = ng * G; j < n; ++j) {
