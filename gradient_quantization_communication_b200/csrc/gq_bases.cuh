@@ -13,7 +13,7 @@
 // chunk each lane forms the values of every 32nd group and puts them in place (base_s_store).
 // Reader: the four codes of a lane (elements 4l .. 4l+3 of a chunk) lie in at most two groups,
 // whose 2B <= 32 bits one 64-bit window of two words holds (base_pos); their digits come from a
-// shared table (base_codes4).
+// shared table (base_run4).
 #pragma once
 
 #include "gq_entropy.cuh"
@@ -138,10 +138,10 @@ __device__ __forceinline__ BasePos base_pos(int e)
     const int j0 = e / g, bit = B * j0;
     return BasePos{bit >> 5, bit & 31, e - j0 * g};
 }
-// The four codes from the two words (lo, hi) at that place.
+// The four codes from the two words (lo, hi) at that place, 4 bits each: code q of the four at
+// bits 4q .. 4q+3 of the result.
 template <int S>
-__device__ __forceinline__ void base_codes4(const DigitTab<S> &t, uint32_t lo, uint32_t hi, const BasePos &ps,
-                                            int (&code)[4])
+__device__ __forceinline__ uint32_t base_run4(const DigitTab<S> &t, uint32_t lo, uint32_t hi, const BasePos &ps)
 {
     constexpr int g = BaseS<S>::g, B = BaseS<S>::B;
     const unsigned long long two = ((unsigned long long)hi << 32 | lo) >> ps.sh;
@@ -149,9 +149,7 @@ __device__ __forceinline__ void base_codes4(const DigitTab<S> &t, uint32_t lo, u
     // the digits of both groups, 4 bits each, the first group's first: element e + q is digit k0 + q
     const unsigned long long dg = (unsigned long long)group_digits<S>(t, (uint32_t)two & mask) |
                                   ((unsigned long long)group_digits<S>(t, (uint32_t)(two >> B) & mask) << (4 * g));
-    const uint32_t run = (uint32_t)(dg >> (4 * ps.k0));
-#pragma unroll
-    for (int q = 0; q < 4; ++q) code[q] = (int)((run >> (4 * q)) & 0xfu);
+    return (uint32_t)(dg >> (4 * ps.k0));
 }
 
 }  // namespace gq

@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_staged(const __gri
 }
 
 // Base-s messages (s = 3, 5, 9; d <= 512): the same items and sum, with each lane's four codes
-// of a chunk taken from the one or two base-s groups that hold them (base_codes4); the code words
+// of a chunk taken from the one or two base-s groups that hold them (base_run4); the code words
 // of kBaseGroup workers are loaded before any is decoded.
 constexpr int kBaseGroup = 4;
 template <bool QSGD, int S, int CPI>
@@ -310,11 +310,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base(const __grid_
                     const float level = QSGD ? __fmul_rn(lv[k], qr) : lv[k];
 #pragma unroll
                     for (int c = 0; c < CPI; ++c) {
-                        int code[4];
-                        base_codes4<S>(tab, lo[k][c], hi[k][c], ps[c], code);
+                        const uint32_t run = base_run4<S>(tab, lo[k][c], hi[k][c], ps[c]);
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, code[e], kWidth));
+                            acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, (int)(run >> (4 * e)), kWidth));
                     }
                 }
             }
@@ -436,11 +435,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) k_decode_base_staged(const 
             for (int c = 0; c < CPI; ++c) {
                 const uint32_t lo = bw[ps[c].wi];
                 const uint32_t hi = ps[c].wi + 1 < nw ? bw[ps[c].wi + 1] : 0u;
-                int code[4];
-                base_codes4<S>(tab, lo, hi, ps[c], code);
+                const uint32_t run = base_run4<S>(tab, lo, hi, ps[c]);
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, code[e], kWidth));
+                    acc[c][e] = __fadd_rn(acc[c][e], __shfl_sync(kFull, level, (int)(run >> (4 * e)), kWidth));
             }
         }
 #pragma unroll
