@@ -139,17 +139,18 @@ __device__ __forceinline__ BasePos base_pos(int e)
     return BasePos{bit >> 5, bit & 31, e - j0 * g};
 }
 // The four codes from the two words (lo, hi) at that place, 4 bits each: code q of the four at
-// bits 4q .. 4q+3 of the result.
+// bits 4q .. 4q+3 of the result (the bits above are the next codes, or 0).  Both groups lie in
+// the low 2B <= 32 bits of the pair shifted down by sh.
 template <int S>
 __device__ __forceinline__ uint32_t base_run4(const DigitTab<S> &t, uint32_t lo, uint32_t hi, const BasePos &ps)
 {
     constexpr int g = BaseS<S>::g, B = BaseS<S>::B;
-    const unsigned long long two = ((unsigned long long)hi << 32 | lo) >> ps.sh;
+    static_assert(2 * B <= 32 && 4 * g < 32, "two groups in one word, a group's digits below bit 32");
+    const uint32_t two = __funnelshift_r(lo, hi, ps.sh);
     constexpr uint32_t mask = (1u << B) - 1u;
-    // the digits of both groups, 4 bits each, the first group's first: element e + q is digit k0 + q
-    const unsigned long long dg = (unsigned long long)group_digits<S>(t, (uint32_t)two & mask) |
-                                  ((unsigned long long)group_digits<S>(t, (uint32_t)(two >> B) & mask) << (4 * g));
-    return (uint32_t)(dg >> (4 * ps.k0));
+    // element e + q is digit k0 + q of the first group, or digit k0 + q - g of the second
+    const uint32_t d1 = group_digits<S>(t, two & mask), d2 = group_digits<S>(t, (two >> B) & mask);
+    return (d1 >> (4 * ps.k0)) | (d2 << (4 * (g - ps.k0)));
 }
 
 }  // namespace gq
